@@ -1,0 +1,434 @@
+"""Throughput of the edge tensor product (forward + VJP) on B200.
+
+One step = the whole hot path on one batch of synthetic input resident in HBM:
+reverse CSR (edges grouped by source) + forward + VJP (grad_x, grad_w, grad_r),
+all through the C ABI (libetp.so). Default workload: 1024 nodes x 128
+neighbours (131072 edges), L = 3, C = 128, 34 paths, fp32.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+Prints one JSON line (rank 0). With N > 1 (torchrun, one process per GPU) every
+rank runs its own replica of the workload (independent problems, no data-path
+collective): weak scaling; the timing is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "edges/s fwd+VJP (L=3, C=128) and achieved HBM GB/s vs roofline on 1 B200"
+UNIT = "edges/s"
+DESCR = {
+    "tiny": "32 nodes, 8 nearest neighbours (256 edges), L=1, C=8",
+    "micro_l2": "1024 nodes x 128 neighbours (131072 edges), L=2, C=128, 15 paths",
+    "micro_l3": "1024 nodes x 128 neighbours (131072 edges), L=3, C=128, 34 paths",
+    "water": "3072-atom water box, r_c = 5 A radius graph, L=2, C=64, 15 paths",
+    "large": "32768 atoms at 0.1/A^3, r_c = 4.5 A radius graph, L=3, C=64, 34 paths",
+}
+KERNEL_SOURCES = ["cg_tensor_products_b200/csrc/etp_kernels.cuh", "cg_tensor_products_b200/csrc/etp_device.cuh"]
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default="micro_l3", choices=sorted(DESCR))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU seconds of the oracle baseline")
+    return ap.parse_args()
+
+
+# ---------------------------------------------------------------------------
+# algorithmic traffic and work (what the method must move / compute)
+def algorithmic(wl, P, nnz):
+    """Bytes and FLOPs per launch of each kernel, counted from the data the method must touch."""
+    N, E, C = wl.N, wl.E, wl.C
+    D = (wl.L + 1) ** 2
+    node = N * D * C * 4
+    fwd_bytes = E * (4 * P * C + 12 + 4) + 2 * node + 4 * (N + 1)
+    bwd_bytes = E * (2 * 4 * P * C + 12 + 4 + 4 + 12) + 3 * node + 4 * (N + 1)
+    return {"fwd_bytes": fwd_bytes, "bwd_bytes": bwd_bytes}
+
+
+def flops(L, paths, nnz_total, C, E):
+    """FLOPs of the sparse-CG schedule the kernels run, per launch:
+    forward 2C(nnz + sum_p d3) per edge (u_p, then the weighted path sum);
+    VJP 2C(2 nnz + 3 sum_p d1) per edge (t_p and dL/dY per coupling entry; w*x,
+    grad_x and grad_w per input component)."""
+    s1 = sum(2 * p[0] + 1 for p in paths)
+    s3 = sum(2 * p[2] + 1 for p in paths)
+    fwd = 2 * C * (nnz_total + s3) * E
+    bwd = 2 * C * (2 * nnz_total + 3 * s1) * E
+    return fwd, bwd
+
+
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    """nvidia-smi samples every 100 ms while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.dev = device_index
+        self.proc = None
+        self.lines = []
+        self.t0 = self.t1 = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-lms", "100", "-i", str(self.dev)], stdout=subprocess.PIPE,
+                                         stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append((time.time(), line.strip()))
+
+    def mark(self, which):
+        setattr(self, which, time.time())
+
+    def stop(self):
+        if self.proc is None:
+            return {"samples": 0, "note": "nvidia-smi unavailable"}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        for ts, line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            rows.append((ts, parts))
+        inside = [p for ts, p in rows if self.t0 is not None and self.t0 - 0.1 <= ts <= self.t1 + 0.1] or \
+            [p for _, p in rows]
+        if not inside:
+            return {"samples": 0}
+        sm = [float(p[1]) for p in inside if p[1].replace(".", "").isdigit()]
+        smax = [float(p[2]) for p in inside if p[2].replace(".", "").isdigit()]
+        reasons = set()
+        for p in inside:
+            for name, val in zip(("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"),
+                                 p[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(inside),
+                "power_w_max": max(float(p[3]) for p in inside if p[3].replace(".", "").isdigit())
+                if any(p[3].replace(".", "").isdigit() for p in inside) else None}
+
+
+def physical_gpu_index(local_rank):
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    if vis:
+        ids = [v.strip() for v in vis.split(",") if v.strip()]
+        if local_rank < len(ids):
+            return ids[local_rank]
+    return str(local_rank)
+
+
+def measured_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel, workload):
+    """dram bytes per launch from a committed ncu capture of the same kernel source, else None."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        ent = d.get(f"{kernel}:{workload}")
+        if ent and ent.get("source_hash") == kernel_source_hash():
+            return ent["bytes_per_launch"]
+    except Exception:
+        pass
+    return None
+
+
+# ---------------------------------------------------------------------------
+def cpu_baseline(wl, seconds):
+    """The FP64 oracle, as it stands, on a bounded sample: fwd rows + VJP of the same edges."""
+    import numpy as np
+
+    import oracle
+
+    tp = oracle.OracleTP(wl.irreps, wl.L, wl.irreps, wl.C)
+    rng = np.random.default_rng(1)
+
+    def run(n_rows):
+        rows = np.sort(rng.choice(wl.N, size=min(n_rows, wl.N), replace=False))
+        edges = np.concatenate([np.arange(wl.row_ptr[i], wl.row_ptr[i + 1]) for i in rows])
+        srcs = np.unique(wl.src[edges])[:n_rows]
+        t0 = time.perf_counter()
+        tp.forward(wl.row_ptr, wl.src, wl.r, wl.x, wl.w, rows=rows)
+        tp.backward(wl.row_ptr, wl.src, wl.r, wl.x, wl.w, wl.g, nodes=srcs, edges=edges)
+        dt = time.perf_counter() - t0
+        # the grad_x sample covers the edges whose source is in srcs
+        n_src_edges = int(np.isin(wl.src, srcs).sum())
+        return dt, len(edges), n_src_edges
+
+    dt, ne, _ = run(2)
+    per_row = max(dt / 2, 1e-3)
+    n_rows = int(max(2, min(wl.N, seconds / per_row)))
+    dt, ne, nse = run(n_rows)
+    return {"value": ne / dt, "unit": "edges/s", "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"{n_rows} random destination rows ({ne} edges): forward of those rows, grad_w and grad_r "
+                      f"of those edges, grad_x of {min(n_rows, len(np.unique(wl.src[:])))} of their sources "
+                      f"({nse} edges); FP64 C loops with OpenMP, harmonics in numpy; {dt:.1f} s"}
+
+
+def reference_arm(args):
+    """The oracle on the host cores: each step a bounded sample of the workload."""
+    import numpy as np
+
+    import oracle
+    import workloads
+
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    wl = workloads.make(args.workload)
+    oracle.build()
+    tp = oracle.OracleTP(wl.irreps, wl.L, wl.irreps, wl.C)
+    rng = np.random.default_rng(2)
+    rows_per_step = 4
+
+    def step():
+        rows = np.sort(rng.choice(wl.N, size=rows_per_step, replace=False))
+        edges = np.concatenate([np.arange(wl.row_ptr[i], wl.row_ptr[i + 1]) for i in rows])
+        tp.forward(wl.row_ptr, wl.src, wl.r, wl.x, wl.w, rows=rows)
+        tp.backward(wl.row_ptr, wl.src, wl.r, wl.x, wl.w, wl.g, nodes=wl.src[edges[:rows_per_step]], edges=edges)
+        return len(edges)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    ne = sum(step() for _ in range(args.steps))
+    dt = time.perf_counter() - t0
+    value = ne / dt
+    cores = oracle.num_threads()
+    sample = f"each step: {rows_per_step} random destination rows of {args.workload} (forward + grad_w + grad_r " \
+             f"of their edges, grad_x of {rows_per_step} sources); FP64 oracle"
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * dt / max(args.steps, 1),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"{args.workload}: {DESCR[args.workload]}", "N": wl.N, "E": wl.E,
+                   "sample": sample},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+# ---------------------------------------------------------------------------
+def main():
+    args = parse()
+    if args.impl == "reference":
+        reference_arm(args)
+        return
+
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    import cg_tensor_products_b200 as etp
+    import workloads
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    wl = workloads.make(args.workload)
+    plan = etp.Plan(wl.irreps, wl.L, wl.irreps, wl.C)
+    nnz_total = len(plan.couplings()[1])
+    N, E = wl.N, wl.E
+    host = {k: torch.from_numpy(np.ascontiguousarray(getattr(wl, k))) for k in ("row_ptr", "src", "r", "x", "w", "g")}
+    d = {k: v.to(dev) for k, v in host.items()}
+    out = torch.empty((N, plan.dim_out, wl.C), device=dev)
+    gx = torch.empty((N, plan.dim_in, wl.C), device=dev)
+    gw = torch.empty((E, plan.n_paths, wl.C), device=dev)
+    gr = torch.empty((E, 3), device=dev)
+    rev_ptr = torch.empty(N + 1, dtype=torch.int32, device=dev)
+    rev_perm = torch.empty(E, dtype=torch.int32, device=dev)
+    dst = torch.empty(E, dtype=torch.int32, device=dev)
+    ws = torch.empty(max(etp.reverse_csr_workspace_size(N, E), 16), dtype=torch.uint8, device=dev)
+    lib = etp._load()
+    stream = torch.cuda.current_stream()
+    sp = etp._stream(stream)
+    P = etp._ptr
+
+    def step(ev=None):
+        if ev:
+            ev[0].record(stream)
+        etp._check(lib.etp_build_reverse_csr(N, E, P(d["row_ptr"]), P(d["src"]), P(rev_ptr), P(rev_perm), P(dst),
+                                             P(ws), ws.numel(), sp), "reverse csr")
+        if ev:
+            ev[1].record(stream)
+        etp._check(lib.etp_forward(plan.handle, N, E, P(d["row_ptr"]), P(d["src"]), P(d["r"]), P(d["x"]), P(d["w"]),
+                                   P(out), sp), "forward")
+        if ev:
+            ev[2].record(stream)
+        etp._check(lib.etp_backward(plan.handle, N, E, P(d["row_ptr"]), P(d["src"]), P(rev_ptr), P(rev_perm), P(dst),
+                                    P(d["r"]), P(d["x"]), P(d["w"]), P(d["g"]), P(gx), P(gw), P(gr), sp), "backward")
+        if ev:
+            ev[3].record(stream)
+
+    for _ in range(max(args.warmup, 0)):
+        step()
+    torch.cuda.synchronize()
+
+    K = args.steps
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
+    sampler = ClockSampler(physical_gpu_index(local_rank))
+    sampler.start()
+    time.sleep(0.3)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    sampler.mark("t0")
+    t_start.record(stream)
+    for k in range(K):
+        step(evs[k])
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    sampler.mark("t1")
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+    total_ms = t_start.elapsed_time(t_end)
+    rc_ms = sum(e[0].elapsed_time(e[1]) for e in evs) / K
+    fwd_ms = sum(e[1].elapsed_time(e[2]) for e in evs) / K
+    bwd_ms = sum(e[2].elapsed_time(e[3]) for e in evs) / K
+    ms_step = total_ms / K
+    if world > 1:
+        t = torch.tensor([ms_step], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)  # timing only, not the data path
+        ms_step = float(t.item())
+    value = world * E / (ms_step / 1e3)
+
+    # roofline of the dominant kernel (the VJP)
+    alg = algorithmic(wl, plan.n_paths, nnz_total)
+    peak, peak_kind = measured_peaks()
+    fl_fwd, fl_bwd = flops(wl.L, plan.paths, nnz_total, wl.C, E)
+    kern = {"reverse_csr_ms": rc_ms, "forward_ms": fwd_ms, "backward_ms": bwd_ms,
+            "forward_GBps": alg["fwd_bytes"] / (fwd_ms * 1e6), "backward_GBps": alg["bwd_bytes"] / (bwd_ms * 1e6),
+            "forward_TFLOPs": fl_fwd / (fwd_ms * 1e9), "backward_TFLOPs": fl_bwd / (bwd_ms * 1e9),
+            "forward_bytes_per_launch": alg["fwd_bytes"], "backward_bytes_per_launch": alg["bwd_bytes"],
+            "forward_flop_per_launch": fl_fwd, "backward_flop_per_launch": fl_bwd}
+    dom = "backward" if bwd_ms >= fwd_ms else "forward"
+    achieved = kern[f"{dom}_GBps"]
+    roofline = {"bound": "hbm", "kernel": f"etp_{'bwd' if dom == 'backward' else 'fwd'}_kernel", "achieved": achieved,
+                "peak": peak, "unit": "GB/s", "frac": achieved / peak, "peak_source": f"{peak_kind} (hbm_gbs)",
+                "traffic": recorded_traffic(f"etp_{'bwd' if dom == 'backward' else 'fwd'}_kernel", args.workload)}
+
+    # end to end through the public API with host buffers (pinned), copies inside the timed region
+    e2e = None
+    if not args.no_e2e:
+        pin = {k: v.pin_memory() for k, v in host.items()}
+        h_out = {"out": torch.empty(out.shape).pin_memory(), "gx": torch.empty(gx.shape).pin_memory(),
+                 "gw": torch.empty(gw.shape).pin_memory(), "gr": torch.empty(gr.shape).pin_memory()}
+        h2d = sum(v.numel() * v.element_size() for v in pin.values())
+        d2h = sum(v.numel() * v.element_size() for v in h_out.values())
+        k_e2e = max(3, min(K, 20))
+
+        def e2e_step():
+            for k, v in pin.items():
+                d[k].copy_(v, non_blocking=True)
+            step()
+            h_out["out"].copy_(out, non_blocking=True)
+            h_out["gx"].copy_(gx, non_blocking=True)
+            h_out["gw"].copy_(gw, non_blocking=True)
+            h_out["gr"].copy_(gr, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(k_e2e):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize()
+        e_ms = a.elapsed_time(b) / k_e2e
+        if world > 1:
+            t = torch.tensor([e_ms], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e_ms = float(t.item())
+        e2e = {"value": world * E / (e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "ms_per_step": e_ms, "steps": k_e2e}
+
+    # kernels launched per step: reverse CSR (count, scan, edge rows, 3 per radix pass) + forward + backward
+    passes = 0
+    while (1 << (8 * passes)) < N and passes < 4:
+        passes += 1
+    rc_launches = (1 if E > 0 else 0) + 1 + (1 if E > 0 else 0) + ((1 if passes == 0 else 3 * passes) if E > 0 else 0)
+    launches = K * (rc_launches + 2)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(wl, args.cpu_seconds)
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    print(json.dumps({
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
+        "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic",
+        "config": {"workload": f"{args.workload}: {DESCR[args.workload]}", "N": N, "E": E, "L": wl.L, "C": wl.C,
+                   "P": plan.n_paths, "cg_nnz": nnz_total,
+                   "step": "reverse CSR + forward + VJP (grad_x, grad_w, grad_r), inputs resident in HBM",
+                   "l2": f"inputs larger than L2 (w = {wl.w.nbytes / 1e9:.2f} GB streamed per pass)",
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+        "roofline": roofline, "kernels": kern, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches,
+        "clocks": clocks,
+    }), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,212 @@
+"""Python binding of libetp.so, the B200 edge-wise equivariant tensor product library.
+
+Argument marshalling only: every step of the computation runs in the library's
+CUDA kernels (see include/etp.h for the operation, layouts and conventions).
+PyTorch supplies device memory and the current stream. There is no CPU path:
+tensors must live on a CUDA device, and a missing library raises.
+
+    plan = Plan("0..3", 3, "0..3", C=128)
+    out = forward(plan, row_ptr, src, r, x, w)
+    rev_ptr, rev_perm, dst = build_reverse_csr(N, row_ptr, src)
+    gx, gw, gr = backward(plan, row_ptr, src, rev_ptr, rev_perm, dst, r, x, w, grad_out)
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libetp.so")
+HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "etp.h")
+
+ETP_OK, ETP_ERR_INVALID_ARG, ETP_ERR_UNSUPPORTED, ETP_ERR_BAD_CSR = 0, 1, 2, 3
+ETP_ERR_CUDA, ETP_ERR_ALLOC, ETP_ERR_WORKSPACE = 4, 5, 6
+ETP_F32 = 0
+CSR_BAD_ENDPOINTS, CSR_NOT_MONOTONE, CSR_SRC_RANGE = 1, 2, 4
+
+_lib = None
+
+
+class EtpError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        msg = _load().etp_status_string(status).decode() if _lib is not None else str(status)
+        super().__init__(f"{where}: {msg} (status {status})")
+
+
+def _load():
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"{LIB_PATH} is missing: build it with `python -m cg_tensor_products_b200.build` "
+                           "(or __graft_entry__.build()); there is no fallback implementation")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, i32, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+    sig = {
+        "etp_plan_create": [ctypes.POINTER(vp), ctypes.c_char_p, i32, ctypes.c_char_p, i32, i32],
+        "etp_plan_info": [vp, vp, vp, vp, vp, vp],
+        "etp_plan_couplings": [vp, vp, vp, vp, vp, vp, vp],
+        "etp_plan_destroy": [vp],
+        "etp_forward": [vp, i32, i32, vp, vp, vp, vp, vp, vp, vp],
+        "etp_backward": [vp, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp],
+        "etp_reverse_csr_workspace_size": [i32, i32, ctypes.POINTER(sz)],
+        "etp_build_reverse_csr": [i32, i32, vp, vp, vp, vp, vp, vp, sz, vp],
+        "etp_validate_csr": [i32, i32, vp, vp, vp, vp],
+        "etp_status_string": [i32],
+    }
+    for name, args in sig.items():
+        fn = getattr(lib, name)
+        fn.argtypes = args
+        fn.restype = ctypes.c_char_p if name == "etp_status_string" else ctypes.c_int
+    _lib = lib
+    return lib
+
+
+def declared_symbols() -> list:
+    """Function names declared in include/etp.h."""
+    with open(HEADER_PATH) as f:
+        txt = f.read()
+    return re.findall(r"ETP_API\s+[\w\s\*]+?\b(etp_\w+)\s*\(", txt)
+
+
+def _check(status: int, where: str):
+    if status != ETP_OK:
+        raise EtpError(status, where)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    import torch
+
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if t is None:
+            continue
+        if not t.is_cuda:
+            raise ValueError("tensors must be CUDA tensors: this library has no CPU path")
+        if not t.is_contiguous():
+            raise ValueError("tensors must be contiguous")
+
+
+class Plan:
+    """A tensor-product plan: irreps in x harmonics 0..sh_lmax -> irreps out, C channels, fp32."""
+
+    def __init__(self, irreps_in: str, sh_lmax: int, irreps_out: str, C: int):
+        lib = _load()
+        h = ctypes.c_void_p()
+        _check(lib.etp_plan_create(ctypes.byref(h), irreps_in.encode(), int(sh_lmax), irreps_out.encode(),
+                                   int(C), ETP_F32), "etp_plan_create")
+        self._h = h
+        self.C = int(C)
+        n_paths, d_in, d_sh, d_out = (ctypes.c_int() for _ in range(4))
+        _check(lib.etp_plan_info(h, ctypes.byref(n_paths), ctypes.byref(d_in), ctypes.byref(d_sh),
+                                 ctypes.byref(d_out), None), "etp_plan_info")
+        self.n_paths, self.dim_in, self.dim_sh, self.dim_out = n_paths.value, d_in.value, d_sh.value, d_out.value
+        arr = (ctypes.c_int * (3 * self.n_paths))()
+        _check(lib.etp_plan_info(h, None, None, None, None, arr), "etp_plan_info")
+        self.paths = [tuple(arr[3 * p:3 * p + 3]) for p in range(self.n_paths)]
+
+    @property
+    def handle(self):
+        return self._h
+
+    def couplings(self):
+        """(path_off, m1, m2, m3, val) of the coefficients compiled into the kernels."""
+        lib = _load()
+        nnz = ctypes.c_int()
+        _check(lib.etp_plan_couplings(self._h, ctypes.byref(nnz), None, None, None, None, None), "couplings")
+        n = nnz.value
+        off = (ctypes.c_int * (self.n_paths + 1))()
+        m1, m2, m3 = ((ctypes.c_int * n)() for _ in range(3))
+        val = (ctypes.c_double * n)()
+        _check(lib.etp_plan_couplings(self._h, ctypes.byref(nnz), off, m1, m2, m3, val), "couplings")
+        return list(off), list(m1), list(m2), list(m3), list(val)
+
+    def close(self):
+        if getattr(self, "_h", None) and _lib is not None:
+            _lib.etp_plan_destroy(self._h)
+        self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def forward(plan: Plan, row_ptr, src, r, x, w, out=None, stream=None):
+    """out[i] = sum over row i of the weighted tensor products (launches etp_forward)."""
+    import torch
+
+    N, E = row_ptr.numel() - 1, src.numel()
+    if out is None:
+        out = torch.empty((N, plan.dim_out, plan.C), device=x.device, dtype=torch.float32)
+    _need_cuda(row_ptr, src, r, x, w, out)
+    _check(_load().etp_forward(plan.handle, N, E, _ptr(row_ptr), _ptr(src), _ptr(r), _ptr(x), _ptr(w), _ptr(out),
+                               _stream(stream)), "etp_forward")
+    return out
+
+
+def backward(plan: Plan, row_ptr, src, rev_ptr, rev_perm, dst, r, x, w, grad_out,
+             want=("x", "w", "r"), grad_x=None, grad_w=None, grad_r=None, stream=None):
+    """(grad_x, grad_w, grad_r) for the cotangent grad_out (launches etp_backward); unwanted ones are None."""
+    import torch
+
+    N, E = row_ptr.numel() - 1, src.numel()
+    dev = x.device
+    if "x" in want and grad_x is None:
+        grad_x = torch.empty((N, plan.dim_in, plan.C), device=dev, dtype=torch.float32)
+    if "w" in want and grad_w is None:
+        grad_w = torch.empty((E, plan.n_paths, plan.C), device=dev, dtype=torch.float32)
+    if "r" in want and grad_r is None:
+        grad_r = torch.empty((E, 3), device=dev, dtype=torch.float32)
+    _need_cuda(row_ptr, src, rev_ptr, rev_perm, dst, r, x, w, grad_out, grad_x, grad_w, grad_r)
+    _check(_load().etp_backward(plan.handle, N, E, _ptr(row_ptr), _ptr(src), _ptr(rev_ptr), _ptr(rev_perm),
+                                _ptr(dst), _ptr(r), _ptr(x), _ptr(w), _ptr(grad_out), _ptr(grad_x), _ptr(grad_w),
+                                _ptr(grad_r), _stream(stream)), "etp_backward")
+    return grad_x, grad_w, grad_r
+
+
+def reverse_csr_workspace_size(N: int, E: int) -> int:
+    b = ctypes.c_size_t()
+    _check(_load().etp_reverse_csr_workspace_size(int(N), int(E), ctypes.byref(b)), "workspace_size")
+    return b.value
+
+
+def build_reverse_csr(N: int, row_ptr, src, with_dst=True, workspace=None, stream=None):
+    """(rev_ptr [N+1], rev_perm [E], dst [E] or None), all int32 on the device (etp_build_reverse_csr)."""
+    import torch
+
+    E = src.numel()
+    dev = row_ptr.device
+    rev_ptr = torch.empty(N + 1, dtype=torch.int32, device=dev)
+    rev_perm = torch.empty(E, dtype=torch.int32, device=dev)
+    dst = torch.empty(E, dtype=torch.int32, device=dev) if with_dst else None
+    nbytes = reverse_csr_workspace_size(N, E)
+    if workspace is None:
+        workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=dev)
+    _need_cuda(row_ptr, src, rev_ptr, rev_perm, dst, workspace)
+    _check(_load().etp_build_reverse_csr(N, E, _ptr(row_ptr), _ptr(src), _ptr(rev_ptr), _ptr(rev_perm), _ptr(dst),
+                                         _ptr(workspace), workspace.numel(), _stream(stream)),
+           "etp_build_reverse_csr")
+    return rev_ptr, rev_perm, dst
+
+
+def validate_csr(N: int, row_ptr, src, stream=None) -> int:
+    """The ETP_CSR_* bits of every problem found in the CSR (0 = valid). Synchronises the stream."""
+    import torch
+
+    flag = torch.empty(1, dtype=torch.int32, device=row_ptr.device)
+    _need_cuda(row_ptr, src, flag)
+    _check(_load().etp_validate_csr(N, src.numel(), _ptr(row_ptr), _ptr(src), _ptr(flag), _stream(stream)),
+           "etp_validate_csr")
+    return int(flag.item())

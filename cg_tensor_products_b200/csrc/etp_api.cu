@@ -1,0 +1,307 @@
+// C ABI of the edge tensor product library (declared in include/etp.h):
+// plan lifecycle, host-side argument checks, and launches on the caller's stream.
+#include <cuda_runtime.h>
+
+#include <cctype>
+#include <cstdint>
+#include <cstring>
+#include <new>
+#include <string>
+#include <vector>
+
+#include "../../include/etp.h"
+#include "etp_device.cuh"
+#include "etp_internal.h"
+
+struct etp_plan_s {
+    int L;
+    bool o3;
+    int C;
+    int P;
+    int D;
+    std::vector<int> paths;  // 3 * P
+};
+
+namespace {
+
+struct Irrep {
+    int l;
+    int parity;  // 0: none, +1: even, -1: odd
+};
+
+// "a..b" | "l[e|o]+l[e|o]+..." ; whitespace ignored. false on a malformed string.
+bool parse_irreps(const char* s, std::vector<Irrep>& out) {
+    out.clear();
+    std::string t;
+    for (const char* c = s; *c; ++c)
+        if (!std::isspace((unsigned char)*c)) t.push_back(*c);
+    if (t.empty()) return false;
+    size_t dots = t.find("..");
+    if (dots != std::string::npos) {
+        std::string a = t.substr(0, dots), b = t.substr(dots + 2);
+        if (a.empty() || b.empty() || a.size() > 3 || b.size() > 3) return false;
+        for (char c : a + b)
+            if (!std::isdigit((unsigned char)c)) return false;
+        int lo = std::stoi(a), hi = std::stoi(b);
+        if (lo > hi) return false;
+        for (int l = lo; l <= hi; ++l) out.push_back({l, 0});
+        return true;
+    }
+    size_t pos = 0;
+    while (pos <= t.size()) {
+        size_t plus = t.find('+', pos);
+        std::string tok = t.substr(pos, plus == std::string::npos ? std::string::npos : plus - pos);
+        if (tok.empty()) return false;
+        int par = 0;
+        if (tok.back() == 'e' || tok.back() == 'o') {
+            par = tok.back() == 'e' ? 1 : -1;
+            tok.pop_back();
+        }
+        if (tok.empty() || tok.size() > 3) return false;
+        for (char c : tok)
+            if (!std::isdigit((unsigned char)c)) return false;
+        out.push_back({std::stoi(tok), par});
+        if (plus == std::string::npos) break;
+        pos = plus + 1;
+    }
+    for (size_t k = 1; k < out.size(); ++k)
+        if (out[k].l <= out[k - 1].l || (out[k].parity == 0) != (out[0].parity == 0)) return false;
+    return true;
+}
+
+// irreps 0..L each once; parities absent everywhere, or natural everywhere.
+// Returns L, or -1 if the list is not of that form.
+int full_range(const std::vector<Irrep>& v, int* parity_mode) {
+    for (size_t k = 0; k < v.size(); ++k) {
+        if (v[k].l != (int)k) return -1;
+        int natural = (k % 2 == 0) ? 1 : -1;
+        if (v[k].parity != 0 && v[k].parity != natural) return -1;
+    }
+    *parity_mode = v[0].parity != 0 ? 1 : 0;
+    return (int)v.size() - 1;
+}
+
+template <int L, bool O3>
+void fill_paths(std::vector<int>& out) {
+    using PS = etp::PathSet<L, O3>;
+    out.clear();
+    for (int p = 0; p < PS::P; ++p) {
+        etp::Path pt = PS::path(p);
+        out.push_back(pt.l1);
+        out.push_back(pt.l2);
+        out.push_back(pt.l3);
+    }
+}
+
+void plan_paths(int L, bool o3, std::vector<int>& out) {
+    switch (L * 2 + (o3 ? 1 : 0)) {
+        case 0: fill_paths<0, false>(out); break;
+        case 1: fill_paths<0, true>(out); break;
+        case 2: fill_paths<1, false>(out); break;
+        case 3: fill_paths<1, true>(out); break;
+        case 4: fill_paths<2, false>(out); break;
+        case 5: fill_paths<2, true>(out); break;
+        case 6: fill_paths<3, false>(out); break;
+        default: fill_paths<3, true>(out); break;
+    }
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+
+etp_status cuda_status(cudaError_t e) { return e == cudaSuccess ? ETP_OK : ETP_ERR_CUDA; }
+
+// teams of C/4 lanes; 4 warps per block
+dim3 node_grid(int N, int team) {
+    long long nodes_per_block = (long long)(etp::kThreadsPerBlock / 32) * (32 / team);
+    return dim3((unsigned)((N + nodes_per_block - 1) / nodes_per_block), 1, 1);
+}
+
+}  // namespace
+
+extern "C" {
+
+etp_status etp_plan_create(etp_plan_t* plan, const char* irreps_in, int sh_lmax, const char* irreps_out, int C,
+                           etp_dtype dtype) {
+    if (!plan || !irreps_in || !irreps_out) return ETP_ERR_INVALID_ARG;
+    *plan = nullptr;
+    std::vector<Irrep> ins, outs;
+    if (!parse_irreps(irreps_in, ins) || !parse_irreps(irreps_out, outs)) return ETP_ERR_INVALID_ARG;
+    if ((ins[0].parity == 0) != (outs[0].parity == 0)) return ETP_ERR_INVALID_ARG;
+    if (sh_lmax < 0 || C <= 0) return ETP_ERR_INVALID_ARG;
+    if (dtype != ETP_F32) return ETP_ERR_UNSUPPORTED;
+    int pm_in = 0, pm_out = 0;
+    int L_in = full_range(ins, &pm_in), L_out = full_range(outs, &pm_out);
+    if (L_in < 0 || L_out != L_in || sh_lmax != L_in || L_in > etp_gen::kLmax) return ETP_ERR_UNSUPPORTED;
+    if (C % 4 != 0) return ETP_ERR_UNSUPPORTED;
+    int C4 = C / 4;
+    if (C4 > 32 || (C4 & (C4 - 1)) != 0) return ETP_ERR_UNSUPPORTED;
+    etp_plan_s* p = new (std::nothrow) etp_plan_s();
+    if (!p) return ETP_ERR_ALLOC;
+    p->L = L_in;
+    p->o3 = pm_in != 0;
+    p->C = C;
+    p->D = (L_in + 1) * (L_in + 1);
+    try {
+        plan_paths(p->L, p->o3, p->paths);
+    } catch (...) {
+        delete p;
+        return ETP_ERR_ALLOC;
+    }
+    p->P = (int)p->paths.size() / 3;
+    *plan = p;
+    return ETP_OK;
+}
+
+etp_status etp_plan_info(etp_plan_t plan, int* n_paths, int* dim_in, int* dim_sh, int* dim_out, int* paths_l1l2l3) {
+    if (!plan) return ETP_ERR_INVALID_ARG;
+    if (n_paths) *n_paths = plan->P;
+    if (dim_in) *dim_in = plan->D;
+    if (dim_sh) *dim_sh = plan->D;
+    if (dim_out) *dim_out = plan->D;
+    if (paths_l1l2l3) std::memcpy(paths_l1l2l3, plan->paths.data(), sizeof(int) * plan->paths.size());
+    return ETP_OK;
+}
+
+etp_status etp_plan_couplings(etp_plan_t plan, int* nnz, int* path_off, int* m1, int* m2, int* m3, double* val) {
+    if (!plan || !nnz) return ETP_ERR_INVALID_ARG;
+    int total = 0;
+    for (int p = 0; p < plan->P; ++p) {
+        const int a = plan->paths[3 * p], b = plan->paths[3 * p + 1], c = plan->paths[3 * p + 2];
+        total += etp_gen::kCgCnt[a][b][c];
+    }
+    *nnz = total;
+    const bool want = path_off || m1 || m2 || m3 || val;
+    if (!want) return ETP_OK;
+    if (!path_off || !m1 || !m2 || !m3 || !val) return ETP_ERR_INVALID_ARG;
+    int k = 0;
+    path_off[0] = 0;
+    for (int p = 0; p < plan->P; ++p) {
+        const int a = plan->paths[3 * p], b = plan->paths[3 * p + 1], c = plan->paths[3 * p + 2];
+        const int off = etp_gen::kCgOff[a][b][c], cnt = etp_gen::kCgCnt[a][b][c];
+        for (int q = 0; q < cnt; ++q, ++k) {
+            m1[k] = etp_gen::kCg[off + q].m1;
+            m2[k] = etp_gen::kCg[off + q].m2;
+            m3[k] = etp_gen::kCg[off + q].m3;
+            val[k] = etp_gen::kCg[off + q].v;
+        }
+        path_off[p + 1] = k;
+    }
+    return ETP_OK;
+}
+
+etp_status etp_plan_destroy(etp_plan_t plan) {
+    delete plan;
+    return ETP_OK;
+}
+
+etp_status etp_forward(etp_plan_t plan, int N, int E, const int32_t* row_ptr, const int32_t* src, const float* r,
+                       const float* x, const float* w, float* out, etp_stream_t stream) {
+    if (!plan || N < 0 || E < 0) return ETP_ERR_INVALID_ARG;
+    if (N == 0) return E == 0 ? ETP_OK : ETP_ERR_INVALID_ARG;
+    if (!row_ptr || !x || !out || !aligned4(row_ptr) || !aligned16(x) || !aligned16(out)) return ETP_ERR_INVALID_ARG;
+    if (E > 0 && (!src || !r || !w || !aligned4(src) || !aligned4(r) || !aligned16(w))) return ETP_ERR_INVALID_ARG;
+    etp::FwdArgs a{N, E, row_ptr, src, r, reinterpret_cast<const float4*>(x), reinterpret_cast<const float4*>(w),
+                   reinterpret_cast<float4*>(out), plan->C / 4, plan->C / 4};
+    const dim3 grid = node_grid(N, a.team);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t err;
+    switch (plan->L) {
+        case 0: err = etp::launch_forward<0>(plan->o3, a, grid, s); break;
+        case 1: err = etp::launch_forward<1>(plan->o3, a, grid, s); break;
+        case 2: err = etp::launch_forward<2>(plan->o3, a, grid, s); break;
+        default: err = etp::launch_forward<3>(plan->o3, a, grid, s); break;
+    }
+    return cuda_status(err);
+}
+
+etp_status etp_backward(etp_plan_t plan, int N, int E, const int32_t* row_ptr, const int32_t* src,
+                        const int32_t* rev_ptr, const int32_t* rev_perm, const int32_t* dst_of_edge, const float* r,
+                        const float* x, const float* w, const float* grad_out, float* grad_x, float* grad_w,
+                        float* grad_r, etp_stream_t stream) {
+    if (!plan || N < 0 || E < 0) return ETP_ERR_INVALID_ARG;
+    if (N == 0) return E == 0 ? ETP_OK : ETP_ERR_INVALID_ARG;
+    if (!row_ptr || !rev_ptr || !x || !grad_out || !aligned4(row_ptr) || !aligned4(rev_ptr) || !aligned16(x) ||
+        !aligned16(grad_out))
+        return ETP_ERR_INVALID_ARG;
+    if (grad_x && !aligned16(grad_x)) return ETP_ERR_INVALID_ARG;
+    if (E > 0) {
+        if (!src || !rev_perm || !r || !w || !aligned4(src) || !aligned4(rev_perm) || !aligned4(r) || !aligned16(w))
+            return ETP_ERR_INVALID_ARG;
+        if ((grad_w && !aligned16(grad_w)) || (grad_r && !aligned4(grad_r)) ||
+            (dst_of_edge && !aligned4(dst_of_edge)))
+            return ETP_ERR_INVALID_ARG;
+    } else {
+        grad_w = nullptr;
+        grad_r = nullptr;
+    }
+    if (!grad_x && !grad_w && !grad_r) return ETP_OK;
+    etp::BwdArgs a{N,
+                   E,
+                   row_ptr,
+                   src,
+                   rev_ptr,
+                   rev_perm,
+                   dst_of_edge,
+                   r,
+                   reinterpret_cast<const float4*>(x),
+                   reinterpret_cast<const float4*>(w),
+                   reinterpret_cast<const float4*>(grad_out),
+                   reinterpret_cast<float4*>(grad_x),
+                   reinterpret_cast<float4*>(grad_w),
+                   grad_r,
+                   plan->C / 4,
+                   plan->C / 4};
+    const dim3 grid = node_grid(N, a.team);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t err;
+    switch (plan->L) {
+        case 0: err = etp::launch_backward<0>(plan->o3, a, grid, s); break;
+        case 1: err = etp::launch_backward<1>(plan->o3, a, grid, s); break;
+        case 2: err = etp::launch_backward<2>(plan->o3, a, grid, s); break;
+        default: err = etp::launch_backward<3>(plan->o3, a, grid, s); break;
+    }
+    return cuda_status(err);
+}
+
+etp_status etp_reverse_csr_workspace_size(int N, int E, size_t* bytes) {
+    if (N < 0 || E < 0 || !bytes) return ETP_ERR_INVALID_ARG;
+    *bytes = etp::reverse_csr_workspace_bytes(N, E);
+    return ETP_OK;
+}
+
+etp_status etp_build_reverse_csr(int N, int E, const int32_t* row_ptr, const int32_t* src, int32_t* rev_ptr,
+                                 int32_t* rev_perm, int32_t* dst_of_edge, void* workspace, size_t workspace_bytes,
+                                 etp_stream_t stream) {
+    if (N < 0 || E < 0) return ETP_ERR_INVALID_ARG;
+    if (N == 0 && E > 0) return ETP_ERR_INVALID_ARG;
+    if (!rev_ptr || !workspace || !aligned4(rev_ptr) || !aligned16(workspace)) return ETP_ERR_INVALID_ARG;
+    if (E > 0 && (!row_ptr || !src || !rev_perm || !aligned4(row_ptr) || !aligned4(src) || !aligned4(rev_perm)))
+        return ETP_ERR_INVALID_ARG;
+    if (dst_of_edge && !aligned4(dst_of_edge)) return ETP_ERR_INVALID_ARG;
+    if (workspace_bytes < etp::reverse_csr_workspace_bytes(N, E)) return ETP_ERR_WORKSPACE;
+    return cuda_status(etp::build_reverse_csr(N, E, row_ptr, src, rev_ptr, rev_perm, dst_of_edge, workspace,
+                                              reinterpret_cast<cudaStream_t>(stream)));
+}
+
+etp_status etp_validate_csr(int N, int E, const int32_t* row_ptr, const int32_t* src, int32_t* d_flag,
+                            etp_stream_t stream) {
+    if (N < 0 || E < 0 || !row_ptr || !d_flag || (E > 0 && !src)) return ETP_ERR_INVALID_ARG;
+    if (!aligned4(row_ptr) || !aligned4(d_flag) || (src && !aligned4(src))) return ETP_ERR_INVALID_ARG;
+    return cuda_status(etp::validate_csr(N, E, row_ptr, src, d_flag, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+const char* etp_status_string(etp_status status) {
+    switch (status) {
+        case ETP_OK: return "ok";
+        case ETP_ERR_INVALID_ARG: return "invalid argument (null, negative size, misaligned pointer or bad string)";
+        case ETP_ERR_UNSUPPORTED: return "unsupported irreps, L, C or dtype (no compiled kernel)";
+        case ETP_ERR_BAD_CSR: return "malformed CSR graph";
+        case ETP_ERR_CUDA: return "CUDA launch or runtime error";
+        case ETP_ERR_ALLOC: return "host allocation failed";
+        case ETP_ERR_WORKSPACE: return "workspace too small";
+    }
+    return "unknown status";
+}
+
+}  // extern "C"

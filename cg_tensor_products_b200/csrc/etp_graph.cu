@@ -1,0 +1,239 @@
+// Graph preprocessing on the device: the reverse CSR (edges grouped by source,
+// stable in edge id), the destination of every edge, and a CSR validator.
+//
+// The reverse grouping is a least-significant-digit radix sort of the source ids
+// with the edge ids as values, 8 bits per pass. Each pass is a stable counting
+// sort over tiles of kTile edges: (1) a per-tile digit histogram, (2) one
+// exclusive scan of the digit-major histogram table, (3) a stable scatter in
+// which one warp walks its tile in order, ranking equal digits inside each
+// 32-edge chunk with __match_any_sync. Stability of every pass makes the result
+// unique: ties (equal sources) stay in increasing edge id, so the output is
+// bit-exact and independent of scheduling. rev_ptr is the exclusive scan of the
+// per-source edge counts.
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "etp_internal.h"
+
+namespace etp {
+namespace {
+
+constexpr int kTile = 4096;
+constexpr int kScanThreads = 1024;
+
+__global__ void count_sources(const int32_t* __restrict__ src, int E, int N, int32_t* __restrict__ cnt) {
+    for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < E; e += gridDim.x * blockDim.x) {
+        int j = src[e];
+        if ((unsigned)j < (unsigned)N) atomicAdd(cnt + j, 1);
+    }
+}
+
+// Exclusive scan of in[0..n) into out[0..n], out[n] = total; one block, in
+// chunks of 4 * kScanThreads. in and out may alias.
+__global__ void __launch_bounds__(kScanThreads) scan_exclusive(const int32_t* in, int32_t* out, int n) {
+    __shared__ int32_t warp_sums[kScanThreads / 32];
+    __shared__ int32_t carry_s;
+    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+    if (tid == 0) carry_s = 0;
+    __syncthreads();
+    for (int base = 0; base < n; base += 4 * kScanThreads) {
+        int v[4];
+        int local = 0;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            int idx = base + tid * 4 + k;
+            v[k] = idx < n ? in[idx] : 0;
+            local += v[k];
+        }
+        int incl = local;
+#pragma unroll
+        for (int s = 1; s < 32; s <<= 1) {
+            int t = __shfl_up_sync(0xffffffffu, incl, s);
+            if (lane >= s) incl += t;
+        }
+        if (lane == 31) warp_sums[wid] = incl;
+        __syncthreads();
+        if (wid == 0) {
+            int ws = warp_sums[lane];
+#pragma unroll
+            for (int s = 1; s < 32; s <<= 1) {
+                int t = __shfl_up_sync(0xffffffffu, ws, s);
+                if (lane >= s) ws += t;
+            }
+            warp_sums[lane] = ws;  // inclusive over warps
+        }
+        __syncthreads();
+        int carry = carry_s;
+        int run = carry + (wid ? warp_sums[wid - 1] : 0) + incl - local;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            int idx = base + tid * 4 + k;
+            if (idx < n) out[idx] = run;
+            run += v[k];
+        }
+        __syncthreads();
+        if (tid == kScanThreads - 1) carry_s = run;
+        __syncthreads();
+    }
+    if (tid == 0) out[n] = carry_s;
+}
+
+// hist[d * n_tiles + t] = number of edges of tile t whose key has digit d.
+__global__ void __launch_bounds__(256) tile_histogram(const int32_t* __restrict__ keys, int E, int shift,
+                                                      int n_tiles, int32_t* __restrict__ hist) {
+    __shared__ int32_t h[256];
+    h[threadIdx.x] = 0;
+    __syncthreads();
+    const int t = blockIdx.x;
+    const int lo = t * kTile, hi = min(E, lo + kTile);
+    for (int e = lo + threadIdx.x; e < hi; e += 256) atomicAdd(h + ((keys[e] >> shift) & 255), 1);
+    __syncthreads();
+    hist[threadIdx.x * n_tiles + t] = h[threadIdx.x];
+}
+
+// Stable scatter of one tile per warp. vals_in == nullptr means the identity
+// (value = edge id).
+__global__ void __launch_bounds__(128) tile_scatter(const int32_t* __restrict__ keys_in,
+                                                    const int32_t* __restrict__ vals_in, int E, int shift,
+                                                    int n_tiles, const int32_t* __restrict__ offsets,
+                                                    int32_t* __restrict__ keys_out, int32_t* __restrict__ vals_out) {
+    __shared__ int32_t base_s[4][256];
+    const int wid = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int t = blockIdx.x * 4 + wid;
+    if (t >= n_tiles) return;  // whole warp leaves together
+    int32_t* base = base_s[wid];
+    for (int d = lane; d < 256; d += 32) base[d] = offsets[d * n_tiles + t];
+    __syncwarp();
+    const int lo = t * kTile, hi = min(E, lo + kTile);
+    const unsigned lt = (1u << lane) - 1u;
+    for (int c = lo; c < hi; c += 32) {
+        const int e = c + lane;
+        const bool act = e < hi;
+        const int key = act ? keys_in[e] : 0;
+        const int val = act ? (vals_in ? vals_in[e] : e) : 0;
+        const int d = act ? ((key >> shift) & 255) : 256 + lane;  // inactive lanes match nobody
+        const unsigned peers = __match_any_sync(0xffffffffu, d);
+        if (act) {
+            const int pos = base[d] + __popc(peers & lt);
+            keys_out[pos] = key;
+            vals_out[pos] = val;
+        }
+        __syncwarp();
+        if (act && lane == __ffs(peers) - 1) base[d] += __popc(peers);
+        __syncwarp();
+    }
+}
+
+__global__ void iota(int32_t* __restrict__ out, int n) {
+    for (int k = blockIdx.x * blockDim.x + threadIdx.x; k < n; k += gridDim.x * blockDim.x) out[k] = k;
+}
+
+__global__ void edge_rows(const int32_t* __restrict__ row_ptr, int N, int E, int32_t* __restrict__ dst) {
+    for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < E; e += gridDim.x * blockDim.x) {
+        int lo = 0, hi = N;  // row_ptr[lo] <= e < row_ptr[hi] on a valid CSR
+        while (hi - lo > 1) {
+            int mid = (lo + hi) >> 1;
+            if (row_ptr[mid] <= e)
+                lo = mid;
+            else
+                hi = mid;
+        }
+        dst[e] = lo;
+    }
+}
+
+__global__ void validate(const int32_t* __restrict__ row_ptr, const int32_t* __restrict__ src, int N, int E,
+                         int32_t* __restrict__ flag) {
+    const int tid = blockIdx.x * blockDim.x + threadIdx.x, stride = gridDim.x * blockDim.x;
+    int bits = 0;
+    if (tid == 0 && (row_ptr[0] != 0 || row_ptr[N] != E)) bits |= 1;
+    for (int i = tid; i < N; i += stride)
+        if (row_ptr[i] > row_ptr[i + 1]) bits |= 2;
+    for (int e = tid; e < E; e += stride) {
+        int j = src[e];
+        if (j < 0 || j >= N) bits |= 4;
+    }
+    if (bits) atomicOr(flag, bits);
+}
+
+inline size_t align16(size_t b) { return (b + 15) & ~size_t(15); }
+inline int grid_for(long long n, int threads) {
+    long long b = (n + threads - 1) / threads;
+    if (b < 1) b = 1;
+    if (b > 148 * 32) b = 148 * 32;
+    return (int)b;
+}
+inline int radix_passes(int N) {
+    int bits = 0;
+    while (bits < 31 && (1ll << bits) < (long long)N) ++bits;  // keys are in [0, N)
+    return (bits + 7) / 8;
+}
+
+}  // namespace
+
+size_t reverse_csr_workspace_bytes(int N, int E) {
+    const int n_tiles = (E + kTile - 1) / kTile;
+    size_t b = 0;
+    b += align16(sizeof(int32_t) * ((size_t)N + 1));      // counts
+    b += 3 * align16(sizeof(int32_t) * (size_t)E);        // keys ping-pong + spare values
+    b += align16(sizeof(int32_t) * (256 * (size_t)n_tiles + 1));  // tile histograms (+ total)
+    return b;
+}
+
+cudaError_t build_reverse_csr(int N, int E, const int32_t* row_ptr, const int32_t* src, int32_t* rev_ptr,
+                              int32_t* rev_perm, int32_t* dst, void* ws, cudaStream_t s) {
+    char* p = static_cast<char*>(ws);
+    int32_t* cnt = reinterpret_cast<int32_t*>(p);
+    p += align16(sizeof(int32_t) * ((size_t)N + 1));
+    int32_t* keys_a = reinterpret_cast<int32_t*>(p);
+    p += align16(sizeof(int32_t) * (size_t)E);
+    int32_t* keys_b = reinterpret_cast<int32_t*>(p);
+    p += align16(sizeof(int32_t) * (size_t)E);
+    int32_t* vals_spare = reinterpret_cast<int32_t*>(p);
+    p += align16(sizeof(int32_t) * (size_t)E);
+    int32_t* hist = reinterpret_cast<int32_t*>(p);
+
+    cudaError_t err;
+    // rev_ptr: exclusive scan of per-source counts
+    if ((err = cudaMemsetAsync(cnt, 0, sizeof(int32_t) * ((size_t)N + 1), s)) != cudaSuccess) return err;
+    if (E > 0) count_sources<<<grid_for(E, 256), 256, 0, s>>>(src, E, N, cnt);
+    scan_exclusive<<<1, kScanThreads, 0, s>>>(cnt, rev_ptr, N);
+    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    if (dst && E > 0) edge_rows<<<grid_for(E, 256), 256, 0, s>>>(row_ptr, N, E, dst);
+    if (E == 0) return cudaGetLastError();
+
+    const int passes = radix_passes(N);
+    if (passes == 0) {  // a single node: every edge has source 0
+        iota<<<grid_for(E, 256), 256, 0, s>>>(rev_perm, E);
+        return cudaGetLastError();
+    }
+    const int n_tiles = (E + kTile - 1) / kTile;
+    // values ping-pong between vals_spare and rev_perm, ending in rev_perm
+    int32_t* vbuf[2] = {passes % 2 ? rev_perm : vals_spare, passes % 2 ? vals_spare : rev_perm};
+    int32_t* kbuf[2] = {keys_a, keys_b};
+    const int32_t* kin = src;
+    const int32_t* vin = nullptr;
+    for (int pass = 0; pass < passes; ++pass) {
+        const int shift = 8 * pass;
+        tile_histogram<<<n_tiles, 256, 0, s>>>(kin, E, shift, n_tiles, hist);
+        scan_exclusive<<<1, kScanThreads, 0, s>>>(hist, hist, 256 * n_tiles);
+        int32_t* kout = kbuf[pass & 1];
+        int32_t* vout = vbuf[pass & 1];
+        tile_scatter<<<(n_tiles + 3) / 4, 128, 0, s>>>(kin, vin, E, shift, n_tiles, hist, kout, vout);
+        kin = kout;
+        vin = vout;
+    }
+    return cudaGetLastError();
+}
+
+cudaError_t validate_csr(int N, int E, const int32_t* row_ptr, const int32_t* src, int32_t* flag,
+                         cudaStream_t s) {
+    cudaError_t err = cudaMemsetAsync(flag, 0, sizeof(int32_t), s);
+    if (err != cudaSuccess) return err;
+    long long work = (long long)(N > E ? N : E);
+    validate<<<grid_for(work, 256), 256, 0, s>>>(row_ptr, src, N, E, flag);
+    return cudaGetLastError();
+}
+
+}  // namespace etp

@@ -1,0 +1,53 @@
+// Internal interface between the C ABI (etp_api.cu) and the kernel translation units.
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include <cstddef>
+#include <cstdint>
+
+namespace etp {
+
+constexpr int kThreadsPerBlock = 128;  // 4 warps; forward and backward kernels
+
+struct FwdArgs {
+    int N, E;
+    const int32_t* row_ptr;
+    const int32_t* src;
+    const float* r;
+    const float4* x;
+    const float4* w;
+    float4* out;
+    int C4;    // C / 4
+    int team;  // lanes per node = C4 (power of two, <= 32)
+};
+
+struct BwdArgs {
+    int N, E;
+    const int32_t* row_ptr;
+    const int32_t* src;
+    const int32_t* rev_ptr;
+    const int32_t* rev_perm;
+    const int32_t* dst;  // may be null
+    const float* r;
+    const float4* x;
+    const float4* w;
+    const float4* g;
+    float4* grad_x;  // may be null
+    float4* grad_w;  // may be null
+    float* grad_r;   // may be null
+    int C4;
+    int team;
+};
+
+template <int L>
+cudaError_t launch_forward(bool o3, const FwdArgs& a, dim3 grid, cudaStream_t s);
+template <int L>
+cudaError_t launch_backward(bool o3, const BwdArgs& a, dim3 grid, cudaStream_t s);
+
+size_t reverse_csr_workspace_bytes(int N, int E);
+cudaError_t build_reverse_csr(int N, int E, const int32_t* row_ptr, const int32_t* src, int32_t* rev_ptr,
+                              int32_t* rev_perm, int32_t* dst, void* ws, cudaStream_t s);
+cudaError_t validate_csr(int N, int E, const int32_t* row_ptr, const int32_t* src, int32_t* flag, cudaStream_t s);
+
+}  // namespace etp

@@ -1,0 +1,174 @@
+/* etp.h - C ABI of the B200 edge-wise equivariant tensor product library.
+ *
+ * One operation, its vector-Jacobian product, and the graph preprocessing they
+ * need. For every directed edge e = (i <- j) of a CSR-by-destination graph:
+ *
+ *   Y(r_e)            real spherical harmonics of the edge vector, l2 = 0..L
+ *   msg_e[l3 m3, c]   = sum_{p = (l1,l2,l3)} w[e,p,c] sum_{m1,m2} CG_p[m1,m2,m3] Y_{l2 m2}(r_e) x[j, l1 m1, c]
+ *   out[i]            = sum over the edges e of row i of msg_e
+ *
+ * Passages this follows (the pages name the operation; they print no formula):
+ *   - "High-performance training and inference for deep equivariant interatomic
+ *     potentials", section "제안 방법": a fused tensor-product kernel whose Wigner
+ *     3-j contraction coefficients are held in compressed sparse form without
+ *     materialised intermediates;
+ *   - "Scaling the leading accuracy of deep equivariant models to biomolecular
+ *     simulations of realistic size", section "提出的方法": strided memory layout
+ *     and a tensor product done as a single contraction;
+ *   - "FlashCart 如何让等变原子间势更快更准?", sections "FlashCart 用笛卡尔内核替代
+ *     球谐耦合" (speed comes from memory access and the aggregation of edge
+ *     contributions) and "生成内核在高阶下胜过球谐基线" (edge convolution, forward
+ *     and vector-Jacobian product);
+ *   - "Machine Learning Interatomic Potentials: Advancing Open-Source Software
+ *     for Efficient and Scalable Molecular Simulation", section "방법론 및
+ *     아키텍처", item 2: dedicated kernels for Clebsch-Gordan tensor products.
+ *
+ * Conventions (the readings this library fixes where the pages are silent):
+ *   - harmonics: component normalisation (sum_m Y_lm^2 = 2l+1), no Condon-Shortley
+ *     phase, m = -l..l, Y_1 = sqrt(3) (y, z, x)/|r|; |r| < 1e-12 gives Y_0 = 1,
+ *     Y_{l>0} = 0 and zero derivative;
+ *   - CG_p: real coupling with sum_{m1,m2} CG^2 = 1 per m3, first nonzero entry in
+ *     lexicographic (m1, m2, m3) order positive; no further path normalisation;
+ *   - paths: every (l1, l2, l3) on the SO(3) triangle |l1-l2| <= l3 <= l1+l2,
+ *     lexicographic; with parity letters in the irreps strings only the paths
+ *     with l1+l2+l3 even (O(3), natural parities);
+ *   - edge vector r_e points from the destination i to the source j;
+ *   - paths into the same l3 are summed into one block; plain segment sum, no
+ *     neighbour normalisation; rows without edges give zeros.
+ *
+ * Layout (all row-major, channel fastest, "D" = (L+1)^2 components, l blocks
+ * ascending, m = -l..l inside a block):
+ *   x, out, grad_out, grad_x : float32 [N][D][C]
+ *   w, grad_w                : float32 [E][P][C]    (P paths in plan order)
+ *   r, grad_r                : float32 [E][3]
+ *   row_ptr int32 [N+1] (row_ptr[0] = 0, row_ptr[N] = E, nondecreasing),
+ *   src int32 [E] (source node of each edge, in [0, N)).
+ * Device pointers must be 16-byte aligned for x, w, out, grad_out, grad_x and
+ * grad_w (they are read and written as float4).
+ *
+ * Ownership and execution: the caller owns every buffer. A plan owns only host
+ * tables (the coupling values are compile-time constants of the kernels).
+ * etp_forward / etp_backward / etp_build_reverse_csr / etp_validate_csr enqueue
+ * work on the given stream and return without synchronising; they allocate no
+ * memory; they overwrite their outputs.
+ *
+ * Errors: arguments that can be checked on the host (NULL pointers, negative
+ * sizes, misalignment, unsupported irreps, L, C or dtype, a too-small workspace)
+ * are rejected before any launch. The CSR's contents live on the device and are
+ * not read by the host: etp_validate_csr checks them and reports through a
+ * device flag. The kernels never trap and never wait on a flag; on an invalid
+ * CSR they stay inside the given buffers (edges and rows out of range are
+ * skipped) and their results are unspecified. A failed launch returns
+ * ETP_ERR_CUDA (cudaGetLastError is consumed).
+ */
+#ifndef ETP_H_
+#define ETP_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define ETP_API __attribute__((visibility("default")))
+#else
+#define ETP_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct etp_plan_s* etp_plan_t;
+typedef struct CUstream_st* etp_stream_t; /* a cudaStream_t; NULL is the legacy default stream */
+
+typedef enum { ETP_F32 = 0 } etp_dtype;
+
+typedef enum {
+    ETP_OK = 0,
+    ETP_ERR_INVALID_ARG = 1, /* NULL, negative size, misaligned pointer, bad string   */
+    ETP_ERR_UNSUPPORTED = 2, /* irreps / L / C / dtype without a compiled kernel        */
+    ETP_ERR_BAD_CSR = 3,     /* reserved for callers that map the validation flag      */
+    ETP_ERR_CUDA = 4,        /* a CUDA launch or query failed                           */
+    ETP_ERR_ALLOC = 5,       /* host allocation of a plan failed                        */
+    ETP_ERR_WORKSPACE = 6    /* workspace smaller than etp_reverse_csr_workspace_size   */
+} etp_status;
+
+/* Bits of the flag written by etp_validate_csr. */
+#define ETP_CSR_BAD_ENDPOINTS 1 /* row_ptr[0] != 0 or row_ptr[N] != E */
+#define ETP_CSR_NOT_MONOTONE 2  /* row_ptr[i] > row_ptr[i+1] for some i */
+#define ETP_CSR_SRC_RANGE 4     /* some src[e] outside [0, N) */
+
+/* Create a plan for the tensor product of node irreps `irreps_in` with the edge
+ * harmonics l2 = 0..sh_lmax into `irreps_out`, C channels each, in `dtype`.
+ * Irreps strings: "0..L", "0+1+...+L", or with parity letters "0e+1o+2e+..."
+ * (natural parities only). Compiled kernels: irreps_in = irreps_out = l 0..L,
+ * sh_lmax = L, L in 0..3; C in {4, 8, 16, 32, 64, 128} (C/4 lanes own a node,
+ * at most one warp); ETP_F32. Anything else: ETP_ERR_UNSUPPORTED (a malformed
+ * string: ETP_ERR_INVALID_ARG). On success *plan is set; free it with
+ * etp_plan_destroy. Host only: needs no GPU. */
+ETP_API etp_status etp_plan_create(etp_plan_t* plan, const char* irreps_in, int sh_lmax,
+                           const char* irreps_out, int C, etp_dtype dtype);
+
+/* Plan shape. Any output pointer may be NULL. paths_l1l2l3, when given, receives
+ * 3*n_paths ints (l1, l2, l3 of each path in kernel order). Host only. */
+ETP_API etp_status etp_plan_info(etp_plan_t plan, int* n_paths, int* dim_in, int* dim_sh, int* dim_out,
+                         int* paths_l1l2l3);
+
+/* The coupling coefficients compiled into the kernels, in sparse form: for path p
+ * the entries k in [path_off[p], path_off[p+1]) couple m1[k], m2[k], m3[k]
+ * (indices 0..2l inside the l1, l2, l3 blocks) with value val[k]. Call with all
+ * arrays NULL to get *nnz; then pass path_off (n_paths+1 ints) and nnz-sized
+ * arrays. Host only. */
+ETP_API etp_status etp_plan_couplings(etp_plan_t plan, int* nnz, int* path_off, int* m1, int* m2, int* m3,
+                              double* val);
+
+/* Free a plan (NULL is accepted). */
+ETP_API etp_status etp_plan_destroy(etp_plan_t plan);
+
+/* Forward: out[i] = sum_{e in row i} msg_e (see above), for all N rows.
+ * x: [N][D][C], w: [E][P][C], r: [E][3], out: [N][D][C] device pointers.
+ * N >= 0, E >= 0; with N = 0 nothing is launched; with E = 0 out is zeroed. */
+ETP_API etp_status etp_forward(etp_plan_t plan, int N, int E, const int32_t* row_ptr, const int32_t* src,
+                       const float* r, const float* x, const float* w, float* out,
+                       etp_stream_t stream);
+
+/* Vector-Jacobian product for the cotangent grad_out = dLoss/d(out), [N][D][C]:
+ *   grad_x[j, l1 m1, c] = sum_{e: src e = j} sum_p w[e,p,c] sum_{m2,m3} CG_p Y_{l2 m2}(r_e) grad_out[dst e, l3 m3, c]
+ *   grad_w[e, p, c]     = sum_{m1,m2,m3} CG_p Y_{l2 m2}(r_e) x[src e, l1 m1, c] grad_out[dst e, l3 m3, c]
+ *   grad_r[e]           = sum_{l2 m2} dLoss/dY_{l2 m2}(e) dY_{l2 m2}/dr_e   (through Y only; r_e . grad_r[e] = 0)
+ * rev_ptr [N+1] / rev_perm [E] group the edges by source, as written by
+ * etp_build_reverse_csr; dst_of_edge [E] (may be NULL: then the row of each edge
+ * is found by binary search in row_ptr). Each of grad_x, grad_w, grad_r may be
+ * NULL to skip it. All outputs are overwritten (sources without edges get zero
+ * grad_x). */
+ETP_API etp_status etp_backward(etp_plan_t plan, int N, int E, const int32_t* row_ptr, const int32_t* src,
+                        const int32_t* rev_ptr, const int32_t* rev_perm, const int32_t* dst_of_edge,
+                        const float* r, const float* x, const float* w, const float* grad_out,
+                        float* grad_x, float* grad_w, float* grad_r, etp_stream_t stream);
+
+/* Bytes of device workspace etp_build_reverse_csr needs for (N, E). */
+ETP_API etp_status etp_reverse_csr_workspace_size(int N, int E, size_t* bytes);
+
+/* Group edges by source, stably in edge id (a counting sort; deterministic):
+ *   rev_ptr[j]..rev_ptr[j+1] indexes rev_perm, the edges with src = j in increasing id;
+ *   dst_of_edge[e] = the CSR row that holds e (may be NULL to skip).
+ * workspace: device memory of at least etp_reverse_csr_workspace_size bytes,
+ * 16-byte aligned, owned by the caller, free to reuse once the stream has passed
+ * this call. Needs a valid CSR (see etp_validate_csr). */
+ETP_API etp_status etp_build_reverse_csr(int N, int E, const int32_t* row_ptr, const int32_t* src,
+                                 int32_t* rev_ptr, int32_t* rev_perm, int32_t* dst_of_edge,
+                                 void* workspace, size_t workspace_bytes, etp_stream_t stream);
+
+/* Check a CSR on the device: zeroes *d_flag (a device int) and ORs in the
+ * ETP_CSR_* bits of every violation found. Read the flag after the stream has
+ * passed this call. */
+ETP_API etp_status etp_validate_csr(int N, int E, const int32_t* row_ptr, const int32_t* src, int32_t* d_flag,
+                            etp_stream_t stream);
+
+/* A static description of a status code. */
+ETP_API const char* etp_status_string(etp_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ETP_H_ */

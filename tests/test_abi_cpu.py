@@ -1,0 +1,127 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports every
+declared symbol, builds plans whose paths and compiled couplings agree with the
+oracle's independent construction, and rejects bad arguments before any launch.
+
+Every call below that passes pointers is built to fail a host check (a NULL, a
+negative size or a misaligned address), so no kernel is ever launched here.
+"""
+import ctypes
+
+import numpy as np
+import pytest
+
+import cg_tensor_products_b200 as etp
+from cg_tensor_products_b200 import build as etp_build
+from oracle import cg, paths
+
+
+@pytest.fixture(scope="module")
+def lib():
+    etp_build.build()
+    return etp._load()
+
+
+def test_exports_every_declared_symbol(lib):
+    names = etp.declared_symbols()
+    assert len(names) == 10
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+@pytest.mark.parametrize("L,o3", [(L, o3) for L in range(4) for o3 in (False, True)])
+def test_plan_paths_match_oracle(lib, L, o3):
+    irreps = "+".join(f"{l}{'eo'[l % 2]}" for l in range(L + 1)) if o3 else f"0..{L}"
+    plan = etp.Plan(irreps, L, irreps, 64)
+    assert plan.paths == paths.enumerate_paths(irreps, L, irreps)
+    assert plan.dim_in == plan.dim_out == (L + 1) ** 2
+
+
+@pytest.mark.parametrize("L", [1, 2, 3])
+def test_compiled_couplings_match_oracle_construction(lib, L):
+    """Racah-formula tables (library) vs invariance construction (oracle): 1e-12."""
+    plan = etp.Plan(f"0..{L}", L, f"0..{L}", 8)
+    off, m1, m2, m3, val = plan.couplings()
+    for p, (l1, l2, l3) in enumerate(plan.paths):
+        T = np.zeros((2 * l1 + 1, 2 * l2 + 1, 2 * l3 + 1))
+        for k in range(off[p], off[p + 1]):
+            T[m1[k], m2[k], m3[k]] = val[k]
+        assert np.max(np.abs(T - cg.real_cg(l1, l2, l3))) < 1e-12, (l1, l2, l3)
+        assert off[p + 1] - off[p] == len(cg.nnz_list(l1, l2, l3))
+
+
+def _create(lib, a, lmax, b, C, dtype=0):
+    h = ctypes.c_void_p()
+    st = lib.etp_plan_create(ctypes.byref(h), a.encode(), lmax, b.encode(), C, dtype)
+    if st == 0:
+        lib.etp_plan_destroy(h)
+    return st
+
+
+def test_plan_create_rejections(lib):
+    assert _create(lib, "0..3", 3, "0..3", 128) == etp.ETP_OK
+    assert _create(lib, "0+1+2", 2, "0+1+2", 64) == etp.ETP_OK
+    assert _create(lib, "0e+1o+2e+3o", 3, "0e+1o+2e+3o", 8) == etp.ETP_OK
+    for C in (4, 8, 16, 32, 64, 128):
+        assert _create(lib, "0..1", 1, "0..1", C) == etp.ETP_OK
+    unsupported = [("0..4", 4, "0..4", 8), ("0..2", 3, "0..2", 8), ("0..2", 2, "0..1", 8), ("1..2", 2, "1..2", 8),
+                   ("0..2", 2, "0..2", 12), ("0..2", 2, "0..2", 256), ("0..2", 2, "0..2", 6),
+                   ("0o+1e", 1, "0o+1e", 8), ("0+2", 2, "0+2", 8)]
+    for args in unsupported:
+        assert _create(lib, *args) == etp.ETP_ERR_UNSUPPORTED, args
+    assert _create(lib, "0..2", 2, "0..2", 8, dtype=3) == etp.ETP_ERR_UNSUPPORTED
+    invalid = [("", 1, "0..1", 8), ("0+x", 1, "0..1", 8), ("0++1", 1, "0..1", 8), ("1+0", 1, "1+0", 8),
+               ("0e+1", 1, "0e+1", 8), ("0e+1o", 1, "0+1", 8), ("0..1", -1, "0..1", 8), ("0..1", 1, "0..1", 0),
+               ("3..1", 1, "0..1", 8)]
+    for args in invalid:
+        assert _create(lib, *args) == etp.ETP_ERR_INVALID_ARG, args
+    assert lib.etp_plan_create(None, b"0..1", 1, b"0..1", 8, 0) == etp.ETP_ERR_INVALID_ARG
+
+
+def test_host_argument_checks(lib):
+    h = ctypes.c_void_p()
+    assert lib.etp_plan_create(ctypes.byref(h), b"0..2", 2, b"0..2", 64, 0) == 0
+    ok = ctypes.c_void_p(0x10000)       # never dereferenced: each call fails a host check
+    bad = ctypes.c_void_p(0x10004)      # not 16-byte aligned
+    F = lib.etp_forward
+    assert F(None, 4, 4, ok, ok, ok, ok, ok, ok, None) == etp.ETP_ERR_INVALID_ARG       # no plan
+    assert F(h, -1, 4, ok, ok, ok, ok, ok, ok, None) == etp.ETP_ERR_INVALID_ARG         # N < 0
+    assert F(h, 4, -2, ok, ok, ok, ok, ok, ok, None) == etp.ETP_ERR_INVALID_ARG         # E < 0
+    assert F(h, 0, 3, ok, ok, ok, ok, ok, ok, None) == etp.ETP_ERR_INVALID_ARG          # edges without nodes
+    assert F(h, 0, 0, None, None, None, None, None, None, None) == etp.ETP_OK           # nothing to do
+    assert F(h, 4, 4, None, ok, ok, ok, ok, ok, None) == etp.ETP_ERR_INVALID_ARG        # row_ptr NULL
+    assert F(h, 4, 4, ok, ok, ok, bad, ok, ok, None) == etp.ETP_ERR_INVALID_ARG         # x misaligned
+    assert F(h, 4, 4, ok, ok, ok, ok, bad, ok, None) == etp.ETP_ERR_INVALID_ARG         # w misaligned
+    assert F(h, 4, 4, ok, ok, ok, ok, ok, bad, None) == etp.ETP_ERR_INVALID_ARG         # out misaligned
+    assert F(h, 4, 4, ok, None, ok, ok, ok, ok, None) == etp.ETP_ERR_INVALID_ARG        # src NULL with E > 0
+    B = lib.etp_backward
+    assert B(h, 4, 4, ok, ok, None, ok, ok, ok, ok, ok, ok, ok, ok, ok, None) == etp.ETP_ERR_INVALID_ARG  # rev_ptr
+    assert B(h, 4, 4, ok, ok, ok, None, ok, ok, ok, ok, ok, ok, ok, ok, None) == etp.ETP_ERR_INVALID_ARG  # rev_perm
+    assert B(h, 4, 4, ok, ok, ok, ok, ok, ok, ok, ok, bad, ok, ok, ok, None) == etp.ETP_ERR_INVALID_ARG   # grad_out
+    assert B(h, 4, 4, ok, ok, ok, ok, ok, ok, ok, ok, ok, ok, bad, ok, None) == etp.ETP_ERR_INVALID_ARG   # grad_w
+    assert B(h, 4, 4, ok, ok, ok, ok, ok, ok, ok, ok, ok, bad, ok, ok, None) == etp.ETP_ERR_INVALID_ARG   # grad_x
+    assert B(h, 4, 4, ok, ok, ok, ok, ok, ok, ok, ok, ok, None, None, None, None) == etp.ETP_OK  # nothing wanted
+    sz = ctypes.c_size_t()
+    assert lib.etp_reverse_csr_workspace_size(10, 100, ctypes.byref(sz)) == 0 and sz.value > 0
+    assert lib.etp_reverse_csr_workspace_size(-1, 100, ctypes.byref(sz)) == etp.ETP_ERR_INVALID_ARG
+    R = lib.etp_build_reverse_csr
+    assert R(10, 100, ok, ok, ok, ok, ok, ok, sz.value - 1, None) == etp.ETP_ERR_WORKSPACE
+    assert R(10, 100, ok, ok, ok, ok, ok, bad, sz.value, None) == etp.ETP_ERR_INVALID_ARG
+    assert R(0, 5, ok, ok, ok, ok, ok, ok, sz.value, None) == etp.ETP_ERR_INVALID_ARG
+    V = lib.etp_validate_csr
+    assert V(10, 100, None, ok, ok, None) == etp.ETP_ERR_INVALID_ARG
+    assert V(10, 100, ok, ok, None, None) == etp.ETP_ERR_INVALID_ARG
+    assert lib.etp_plan_destroy(h) == 0
+    assert lib.etp_plan_destroy(None) == 0
+    for s in range(7):
+        assert lib.etp_status_string(s)
+    assert lib.etp_status_string(99) == b"unknown status"
+
+
+def test_binding_refuses_cpu_tensors(lib):
+    import torch
+
+    plan = etp.Plan("0..1", 1, "0..1", 8)
+    row_ptr = torch.zeros(3, dtype=torch.int32)
+    with pytest.raises(ValueError):
+        etp.forward(plan, row_ptr, torch.zeros(0, dtype=torch.int32), torch.zeros(0, 3),
+                    torch.zeros(2, 4, 8), torch.zeros(0, 5, 8), out=torch.zeros(2, 4, 8))

@@ -1,0 +1,179 @@
+"""GPU parity: the CUDA path (through the C ABI) against the FP64 oracle.
+
+Forward <= 1e-5 and VJP <= 1e-4 in max-normalised error per output tensor;
+reverse CSR and edge rows bit-exact. Full comparisons at sizes the oracle runs
+in seconds (several blocks, ragged tails, empty rows, isolated sources,
+duplicate edges); sampled comparisons at the full workload sizes.
+"""
+import numpy as np
+import pytest
+import torch
+
+import cg_tensor_products_b200 as etp
+import oracle
+import workloads
+from cg_tensor_products_b200 import build as etp_build
+from gpu_helpers import (check_errs, check_reverse_csr, compare_full, compare_sampled, rel_err, run_gpu, to_dev)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    etp_build.build()
+    oracle.build()
+
+
+@pytest.mark.parametrize("name", ["tiny", "micro_l2", "water"])
+def test_workload_full(name):
+    wl = workloads.make(name)
+    res = run_gpu(wl)
+    check_reverse_csr(wl, res)
+    errs = compare_full(wl, res)
+    print(name, errs)
+    check_errs(errs)
+
+
+@pytest.mark.parametrize("name", ["micro_l3", "large"])
+def test_workload_full_size_sampled(name):
+    wl = workloads.make(name)
+    res = run_gpu(wl)
+    check_reverse_csr(wl, res)
+    errs = compare_sampled(wl, res)
+    print(name, errs)
+    check_errs(errs)
+    # invariant at any size: the derivative goes through the direction only
+    r = torch.from_numpy(wl.r).cuda().double()
+    radial = (res["grad_r"].double() * r).sum(1).abs().max().item()
+    scale = (res["grad_r"].double().norm(dim=1) * r.norm(dim=1)).max().item()
+    assert radial <= 1e-5 * scale
+
+
+def test_l3_c128_reduced_full():
+    """The benchmark's shape (L = 3, C = 128, 128 neighbours) on 200 nodes: full comparison."""
+    rng = np.random.default_rng(7)
+    n, k = 200, 128
+    dst = np.repeat(np.arange(n), k)
+    src = np.concatenate([np.sort(rng.choice(n, k, replace=False)) for _ in range(n)])
+    row_ptr, src_s, order = workloads.csr_from_pairs(n, dst, src)
+    E = len(src_s)
+    wl = workloads.Workload("l3c128", 3, 128, 34, row_ptr, src_s, (2 * rng.standard_normal((E, 3))).astype(np.float32),
+                            rng.standard_normal((n, 16, 128), dtype=np.float32),
+                            (rng.standard_normal((E, 34, 128), dtype=np.float32) / np.float32(np.sqrt(34))),
+                            rng.standard_normal((n, 16, 128), dtype=np.float32))
+    res = run_gpu(wl)
+    check_reverse_csr(wl, res)
+    errs = compare_full(wl, res)
+    print(errs)
+    check_errs(errs)
+
+
+SPECS = [(L, o3, C) for L in range(4) for o3 in (False, True) for C in (4, 8, 16, 32, 64, 128)]
+
+
+@pytest.mark.parametrize("L,o3,C", SPECS)
+def test_every_compiled_spec_ragged_multigraph(L, o3, C):
+    irreps = "+".join(f"{l}{'eo'[l % 2]}" for l in range(L + 1)) if o3 else f"0..{L}"
+    P = len(oracle.paths.enumerate_paths(irreps, L, irreps))
+    rng = np.random.default_rng(100 * L + C + (7 if o3 else 0))
+    wl = workloads.random_graph(rng, 37, 300, L, C, P)
+    res = run_gpu(wl, irreps=irreps, with_dst=(C % 8 == 0))   # half the cases find rows by binary search
+    check_reverse_csr(wl, res)
+    errs = compare_full(wl, res, irreps=irreps)
+    check_errs(errs)
+    empty = np.flatnonzero(np.diff(wl.row_ptr) == 0)
+    assert len(empty) and torch.all(res["out"][torch.from_numpy(empty).cuda()] == 0)
+    iso = np.setdiff1d(np.arange(wl.N), wl.src)
+    assert len(iso) and torch.all(res["grad_x"][torch.from_numpy(iso).cuda()] == 0)
+
+
+@pytest.mark.parametrize("want", [("w",), ("r",), ("x",), ("w", "r")])
+def test_subsets_of_gradients(want):
+    rng = np.random.default_rng(3)
+    wl = workloads.random_graph(rng, 50, 400, 2, 32, 15)
+    res = run_gpu(wl, want=want)
+    full = run_gpu(wl)
+    for k, key in (("x", "grad_x"), ("w", "grad_w"), ("r", "grad_r")):
+        if k in want:
+            assert torch.equal(res[key], full[key])
+        else:
+            assert res[key] is None
+
+
+def test_no_edges():
+    n = 9
+    wl = workloads.Workload("empty", 2, 16, 15, np.zeros(n + 1, np.int32), np.zeros(0, np.int32),
+                            np.zeros((0, 3), np.float32), np.ones((n, 9, 16), np.float32),
+                            np.zeros((0, 15, 16), np.float32), np.ones((n, 9, 16), np.float32))
+    res = run_gpu(wl)
+    assert torch.all(res["out"] == 0) and torch.all(res["grad_x"] == 0)
+    assert res["grad_w"].shape == (0, 15, 16) and res["grad_r"].shape == (0, 3)
+    assert torch.all(res["rev_ptr"] == 0)
+
+
+def test_zero_length_edge_vectors():
+    rng = np.random.default_rng(4)
+    wl = workloads.random_graph(rng, 20, 120, 3, 8, 34)
+    wl.r[::7] = 0.0
+    res = run_gpu(wl)
+    check_errs(compare_full(wl, res))
+    assert torch.all(res["grad_r"][::7] == 0)
+
+
+def test_non_default_stream_and_repeat_determinism():
+    wl = workloads.random_graph(np.random.default_rng(5), 64, 2000, 3, 64, 34)
+    a = run_gpu(wl)
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        b = run_gpu(wl)
+    s.synchronize()
+    for k in ("out", "grad_x", "grad_w", "grad_r", "rev_perm"):
+        assert torch.equal(a[k], b[k]), k     # same launch shape, same order of sums
+
+
+@pytest.mark.parametrize("n,e", [(1, 0), (1, 50), (2, 7), (256, 5000), (257, 5000), (70000, 300000),
+                                 (3, 10000)])
+def test_reverse_csr_bit_exact(n, e):
+    rng = np.random.default_rng(n + e)
+    dst = rng.integers(0, n, e)
+    src = rng.integers(0, n, e)
+    row_ptr, s, _ = workloads.csr_from_pairs(n, dst, src)
+    rp, perm, d = etp.build_reverse_csr(n, torch.from_numpy(row_ptr).cuda(), torch.from_numpy(s).cuda())
+    o_rp, o_perm, o_d = oracle.reverse_csr(n, row_ptr, s)
+    assert np.array_equal(rp.cpu().numpy(), o_rp)
+    assert np.array_equal(perm.cpu().numpy(), o_perm)
+    assert np.array_equal(d.cpu().numpy(), o_d)
+
+
+def test_validate_csr_flags():
+    dev = "cuda:0"
+    rp = torch.tensor([0, 2, 3, 5], dtype=torch.int32, device=dev)
+    src = torch.tensor([1, 2, 0, 0, 1], dtype=torch.int32, device=dev)
+    assert etp.validate_csr(3, rp, src) == 0
+    assert etp.validate_csr(3, torch.tensor([1, 2, 3, 5], dtype=torch.int32, device=dev), src) & etp.CSR_BAD_ENDPOINTS
+    assert etp.validate_csr(3, torch.tensor([0, 2, 3, 4], dtype=torch.int32, device=dev), src) & etp.CSR_BAD_ENDPOINTS
+    assert etp.validate_csr(3, torch.tensor([0, 3, 2, 5], dtype=torch.int32, device=dev), src) == etp.CSR_NOT_MONOTONE
+    assert etp.validate_csr(3, rp, torch.tensor([1, 2, 3, 0, 1], dtype=torch.int32, device=dev)) == etp.CSR_SRC_RANGE
+    assert etp.validate_csr(3, rp, torch.tensor([1, -1, 0, 0, 1], dtype=torch.int32, device=dev)) == etp.CSR_SRC_RANGE
+
+
+def test_out_of_range_sources_are_skipped_not_faulted():
+    """An invalid src (caught by validate_csr) must not make the kernels leave their buffers."""
+    rng = np.random.default_rng(6)
+    wl = workloads.random_graph(rng, 16, 100, 1, 8, 5)
+    t = to_dev(wl)
+    bad_src = t["src"].clone()
+    bad_src[::9] = 1 << 20
+    plan = etp.Plan("0..1", 1, "0..1", 8)
+    assert etp.validate_csr(wl.N, t["row_ptr"], bad_src) == etp.CSR_SRC_RANGE
+    out = etp.forward(plan, t["row_ptr"], bad_src, t["r"], t["x"], t["w"])
+    torch.cuda.synchronize()
+    keep = np.ones(wl.E, bool)
+    keep[::9] = False
+    # the same graph with those edges given zero weight is the reference
+    w0 = wl.w.copy()
+    w0[~keep] = 0
+    ref = oracle.OracleTP("0..1", 1, "0..1", 8).forward(wl.row_ptr, wl.src, wl.r, wl.x, w0)
+    assert rel_err(out, ref) <= 1e-5
