@@ -47,6 +47,7 @@ def parse():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--workload", default="micro_l3", choices=sorted(DESCR))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--nodes", type=int, default=None, help="micro workloads: node count (128 neighbours each)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU seconds of the oracle baseline")
@@ -278,7 +279,7 @@ def main():
     if world > 1:
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
 
-    wl = workloads.make(args.workload)
+    wl = workloads.make(args.workload, n_nodes=args.nodes)
     plan = etp.Plan(wl.irreps, wl.L, wl.irreps, wl.C)
     nnz_total = len(plan.couplings()[1])
     N, E = wl.N, wl.E
@@ -420,7 +421,8 @@ def main():
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
         "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
         "data": "synthetic",
-        "config": {"workload": f"{args.workload}: {DESCR[args.workload]}", "N": N, "E": E, "L": wl.L, "C": wl.C,
+        "config": {"workload": f"{args.workload}: {DESCR[args.workload]}" + (f" (reduced to {N} nodes)" if args.nodes else ""),
+                   "N": N, "E": E, "L": wl.L, "C": wl.C,
                    "P": plan.n_paths, "cg_nnz": nnz_total,
                    "step": "reverse CSR + forward + VJP (grad_x, grad_w, grad_r), inputs resident in HBM",
                    "l2": f"inputs larger than L2 (w = {wl.w.nbytes / 1e9:.2f} GB streamed per pass)",

@@ -129,8 +129,8 @@ def _geometry_tiny(rng):
     return row_ptr, src_sorted, r.astype(np.float32)
 
 
-def _geometry_micro(rng):
-    n, k = 1024, 128
+def _geometry_micro(rng, n=1024):
+    k = 128
     dst = np.repeat(np.arange(n), k)
     src = np.empty(n * k, dtype=np.int64)
     for i in range(n):
@@ -210,8 +210,11 @@ def radial_mlp_weights(rng, r: np.ndarray, rc: float, P: int, C: int,
     return out.reshape(len(d), P, C)
 
 
-def make(name: str, seed: int = 0) -> Workload:
-    """Build one named workload from numpy.random.default_rng(seed)."""
+def make(name: str, seed: int = 0, n_nodes: int | None = None) -> Workload:
+    """Build one named workload from numpy.random.default_rng(seed).
+
+    n_nodes (micro workloads only) shrinks the node count, keeping 128 neighbours
+    per node (profiling captures use it to stay small)."""
     spec = SPECS[name]
     L, C = spec["L"], spec["C"]
     P = N_PATHS_SO3[L]
@@ -220,7 +223,7 @@ def make(name: str, seed: int = 0) -> Workload:
     if name == "tiny":
         row_ptr, src, r = _geometry_tiny(rng)
     elif name in ("micro_l2", "micro_l3"):
-        row_ptr, src, r = _geometry_micro(rng)
+        row_ptr, src, r = _geometry_micro(rng, n_nodes or 1024)
     elif name == "water":
         row_ptr, src, r64, rc = _geometry_water(rng)
         r = r64.astype(np.float32)
