@@ -21,7 +21,8 @@ LIB_PATH = os.path.join(_HERE, "libetp.so")
 HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "etp.h")
 
 ETP_OK, ETP_ERR_INVALID_ARG, ETP_ERR_UNSUPPORTED, ETP_ERR_BAD_CSR = 0, 1, 2, 3
-ETP_ERR_CUDA, ETP_ERR_ALLOC, ETP_ERR_WORKSPACE = 4, 5, 6
+ETP_ERR_CUDA, ETP_ERR_ALLOC, ETP_ERR_WORKSPACE, ETP_ERR_TOO_LARGE = 4, 5, 6, 7
+STATIC_MAX_NODES = STATIC_MAX_EDGES = 1 << 18
 ETP_F32 = 0
 CSR_BAD_ENDPOINTS, CSR_NOT_MONOTONE, CSR_SRC_RANGE = 1, 2, 4
 
@@ -53,6 +54,7 @@ def _load():
         "etp_backward": [vp, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp],
         "etp_reverse_csr_workspace_size": [i32, i32, ctypes.POINTER(sz)],
         "etp_build_reverse_csr": [i32, i32, vp, vp, vp, vp, vp, vp, sz, vp],
+        "etp_build_reverse_csr_static": [i32, i32, vp, vp, vp, vp, vp, vp],
         "etp_validate_csr": [i32, i32, vp, vp, vp, vp],
         "etp_status_string": [i32],
     }
@@ -198,6 +200,22 @@ def build_reverse_csr(N: int, row_ptr, src, with_dst=True, workspace=None, strea
     _check(_load().etp_build_reverse_csr(N, E, _ptr(row_ptr), _ptr(src), _ptr(rev_ptr), _ptr(rev_perm), _ptr(dst),
                                          _ptr(workspace), workspace.numel(), _stream(stream)),
            "etp_build_reverse_csr")
+    return rev_ptr, rev_perm, dst
+
+
+def build_reverse_csr_static(N: int, row_ptr, src, with_dst=True, stream=None):
+    """As build_reverse_csr, with the library's fixed device scratch instead of a workspace
+    (etp_build_reverse_csr_static; N, E <= 2^18; calls that overlap on the GPU race)."""
+    import torch
+
+    E = src.numel()
+    dev = row_ptr.device
+    rev_ptr = torch.empty(N + 1, dtype=torch.int32, device=dev)
+    rev_perm = torch.empty(E, dtype=torch.int32, device=dev)
+    dst = torch.empty(E, dtype=torch.int32, device=dev) if with_dst else None
+    _need_cuda(row_ptr, src, rev_ptr, rev_perm, dst)
+    _check(_load().etp_build_reverse_csr_static(N, E, _ptr(row_ptr), _ptr(src), _ptr(rev_ptr), _ptr(rev_perm),
+                                                _ptr(dst), _stream(stream)), "etp_build_reverse_csr_static")
     return rev_ptr, rev_perm, dst
 
 

@@ -300,6 +300,7 @@ const char* etp_status_string(etp_status status) {
         case ETP_ERR_CUDA: return "CUDA launch or runtime error";
         case ETP_ERR_ALLOC: return "host allocation failed";
         case ETP_ERR_WORKSPACE: return "workspace too small";
+        case ETP_ERR_TOO_LARGE: return "N or E above the fixed scratch limit of the static-scratch variant";
     }
     return "unknown status";
 }

@@ -19,7 +19,7 @@
 namespace etp {
 namespace {
 
-constexpr int kTile = 4096;
+constexpr int kTile = kRadixTile;
 constexpr int kScanThreads = 1024;
 
 __global__ void count_sources(const int32_t* __restrict__ src, int E, int N, int32_t* __restrict__ cnt) {
@@ -172,14 +172,7 @@ inline int radix_passes(int N) {
 
 }  // namespace
 
-size_t reverse_csr_workspace_bytes(int N, int E) {
-    const int n_tiles = (E + kTile - 1) / kTile;
-    size_t b = 0;
-    b += align16(sizeof(int32_t) * ((size_t)N + 1));      // counts
-    b += 3 * align16(sizeof(int32_t) * (size_t)E);        // keys ping-pong + spare values
-    b += align16(sizeof(int32_t) * (256 * (size_t)n_tiles + 1));  // tile histograms (+ total)
-    return b;
-}
+size_t reverse_csr_workspace_bytes(int N, int E) { return reverse_csr_workspace_bytes_for(N, E); }
 
 cudaError_t build_reverse_csr(int N, int E, const int32_t* row_ptr, const int32_t* src, int32_t* rev_ptr,
                               int32_t* rev_perm, int32_t* dst, void* ws, cudaStream_t s) {

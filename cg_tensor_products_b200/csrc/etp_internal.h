@@ -45,6 +45,15 @@ cudaError_t launch_forward(bool o3, const FwdArgs& a, dim3 grid, cudaStream_t s)
 template <int L>
 cudaError_t launch_backward(bool o3, const BwdArgs& a, dim3 grid, cudaStream_t s);
 
+// Reverse CSR workspace: per-source counts, two key buffers, one value buffer,
+// and the digit-major table of per-tile histograms (tiles of kRadixTile edges).
+constexpr int kRadixTile = 4096;
+constexpr size_t align16_bytes(size_t b) { return (b + 15) & ~size_t(15); }
+constexpr size_t reverse_csr_workspace_bytes_for(long long N, long long E) {
+    return align16_bytes(4 * (size_t)(N + 1)) + 3 * align16_bytes(4 * (size_t)E) +
+           align16_bytes(4 * (256 * (size_t)((E + kRadixTile - 1) / kRadixTile) + 1));
+}
+
 size_t reverse_csr_workspace_bytes(int N, int E);
 cudaError_t build_reverse_csr(int N, int E, const int32_t* row_ptr, const int32_t* src, int32_t* rev_ptr,
                               int32_t* rev_perm, int32_t* dst, void* ws, cudaStream_t s);

@@ -89,7 +89,8 @@ typedef enum {
     ETP_ERR_BAD_CSR = 3,     /* reserved for callers that map the validation flag      */
     ETP_ERR_CUDA = 4,        /* a CUDA launch or query failed                           */
     ETP_ERR_ALLOC = 5,       /* host allocation of a plan failed                        */
-    ETP_ERR_WORKSPACE = 6    /* workspace smaller than etp_reverse_csr_workspace_size   */
+    ETP_ERR_WORKSPACE = 6,   /* workspace smaller than etp_reverse_csr_workspace_size   */
+    ETP_ERR_TOO_LARGE = 7    /* N or E above the fixed scratch of the _static variant   */
 } etp_status;
 
 /* Bits of the flag written by etp_validate_csr. */
@@ -157,6 +158,30 @@ ETP_API etp_status etp_reverse_csr_workspace_size(int N, int E, size_t* bytes);
 ETP_API etp_status etp_build_reverse_csr(int N, int E, const int32_t* row_ptr, const int32_t* src,
                                  int32_t* rev_ptr, int32_t* rev_perm, int32_t* dst_of_edge,
                                  void* workspace, size_t workspace_bytes, etp_stream_t stream);
+
+/* Limits of etp_build_reverse_csr_static and the size of its scratch array. */
+#define ETP_STATIC_MAX_NODES (1 << 18)
+#define ETP_STATIC_MAX_EDGES (1 << 18)
+#define ETP_STATIC_SCRATCH_BYTES 4259872 /* device bytes held on every GPU that loads the library */
+
+/* etp_build_reverse_csr without a workspace argument and without allocating:
+ * for callers that cannot allocate device memory where they need the reverse
+ * CSR (a plugin inside a host program that owns the GPU memory budget, or a
+ * time-critical loop that must not call cudaMalloc, which may synchronise the
+ * device). The pages have no counterpart of this call; it is a deployment
+ * convenience of this library.
+ * Same arguments, outputs and result as etp_build_reverse_csr. The scratch is a
+ * fixed file-scope device array of ETP_STATIC_SCRATCH_BYTES, present on every GPU
+ * that loads the library until the process exits. N > ETP_STATIC_MAX_NODES or
+ * E > ETP_STATIC_MAX_EDGES returns ETP_ERR_TOO_LARGE before any launch. The
+ * first call on a device (the current device) looks up the array's device
+ * address for that device; make that first call before any stream capture on
+ * it. All calls share the one array: calls whose work overlaps on the GPU
+ * (unordered streams or threads) race and give wrong results; calls ordered on
+ * one stream are safe. */
+ETP_API etp_status etp_build_reverse_csr_static(int N, int E, const int32_t* row_ptr, const int32_t* src,
+                                                int32_t* rev_ptr, int32_t* rev_perm, int32_t* dst_of_edge,
+                                                etp_stream_t stream);
 
 /* Check a CSR on the device: zeroes *d_flag (a device int) and ORs in the
  * ETP_CSR_* bits of every violation found. Read the flag after the stream has

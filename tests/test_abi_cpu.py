@@ -23,7 +23,7 @@ def lib():
 
 def test_exports_every_declared_symbol(lib):
     names = etp.declared_symbols()
-    assert len(names) == 10
+    assert len(names) == 11
     for n in names:
         assert hasattr(lib, n), n
 
@@ -107,12 +107,17 @@ def test_host_argument_checks(lib):
     assert R(10, 100, ok, ok, ok, ok, ok, ok, sz.value - 1, None) == etp.ETP_ERR_WORKSPACE
     assert R(10, 100, ok, ok, ok, ok, ok, bad, sz.value, None) == etp.ETP_ERR_INVALID_ARG
     assert R(0, 5, ok, ok, ok, ok, ok, ok, sz.value, None) == etp.ETP_ERR_INVALID_ARG
+    S = lib.etp_build_reverse_csr_static
+    assert S(10, (1 << 18) + 1, ok, ok, ok, ok, ok, None) == etp.ETP_ERR_TOO_LARGE
+    assert S((1 << 18) + 1, 10, ok, ok, ok, ok, ok, None) == etp.ETP_ERR_TOO_LARGE
+    assert S(10, 100, ok, ok, ctypes.c_void_p(0x10002), ok, ok, None) == etp.ETP_ERR_INVALID_ARG  # rev_ptr
+    assert S(-1, 100, ok, ok, ok, ok, ok, None) == etp.ETP_ERR_INVALID_ARG
     V = lib.etp_validate_csr
     assert V(10, 100, None, ok, ok, None) == etp.ETP_ERR_INVALID_ARG
     assert V(10, 100, ok, ok, None, None) == etp.ETP_ERR_INVALID_ARG
     assert lib.etp_plan_destroy(h) == 0
     assert lib.etp_plan_destroy(None) == 0
-    for s in range(7):
+    for s in range(8):
         assert lib.etp_status_string(s)
     assert lib.etp_status_string(99) == b"unknown status"
 
