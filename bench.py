@@ -37,7 +37,7 @@ DESCR = {
     "water": "3072-atom water box, r_c = 5 A radius graph, L=2, C=64, 15 paths",
     "large": "32768 atoms at 0.1/A^3, r_c = 4.5 A radius graph, L=3, C=64, 34 paths",
 }
-KERNEL_SOURCES = ["cg_tensor_products_b200/csrc/etp_kernels.cuh", "cg_tensor_products_b200/csrc/etp_device.cuh"]
+KERNEL_SOURCES = ["cg_tensor_products_b200/csrc/etp_frame.cuh", "cg_tensor_products_b200/csrc/etp_device.cuh"]
 
 
 def parse():

@@ -18,8 +18,9 @@ struct FwdArgs {
     const float4* x;
     const float4* w;
     float4* out;
-    int C4;    // C / 4
-    int team;  // lanes per node = C4 (power of two, <= 32)
+    int C4;      // C / 4
+    int team;    // lanes per team = min(32, C/2), a power of two
+    int slices;  // teams per node = C / (2 team): 1, or 2 when C = 128
 };
 
 struct BwdArgs {
@@ -38,12 +39,21 @@ struct BwdArgs {
     float* grad_r;   // may be null
     int C4;
     int team;
+    int slices;
 };
 
+// Launch geometry shared by the forward and backward kernels: teams of
+// min(32, C/2) lanes, each lane two channels; C/(2 team) teams per node.
+struct LaunchShape {
+    int team, slices, nodes_per_block;
+    size_t smem_bytes;
+};
+LaunchShape launch_shape(int C, int N);
+
 template <int L>
-cudaError_t launch_forward(bool o3, const FwdArgs& a, dim3 grid, cudaStream_t s);
+cudaError_t launch_forward(bool o3, const FwdArgs& a, dim3 grid, size_t smem, cudaStream_t s);
 template <int L>
-cudaError_t launch_backward(bool o3, const BwdArgs& a, dim3 grid, cudaStream_t s);
+cudaError_t launch_backward(bool o3, const BwdArgs& a, dim3 grid, size_t smem, cudaStream_t s);
 
 // Reverse CSR workspace: per-source counts, two key buffers, one value buffer,
 // and the digit-major table of per-tile histograms (tiles of kRadixTile edges).

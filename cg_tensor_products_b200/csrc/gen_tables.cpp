@@ -26,6 +26,20 @@
 //
 // The output header lists, for every (l1, l2, l3) with l <= kLmax on the SO(3)
 // triangle, the nonzero entries (m1, m2, m3, value) with indices 0..2l.
+//
+// It also writes the tables of the edge-aligned frame used by the kernels. For
+// an edge with unit vector u, a rotation R with R u = z maps the harmonics to
+// Y(z) = sqrt(2l+1) delta_{m,0}; by the equivariance of every coupling,
+//   CG_p(x, Y(u)) = D_l3(R)^T B_p D_l1(R) x,   B_p[m3, m1] = sqrt(2 l2 + 1) CG_p[m1, 0, m3],
+// and B_p is nonzero only at m1 = m3 (l1+l2+l3 even) or m1 = -m3 (odd), with
+// B_p[m, m] = B_p[-m, -m] = b_p(|m|) (even) or B_p[mu, -mu] = -B_p[-mu, mu] = b_p(mu)
+// (odd). Written: b_p(mu) for mu = 0..min(l1, l3); the real-basis rotation
+// generators J_x, J_y (d/de Y(exp(e [a]x) r) = J_a Y(r)), obtained from the
+// Condon-Shortley ladder operators, (a x r).grad = i a.L, L_+- Y^m =
+// sqrt((l -+ m)(l +- m + 1)) Y^(m+-1), through the same change of basis; and, for
+// the Wigner matrices D_l(R) (Y_l(R r) = D_l(R) Y_l(r)), 7 fixed unit vectors p_k
+// and A_l^-1 with A_l = [Y_l(p_1) .. Y_l(p_2l+1)], so that
+// D_l(R) = [Y_l(R p_1) .. Y_l(R p_2l+1)] A_l^-1.
 #include <cmath>
 #include <complex>
 #include <cstdio>
@@ -152,6 +166,99 @@ std::vector<Nz> real_cg(int l1, int l2, int l3) {
     return out;
 }
 
+// ---------------------------------------------------------------------------
+// Real spherical harmonics of a unit vector (component normalisation, no
+// Condon-Shortley phase), long double: Y_lm = K_lm Pi_l^|m|(z) {Re,1,Im}(x+iy)^|m|.
+std::vector<ld> real_sh(int L, ld x, ld y, ld z) {
+    std::vector<ld> Y((L + 1) * (L + 1));
+    std::vector<ld> Cm(L + 1), Sm(L + 1);
+    Cm[0] = 1;
+    Sm[0] = 0;
+    for (int m = 1; m <= L; ++m) {
+        Cm[m] = x * Cm[m - 1] - y * Sm[m - 1];
+        Sm[m] = x * Sm[m - 1] + y * Cm[m - 1];
+    }
+    std::vector<std::vector<ld>> Pi(L + 1, std::vector<ld>(L + 1, 0));
+    for (int m = 0; m <= L; ++m) {
+        ld df = 1;
+        for (int k = 2 * m - 1; k > 1; k -= 2) df *= k;
+        Pi[m][m] = df;
+        if (m + 1 <= L) Pi[m + 1][m] = (2 * m + 1) * z * Pi[m][m];
+        for (int l = m + 2; l <= L; ++l) Pi[l][m] = ((2 * l - 1) * z * Pi[l - 1][m] - (l + m - 1) * Pi[l - 2][m]) / (l - m);
+    }
+    for (int l = 0; l <= L; ++l)
+        for (int m = -l; m <= l; ++m) {
+            int mu = std::abs(m);
+            ld k = std::sqrt((2 * l + 1) * fact(l - mu) / fact(l + mu)) * (mu ? std::sqrt((ld)2) : 1);
+            ld az = m > 0 ? Cm[mu] : (m < 0 ? Sm[mu] : 1);
+            Y[l * l + l + m] = k * Pi[l][mu] * az;
+        }
+    return Y;
+}
+
+// Gauss-Jordan inverse with partial pivoting (n <= 7).
+bool invert(std::vector<ld>& A, int n) {
+    std::vector<ld> I(n * n, 0);
+    for (int i = 0; i < n; ++i) I[i * n + i] = 1;
+    for (int c = 0; c < n; ++c) {
+        int piv = c;
+        for (int r = c + 1; r < n; ++r)
+            if (std::fabs(A[r * n + c]) > std::fabs(A[piv * n + c])) piv = r;
+        if (std::fabs(A[piv * n + c]) < 1e-12L) return false;
+        for (int k = 0; k < n; ++k) {
+            std::swap(A[c * n + k], A[piv * n + k]);
+            std::swap(I[c * n + k], I[piv * n + k]);
+        }
+        ld d = A[c * n + c];
+        for (int k = 0; k < n; ++k) {
+            A[c * n + k] /= d;
+            I[c * n + k] /= d;
+        }
+        for (int r = 0; r < n; ++r)
+            if (r != c) {
+                ld f = A[r * n + c];
+                for (int k = 0; k < n; ++k) {
+                    A[r * n + k] -= f * A[c * n + k];
+                    I[r * n + k] -= f * I[c * n + k];
+                }
+            }
+    }
+    A = I;
+    return true;
+}
+
+// Real-basis generator J_a (a = 0: x, 1: y) of degree l: U J^C U^dagger with
+// J^C_x[m, m+-1] = (i/2) c_+-(m), J^C_y[m, m+1] = c_+(m)/2, J^C_y[m, m-1] = -c_-(m)/2.
+std::vector<ld> real_generator(int l, int axis) {
+    int d = 2 * l + 1;
+    std::vector<cld> Jc(d * d, cld(0, 0));
+    for (int m = -l; m <= l; ++m) {
+        ld cp = std::sqrt((ld)(l - m) * (l + m + 1)), cm = std::sqrt((ld)(l + m) * (l - m + 1));
+        if (m + 1 <= l) Jc[(m + l) * d + (m + 1 + l)] = axis == 0 ? cld(0, cp / 2) : cld(cp / 2, 0);
+        if (m - 1 >= -l) Jc[(m + l) * d + (m - 1 + l)] = axis == 0 ? cld(0, cm / 2) : cld(-cm / 2, 0);
+    }
+    auto U = real_from_complex(l);
+    std::vector<ld> J(d * d);
+    for (int a = 0; a < d; ++a)
+        for (int b = 0; b < d; ++b) {
+            cld acc(0, 0);
+            for (int i = 0; i < d; ++i)
+                for (int j = 0; j < d; ++j) acc += U[a * d + i] * Jc[i * d + j] * std::conj(U[b * d + j]);
+            if (std::fabs(acc.imag()) > 1e-15L) {
+                std::fprintf(stderr, "generator l=%d axis=%d is not real\n", l, axis);
+                std::exit(1);
+            }
+            J[a * d + b] = std::fabs(acc.real()) < 1e-15L ? 0 : acc.real();
+        }
+    for (int a = 0; a < d; ++a)
+        for (int b = 0; b < d; ++b)
+            if (std::fabs(J[a * d + b] + J[b * d + a]) > 1e-15L) {
+                std::fprintf(stderr, "generator l=%d axis=%d is not antisymmetric\n", l, axis);
+                std::exit(1);
+            }
+    return J;
+}
+
 }  // namespace
 
 int main(int argc, char** argv) {
@@ -191,6 +298,134 @@ int main(int argc, char** argv) {
                 for (int c = 0; c <= kLmax; ++c)
                     std::fprintf(f, "%d%s", pass ? cnt[a][b][c] : off[a][b][c], c < kLmax ? ", " : "");
                 std::fprintf(f, "}%s", b < kLmax ? ", " : "");
+            }
+            std::fprintf(f, "},\n");
+        }
+        std::fprintf(f, "};\n\n");
+    }
+    // --- edge-aligned frame: b_p(mu) --------------------------------------
+    std::fprintf(f, "// b[l1][l2][l3][mu]: the m2 = 0 slice of the coupling in the edge frame (see gen_tables.cpp)\n");
+    std::fprintf(f, "constexpr double kFrameB[%d][%d][%d][%d] = {\n", kLmax + 1, kLmax + 1, kLmax + 1, kLmax + 1);
+    for (int a = 0; a <= kLmax; ++a) {
+        std::fprintf(f, "    {");
+        for (int b = 0; b <= kLmax; ++b) {
+            std::fprintf(f, "{");
+            for (int c = 0; c <= kLmax; ++c) {
+                std::vector<ld> dense((2 * a + 1) * (2 * b + 1) * (2 * c + 1), 0);
+                int d2 = 2 * b + 1, d3 = 2 * c + 1;
+                for (auto& z : real_cg(a, b, c)) dense[(z.m1 * d2 + z.m2) * d3 + z.m3] = z.v;
+                auto at = [&](int m1, int m3) { return dense[((m1 + a) * d2 + b) * d3 + (m3 + c)] * std::sqrt((ld)(2 * b + 1)); };
+                const bool odd = (a + b + c) % 2 == 1;
+                const int mn = a < c ? a : c;
+                // structure check: B nonzero only at m1 = +-m3 with the stated symmetry
+                for (int m1 = -a; m1 <= a; ++m1)
+                    for (int m3 = -c; m3 <= c; ++m3) {
+                        ld v = at(m1, m3);
+                        bool allowed = odd ? (m1 == -m3 && m3 != 0) : (m1 == m3);
+                        if (!allowed && std::fabs(v) > 1e-15L) {
+                            std::fprintf(stderr, "frame coupling (%d,%d,%d) has an entry off its pattern\n", a, b, c);
+                            return 1;
+                        }
+                    }
+                std::fprintf(f, "{");
+                for (int mu = 0; mu <= kLmax; ++mu) {
+                    ld v = 0;
+                    if (mu <= mn && !(c < std::abs(a - b) || c > a + b)) {
+                        if (!odd) {
+                            v = at(mu, mu);
+                            if (std::fabs(at(-mu, -mu) - v) > 1e-15L) { std::fprintf(stderr, "even symmetry\n"); return 1; }
+                        } else if (mu > 0) {
+                            v = at(-mu, mu);
+                            if (std::fabs(at(mu, -mu) + v) > 1e-15L) { std::fprintf(stderr, "odd symmetry\n"); return 1; }
+                        }
+                    }
+                    std::fprintf(f, "%.21Lg%s", v, mu < kLmax ? ", " : "");
+                }
+                std::fprintf(f, "}%s", c < kLmax ? ", " : "");
+            }
+            std::fprintf(f, "}%s", b < kLmax ? ", " : "");
+        }
+        std::fprintf(f, "},\n");
+    }
+    std::fprintf(f, "};\n\n");
+    // --- generators J_x, J_y -------------------------------------------------
+    std::fprintf(f, "// kGen[axis][l][a][b]: real-basis rotation generators (axis 0: x, 1: y), d/de Y(exp(e[a]x) r) = J Y(r)\n");
+    std::fprintf(f, "constexpr double kGen[2][%d][7][7] = {\n", kLmax + 1);
+    for (int ax = 0; ax < 2; ++ax) {
+        std::fprintf(f, "    {");
+        for (int l = 0; l <= kLmax; ++l) {
+            auto J = real_generator(l, ax);
+            int d = 2 * l + 1;
+            std::fprintf(f, "{");
+            for (int a = 0; a < 7; ++a) {
+                std::fprintf(f, "{");
+                for (int b = 0; b < 7; ++b) std::fprintf(f, "%.21Lg%s", (a < d && b < d) ? J[a * d + b] : (ld)0, b < 6 ? ", " : "");
+                std::fprintf(f, "}%s", a < 6 ? ", " : "");
+            }
+            std::fprintf(f, "}%s", l < kLmax ? ", " : "");
+        }
+        std::fprintf(f, "},\n");
+    }
+    std::fprintf(f, "};\n\n");
+    // --- Wigner fitting points and inverses ---------------------------------
+    {
+        unsigned long long st = 0x9E3779B97F4A7C15ull;
+        auto uni = [&]() {
+            st = st * 6364136223846793005ull + 1442695040888963407ull;
+            return (ld)((st >> 11) & ((1ull << 53) - 1)) / (ld)(1ull << 53);
+        };
+        ld best = 1e300L;
+        std::vector<ld> best_pts, best_inv[kLmax + 1];
+        for (int trial = 0; trial < 4000; ++trial) {
+            std::vector<ld> pts(3 * 7);
+            for (int k = 0; k < 7; ++k) {
+                ld zz = 2 * uni() - 1, ph = 2 * 3.14159265358979323846264338327950288L * uni();
+                ld rr = std::sqrt(1 - zz * zz);
+                pts[3 * k] = rr * std::cos(ph);
+                pts[3 * k + 1] = rr * std::sin(ph);
+                pts[3 * k + 2] = zz;
+            }
+            ld worst = 0;
+            std::vector<ld> inv[kLmax + 1];
+            bool ok = true;
+            for (int l = 2; l <= kLmax && ok; ++l) {
+                int d = 2 * l + 1;
+                std::vector<ld> A(d * d);
+                for (int k = 0; k < d; ++k) {
+                    auto Y = real_sh(l, pts[3 * k], pts[3 * k + 1], pts[3 * k + 2]);
+                    for (int m = 0; m < d; ++m) A[m * d + k] = Y[l * l + m];  // column k = Y_l(p_k)
+                }
+                ld na = 0;
+                for (auto v : A) na += v * v;
+                std::vector<ld> Ai = A;
+                if (!invert(Ai, d)) { ok = false; break; }
+                ld ni = 0;
+                for (auto v : Ai) ni += v * v;
+                ld cond = std::sqrt(na * ni);
+                if (cond > worst) worst = cond;
+                inv[l] = Ai;
+            }
+            if (ok && worst < best) {
+                best = worst;
+                best_pts = pts;
+                for (int l = 2; l <= kLmax; ++l) best_inv[l] = inv[l];
+            }
+        }
+        std::fprintf(f, "// Wigner matrices by fitting: D_l(R) = [Y_l(R p_1) .. Y_l(R p_2l+1)] A_l^-1 (Frobenius condition %.3Lf)\n", best);
+        std::fprintf(f, "constexpr double kFitPoints[7][3] = {\n");
+        for (int k = 0; k < 7; ++k)
+            std::fprintf(f, "    {%.21Lg, %.21Lg, %.21Lg},\n", best_pts[3 * k], best_pts[3 * k + 1], best_pts[3 * k + 2]);
+        std::fprintf(f, "};\n");
+        std::fprintf(f, "// kFitInv[l][k][b] = (A_l^-1)[k][b], zero-padded to 7 x 7 (l = 2, 3; rows 0, 1 unused)\n");
+        std::fprintf(f, "constexpr double kFitInv[%d][7][7] = {\n", kLmax + 1);
+        for (int l = 0; l <= kLmax; ++l) {
+            int d = 2 * l + 1;
+            std::fprintf(f, "    {");
+            for (int k = 0; k < 7; ++k) {
+                std::fprintf(f, "{");
+                for (int b = 0; b < 7; ++b)
+                    std::fprintf(f, "%.21Lg%s", (l >= 2 && k < d && b < d) ? best_inv[l][k * d + b] : (ld)0, b < 6 ? ", " : "");
+                std::fprintf(f, "}%s", k < 6 ? ", " : "");
             }
             std::fprintf(f, "},\n");
         }
