@@ -111,9 +111,6 @@ bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0
 
 etp_status cuda_status(cudaError_t e) { return e == cudaSuccess ? ETP_OK : ETP_ERR_CUDA; }
 
-dim3 node_grid(int N, const etp::LaunchShape& sh) {
-    return dim3((unsigned)((N + sh.nodes_per_block - 1) / sh.nodes_per_block), 1, 1);
-}
 
 }  // namespace
 
@@ -199,17 +196,18 @@ etp_status etp_forward(etp_plan_t plan, int N, int E, const int32_t* row_ptr, co
     if (N == 0) return E == 0 ? ETP_OK : ETP_ERR_INVALID_ARG;
     if (!row_ptr || !x || !out || !aligned4(row_ptr) || !aligned16(x) || !aligned16(out)) return ETP_ERR_INVALID_ARG;
     if (E > 0 && (!src || !r || !w || !aligned4(src) || !aligned4(r) || !aligned16(w))) return ETP_ERR_INVALID_ARG;
-    const etp::LaunchShape sh = etp::launch_shape(plan->C, N);
-    etp::FwdArgs a{N, E, row_ptr, src, r, reinterpret_cast<const float4*>(x), reinterpret_cast<const float4*>(w),
-                   reinterpret_cast<float4*>(out), plan->C / 4, sh.team, sh.slices};
-    const dim3 grid = node_grid(N, sh);
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    cudaError_t err;
+    // rows cut by a task boundary are reduced onto zeros; empty rows stay zero
+    cudaError_t err = cudaMemsetAsync(out, 0, sizeof(float) * (size_t)N * plan->D * plan->C, s);
+    if (err != cudaSuccess || E == 0) return cuda_status(err);
+    const etp::LaunchShape sh = etp::launch_shape(plan->C, plan->L, plan->o3, false, E, N);
+    etp::FwdArgs a{N, E, row_ptr, src, r, reinterpret_cast<const float4*>(x), reinterpret_cast<const float4*>(w),
+                   reinterpret_cast<float4*>(out), plan->C / 4, sh.team, sh.slices, sh.ntasks};
     switch (plan->L) {
-        case 0: err = etp::launch_forward<0>(plan->o3, a, grid, sh.smem_bytes, s); break;
-        case 1: err = etp::launch_forward<1>(plan->o3, a, grid, sh.smem_bytes, s); break;
-        case 2: err = etp::launch_forward<2>(plan->o3, a, grid, sh.smem_bytes, s); break;
-        default: err = etp::launch_forward<3>(plan->o3, a, grid, sh.smem_bytes, s); break;
+        case 0: err = etp::launch_forward<0>(plan->o3, a, sh.grid, sh.smem_bytes, s); break;
+        case 1: err = etp::launch_forward<1>(plan->o3, a, sh.grid, sh.smem_bytes, s); break;
+        case 2: err = etp::launch_forward<2>(plan->o3, a, sh.grid, sh.smem_bytes, s); break;
+        default: err = etp::launch_forward<3>(plan->o3, a, sh.grid, sh.smem_bytes, s); break;
     }
     return cuda_status(err);
 }
@@ -235,6 +233,12 @@ etp_status etp_backward(etp_plan_t plan, int N, int E, const int32_t* row_ptr, c
         grad_r = nullptr;
     }
     if (!grad_x && !grad_w && !grad_r) return ETP_OK;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t err = cudaSuccess;
+    // source rows cut by a task boundary are reduced onto zeros; sources without edges stay zero
+    if (grad_x) err = cudaMemsetAsync(grad_x, 0, sizeof(float) * (size_t)N * plan->D * plan->C, s);
+    if (err != cudaSuccess || E == 0) return cuda_status(err);
+    const etp::LaunchShape sh = etp::launch_shape(plan->C, plan->L, plan->o3, true, E, N);
     etp::BwdArgs a{N,
                    E,
                    row_ptr,
@@ -250,19 +254,14 @@ etp_status etp_backward(etp_plan_t plan, int N, int E, const int32_t* row_ptr, c
                    reinterpret_cast<float4*>(grad_w),
                    grad_r,
                    plan->C / 4,
-                   0,
-                   0};
-    const etp::LaunchShape sh = etp::launch_shape(plan->C, N);
-    a.team = sh.team;
-    a.slices = sh.slices;
-    const dim3 grid = node_grid(N, sh);
-    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    cudaError_t err;
+                   sh.team,
+                   sh.slices,
+                   sh.ntasks};
     switch (plan->L) {
-        case 0: err = etp::launch_backward<0>(plan->o3, a, grid, sh.smem_bytes, s); break;
-        case 1: err = etp::launch_backward<1>(plan->o3, a, grid, sh.smem_bytes, s); break;
-        case 2: err = etp::launch_backward<2>(plan->o3, a, grid, sh.smem_bytes, s); break;
-        default: err = etp::launch_backward<3>(plan->o3, a, grid, sh.smem_bytes, s); break;
+        case 0: err = etp::launch_backward<0>(plan->o3, a, sh.grid, sh.smem_bytes, s); break;
+        case 1: err = etp::launch_backward<1>(plan->o3, a, sh.grid, sh.smem_bytes, s); break;
+        case 2: err = etp::launch_backward<2>(plan->o3, a, sh.grid, sh.smem_bytes, s); break;
+        default: err = etp::launch_backward<3>(plan->o3, a, sh.grid, sh.smem_bytes, s); break;
     }
     return cuda_status(err);
 }

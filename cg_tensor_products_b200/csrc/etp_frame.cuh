@@ -52,7 +52,7 @@ __device__ __forceinline__ int row_of_edge(const int32_t* __restrict__ row_ptr, 
 
 namespace frame {
 
-constexpr int kThreads = kThreadsPerBlock;  // 4 warps
+constexpr int kThreads = kThreadsPerBlock;  // 2 warps
 constexpr int kYbufFloats = 7 * 12;         // harmonics l = 2, 3 at the 7 fitting points
 constexpr int kDbufFloats = 96;             // D_2 (5 rows x 8) then D_3 (7 rows x 8)
 constexpr int kTeamFloats = kYbufFloats + kDbufFloats;
@@ -61,6 +61,15 @@ constexpr int kFitStride = 128;             // shared-memory floats reserved for
 // Team buffers are read with 16-byte vector loads: every offset must keep 16-byte alignment.
 static_assert(kFitStride >= kFitFloats && kFitStride % 4 == 0, "fit table stride");
 static_assert(kYbufFloats % 4 == 0 && kTeamFloats % 4 == 0, "team buffer alignment");
+constexpr int kHeaderFloats = kFitStride + 8;  // fit table, then the grad_r slice partials
+constexpr int kRingFwd = 24;                   // weight-ring slots (paths) per team, forward
+constexpr int kRingBwd = 8;                    // and backward (its node rows take more room)
+// Floats of one team's shared buffers: harmonics and Wigner matrices, `rows`
+// node-row buffers of D x T float2, and the weight ring.
+constexpr int team_floats(int D, int T, int rows, int ring) {
+    return kTeamFloats + rows * D * T * 2 + ring * T * 2;
+}
+static_assert(kHeaderFloats % 4 == 0, "header alignment");
 
 // ---------------------------------------------------------------------------
 // compile-time tables
@@ -114,13 +123,6 @@ __device__ __forceinline__ float4 lds4(const float* p) {
     return v;
 }
 
-__device__ __forceinline__ float2 ld_stream2(const float2* p, uint64_t pol) {
-    float2 v;
-    asm("ld.global.nc.L1::no_allocate.L2::cache_hint.v2.f32 {%0, %1}, [%2], %3;"
-        : "=f"(v.x), "=f"(v.y)
-        : "l"(p), "l"(pol));
-    return v;
-}
 __device__ __forceinline__ void st_stream2(float2* p, float2 v, uint64_t pol) {
     asm volatile("st.global.L2::cache_hint.v2.f32 [%0], {%1, %2}, %3;" ::"l"(p), "f"(v.x), "f"(v.y), "l"(pol)
                  : "memory");
@@ -257,12 +259,146 @@ __device__ __forceinline__ void rotate_all(const Frame& f, const float* dbuf, co
     });
 }
 
+// ---------------------------------------------------------------------------
+// Streaming of the per-edge weights: every lane copies its own two channels of
+// each path into a ring of shared-memory slots with cp.async, a fixed number of
+// paths (DIST) ahead of their use, in the order the kernels consume them
+// (l3 outer, l1, l2 inner). Each consumption step issues one copy group and
+// waits until the group holding the step's own path has landed, so that DIST
+// copies stay in flight without holding registers. A lane reads back only what
+// it copied itself, so no cross-lane synchronisation is needed. The next edge's
+// node row (x for the forward, grad_out for the backward) rides in the group of
+// the first step of the current edge.
+__device__ __forceinline__ unsigned smem_u32(const void* p) { return (unsigned)__cvta_generic_to_shared(p); }
+__device__ __forceinline__ void cp_async8(const void* smem, const void* gmem) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(smem_u32(smem)), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+__device__ __forceinline__ float2 lds2(const float2* p) {
+    float2 v;
+    asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(smem_u32(p)));
+    return v;
+}
+
+// Consumption order of the paths within an edge (l3 outer, l1, l2 inner).
+template <int L, bool O3>
+struct Order {
+    static constexpr int P = PathSet<L, O3>::P;
+    static constexpr int path_at(int k) {
+        int n = 0;
+        for (int c = 0; c <= L; ++c)
+            for (int a = 0; a <= L; ++a)
+                for (int b = 0; b <= L; ++b)
+                    if (PathSet<L, O3>::allowed(a, b, c)) {
+                        if (n == k) return path_index<L, O3>(a, b, c);
+                        ++n;
+                    }
+        return -1;
+    }
+    static constexpr int pos(int l1, int l2, int l3) {
+        int n = 0;
+        for (int c = 0; c <= L; ++c)
+            for (int a = 0; a <= L; ++a)
+                for (int b = 0; b <= L; ++b)
+                    if (PathSet<L, O3>::allowed(a, b, c)) {
+                        if (a == l1 && b == l2 && c == l3) return n;
+                        ++n;
+                    }
+        return -1;
+    }
+};
+
+// Parts of an edge's weights in consumption order: NQ parts of PP paths. PP is
+// odd, so the lane-major slots (lane t's paths at t * PP + k) are read and
+// written without shared-memory bank conflicts.
+template <int L, bool O3>
+struct Parts {
+    static constexpr int P = PathSet<L, O3>::P;
+    static constexpr int NQ0 = P < 4 ? P : 4;
+    static constexpr int PP = ((P + NQ0 - 1) / NQ0) | 1;
+    static constexpr int NQ = (P + PP - 1) / PP;
+    static constexpr int begin(int q) { return q * PP; }
+    static constexpr int end(int q) { return (q + 1) * PP < P ? (q + 1) * PP : P; }
+    static constexpr int ring_float2(int T) { return (NQ + 1) * PP * T; }
+};
+
+// The weight pipe of one team: a ring of NQ + 1 part slots. Part q of the next
+// edge is issued when part q of the current edge starts (one edge of lead), into
+// the slot the previous part has just released; one cp.async group per part.
+// Group bookkeeping (groups numbered in issue order, part q of edge i is group
+// i NQ + q): at the start of an edge the groups of its part 0 (which also holds
+// its node rows) are complete after wait_group(NQ - 1); at the start of part q,
+// after issuing the group of the next edge's part q, wait_group(NQ) leaves the
+// current part complete.
+template <int L, bool O3>
+struct Pipe {
+    using PT = Parts<L, O3>;
+    static constexpr int P = PT::P, NQ = PT::NQ, PP = PT::PP;
+    float2* ring;          // (NQ + 1) slots of PP x T float2, lane-major
+    int T, tl, C2;
+    int slot0;             // slot of part 0 of the current edge
+    const float2* w_next;  // this lane's weights of the next edge, or nullptr
+
+    __device__ __forceinline__ float2* lane_slot(int slot) { return ring + (slot * T + tl) * PP; }
+
+    template <int q>
+    __device__ __forceinline__ void issue_part(const float2* w, int slot) {
+        float2* dst = lane_slot(slot);
+        static_for<PT::begin(q), PT::end(q)>([&](auto kc) {
+            constexpr int k = decltype(kc)::value;
+            cp_async8(dst + (k - PT::begin(q)), w + Order<L, O3>::path_at(k) * C2);
+        });
+    }
+
+    // First edge: all its parts, its node rows (issued by `rows`) in the first group.
+    template <class Rows>
+    __device__ __forceinline__ void prologue(const float2* w_first, Rows&& rows) {
+        slot0 = 0;
+        static_for<0, NQ>([&](auto qc) {
+            constexpr int q = decltype(qc)::value;
+            if (w_first) issue_part<q>(w_first, q);
+            if constexpr (q == 0) rows();
+            cp_async_commit();
+        });
+    }
+
+    __device__ __forceinline__ void edge_begin() { cp_async_wait<NQ - 1>(); }
+
+    // Start of part q of the current edge: issue the next edge's part q (and at
+    // q = 0 its node rows), wait for the current part.
+    template <int q, class Rows>
+    __device__ __forceinline__ void part_begin(Rows&& next_rows) {
+        if (w_next) issue_part<q>(w_next, (slot0 + q + NQ) % (NQ + 1));
+        if constexpr (q == 0) next_rows();
+        cp_async_commit();
+        cp_async_wait<NQ>();
+    }
+
+    // Weight of consumption position k (its part has begun).
+    template <int k>
+    __device__ __forceinline__ float2 w_at() {
+        constexpr int q = k / PP;
+        return lds2(lane_slot((slot0 + q) % (NQ + 1)) + (k - q * PP));
+    }
+
+    __device__ __forceinline__ void edge_end(const float2* next_after) {
+        slot0 = (slot0 + NQ) % (NQ + 1);
+        w_next = next_after;
+    }
+};
+
 // Combined frame weights of the (l1, l3) group for this lane's channels:
-// We[mu] = sum over even paths (l1, l2, l3) of b_p(mu) w_p, Wo[mu] likewise for odd
-// paths; degenerate edges keep only l2 = 0.
-template <int L, bool O3, int l1, int l3>
-__device__ __forceinline__ void group_weights(const float2* __restrict__ we, int C2, uint64_t pol, bool degenerate,
-                                              float2 (&We)[4], float2 (&Wo)[4], float2 (&wp)[L + 1]) {
+// We[mu] = sum over even paths (l1, l2, l3) of b_p(mu) w_p, Wo[mu] likewise for
+// odd paths; degenerate edges keep only l2 = 0. Part boundaries inside the group
+// advance the pipe.
+template <int L, bool O3, int l1, int l3, class Rows>
+__device__ __forceinline__ void group_weights(Pipe<L, O3>& pp, Rows&& next_rows, bool degenerate, float2 (&We)[4],
+                                              float2 (&Wo)[4]) {
 #pragma unroll
     for (int m = 0; m < 4; ++m) {
         We[m] = f2_zero();
@@ -271,10 +407,11 @@ __device__ __forceinline__ void group_weights(const float2* __restrict__ we, int
     static_for<0, L + 1>([&](auto l2c) {
         constexpr int l2 = decltype(l2c)::value;
         if constexpr (PathSet<L, O3>::allowed(l1, l2, l3)) {
-            constexpr int p = path_index<L, O3>(l1, l2, l3);
-            float2 w = ld_stream2(we + p * C2, pol);
+            constexpr int k = Order<L, O3>::pos(l1, l2, l3);
+            constexpr int PP = Parts<L, O3>::PP;
+            if constexpr (k % PP == 0) pp.template part_begin<k / PP>(next_rows);
+            float2 w = pp.template w_at<k>();
             if (l2 > 0 && degenerate) w = f2_zero();
-            wp[l2] = w;
             constexpr bool odd = (l1 + l2 + l3) % 2 == 1;
             static_for<0, cmin(l1, l3) + 1>([&](auto mc) {
                 constexpr int mu = decltype(mc)::value;
@@ -347,8 +484,12 @@ __device__ __forceinline__ float gen_form(const float2* v, const float2* s) {
 }
 
 // ---------------------------------------------------------------------------
+// Work decomposition: equal contiguous ranges of edges ("tasks"), one per team
+// (or per pair of slice teams when C = 128, the block's two warps). Rows cut by a
+// range boundary are combined by vector reductions on a zeroed output; rows
+// inside a range are stored once.
 struct Geometry {
-    int T, S, team_in_block, node, slice, tl;
+    int T, S, team_in_block, task, slice, tl;
     unsigned tmask;
 };
 
@@ -359,12 +500,48 @@ __device__ __forceinline__ Geometry geometry(int team_lanes, int slices) {
     g.S = slices;
     g.tl = lane & (team_lanes - 1);
     g.team_in_block = warp * (32 / team_lanes) + lane / team_lanes;
-    const int nodes_per_block = (kThreads / team_lanes) / slices;
-    g.node = blockIdx.x * nodes_per_block + g.team_in_block / slices;
+    const int tasks_per_block = (kThreads / team_lanes) / slices;
+    g.task = blockIdx.x * tasks_per_block + g.team_in_block / slices;
     g.slice = g.team_in_block % slices;
     const unsigned ones = team_lanes == 32 ? 0xffffffffu : ((1u << team_lanes) - 1u);
     g.tmask = ones << (lane & ~(team_lanes - 1) & 31);
     return g;
+}
+
+// [k0, k1): the task's share of n items.
+__device__ __forceinline__ void task_range(long long n, int task, int ntasks, int& k0, int& k1) {
+    k0 = (int)(n * task / ntasks);
+    k1 = (int)(n * (task + 1) / ntasks);
+}
+
+// largest i in [0, n) with ptr[i] <= k (ptr nondecreasing, ptr[0] <= k)
+__device__ __forceinline__ int segment_of(const int32_t* __restrict__ ptr, int n, int k) {
+    int lo = 0, hi = n;
+    while (hi - lo > 1) {
+        int mid = (lo + hi) >> 1;
+        if (__ldg(ptr + mid) <= k)
+            lo = mid;
+        else
+            hi = mid;
+    }
+    return lo;
+}
+
+__device__ __forceinline__ void red_add2(float2* p, float2 v) {
+    asm volatile("red.global.add.v2.f32 [%0], {%1, %2};" ::"l"(p), "f"(v.x), "f"(v.y) : "memory");
+}
+
+// Store a row accumulator: plainly when the task owns the whole row, else by
+// vector reduction onto the zeroed output.
+template <int D>
+__device__ __forceinline__ void flush_row(float2* row, int C2, const float2 (&acc)[D], bool whole) {
+#pragma unroll
+    for (int k = 0; k < D; ++k) {
+        if (whole)
+            row[k * C2] = acc[k];
+        else
+            red_add2(row + k * C2, acc[k]);
+    }
 }
 
 // The fitting points and inverses as one constant-memory table, built at
@@ -396,44 +573,78 @@ __device__ __forceinline__ void load_fit_tables(float* fit) {
 
 }  // namespace frame
 
+
 // ===========================================================================
+// Forward: task = a contiguous range of CSR (destination-ordered) edges.
 template <int L, bool O3>
-__global__ void __launch_bounds__(frame::kThreads, 2) etp_fwd_frame_kernel(FwdArgs a) {
+__global__ void __launch_bounds__(frame::kThreads, 4) etp_fwd_frame_kernel(FwdArgs a) {
     using namespace frame;
+    using PT = Parts<L, O3>;
     constexpr int D = (L + 1) * (L + 1);
+    constexpr int P = PT::P;
     extern __shared__ __align__(16) float smem[];
-    float* fit = smem;
-    load_fit_tables(fit);
+    load_fit_tables(smem);
     const Geometry G = geometry(a.team, a.slices);
-    if (G.node >= a.N) return;
-    float* ybuf = smem + kFitStride + G.team_in_block * kTeamFloats;
-    float* dbuf = ybuf + kYbufFloats;
+    if (G.task >= a.ntasks) return;  // the slice teams of a task leave together
+    int k0, k1;
+    task_range(a.E, G.task, a.ntasks, k0, k1);
+    if (k0 >= k1) return;
+    float* team = smem + kHeaderFloats + G.team_in_block * team_floats(D, G.T, 1, PT::ring_float2(G.T) / G.T);
+    float* ybuf = team;
+    float* dbuf = team + kYbufFloats;
+    float2* xbuf = reinterpret_cast<float2*>(team + kYbufFloats + kDbufFloats);
+    float2* ring = xbuf + D * G.T;
     const int C2 = a.C4 * 2;
     const int cp = G.slice * G.T + G.tl;
-    const uint64_t pol = l2_evict_first_policy();
     const float2* x2 = reinterpret_cast<const float2*>(a.x);
     const float2* w2 = reinterpret_cast<const float2*>(a.w);
+    float2* out2 = reinterpret_cast<float2*>(a.out);
 
-    int e0 = __ldg(a.row_ptr + G.node), e1 = __ldg(a.row_ptr + G.node + 1);
-    e0 = max(e0, 0);
-    e1 = min(e1, a.E);
+    auto w_of = [&](int e) -> const float2* { return e < k1 ? w2 + (size_t)e * P * C2 + cp : nullptr; };
+    auto copy_x = [&](int j) {  // an out-of-range source reads row 0 and is zeroed later
+        const float2* src = x2 + (size_t)((unsigned)j < (unsigned)a.N ? j : 0) * D * C2 + cp;
+#pragma unroll
+        for (int k = 0; k < D; ++k) cp_async8(xbuf + k * G.T + G.tl, src + k * C2);
+    };
+
+    int row = segment_of(a.row_ptr, a.N, k0);
+    int row_lo = __ldg(a.row_ptr + row), row_hi = __ldg(a.row_ptr + row + 1);
+    int j_cur = __ldg(a.src + k0);
+    Pipe<L, O3> pp{ring, G.T, G.tl, C2, 0, w_of(k0 + 1)};
+    pp.prologue(w_of(k0), [&] { copy_x(j_cur); });
 
     float2 acc[D];
 #pragma unroll
     for (int k = 0; k < D; ++k) acc[k] = f2_zero();
 
-    for (int e = e0; e < e1; ++e) {
-        const int j = __ldg(a.src + e);
-        if ((unsigned)j >= (unsigned)a.N) continue;  // uniform over the team
+    for (int e = k0; e < k1; ++e) {
+        while (e >= row_hi && row < a.N - 1) {  // the edge opens a later row: store the finished one
+            if (row_hi > max(row_lo, k0)) {
+                flush_row<D>(out2 + (size_t)row * D * C2 + cp, C2, acc, row_lo >= k0);
+#pragma unroll
+                for (int k = 0; k < D; ++k) acc[k] = f2_zero();
+            }
+            ++row;
+            row_lo = row_hi;
+            row_hi = __ldg(a.row_ptr + row + 1);
+        }
+        const bool has_next = e + 1 < k1;
+        const int j_next = has_next ? __ldg(a.src + e + 1) : 0;
+        pp.edge_begin();
         const Frame f = make_frame(__ldg(a.r + 3 * (size_t)e), __ldg(a.r + 3 * (size_t)e + 1),
                                    __ldg(a.r + 3 * (size_t)e + 2));
-        float2 xv[D], xp[D];
-        const float2* xj = x2 + (size_t)j * D * C2 + cp;
+        team_wigner<L>(f, G.tl, G.T, G.tmask, ybuf, dbuf, smem);
+        float2 xp[D];
+        {
+            float2 xv[D];
+            const bool valid = (unsigned)j_cur < (unsigned)a.N;  // an invalid source contributes nothing
 #pragma unroll
-        for (int k = 0; k < D; ++k) xv[k] = __ldg(xj + k * C2);
-        team_wigner<L>(f, G.tl, G.T, G.tmask, ybuf, dbuf, fit + 0);
-        rotate_all<L>(f, dbuf, xv, xp);
-        const float2* we = w2 + (size_t)e * PathSet<L, O3>::P * C2 + cp;
+            for (int k = 0; k < D; ++k) xv[k] = valid ? lds2(xbuf + k * G.T + G.tl) : f2_zero();
+            rotate_all<L>(f, dbuf, xv, xp);
+        }
+        auto next_rows = [&] {
+            if (has_next) copy_x(j_next);
+        };
         static_for<0, L + 1>([&](auto l3c) {
             constexpr int l3 = decltype(l3c)::value;
             float2 y[2 * l3 + 1];
@@ -442,156 +653,204 @@ __global__ void __launch_bounds__(frame::kThreads, 2) etp_fwd_frame_kernel(FwdAr
             static_for<0, L + 1>([&](auto l1c) {
                 constexpr int l1 = decltype(l1c)::value;
                 if constexpr (has_type<L, O3>(l1, l3, 0) || has_type<L, O3>(l1, l3, 1)) {
-                    float2 We[4], Wo[4], wp[L + 1];
-                    group_weights<L, O3, l1, l3>(we, C2, pol, f.degenerate, We, Wo, wp);
+                    float2 We[4], Wo[4];
+                    group_weights<L, O3, l1, l3>(pp, next_rows, f.degenerate, We, Wo);
                     apply_M<L, O3, l1, l3>(We, Wo, xp + l1 * l1, y);
                 }
             });
             rotate<l3, true, true>(f, dbuf, y, acc + l3 * l3);
         });
+        pp.edge_end(w_of(e + 2));
+        j_cur = j_next;
     }
-    float2* o = reinterpret_cast<float2*>(a.out) + (size_t)G.node * D * C2 + cp;
-#pragma unroll
-    for (int k = 0; k < D; ++k) o[k * C2] = acc[k];
+    cp_async_wait_all();
+    flush_row<D>(out2 + (size_t)row * D * C2 + cp, C2, acc, row_lo >= k0 && row_hi <= k1);
 }
 
 // ===========================================================================
+// Backward: task = a contiguous range of reverse-CSR (source-ordered) positions.
 template <int L, bool O3>
-__global__ void __launch_bounds__(frame::kThreads, 2) etp_bwd_frame_kernel(BwdArgs a) {
+__global__ void __launch_bounds__(frame::kThreads, 4) etp_bwd_frame_kernel(BwdArgs a) {
     using namespace frame;
+    using PT = Parts<L, O3>;
     constexpr int D = (L + 1) * (L + 1);
+    constexpr int P = PT::P;
     extern __shared__ __align__(16) float smem[];
-    float* fit = smem;
-    load_fit_tables(fit);
+    load_fit_tables(smem);
     const Geometry G = geometry(a.team, a.slices);
-    if (G.node >= a.N) return;  // both slices of a node leave together
-    float* ybuf = smem + kFitStride + G.team_in_block * kTeamFloats;
-    float* dbuf = ybuf + kYbufFloats;
-    // slice partials of grad_r (two nodes per block when S = 2), double-buffered by edge parity
-    float* comb = smem + kFitStride + (kThreads / G.T) * kTeamFloats;
+    if (G.task >= a.ntasks) return;  // the slice teams of a task leave together
+    int k0, k1;
+    task_range(a.E, G.task, a.ntasks, k0, k1);
+    if (k0 >= k1) return;
+    float* comb = smem + kFitStride;  // slice partials of grad_r, double-buffered by edge parity
+    float* team = smem + kHeaderFloats + G.team_in_block * team_floats(D, G.T, 2, PT::ring_float2(G.T) / G.T);
+    float* ybuf = team;
+    float* dbuf = team + kYbufFloats;
+    float2* xbuf = reinterpret_cast<float2*>(team + kYbufFloats + kDbufFloats);
+    float2* gbuf = xbuf + D * G.T;
+    float2* ring = gbuf + D * G.T;
     const int C2 = a.C4 * 2;
     const int cp = G.slice * G.T + G.tl;
-    const uint64_t pol = l2_evict_first_policy();
+    const uint64_t pol_w = l2_evict_first_policy();
     const float2* x2 = reinterpret_cast<const float2*>(a.x);
     const float2* g2 = reinterpret_cast<const float2*>(a.g);
     const float2* w2 = reinterpret_cast<const float2*>(a.w);
     float2* gw2 = reinterpret_cast<float2*>(a.grad_w);
+    float2* gx2 = reinterpret_cast<float2*>(a.grad_x);
     const bool want_w = a.grad_w != nullptr;
     const bool want_r = a.grad_r != nullptr;
 
-    const int q0 = max(__ldg(a.rev_ptr + G.node), 0);
-    const int q1 = min(__ldg(a.rev_ptr + G.node + 1), a.E);
-
-    float2 xv[D], gx[D];
-    {
-        const float2* xj = x2 + (size_t)G.node * D * C2 + cp;
+    // position q of the reverse order -> edge; out-of-range edges and rows map to
+    // valid addresses and are marked invalid (they contribute and store nothing)
+    auto edge_at = [&](int q) -> int { return __ldg(a.rev_perm + q); };
+    auto valid_edge = [&](int e) { return (unsigned)e < (unsigned)a.E; };
+    auto dst_of = [&](int e) -> int {
+        if (!valid_edge(e)) return -1;
+        return a.dst ? __ldg(a.dst + e) : row_of_edge(a.row_ptr, a.N, e);
+    };
+    auto w_of = [&](int q) -> const float2* {
+        if (q >= k1) return nullptr;
+        const int e = edge_at(q);
+        return w2 + (size_t)(valid_edge(e) ? e : 0) * P * C2 + cp;
+    };
+    auto copy_rows = [&](int j, int i) {
+        const float2* xs = x2 + (size_t)j * D * C2 + cp;
+        const float2* gs = g2 + (size_t)((unsigned)i < (unsigned)a.N ? i : 0) * D * C2 + cp;
 #pragma unroll
         for (int k = 0; k < D; ++k) {
-            xv[k] = __ldg(xj + k * C2);
-            gx[k] = f2_zero();
+            cp_async8(xbuf + k * G.T + G.tl, xs + k * C2);
+            cp_async8(gbuf + k * G.T + G.tl, gs + k * C2);
         }
-    }
-    const int node_in_block = G.team_in_block / G.S;
+    };
 
-    for (int q = q0, it = 0; q < q1; ++q, ++it) {
-        const int e = __ldg(a.rev_perm + q);
-        bool ok = (unsigned)e < (unsigned)a.E;
-        int i = 0;
-        if (ok) {
-            i = a.dst ? __ldg(a.dst + e) : row_of_edge(a.row_ptr, a.N, e);
-            ok = (unsigned)i < (unsigned)a.N;
+    int row = segment_of(a.rev_ptr, a.N, k0);  // source node of position k0
+    int row_lo = __ldg(a.rev_ptr + row), row_hi = __ldg(a.rev_ptr + row + 1);
+    int e_cur = edge_at(k0);
+    int i_cur = dst_of(e_cur);
+    Pipe<L, O3> pp{ring, G.T, G.tl, C2, 0, w_of(k0 + 1)};
+    pp.prologue(w_of(k0), [&] { copy_rows(row, i_cur); });
+
+    float2 gx[D];
+#pragma unroll
+    for (int k = 0; k < D; ++k) gx[k] = f2_zero();
+
+    for (int q = k0, it = 0; q < k1; ++q, ++it) {
+        while (q >= row_hi && row < a.N - 1) {  // the position opens a later source row: store the finished one
+            if (row_hi > max(row_lo, k0)) {
+                if (gx2) flush_row<D>(gx2 + (size_t)row * D * C2 + cp, C2, gx, row_lo >= k0);
+#pragma unroll
+                for (int k = 0; k < D; ++k) gx[k] = f2_zero();
+            }
+            ++row;
+            row_lo = row_hi;
+            row_hi = __ldg(a.rev_ptr + row + 1);
         }
-        float sx = 0.f, sy = 0.f;  // dL/de_x, dL/de_y over this lane's channels
+        // the next position's source row and destination (for the row prefetch)
+        const bool has_next = q + 1 < k1;
+        int row_next = row, e_next = 0, i_next = 0;
+        if (has_next) {
+            int hi = row_hi;
+            while (q + 1 >= hi && row_next < a.N - 1) hi = __ldg(a.rev_ptr + (++row_next) + 1);
+            e_next = edge_at(q + 1);
+            i_next = dst_of(e_next);
+        }
+        const bool ok = valid_edge(e_cur) && (unsigned)i_cur < (unsigned)a.N;
+        pp.edge_begin();
         Frame f = make_frame(0.f, 0.f, 1.f);
-        if (ok) {
-            f = make_frame(__ldg(a.r + 3 * (size_t)e), __ldg(a.r + 3 * (size_t)e + 1),
-                           __ldg(a.r + 3 * (size_t)e + 2));
-            team_wigner<L>(f, G.tl, G.T, G.tmask, ybuf, dbuf, fit);
-            float2 xp[D], z[D];
-            rotate_all<L>(f, dbuf, xv, xp);
+        if (ok)
+            f = make_frame(__ldg(a.r + 3 * (size_t)e_cur), __ldg(a.r + 3 * (size_t)e_cur + 1),
+                           __ldg(a.r + 3 * (size_t)e_cur + 2));
+        team_wigner<L>(f, G.tl, G.T, G.tmask, ybuf, dbuf, smem);
+        float2 xp[D], gp[D], z[D];
+        {
+            float2 v[D];
 #pragma unroll
-            for (int k = 0; k < D; ++k) z[k] = f2_zero();
-            const float2* gi = g2 + (size_t)i * D * C2 + cp;
-            const float2* we = w2 + (size_t)e * PathSet<L, O3>::P * C2 + cp;
-            float2* gwe = want_w ? gw2 + (size_t)e * PathSet<L, O3>::P * C2 + cp : nullptr;
-            static_for<0, L + 1>([&](auto l3c) {
-                constexpr int l3 = decltype(l3c)::value;
-                constexpr int d3 = 2 * l3 + 1;
-                float2 gv[d3], gp[d3], y[d3];
+            for (int k = 0; k < D; ++k) v[k] = ok ? lds2(xbuf + k * G.T + G.tl) : f2_zero();
+            rotate_all<L>(f, dbuf, v, xp);
 #pragma unroll
-                for (int m = 0; m < d3; ++m) {
-                    gv[m] = __ldg(gi + (l3 * l3 + m) * C2);
-                    y[m] = f2_zero();
-                }
-                rotate<l3, false, false>(f, dbuf, gv, gp);
-                static_for<0, L + 1>([&](auto l1c) {
-                    constexpr int l1 = decltype(l1c)::value;
-                    if constexpr (has_type<L, O3>(l1, l3, 0) || has_type<L, O3>(l1, l3, 1)) {
-                        float2 We[4], Wo[4], wp[L + 1];
-                        group_weights<L, O3, l1, l3>(we, C2, pol, f.degenerate, We, Wo, wp);
-                        apply_M<L, O3, l1, l3>(We, Wo, xp + l1 * l1, y);
-                        apply_MT<L, O3, l1, l3>(We, Wo, gp, z + l1 * l1);
-                        if (want_w) {
-                            // products of the frame components coupled by B_p, symmetrised in +-mu
-                            constexpr int mn = cmin(l1, l3);
-                            float2 Pe[4], Po[4];
-                            static_for<0, mn + 1>([&](auto mc) {
-                                constexpr int mu = decltype(mc)::value;
-                                const float2 a1 = gp[l3 + mu], a2 = gp[l3 - mu];
-                                const float2 b1 = xp[l1 * l1 + l1 + mu], b2 = xp[l1 * l1 + l1 - mu];
-                                if constexpr (mu == 0) {
-                                    Pe[0] = make_float2(a1.x * b1.x, a1.y * b1.y);
-                                    Po[0] = f2_zero();
-                                } else {
-                                    Pe[mu] = make_float2(fmaf(a1.x, b1.x, a2.x * b2.x), fmaf(a1.y, b1.y, a2.y * b2.y));
-                                    Po[mu] = make_float2(fmaf(a1.x, b2.x, -a2.x * b1.x), fmaf(a1.y, b2.y, -a2.y * b1.y));
-                                }
-                            });
-                            static_for<0, L + 1>([&](auto l2c) {
-                                constexpr int l2 = decltype(l2c)::value;
-                                if constexpr (PathSet<L, O3>::allowed(l1, l2, l3)) {
-                                    constexpr int p = path_index<L, O3>(l1, l2, l3);
-                                    constexpr bool odd = (l1 + l2 + l3) % 2 == 1;
-                                    float2 gw = f2_zero();
-                                    static_for<0, mn + 1>([&](auto mc) {
-                                        constexpr int mu = decltype(mc)::value;
-                                        constexpr float b = (float)etp_gen::kFrameB[l1][l2][l3][mu];
-                                        if constexpr (b != 0.f) f2_fma(gw, b, odd ? Po[mu] : Pe[mu]);
-                                    });
-                                    if (l2 > 0 && f.degenerate) gw = f2_zero();
-                                    st_stream2(gwe + p * C2, gw, pol);
-                                }
-                            });
-                        }
-                    }
-                });
-                if (want_r) {
-                    sx += gen_form<l3, 0>(gp, y);
-                    sy += gen_form<l3, 1>(gp, y);
-                }
-            });
+            for (int k = 0; k < D; ++k) v[k] = ok ? lds2(gbuf + k * G.T + G.tl) : f2_zero();
+            rotate_all<L>(f, dbuf, v, gp);
+        }
+#pragma unroll
+        for (int k = 0; k < D; ++k) z[k] = f2_zero();
+        auto next_rows = [&] {
+            if (has_next) copy_rows(row_next, i_next);
+        };
+        float2* gwe = (want_w && ok) ? gw2 + (size_t)e_cur * P * C2 + cp : nullptr;
+        float sx = 0.f, sy = 0.f;  // dL/de_x, dL/de_y over this lane's channels
+        static_for<0, L + 1>([&](auto l3c) {
+            constexpr int l3 = decltype(l3c)::value;
+            constexpr int d3 = 2 * l3 + 1;
+            float2 y[d3];
+#pragma unroll
+            for (int m = 0; m < d3; ++m) y[m] = f2_zero();
             static_for<0, L + 1>([&](auto l1c) {
                 constexpr int l1 = decltype(l1c)::value;
-                if (want_r) {
-                    sx += gen_form<l1, 0>(xp + l1 * l1, z + l1 * l1);
-                    sy += gen_form<l1, 1>(xp + l1 * l1, z + l1 * l1);
+                if constexpr (has_type<L, O3>(l1, l3, 0) || has_type<L, O3>(l1, l3, 1)) {
+                    float2 We[4], Wo[4];
+                    group_weights<L, O3, l1, l3>(pp, next_rows, f.degenerate, We, Wo);
+                    apply_M<L, O3, l1, l3>(We, Wo, xp + l1 * l1, y);
+                    apply_MT<L, O3, l1, l3>(We, Wo, gp + l3 * l3, z + l1 * l1);
+                    if (gwe) {
+                        // products of the frame components coupled by B_p, symmetrised in +-mu
+                        constexpr int mn = cmin(l1, l3);
+                        float2 Pe[4], Po[4];
+                        static_for<0, mn + 1>([&](auto mc) {
+                            constexpr int mu = decltype(mc)::value;
+                            const float2 a1 = gp[l3 * l3 + l3 + mu], a2 = gp[l3 * l3 + l3 - mu];
+                            const float2 b1 = xp[l1 * l1 + l1 + mu], b2 = xp[l1 * l1 + l1 - mu];
+                            if constexpr (mu == 0) {
+                                Pe[0] = make_float2(a1.x * b1.x, a1.y * b1.y);
+                                Po[0] = f2_zero();
+                            } else {
+                                Pe[mu] = make_float2(fmaf(a1.x, b1.x, a2.x * b2.x), fmaf(a1.y, b1.y, a2.y * b2.y));
+                                Po[mu] = make_float2(fmaf(a1.x, b2.x, -a2.x * b1.x), fmaf(a1.y, b2.y, -a2.y * b1.y));
+                            }
+                        });
+                        static_for<0, L + 1>([&](auto l2c) {
+                            constexpr int l2 = decltype(l2c)::value;
+                            if constexpr (PathSet<L, O3>::allowed(l1, l2, l3)) {
+                                constexpr int p = path_index<L, O3>(l1, l2, l3);
+                                constexpr bool odd = (l1 + l2 + l3) % 2 == 1;
+                                float2 gw = f2_zero();
+                                static_for<0, mn + 1>([&](auto mc) {
+                                    constexpr int mu = decltype(mc)::value;
+                                    constexpr float b = (float)etp_gen::kFrameB[l1][l2][l3][mu];
+                                    if constexpr (b != 0.f) f2_fma(gw, b, odd ? Po[mu] : Pe[mu]);
+                                });
+                                if (l2 > 0 && f.degenerate) gw = f2_zero();
+                                st_stream2(gwe + p * C2, gw, pol_w);
+                            }
+                        });
+                    }
                 }
-                rotate<l1, true, true>(f, dbuf, z + l1 * l1, gx + l1 * l1);
             });
-        }
+            if (want_r) {
+                sx += gen_form<l3, 0>(gp + l3 * l3, y);
+                sy += gen_form<l3, 1>(gp + l3 * l3, y);
+            }
+        });
+        static_for<0, L + 1>([&](auto l1c) {
+            constexpr int l1 = decltype(l1c)::value;
+            if (want_r) {
+                sx += gen_form<l1, 0>(xp + l1 * l1, z + l1 * l1);
+                sy += gen_form<l1, 1>(xp + l1 * l1, z + l1 * l1);
+            }
+            rotate<l1, true, true>(f, dbuf, z + l1 * l1, gx + l1 * l1);
+        });
         if (want_r) {
-            // sum over the team's lanes, then over the node's slices
+            // sum over the team's lanes, then over the task's two slices (the block's two warps)
             for (int s = 1; s < G.T; s <<= 1) {
                 sx += __shfl_xor_sync(G.tmask, sx, s);
                 sy += __shfl_xor_sync(G.tmask, sy, s);
             }
             if (G.S == 2) {
-                float* slot = comb + (node_in_block * 2 + (it & 1)) * 2;
+                float* slot = comb + (it & 1) * 2;
                 if (G.slice == 1 && G.tl == 0) {
                     slot[0] = sx;
                     slot[1] = sy;
                 }
-                asm volatile("bar.sync %0, %1;" ::"r"(1 + node_in_block), "r"(64) : "memory");
+                __syncthreads();
                 if (G.slice == 0) {
                     sx += slot[0];
                     sy += slot[1];
@@ -600,18 +859,46 @@ __global__ void __launch_bounds__(frame::kThreads, 2) etp_bwd_frame_kernel(BwdAr
             if (ok && G.slice == 0 && G.tl == 0) {
                 // grad_r = R^T (dL/de_y, -dL/de_x, 0) / |r|
                 const float gu0 = sy * f.inv_rho, gu1 = -sx * f.inv_rho;
-                float* gr = a.grad_r + 3 * (size_t)e;
+                float* gr = a.grad_r + 3 * (size_t)e_cur;
                 gr[0] = f.R[0] * gu0 + f.R[3] * gu1;
                 gr[1] = f.R[1] * gu0 + f.R[4] * gu1;
                 gr[2] = f.R[2] * gu0 + f.R[5] * gu1;
             }
         }
+        pp.edge_end(w_of(q + 2));
+        e_cur = e_next;
+        i_cur = i_next;
     }
-    if (a.grad_x) {
-        float2* o = reinterpret_cast<float2*>(a.grad_x) + (size_t)G.node * D * C2 + cp;
-#pragma unroll
-        for (int k = 0; k < D; ++k) o[k * C2] = gx[k];
-    }
+    cp_async_wait_all();
+    if (gx2) flush_row<D>(gx2 + (size_t)row * D * C2 + cp, C2, gx, row_lo >= k0 && row_hi <= k1);
+}
+
+namespace frame {
+template <int L, bool O3>
+constexpr size_t smem_bytes_for(int T, bool backward) {
+    constexpr int D = (L + 1) * (L + 1);
+    const int teams = kThreads / T;
+    return sizeof(float) *
+           (size_t)(kHeaderFloats + teams * team_floats(D, T, backward ? 2 : 1, Parts<L, O3>::ring_float2(T) / T));
+}
+}  // namespace frame
+
+template <int L>
+size_t smem_bytes(bool o3, int T, bool backward) {
+    return o3 ? frame::smem_bytes_for<L, true>(T, backward) : frame::smem_bytes_for<L, false>(T, backward);
+}
+
+template <int L>
+int blocks_per_sm(bool o3, bool backward, size_t smem) {
+    int n = 0;
+    const void* k;
+    if (backward)
+        k = o3 ? (const void*)etp_bwd_frame_kernel<L, true> : (const void*)etp_bwd_frame_kernel<L, false>;
+    else
+        k = o3 ? (const void*)etp_fwd_frame_kernel<L, true> : (const void*)etp_fwd_frame_kernel<L, false>;
+    cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, 160 * 1024);
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k, frame::kThreads, smem) != cudaSuccess) n = 1;
+    return n < 1 ? 1 : n;
 }
 
 template <int L>

@@ -8,7 +8,7 @@
 
 namespace etp {
 
-constexpr int kThreadsPerBlock = 128;  // 4 warps; forward and backward kernels
+constexpr int kThreadsPerBlock = 64;  // 2 warps; forward and backward kernels
 
 struct FwdArgs {
     int N, E;
@@ -20,7 +20,8 @@ struct FwdArgs {
     float4* out;
     int C4;      // C / 4
     int team;    // lanes per team = min(32, C/2), a power of two
-    int slices;  // teams per node = C / (2 team): 1, or 2 when C = 128
+    int slices;  // teams per task = C / (2 team): 1, or 2 when C = 128
+    int ntasks;  // equal contiguous edge ranges
 };
 
 struct BwdArgs {
@@ -40,15 +41,23 @@ struct BwdArgs {
     int C4;
     int team;
     int slices;
+    int ntasks;
 };
 
 // Launch geometry shared by the forward and backward kernels: teams of
-// min(32, C/2) lanes, each lane two channels; C/(2 team) teams per node.
+// min(32, C/2) lanes, each lane two channels; C/(2 team) teams per task (a
+// contiguous range of edges); as many tasks as fill the GPU once.
 struct LaunchShape {
-    int team, slices, nodes_per_block;
+    int team, slices, tasks_per_block, ntasks;
     size_t smem_bytes;
+    dim3 grid;
 };
-LaunchShape launch_shape(int C, int N);
+LaunchShape launch_shape(int C, int L, bool o3, bool backward, int E, int N);
+
+template <int L>
+size_t smem_bytes(bool o3, int T, bool backward);
+template <int L>
+int blocks_per_sm(bool o3, bool backward, size_t smem);
 
 template <int L>
 cudaError_t launch_forward(bool o3, const FwdArgs& a, dim3 grid, size_t smem, cudaStream_t s);

@@ -9,4 +9,6 @@
 namespace etp {
 template cudaError_t launch_forward<ETP_L>(bool, const FwdArgs&, dim3, size_t, cudaStream_t);
 template cudaError_t launch_backward<ETP_L>(bool, const BwdArgs&, dim3, size_t, cudaStream_t);
+template size_t smem_bytes<ETP_L>(bool, int, bool);
+template int blocks_per_sm<ETP_L>(bool, bool, size_t);
 }  // namespace etp

@@ -1,16 +1,61 @@
 // Launch geometry of the forward and backward kernels (host side).
+#include <atomic>
+
 #include "etp_frame.cuh"
 
 namespace etp {
+namespace {
 
-LaunchShape launch_shape(int C, int N) {
-    (void)N;
+// Resident blocks per SM of each kernel specialisation, per device (computed once).
+std::atomic<int> g_occupancy[16][4][2][2][6];
+std::atomic<int> g_sms[16];
+
+int log2i(int t) {
+    int k = 0;
+    while ((1 << k) < t) ++k;
+    return k;
+}
+
+}  // namespace
+
+LaunchShape launch_shape(int C, int L, bool o3, bool backward, int E, int N) {
     LaunchShape s;
     s.team = C / 2 < 32 ? C / 2 : 32;
     s.slices = C / (2 * s.team);
-    s.nodes_per_block = (frame::kThreads / s.team) / s.slices;
-    const int teams = frame::kThreads / s.team;
-    s.smem_bytes = sizeof(float) * (frame::kFitStride + teams * frame::kTeamFloats + 8);
+    s.tasks_per_block = (frame::kThreads / s.team) / s.slices;
+    switch (L) {
+        case 0: s.smem_bytes = smem_bytes<0>(o3, s.team, backward); break;
+        case 1: s.smem_bytes = smem_bytes<1>(o3, s.team, backward); break;
+        case 2: s.smem_bytes = smem_bytes<2>(o3, s.team, backward); break;
+        default: s.smem_bytes = smem_bytes<3>(o3, s.team, backward); break;
+    }
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 16) dev = 0;
+    int sms = g_sms[dev].load();
+    if (sms == 0) {
+        if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 1) sms = 1;
+        g_sms[dev].store(sms);
+    }
+    std::atomic<int>& occ = g_occupancy[dev][L & 3][o3 ? 1 : 0][backward ? 1 : 0][log2i(s.team) % 6];
+    int bps = occ.load();
+    if (bps == 0) {
+        switch (L) {
+            case 0: bps = blocks_per_sm<0>(o3, backward, s.smem_bytes); break;
+            case 1: bps = blocks_per_sm<1>(o3, backward, s.smem_bytes); break;
+            case 2: bps = blocks_per_sm<2>(o3, backward, s.smem_bytes); break;
+            default: bps = blocks_per_sm<3>(o3, backward, s.smem_bytes); break;
+        }
+        occ.store(bps);
+    }
+    // One wave of tasks, at least 16 edges each and no more tasks than rows: a
+    // row longer than a task is cut more than once, and its pieces are then
+    // summed in a run-dependent order (still correct, not bitwise repeatable).
+    long long cap = (long long)sms * bps * s.tasks_per_block;
+    long long want = ((long long)E + 15) / 16;
+    if (want > N) want = N;
+    long long nt = want < cap ? want : cap;
+    s.ntasks = (int)(nt < 1 ? 1 : nt);
+    s.grid = dim3((unsigned)((s.ntasks + s.tasks_per_block - 1) / s.tasks_per_block), 1, 1);
     return s;
 }
 

@@ -96,10 +96,12 @@ def test_subsets_of_gradients(want):
     res = run_gpu(wl, want=want)
     full = run_gpu(wl)
     for k, key in (("x", "grad_x"), ("w", "grad_w"), ("r", "grad_r")):
-        if k in want:
-            assert torch.equal(res[key], full[key])
-        else:
+        if k not in want:
             assert res[key] is None
+        elif key == "grad_x":   # node sums: pieces of a row cut twice may be reduced in another order
+            assert rel_err(res[key], full[key].double().cpu().numpy()) <= 1e-6
+        else:
+            assert torch.equal(res[key], full[key])
 
 
 def test_no_edges():
@@ -122,15 +124,38 @@ def test_zero_length_edge_vectors():
     assert torch.all(res["grad_r"][::7] == 0)
 
 
-def test_non_default_stream_and_repeat_determinism():
+def test_non_default_stream_and_repeatability():
+    """A second run on another stream: per-edge outputs and the reverse CSR are
+    bit-identical; node sums may differ in the last bits when a row is cut into
+    more than two tasks (its pieces are reduced in a run-dependent order)."""
     wl = workloads.random_graph(np.random.default_rng(5), 64, 2000, 3, 64, 34)
     a = run_gpu(wl)
     s = torch.cuda.Stream()
     with torch.cuda.stream(s):
         b = run_gpu(wl)
     s.synchronize()
-    for k in ("out", "grad_x", "grad_w", "grad_r", "rev_perm"):
-        assert torch.equal(a[k], b[k]), k     # same launch shape, same order of sums
+    for k in ("grad_w", "grad_r", "rev_ptr", "rev_perm", "dst"):
+        assert torch.equal(a[k], b[k]), k
+    for k in ("out", "grad_x"):
+        assert rel_err(a[k], b[k].double().cpu().numpy()) <= 1e-6, k
+
+
+def test_bitwise_repeatable_on_the_benchmark_graph_shape():
+    """Rows no longer than a task (as in every named workload) are cut at most
+    once, so all outputs repeat bit for bit."""
+    rng = np.random.default_rng(9)
+    n, k = 300, 128
+    dst = np.repeat(np.arange(n), k)
+    src = np.concatenate([np.sort(rng.choice(n, k, replace=False)) for _ in range(n)])
+    row_ptr, src_s, _ = workloads.csr_from_pairs(n, dst, src)
+    E = len(src_s)
+    wl = workloads.Workload("rep", 2, 128, 15, row_ptr, src_s, rng.standard_normal((E, 3), dtype=np.float32),
+                            rng.standard_normal((n, 9, 128), dtype=np.float32),
+                            rng.standard_normal((E, 15, 128), dtype=np.float32),
+                            rng.standard_normal((n, 9, 128), dtype=np.float32))
+    a, b = run_gpu(wl), run_gpu(wl)
+    for key in ("out", "grad_x", "grad_w", "grad_r"):
+        assert torch.equal(a[key], b[key]), key
 
 
 @pytest.mark.parametrize("n,e", [(1, 0), (1, 50), (2, 7), (256, 5000), (257, 5000), (70000, 300000),
