@@ -3,10 +3,11 @@
 //
 // The reverse grouping is a least-significant-digit radix sort of the source ids
 // with the edge ids as values, 8 bits per pass. Each pass is a stable counting
-// sort over tiles of kTile edges: (1) a per-tile digit histogram, (2) one
-// exclusive scan of the digit-major histogram table, (3) a stable scatter in
-// which one warp walks its tile in order, ranking equal digits inside each
-// 32-edge chunk with __match_any_sync. Stability of every pass makes the result
+// sort over tiles of kTile edges: (1) a per-tile digit histogram, (2) an
+// exclusive scan of the histogram table in (digit, tile) order, (3) a stable
+// scatter in which four warps split a tile into quarters, offset each other by
+// their digit counts, and walk their quarter in order, ranking equal digits
+// inside each 32-edge chunk with __match_any_sync. Stability of every pass makes the result
 // unique: ties (equal sources) stay in increasing edge id, so the output is
 // bit-exact and independent of scheduling. rev_ptr is the exclusive scan of the
 // per-source edge counts.
@@ -79,9 +80,46 @@ __global__ void __launch_bounds__(kScanThreads) scan_exclusive(const int32_t* in
     if (tid == 0) out[n] = carry_s;
 }
 
-// hist[d * n_tiles + t] = number of edges of tile t whose key has digit d.
+// Exclusive scan, in place, of the per-tile digit counts in tile-major order
+// hist[t * 256 + d], in the order (digit, tile): one block of 256 threads, thread
+// d runs down its digit over the tiles (coalesced rows, loads batched by 8),
+// then the 256 digit totals are scanned and added back. hist[256 * n_tiles] = total.
+__global__ void __launch_bounds__(256) scan_digit_columns(int32_t* hist, int n_tiles) {
+    __shared__ int32_t tot[256];
+    const int d = threadIdx.x;
+    int run = 0;
+    int t = 0;
+    for (; t + 8 <= n_tiles; t += 8) {
+        int v[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) v[k] = hist[(size_t)(t + k) * 256 + d];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            hist[(size_t)(t + k) * 256 + d] = run;
+            run += v[k];
+        }
+    }
+    for (; t < n_tiles; ++t) {
+        const int v = hist[(size_t)t * 256 + d];
+        hist[(size_t)t * 256 + d] = run;
+        run += v;
+    }
+    tot[d] = run;
+    __syncthreads();
+    for (int s = 1; s < 256; s <<= 1) {  // inclusive scan of the totals
+        const int v = d >= s ? tot[d - s] : 0;
+        __syncthreads();
+        tot[d] += v;
+        __syncthreads();
+    }
+    const int base = d ? tot[d - 1] : 0;
+    for (t = 0; t < n_tiles; ++t) hist[(size_t)t * 256 + d] += base;
+    if (d == 255) hist[256 * (size_t)n_tiles] = tot[255];
+}
+
+// hist[t * 256 + d] = number of edges of tile t whose key has digit d.
 __global__ void __launch_bounds__(256) tile_histogram(const int32_t* __restrict__ keys, int E, int shift,
-                                                      int n_tiles, int32_t* __restrict__ hist) {
+                                                      int32_t* __restrict__ hist) {
     __shared__ int32_t h[256];
     h[threadIdx.x] = 0;
     __syncthreads();
@@ -89,23 +127,41 @@ __global__ void __launch_bounds__(256) tile_histogram(const int32_t* __restrict_
     const int lo = t * kTile, hi = min(E, lo + kTile);
     for (int e = lo + threadIdx.x; e < hi; e += 256) atomicAdd(h + ((keys[e] >> shift) & 255), 1);
     __syncthreads();
-    hist[threadIdx.x * n_tiles + t] = h[threadIdx.x];
+    hist[(size_t)t * 256 + threadIdx.x] = h[threadIdx.x];
 }
 
-// Stable scatter of one tile per warp. vals_in == nullptr means the identity
-// (value = edge id).
+// Stable scatter of one tile per block of 4 warps: warp w takes the w-th quarter
+// of the tile; (1) each warp counts its digits, (2) the per-digit counts are
+// prefix-summed over the warps on top of the tile's scanned offsets, (3) each
+// warp walks its quarter in order, ranking equal digits inside 32-edge chunks
+// with __match_any_sync. vals_in == nullptr means the identity (value = edge id).
 __global__ void __launch_bounds__(128) tile_scatter(const int32_t* __restrict__ keys_in,
                                                     const int32_t* __restrict__ vals_in, int E, int shift,
-                                                    int n_tiles, const int32_t* __restrict__ offsets,
+                                                    const int32_t* __restrict__ offsets,
                                                     int32_t* __restrict__ keys_out, int32_t* __restrict__ vals_out) {
-    __shared__ int32_t base_s[4][256];
+    __shared__ int32_t cnt[4][256];
     const int wid = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int t = blockIdx.x * 4 + wid;
-    if (t >= n_tiles) return;  // whole warp leaves together
-    int32_t* base = base_s[wid];
-    for (int d = lane; d < 256; d += 32) base[d] = offsets[d * n_tiles + t];
+    const int t = blockIdx.x;
+    constexpr int kQuarter = kTile / 4;
+    const int lo = t * kTile + wid * kQuarter, hi = min(E, lo + kQuarter);
+    for (int d = lane; d < 256; d += 32) cnt[wid][d] = 0;
     __syncwarp();
-    const int lo = t * kTile, hi = min(E, lo + kTile);
+    for (int c = lo; c < hi; c += 32) {
+        const int e = c + lane;
+        if (e < hi) atomicAdd(&cnt[wid][(keys_in[e] >> shift) & 255], 1);
+    }
+    __syncthreads();
+    for (int d = threadIdx.x; d < 256; d += 128) {  // warp-exclusive prefix per digit
+        int run = offsets[(size_t)t * 256 + d];
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+            const int v = cnt[w][d];
+            cnt[w][d] = run;
+            run += v;
+        }
+    }
+    __syncthreads();
+    int32_t* base = cnt[wid];
     const unsigned lt = (1u << lane) - 1u;
     for (int c = lo; c < hi; c += 32) {
         const int e = c + lane;
@@ -209,11 +265,11 @@ cudaError_t build_reverse_csr(int N, int E, const int32_t* row_ptr, const int32_
     const int32_t* vin = nullptr;
     for (int pass = 0; pass < passes; ++pass) {
         const int shift = 8 * pass;
-        tile_histogram<<<n_tiles, 256, 0, s>>>(kin, E, shift, n_tiles, hist);
-        scan_exclusive<<<1, kScanThreads, 0, s>>>(hist, hist, 256 * n_tiles);
+        tile_histogram<<<n_tiles, 256, 0, s>>>(kin, E, shift, hist);
+        scan_digit_columns<<<1, 256, 0, s>>>(hist, n_tiles);
         int32_t* kout = kbuf[pass & 1];
         int32_t* vout = vbuf[pass & 1];
-        tile_scatter<<<(n_tiles + 3) / 4, 128, 0, s>>>(kin, vin, E, shift, n_tiles, hist, kout, vout);
+        tile_scatter<<<n_tiles, 128, 0, s>>>(kin, vin, E, shift, hist, kout, vout);
         kin = kout;
         vin = vout;
     }

@@ -66,7 +66,7 @@ cudaError_t launch_backward(bool o3, const BwdArgs& a, dim3 grid, size_t smem, c
 
 // Reverse CSR workspace: per-source counts, two key buffers, one value buffer,
 // and the digit-major table of per-tile histograms (tiles of kRadixTile edges).
-constexpr int kRadixTile = 4096;
+constexpr int kRadixTile = 1024;
 constexpr size_t align16_bytes(size_t b) { return (b + 15) & ~size_t(15); }
 constexpr size_t reverse_csr_workspace_bytes_for(long long N, long long E) {
     return align16_bytes(4 * (size_t)(N + 1)) + 3 * align16_bytes(4 * (size_t)E) +
