@@ -56,6 +56,7 @@ def _load():
         "etp_build_reverse_csr": [i32, i32, vp, vp, vp, vp, vp, vp, sz, vp],
         "etp_build_reverse_csr_static": [i32, i32, vp, vp, vp, vp, vp, vp],
         "etp_validate_csr": [i32, i32, vp, vp, vp, vp],
+        "etp_device_fault": [vp],
         "etp_status_string": [i32],
     }
     for name, args in sig.items():
@@ -217,6 +218,13 @@ def build_reverse_csr_static(N: int, row_ptr, src, with_dst=True, stream=None):
     _check(_load().etp_build_reverse_csr_static(N, E, _ptr(row_ptr), _ptr(src), _ptr(rev_ptr), _ptr(rev_perm),
                                                 _ptr(dst), _stream(stream)), "etp_build_reverse_csr_static")
     return rev_ptr, rev_perm, dst
+
+
+def device_fault() -> int:
+    """1 if a bounded wait inside a kernel ran out since the last call (never expected); clears it."""
+    f = ctypes.c_int()
+    _check(_load().etp_device_fault(ctypes.byref(f)), "etp_device_fault")
+    return f.value
 
 
 def validate_csr(N: int, row_ptr, src, stream=None) -> int:

@@ -9,7 +9,7 @@
 #include <string>
 #include <vector>
 
-#include "../../include/etp.h"
+#include "etp.h"
 #include "etp_device.cuh"
 #include "etp_internal.h"
 
@@ -291,6 +291,16 @@ etp_status etp_validate_csr(int N, int E, const int32_t* row_ptr, const int32_t*
     if (N < 0 || E < 0 || !row_ptr || !d_flag || (E > 0 && !src)) return ETP_ERR_INVALID_ARG;
     if (!aligned4(row_ptr) || !aligned4(d_flag) || (src && !aligned4(src))) return ETP_ERR_INVALID_ARG;
     return cuda_status(etp::validate_csr(N, E, row_ptr, src, d_flag, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+etp_status etp_device_fault(int* fault) {
+    if (!fault) return ETP_ERR_INVALID_ARG;
+    if (cudaDeviceSynchronize() != cudaSuccess) return ETP_ERR_CUDA;
+    const int f0 = etp::read_and_clear_fault<0>(), f1 = etp::read_and_clear_fault<1>();
+    const int f2 = etp::read_and_clear_fault<2>(), f3 = etp::read_and_clear_fault<3>();
+    if (f0 < 0 || f1 < 0 || f2 < 0 || f3 < 0) return ETP_ERR_CUDA;
+    *fault = f0 | f1 | f2 | f3;
+    return ETP_OK;
 }
 
 const char* etp_status_string(etp_status status) {

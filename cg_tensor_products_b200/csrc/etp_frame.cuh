@@ -54,7 +54,7 @@ namespace frame {
 
 constexpr int kThreads = kThreadsPerBlock;  // 2 warps
 constexpr int kYbufFloats = 7 * 12;         // harmonics l = 2, 3 at the 7 fitting points
-constexpr int kDbufFloats = 96;             // D_2 (5 rows x 8) then D_3 (7 rows x 8)
+constexpr int kDbufFloats = 192;            // D_2 (5 rows) then D_3 (7 rows), rows of 8 duplicated pairs
 constexpr int kTeamFloats = kYbufFloats + kDbufFloats;
 constexpr int kFitFloats = 24 + 2 * 49;     // points (padded) + A_2^-1, A_3^-1 (7 x 7 each)
 constexpr int kFitStride = 128;             // shared-memory floats reserved for the fit table
@@ -62,14 +62,14 @@ constexpr int kFitStride = 128;             // shared-memory floats reserved for
 static_assert(kFitStride >= kFitFloats && kFitStride % 4 == 0, "fit table stride");
 static_assert(kYbufFloats % 4 == 0 && kTeamFloats % 4 == 0, "team buffer alignment");
 constexpr int kHeaderFloats = kFitStride + 8;  // fit table, then the grad_r slice partials
-constexpr int kRingFwd = 24;                   // weight-ring slots (paths) per team, forward
-constexpr int kRingBwd = 8;                    // and backward (its node rows take more room)
-// Floats of one team's shared buffers: harmonics and Wigner matrices, `rows`
-// node-row buffers of D x T float2, and the weight ring.
-constexpr int team_floats(int D, int T, int rows, int ring) {
-    return kTeamFloats + rows * D * T * 2 + ring * T * 2;
-}
 static_assert(kHeaderFloats % 4 == 0, "header alignment");
+// Shared memory of one task group (the S teams of a task): 32 floats of
+// mbarriers, then two edge-weight buffers of P*C floats and `rows` node-row
+// buffers of D*C floats (all 16-byte aligned: P*C and D*C are multiples of 4).
+constexpr int kBarFloats = 32;
+constexpr int group_floats(int P, int D, int C, int rows) { return kBarFloats + 2 * P * C + rows * D * C; }
+// The backward's per-team buffers add this lane-owned x and grad_out rows (D x T float2 each).
+constexpr int bwd_team_floats(int D, int T) { return kTeamFloats + 2 * D * T * 2; }
 
 // ---------------------------------------------------------------------------
 // compile-time tables
@@ -94,18 +94,21 @@ constexpr bool has_type(int l1, int l3, int odd) {
     return false;
 }
 
+// Two channels per lane: packed fp32x2 arithmetic (one instruction for both
+// channels, each half rounded exactly as fmaf / fadd / fmul).
+__device__ __forceinline__ float2 f2_dup(float s) { return make_float2(s, s); }
+// scalar (usually a compile-time constant, kept as an immediate) times a pair
 __device__ __forceinline__ void f2_fma(float2& acc, float s, float2 v) {
     acc.x = fmaf(s, v.x, acc.x);
     acc.y = fmaf(s, v.y, acc.y);
 }
-__device__ __forceinline__ void f2_fma(float2& acc, float2 a, float2 b) {
-    acc.x = fmaf(a.x, b.x, acc.x);
-    acc.y = fmaf(a.y, b.y, acc.y);
-}
+__device__ __forceinline__ void f2_fma(float2& acc, float2 a, float2 b) { acc = __ffma2_rn(a, b, acc); }
 __device__ __forceinline__ void f2_fms(float2& acc, float2 a, float2 b) {  // acc -= a * b
     acc.x = fmaf(-a.x, b.x, acc.x);
     acc.y = fmaf(-a.y, b.y, acc.y);
 }
+__device__ __forceinline__ float2 f2_mul(float2 a, float2 b) { return __fmul2_rn(a, b); }
+__device__ __forceinline__ float2 f2_add(float2 a, float2 b) { return __fadd2_rn(a, b); }
 __device__ __forceinline__ float2 f2_zero() { return make_float2(0.f, 0.f); }
 
 // Shared-memory read that the compiler must issue where it stands: the Wigner
@@ -148,7 +151,7 @@ __device__ __forceinline__ Frame make_frame(float rx, float ry, float rz) {
     const float x = f.degenerate ? 0.f : rx * inv, y = f.degenerate ? 0.f : ry * inv;
     const float z = f.degenerate ? 1.f : rz * inv;
     const float s = copysignf(1.f, z);
-    const float a = -1.f / (s + z);
+    const float a = -__frcp_rn(s + z);
     const float b = x * y * a;
     f.R[0] = 1.f + s * x * x * a;
     f.R[1] = s * b;
@@ -188,27 +191,31 @@ __device__ __forceinline__ void team_wigner(const Frame& f, int tl, int T, unsig
             for (int c = 4; c < (L + 1) * (L + 1); ++c) ybuf[k * 12 + (c - 4)] = Y[c];
         }
         __syncwarp(tmask);
-        constexpr int n2 = 25, n3 = L >= 3 ? 49 : 0;
         const float* inv2 = fit + 24;
         const float* inv3 = fit + 24 + 49;
-        for (int idx = tl; idx < n2 + n3; idx += T) {
-            const bool is3 = idx >= n2;
-            const int j = is3 ? idx - n2 : idx;
-            const int d = is3 ? 7 : 5;
-            const int a = j / d, b = j - a * d;
-            const float* inv = is3 ? inv3 : inv2;
-            const int yoff = is3 ? 5 : 0;
+        for (int idx = tl; idx < 25; idx += T) {
+            const int a = idx / 5, b = idx - 5 * (idx / 5);
             float v = 0.f;
 #pragma unroll
-            for (int k = 0; k < NP; ++k) v = fmaf(ybuf[k * 12 + yoff + a], inv[k * 7 + b], v);
-            dbuf[(is3 ? 40 : 0) + a * 8 + b] = v;
+            for (int k = 0; k < 5; ++k) v = fmaf(ybuf[k * 12 + a], inv2[k * 7 + b], v);
+            reinterpret_cast<float2*>(dbuf + a * 16)[b] = make_float2(v, v);
+        }
+        if constexpr (L >= 3) {
+            for (int idx = tl; idx < 49; idx += T) {
+                const int a = idx / 7, b = idx - 7 * (idx / 7);
+                float v = 0.f;
+#pragma unroll
+                for (int k = 0; k < 7; ++k) v = fmaf(ybuf[k * 12 + 5 + a], inv3[k * 7 + b], v);
+                reinterpret_cast<float2*>(dbuf + 80 + a * 16)[b] = make_float2(v, v);
+            }
         }
         __syncwarp(tmask);
     }
 }
 
 // out = D_l in  (TRANS = false)   or   out (+)= D_l^T in  (TRANS = true, ACC adds)
-// D_2, D_3 rows are 8 floats apart in the team buffer and read as two float4.
+// D_2, D_3 rows are 16 floats apart in the team buffer (8 duplicated pairs),
+// read as float4 = two pairs.
 template <int l, bool TRANS, bool ACC>
 __device__ __forceinline__ void rotate(const Frame& f, const float* __restrict__ dbuf, const float2* in, float2* out) {
     constexpr int d = 2 * l + 1;
@@ -220,33 +227,34 @@ __device__ __forceinline__ void rotate(const Frame& f, const float* __restrict__
     } else {
 #pragma unroll
         for (int a = 0; a < d; ++a) {
-            float row[8];
+            float2 row[8];
             if constexpr (l == 1) {
 #pragma unroll
-                for (int b = 0; b < d; ++b) row[b] = d1(f, a, b);
+                for (int b = 0; b < d; ++b) row[b] = f2_dup(d1(f, a, b));
             } else {
-                const float4 lo = lds4(dbuf + (l == 2 ? 0 : 40) + a * 8);
-                const float4 hi = lds4(dbuf + (l == 2 ? 0 : 40) + a * 8 + 4);
-                row[0] = lo.x, row[1] = lo.y, row[2] = lo.z, row[3] = lo.w;
-                row[4] = hi.x, row[5] = hi.y, row[6] = hi.z, row[7] = hi.w;
+                const float* base = dbuf + (l == 2 ? 0 : 80) + a * 16;
+#pragma unroll
+                for (int h = 0; h < (d + 1) / 2; ++h) {
+                    const float4 q = lds4(base + 4 * h);
+                    row[2 * h] = make_float2(q.x, q.y);
+                    row[2 * h + 1] = make_float2(q.z, q.w);
+                }
             }
 #pragma unroll
             for (int b = 0; b < d; ++b) {
                 if constexpr (TRANS)
-                    f2_fma(tmp[b], row[b], in[a]);
+                    tmp[b] = __ffma2_rn(row[b], in[a], tmp[b]);
                 else
-                    f2_fma(tmp[a], row[b], in[b]);
+                    tmp[a] = __ffma2_rn(row[b], in[b], tmp[a]);
             }
         }
     }
 #pragma unroll
     for (int a = 0; a < d; ++a) {
-        if constexpr (ACC) {
-            out[a].x += tmp[a].x;
-            out[a].y += tmp[a].y;
-        } else {
+        if constexpr (ACC)
+            out[a] = f2_add(out[a], tmp[a]);
+        else
             out[a] = tmp[a];
-        }
     }
 }
 
@@ -260,144 +268,65 @@ __device__ __forceinline__ void rotate_all(const Frame& f, const float* dbuf, co
 }
 
 // ---------------------------------------------------------------------------
-// Streaming of the per-edge weights: every lane copies its own two channels of
-// each path into a ring of shared-memory slots with cp.async, a fixed number of
-// paths (DIST) ahead of their use, in the order the kernels consume them
-// (l3 outer, l1, l2 inner). Each consumption step issues one copy group and
-// waits until the group holding the step's own path has landed, so that DIST
-// copies stay in flight without holding registers. A lane reads back only what
-// it copied itself, so no cross-lane synchronisation is needed. The next edge's
-// node row (x for the forward, grad_out for the backward) rides in the group of
-// the first step of the current edge.
+// Streaming of the per-edge weights and node rows with the bulk-copy (TMA) engine:
+// one producer lane per task group issues cp.async.bulk copies of whole rows
+// (an edge's weights are P*C contiguous floats, a node row D*C) into shared
+// memory, completing on an mbarrier by transaction count; consumers wait on the
+// barrier's phase. Every wait is bounded: on time-out the kernel raises a fault
+// flag and carries on with whatever the buffer holds (stays in bounds, finishes).
 __device__ __forceinline__ unsigned smem_u32(const void* p) { return (unsigned)__cvta_generic_to_shared(p); }
-__device__ __forceinline__ void cp_async8(const void* smem, const void* gmem) {
-    asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(smem_u32(smem)), "l"(gmem) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 __device__ __forceinline__ float2 lds2(const float2* p) {
     float2 v;
     asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(smem_u32(p)));
     return v;
 }
+__device__ __forceinline__ void mbar_init(uint64_t* bar, unsigned count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_fence_init() { asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory"); }
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, unsigned bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
+}
+// 16-byte-aligned addresses, bytes a multiple of 16
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, unsigned bytes, uint64_t* bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                     smem_u32(dst)),
+                 "l"(src), "r"(bytes), "r"(smem_u32(bar))
+                 : "memory");
+}
+// Per-lane 8-byte asynchronous copies (the backward's node rows: each lane copies
+// and later reads only its own channels, so no cross-lane synchronisation).
+__device__ __forceinline__ void cp_async8(void* smem, const void* gmem) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(smem_u32(smem)), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
-// Consumption order of the paths within an edge (l3 outer, l1, l2 inner).
-template <int L, bool O3>
-struct Order {
-    static constexpr int P = PathSet<L, O3>::P;
-    static constexpr int path_at(int k) {
-        int n = 0;
-        for (int c = 0; c <= L; ++c)
-            for (int a = 0; a <= L; ++a)
-                for (int b = 0; b <= L; ++b)
-                    if (PathSet<L, O3>::allowed(a, b, c)) {
-                        if (n == k) return path_index<L, O3>(a, b, c);
-                        ++n;
-                    }
-        return -1;
+constexpr int kWaitLimit = 1 << 20;  // polls of mbarrier.try_wait before giving up
+__device__ int g_fault;              // set when a bounded wait ran out (never expected)
+// Wait for a phase of `bar`; `live` turns false (and the flag is raised) when the
+// bound runs out, after which the caller's later waits return at once.
+__device__ __forceinline__ void mbar_wait(uint64_t* bar, unsigned parity, bool& live) {
+    if (!live) return;
+    for (int i = 0; i < kWaitLimit; ++i) {
+        unsigned done;
+        asm volatile(
+            "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}"
+            : "=r"(done)
+            : "r"(smem_u32(bar)), "r"(parity)
+            : "memory");
+        if (done) return;
     }
-    static constexpr int pos(int l1, int l2, int l3) {
-        int n = 0;
-        for (int c = 0; c <= L; ++c)
-            for (int a = 0; a <= L; ++a)
-                for (int b = 0; b <= L; ++b)
-                    if (PathSet<L, O3>::allowed(a, b, c)) {
-                        if (a == l1 && b == l2 && c == l3) return n;
-                        ++n;
-                    }
-        return -1;
-    }
-};
-
-// Parts of an edge's weights in consumption order: NQ parts of PP paths. PP is
-// odd, so the lane-major slots (lane t's paths at t * PP + k) are read and
-// written without shared-memory bank conflicts.
-template <int L, bool O3>
-struct Parts {
-    static constexpr int P = PathSet<L, O3>::P;
-    static constexpr int NQ0 = P < 4 ? P : 4;
-    static constexpr int PP = ((P + NQ0 - 1) / NQ0) | 1;
-    static constexpr int NQ = (P + PP - 1) / PP;
-    static constexpr int begin(int q) { return q * PP; }
-    static constexpr int end(int q) { return (q + 1) * PP < P ? (q + 1) * PP : P; }
-    static constexpr int ring_float2(int T) { return (NQ + 1) * PP * T; }
-};
-
-// The weight pipe of one team: a ring of NQ + 1 part slots. Part q of the next
-// edge is issued when part q of the current edge starts (one edge of lead), into
-// the slot the previous part has just released; one cp.async group per part.
-// Group bookkeeping (groups numbered in issue order, part q of edge i is group
-// i NQ + q): at the start of an edge the groups of its part 0 (which also holds
-// its node rows) are complete after wait_group(NQ - 1); at the start of part q,
-// after issuing the group of the next edge's part q, wait_group(NQ) leaves the
-// current part complete.
-template <int L, bool O3>
-struct Pipe {
-    using PT = Parts<L, O3>;
-    static constexpr int P = PT::P, NQ = PT::NQ, PP = PT::PP;
-    float2* ring;          // (NQ + 1) slots of PP x T float2, lane-major
-    int T, tl, C2;
-    int slot0;             // slot of part 0 of the current edge
-    const float2* w_next;  // this lane's weights of the next edge, or nullptr
-
-    __device__ __forceinline__ float2* lane_slot(int slot) { return ring + (slot * T + tl) * PP; }
-
-    template <int q>
-    __device__ __forceinline__ void issue_part(const float2* w, int slot) {
-        float2* dst = lane_slot(slot);
-        static_for<PT::begin(q), PT::end(q)>([&](auto kc) {
-            constexpr int k = decltype(kc)::value;
-            cp_async8(dst + (k - PT::begin(q)), w + Order<L, O3>::path_at(k) * C2);
-        });
-    }
-
-    // First edge: all its parts, its node rows (issued by `rows`) in the first group.
-    template <class Rows>
-    __device__ __forceinline__ void prologue(const float2* w_first, Rows&& rows) {
-        slot0 = 0;
-        static_for<0, NQ>([&](auto qc) {
-            constexpr int q = decltype(qc)::value;
-            if (w_first) issue_part<q>(w_first, q);
-            if constexpr (q == 0) rows();
-            cp_async_commit();
-        });
-    }
-
-    __device__ __forceinline__ void edge_begin() { cp_async_wait<NQ - 1>(); }
-
-    // Start of part q of the current edge: issue the next edge's part q (and at
-    // q = 0 its node rows), wait for the current part.
-    template <int q, class Rows>
-    __device__ __forceinline__ void part_begin(Rows&& next_rows) {
-        if (w_next) issue_part<q>(w_next, (slot0 + q + NQ) % (NQ + 1));
-        if constexpr (q == 0) next_rows();
-        cp_async_commit();
-        cp_async_wait<NQ>();
-    }
-
-    // Weight of consumption position k (its part has begun).
-    template <int k>
-    __device__ __forceinline__ float2 w_at() {
-        constexpr int q = k / PP;
-        return lds2(lane_slot((slot0 + q) % (NQ + 1)) + (k - q * PP));
-    }
-
-    __device__ __forceinline__ void edge_end(const float2* next_after) {
-        slot0 = (slot0 + NQ) % (NQ + 1);
-        w_next = next_after;
-    }
-};
+    live = false;
+    atomicOr(&g_fault, 1);
+}
 
 // Combined frame weights of the (l1, l3) group for this lane's channels:
 // We[mu] = sum over even paths (l1, l2, l3) of b_p(mu) w_p, Wo[mu] likewise for
-// odd paths; degenerate edges keep only l2 = 0. Part boundaries inside the group
-// advance the pipe.
-template <int L, bool O3, int l1, int l3, class Rows>
-__device__ __forceinline__ void group_weights(Pipe<L, O3>& pp, Rows&& next_rows, bool degenerate, float2 (&We)[4],
+// odd paths; degenerate edges keep only l2 = 0. `wrow` is the edge's weight row
+// in shared memory as float2, offset to this lane's channel pair.
+template <int L, bool O3, int l1, int l3>
+__device__ __forceinline__ void group_weights(const float2* wrow, int C2, bool degenerate, float2 (&We)[4],
                                               float2 (&Wo)[4]) {
 #pragma unroll
     for (int m = 0; m < 4; ++m) {
@@ -407,10 +336,8 @@ __device__ __forceinline__ void group_weights(Pipe<L, O3>& pp, Rows&& next_rows,
     static_for<0, L + 1>([&](auto l2c) {
         constexpr int l2 = decltype(l2c)::value;
         if constexpr (PathSet<L, O3>::allowed(l1, l2, l3)) {
-            constexpr int k = Order<L, O3>::pos(l1, l2, l3);
-            constexpr int PP = Parts<L, O3>::PP;
-            if constexpr (k % PP == 0) pp.template part_begin<k / PP>(next_rows);
-            float2 w = pp.template w_at<k>();
+            constexpr int p = path_index<L, O3>(l1, l2, l3);
+            float2 w = lds2(wrow + p * C2);
             if (l2 > 0 && degenerate) w = f2_zero();
             constexpr bool odd = (l1 + l2 + l3) % 2 == 1;
             static_for<0, cmin(l1, l3) + 1>([&](auto mc) {
@@ -465,18 +392,20 @@ __device__ __forceinline__ void apply_MT(const float2 (&We)[4], const float2 (&W
     }
 }
 
-// sum over the lane's channels of  -(J_a v)^T s  for a block of degree l:  -sum J[m][m'] v[m'] s[m]
+// -(J_a v)^T s for a block of degree l, per channel of the lane:
+//   -sum_{m,m'} J[m][m'] v[m'] s[m] = -sum_{m < m'} J[m][m'] (v[m'] s[m] - v[m] s[m'])   (J antisymmetric)
 template <int l, int axis>
-__device__ __forceinline__ float gen_form(const float2* v, const float2* s) {
-    float acc = 0.f;
+__device__ __forceinline__ float2 gen_form(const float2* v, const float2* s) {
+    float2 acc = f2_zero();
     static_for<0, 2 * l + 1>([&](auto ac) {
         constexpr int a = decltype(ac)::value;
-        static_for<0, 2 * l + 1>([&](auto bc) {
+        static_for<a + 1, 2 * l + 1>([&](auto bc) {
             constexpr int b = decltype(bc)::value;
             constexpr float J = (float)etp_gen::kGen[axis][l][a][b];
             if constexpr (J != 0.f) {
-                acc = fmaf(-J, v[b].x * s[a].x, acc);
-                acc = fmaf(-J, v[b].y * s[a].y, acc);
+                float2 t = f2_mul(v[b], s[a]);
+                f2_fms(t, v[a], s[b]);
+                f2_fma(acc, -J, t);
             }
         });
     });
@@ -575,13 +504,14 @@ __device__ __forceinline__ void load_fit_tables(float* fit) {
 
 
 // ===========================================================================
-// Forward: task = a contiguous range of CSR (destination-ordered) edges.
+// Forward: task = a contiguous range of CSR (destination-ordered) edges. Per edge,
+// the producer lane bulk-copies the next edge's weight row and source row into
+// the other of two buffers while the group computes this edge.
 template <int L, bool O3>
 __global__ void __launch_bounds__(frame::kThreads, 4) etp_fwd_frame_kernel(FwdArgs a) {
     using namespace frame;
-    using PT = Parts<L, O3>;
     constexpr int D = (L + 1) * (L + 1);
-    constexpr int P = PT::P;
+    constexpr int P = PathSet<L, O3>::P;
     extern __shared__ __align__(16) float smem[];
     load_fit_tables(smem);
     const Geometry G = geometry(a.team, a.slices);
@@ -589,35 +519,49 @@ __global__ void __launch_bounds__(frame::kThreads, 4) etp_fwd_frame_kernel(FwdAr
     int k0, k1;
     task_range(a.E, G.task, a.ntasks, k0, k1);
     if (k0 >= k1) return;
-    float* team = smem + kHeaderFloats + G.team_in_block * team_floats(D, G.T, 1, PT::ring_float2(G.T) / G.T);
+    const int C2 = a.C4 * 2, C = 2 * C2;
+    const int ngroups = (kThreads / G.T) / G.S;
+    float* gbase = smem + kHeaderFloats + (G.team_in_block / G.S) * group_floats(P, D, C, 2);
+    uint64_t* bar = reinterpret_cast<uint64_t*>(gbase);
+    float* wbuf = gbase + kBarFloats;
+    float* xbuf = wbuf + 2 * P * C;
+    float* team = smem + kHeaderFloats + ngroups * group_floats(P, D, C, 2) + G.team_in_block * kTeamFloats;
     float* ybuf = team;
     float* dbuf = team + kYbufFloats;
-    float2* xbuf = reinterpret_cast<float2*>(team + kYbufFloats + kDbufFloats);
-    float2* ring = xbuf + D * G.T;
-    const int C2 = a.C4 * 2;
+    const bool producer = G.slice == 0 && G.tl == 0;
     const int cp = G.slice * G.T + G.tl;
-    const float2* x2 = reinterpret_cast<const float2*>(a.x);
-    const float2* w2 = reinterpret_cast<const float2*>(a.w);
     float2* out2 = reinterpret_cast<float2*>(a.out);
-
-    auto w_of = [&](int e) -> const float2* { return e < k1 ? w2 + (size_t)e * P * C2 + cp : nullptr; };
-    auto copy_x = [&](int j) {  // an out-of-range source reads row 0 and is zeroed later
-        const float2* src = x2 + (size_t)((unsigned)j < (unsigned)a.N ? j : 0) * D * C2 + cp;
-#pragma unroll
-        for (int k = 0; k < D; ++k) cp_async8(xbuf + k * G.T + G.tl, src + k * C2);
+    auto group_sync = [&] {
+        if (G.S == 2)
+            __syncthreads();  // the block is exactly this task's two warps
+        else
+            __syncwarp(G.tmask);
     };
+    const unsigned wbytes = 4u * P * C, xbytes = 4u * D * C;
+    auto issue = [&](int e, int slot) {
+        int j = __ldg(a.src + e);
+        j = (unsigned)j < (unsigned)a.N ? j : 0;
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        mbar_expect_tx(&bar[slot], wbytes + xbytes);
+        bulk_g2s(wbuf + slot * P * C, reinterpret_cast<const float*>(a.w) + (size_t)e * P * C, wbytes, &bar[slot]);
+        bulk_g2s(xbuf + slot * D * C, reinterpret_cast<const float*>(a.x) + (size_t)j * D * C, xbytes, &bar[slot]);
+    };
+    if (producer) {
+        mbar_init(&bar[0], 1);
+        mbar_init(&bar[1], 1);
+        mbar_fence_init();
+    }
+    group_sync();
+    if (producer) issue(k0, 0);
+    bool live = true;
 
     int row = segment_of(a.row_ptr, a.N, k0);
     int row_lo = __ldg(a.row_ptr + row), row_hi = __ldg(a.row_ptr + row + 1);
-    int j_cur = __ldg(a.src + k0);
-    Pipe<L, O3> pp{ring, G.T, G.tl, C2, 0, w_of(k0 + 1)};
-    pp.prologue(w_of(k0), [&] { copy_x(j_cur); });
-
     float2 acc[D];
 #pragma unroll
     for (int k = 0; k < D; ++k) acc[k] = f2_zero();
 
-    for (int e = k0; e < k1; ++e) {
+    for (int e = k0, it = 0; e < k1; ++e, ++it) {
         while (e >= row_hi && row < a.N - 1) {  // the edge opens a later row: store the finished one
             if (row_hi > max(row_lo, k0)) {
                 flush_row<D>(out2 + (size_t)row * D * C2 + cp, C2, acc, row_lo >= k0);
@@ -628,23 +572,22 @@ __global__ void __launch_bounds__(frame::kThreads, 4) etp_fwd_frame_kernel(FwdAr
             row_lo = row_hi;
             row_hi = __ldg(a.row_ptr + row + 1);
         }
-        const bool has_next = e + 1 < k1;
-        const int j_next = has_next ? __ldg(a.src + e + 1) : 0;
-        pp.edge_begin();
+        const int slot = it & 1;
+        if (producer && e + 1 < k1) issue(e + 1, slot ^ 1);
+        const bool valid = (unsigned)__ldg(a.src + e) < (unsigned)a.N;  // an invalid source contributes nothing
         const Frame f = make_frame(__ldg(a.r + 3 * (size_t)e), __ldg(a.r + 3 * (size_t)e + 1),
                                    __ldg(a.r + 3 * (size_t)e + 2));
         team_wigner<L>(f, G.tl, G.T, G.tmask, ybuf, dbuf, smem);
+        mbar_wait(&bar[slot], (it >> 1) & 1, live);
+        const float2* xs = reinterpret_cast<const float2*>(xbuf + slot * D * C) + cp;
+        const float2* ws = reinterpret_cast<const float2*>(wbuf + slot * P * C) + cp;
         float2 xp[D];
         {
             float2 xv[D];
-            const bool valid = (unsigned)j_cur < (unsigned)a.N;  // an invalid source contributes nothing
 #pragma unroll
-            for (int k = 0; k < D; ++k) xv[k] = valid ? lds2(xbuf + k * G.T + G.tl) : f2_zero();
+            for (int k = 0; k < D; ++k) xv[k] = valid ? lds2(xs + k * C2) : f2_zero();
             rotate_all<L>(f, dbuf, xv, xp);
         }
-        auto next_rows = [&] {
-            if (has_next) copy_x(j_next);
-        };
         static_for<0, L + 1>([&](auto l3c) {
             constexpr int l3 = decltype(l3c)::value;
             float2 y[2 * l3 + 1];
@@ -654,27 +597,27 @@ __global__ void __launch_bounds__(frame::kThreads, 4) etp_fwd_frame_kernel(FwdAr
                 constexpr int l1 = decltype(l1c)::value;
                 if constexpr (has_type<L, O3>(l1, l3, 0) || has_type<L, O3>(l1, l3, 1)) {
                     float2 We[4], Wo[4];
-                    group_weights<L, O3, l1, l3>(pp, next_rows, f.degenerate, We, Wo);
+                    group_weights<L, O3, l1, l3>(ws, C2, f.degenerate, We, Wo);
                     apply_M<L, O3, l1, l3>(We, Wo, xp + l1 * l1, y);
                 }
             });
             rotate<l3, true, true>(f, dbuf, y, acc + l3 * l3);
         });
-        pp.edge_end(w_of(e + 2));
-        j_cur = j_next;
+        group_sync();  // this slot's buffers are free for the edge after next
     }
-    cp_async_wait_all();
     flush_row<D>(out2 + (size_t)row * D * C2 + cp, C2, acc, row_lo >= k0 && row_hi <= k1);
 }
 
 // ===========================================================================
 // Backward: task = a contiguous range of reverse-CSR (source-ordered) positions.
+// Weight rows are double-buffered like the forward's; the node rows (x of the
+// source, grad_out of the destination) are single-buffered and refilled for the
+// next edge as soon as this edge has rotated them into registers.
 template <int L, bool O3>
 __global__ void __launch_bounds__(frame::kThreads, 4) etp_bwd_frame_kernel(BwdArgs a) {
     using namespace frame;
-    using PT = Parts<L, O3>;
     constexpr int D = (L + 1) * (L + 1);
-    constexpr int P = PT::P;
+    constexpr int P = PathSet<L, O3>::P;
     extern __shared__ __align__(16) float smem[];
     load_fit_tables(smem);
     const Geometry G = geometry(a.team, a.slices);
@@ -682,23 +625,30 @@ __global__ void __launch_bounds__(frame::kThreads, 4) etp_bwd_frame_kernel(BwdAr
     int k0, k1;
     task_range(a.E, G.task, a.ntasks, k0, k1);
     if (k0 >= k1) return;
+    const int C2 = a.C4 * 2, C = 2 * C2;
+    const int ngroups = (kThreads / G.T) / G.S;
     float* comb = smem + kFitStride;  // slice partials of grad_r, double-buffered by edge parity
-    float* team = smem + kHeaderFloats + G.team_in_block * team_floats(D, G.T, 2, PT::ring_float2(G.T) / G.T);
+    float* gbase = smem + kHeaderFloats + (G.team_in_block / G.S) * group_floats(P, D, C, 0);
+    uint64_t* bar = reinterpret_cast<uint64_t*>(gbase);  // [0], [1]: weight buffers
+    float* wbuf = gbase + kBarFloats;
+    float* team = smem + kHeaderFloats + ngroups * group_floats(P, D, C, 0) + G.team_in_block * bwd_team_floats(D, G.T);
     float* ybuf = team;
     float* dbuf = team + kYbufFloats;
-    float2* xbuf = reinterpret_cast<float2*>(team + kYbufFloats + kDbufFloats);
-    float2* gbuf = xbuf + D * G.T;
-    float2* ring = gbuf + D * G.T;
-    const int C2 = a.C4 * 2;
+    float2* xrow = reinterpret_cast<float2*>(team + kTeamFloats);  // this lane's channels of x[src], D x T
+    float2* grow = xrow + D * G.T;                                  // and of grad_out[dst]
+    const bool producer = G.slice == 0 && G.tl == 0;
     const int cp = G.slice * G.T + G.tl;
     const uint64_t pol_w = l2_evict_first_policy();
-    const float2* x2 = reinterpret_cast<const float2*>(a.x);
-    const float2* g2 = reinterpret_cast<const float2*>(a.g);
-    const float2* w2 = reinterpret_cast<const float2*>(a.w);
     float2* gw2 = reinterpret_cast<float2*>(a.grad_w);
     float2* gx2 = reinterpret_cast<float2*>(a.grad_x);
     const bool want_w = a.grad_w != nullptr;
     const bool want_r = a.grad_r != nullptr;
+    auto group_sync = [&] {
+        if (G.S == 2)
+            __syncthreads();  // the block is exactly this task's two warps
+        else
+            __syncwarp(G.tmask);
+    };
 
     // position q of the reverse order -> edge; out-of-range edges and rows map to
     // valid addresses and are marked invalid (they contribute and store nothing)
@@ -708,27 +658,42 @@ __global__ void __launch_bounds__(frame::kThreads, 4) etp_bwd_frame_kernel(BwdAr
         if (!valid_edge(e)) return -1;
         return a.dst ? __ldg(a.dst + e) : row_of_edge(a.row_ptr, a.N, e);
     };
-    auto w_of = [&](int q) -> const float2* {
-        if (q >= k1) return nullptr;
-        const int e = edge_at(q);
-        return w2 + (size_t)(valid_edge(e) ? e : 0) * P * C2 + cp;
+    const unsigned wbytes = 4u * P * C, xbytes = 4u * D * C;
+    auto issue_w = [&](int e, int slot) {
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        mbar_expect_tx(&bar[slot], wbytes);
+        bulk_g2s(wbuf + slot * P * C, reinterpret_cast<const float*>(a.w) + (size_t)(valid_edge(e) ? e : 0) * P * C,
+                 wbytes, &bar[slot]);
     };
-    auto copy_rows = [&](int j, int i) {
+    const float2* x2 = reinterpret_cast<const float2*>(a.x);
+    const float2* g2 = reinterpret_cast<const float2*>(a.g);
+    auto copy_x = [&](int j) {
         const float2* xs = x2 + (size_t)j * D * C2 + cp;
+#pragma unroll
+        for (int k = 0; k < D; ++k) cp_async8(xrow + k * G.T + G.tl, xs + k * C2);
+        cp_async_commit();
+    };
+    auto copy_g = [&](int i) {
         const float2* gs = g2 + (size_t)((unsigned)i < (unsigned)a.N ? i : 0) * D * C2 + cp;
 #pragma unroll
-        for (int k = 0; k < D; ++k) {
-            cp_async8(xbuf + k * G.T + G.tl, xs + k * C2);
-            cp_async8(gbuf + k * G.T + G.tl, gs + k * C2);
-        }
+        for (int k = 0; k < D; ++k) cp_async8(grow + k * G.T + G.tl, gs + k * C2);
+        cp_async_commit();
     };
 
     int row = segment_of(a.rev_ptr, a.N, k0);  // source node of position k0
     int row_lo = __ldg(a.rev_ptr + row), row_hi = __ldg(a.rev_ptr + row + 1);
     int e_cur = edge_at(k0);
     int i_cur = dst_of(e_cur);
-    Pipe<L, O3> pp{ring, G.T, G.tl, C2, 0, w_of(k0 + 1)};
-    pp.prologue(w_of(k0), [&] { copy_rows(row, i_cur); });
+    if (producer) {
+        mbar_init(&bar[0], 1);
+        mbar_init(&bar[1], 1);
+        mbar_fence_init();
+    }
+    group_sync();
+    if (producer) issue_w(e_cur, 0);
+    copy_x(row);
+    copy_g(i_cur);
+    bool live = true;
 
     float2 gx[D];
 #pragma unroll
@@ -745,7 +710,7 @@ __global__ void __launch_bounds__(frame::kThreads, 4) etp_bwd_frame_kernel(BwdAr
             row_lo = row_hi;
             row_hi = __ldg(a.rev_ptr + row + 1);
         }
-        // the next position's source row and destination (for the row prefetch)
+        // the next position's source row, edge and destination (for the prefetches)
         const bool has_next = q + 1 < k1;
         int row_next = row, e_next = 0, i_next = 0;
         if (has_next) {
@@ -754,57 +719,62 @@ __global__ void __launch_bounds__(frame::kThreads, 4) etp_bwd_frame_kernel(BwdAr
             e_next = edge_at(q + 1);
             i_next = dst_of(e_next);
         }
+        const int slot = it & 1;
+        if (producer && has_next) issue_w(e_next, slot ^ 1);
         const bool ok = valid_edge(e_cur) && (unsigned)i_cur < (unsigned)a.N;
-        pp.edge_begin();
         Frame f = make_frame(0.f, 0.f, 1.f);
         if (ok)
             f = make_frame(__ldg(a.r + 3 * (size_t)e_cur), __ldg(a.r + 3 * (size_t)e_cur + 1),
                            __ldg(a.r + 3 * (size_t)e_cur + 2));
         team_wigner<L>(f, G.tl, G.T, G.tmask, ybuf, dbuf, smem);
-        float2 xp[D], gp[D], z[D];
+        float2 xp[D], z[D];
+        cp_async_wait_all();  // this edge's node rows (this lane's copies)
         {
             float2 v[D];
 #pragma unroll
-            for (int k = 0; k < D; ++k) v[k] = ok ? lds2(xbuf + k * G.T + G.tl) : f2_zero();
+            for (int k = 0; k < D; ++k) v[k] = ok ? lds2(xrow + k * G.T + G.tl) : f2_zero();
             rotate_all<L>(f, dbuf, v, xp);
-#pragma unroll
-            for (int k = 0; k < D; ++k) v[k] = ok ? lds2(gbuf + k * G.T + G.tl) : f2_zero();
-            rotate_all<L>(f, dbuf, v, gp);
         }
+        if (has_next && row_next != row) copy_x(row_next);  // x row of the next source, behind this edge's reads
 #pragma unroll
         for (int k = 0; k < D; ++k) z[k] = f2_zero();
-        auto next_rows = [&] {
-            if (has_next) copy_rows(row_next, i_next);
-        };
+        mbar_wait(&bar[slot], (it >> 1) & 1, live);
+        const float2* ws = reinterpret_cast<const float2*>(wbuf + slot * P * C) + cp;
         float2* gwe = (want_w && ok) ? gw2 + (size_t)e_cur * P * C2 + cp : nullptr;
-        float sx = 0.f, sy = 0.f;  // dL/de_x, dL/de_y over this lane's channels
+        float2 sx2 = f2_zero(), sy2 = f2_zero();  // dL/de_x, dL/de_y per channel of this lane
         static_for<0, L + 1>([&](auto l3c) {
             constexpr int l3 = decltype(l3c)::value;
             constexpr int d3 = 2 * l3 + 1;
-            float2 y[d3];
+            float2 y[d3], gp[d3];  // gp: this block of grad_out rotated into the frame
+            {
+                float2 v[d3];
+#pragma unroll
+                for (int m = 0; m < d3; ++m) v[m] = ok ? lds2(grow + (l3 * l3 + m) * G.T + G.tl) : f2_zero();
+                rotate<l3, false, false>(f, dbuf, v, gp);
+            }
 #pragma unroll
             for (int m = 0; m < d3; ++m) y[m] = f2_zero();
             static_for<0, L + 1>([&](auto l1c) {
                 constexpr int l1 = decltype(l1c)::value;
                 if constexpr (has_type<L, O3>(l1, l3, 0) || has_type<L, O3>(l1, l3, 1)) {
                     float2 We[4], Wo[4];
-                    group_weights<L, O3, l1, l3>(pp, next_rows, f.degenerate, We, Wo);
+                    group_weights<L, O3, l1, l3>(ws, C2, f.degenerate, We, Wo);
                     apply_M<L, O3, l1, l3>(We, Wo, xp + l1 * l1, y);
-                    apply_MT<L, O3, l1, l3>(We, Wo, gp + l3 * l3, z + l1 * l1);
+                    apply_MT<L, O3, l1, l3>(We, Wo, gp, z + l1 * l1);
                     if (gwe) {
                         // products of the frame components coupled by B_p, symmetrised in +-mu
                         constexpr int mn = cmin(l1, l3);
                         float2 Pe[4], Po[4];
                         static_for<0, mn + 1>([&](auto mc) {
                             constexpr int mu = decltype(mc)::value;
-                            const float2 a1 = gp[l3 * l3 + l3 + mu], a2 = gp[l3 * l3 + l3 - mu];
+                            const float2 a1 = gp[l3 + mu], a2 = gp[l3 - mu];
                             const float2 b1 = xp[l1 * l1 + l1 + mu], b2 = xp[l1 * l1 + l1 - mu];
                             if constexpr (mu == 0) {
-                                Pe[0] = make_float2(a1.x * b1.x, a1.y * b1.y);
+                                Pe[0] = f2_mul(a1, b1);
                                 Po[0] = f2_zero();
                             } else {
-                                Pe[mu] = make_float2(fmaf(a1.x, b1.x, a2.x * b2.x), fmaf(a1.y, b1.y, a2.y * b2.y));
-                                Po[mu] = make_float2(fmaf(a1.x, b2.x, -a2.x * b1.x), fmaf(a1.y, b2.y, -a2.y * b1.y));
+                                Pe[mu] = __ffma2_rn(a1, b1, f2_mul(a2, b2));
+                                Po[mu] = __ffma2_rn(a1, b2, f2_mul(make_float2(-a2.x, -a2.y), b1));
                             }
                         });
                         static_for<0, L + 1>([&](auto l2c) {
@@ -826,66 +796,67 @@ __global__ void __launch_bounds__(frame::kThreads, 4) etp_bwd_frame_kernel(BwdAr
                 }
             });
             if (want_r) {
-                sx += gen_form<l3, 0>(gp + l3 * l3, y);
-                sy += gen_form<l3, 1>(gp + l3 * l3, y);
+                sx2 = f2_add(sx2, gen_form<l3, 0>(gp, y));
+                sy2 = f2_add(sy2, gen_form<l3, 1>(gp, y));
             }
         });
+        if (has_next) copy_g(i_next);  // grad_out row of the next destination, behind this edge's reads
         static_for<0, L + 1>([&](auto l1c) {
             constexpr int l1 = decltype(l1c)::value;
             if (want_r) {
-                sx += gen_form<l1, 0>(xp + l1 * l1, z + l1 * l1);
-                sy += gen_form<l1, 1>(xp + l1 * l1, z + l1 * l1);
+                sx2 = f2_add(sx2, gen_form<l1, 0>(xp + l1 * l1, z + l1 * l1));
+                sy2 = f2_add(sy2, gen_form<l1, 1>(xp + l1 * l1, z + l1 * l1));
             }
             rotate<l1, true, true>(f, dbuf, z + l1 * l1, gx + l1 * l1);
         });
+        // sum dL/de over the lane's channels and the team's lanes; the second
+        // slice (C = 128) hands its sum over through shared memory at the sync
+        float sx = sx2.x + sx2.y, sy = sy2.x + sy2.y;
         if (want_r) {
-            // sum over the team's lanes, then over the task's two slices (the block's two warps)
             for (int s = 1; s < G.T; s <<= 1) {
                 sx += __shfl_xor_sync(G.tmask, sx, s);
                 sy += __shfl_xor_sync(G.tmask, sy, s);
             }
-            if (G.S == 2) {
-                float* slot = comb + (it & 1) * 2;
-                if (G.slice == 1 && G.tl == 0) {
-                    slot[0] = sx;
-                    slot[1] = sy;
-                }
-                __syncthreads();
-                if (G.slice == 0) {
-                    sx += slot[0];
-                    sy += slot[1];
-                }
-            }
-            if (ok && G.slice == 0 && G.tl == 0) {
-                // grad_r = R^T (dL/de_y, -dL/de_x, 0) / |r|
-                const float gu0 = sy * f.inv_rho, gu1 = -sx * f.inv_rho;
-                float* gr = a.grad_r + 3 * (size_t)e_cur;
-                gr[0] = f.R[0] * gu0 + f.R[3] * gu1;
-                gr[1] = f.R[1] * gu0 + f.R[4] * gu1;
-                gr[2] = f.R[2] * gu0 + f.R[5] * gu1;
+            if (G.S == 2 && G.slice == 1 && G.tl == 0) {
+                comb[(it & 1) * 2] = sx;
+                comb[(it & 1) * 2 + 1] = sy;
             }
         }
-        pp.edge_end(w_of(q + 2));
+        group_sync();  // weight buffer free for the edge after next; slice partials visible
+        if (want_r && ok && G.slice == 0 && G.tl == 0) {
+            if (G.S == 2) {
+                sx += comb[(it & 1) * 2];
+                sy += comb[(it & 1) * 2 + 1];
+            }
+            // grad_r = R^T (dL/de_y, -dL/de_x, 0) / |r|
+            const float gu0 = sy * f.inv_rho, gu1 = -sx * f.inv_rho;
+            float* gr = a.grad_r + 3 * (size_t)e_cur;
+            gr[0] = f.R[0] * gu0 + f.R[3] * gu1;
+            gr[1] = f.R[1] * gu0 + f.R[4] * gu1;
+            gr[2] = f.R[2] * gu0 + f.R[5] * gu1;
+        }
         e_cur = e_next;
         i_cur = i_next;
     }
-    cp_async_wait_all();
     if (gx2) flush_row<D>(gx2 + (size_t)row * D * C2 + cp, C2, gx, row_lo >= k0 && row_hi <= k1);
 }
 
 namespace frame {
 template <int L, bool O3>
-constexpr size_t smem_bytes_for(int T, bool backward) {
+constexpr size_t smem_bytes_for(int C, int T, bool backward) {
     constexpr int D = (L + 1) * (L + 1);
+    constexpr int P = PathSet<L, O3>::P;
     const int teams = kThreads / T;
-    return sizeof(float) *
-           (size_t)(kHeaderFloats + teams * team_floats(D, T, backward ? 2 : 1, Parts<L, O3>::ring_float2(T) / T));
+    const int S = C / (2 * T);
+    const int groups = teams / S;
+    return sizeof(float) * (size_t)(kHeaderFloats + groups * group_floats(P, D, C, backward ? 0 : 2) +
+                                    teams * (backward ? bwd_team_floats(D, T) : kTeamFloats));
 }
 }  // namespace frame
 
 template <int L>
-size_t smem_bytes(bool o3, int T, bool backward) {
-    return o3 ? frame::smem_bytes_for<L, true>(T, backward) : frame::smem_bytes_for<L, false>(T, backward);
+size_t smem_bytes(bool o3, int C, int T, bool backward) {
+    return o3 ? frame::smem_bytes_for<L, true>(C, T, backward) : frame::smem_bytes_for<L, false>(C, T, backward);
 }
 
 template <int L>
@@ -896,7 +867,7 @@ int blocks_per_sm(bool o3, bool backward, size_t smem) {
         k = o3 ? (const void*)etp_bwd_frame_kernel<L, true> : (const void*)etp_bwd_frame_kernel<L, false>;
     else
         k = o3 ? (const void*)etp_fwd_frame_kernel<L, true> : (const void*)etp_fwd_frame_kernel<L, false>;
-    cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, 160 * 1024);
+    cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k, frame::kThreads, smem) != cudaSuccess) n = 1;
     return n < 1 ? 1 : n;
 }
@@ -918,5 +889,6 @@ cudaError_t launch_backward(bool o3, const BwdArgs& a, dim3 grid, size_t smem, c
         etp_bwd_frame_kernel<L, false><<<grid, frame::kThreads, smem, s>>>(a);
     return cudaGetLastError();
 }
+
 
 }  // namespace etp

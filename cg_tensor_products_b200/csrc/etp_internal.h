@@ -55,7 +55,9 @@ struct LaunchShape {
 LaunchShape launch_shape(int C, int L, bool o3, bool backward, int E, int N);
 
 template <int L>
-size_t smem_bytes(bool o3, int T, bool backward);
+size_t smem_bytes(bool o3, int C, int T, bool backward);
+template <int L>
+int read_and_clear_fault();
 template <int L>
 int blocks_per_sm(bool o3, bool backward, size_t smem);
 

@@ -24,10 +24,10 @@ LaunchShape launch_shape(int C, int L, bool o3, bool backward, int E, int N) {
     s.slices = C / (2 * s.team);
     s.tasks_per_block = (frame::kThreads / s.team) / s.slices;
     switch (L) {
-        case 0: s.smem_bytes = smem_bytes<0>(o3, s.team, backward); break;
-        case 1: s.smem_bytes = smem_bytes<1>(o3, s.team, backward); break;
-        case 2: s.smem_bytes = smem_bytes<2>(o3, s.team, backward); break;
-        default: s.smem_bytes = smem_bytes<3>(o3, s.team, backward); break;
+        case 0: s.smem_bytes = smem_bytes<0>(o3, C, s.team, backward); break;
+        case 1: s.smem_bytes = smem_bytes<1>(o3, C, s.team, backward); break;
+        case 2: s.smem_bytes = smem_bytes<2>(o3, C, s.team, backward); break;
+        default: s.smem_bytes = smem_bytes<3>(o3, C, s.team, backward); break;
     }
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 16) dev = 0;

@@ -29,7 +29,7 @@
 #include <cstdint>
 #include <mutex>
 
-#include "../../include/etp.h"
+#include "etp.h"
 #include "etp_internal.h"
 
 namespace {

@@ -189,6 +189,13 @@ ETP_API etp_status etp_build_reverse_csr_static(int N, int E, const int32_t* row
 ETP_API etp_status etp_validate_csr(int N, int E, const int32_t* row_ptr, const int32_t* src, int32_t* d_flag,
                             etp_stream_t stream);
 
+/* Kernel fault report: every wait inside the kernels (on an asynchronous bulk
+ * copy) is bounded; if one ever runs out, the kernel raises a flag, finishes its
+ * work with the data it has (staying inside its buffers) and returns, instead of
+ * hanging. This call synchronises the current device, returns the flag in
+ * *fault (0: no wait ran out since the last call) and clears it. */
+ETP_API etp_status etp_device_fault(int* fault);
+
 /* A static description of a status code. */
 ETP_API const char* etp_status_string(etp_status status);
 

@@ -36,6 +36,7 @@ def run_gpu(wl, irreps=None, with_dst=True, want=("x", "w", "r")):
     gx, gw, gr = etp.backward(plan, t["row_ptr"], t["src"], rev_ptr, rev_perm, dst, t["r"], t["x"], t["w"], t["g"],
                               want=want)
     torch.cuda.synchronize()
+    assert etp.device_fault() == 0, "a bounded wait inside a kernel ran out"
     return dict(plan=plan, out=out, rev_ptr=rev_ptr, rev_perm=rev_perm, dst=dst, grad_x=gx, grad_w=gw, grad_r=gr)
 
 

@@ -23,7 +23,7 @@ def lib():
 
 def test_exports_every_declared_symbol(lib):
     names = etp.declared_symbols()
-    assert len(names) == 11
+    assert len(names) == 12
     for n in names:
         assert hasattr(lib, n), n
 
@@ -117,6 +117,7 @@ def test_host_argument_checks(lib):
     assert V(10, 100, ok, ok, None, None) == etp.ETP_ERR_INVALID_ARG
     assert lib.etp_plan_destroy(h) == 0
     assert lib.etp_plan_destroy(None) == 0
+    assert lib.etp_device_fault(None) == etp.ETP_ERR_INVALID_ARG
     for s in range(8):
         assert lib.etp_status_string(s)
     assert lib.etp_status_string(99) == b"unknown status"
