@@ -323,11 +323,10 @@ __device__ __forceinline__ void mbar_wait(uint64_t* bar, unsigned parity, bool& 
 
 // Combined frame weights of the (l1, l3) group for this lane's channels:
 // We[mu] = sum over even paths (l1, l2, l3) of b_p(mu) w_p, Wo[mu] likewise for
-// odd paths; degenerate edges keep only l2 = 0. `wrow` is the edge's weight row
-// in shared memory as float2, offset to this lane's channel pair.
+// odd paths. `wrow` is the edge's weight row in shared memory as float2, offset
+// to this lane's channel pair.
 template <int L, bool O3, int l1, int l3>
-__device__ __forceinline__ void group_weights(const float2* wrow, int C2, bool degenerate, float2 (&We)[4],
-                                              float2 (&Wo)[4]) {
+__device__ __forceinline__ void group_weights(const float2* wrow, int C2, float2 (&We)[4], float2 (&Wo)[4]) {
 #pragma unroll
     for (int m = 0; m < 4; ++m) {
         We[m] = f2_zero();
@@ -337,8 +336,7 @@ __device__ __forceinline__ void group_weights(const float2* wrow, int C2, bool d
         constexpr int l2 = decltype(l2c)::value;
         if constexpr (PathSet<L, O3>::allowed(l1, l2, l3)) {
             constexpr int p = path_index<L, O3>(l1, l2, l3);
-            float2 w = lds2(wrow + p * C2);
-            if (l2 > 0 && degenerate) w = f2_zero();
+            const float2 w = lds2(wrow + p * C2);
             constexpr bool odd = (l1 + l2 + l3) % 2 == 1;
             static_for<0, cmin(l1, l3) + 1>([&](auto mc) {
                 constexpr int mu = decltype(mc)::value;
@@ -506,8 +504,9 @@ __device__ __forceinline__ void load_fit_tables(float* fit) {
 // ===========================================================================
 // Forward: task = a contiguous range of CSR (destination-ordered) edges. Per edge,
 // the producer lane bulk-copies the next edge's weight row and source row into
-// the other of two buffers while the group computes this edge.
-template <int L, bool O3>
+// the other of two buffers while the group computes this edge. C2T is the
+// compile-time channel-pair count (0: taken from the arguments).
+template <int L, bool O3, int C2T>
 __global__ void __launch_bounds__(frame::kThreads, 4) etp_fwd_frame_kernel(FwdArgs a) {
     using namespace frame;
     constexpr int D = (L + 1) * (L + 1);
@@ -519,7 +518,7 @@ __global__ void __launch_bounds__(frame::kThreads, 4) etp_fwd_frame_kernel(FwdAr
     int k0, k1;
     task_range(a.E, G.task, a.ntasks, k0, k1);
     if (k0 >= k1) return;
-    const int C2 = a.C4 * 2, C = 2 * C2;
+    const int C2 = C2T ? C2T : a.C4 * 2, C = 2 * C2;
     const int ngroups = (kThreads / G.T) / G.S;
     float* gbase = smem + kHeaderFloats + (G.team_in_block / G.S) * group_floats(P, D, C, 2);
     uint64_t* bar = reinterpret_cast<uint64_t*>(gbase);
@@ -577,32 +576,42 @@ __global__ void __launch_bounds__(frame::kThreads, 4) etp_fwd_frame_kernel(FwdAr
         const bool valid = (unsigned)__ldg(a.src + e) < (unsigned)a.N;  // an invalid source contributes nothing
         const Frame f = make_frame(__ldg(a.r + 3 * (size_t)e), __ldg(a.r + 3 * (size_t)e + 1),
                                    __ldg(a.r + 3 * (size_t)e + 2));
-        team_wigner<L>(f, G.tl, G.T, G.tmask, ybuf, dbuf, smem);
+        if (!f.degenerate) team_wigner<L>(f, G.tl, G.T, G.tmask, ybuf, dbuf, smem);
         mbar_wait(&bar[slot], (it >> 1) & 1, live);
         const float2* xs = reinterpret_cast<const float2*>(xbuf + slot * D * C) + cp;
         const float2* ws = reinterpret_cast<const float2*>(wbuf + slot * P * C) + cp;
-        float2 xp[D];
-        {
-            float2 xv[D];
+        if (valid && !f.degenerate) {
+            float2 xp[D];
+            {
+                float2 xv[D];
 #pragma unroll
-            for (int k = 0; k < D; ++k) xv[k] = valid ? lds2(xs + k * C2) : f2_zero();
-            rotate_all<L>(f, dbuf, xv, xp);
-        }
-        static_for<0, L + 1>([&](auto l3c) {
-            constexpr int l3 = decltype(l3c)::value;
-            float2 y[2 * l3 + 1];
+                for (int k = 0; k < D; ++k) xv[k] = lds2(xs + k * C2);
+                rotate_all<L>(f, dbuf, xv, xp);
+            }
+            static_for<0, L + 1>([&](auto l3c) {
+                constexpr int l3 = decltype(l3c)::value;
+                float2 y[2 * l3 + 1];
 #pragma unroll
-            for (int m = 0; m < 2 * l3 + 1; ++m) y[m] = f2_zero();
-            static_for<0, L + 1>([&](auto l1c) {
-                constexpr int l1 = decltype(l1c)::value;
-                if constexpr (has_type<L, O3>(l1, l3, 0) || has_type<L, O3>(l1, l3, 1)) {
-                    float2 We[4], Wo[4];
-                    group_weights<L, O3, l1, l3>(ws, C2, f.degenerate, We, Wo);
-                    apply_M<L, O3, l1, l3>(We, Wo, xp + l1 * l1, y);
-                }
+                for (int m = 0; m < 2 * l3 + 1; ++m) y[m] = f2_zero();
+                static_for<0, L + 1>([&](auto l1c) {
+                    constexpr int l1 = decltype(l1c)::value;
+                    if constexpr (has_type<L, O3>(l1, l3, 0) || has_type<L, O3>(l1, l3, 1)) {
+                        float2 We[4], Wo[4];
+                        group_weights<L, O3, l1, l3>(ws, C2, We, Wo);
+                        apply_M<L, O3, l1, l3>(We, Wo, xp + l1 * l1, y);
+                    }
+                });
+                rotate<l3, true, true>(f, dbuf, y, acc + l3 * l3);
             });
-            rotate<l3, true, true>(f, dbuf, y, acc + l3 * l3);
-        });
+        } else if (valid) {
+            // no direction: only the paths (l, 0, l) act, each as the identity
+            static_for<0, L + 1>([&](auto lc) {
+                constexpr int l = decltype(lc)::value;
+                const float2 w = lds2(ws + path_index<L, O3>(l, 0, l) * C2);
+#pragma unroll
+                for (int m = 0; m < 2 * l + 1; ++m) f2_fma(acc[l * l + m], w, lds2(xs + (l * l + m) * C2));
+            });
+        }
         group_sync();  // this slot's buffers are free for the edge after next
     }
     flush_row<D>(out2 + (size_t)row * D * C2 + cp, C2, acc, row_lo >= k0 && row_hi <= k1);
@@ -610,10 +619,11 @@ __global__ void __launch_bounds__(frame::kThreads, 4) etp_fwd_frame_kernel(FwdAr
 
 // ===========================================================================
 // Backward: task = a contiguous range of reverse-CSR (source-ordered) positions.
-// Weight rows are double-buffered like the forward's; the node rows (x of the
-// source, grad_out of the destination) are single-buffered and refilled for the
-// next edge as soon as this edge has rotated them into registers.
-template <int L, bool O3>
+// Weight rows are bulk-copied into two buffers like the forward's; the node rows
+// (x of the source, grad_out of the destination) are copied lane by lane
+// (cp.async) into lane-owned buffers, refilled for the next edge as soon as this
+// edge has read them.
+template <int L, bool O3, int C2T>
 __global__ void __launch_bounds__(frame::kThreads, 4) etp_bwd_frame_kernel(BwdArgs a) {
     using namespace frame;
     constexpr int D = (L + 1) * (L + 1);
@@ -625,7 +635,7 @@ __global__ void __launch_bounds__(frame::kThreads, 4) etp_bwd_frame_kernel(BwdAr
     int k0, k1;
     task_range(a.E, G.task, a.ntasks, k0, k1);
     if (k0 >= k1) return;
-    const int C2 = a.C4 * 2, C = 2 * C2;
+    const int C2 = C2T ? C2T : a.C4 * 2, C = 2 * C2;
     const int ngroups = (kThreads / G.T) / G.S;
     float* comb = smem + kFitStride;  // slice partials of grad_r, double-buffered by edge parity
     float* gbase = smem + kHeaderFloats + (G.team_in_block / G.S) * group_floats(P, D, C, 0);
@@ -658,7 +668,7 @@ __global__ void __launch_bounds__(frame::kThreads, 4) etp_bwd_frame_kernel(BwdAr
         if (!valid_edge(e)) return -1;
         return a.dst ? __ldg(a.dst + e) : row_of_edge(a.row_ptr, a.N, e);
     };
-    const unsigned wbytes = 4u * P * C, xbytes = 4u * D * C;
+    const unsigned wbytes = 4u * P * C;
     auto issue_w = [&](int e, int slot) {
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         mbar_expect_tx(&bar[slot], wbytes);
@@ -726,89 +736,118 @@ __global__ void __launch_bounds__(frame::kThreads, 4) etp_bwd_frame_kernel(BwdAr
         if (ok)
             f = make_frame(__ldg(a.r + 3 * (size_t)e_cur), __ldg(a.r + 3 * (size_t)e_cur + 1),
                            __ldg(a.r + 3 * (size_t)e_cur + 2));
-        team_wigner<L>(f, G.tl, G.T, G.tmask, ybuf, dbuf, smem);
-        float2 xp[D], z[D];
+        if (ok && !f.degenerate) team_wigner<L>(f, G.tl, G.T, G.tmask, ybuf, dbuf, smem);
         cp_async_wait_all();  // this edge's node rows (this lane's copies)
-        {
-            float2 v[D];
-#pragma unroll
-            for (int k = 0; k < D; ++k) v[k] = ok ? lds2(xrow + k * G.T + G.tl) : f2_zero();
-            rotate_all<L>(f, dbuf, v, xp);
-        }
-        if (has_next && row_next != row) copy_x(row_next);  // x row of the next source, behind this edge's reads
-#pragma unroll
-        for (int k = 0; k < D; ++k) z[k] = f2_zero();
         mbar_wait(&bar[slot], (it >> 1) & 1, live);
         const float2* ws = reinterpret_cast<const float2*>(wbuf + slot * P * C) + cp;
         float2* gwe = (want_w && ok) ? gw2 + (size_t)e_cur * P * C2 + cp : nullptr;
         float2 sx2 = f2_zero(), sy2 = f2_zero();  // dL/de_x, dL/de_y per channel of this lane
-        static_for<0, L + 1>([&](auto l3c) {
-            constexpr int l3 = decltype(l3c)::value;
-            constexpr int d3 = 2 * l3 + 1;
-            float2 y[d3], gp[d3];  // gp: this block of grad_out rotated into the frame
+        if (ok && !f.degenerate) {
+            float2 xp[D], z[D];
             {
-                float2 v[d3];
+                float2 v[D];
 #pragma unroll
-                for (int m = 0; m < d3; ++m) v[m] = ok ? lds2(grow + (l3 * l3 + m) * G.T + G.tl) : f2_zero();
-                rotate<l3, false, false>(f, dbuf, v, gp);
+                for (int k = 0; k < D; ++k) v[k] = lds2(xrow + k * G.T + G.tl);
+                rotate_all<L>(f, dbuf, v, xp);
             }
+            if (has_next && row_next != row) copy_x(row_next);  // next source's x row, behind this edge's reads
 #pragma unroll
-            for (int m = 0; m < d3; ++m) y[m] = f2_zero();
-            static_for<0, L + 1>([&](auto l1c) {
-                constexpr int l1 = decltype(l1c)::value;
-                if constexpr (has_type<L, O3>(l1, l3, 0) || has_type<L, O3>(l1, l3, 1)) {
-                    float2 We[4], Wo[4];
-                    group_weights<L, O3, l1, l3>(ws, C2, f.degenerate, We, Wo);
-                    apply_M<L, O3, l1, l3>(We, Wo, xp + l1 * l1, y);
-                    apply_MT<L, O3, l1, l3>(We, Wo, gp, z + l1 * l1);
-                    if (gwe) {
-                        // products of the frame components coupled by B_p, symmetrised in +-mu
-                        constexpr int mn = cmin(l1, l3);
-                        float2 Pe[4], Po[4];
-                        static_for<0, mn + 1>([&](auto mc) {
-                            constexpr int mu = decltype(mc)::value;
-                            const float2 a1 = gp[l3 + mu], a2 = gp[l3 - mu];
-                            const float2 b1 = xp[l1 * l1 + l1 + mu], b2 = xp[l1 * l1 + l1 - mu];
-                            if constexpr (mu == 0) {
-                                Pe[0] = f2_mul(a1, b1);
-                                Po[0] = f2_zero();
-                            } else {
-                                Pe[mu] = __ffma2_rn(a1, b1, f2_mul(a2, b2));
-                                Po[mu] = __ffma2_rn(a1, b2, f2_mul(make_float2(-a2.x, -a2.y), b1));
-                            }
-                        });
-                        static_for<0, L + 1>([&](auto l2c) {
-                            constexpr int l2 = decltype(l2c)::value;
-                            if constexpr (PathSet<L, O3>::allowed(l1, l2, l3)) {
-                                constexpr int p = path_index<L, O3>(l1, l2, l3);
-                                constexpr bool odd = (l1 + l2 + l3) % 2 == 1;
-                                float2 gw = f2_zero();
-                                static_for<0, mn + 1>([&](auto mc) {
-                                    constexpr int mu = decltype(mc)::value;
-                                    constexpr float b = (float)etp_gen::kFrameB[l1][l2][l3][mu];
-                                    if constexpr (b != 0.f) f2_fma(gw, b, odd ? Po[mu] : Pe[mu]);
-                                });
-                                if (l2 > 0 && f.degenerate) gw = f2_zero();
-                                st_stream2(gwe + p * C2, gw, pol_w);
-                            }
-                        });
+            for (int k = 0; k < D; ++k) z[k] = f2_zero();
+            static_for<0, L + 1>([&](auto l3c) {
+                constexpr int l3 = decltype(l3c)::value;
+                constexpr int d3 = 2 * l3 + 1;
+                float2 y[d3], gp[d3];  // gp: this block of grad_out rotated into the frame
+                {
+                    float2 v[d3];
+#pragma unroll
+                    for (int m = 0; m < d3; ++m) v[m] = lds2(grow + (l3 * l3 + m) * G.T + G.tl);
+                    rotate<l3, false, false>(f, dbuf, v, gp);
+                }
+#pragma unroll
+                for (int m = 0; m < d3; ++m) y[m] = f2_zero();
+                static_for<0, L + 1>([&](auto l1c) {
+                    constexpr int l1 = decltype(l1c)::value;
+                    if constexpr (has_type<L, O3>(l1, l3, 0) || has_type<L, O3>(l1, l3, 1)) {
+                        float2 We[4], Wo[4];
+                        group_weights<L, O3, l1, l3>(ws, C2, We, Wo);
+                        apply_M<L, O3, l1, l3>(We, Wo, xp + l1 * l1, y);
+                        apply_MT<L, O3, l1, l3>(We, Wo, gp, z + l1 * l1);
+                        if (gwe) {
+                            // products of the frame components coupled by B_p, symmetrised in +-mu
+                            constexpr int mn = cmin(l1, l3);
+                            float2 Pe[4], Po[4];
+                            static_for<0, mn + 1>([&](auto mc) {
+                                constexpr int mu = decltype(mc)::value;
+                                const float2 a1 = gp[l3 + mu], a2 = gp[l3 - mu];
+                                const float2 b1 = xp[l1 * l1 + l1 + mu], b2 = xp[l1 * l1 + l1 - mu];
+                                if constexpr (mu == 0) {
+                                    Pe[0] = f2_mul(a1, b1);
+                                    Po[0] = f2_zero();
+                                } else {
+                                    Pe[mu] = __ffma2_rn(a1, b1, f2_mul(a2, b2));
+                                    Po[mu] = f2_mul(a1, b2);
+                                    f2_fms(Po[mu], a2, b1);
+                                }
+                            });
+                            static_for<0, L + 1>([&](auto l2c) {
+                                constexpr int l2 = decltype(l2c)::value;
+                                if constexpr (PathSet<L, O3>::allowed(l1, l2, l3)) {
+                                    constexpr int p = path_index<L, O3>(l1, l2, l3);
+                                    constexpr bool odd = (l1 + l2 + l3) % 2 == 1;
+                                    float2 gw = f2_zero();
+                                    static_for<0, mn + 1>([&](auto mc) {
+                                        constexpr int mu = decltype(mc)::value;
+                                        constexpr float b = (float)etp_gen::kFrameB[l1][l2][l3][mu];
+                                        if constexpr (b != 0.f) f2_fma(gw, b, odd ? Po[mu] : Pe[mu]);
+                                    });
+                                    st_stream2(gwe + p * C2, gw, pol_w);
+                                }
+                            });
+                        }
                     }
+                });
+                if (want_r) {
+                    sx2 = f2_add(sx2, gen_form<l3, 0>(gp, y));
+                    sy2 = f2_add(sy2, gen_form<l3, 1>(gp, y));
                 }
             });
-            if (want_r) {
-                sx2 = f2_add(sx2, gen_form<l3, 0>(gp, y));
-                sy2 = f2_add(sy2, gen_form<l3, 1>(gp, y));
+            if (has_next) copy_g(i_next);  // next destination's grad_out row, behind this edge's reads
+            static_for<0, L + 1>([&](auto l1c) {
+                constexpr int l1 = decltype(l1c)::value;
+                if (want_r) {
+                    sx2 = f2_add(sx2, gen_form<l1, 0>(xp + l1 * l1, z + l1 * l1));
+                    sy2 = f2_add(sy2, gen_form<l1, 1>(xp + l1 * l1, z + l1 * l1));
+                }
+                rotate<l1, true, true>(f, dbuf, z + l1 * l1, gx + l1 * l1);
+            });
+        } else {
+            // an invalid edge contributes nothing; a degenerate one (no direction)
+            // only through the paths (l, 0, l), each the identity, and has grad_r = 0
+            if (ok) {
+                static_for<0, L + 1>([&](auto lc) {
+                    constexpr int l = decltype(lc)::value;
+                    constexpr int p0 = path_index<L, O3>(l, 0, l);
+                    const float2 w = lds2(ws + p0 * C2);
+                    float2 gw = f2_zero();
+#pragma unroll
+                    for (int m = 0; m < 2 * l + 1; ++m) {
+                        const float2 gv = lds2(grow + (l * l + m) * G.T + G.tl);
+                        f2_fma(gx[l * l + m], w, gv);
+                        f2_fma(gw, lds2(xrow + (l * l + m) * G.T + G.tl), gv);
+                    }
+                    if (gwe) st_stream2(gwe + p0 * C2, gw, pol_w);
+                });
+                if (gwe) {
+                    static_for<0, P>([&](auto pc) {
+                        constexpr int p = decltype(pc)::value;
+                        constexpr Path pt = PathSet<L, O3>::path(p);
+                        if constexpr (pt.l2 > 0) st_stream2(gwe + p * C2, f2_zero(), pol_w);
+                    });
+                }
             }
-        });
-        if (has_next) copy_g(i_next);  // grad_out row of the next destination, behind this edge's reads
-        static_for<0, L + 1>([&](auto l1c) {
-            constexpr int l1 = decltype(l1c)::value;
-            if (want_r) {
-                sx2 = f2_add(sx2, gen_form<l1, 0>(xp + l1 * l1, z + l1 * l1));
-                sy2 = f2_add(sy2, gen_form<l1, 1>(xp + l1 * l1, z + l1 * l1));
-            }
-            rotate<l1, true, true>(f, dbuf, z + l1 * l1, gx + l1 * l1);
-        });
+            if (has_next && row_next != row) copy_x(row_next);
+            if (has_next) copy_g(i_next);
+        }
         // sum dL/de over the lane's channels and the team's lanes; the second
         // slice (C = 128) hands its sum over through shared memory at the sync
         float sx = sx2.x + sx2.y, sy = sy2.x + sy2.y;
@@ -828,7 +867,7 @@ __global__ void __launch_bounds__(frame::kThreads, 4) etp_bwd_frame_kernel(BwdAr
                 sx += comb[(it & 1) * 2];
                 sy += comb[(it & 1) * 2 + 1];
             }
-            // grad_r = R^T (dL/de_y, -dL/de_x, 0) / |r|
+            // grad_r = R^T (dL/de_y, -dL/de_x, 0) / |r|   (0 for a degenerate edge: inv_rho = 0)
             const float gu0 = sy * f.inv_rho, gu1 = -sx * f.inv_rho;
             float* gr = a.grad_r + 3 * (size_t)e_cur;
             gr[0] = f.R[0] * gu0 + f.R[3] * gu1;
@@ -838,6 +877,7 @@ __global__ void __launch_bounds__(frame::kThreads, 4) etp_bwd_frame_kernel(BwdAr
         e_cur = e_next;
         i_cur = i_next;
     }
+    cp_async_wait_all();
     if (gx2) flush_row<D>(gx2 + (size_t)row * D * C2 + cp, C2, gx, row_lo >= k0 && row_hi <= k1);
 }
 
@@ -859,14 +899,22 @@ size_t smem_bytes(bool o3, int C, int T, bool backward) {
     return o3 ? frame::smem_bytes_for<L, true>(C, T, backward) : frame::smem_bytes_for<L, false>(C, T, backward);
 }
 
+// Kernel of a specialisation: compile-time channel pairs for C = 128 and C = 64.
+template <int L, bool O3, int C2T>
+const void* kernel_of(bool backward) {
+    return backward ? (const void*)etp_bwd_frame_kernel<L, O3, C2T> : (const void*)etp_fwd_frame_kernel<L, O3, C2T>;
+}
 template <int L>
-int blocks_per_sm(bool o3, bool backward, size_t smem) {
+const void* kernel_for(bool o3, bool backward, int C2) {
+    if (C2 == 64) return o3 ? kernel_of<L, true, 64>(backward) : kernel_of<L, false, 64>(backward);
+    if (C2 == 32) return o3 ? kernel_of<L, true, 32>(backward) : kernel_of<L, false, 32>(backward);
+    return o3 ? kernel_of<L, true, 0>(backward) : kernel_of<L, false, 0>(backward);
+}
+
+template <int L>
+int blocks_per_sm(bool o3, bool backward, int C, size_t smem) {
     int n = 0;
-    const void* k;
-    if (backward)
-        k = o3 ? (const void*)etp_bwd_frame_kernel<L, true> : (const void*)etp_bwd_frame_kernel<L, false>;
-    else
-        k = o3 ? (const void*)etp_fwd_frame_kernel<L, true> : (const void*)etp_fwd_frame_kernel<L, false>;
+    const void* k = kernel_for<L>(o3, backward, C / 2);
     cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k, frame::kThreads, smem) != cudaSuccess) n = 1;
     return n < 1 ? 1 : n;
@@ -874,21 +922,14 @@ int blocks_per_sm(bool o3, bool backward, size_t smem) {
 
 template <int L>
 cudaError_t launch_forward(bool o3, const FwdArgs& a, dim3 grid, size_t smem, cudaStream_t s) {
-    if (o3)
-        etp_fwd_frame_kernel<L, true><<<grid, frame::kThreads, smem, s>>>(a);
-    else
-        etp_fwd_frame_kernel<L, false><<<grid, frame::kThreads, smem, s>>>(a);
-    return cudaGetLastError();
+    void* args[] = {const_cast<FwdArgs*>(&a)};
+    return cudaLaunchKernel(kernel_for<L>(o3, false, a.C4 * 2), grid, dim3(frame::kThreads), args, smem, s);
 }
 
 template <int L>
 cudaError_t launch_backward(bool o3, const BwdArgs& a, dim3 grid, size_t smem, cudaStream_t s) {
-    if (o3)
-        etp_bwd_frame_kernel<L, true><<<grid, frame::kThreads, smem, s>>>(a);
-    else
-        etp_bwd_frame_kernel<L, false><<<grid, frame::kThreads, smem, s>>>(a);
-    return cudaGetLastError();
+    void* args[] = {const_cast<BwdArgs*>(&a)};
+    return cudaLaunchKernel(kernel_for<L>(o3, true, a.C4 * 2), grid, dim3(frame::kThreads), args, smem, s);
 }
-
 
 }  // namespace etp

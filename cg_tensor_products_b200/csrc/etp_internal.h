@@ -59,7 +59,7 @@ size_t smem_bytes(bool o3, int C, int T, bool backward);
 template <int L>
 int read_and_clear_fault();
 template <int L>
-int blocks_per_sm(bool o3, bool backward, size_t smem);
+int blocks_per_sm(bool o3, bool backward, int C, size_t smem);
 
 template <int L>
 cudaError_t launch_forward(bool o3, const FwdArgs& a, dim3 grid, size_t smem, cudaStream_t s);

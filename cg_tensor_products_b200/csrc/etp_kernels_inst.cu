@@ -20,5 +20,5 @@ int read_and_clear_fault<ETP_L>() {
     cudaMemcpyToSymbol(frame::g_fault, &zero, sizeof(int));
     return v;
 }
-template int blocks_per_sm<ETP_L>(bool, bool, size_t);
+template int blocks_per_sm<ETP_L>(bool, bool, int, size_t);
 }  // namespace etp
