@@ -49,6 +49,8 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--nodes", type=int, default=None, help="micro workloads: node count (128 neighbours each)")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-frames", action="store_true",
+                    help="kernels build the edge frames themselves (no etp_edge_frames pass)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU seconds of the oracle baseline")
     return ap.parse_args()
@@ -170,17 +172,29 @@ def kernel_source_hash():
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(kernel, workload):
-    """dram bytes per launch from a committed ncu capture of the same kernel source, else None."""
-    path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+def recorded_traffic(kernel, framed, workload, n_nodes):
+    """DRAM bytes (read + write) per launch from a committed ncu capture of the same
+    kernel source and launch, else None. The summaries under profiles/ carry lines
+    `traffic: <kernel> framed=<0|1> workload=<name> nodes=<N> source=<hash> bytes=<B>`."""
+    want = {"kernel": kernel, "framed": str(int(framed)), "workload": workload, "nodes": str(n_nodes),
+            "source": kernel_source_hash()}
+    pdir = os.path.join(ROOT, "profiles")
     try:
-        with open(path) as f:
-            d = json.load(f)
-        ent = d.get(f"{kernel}:{workload}")
-        if ent and ent.get("source_hash") == kernel_source_hash():
-            return ent["bytes_per_launch"]
-    except Exception:
-        pass
+        names = sorted(os.listdir(pdir))
+    except OSError:
+        return None
+    for name in names:
+        if not name.endswith((".md", ".txt")):
+            continue
+        with open(os.path.join(pdir, name)) as f:
+            for line in f:
+                line = line.strip().strip("`")
+                if not line.startswith("traffic: "):
+                    continue
+                parts = line[len("traffic: "):].split()
+                kv = dict(p.split("=", 1) for p in parts[1:] if "=" in p)
+                if parts and parts[0] == kernel and all(kv.get(k) == v for k, v in want.items() if k != "kernel"):
+                    return float(kv["bytes"])
     return None
 
 
@@ -298,6 +312,8 @@ def main():
     rev_perm = torch.empty(E, dtype=torch.int32, device=dev)
     dst = torch.empty(E, dtype=torch.int32, device=dev)
     ws = torch.empty(max(etp.reverse_csr_workspace_size(N, E), 16), dtype=torch.uint8, device=dev)
+    framed = not args.no_frames
+    frames = torch.empty((E, etp.FRAME_FLOATS), device=dev) if framed else None
     lib = etp._load()
     stream = torch.cuda.current_stream()
     sp = etp._stream(stream)
@@ -310,21 +326,26 @@ def main():
                                              P(ws), ws.numel(), sp), "reverse csr")
         if ev:
             ev[1].record(stream)
-        etp._check(lib.etp_forward(plan.handle, N, E, P(d["row_ptr"]), P(d["src"]), P(d["r"]), P(d["x"]), P(d["w"]),
-                                   P(out), sp), "forward")
+        if framed:
+            etp._check(lib.etp_edge_frames(plan.handle, E, P(d["r"]), P(frames), sp), "edge frames")
         if ev:
             ev[2].record(stream)
-        etp._check(lib.etp_backward(plan.handle, N, E, P(d["row_ptr"]), P(d["src"]), P(rev_ptr), P(rev_perm), P(dst),
-                                    P(d["r"]), P(d["x"]), P(d["w"]), P(d["g"]), P(gx), P(gw), P(gr), sp), "backward")
+        etp._check(lib.etp_forward(plan.handle, N, E, P(d["row_ptr"]), P(d["src"]), P(d["r"]), P(frames), P(d["x"]),
+                                   P(d["w"]), P(out), sp), "forward")
         if ev:
             ev[3].record(stream)
+        etp._check(lib.etp_backward(plan.handle, N, E, P(d["row_ptr"]), P(d["src"]), P(rev_ptr), P(rev_perm), P(dst),
+                                    P(d["r"]), P(frames), P(d["x"]), P(d["w"]), P(d["g"]), P(gx), P(gw), P(gr), sp),
+                       "backward")
+        if ev:
+            ev[4].record(stream)
 
     for _ in range(max(args.warmup, 0)):
         step()
     torch.cuda.synchronize()
 
     K = args.steps
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(K)]
     sampler = ClockSampler(physical_gpu_index(local_rank))
     sampler.start()
     time.sleep(0.3)
@@ -345,8 +366,9 @@ def main():
     clocks = sampler.stop()
     total_ms = t_start.elapsed_time(t_end)
     rc_ms = sum(e[0].elapsed_time(e[1]) for e in evs) / K
-    fwd_ms = sum(e[1].elapsed_time(e[2]) for e in evs) / K
-    bwd_ms = sum(e[2].elapsed_time(e[3]) for e in evs) / K
+    fr_ms = sum(e[1].elapsed_time(e[2]) for e in evs) / K
+    fwd_ms = sum(e[2].elapsed_time(e[3]) for e in evs) / K
+    bwd_ms = sum(e[3].elapsed_time(e[4]) for e in evs) / K
     ms_step = total_ms / K
     if world > 1:
         t = torch.tensor([ms_step], device=dev)
@@ -358,16 +380,19 @@ def main():
     alg = algorithmic(wl, plan.n_paths, nnz_total)
     peak, peak_kind = measured_peaks()
     fl_fwd, fl_bwd = flops(wl.L, plan.paths, nnz_total, wl.C, E)
-    kern = {"reverse_csr_ms": rc_ms, "forward_ms": fwd_ms, "backward_ms": bwd_ms,
+    kern = {"reverse_csr_ms": rc_ms, "edge_frames_ms": fr_ms if framed else None,
+            "forward_ms": fwd_ms, "backward_ms": bwd_ms,
             "forward_GBps": alg["fwd_bytes"] / (fwd_ms * 1e6), "backward_GBps": alg["bwd_bytes"] / (bwd_ms * 1e6),
             "forward_equiv_TFLOPs": fl_fwd / (fwd_ms * 1e9), "backward_equiv_TFLOPs": fl_bwd / (bwd_ms * 1e9),
             "forward_bytes_per_launch": alg["fwd_bytes"], "backward_bytes_per_launch": alg["bwd_bytes"],
             "forward_sparse_cg_flop_per_launch": fl_fwd, "backward_sparse_cg_flop_per_launch": fl_bwd}
     dom = "backward" if bwd_ms >= fwd_ms else "forward"
     achieved = kern[f"{dom}_GBps"]
-    roofline = {"bound": "hbm", "kernel": f"etp_{'bwd' if dom == 'backward' else 'fwd'}_kernel", "achieved": achieved,
-                "peak": peak, "unit": "GB/s", "frac": achieved / peak, "peak_source": f"{peak_kind} (hbm_gbs)",
-                "traffic": recorded_traffic(f"etp_{'bwd' if dom == 'backward' else 'fwd'}_kernel", args.workload)}
+    kname = f"etp_{'bwd' if dom == 'backward' else 'fwd'}_frame_kernel"
+    roofline = {"bound": "hbm", "kernel": f"{kname} ({'frames given' if framed else 'frames built in the kernel'})",
+                "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                "peak_source": f"{peak_kind} (hbm_gbs, burst copy)",
+                "traffic": recorded_traffic(kname, framed, args.workload, N)}
 
     # end to end through the public API with host buffers (pinned), copies inside the timed region
     e2e = None
@@ -411,7 +436,7 @@ def main():
     while (1 << (8 * passes)) < N and passes < 4:
         passes += 1
     rc_launches = (1 if E > 0 else 0) + 1 + (1 if E > 0 else 0) + ((1 if passes == 0 else 3 * passes) if E > 0 else 0)
-    launches = K * (rc_launches + 2)
+    launches = K * (rc_launches + 2 + (1 if framed and E > 0 else 0))
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -429,7 +454,8 @@ def main():
         "config": {"workload": f"{args.workload}: {DESCR[args.workload]}" + (f" (reduced to {N} nodes)" if args.nodes else ""),
                    "N": N, "E": E, "L": wl.L, "C": wl.C,
                    "P": plan.n_paths, "cg_nnz": nnz_total,
-                   "step": "reverse CSR + forward + VJP (grad_x, grad_w, grad_r), inputs resident in HBM",
+                   "step": ("reverse CSR + " + ("edge frames + " if framed else "") +
+                            "forward + VJP (grad_x, grad_w, grad_r), inputs resident in HBM"),
                    "l2": f"inputs larger than L2 (w = {wl.w.nbytes / 1e9:.2f} GB streamed per pass)",
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
         "roofline": roofline, "kernels": kern, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches,

@@ -23,6 +23,7 @@ HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "etp.h")
 ETP_OK, ETP_ERR_INVALID_ARG, ETP_ERR_UNSUPPORTED, ETP_ERR_BAD_CSR = 0, 1, 2, 3
 ETP_ERR_CUDA, ETP_ERR_ALLOC, ETP_ERR_WORKSPACE, ETP_ERR_TOO_LARGE = 4, 5, 6, 7
 STATIC_MAX_NODES = STATIC_MAX_EDGES = 1 << 18
+FRAME_FLOATS = 88  # floats of one edge frame record (ETP_FRAME_FLOATS)
 ETP_F32 = 0
 CSR_BAD_ENDPOINTS, CSR_NOT_MONOTONE, CSR_SRC_RANGE = 1, 2, 4
 
@@ -50,8 +51,9 @@ def _load():
         "etp_plan_info": [vp, vp, vp, vp, vp, vp],
         "etp_plan_couplings": [vp, vp, vp, vp, vp, vp, vp],
         "etp_plan_destroy": [vp],
-        "etp_forward": [vp, i32, i32, vp, vp, vp, vp, vp, vp, vp],
-        "etp_backward": [vp, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp],
+        "etp_edge_frames": [vp, i32, vp, vp, vp],
+        "etp_forward": [vp, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp],
+        "etp_backward": [vp, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp],
         "etp_reverse_csr_workspace_size": [i32, i32, ctypes.POINTER(sz)],
         "etp_build_reverse_csr": [i32, i32, vp, vp, vp, vp, vp, vp, sz, vp],
         "etp_build_reverse_csr_static": [i32, i32, vp, vp, vp, vp, vp, vp],
@@ -146,21 +148,34 @@ class Plan:
             pass
 
 
-def forward(plan: Plan, row_ptr, src, r, x, w, out=None, stream=None):
-    """out[i] = sum over row i of the weighted tensor products (launches etp_forward)."""
+def edge_frames(plan: Plan, r, frames=None, stream=None):
+    """Per-edge frame records [E][FRAME_FLOATS] for r (launches etp_edge_frames)."""
+    import torch
+
+    E = r.shape[0]
+    if frames is None:
+        frames = torch.empty((E, FRAME_FLOATS), device=r.device, dtype=torch.float32)
+    _need_cuda(r, frames)
+    _check(_load().etp_edge_frames(plan.handle, E, _ptr(r), _ptr(frames), _stream(stream)), "etp_edge_frames")
+    return frames
+
+
+def forward(plan: Plan, row_ptr, src, r, x, w, out=None, frames=None, stream=None):
+    """out[i] = sum over row i of the weighted tensor products (launches etp_forward).
+    frames: None, or edge_frames(plan, r) (then the kernel reads those instead of building them)."""
     import torch
 
     N, E = row_ptr.numel() - 1, src.numel()
     if out is None:
         out = torch.empty((N, plan.dim_out, plan.C), device=x.device, dtype=torch.float32)
-    _need_cuda(row_ptr, src, r, x, w, out)
-    _check(_load().etp_forward(plan.handle, N, E, _ptr(row_ptr), _ptr(src), _ptr(r), _ptr(x), _ptr(w), _ptr(out),
-                               _stream(stream)), "etp_forward")
+    _need_cuda(row_ptr, src, r, frames, x, w, out)
+    _check(_load().etp_forward(plan.handle, N, E, _ptr(row_ptr), _ptr(src), _ptr(r), _ptr(frames), _ptr(x), _ptr(w),
+                               _ptr(out), _stream(stream)), "etp_forward")
     return out
 
 
 def backward(plan: Plan, row_ptr, src, rev_ptr, rev_perm, dst, r, x, w, grad_out,
-             want=("x", "w", "r"), grad_x=None, grad_w=None, grad_r=None, stream=None):
+             want=("x", "w", "r"), grad_x=None, grad_w=None, grad_r=None, frames=None, stream=None):
     """(grad_x, grad_w, grad_r) for the cotangent grad_out (launches etp_backward); unwanted ones are None."""
     import torch
 
@@ -172,10 +187,10 @@ def backward(plan: Plan, row_ptr, src, rev_ptr, rev_perm, dst, r, x, w, grad_out
         grad_w = torch.empty((E, plan.n_paths, plan.C), device=dev, dtype=torch.float32)
     if "r" in want and grad_r is None:
         grad_r = torch.empty((E, 3), device=dev, dtype=torch.float32)
-    _need_cuda(row_ptr, src, rev_ptr, rev_perm, dst, r, x, w, grad_out, grad_x, grad_w, grad_r)
+    _need_cuda(row_ptr, src, rev_ptr, rev_perm, dst, r, frames, x, w, grad_out, grad_x, grad_w, grad_r)
     _check(_load().etp_backward(plan.handle, N, E, _ptr(row_ptr), _ptr(src), _ptr(rev_ptr), _ptr(rev_perm),
-                                _ptr(dst), _ptr(r), _ptr(x), _ptr(w), _ptr(grad_out), _ptr(grad_x), _ptr(grad_w),
-                                _ptr(grad_r), _stream(stream)), "etp_backward")
+                                _ptr(dst), _ptr(r), _ptr(frames), _ptr(x), _ptr(w), _ptr(grad_out), _ptr(grad_x),
+                                _ptr(grad_w), _ptr(grad_r), _stream(stream)), "etp_backward")
     return grad_x, grad_w, grad_r
 
 

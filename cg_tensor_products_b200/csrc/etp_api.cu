@@ -190,19 +190,46 @@ etp_status etp_plan_destroy(etp_plan_t plan) {
     return ETP_OK;
 }
 
+etp_status etp_edge_frames(etp_plan_t plan, int E, const float* r, float* frames, etp_stream_t stream) {
+    if (!plan || E < 0) return ETP_ERR_INVALID_ARG;
+    if (E == 0) return ETP_OK;
+    if (!r || !frames || !aligned4(r) || !aligned16(frames)) return ETP_ERR_INVALID_ARG;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t err;
+    switch (plan->L) {
+        case 0: err = etp::launch_edge_frames<0>(E, r, frames, s); break;
+        case 1: err = etp::launch_edge_frames<1>(E, r, frames, s); break;
+        case 2: err = etp::launch_edge_frames<2>(E, r, frames, s); break;
+        default: err = etp::launch_edge_frames<3>(E, r, frames, s); break;
+    }
+    return cuda_status(err);
+}
+
 etp_status etp_forward(etp_plan_t plan, int N, int E, const int32_t* row_ptr, const int32_t* src, const float* r,
-                       const float* x, const float* w, float* out, etp_stream_t stream) {
+                       const float* frames, const float* x, const float* w, float* out, etp_stream_t stream) {
     if (!plan || N < 0 || E < 0) return ETP_ERR_INVALID_ARG;
     if (N == 0) return E == 0 ? ETP_OK : ETP_ERR_INVALID_ARG;
     if (!row_ptr || !x || !out || !aligned4(row_ptr) || !aligned16(x) || !aligned16(out)) return ETP_ERR_INVALID_ARG;
-    if (E > 0 && (!src || !r || !w || !aligned4(src) || !aligned4(r) || !aligned16(w))) return ETP_ERR_INVALID_ARG;
+    if (E > 0 && (!src || !w || !aligned4(src) || !aligned16(w))) return ETP_ERR_INVALID_ARG;
+    if (E > 0 && (frames ? !aligned16(frames) : (!r || !aligned4(r)))) return ETP_ERR_INVALID_ARG;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     // rows cut by a task boundary are reduced onto zeros; empty rows stay zero
     cudaError_t err = cudaMemsetAsync(out, 0, sizeof(float) * (size_t)N * plan->D * plan->C, s);
     if (err != cudaSuccess || E == 0) return cuda_status(err);
-    const etp::LaunchShape sh = etp::launch_shape(plan->C, plan->L, plan->o3, false, E, N);
-    etp::FwdArgs a{N, E, row_ptr, src, r, reinterpret_cast<const float4*>(x), reinterpret_cast<const float4*>(w),
-                   reinterpret_cast<float4*>(out), plan->C / 4, sh.team, sh.slices, sh.ntasks};
+    const etp::LaunchShape sh = etp::launch_shape(plan->C, plan->L, plan->o3, false, frames != nullptr, E, N);
+    etp::FwdArgs a{N,
+                   E,
+                   row_ptr,
+                   src,
+                   r,
+                   frames,
+                   reinterpret_cast<const float4*>(x),
+                   reinterpret_cast<const float4*>(w),
+                   reinterpret_cast<float4*>(out),
+                   plan->C / 4,
+                   sh.team,
+                   sh.slices,
+                   sh.ntasks};
     switch (plan->L) {
         case 0: err = etp::launch_forward<0>(plan->o3, a, sh.grid, sh.smem_bytes, s); break;
         case 1: err = etp::launch_forward<1>(plan->o3, a, sh.grid, sh.smem_bytes, s); break;
@@ -214,8 +241,8 @@ etp_status etp_forward(etp_plan_t plan, int N, int E, const int32_t* row_ptr, co
 
 etp_status etp_backward(etp_plan_t plan, int N, int E, const int32_t* row_ptr, const int32_t* src,
                         const int32_t* rev_ptr, const int32_t* rev_perm, const int32_t* dst_of_edge, const float* r,
-                        const float* x, const float* w, const float* grad_out, float* grad_x, float* grad_w,
-                        float* grad_r, etp_stream_t stream) {
+                        const float* frames, const float* x, const float* w, const float* grad_out, float* grad_x,
+                        float* grad_w, float* grad_r, etp_stream_t stream) {
     if (!plan || N < 0 || E < 0) return ETP_ERR_INVALID_ARG;
     if (N == 0) return E == 0 ? ETP_OK : ETP_ERR_INVALID_ARG;
     if (!row_ptr || !rev_ptr || !x || !grad_out || !aligned4(row_ptr) || !aligned4(rev_ptr) || !aligned16(x) ||
@@ -223,8 +250,9 @@ etp_status etp_backward(etp_plan_t plan, int N, int E, const int32_t* row_ptr, c
         return ETP_ERR_INVALID_ARG;
     if (grad_x && !aligned16(grad_x)) return ETP_ERR_INVALID_ARG;
     if (E > 0) {
-        if (!src || !rev_perm || !r || !w || !aligned4(src) || !aligned4(rev_perm) || !aligned4(r) || !aligned16(w))
+        if (!src || !rev_perm || !w || !aligned4(src) || !aligned4(rev_perm) || !aligned16(w))
             return ETP_ERR_INVALID_ARG;
+        if (frames ? !aligned16(frames) : (!r || !aligned4(r))) return ETP_ERR_INVALID_ARG;
         if ((grad_w && !aligned16(grad_w)) || (grad_r && !aligned4(grad_r)) ||
             (dst_of_edge && !aligned4(dst_of_edge)))
             return ETP_ERR_INVALID_ARG;
@@ -238,7 +266,7 @@ etp_status etp_backward(etp_plan_t plan, int N, int E, const int32_t* row_ptr, c
     // source rows cut by a task boundary are reduced onto zeros; sources without edges stay zero
     if (grad_x) err = cudaMemsetAsync(grad_x, 0, sizeof(float) * (size_t)N * plan->D * plan->C, s);
     if (err != cudaSuccess || E == 0) return cuda_status(err);
-    const etp::LaunchShape sh = etp::launch_shape(plan->C, plan->L, plan->o3, true, E, N);
+    const etp::LaunchShape sh = etp::launch_shape(plan->C, plan->L, plan->o3, true, frames != nullptr, E, N);
     etp::BwdArgs a{N,
                    E,
                    row_ptr,
@@ -247,6 +275,7 @@ etp_status etp_backward(etp_plan_t plan, int N, int E, const int32_t* row_ptr, c
                    rev_perm,
                    dst_of_edge,
                    r,
+                   frames,
                    reinterpret_cast<const float4*>(x),
                    reinterpret_cast<const float4*>(w),
                    reinterpret_cast<const float4*>(grad_out),

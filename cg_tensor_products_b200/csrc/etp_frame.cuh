@@ -33,6 +33,7 @@
 #pragma once
 
 #include "etp_device.cuh"
+#include "etp.h"
 #include "etp_internal.h"
 
 namespace etp {
@@ -67,7 +68,16 @@ static_assert(kHeaderFloats % 4 == 0, "header alignment");
 // mbarriers, then two edge-weight buffers of P*C floats and `rows` node-row
 // buffers of D*C floats (all 16-byte aligned: P*C and D*C are multiples of 4).
 constexpr int kBarFloats = 32;
-constexpr int group_floats(int P, int D, int C, int rows) { return kBarFloats + 2 * P * C + rows * D * C; }
+// Edge frame record (floats): D_2 row-major [0, 25), D_3 row-major [25, 74), R
+// row-major [76, 85), 1/|r| at 85, the zero-length flag (1 or 0) at 86. With
+// frames given, a group also holds two records, one per weight buffer.
+constexpr int kFrameFloats = 88;
+constexpr int kFrameD3 = 25, kFrameR = 76, kFrameInvRho = 85, kFrameDegen = 86;
+static_assert(kFrameFloats % 4 == 0 && kFrameR % 4 == 0, "frame record alignment");
+static_assert(kFrameFloats == ETP_FRAME_FLOATS, "etp.h states the record size");
+constexpr int group_floats(int P, int D, int C, int rows, bool framed) {
+    return kBarFloats + 2 * P * C + rows * D * C + (framed ? 2 * kFrameFloats : 0);
+}
 // The backward's per-team buffers add this lane-owned x and grad_out rows (D x T float2 each).
 constexpr int bwd_team_floats(int D, int T) { return kTeamFloats + 2 * D * T * 2; }
 
@@ -142,6 +152,10 @@ struct Frame {
     float inv_rho;
     bool degenerate;
 };
+
+__device__ __forceinline__ float3 load_r(const float* r, int e) {
+    return make_float3(__ldg(r + 3 * (size_t)e), __ldg(r + 3 * (size_t)e + 1), __ldg(r + 3 * (size_t)e + 2));
+}
 
 __device__ __forceinline__ Frame make_frame(float rx, float ry, float rz) {
     Frame f;
@@ -498,6 +512,109 @@ __device__ __forceinline__ void load_fit_tables(float* fit) {
     __syncthreads();
 }
 
+// The frame of an edge read back from its record in shared memory.
+__device__ __forceinline__ Frame frame_of(const float* fb) {
+    Frame f;
+    const float4 q0 = lds4(fb + kFrameR), q1 = lds4(fb + kFrameR + 4), q2 = lds4(fb + kFrameR + 8);
+    f.R[0] = q0.x, f.R[1] = q0.y, f.R[2] = q0.z, f.R[3] = q0.w;
+    f.R[4] = q1.x, f.R[5] = q1.y, f.R[6] = q1.z, f.R[7] = q1.w;
+    f.R[8] = q2.x;
+    f.inv_rho = q2.y;
+    f.degenerate = q2.z != 0.f;
+    return f;
+}
+
+// The record's D_2, D_3 copied into the team's rotation buffer as duplicated
+// pairs (the layout `rotate` reads).
+template <int L>
+__device__ __forceinline__ void expand_wigner(const float* fb, int tl, int T, unsigned tmask, float* dbuf) {
+    if constexpr (L >= 2) {
+        constexpr int n = L >= 3 ? kFrameD3 + 49 : kFrameD3;
+        for (int idx = tl; idx < n; idx += T) {
+            const float v = lds(fb + idx);
+            int off;
+            if (idx < kFrameD3) {
+                const int a = idx / 5;
+                off = a * 16 + 2 * (idx - 5 * a);
+            } else {
+                const int k = idx - kFrameD3, a = k / 7;
+                off = 80 + a * 16 + 2 * (k - 7 * a);
+            }
+            *reinterpret_cast<float2*>(dbuf + off) = make_float2(v, v);
+        }
+        __syncwarp(tmask);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Edge frames: one thread per edge builds the edge's record (R, 1/|r|, the
+// zero-length flag, and D_2, D_3 of R fitted from the harmonics at the fixed
+// points, in the same operation order as the in-kernel build); the block's
+// records are staged in shared memory and leave as one contiguous write.
+constexpr int kFrameBlock = 128;
+template <int L>
+__global__ void __launch_bounds__(kFrameBlock) etp_edge_frames_kernel(int E, const float* __restrict__ r,
+                                                                       float4* __restrict__ frames) {
+    __shared__ __align__(16) float stage[kFrameBlock * kFrameFloats];
+    const int e0 = blockIdx.x * kFrameBlock;
+    const int e = e0 + threadIdx.x;
+    if (e < E) {
+        const float3 rv = load_r(r, e);
+        const Frame f = make_frame(rv.x, rv.y, rv.z);
+        float d2[25], d3[49];
+#pragma unroll
+        for (int i = 0; i < 25; ++i) d2[i] = 0.f;
+#pragma unroll
+        for (int i = 0; i < 49; ++i) d3[i] = 0.f;
+        if constexpr (L >= 2) {
+            if (!f.degenerate) {
+#pragma unroll
+                for (int k = 0; k < 2 * L + 1; ++k) {
+                    const float px = c_fit.v[3 * k], py = c_fit.v[3 * k + 1], pz = c_fit.v[3 * k + 2];
+                    const float qx = f.R[0] * px + f.R[1] * py + f.R[2] * pz;
+                    const float qy = f.R[3] * px + f.R[4] * py + f.R[5] * pz;
+                    const float qz = f.R[6] * px + f.R[7] * py + f.R[8] * pz;
+                    float Y[(L + 1) * (L + 1)];
+                    sh_unit<L, float>(qx, qy, qz, Y);
+                    if (k < 5) {
+#pragma unroll
+                        for (int a = 0; a < 5; ++a)
+#pragma unroll
+                            for (int b = 0; b < 5; ++b)
+                                d2[a * 5 + b] = fmaf(Y[4 + a], c_fit.v[24 + k * 7 + b], d2[a * 5 + b]);
+                    }
+                    if constexpr (L >= 3) {
+#pragma unroll
+                        for (int a = 0; a < 7; ++a)
+#pragma unroll
+                            for (int b = 0; b < 7; ++b)
+                                d3[a * 7 + b] = fmaf(Y[9 + a], c_fit.v[73 + k * 7 + b], d3[a * 7 + b]);
+                    }
+                }
+            }
+        }
+        float4* rec = reinterpret_cast<float4*>(stage + threadIdx.x * kFrameFloats);
+        float v[kFrameFloats];
+#pragma unroll
+        for (int i = 0; i < kFrameFloats; ++i) v[i] = 0.f;
+#pragma unroll
+        for (int i = 0; i < 25; ++i) v[i] = d2[i];
+#pragma unroll
+        for (int i = 0; i < 49; ++i) v[kFrameD3 + i] = d3[i];
+#pragma unroll
+        for (int i = 0; i < 9; ++i) v[kFrameR + i] = f.R[i];
+        v[kFrameInvRho] = f.inv_rho;
+        v[kFrameDegen] = f.degenerate ? 1.f : 0.f;
+#pragma unroll
+        for (int i = 0; i < kFrameFloats / 4; ++i) rec[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+    }
+    __syncthreads();
+    const int n = min(kFrameBlock, E - e0) * (kFrameFloats / 4);
+    float4* dst = frames + (size_t)e0 * (kFrameFloats / 4);
+    const float4* st = reinterpret_cast<const float4*>(stage);
+    for (int i = threadIdx.x; i < n; i += kFrameBlock) dst[i] = st[i];
+}
+
 }  // namespace frame
 
 
@@ -505,14 +622,15 @@ __device__ __forceinline__ void load_fit_tables(float* fit) {
 // Forward: task = a contiguous range of CSR (destination-ordered) edges. Per edge,
 // the producer lane bulk-copies the next edge's weight row and source row into
 // the other of two buffers while the group computes this edge. C2T is the
-// compile-time channel-pair count (0: taken from the arguments).
-template <int L, bool O3, int C2T>
+// compile-time channel-pair count (0: taken from the arguments). FR: the edges'
+// frame records are given (copied with the weights) instead of built here.
+template <int L, bool O3, int C2T, bool FR>
 __global__ void __launch_bounds__(frame::kThreads, 4) etp_fwd_frame_kernel(FwdArgs a) {
     using namespace frame;
     constexpr int D = (L + 1) * (L + 1);
     constexpr int P = PathSet<L, O3>::P;
     extern __shared__ __align__(16) float smem[];
-    load_fit_tables(smem);
+    if constexpr (!FR) load_fit_tables(smem);
     const Geometry G = geometry(a.team, a.slices);
     if (G.task >= a.ntasks) return;  // the slice teams of a task leave together
     int k0, k1;
@@ -520,11 +638,13 @@ __global__ void __launch_bounds__(frame::kThreads, 4) etp_fwd_frame_kernel(FwdAr
     if (k0 >= k1) return;
     const int C2 = C2T ? C2T : a.C4 * 2, C = 2 * C2;
     const int ngroups = (kThreads / G.T) / G.S;
-    float* gbase = smem + kHeaderFloats + (G.team_in_block / G.S) * group_floats(P, D, C, 2);
+    const int gfloats = group_floats(P, D, C, 2, FR);
+    float* gbase = smem + kHeaderFloats + (G.team_in_block / G.S) * gfloats;
     uint64_t* bar = reinterpret_cast<uint64_t*>(gbase);
     float* wbuf = gbase + kBarFloats;
     float* xbuf = wbuf + 2 * P * C;
-    float* team = smem + kHeaderFloats + ngroups * group_floats(P, D, C, 2) + G.team_in_block * kTeamFloats;
+    float* fbuf = xbuf + 2 * D * C;  // two frame records (FR)
+    float* team = smem + kHeaderFloats + ngroups * gfloats + G.team_in_block * kTeamFloats;
     float* ybuf = team;
     float* dbuf = team + kYbufFloats;
     const bool producer = G.slice == 0 && G.tl == 0;
@@ -536,14 +656,15 @@ __global__ void __launch_bounds__(frame::kThreads, 4) etp_fwd_frame_kernel(FwdAr
         else
             __syncwarp(G.tmask);
     };
-    const unsigned wbytes = 4u * P * C, xbytes = 4u * D * C;
-    auto issue = [&](int e, int slot) {
-        int j = __ldg(a.src + e);
+    const unsigned wbytes = 4u * P * C, xbytes = 4u * D * C, fbytes = FR ? 4u * kFrameFloats : 0u;
+    auto issue = [&](int e, int j, int slot) {
         j = (unsigned)j < (unsigned)a.N ? j : 0;
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        mbar_expect_tx(&bar[slot], wbytes + xbytes);
+        mbar_expect_tx(&bar[slot], wbytes + xbytes + fbytes);
         bulk_g2s(wbuf + slot * P * C, reinterpret_cast<const float*>(a.w) + (size_t)e * P * C, wbytes, &bar[slot]);
         bulk_g2s(xbuf + slot * D * C, reinterpret_cast<const float*>(a.x) + (size_t)j * D * C, xbytes, &bar[slot]);
+        if constexpr (FR)
+            bulk_g2s(fbuf + slot * kFrameFloats, a.frames + (size_t)e * kFrameFloats, fbytes, &bar[slot]);
     };
     if (producer) {
         mbar_init(&bar[0], 1);
@@ -551,7 +672,12 @@ __global__ void __launch_bounds__(frame::kThreads, 4) etp_fwd_frame_kernel(FwdAr
         mbar_fence_init();
     }
     group_sync();
-    if (producer) issue(k0, 0);
+    // source indices one and two edges ahead and the next edge vector are loaded
+    // an edge early, so their latency hides behind an edge of compute
+    int j_cur = __ldg(a.src + k0);
+    int j_next = k0 + 1 < k1 ? __ldg(a.src + k0 + 1) : 0;
+    float3 r_cur = FR ? make_float3(0.f, 0.f, 1.f) : load_r(a.r, k0);
+    if (producer) issue(k0, j_cur, 0);
     bool live = true;
 
     int row = segment_of(a.row_ptr, a.N, k0);
@@ -572,12 +698,21 @@ __global__ void __launch_bounds__(frame::kThreads, 4) etp_fwd_frame_kernel(FwdAr
             row_hi = __ldg(a.row_ptr + row + 1);
         }
         const int slot = it & 1;
-        if (producer && e + 1 < k1) issue(e + 1, slot ^ 1);
-        const bool valid = (unsigned)__ldg(a.src + e) < (unsigned)a.N;  // an invalid source contributes nothing
-        const Frame f = make_frame(__ldg(a.r + 3 * (size_t)e), __ldg(a.r + 3 * (size_t)e + 1),
-                                   __ldg(a.r + 3 * (size_t)e + 2));
-        if (!f.degenerate) team_wigner<L>(f, G.tl, G.T, G.tmask, ybuf, dbuf, smem);
-        mbar_wait(&bar[slot], (it >> 1) & 1, live);
+        if (producer && e + 1 < k1) issue(e + 1, j_next, slot ^ 1);
+        const int j_after = e + 2 < k1 ? __ldg(a.src + e + 2) : 0;
+        const float3 r_next = (!FR && e + 1 < k1) ? load_r(a.r, e + 1) : r_cur;
+        const bool valid = (unsigned)j_cur < (unsigned)a.N;  // an invalid source contributes nothing
+        Frame f;
+        if constexpr (FR) {
+            mbar_wait(&bar[slot], (it >> 1) & 1, live);
+            const float* fb = fbuf + slot * kFrameFloats;
+            f = frame_of(fb);
+            if (!f.degenerate) expand_wigner<L>(fb, G.tl, G.T, G.tmask, dbuf);
+        } else {
+            f = make_frame(r_cur.x, r_cur.y, r_cur.z);
+            if (!f.degenerate) team_wigner<L>(f, G.tl, G.T, G.tmask, ybuf, dbuf, smem);
+            mbar_wait(&bar[slot], (it >> 1) & 1, live);
+        }
         const float2* xs = reinterpret_cast<const float2*>(xbuf + slot * D * C) + cp;
         const float2* ws = reinterpret_cast<const float2*>(wbuf + slot * P * C) + cp;
         if (valid && !f.degenerate) {
@@ -613,6 +748,9 @@ __global__ void __launch_bounds__(frame::kThreads, 4) etp_fwd_frame_kernel(FwdAr
             });
         }
         group_sync();  // this slot's buffers are free for the edge after next
+        j_cur = j_next;
+        j_next = j_after;
+        r_cur = r_next;
     }
     flush_row<D>(out2 + (size_t)row * D * C2 + cp, C2, acc, row_lo >= k0 && row_hi <= k1);
 }
@@ -622,14 +760,14 @@ __global__ void __launch_bounds__(frame::kThreads, 4) etp_fwd_frame_kernel(FwdAr
 // Weight rows are bulk-copied into two buffers like the forward's; the node rows
 // (x of the source, grad_out of the destination) are copied lane by lane
 // (cp.async) into lane-owned buffers, refilled for the next edge as soon as this
-// edge has read them.
-template <int L, bool O3, int C2T>
+// edge has read them. FR: frame records given, as in the forward.
+template <int L, bool O3, int C2T, bool FR>
 __global__ void __launch_bounds__(frame::kThreads, 4) etp_bwd_frame_kernel(BwdArgs a) {
     using namespace frame;
     constexpr int D = (L + 1) * (L + 1);
     constexpr int P = PathSet<L, O3>::P;
     extern __shared__ __align__(16) float smem[];
-    load_fit_tables(smem);
+    if constexpr (!FR) load_fit_tables(smem);
     const Geometry G = geometry(a.team, a.slices);
     if (G.task >= a.ntasks) return;  // the slice teams of a task leave together
     int k0, k1;
@@ -638,10 +776,12 @@ __global__ void __launch_bounds__(frame::kThreads, 4) etp_bwd_frame_kernel(BwdAr
     const int C2 = C2T ? C2T : a.C4 * 2, C = 2 * C2;
     const int ngroups = (kThreads / G.T) / G.S;
     float* comb = smem + kFitStride;  // slice partials of grad_r, double-buffered by edge parity
-    float* gbase = smem + kHeaderFloats + (G.team_in_block / G.S) * group_floats(P, D, C, 0);
+    const int gfloats = group_floats(P, D, C, 0, FR);
+    float* gbase = smem + kHeaderFloats + (G.team_in_block / G.S) * gfloats;
     uint64_t* bar = reinterpret_cast<uint64_t*>(gbase);  // [0], [1]: weight buffers
     float* wbuf = gbase + kBarFloats;
-    float* team = smem + kHeaderFloats + ngroups * group_floats(P, D, C, 0) + G.team_in_block * bwd_team_floats(D, G.T);
+    float* fbuf = wbuf + 2 * P * C;  // two frame records (FR)
+    float* team = smem + kHeaderFloats + ngroups * gfloats + G.team_in_block * bwd_team_floats(D, G.T);
     float* ybuf = team;
     float* dbuf = team + kYbufFloats;
     float2* xrow = reinterpret_cast<float2*>(team + kTeamFloats);  // this lane's channels of x[src], D x T
@@ -668,12 +808,14 @@ __global__ void __launch_bounds__(frame::kThreads, 4) etp_bwd_frame_kernel(BwdAr
         if (!valid_edge(e)) return -1;
         return a.dst ? __ldg(a.dst + e) : row_of_edge(a.row_ptr, a.N, e);
     };
-    const unsigned wbytes = 4u * P * C;
+    const unsigned wbytes = 4u * P * C, fbytes = FR ? 4u * kFrameFloats : 0u;
     auto issue_w = [&](int e, int slot) {
+        e = valid_edge(e) ? e : 0;
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        mbar_expect_tx(&bar[slot], wbytes);
-        bulk_g2s(wbuf + slot * P * C, reinterpret_cast<const float*>(a.w) + (size_t)(valid_edge(e) ? e : 0) * P * C,
-                 wbytes, &bar[slot]);
+        mbar_expect_tx(&bar[slot], wbytes + fbytes);
+        bulk_g2s(wbuf + slot * P * C, reinterpret_cast<const float*>(a.w) + (size_t)e * P * C, wbytes, &bar[slot]);
+        if constexpr (FR)
+            bulk_g2s(fbuf + slot * kFrameFloats, a.frames + (size_t)e * kFrameFloats, fbytes, &bar[slot]);
     };
     const float2* x2 = reinterpret_cast<const float2*>(a.x);
     const float2* g2 = reinterpret_cast<const float2*>(a.g);
@@ -692,8 +834,12 @@ __global__ void __launch_bounds__(frame::kThreads, 4) etp_bwd_frame_kernel(BwdAr
 
     int row = segment_of(a.rev_ptr, a.N, k0);  // source node of position k0
     int row_lo = __ldg(a.rev_ptr + row), row_hi = __ldg(a.rev_ptr + row + 1);
+    // the edge of the next position and the destination and vector of the next
+    // edge are loaded an edge early (the position after next: two early)
     int e_cur = edge_at(k0);
     int i_cur = dst_of(e_cur);
+    int e_next = k0 + 1 < k1 ? edge_at(k0 + 1) : 0;
+    float3 r_cur = FR ? make_float3(0.f, 0.f, 1.f) : load_r(a.r, valid_edge(e_cur) ? e_cur : 0);
     if (producer) {
         mbar_init(&bar[0], 1);
         mbar_init(&bar[1], 1);
@@ -722,23 +868,30 @@ __global__ void __launch_bounds__(frame::kThreads, 4) etp_bwd_frame_kernel(BwdAr
         }
         // the next position's source row, edge and destination (for the prefetches)
         const bool has_next = q + 1 < k1;
-        int row_next = row, e_next = 0, i_next = 0;
+        const int slot = it & 1;
+        if (producer && has_next) issue_w(e_next, slot ^ 1);
+        int row_next = row;
         if (has_next) {
             int hi = row_hi;
             while (q + 1 >= hi && row_next < a.N - 1) hi = __ldg(a.rev_ptr + (++row_next) + 1);
-            e_next = edge_at(q + 1);
-            i_next = dst_of(e_next);
         }
-        const int slot = it & 1;
-        if (producer && has_next) issue_w(e_next, slot ^ 1);
+        const int e_after = q + 2 < k1 ? edge_at(q + 2) : 0;
+        const int i_next = has_next ? dst_of(e_next) : 0;
+        const float3 r_next = (!FR && has_next) ? load_r(a.r, valid_edge(e_next) ? e_next : 0) : r_cur;
         const bool ok = valid_edge(e_cur) && (unsigned)i_cur < (unsigned)a.N;
-        Frame f = make_frame(0.f, 0.f, 1.f);
-        if (ok)
-            f = make_frame(__ldg(a.r + 3 * (size_t)e_cur), __ldg(a.r + 3 * (size_t)e_cur + 1),
-                           __ldg(a.r + 3 * (size_t)e_cur + 2));
-        if (ok && !f.degenerate) team_wigner<L>(f, G.tl, G.T, G.tmask, ybuf, dbuf, smem);
-        cp_async_wait_all();  // this edge's node rows (this lane's copies)
-        mbar_wait(&bar[slot], (it >> 1) & 1, live);
+        Frame f;
+        if constexpr (FR) {
+            cp_async_wait_all();  // this edge's node rows (this lane's copies)
+            mbar_wait(&bar[slot], (it >> 1) & 1, live);
+            const float* fb = fbuf + slot * kFrameFloats;
+            f = frame_of(fb);
+            if (ok && !f.degenerate) expand_wigner<L>(fb, G.tl, G.T, G.tmask, dbuf);
+        } else {
+            f = ok ? make_frame(r_cur.x, r_cur.y, r_cur.z) : make_frame(0.f, 0.f, 1.f);
+            if (ok && !f.degenerate) team_wigner<L>(f, G.tl, G.T, G.tmask, ybuf, dbuf, smem);
+            cp_async_wait_all();  // this edge's node rows (this lane's copies)
+            mbar_wait(&bar[slot], (it >> 1) & 1, live);
+        }
         const float2* ws = reinterpret_cast<const float2*>(wbuf + slot * P * C) + cp;
         float2* gwe = (want_w && ok) ? gw2 + (size_t)e_cur * P * C2 + cp : nullptr;
         float2 sx2 = f2_zero(), sy2 = f2_zero();  // dL/de_x, dL/de_y per channel of this lane
@@ -876,6 +1029,8 @@ __global__ void __launch_bounds__(frame::kThreads, 4) etp_bwd_frame_kernel(BwdAr
         }
         e_cur = e_next;
         i_cur = i_next;
+        e_next = e_after;
+        r_cur = r_next;
     }
     cp_async_wait_all();
     if (gx2) flush_row<D>(gx2 + (size_t)row * D * C2 + cp, C2, gx, row_lo >= k0 && row_hi <= k1);
@@ -883,38 +1038,44 @@ __global__ void __launch_bounds__(frame::kThreads, 4) etp_bwd_frame_kernel(BwdAr
 
 namespace frame {
 template <int L, bool O3>
-constexpr size_t smem_bytes_for(int C, int T, bool backward) {
+constexpr size_t smem_bytes_for(int C, int T, bool backward, bool framed) {
     constexpr int D = (L + 1) * (L + 1);
     constexpr int P = PathSet<L, O3>::P;
     const int teams = kThreads / T;
     const int S = C / (2 * T);
     const int groups = teams / S;
-    return sizeof(float) * (size_t)(kHeaderFloats + groups * group_floats(P, D, C, backward ? 0 : 2) +
+    return sizeof(float) * (size_t)(kHeaderFloats + groups * group_floats(P, D, C, backward ? 0 : 2, framed) +
                                     teams * (backward ? bwd_team_floats(D, T) : kTeamFloats));
 }
 }  // namespace frame
 
 template <int L>
-size_t smem_bytes(bool o3, int C, int T, bool backward) {
-    return o3 ? frame::smem_bytes_for<L, true>(C, T, backward) : frame::smem_bytes_for<L, false>(C, T, backward);
+size_t smem_bytes(bool o3, int C, int T, bool backward, bool framed) {
+    return o3 ? frame::smem_bytes_for<L, true>(C, T, backward, framed)
+              : frame::smem_bytes_for<L, false>(C, T, backward, framed);
 }
 
-// Kernel of a specialisation: compile-time channel pairs for C = 128 and C = 64.
+// Kernel of a specialisation: compile-time channel pairs for C = 128 and C = 64;
+// frame records given or built in the kernel.
 template <int L, bool O3, int C2T>
-const void* kernel_of(bool backward) {
-    return backward ? (const void*)etp_bwd_frame_kernel<L, O3, C2T> : (const void*)etp_fwd_frame_kernel<L, O3, C2T>;
+const void* kernel_of(bool backward, bool framed) {
+    if (framed)
+        return backward ? (const void*)etp_bwd_frame_kernel<L, O3, C2T, true>
+                        : (const void*)etp_fwd_frame_kernel<L, O3, C2T, true>;
+    return backward ? (const void*)etp_bwd_frame_kernel<L, O3, C2T, false>
+                    : (const void*)etp_fwd_frame_kernel<L, O3, C2T, false>;
 }
 template <int L>
-const void* kernel_for(bool o3, bool backward, int C2) {
-    if (C2 == 64) return o3 ? kernel_of<L, true, 64>(backward) : kernel_of<L, false, 64>(backward);
-    if (C2 == 32) return o3 ? kernel_of<L, true, 32>(backward) : kernel_of<L, false, 32>(backward);
-    return o3 ? kernel_of<L, true, 0>(backward) : kernel_of<L, false, 0>(backward);
+const void* kernel_for(bool o3, bool backward, bool framed, int C2) {
+    if (C2 == 64) return o3 ? kernel_of<L, true, 64>(backward, framed) : kernel_of<L, false, 64>(backward, framed);
+    if (C2 == 32) return o3 ? kernel_of<L, true, 32>(backward, framed) : kernel_of<L, false, 32>(backward, framed);
+    return o3 ? kernel_of<L, true, 0>(backward, framed) : kernel_of<L, false, 0>(backward, framed);
 }
 
 template <int L>
-int blocks_per_sm(bool o3, bool backward, int C, size_t smem) {
+int blocks_per_sm(bool o3, bool backward, bool framed, int C, size_t smem) {
     int n = 0;
-    const void* k = kernel_for<L>(o3, backward, C / 2);
+    const void* k = kernel_for<L>(o3, backward, framed, C / 2);
     cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k, frame::kThreads, smem) != cudaSuccess) n = 1;
     return n < 1 ? 1 : n;
@@ -923,13 +1084,23 @@ int blocks_per_sm(bool o3, bool backward, int C, size_t smem) {
 template <int L>
 cudaError_t launch_forward(bool o3, const FwdArgs& a, dim3 grid, size_t smem, cudaStream_t s) {
     void* args[] = {const_cast<FwdArgs*>(&a)};
-    return cudaLaunchKernel(kernel_for<L>(o3, false, a.C4 * 2), grid, dim3(frame::kThreads), args, smem, s);
+    return cudaLaunchKernel(kernel_for<L>(o3, false, a.frames != nullptr, a.C4 * 2), grid, dim3(frame::kThreads), args,
+                            smem, s);
 }
 
 template <int L>
 cudaError_t launch_backward(bool o3, const BwdArgs& a, dim3 grid, size_t smem, cudaStream_t s) {
     void* args[] = {const_cast<BwdArgs*>(&a)};
-    return cudaLaunchKernel(kernel_for<L>(o3, true, a.C4 * 2), grid, dim3(frame::kThreads), args, smem, s);
+    return cudaLaunchKernel(kernel_for<L>(o3, true, a.frames != nullptr, a.C4 * 2), grid, dim3(frame::kThreads), args,
+                            smem, s);
+}
+
+template <int L>
+cudaError_t launch_edge_frames(int E, const float* r, float* frames, cudaStream_t s) {
+    if (E == 0) return cudaSuccess;
+    const unsigned blocks = (unsigned)((E + frame::kFrameBlock - 1) / frame::kFrameBlock);
+    frame::etp_edge_frames_kernel<L><<<blocks, frame::kFrameBlock, 0, s>>>(E, r, reinterpret_cast<float4*>(frames));
+    return cudaGetLastError();
 }
 
 }  // namespace etp

@@ -15,6 +15,7 @@ struct FwdArgs {
     const int32_t* row_ptr;
     const int32_t* src;
     const float* r;
+    const float* frames;  // may be null: frames built in the kernel
     const float4* x;
     const float4* w;
     float4* out;
@@ -32,6 +33,7 @@ struct BwdArgs {
     const int32_t* rev_perm;
     const int32_t* dst;  // may be null
     const float* r;
+    const float* frames;  // may be null: frames built in the kernel
     const float4* x;
     const float4* w;
     const float4* g;
@@ -52,19 +54,21 @@ struct LaunchShape {
     size_t smem_bytes;
     dim3 grid;
 };
-LaunchShape launch_shape(int C, int L, bool o3, bool backward, int E, int N);
+LaunchShape launch_shape(int C, int L, bool o3, bool backward, bool framed, int E, int N);
 
 template <int L>
-size_t smem_bytes(bool o3, int C, int T, bool backward);
+size_t smem_bytes(bool o3, int C, int T, bool backward, bool framed);
 template <int L>
 int read_and_clear_fault();
 template <int L>
-int blocks_per_sm(bool o3, bool backward, int C, size_t smem);
+int blocks_per_sm(bool o3, bool backward, bool framed, int C, size_t smem);
 
 template <int L>
 cudaError_t launch_forward(bool o3, const FwdArgs& a, dim3 grid, size_t smem, cudaStream_t s);
 template <int L>
 cudaError_t launch_backward(bool o3, const BwdArgs& a, dim3 grid, size_t smem, cudaStream_t s);
+template <int L>
+cudaError_t launch_edge_frames(int E, const float* r, float* frames, cudaStream_t s);
 
 // Reverse CSR workspace: per-source counts, two key buffers, one value buffer,
 // and the digit-major table of per-tile histograms (tiles of kRadixTile edges).

@@ -9,7 +9,8 @@
 namespace etp {
 template cudaError_t launch_forward<ETP_L>(bool, const FwdArgs&, dim3, size_t, cudaStream_t);
 template cudaError_t launch_backward<ETP_L>(bool, const BwdArgs&, dim3, size_t, cudaStream_t);
-template size_t smem_bytes<ETP_L>(bool, int, int, bool);
+template size_t smem_bytes<ETP_L>(bool, int, int, bool, bool);
+template cudaError_t launch_edge_frames<ETP_L>(int, const float*, float*, cudaStream_t);
 
 // The fault flag of this specialisation's kernels.
 template <>
@@ -20,5 +21,5 @@ int read_and_clear_fault<ETP_L>() {
     cudaMemcpyToSymbol(frame::g_fault, &zero, sizeof(int));
     return v;
 }
-template int blocks_per_sm<ETP_L>(bool, bool, int, size_t);
+template int blocks_per_sm<ETP_L>(bool, bool, bool, int, size_t);
 }  // namespace etp

@@ -7,7 +7,7 @@ namespace etp {
 namespace {
 
 // Resident blocks per SM of each kernel specialisation, per device (computed once).
-std::atomic<int> g_occupancy[16][4][2][2][8];
+std::atomic<int> g_occupancy[16][4][2][2][2][8];
 std::atomic<int> g_sms[16];
 
 int log2i(int t) {
@@ -18,16 +18,16 @@ int log2i(int t) {
 
 }  // namespace
 
-LaunchShape launch_shape(int C, int L, bool o3, bool backward, int E, int N) {
+LaunchShape launch_shape(int C, int L, bool o3, bool backward, bool framed, int E, int N) {
     LaunchShape s;
     s.team = C / 2 < 32 ? C / 2 : 32;
     s.slices = C / (2 * s.team);
     s.tasks_per_block = (frame::kThreads / s.team) / s.slices;
     switch (L) {
-        case 0: s.smem_bytes = smem_bytes<0>(o3, C, s.team, backward); break;
-        case 1: s.smem_bytes = smem_bytes<1>(o3, C, s.team, backward); break;
-        case 2: s.smem_bytes = smem_bytes<2>(o3, C, s.team, backward); break;
-        default: s.smem_bytes = smem_bytes<3>(o3, C, s.team, backward); break;
+        case 0: s.smem_bytes = smem_bytes<0>(o3, C, s.team, backward, framed); break;
+        case 1: s.smem_bytes = smem_bytes<1>(o3, C, s.team, backward, framed); break;
+        case 2: s.smem_bytes = smem_bytes<2>(o3, C, s.team, backward, framed); break;
+        default: s.smem_bytes = smem_bytes<3>(o3, C, s.team, backward, framed); break;
     }
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 16) dev = 0;
@@ -36,14 +36,14 @@ LaunchShape launch_shape(int C, int L, bool o3, bool backward, int E, int N) {
         if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 1) sms = 1;
         g_sms[dev].store(sms);
     }
-    std::atomic<int>& occ = g_occupancy[dev][L & 3][o3 ? 1 : 0][backward ? 1 : 0][log2i(C) % 8];
+    std::atomic<int>& occ = g_occupancy[dev][L & 3][o3 ? 1 : 0][backward ? 1 : 0][framed ? 1 : 0][log2i(C) % 8];
     int bps = occ.load();
     if (bps == 0) {
         switch (L) {
-            case 0: bps = blocks_per_sm<0>(o3, backward, C, s.smem_bytes); break;
-            case 1: bps = blocks_per_sm<1>(o3, backward, C, s.smem_bytes); break;
-            case 2: bps = blocks_per_sm<2>(o3, backward, C, s.smem_bytes); break;
-            default: bps = blocks_per_sm<3>(o3, backward, C, s.smem_bytes); break;
+            case 0: bps = blocks_per_sm<0>(o3, backward, framed, C, s.smem_bytes); break;
+            case 1: bps = blocks_per_sm<1>(o3, backward, framed, C, s.smem_bytes); break;
+            case 2: bps = blocks_per_sm<2>(o3, backward, framed, C, s.smem_bytes); break;
+            default: bps = blocks_per_sm<3>(o3, backward, framed, C, s.smem_bytes); break;
         }
         occ.store(bps);
     }

@@ -43,12 +43,13 @@
  *   r, grad_r                : float32 [E][3]
  *   row_ptr int32 [N+1] (row_ptr[0] = 0, row_ptr[N] = E, nondecreasing),
  *   src int32 [E] (source node of each edge, in [0, N)).
- * Device pointers must be 16-byte aligned for x, w, out, grad_out, grad_x and
- * grad_w (they are read and written as float4).
+ * Device pointers must be 16-byte aligned for x, w, out, grad_out, grad_x,
+ * grad_w and frames (they are moved in 16-byte units).
  *
  * Ownership and execution: the caller owns every buffer. A plan owns only host
  * tables (the coupling values are compile-time constants of the kernels).
- * etp_forward / etp_backward / etp_build_reverse_csr / etp_validate_csr enqueue
+ * etp_edge_frames / etp_forward / etp_backward / etp_build_reverse_csr /
+ * etp_validate_csr enqueue
  * work on the given stream and return without synchronising; they allocate no
  * memory; they overwrite their outputs.
  *
@@ -125,11 +126,31 @@ ETP_API etp_status etp_plan_couplings(etp_plan_t plan, int* nnz, int* path_off, 
 /* Free a plan (NULL is accepted). */
 ETP_API etp_status etp_plan_destroy(etp_plan_t plan);
 
+/* Floats in the frame record of one edge (see etp_edge_frames). */
+#define ETP_FRAME_FLOATS 88
+
+/* Edge frames: for every edge, the rotation R that takes the edge direction to
+ * the z axis, 1/|r|, a zero-length flag, and the Wigner matrices D_2(R), D_3(R)
+ * of the real harmonics, written as a record of ETP_FRAME_FLOATS floats.
+ * The tensor product is evaluated in this frame: there the harmonics of the edge
+ * are those of z, nonzero for m2 = 0 only, so each path couples the rotated x
+ * through few coefficients (this library's reading of the pages' sparse
+ * Clebsch-Gordan contraction: the rotation is a change of basis, the result the
+ * same). The records depend on r only; computed once, they serve both
+ * etp_forward and etp_backward for the same r, which then skip building the
+ * frames themselves. The record layout is private to the library.
+ * frames: device float32 [E][ETP_FRAME_FLOATS], 16-byte aligned, owned by the
+ * caller; r: [E][3]. E = 0 launches nothing. */
+ETP_API etp_status etp_edge_frames(etp_plan_t plan, int E, const float* r, float* frames, etp_stream_t stream);
+
 /* Forward: out[i] = sum_{e in row i} msg_e (see above), for all N rows.
  * x: [N][D][C], w: [E][P][C], r: [E][3], out: [N][D][C] device pointers.
- * N >= 0, E >= 0; with N = 0 nothing is launched; with E = 0 out is zeroed. */
+ * frames: NULL (the kernel builds each edge's frame from r), or the records
+ * etp_edge_frames wrote for this r and plan's L (then r is not read and may be
+ * NULL). N >= 0, E >= 0; with N = 0 nothing is launched; with E = 0 out is
+ * zeroed. */
 ETP_API etp_status etp_forward(etp_plan_t plan, int N, int E, const int32_t* row_ptr, const int32_t* src,
-                       const float* r, const float* x, const float* w, float* out,
+                       const float* r, const float* frames, const float* x, const float* w, float* out,
                        etp_stream_t stream);
 
 /* Vector-Jacobian product for the cotangent grad_out = dLoss/d(out), [N][D][C]:
@@ -138,13 +159,15 @@ ETP_API etp_status etp_forward(etp_plan_t plan, int N, int E, const int32_t* row
  *   grad_r[e]           = sum_{l2 m2} dLoss/dY_{l2 m2}(e) dY_{l2 m2}/dr_e   (through Y only; r_e . grad_r[e] = 0)
  * rev_ptr [N+1] / rev_perm [E] group the edges by source, as written by
  * etp_build_reverse_csr; dst_of_edge [E] (may be NULL: then the row of each edge
- * is found by binary search in row_ptr). Each of grad_x, grad_w, grad_r may be
+ * is found by binary search in row_ptr). frames: as in etp_forward (with
+ * frames, r is not read and may be NULL). Each of grad_x, grad_w, grad_r may be
  * NULL to skip it. All outputs are overwritten (sources without edges get zero
  * grad_x). */
 ETP_API etp_status etp_backward(etp_plan_t plan, int N, int E, const int32_t* row_ptr, const int32_t* src,
                         const int32_t* rev_ptr, const int32_t* rev_perm, const int32_t* dst_of_edge,
-                        const float* r, const float* x, const float* w, const float* grad_out,
-                        float* grad_x, float* grad_w, float* grad_r, etp_stream_t stream);
+                        const float* r, const float* frames, const float* x, const float* w,
+                        const float* grad_out, float* grad_x, float* grad_w, float* grad_r,
+                        etp_stream_t stream);
 
 /* Bytes of device workspace etp_build_reverse_csr needs for (N, E). */
 ETP_API etp_status etp_reverse_csr_workspace_size(int N, int E, size_t* bytes);

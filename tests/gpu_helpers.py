@@ -27,17 +27,23 @@ def to_dev(wl, dev="cuda:0"):
             for k in ("row_ptr", "src", "r", "x", "w", "g")}
 
 
-def run_gpu(wl, irreps=None, with_dst=True, want=("x", "w", "r")):
+def run_gpu(wl, irreps=None, with_dst=True, want=("x", "w", "r"), framed=False):
+    """Forward, reverse CSR and VJP through the binding. framed: the edge frames
+    are built once by etp_edge_frames and both kernels read them (r is then not
+    passed to the kernels at all)."""
     irreps = irreps or wl.irreps
     plan = etp.Plan(irreps, wl.L, irreps, wl.C)
     t = to_dev(wl)
-    out = etp.forward(plan, t["row_ptr"], t["src"], t["r"], t["x"], t["w"])
+    frames = etp.edge_frames(plan, t["r"]) if framed else None
+    r = None if framed else t["r"]
+    out = etp.forward(plan, t["row_ptr"], t["src"], r, t["x"], t["w"], frames=frames)
     rev_ptr, rev_perm, dst = etp.build_reverse_csr(wl.N, t["row_ptr"], t["src"], with_dst=with_dst)
-    gx, gw, gr = etp.backward(plan, t["row_ptr"], t["src"], rev_ptr, rev_perm, dst, t["r"], t["x"], t["w"], t["g"],
-                              want=want)
+    gx, gw, gr = etp.backward(plan, t["row_ptr"], t["src"], rev_ptr, rev_perm, dst, r, t["x"], t["w"], t["g"],
+                              want=want, frames=frames)
     torch.cuda.synchronize()
     assert etp.device_fault() == 0, "a bounded wait inside a kernel ran out"
-    return dict(plan=plan, out=out, rev_ptr=rev_ptr, rev_perm=rev_perm, dst=dst, grad_x=gx, grad_w=gw, grad_r=gr)
+    return dict(plan=plan, out=out, rev_ptr=rev_ptr, rev_perm=rev_perm, dst=dst, grad_x=gx, grad_w=gw, grad_r=gr,
+                frames=frames)
 
 
 def compare_full(wl, res, irreps=None):

@@ -23,7 +23,7 @@ def lib():
 
 def test_exports_every_declared_symbol(lib):
     names = etp.declared_symbols()
-    assert len(names) == 12
+    assert len(names) == 13
     for n in names:
         assert hasattr(lib, n), n
 
@@ -83,23 +83,33 @@ def test_host_argument_checks(lib):
     ok = ctypes.c_void_p(0x10000)       # never dereferenced: each call fails a host check
     bad = ctypes.c_void_p(0x10004)      # not 16-byte aligned
     F = lib.etp_forward
-    assert F(None, 4, 4, ok, ok, ok, ok, ok, ok, None) == etp.ETP_ERR_INVALID_ARG       # no plan
-    assert F(h, -1, 4, ok, ok, ok, ok, ok, ok, None) == etp.ETP_ERR_INVALID_ARG         # N < 0
-    assert F(h, 4, -2, ok, ok, ok, ok, ok, ok, None) == etp.ETP_ERR_INVALID_ARG         # E < 0
-    assert F(h, 0, 3, ok, ok, ok, ok, ok, ok, None) == etp.ETP_ERR_INVALID_ARG          # edges without nodes
-    assert F(h, 0, 0, None, None, None, None, None, None, None) == etp.ETP_OK           # nothing to do
-    assert F(h, 4, 4, None, ok, ok, ok, ok, ok, None) == etp.ETP_ERR_INVALID_ARG        # row_ptr NULL
-    assert F(h, 4, 4, ok, ok, ok, bad, ok, ok, None) == etp.ETP_ERR_INVALID_ARG         # x misaligned
-    assert F(h, 4, 4, ok, ok, ok, ok, bad, ok, None) == etp.ETP_ERR_INVALID_ARG         # w misaligned
-    assert F(h, 4, 4, ok, ok, ok, ok, ok, bad, None) == etp.ETP_ERR_INVALID_ARG         # out misaligned
-    assert F(h, 4, 4, ok, None, ok, ok, ok, ok, None) == etp.ETP_ERR_INVALID_ARG        # src NULL with E > 0
+    assert F(None, 4, 4, ok, ok, ok, None, ok, ok, ok, None) == etp.ETP_ERR_INVALID_ARG       # no plan
+    assert F(h, -1, 4, ok, ok, ok, None, ok, ok, ok, None) == etp.ETP_ERR_INVALID_ARG         # N < 0
+    assert F(h, 4, -2, ok, ok, ok, None, ok, ok, ok, None) == etp.ETP_ERR_INVALID_ARG         # E < 0
+    assert F(h, 0, 3, ok, ok, ok, None, ok, ok, ok, None) == etp.ETP_ERR_INVALID_ARG          # edges without nodes
+    assert F(h, 0, 0, None, None, None, None, None, None, None, None) == etp.ETP_OK           # nothing to do
+    assert F(h, 4, 4, None, ok, ok, None, ok, ok, ok, None) == etp.ETP_ERR_INVALID_ARG        # row_ptr NULL
+    assert F(h, 4, 4, ok, ok, ok, None, bad, ok, ok, None) == etp.ETP_ERR_INVALID_ARG         # x misaligned
+    assert F(h, 4, 4, ok, ok, ok, None, ok, bad, ok, None) == etp.ETP_ERR_INVALID_ARG         # w misaligned
+    assert F(h, 4, 4, ok, ok, ok, None, ok, ok, bad, None) == etp.ETP_ERR_INVALID_ARG         # out misaligned
+    assert F(h, 4, 4, ok, None, ok, None, ok, ok, ok, None) == etp.ETP_ERR_INVALID_ARG        # src NULL with E > 0
+    assert F(h, 4, 4, ok, ok, None, None, ok, ok, ok, None) == etp.ETP_ERR_INVALID_ARG     # neither r nor frames
+    assert F(h, 4, 4, ok, ok, None, bad, ok, ok, ok, None) == etp.ETP_ERR_INVALID_ARG      # frames misaligned
     B = lib.etp_backward
-    assert B(h, 4, 4, ok, ok, None, ok, ok, ok, ok, ok, ok, ok, ok, ok, None) == etp.ETP_ERR_INVALID_ARG  # rev_ptr
-    assert B(h, 4, 4, ok, ok, ok, None, ok, ok, ok, ok, ok, ok, ok, ok, None) == etp.ETP_ERR_INVALID_ARG  # rev_perm
-    assert B(h, 4, 4, ok, ok, ok, ok, ok, ok, ok, ok, bad, ok, ok, ok, None) == etp.ETP_ERR_INVALID_ARG   # grad_out
-    assert B(h, 4, 4, ok, ok, ok, ok, ok, ok, ok, ok, ok, ok, bad, ok, None) == etp.ETP_ERR_INVALID_ARG   # grad_w
-    assert B(h, 4, 4, ok, ok, ok, ok, ok, ok, ok, ok, ok, bad, ok, ok, None) == etp.ETP_ERR_INVALID_ARG   # grad_x
-    assert B(h, 4, 4, ok, ok, ok, ok, ok, ok, ok, ok, ok, None, None, None, None) == etp.ETP_OK  # nothing wanted
+    assert B(h, 4, 4, ok, ok, None, ok, ok, ok, None, ok, ok, ok, ok, ok, ok, None) == etp.ETP_ERR_INVALID_ARG  # rev_ptr
+    assert B(h, 4, 4, ok, ok, ok, None, ok, ok, None, ok, ok, ok, ok, ok, ok, None) == etp.ETP_ERR_INVALID_ARG  # rev_perm
+    assert B(h, 4, 4, ok, ok, ok, ok, ok, ok, None, ok, ok, bad, ok, ok, ok, None) == etp.ETP_ERR_INVALID_ARG   # grad_out
+    assert B(h, 4, 4, ok, ok, ok, ok, ok, ok, None, ok, ok, ok, ok, bad, ok, None) == etp.ETP_ERR_INVALID_ARG   # grad_w
+    assert B(h, 4, 4, ok, ok, ok, ok, ok, ok, None, ok, ok, ok, bad, ok, ok, None) == etp.ETP_ERR_INVALID_ARG   # grad_x
+    assert B(h, 4, 4, ok, ok, ok, ok, ok, ok, None, ok, ok, ok, None, None, None, None) == etp.ETP_OK  # nothing wanted
+    assert B(h, 4, 4, ok, ok, ok, ok, ok, None, None, ok, ok, ok, ok, ok, ok, None) == etp.ETP_ERR_INVALID_ARG  # no r/frames
+    assert B(h, 4, 4, ok, ok, ok, ok, ok, None, bad, ok, ok, ok, ok, ok, ok, None) == etp.ETP_ERR_INVALID_ARG   # frames
+    G = lib.etp_edge_frames
+    assert G(None, 4, ok, ok, None) == etp.ETP_ERR_INVALID_ARG      # no plan
+    assert G(h, -1, ok, ok, None) == etp.ETP_ERR_INVALID_ARG        # E < 0
+    assert G(h, 4, None, ok, None) == etp.ETP_ERR_INVALID_ARG       # r NULL
+    assert G(h, 4, ok, bad, None) == etp.ETP_ERR_INVALID_ARG        # frames misaligned
+    assert G(h, 0, None, None, None) == etp.ETP_OK                  # nothing to do
     sz = ctypes.c_size_t()
     assert lib.etp_reverse_csr_workspace_size(10, 100, ctypes.byref(sz)) == 0 and sz.value > 0
     assert lib.etp_reverse_csr_workspace_size(-1, 100, ctypes.byref(sz)) == etp.ETP_ERR_INVALID_ARG

@@ -11,6 +11,7 @@ import torch
 
 import cg_tensor_products_b200 as etp
 import oracle
+import oracle.cg
 import workloads
 from cg_tensor_products_b200 import build as etp_build
 from gpu_helpers import (check_errs, check_reverse_csr, compare_full, compare_sampled, rel_err, run_gpu, to_dev)
@@ -26,20 +27,22 @@ def _built():
     oracle.build()
 
 
+@pytest.mark.parametrize("framed", [False, True])
 @pytest.mark.parametrize("name", ["tiny", "micro_l2", "water"])
-def test_workload_full(name):
+def test_workload_full(name, framed):
     wl = workloads.make(name)
-    res = run_gpu(wl)
+    res = run_gpu(wl, framed=framed)
     check_reverse_csr(wl, res)
     errs = compare_full(wl, res)
     print(name, errs)
     check_errs(errs)
 
 
+@pytest.mark.parametrize("framed", [False, True])
 @pytest.mark.parametrize("name", ["micro_l3", "large"])
-def test_workload_full_size_sampled(name):
+def test_workload_full_size_sampled(name, framed):
     wl = workloads.make(name)
-    res = run_gpu(wl)
+    res = run_gpu(wl, framed=framed)
     check_reverse_csr(wl, res)
     errs = compare_sampled(wl, res)
     print(name, errs)
@@ -51,7 +54,8 @@ def test_workload_full_size_sampled(name):
     assert radial <= 1e-5 * scale
 
 
-def test_l3_c128_reduced_full():
+@pytest.mark.parametrize("framed", [False, True])
+def test_l3_c128_reduced_full(framed):
     """The benchmark's shape (L = 3, C = 128, 128 neighbours) on 200 nodes: full comparison."""
     rng = np.random.default_rng(7)
     n, k = 200, 128
@@ -63,7 +67,7 @@ def test_l3_c128_reduced_full():
                             rng.standard_normal((n, 16, 128), dtype=np.float32),
                             (rng.standard_normal((E, 34, 128), dtype=np.float32) / np.float32(np.sqrt(34))),
                             rng.standard_normal((n, 16, 128), dtype=np.float32))
-    res = run_gpu(wl)
+    res = run_gpu(wl, framed=framed)
     check_reverse_csr(wl, res)
     errs = compare_full(wl, res)
     print(errs)
@@ -73,13 +77,14 @@ def test_l3_c128_reduced_full():
 SPECS = [(L, o3, C) for L in range(4) for o3 in (False, True) for C in (4, 8, 16, 32, 64, 128)]
 
 
+@pytest.mark.parametrize("framed", [False, True])
 @pytest.mark.parametrize("L,o3,C", SPECS)
-def test_every_compiled_spec_ragged_multigraph(L, o3, C):
+def test_every_compiled_spec_ragged_multigraph(L, o3, C, framed):
     irreps = "+".join(f"{l}{'eo'[l % 2]}" for l in range(L + 1)) if o3 else f"0..{L}"
     P = len(oracle.paths.enumerate_paths(irreps, L, irreps))
     rng = np.random.default_rng(100 * L + C + (7 if o3 else 0))
     wl = workloads.random_graph(rng, 37, 300, L, C, P)
-    res = run_gpu(wl, irreps=irreps, with_dst=(C % 8 == 0))   # half the cases find rows by binary search
+    res = run_gpu(wl, irreps=irreps, with_dst=(C % 8 == 0), framed=framed)  # half: rows by binary search
     check_reverse_csr(wl, res)
     errs = compare_full(wl, res, irreps=irreps)
     check_errs(errs)
@@ -115,11 +120,13 @@ def test_no_edges():
     assert torch.all(res["rev_ptr"] == 0)
 
 
-def test_zero_length_edge_vectors():
+@pytest.mark.parametrize("C", [8, 128])
+@pytest.mark.parametrize("framed", [False, True])
+def test_zero_length_edge_vectors(framed, C):
     rng = np.random.default_rng(4)
-    wl = workloads.random_graph(rng, 20, 120, 3, 8, 34)
+    wl = workloads.random_graph(rng, 20, 120, 3, C, 34)
     wl.r[::7] = 0.0
-    res = run_gpu(wl)
+    res = run_gpu(wl, framed=framed)
     check_errs(compare_full(wl, res))
     assert torch.all(res["grad_r"][::7] == 0)
 
@@ -204,3 +211,45 @@ def test_out_of_range_sources_are_skipped_not_faulted():
     w0[~keep] = 0
     ref = oracle.OracleTP("0..1", 1, "0..1", 8).forward(wl.row_ptr, wl.src, wl.r, wl.x, w0)
     assert rel_err(out, ref) <= 1e-5
+
+
+@pytest.mark.parametrize("L", [0, 1, 2, 3])
+def test_edge_frame_records(L):
+    """The frame record of each edge: R a proper rotation taking r/|r| to z,
+    1/|r|, the zero-length flag, and D_2, D_3 equal to the oracle's Wigner
+    matrices of that R (Y_l(R u) = D_l(R) Y_l(u))."""
+    rng = np.random.default_rng(11 + L)
+    E = 300
+    r = rng.standard_normal((E, 3)).astype(np.float32) * rng.uniform(0.1, 5.0, (E, 1)).astype(np.float32)
+    r[5] = 0.0
+    r[17] = (1e-14, 0.0, 0.0)
+    r[30] = (0.0, 0.0, -2.5)   # on the axis opposite z
+    r[31] = (0.0, 0.0, 3.0)
+    plan = etp.Plan(f"0..{L}", L, f"0..{L}", 8)
+    fr = etp.edge_frames(plan, torch.from_numpy(r).cuda())
+    torch.cuda.synchronize()
+    fr = fr.cpu().numpy().astype(np.float64)
+    assert fr.shape == (E, etp.FRAME_FLOATS)
+    n = np.linalg.norm(r.astype(np.float64), axis=1)
+    for e in range(E):
+        R = fr[e, 76:85].reshape(3, 3)
+        if n[e] < 1e-12:
+            assert fr[e, 86] == 1.0 and fr[e, 85] == 0.0
+            assert np.allclose(R, np.eye(3))
+            continue
+        assert fr[e, 86] == 0.0
+        assert abs(fr[e, 85] * n[e] - 1) < 1e-6
+        assert np.abs(R @ R.T - np.eye(3)).max() < 1e-6 and abs(np.linalg.det(R) - 1) < 1e-6
+        assert np.abs(R @ (r[e] / n[e]) - np.array([0.0, 0.0, 1.0])).max() < 1e-6
+        if L >= 2:
+            assert np.abs(fr[e, 0:25].reshape(5, 5) - oracle.cg.wigner_d(2, R)).max() < 2e-5, e
+        if L >= 3:
+            assert np.abs(fr[e, 25:74].reshape(7, 7) - oracle.cg.wigner_d(3, R)).max() < 2e-5, e
+
+
+def test_framed_and_unframed_agree():
+    """Both kernel variants evaluate the same frames: results agree to rounding."""
+    wl = workloads.random_graph(np.random.default_rng(12), 80, 3000, 3, 128, 34)
+    a, b = run_gpu(wl), run_gpu(wl, framed=True)
+    for k in ("out", "grad_x", "grad_w", "grad_r"):
+        assert rel_err(a[k], b[k].double().cpu().numpy()) <= 1e-6, k
