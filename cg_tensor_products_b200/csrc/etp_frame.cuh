@@ -308,6 +308,16 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, unsigned by
                  "l"(src), "r"(bytes), "r"(smem_u32(bar))
                  : "memory");
 }
+// The same with an L2 evict-first hint: for the edge weights, read once per pass,
+// so that they do not push the node rows (read by many edges) out of L2.
+__device__ __forceinline__ void bulk_g2s_stream(void* dst, const void* src, unsigned bytes, uint64_t* bar,
+                                                uint64_t pol) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;" ::"r"(
+            smem_u32(dst)),
+        "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(pol)
+        : "memory");
+}
 // Per-lane 8-byte asynchronous copies (the backward's node rows: each lane copies
 // and later reads only its own channels, so no cross-lane synchronisation).
 __device__ __forceinline__ void cp_async8(void* smem, const void* gmem) {
@@ -657,11 +667,13 @@ __global__ void __launch_bounds__(frame::kThreads, 4) etp_fwd_frame_kernel(FwdAr
             __syncwarp(G.tmask);
     };
     const unsigned wbytes = 4u * P * C, xbytes = 4u * D * C, fbytes = FR ? 4u * kFrameFloats : 0u;
+    const uint64_t pol_w = l2_evict_first_policy();
     auto issue = [&](int e, int j, int slot) {
         j = (unsigned)j < (unsigned)a.N ? j : 0;
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         mbar_expect_tx(&bar[slot], wbytes + xbytes + fbytes);
-        bulk_g2s(wbuf + slot * P * C, reinterpret_cast<const float*>(a.w) + (size_t)e * P * C, wbytes, &bar[slot]);
+        bulk_g2s_stream(wbuf + slot * P * C, reinterpret_cast<const float*>(a.w) + (size_t)e * P * C, wbytes, &bar[slot],
+                        pol_w);
         bulk_g2s(xbuf + slot * D * C, reinterpret_cast<const float*>(a.x) + (size_t)j * D * C, xbytes, &bar[slot]);
         if constexpr (FR)
             bulk_g2s(fbuf + slot * kFrameFloats, a.frames + (size_t)e * kFrameFloats, fbytes, &bar[slot]);
@@ -813,7 +825,8 @@ __global__ void __launch_bounds__(frame::kThreads, 4) etp_bwd_frame_kernel(BwdAr
         e = valid_edge(e) ? e : 0;
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         mbar_expect_tx(&bar[slot], wbytes + fbytes);
-        bulk_g2s(wbuf + slot * P * C, reinterpret_cast<const float*>(a.w) + (size_t)e * P * C, wbytes, &bar[slot]);
+        bulk_g2s_stream(wbuf + slot * P * C, reinterpret_cast<const float*>(a.w) + (size_t)e * P * C, wbytes, &bar[slot],
+                        pol_w);
         if constexpr (FR)
             bulk_g2s(fbuf + slot * kFrameFloats, a.frames + (size_t)e * kFrameFloats, fbytes, &bar[slot]);
     };
