@@ -247,19 +247,30 @@ def reference_arm(args):
     oracle.build()
     tp = oracle.OracleTP(wl.irreps, wl.L, wl.irreps, wl.C)
     rng = np.random.default_rng(2)
-    rows_per_step = 4
 
-    def step():
-        rows = np.sort(rng.choice(wl.N, size=rows_per_step, replace=False))
+    def step(n_rows):
+        rows = np.sort(rng.choice(wl.N, size=n_rows, replace=False))
         edges = np.concatenate([np.arange(wl.row_ptr[i], wl.row_ptr[i + 1]) for i in rows])
         tp.forward(wl.row_ptr, wl.src, wl.r, wl.x, wl.w, rows=rows)
-        tp.backward(wl.row_ptr, wl.src, wl.r, wl.x, wl.w, wl.g, nodes=wl.src[edges[:rows_per_step]], edges=edges)
+        tp.backward(wl.row_ptr, wl.src, wl.r, wl.x, wl.w, wl.g, nodes=wl.src[edges[:n_rows]], edges=edges)
         return len(edges)
 
+    # a step's time ~ a + b rows (a: the oracle's harmonics of every edge); size each step so that the whole
+    # run (warm-up + timed steps) takes about two minutes, and at most 2.5 s a step
+    t_a = time.perf_counter()
+    step(2)
+    t_b = time.perf_counter()
+    step(10)
+    t_c = time.perf_counter()
+    b = max(((t_c - t_b) - (t_b - t_a)) / 8, 1e-4)
+    a = max((t_b - t_a) - 2 * b, 0.0)
+    budget = min(2.5, 120.0 / max(args.steps + args.warmup, 1))
+    rows_per_step = int(max(1, min(wl.N, (budget - a) / b)))
+
     for _ in range(args.warmup):
-        step()
+        step(rows_per_step)
     t0 = time.perf_counter()
-    ne = sum(step() for _ in range(args.steps))
+    ne = sum(step(rows_per_step) for _ in range(args.steps))
     dt = time.perf_counter() - t0
     value = ne / dt
     cores = oracle.num_threads()

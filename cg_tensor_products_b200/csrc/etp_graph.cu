@@ -1,7 +1,13 @@
 // Graph preprocessing on the device: the reverse CSR (edges grouped by source,
 // stable in edge id), the destination of every edge, and a CSR validator.
 //
-// The reverse grouping is a least-significant-digit radix sort of the source ids
+// Up to kOnePassMaxNodes sources the grouping is one stable counting pass: the
+// count of every (source, tile of kTile edges) pair in a source-major table, one
+// exclusive scan of that table (which also yields rev_ptr: the entry of tile 0 of
+// each source), and a stable scatter of each tile. An out-of-range source counts
+// as source N, so every position is written.
+//
+// Otherwise the reverse grouping is a least-significant-digit radix sort of the source ids
 // with the edge ids as values, 8 bits per pass. Each pass is a stable counting
 // sort over tiles of kTile edges: (1) a per-tile digit histogram, (2) an
 // exclusive scan of the histogram table in (digit, tile) order, (3) a stable
@@ -181,6 +187,144 @@ __global__ void __launch_bounds__(128) tile_scatter(const int32_t* __restrict__ 
     }
 }
 
+// ---------------------------------------------------------------------------
+// One-pass grouping. Bucket of an edge: its source, or N when out of range.
+__device__ __forceinline__ int bucket_of(int j, int N) { return (unsigned)j < (unsigned)N ? j : N; }
+
+// table[b * n_tiles + t] = edges of tile t in bucket b, for b = 0..N.
+__global__ void __launch_bounds__(256) tile_counts(const int32_t* __restrict__ src, int E, int N, int n_tiles,
+                                                   int32_t* __restrict__ table) {
+    __shared__ int32_t h[kOnePassMaxNodes + 1];
+    for (int b = threadIdx.x; b <= N; b += 256) h[b] = 0;
+    __syncthreads();
+    const int t = blockIdx.x;
+    const int lo = t * kTile, hi = min(E, lo + kTile);
+    for (int e = lo + threadIdx.x; e < hi; e += 256) atomicAdd(h + bucket_of(src[e], N), 1);
+    __syncthreads();
+    for (int b = threadIdx.x; b <= N; b += 256) table[(size_t)b * n_tiles + t] = h[b];
+}
+
+// Block-wide exclusive scan of one value per thread (1024 threads); returns the
+// thread's exclusive prefix and writes the block total to *total.
+__device__ __forceinline__ int block_exclusive_1024(int v, int32_t* warp_tot, int* total) {
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    int incl = v;
+#pragma unroll
+    for (int s = 1; s < 32; s <<= 1) {
+        const int u = __shfl_up_sync(0xffffffffu, incl, s);
+        if (lane >= s) incl += u;
+    }
+    if (lane == 31) warp_tot[wid] = incl;
+    __syncthreads();
+    if (wid == 0) {
+        int w = warp_tot[lane];
+#pragma unroll
+        for (int s = 1; s < 32; s <<= 1) {
+            const int u = __shfl_up_sync(0xffffffffu, w, s);
+            if (lane >= s) w += u;
+        }
+        warp_tot[lane] = w;  // inclusive over warps
+    }
+    __syncthreads();
+    const int excl = (wid ? warp_tot[wid - 1] : 0) + incl - v;
+    *total = warp_tot[31];
+    return excl;
+}
+
+// In-place exclusive scan of each chunk of kScanChunk entries (8 per thread);
+// part[chunk] = the chunk's total.
+__global__ void __launch_bounds__(1024) scan_chunks(int32_t* __restrict__ a, long long n,
+                                                    int32_t* __restrict__ part) {
+    __shared__ int32_t warp_tot[32];
+    const long long base = (long long)blockIdx.x * kScanChunk + 8ll * threadIdx.x;
+    int v[8];
+    int sum = 0;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+        v[k] = base + k < n ? a[base + k] : 0;
+        sum += v[k];
+    }
+    int total;
+    int run = block_exclusive_1024(sum, warp_tot, &total);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+        if (base + k < n) a[base + k] = run;
+        run += v[k];
+    }
+    if (threadIdx.x == 0) part[blockIdx.x] = total;
+}
+
+// Exclusive scan of the chunk totals (one block, in place; part[nb] = total), then
+// rev_ptr[b] = scanned table entry of (b, tile 0) for b = 0..N.
+__global__ void __launch_bounds__(1024) scan_parts_rev_ptr(int32_t* __restrict__ part, int nb,
+                                                           const int32_t* __restrict__ table, int n_tiles, int N,
+                                                           int32_t* __restrict__ rev_ptr) {
+    __shared__ int32_t warp_tot[32];
+    __shared__ int32_t carry;
+    if (threadIdx.x == 0) carry = 0;
+    __syncthreads();
+    for (int b0 = 0; b0 < nb; b0 += 1024) {
+        const int i = b0 + threadIdx.x;
+        const int v = i < nb ? part[i] : 0;
+        int total;
+        const int ex = block_exclusive_1024(v, warp_tot, &total);
+        const int c = carry;
+        if (i < nb) part[i] = c + ex;
+        __syncthreads();
+        if (threadIdx.x == 0) carry = c + total;
+        __syncthreads();
+    }
+    if (threadIdx.x == 0) part[nb] = carry;
+    __syncthreads();
+    for (int b = threadIdx.x; b <= N; b += 1024) {
+        const long long idx = (long long)b * n_tiles;
+        rev_ptr[b] = table[idx] + part[idx / kScanChunk];
+    }
+}
+
+// Stable scatter of one tile per block of 4 warps (as tile_scatter, with the
+// bucket of the full source id): rev_perm[pos] = edge id.
+__global__ void __launch_bounds__(128) tile_scatter_one_pass(const int32_t* __restrict__ src, int E, int N,
+                                                             int n_tiles, const int32_t* __restrict__ table,
+                                                             const int32_t* __restrict__ part,
+                                                             int32_t* __restrict__ rev_perm) {
+    __shared__ int32_t cnt[4][kOnePassMaxNodes + 1];
+    const int wid = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int t = blockIdx.x;
+    constexpr int kQuarter = kTile / 4;
+    const int lo = t * kTile + wid * kQuarter, hi = min(E, lo + kQuarter);
+    for (int b = lane; b <= N; b += 32) cnt[wid][b] = 0;
+    __syncwarp();
+    for (int c = lo; c < hi; c += 32) {
+        const int e = c + lane;
+        if (e < hi) atomicAdd(&cnt[wid][bucket_of(src[e], N)], 1);
+    }
+    __syncthreads();
+    for (int b = threadIdx.x; b <= N; b += 128) {  // warp-exclusive prefix per bucket
+        const long long idx = (long long)b * n_tiles + t;
+        int run = table[idx] + part[idx / kScanChunk];
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+            const int v = cnt[w][b];
+            cnt[w][b] = run;
+            run += v;
+        }
+    }
+    __syncthreads();
+    int32_t* base = cnt[wid];
+    const unsigned lt = (1u << lane) - 1u;
+    for (int c = lo; c < hi; c += 32) {
+        const int e = c + lane;
+        const bool act = e < hi;
+        const int b = act ? bucket_of(src[e], N) : kOnePassMaxNodes + 1 + lane;  // inactive lanes match nobody
+        const unsigned peers = __match_any_sync(0xffffffffu, b);
+        if (act) rev_perm[base[b] + __popc(peers & lt)] = e;
+        __syncwarp();
+        if (act && lane == __ffs(peers) - 1) base[b] += __popc(peers);
+        __syncwarp();
+    }
+}
+
 __global__ void iota(int32_t* __restrict__ out, int n) {
     for (int k = blockIdx.x * blockDim.x + threadIdx.x; k < n; k += gridDim.x * blockDim.x) out[k] = k;
 }
@@ -231,7 +375,20 @@ inline int radix_passes(int N) {
 size_t reverse_csr_workspace_bytes(int N, int E) { return reverse_csr_workspace_bytes_for(N, E); }
 
 cudaError_t build_reverse_csr(int N, int E, const int32_t* row_ptr, const int32_t* src, int32_t* rev_ptr,
-                              int32_t* rev_perm, int32_t* dst, void* ws, cudaStream_t s) {
+                              int32_t* rev_perm, int32_t* dst, void* ws, cudaStream_t s, bool one_pass) {
+    if (one_pass && reverse_csr_one_pass(N, E)) {
+        const int n_tiles = (int)radix_tiles(E);
+        const long long n = (long long)(N + 1) * n_tiles;
+        const int nb = (int)((n + kScanChunk - 1) / kScanChunk);
+        int32_t* table = static_cast<int32_t*>(ws);
+        int32_t* part = reinterpret_cast<int32_t*>(static_cast<char*>(ws) + align16(sizeof(int32_t) * (size_t)n));
+        tile_counts<<<n_tiles, 256, 0, s>>>(src, E, N, n_tiles, table);
+        scan_chunks<<<nb, 1024, 0, s>>>(table, n, part);
+        scan_parts_rev_ptr<<<1, 1024, 0, s>>>(part, nb, table, n_tiles, N, rev_ptr);
+        tile_scatter_one_pass<<<n_tiles, 128, 0, s>>>(src, E, N, n_tiles, table, part, rev_perm);
+        if (dst) edge_rows<<<grid_for(E, 256), 256, 0, s>>>(row_ptr, N, E, dst);
+        return cudaGetLastError();
+    }
     char* p = static_cast<char*>(ws);
     int32_t* cnt = reinterpret_cast<int32_t*>(p);
     p += align16(sizeof(int32_t) * ((size_t)N + 1));

@@ -70,18 +70,37 @@ cudaError_t launch_backward(bool o3, const BwdArgs& a, dim3 grid, size_t smem, c
 template <int L>
 cudaError_t launch_edge_frames(int E, const float* r, float* frames, cudaStream_t s);
 
-// Reverse CSR workspace: per-source counts, two key buffers, one value buffer,
-// and the digit-major table of per-tile histograms (tiles of kRadixTile edges).
+// Reverse CSR workspace. Up to kOnePassMaxNodes sources (and a bounded table)
+// the grouping is one stable counting pass over a (source, tile) count table;
+// otherwise a radix sort of the source ids, 8 bits per pass, whose workspace is
+// per-source counts, two key buffers, one value buffer and the digit-major table
+// of per-tile histograms (tiles of kRadixTile edges).
 constexpr int kRadixTile = 1024;
+constexpr int kOnePassMaxNodes = 2048;
+constexpr long long kOnePassMaxEntries = 1ll << 22;
+constexpr int kScanChunk = 8192;  // table entries scanned per block
 constexpr size_t align16_bytes(size_t b) { return (b + 15) & ~size_t(15); }
-constexpr size_t reverse_csr_workspace_bytes_for(long long N, long long E) {
-    return align16_bytes(4 * (size_t)(N + 1)) + 3 * align16_bytes(4 * (size_t)E) +
-           align16_bytes(4 * (256 * (size_t)((E + kRadixTile - 1) / kRadixTile) + 1));
+constexpr long long radix_tiles(long long E) { return (E + kRadixTile - 1) / kRadixTile; }
+constexpr bool reverse_csr_one_pass(long long N, long long E) {
+    return N >= 1 && N <= kOnePassMaxNodes && E > 0 && (N + 1) * radix_tiles(E) <= kOnePassMaxEntries;
 }
-
+constexpr size_t radix_workspace_bytes_for(long long N, long long E) {
+    return align16_bytes(4 * (size_t)(N + 1)) + 3 * align16_bytes(4 * (size_t)E) +
+           align16_bytes(4 * (256 * (size_t)radix_tiles(E) + 1));
+}
+constexpr size_t one_pass_workspace_bytes_for(long long N, long long E) {
+    return align16_bytes(4 * (size_t)((N + 1) * radix_tiles(E))) +
+           align16_bytes(4 * (size_t)((N + 1) * radix_tiles(E) / kScanChunk + 2));
+}
+constexpr size_t reverse_csr_workspace_bytes_for(long long N, long long E) {
+    return reverse_csr_one_pass(N, E) ? one_pass_workspace_bytes_for(N, E) : radix_workspace_bytes_for(N, E);
+}
 size_t reverse_csr_workspace_bytes(int N, int E);
+// one_pass: allow the one-pass grouping when it applies (the workspace must then
+// hold reverse_csr_workspace_bytes_for); false: always the radix sort (workspace
+// radix_workspace_bytes_for).
 cudaError_t build_reverse_csr(int N, int E, const int32_t* row_ptr, const int32_t* src, int32_t* rev_ptr,
-                              int32_t* rev_perm, int32_t* dst, void* ws, cudaStream_t s);
+                              int32_t* rev_perm, int32_t* dst, void* ws, cudaStream_t s, bool one_pass = true);
 cudaError_t validate_csr(int N, int E, const int32_t* row_ptr, const int32_t* src, int32_t* flag, cudaStream_t s);
 
 }  // namespace etp

@@ -35,7 +35,7 @@
 namespace {
 
 constexpr size_t kStaticScratchBytes =
-    etp::reverse_csr_workspace_bytes_for(ETP_STATIC_MAX_NODES, ETP_STATIC_MAX_EDGES);
+    etp::radix_workspace_bytes_for(ETP_STATIC_MAX_NODES, ETP_STATIC_MAX_EDGES);
 static_assert(kStaticScratchBytes == ETP_STATIC_SCRATCH_BYTES, "etp.h states the scratch size");
 
 static __device__ __align__(256) unsigned char g_reverse_csr_scratch[kStaticScratchBytes];
@@ -77,7 +77,9 @@ extern "C" ETP_API etp_status etp_build_reverse_csr_static(int N, int E, const i
     if (dst_of_edge && (reinterpret_cast<uintptr_t>(dst_of_edge) & mis4)) return ETP_ERR_INVALID_ARG;
     void* ws = nullptr;
     if (scratch_address(&ws) != cudaSuccess) return ETP_ERR_CUDA;
+    // always the radix path: its scratch need grows with N and E, so the array sized
+    // for the limits covers every admitted call
     cudaError_t err = etp::build_reverse_csr(N, E, row_ptr, src, rev_ptr, rev_perm, dst_of_edge, ws,
-                                             reinterpret_cast<cudaStream_t>(stream));
+                                             reinterpret_cast<cudaStream_t>(stream), false);
     return err == cudaSuccess ? ETP_OK : ETP_ERR_CUDA;
 }

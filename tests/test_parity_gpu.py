@@ -168,7 +168,8 @@ def test_bitwise_repeatable_when_rows_fit_a_task():
 
 
 @pytest.mark.parametrize("n,e", [(1, 0), (1, 50), (2, 7), (256, 5000), (257, 5000), (70000, 300000),
-                                 (3, 10000)])
+                                 (3, 10000), (2048, 200000), (2049, 200000), (1024, 131072),
+                                 (1500, 2_200_000)])
 def test_reverse_csr_bit_exact(n, e):
     rng = np.random.default_rng(n + e)
     dst = rng.integers(0, n, e)
@@ -253,3 +254,26 @@ def test_framed_and_unframed_agree():
     a, b = run_gpu(wl), run_gpu(wl, framed=True)
     for k in ("out", "grad_x", "grad_w", "grad_r"):
         assert rel_err(a[k], b[k].double().cpu().numpy()) <= 1e-6, k
+
+
+@pytest.mark.parametrize("n", [100, 5000])
+def test_reverse_csr_with_out_of_range_sources(n):
+    """Sources outside [0, N) (an invalid CSR) are grouped after all valid ones:
+    rev_ptr[N] counts the valid edges, the valid part matches the stable grouping
+    of the valid edges, and rev_perm stays a permutation (nothing out of bounds)."""
+    rng = np.random.default_rng(n)
+    e = 20000
+    dst = rng.integers(0, n, e)
+    src = rng.integers(0, n, e)
+    row_ptr, s, _ = workloads.csr_from_pairs(n, dst, src)
+    s = s.copy()
+    bad = rng.random(e) < 0.05
+    s[bad] = np.where(rng.random(bad.sum()) < 0.5, -3, n + 7)
+    rp, perm, d = etp.build_reverse_csr(n, torch.from_numpy(row_ptr).cuda(), torch.from_numpy(s).cuda())
+    rp, perm = rp.cpu().numpy(), perm.cpu().numpy()
+    valid = np.flatnonzero(~bad)
+    order = valid[np.argsort(s[valid], kind="stable")]
+    assert rp[n] == len(valid)
+    assert np.array_equal(perm[:len(valid)], order)
+    assert np.array_equal(np.sort(perm), np.arange(e))
+    assert np.array_equal(rp, np.concatenate([[0], np.cumsum(np.bincount(s[valid], minlength=n))]))
