@@ -272,6 +272,50 @@ __device__ __forceinline__ void rotate(const Frame& f, const float* __restrict__
     }
 }
 
+// Two vectors rotated by the same D_l (each row loaded once, two FMA streams).
+template <int l>
+__device__ __forceinline__ void rotate2(const Frame& f, const float* __restrict__ dbuf, const float2* in1,
+                                        const float2* in2, float2* out1, float2* out2) {
+    constexpr int d = 2 * l + 1;
+    if constexpr (l == 0) {
+        out1[0] = in1[0];
+        out2[0] = in2[0];
+    } else {
+#pragma unroll
+        for (int a = 0; a < d; ++a) {
+            float2 row[8];
+            if constexpr (l == 1) {
+#pragma unroll
+                for (int b = 0; b < d; ++b) row[b] = f2_dup(d1(f, a, b));
+            } else {
+                const float* base = dbuf + (l == 2 ? 0 : 80) + a * 16;
+#pragma unroll
+                for (int h = 0; h < (d + 1) / 2; ++h) {
+                    const float4 q = lds4(base + 4 * h);
+                    row[2 * h] = make_float2(q.x, q.y);
+                    row[2 * h + 1] = make_float2(q.z, q.w);
+                }
+            }
+            float2 t1 = f2_zero(), t2 = f2_zero();
+#pragma unroll
+            for (int b = 0; b < d; ++b) {
+                t1 = __ffma2_rn(row[b], in1[b], t1);
+                t2 = __ffma2_rn(row[b], in2[b], t2);
+            }
+            out1[a] = t1;
+            out2[a] = t2;
+        }
+    }
+}
+template <int L>
+__device__ __forceinline__ void rotate_all2(const Frame& f, const float* dbuf, const float2* in1, const float2* in2,
+                                            float2* out1, float2* out2) {
+    static_for<0, L + 1>([&](auto lc) {
+        constexpr int l = decltype(lc)::value;
+        rotate2<l>(f, dbuf, in1 + l * l, in2 + l * l, out1 + l * l, out2 + l * l);
+    });
+}
+
 // Rotate every l block of a [D] float2 vector into the frame.
 template <int L>
 __device__ __forceinline__ void rotate_all(const Frame& f, const float* dbuf, const float2* in, float2* out) {
@@ -909,26 +953,24 @@ __global__ void __launch_bounds__(frame::kThreads, 4) etp_bwd_frame_kernel(BwdAr
         float2* gwe = (want_w && ok) ? gw2 + (size_t)e_cur * P * C2 + cp : nullptr;
         float2 sx2 = f2_zero(), sy2 = f2_zero();  // dL/de_x, dL/de_y per channel of this lane
         if (ok && !f.degenerate) {
-            float2 xp[D], z[D];
+            float2 xp[D], gpa[D], z[D];
             {
-                float2 v[D];
+                float2 v[D], u[D];
 #pragma unroll
                 for (int k = 0; k < D; ++k) v[k] = lds2(xrow + k * G.T + G.tl);
-                rotate_all<L>(f, dbuf, v, xp);
+#pragma unroll
+                for (int k = 0; k < D; ++k) u[k] = lds2(grow + k * G.T + G.tl);
+                rotate_all2<L>(f, dbuf, v, u, xp, gpa);
             }
             if (has_next && row_next != row) copy_x(row_next);  // next source's x row, behind this edge's reads
+            if (has_next) copy_g(i_next);
 #pragma unroll
             for (int k = 0; k < D; ++k) z[k] = f2_zero();
             static_for<0, L + 1>([&](auto l3c) {
                 constexpr int l3 = decltype(l3c)::value;
                 constexpr int d3 = 2 * l3 + 1;
-                float2 y[d3], gp[d3];  // gp: this block of grad_out rotated into the frame
-                {
-                    float2 v[d3];
-#pragma unroll
-                    for (int m = 0; m < d3; ++m) v[m] = lds2(grow + (l3 * l3 + m) * G.T + G.tl);
-                    rotate<l3, false, false>(f, dbuf, v, gp);
-                }
+                float2 y[d3];
+                const float2* gp = gpa + l3 * l3;
 #pragma unroll
                 for (int m = 0; m < d3; ++m) y[m] = f2_zero();
                 static_for<0, L + 1>([&](auto l1c) {
@@ -977,7 +1019,6 @@ __global__ void __launch_bounds__(frame::kThreads, 4) etp_bwd_frame_kernel(BwdAr
                     sy2 = f2_add(sy2, gen_form<l3, 1>(gp, y));
                 }
             });
-            if (has_next) copy_g(i_next);  // next destination's grad_out row, behind this edge's reads
             static_for<0, L + 1>([&](auto l1c) {
                 constexpr int l1 = decltype(l1c)::value;
                 if (want_r) {
