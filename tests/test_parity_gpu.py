@@ -277,3 +277,25 @@ def test_reverse_csr_with_out_of_range_sources(n):
     assert np.array_equal(perm[:len(valid)], order)
     assert np.array_equal(np.sort(perm), np.arange(e))
     assert np.array_equal(rp, np.concatenate([[0], np.cumsum(np.bincount(s[valid], minlength=n))]))
+
+
+@pytest.mark.parametrize("framed", [False, True])
+def test_hub_rows_cut_across_many_tasks(framed):
+    """A destination with 20,000 edges and a source with 20,000 edges among 64 nodes:
+    the tasks are equal edge ranges, so both hub rows are cut across ~30 tasks and
+    their pieces are combined on the zeroed outputs."""
+    rng = np.random.default_rng(21)
+    n, hub = 64, 20000
+    dst = np.concatenate([np.zeros(hub, np.int64), rng.integers(0, n, hub), rng.integers(0, n, 3000)])
+    src = np.concatenate([rng.integers(0, n, hub), np.ones(hub, np.int64), rng.integers(0, n, 3000)])
+    row_ptr, s, _ = workloads.csr_from_pairs(n, dst, src)
+    E = len(s)
+    wl = workloads.Workload("hubs", 3, 32, 34, row_ptr, s, rng.standard_normal((E, 3), dtype=np.float32),
+                            rng.standard_normal((n, 16, 32), dtype=np.float32),
+                            rng.standard_normal((E, 34, 32), dtype=np.float32) / np.float32(np.sqrt(34)),
+                            rng.standard_normal((n, 16, 32), dtype=np.float32))
+    res = run_gpu(wl, framed=framed)
+    check_reverse_csr(wl, res)
+    errs = compare_full(wl, res)
+    print(errs)
+    check_errs(errs)
