@@ -396,6 +396,26 @@ def main():
                 "peak_source": f"{peak_kind} (hbm_gbs, burst copy)",
                 "traffic": recorded_traffic(kname, framed, args.workload, N)}
 
+    # force assembly from grad_r (a separate call, not part of the step): forces and per-atom virials
+    forces_t = torch.empty((N, 3), device=dev)
+    virial_t = torch.empty((N, 9), device=dev)
+
+    def forces_call():
+        etp._check(lib.etp_assemble_forces(N, E, P(d["row_ptr"]), P(rev_ptr), P(rev_perm), P(d["r"]), P(gr),
+                                           P(forces_t), P(virial_t), sp), "assemble forces")
+
+    for _ in range(3):
+        forces_call()
+    fa, fb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    fa.record(stream)
+    for _ in range(20):
+        forces_call()
+    fb.record(stream)
+    torch.cuda.synchronize()
+    f_ms = fa.elapsed_time(fb) / 20
+    kern["assemble_forces_ms"] = f_ms
+    kern["assemble_forces_GBps"] = (40 * E + 48 * N + 8) / (f_ms * 1e6)
+
     # the same kernel against the nominal FP32 rate at the clock seen under load (148 SMs x 128 FMA lanes x 2):
     # the method's sparse-CG FLOP count, which the edge-frame schedule undercuts (it executes fewer)
     sms = torch.cuda.get_device_properties(dev).multi_processor_count
@@ -447,7 +467,7 @@ def main():
         while (1 << (8 * passes)) < N and passes < 4:
             passes += 1
         rc_launches = (1 if E > 0 else 0) + 1 + (1 if E > 0 else 0) + ((1 if passes == 0 else 3 * passes) if E > 0 else 0)
-    launches = K * (rc_launches + 2 + (1 if framed and E > 0 else 0))
+    launches = K * (rc_launches + 2 + (1 if framed and E > 0 else 0))  # in the timed steps
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

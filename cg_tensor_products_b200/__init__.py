@@ -54,6 +54,7 @@ def _load():
         "etp_edge_frames": [vp, i32, vp, vp, vp],
         "etp_forward": [vp, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp],
         "etp_backward": [vp, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp],
+        "etp_assemble_forces": [i32, i32, vp, vp, vp, vp, vp, vp, vp, vp],
         "etp_reverse_csr_workspace_size": [i32, i32, ctypes.POINTER(sz)],
         "etp_build_reverse_csr": [i32, i32, vp, vp, vp, vp, vp, vp, sz, vp],
         "etp_build_reverse_csr_static": [i32, i32, vp, vp, vp, vp, vp, vp],
@@ -192,6 +193,24 @@ def backward(plan: Plan, row_ptr, src, rev_ptr, rev_perm, dst, r, x, w, grad_out
                                 _ptr(dst), _ptr(r), _ptr(frames), _ptr(x), _ptr(w), _ptr(grad_out), _ptr(grad_x),
                                 _ptr(grad_w), _ptr(grad_r), _stream(stream)), "etp_backward")
     return grad_x, grad_w, grad_r
+
+
+def assemble_forces(N: int, row_ptr, rev_ptr, rev_perm, grad_r, r=None, forces=None, virial=None, stream=None):
+    """(forces [N, 3], virial [N, 3, 3] or None) from grad_r = dE/dr (etp_assemble_forces).
+    The per-atom virial is computed when r is given."""
+    import torch
+
+    E = grad_r.shape[0]
+    dev = grad_r.device
+    if forces is None:
+        forces = torch.empty((N, 3), device=dev, dtype=torch.float32)
+    if r is not None and virial is None:
+        virial = torch.empty((N, 3, 3), device=dev, dtype=torch.float32)
+    _need_cuda(row_ptr, rev_ptr, rev_perm, grad_r, r, forces, virial)
+    _check(_load().etp_assemble_forces(int(N), int(E), _ptr(row_ptr), _ptr(rev_ptr), _ptr(rev_perm), _ptr(r),
+                                       _ptr(grad_r), _ptr(forces), _ptr(virial), _stream(stream)),
+           "etp_assemble_forces")
+    return forces, virial
 
 
 def reverse_csr_workspace_size(N: int, E: int) -> int:

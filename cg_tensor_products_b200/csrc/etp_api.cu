@@ -295,6 +295,19 @@ etp_status etp_backward(etp_plan_t plan, int N, int E, const int32_t* row_ptr, c
     return cuda_status(err);
 }
 
+etp_status etp_assemble_forces(int N, int E, const int32_t* row_ptr, const int32_t* rev_ptr, const int32_t* rev_perm,
+                               const float* r, const float* grad_r, float* forces, float* virial, etp_stream_t stream) {
+    if (N < 0 || E < 0) return ETP_ERR_INVALID_ARG;
+    if (N == 0) return E == 0 ? ETP_OK : ETP_ERR_INVALID_ARG;
+    if (!row_ptr || !rev_ptr || !forces || !aligned4(row_ptr) || !aligned4(rev_ptr) || !aligned4(forces))
+        return ETP_ERR_INVALID_ARG;
+    if (virial && !aligned4(virial)) return ETP_ERR_INVALID_ARG;
+    if (E > 0 && (!rev_perm || !grad_r || !aligned4(rev_perm) || !aligned4(grad_r))) return ETP_ERR_INVALID_ARG;
+    if (E > 0 && virial && (!r || !aligned4(r))) return ETP_ERR_INVALID_ARG;
+    return cuda_status(etp::assemble_forces(N, E, row_ptr, rev_ptr, rev_perm, r, grad_r, forces, virial,
+                                            reinterpret_cast<cudaStream_t>(stream)));
+}
+
 etp_status etp_reverse_csr_workspace_size(int N, int E, size_t* bytes) {
     if (N < 0 || E < 0 || !bytes) return ETP_ERR_INVALID_ARG;
     *bytes = etp::reverse_csr_workspace_bytes(N, E);

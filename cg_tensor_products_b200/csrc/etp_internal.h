@@ -101,6 +101,8 @@ size_t reverse_csr_workspace_bytes(int N, int E);
 // radix_workspace_bytes_for).
 cudaError_t build_reverse_csr(int N, int E, const int32_t* row_ptr, const int32_t* src, int32_t* rev_ptr,
                               int32_t* rev_perm, int32_t* dst, void* ws, cudaStream_t s, bool one_pass = true);
+cudaError_t assemble_forces(int N, int E, const int32_t* row_ptr, const int32_t* rev_ptr, const int32_t* rev_perm,
+                            const float* r, const float* grad_r, float* forces, float* virial, cudaStream_t s);
 cudaError_t validate_csr(int N, int E, const int32_t* row_ptr, const int32_t* src, int32_t* flag, cudaStream_t s);
 
 }  // namespace etp

@@ -169,6 +169,24 @@ ETP_API etp_status etp_backward(etp_plan_t plan, int N, int E, const int32_t* ro
                         const float* grad_out, float* grad_x, float* grad_w, float* grad_r,
                         etp_stream_t stream);
 
+/* Atom forces and per-atom virials from per-edge energy derivatives.
+ * The pages evaluate models on energies and forces ("FlashCart 如何让等变原子间势更快更准?",
+ * section "560 万参数模型胜过 1.89 亿参数 transformer"); forces are minus the position
+ * gradient of the energy. With r_e = pos[src e] - pos[dst e] (plus a fixed periodic
+ * shift) and grad_r[e] = dE/dr_e (etp_backward's grad_r, plus whatever other terms
+ * of dE/dr_e the caller adds):
+ *   forces[k]          = sum_{e: dst e = k} grad_r[e] - sum_{e: src e = k} grad_r[e]
+ *   virial[k][a][b]    = sum_{e: dst e = k} grad_r[e][a] * r[e][b]
+ * (summed over k, the virial is dE/d(eps_ab) under the strain r -> (I + eps) r of
+ * every edge vector; each edge's term is assigned to its destination atom).
+ * row_ptr [N+1] and src define the CSR by destination; rev_ptr [N+1], rev_perm [E]
+ * are etp_build_reverse_csr's output for it. forces: float32 [N][3]; virial:
+ * float32 [N][3][3] or NULL (then r may be NULL). Every sum is taken in a fixed
+ * order: results repeat bit for bit. Overwrites its outputs; allocates nothing. */
+ETP_API etp_status etp_assemble_forces(int N, int E, const int32_t* row_ptr, const int32_t* rev_ptr,
+                                       const int32_t* rev_perm, const float* r, const float* grad_r,
+                                       float* forces, float* virial, etp_stream_t stream);
+
 /* Bytes of device workspace etp_build_reverse_csr needs for (N, E). */
 ETP_API etp_status etp_reverse_csr_workspace_size(int N, int E, size_t* bytes);
 

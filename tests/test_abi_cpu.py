@@ -23,7 +23,7 @@ def lib():
 
 def test_exports_every_declared_symbol(lib):
     names = etp.declared_symbols()
-    assert len(names) == 13
+    assert len(names) == 14
     for n in names:
         assert hasattr(lib, n), n
 
@@ -110,6 +110,14 @@ def test_host_argument_checks(lib):
     assert G(h, 4, None, ok, None) == etp.ETP_ERR_INVALID_ARG       # r NULL
     assert G(h, 4, ok, bad, None) == etp.ETP_ERR_INVALID_ARG        # frames misaligned
     assert G(h, 0, None, None, None) == etp.ETP_OK                  # nothing to do
+    A = lib.etp_assemble_forces
+    assert A(-1, 4, ok, ok, ok, ok, ok, ok, None, None) == etp.ETP_ERR_INVALID_ARG      # N < 0
+    assert A(0, 4, ok, ok, ok, ok, ok, ok, None, None) == etp.ETP_ERR_INVALID_ARG       # edges without nodes
+    assert A(0, 0, None, None, None, None, None, None, None, None) == etp.ETP_OK        # nothing to do
+    assert A(4, 4, ok, ok, ok, ok, ok, None, None, None) == etp.ETP_ERR_INVALID_ARG     # forces NULL
+    assert A(4, 4, ok, ok, None, ok, ok, ok, None, None) == etp.ETP_ERR_INVALID_ARG     # rev_perm NULL
+    assert A(4, 4, ok, ok, ok, None, ok, ok, ok, None) == etp.ETP_ERR_INVALID_ARG       # virial without r
+    assert A(4, 4, ok, ok, ok, ok, ctypes.c_void_p(0x10002), ok, None, None) == etp.ETP_ERR_INVALID_ARG  # grad_r
     sz = ctypes.c_size_t()
     assert lib.etp_reverse_csr_workspace_size(10, 100, ctypes.byref(sz)) == 0 and sz.value > 0
     assert lib.etp_reverse_csr_workspace_size(-1, 100, ctypes.byref(sz)) == etp.ETP_ERR_INVALID_ARG

@@ -14,7 +14,8 @@ import oracle
 import oracle.cg
 import workloads
 from cg_tensor_products_b200 import build as etp_build
-from gpu_helpers import (check_errs, check_reverse_csr, compare_full, compare_sampled, rel_err, run_gpu, to_dev)
+from gpu_helpers import (VJP_TOL, check_errs, check_reverse_csr, compare_full, compare_sampled, rel_err, run_gpu,
+                         to_dev)
 
 pytestmark = pytest.mark.gpu
 
@@ -299,3 +300,33 @@ def test_hub_rows_cut_across_many_tasks(framed):
     errs = compare_full(wl, res)
     print(errs)
     check_errs(errs)
+
+
+@pytest.mark.parametrize("name", ["tiny", "water", "micro_l3"])
+def test_assembled_forces_match_oracle(name):
+    """Forces and per-atom virials from the GPU's grad_r against the oracle's
+    assembly of the oracle's grad_r (VJP tolerance), momentum conservation, and
+    bit-for-bit repetition."""
+    wl = workloads.make(name)
+    res = run_gpu(wl, framed=True)
+    r = torch.from_numpy(wl.r).cuda()
+    rp = torch.from_numpy(wl.row_ptr).cuda()
+    F, V = etp.assemble_forces(wl.N, rp, res["rev_ptr"], res["rev_perm"], res["grad_r"], r=r)
+    F2, V2 = etp.assemble_forces(wl.N, rp, res["rev_ptr"], res["rev_perm"], res["grad_r"], r=r)
+    F3, V3 = etp.assemble_forces(wl.N, rp, res["rev_ptr"], res["rev_perm"], res["grad_r"])
+    torch.cuda.synchronize()
+    assert torch.equal(F, F2) and torch.equal(V, V2) and torch.equal(F, F3) and V3 is None
+    tp = oracle.OracleTP(wl.irreps, wl.L, wl.irreps, wl.C)
+    if name == "micro_l3":   # grad_r of a sample of edges is enough to pin the oracle side here
+        edges = np.arange(wl.E)
+        g_ref = np.concatenate([tp.backward(wl.row_ptr, wl.src, wl.r, wl.x, wl.w, wl.g, nodes=np.arange(1),
+                                            edges=edges[k:k + 32768], want=("r",))["grad_r"]
+                                for k in range(0, wl.E, 32768)])
+    else:
+        g_ref = tp.backward(wl.row_ptr, wl.src, wl.r, wl.x, wl.w, wl.g, want=("r",))["grad_r"]
+    F_ref, V_ref = oracle.assemble_forces(wl.N, wl.row_ptr, wl.src, wl.r, g_ref)
+    assert rel_err(F, F_ref) <= VJP_TOL and rel_err(V, V_ref) <= VJP_TOL
+    # the GPU assembly itself, on the GPU's own grad_r, to fp32 summation accuracy
+    F_own, V_own = oracle.assemble_forces(wl.N, wl.row_ptr, wl.src, wl.r, res["grad_r"].double().cpu().numpy())
+    assert rel_err(F, F_own) <= 1e-5 and rel_err(V, V_own) <= 1e-5
+    assert F.double().sum(0).abs().max().item() <= 1e-5 * res["grad_r"].double().abs().sum().item()
