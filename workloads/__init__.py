@@ -177,8 +177,8 @@ def _geometry_water(rng, rc=5.0):
     return row_ptr, src_sorted, r, rc
 
 
-def _geometry_large(rng, rc=4.5):
-    n, dens = 32768, 0.1
+def _geometry_large(rng, rc=4.5, n=32768):
+    dens = 0.1
     box = (n / dens) ** (1.0 / 3.0)
     pos = rng.uniform(0.0, box, size=(n, 3))
     dst, src = radius_pairs(pos, box, rc)
@@ -213,8 +213,9 @@ def radial_mlp_weights(rng, r: np.ndarray, rc: float, P: int, C: int,
 def make(name: str, seed: int = 0, n_nodes: int | None = None) -> Workload:
     """Build one named workload from numpy.random.default_rng(seed).
 
-    n_nodes (micro workloads only) shrinks the node count, keeping 128 neighbours
-    per node (profiling captures use it to stay small)."""
+    n_nodes (micro and large workloads) shrinks the node count: micro keeps 128
+    neighbours per node, large keeps its density and cutoff (about 38 neighbours);
+    profiling captures use it to stay small."""
     spec = SPECS[name]
     L, C = spec["L"], spec["C"]
     P = N_PATHS_SO3[L]
@@ -228,7 +229,7 @@ def make(name: str, seed: int = 0, n_nodes: int | None = None) -> Workload:
         row_ptr, src, r64, rc = _geometry_water(rng)
         r = r64.astype(np.float32)
     elif name == "large":
-        row_ptr, src, r64 = _geometry_large(rng)
+        row_ptr, src, r64 = _geometry_large(rng, n=n_nodes or 32768)
         r = r64.astype(np.float32)
     else:
         raise KeyError(name)
