@@ -311,11 +311,18 @@ def main():
     nnz_total = len(plan.couplings()[1])
     N, E = wl.N, wl.E
     host = {k: torch.from_numpy(np.ascontiguousarray(getattr(wl, k))) for k in ("row_ptr", "src", "r", "x", "w", "g")}
-    d = {k: v.to(dev) for k, v in host.items()}
-    out = torch.empty((N, plan.dim_out, wl.C), device=dev)
-    gx = torch.empty((N, plan.dim_in, wl.C), device=dev)
-    gw = torch.empty((E, plan.n_paths, wl.C), device=dev)
-    gr = torch.empty((E, 3), device=dev)
+
+    def io_buffers():
+        """A step's inputs (a device copy of `host`) and outputs."""
+        b = {k: v.to(dev) for k, v in host.items()}
+        b["out"] = torch.empty((N, plan.dim_out, wl.C), device=dev)
+        b["gx"] = torch.empty((N, plan.dim_in, wl.C), device=dev)
+        b["gw"] = torch.empty((E, plan.n_paths, wl.C), device=dev)
+        b["gr"] = torch.empty((E, 3), device=dev)
+        return b
+
+    d = io_buffers()
+    out, gx, gw, gr = d["out"], d["gx"], d["gw"], d["gr"]
     rev_ptr = torch.empty(N + 1, dtype=torch.int32, device=dev)
     rev_perm = torch.empty(E, dtype=torch.int32, device=dev)
     dst = torch.empty(E, dtype=torch.int32, device=dev)
@@ -327,26 +334,31 @@ def main():
     sp = etp._stream(stream)
     P = etp._ptr
 
-    def step(ev=None):
+    def step(ev=None, b=None, s=None):
+        """One pass of the path on the buffers b (default d) and stream s (default the current one); the reverse
+        CSR, frames and workspace are shared scratch (every use is ordered on the one compute stream)."""
+        b = d if b is None else b
+        s = stream if s is None else s
+        spp = etp._stream(s)
         if ev:
-            ev[0].record(stream)
-        etp._check(lib.etp_build_reverse_csr(N, E, P(d["row_ptr"]), P(d["src"]), P(rev_ptr), P(rev_perm), P(dst),
-                                             P(ws), ws.numel(), sp), "reverse csr")
+            ev[0].record(s)
+        etp._check(lib.etp_build_reverse_csr(N, E, P(b["row_ptr"]), P(b["src"]), P(rev_ptr), P(rev_perm), P(dst),
+                                             P(ws), ws.numel(), spp), "reverse csr")
         if ev:
-            ev[1].record(stream)
+            ev[1].record(s)
         if framed:
-            etp._check(lib.etp_edge_frames(plan.handle, E, P(d["r"]), P(frames), sp), "edge frames")
+            etp._check(lib.etp_edge_frames(plan.handle, E, P(b["r"]), P(frames), spp), "edge frames")
         if ev:
-            ev[2].record(stream)
-        etp._check(lib.etp_forward(plan.handle, N, E, P(d["row_ptr"]), P(d["src"]), P(d["r"]), P(frames), P(d["x"]),
-                                   P(d["w"]), P(out), sp), "forward")
+            ev[2].record(s)
+        etp._check(lib.etp_forward(plan.handle, N, E, P(b["row_ptr"]), P(b["src"]), P(b["r"]), P(frames), P(b["x"]),
+                                   P(b["w"]), P(b["out"]), spp), "forward")
         if ev:
-            ev[3].record(stream)
-        etp._check(lib.etp_backward(plan.handle, N, E, P(d["row_ptr"]), P(d["src"]), P(rev_ptr), P(rev_perm), P(dst),
-                                    P(d["r"]), P(frames), P(d["x"]), P(d["w"]), P(d["g"]), P(gx), P(gw), P(gr), sp),
-                       "backward")
+            ev[3].record(s)
+        etp._check(lib.etp_backward(plan.handle, N, E, P(b["row_ptr"]), P(b["src"]), P(rev_ptr), P(rev_perm), P(dst),
+                                    P(b["r"]), P(frames), P(b["x"]), P(b["w"]), P(b["g"]), P(b["gx"]), P(b["gw"]),
+                                    P(b["gr"]), spp), "backward")
         if ev:
-            ev[4].record(stream)
+            ev[4].record(s)
 
     for _ in range(max(args.warmup, 0)):
         step()
@@ -425,37 +437,61 @@ def main():
     fp32 = {"kernel": kname, "equiv_tflops": eq, "nominal_peak_tflops": fp32_peak, "frac": eq / fp32_peak,
             "note": f"nominal = {sms} SMs x 128 lanes x 2 flop x {mhz:.0f} MHz; flop = the method's sparse-CG count"}
 
-    # end to end through the public API with host buffers (pinned), copies inside the timed region
+    # end to end through the public API with host buffers (pinned): every step copies its inputs host -> device,
+    # runs the path and copies its outputs device -> host, all inside the timed region. Steps are pipelined the
+    # way a user streaming batches would run them: two sets of device buffers alternate, the input copies run
+    # on one stream, the path on another and the output copies on a third, so step k+1's inputs and step k-1's
+    # outputs cross PCIe (both directions at once) while step k computes.
     e2e = None
     if not args.no_e2e:
         pin = {k: v.pin_memory() for k, v in host.items()}
-        h_out = {"out": torch.empty(out.shape).pin_memory(), "gx": torch.empty(gx.shape).pin_memory(),
-                 "gw": torch.empty(gw.shape).pin_memory(), "gr": torch.empty(gr.shape).pin_memory()}
+        h_out = {k: torch.empty(d[k].shape).pin_memory() for k in ("out", "gx", "gw", "gr")}
         h2d = sum(v.numel() * v.element_size() for v in pin.values())
         d2h = sum(v.numel() * v.element_size() for v in h_out.values())
         k_e2e = max(3, min(K, 20))
+        sets = [d, io_buffers()]
+        s_in, s_comp, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
 
-        def e2e_step():
-            for k, v in pin.items():
-                d[k].copy_(v, non_blocking=True)
-            step()
-            h_out["out"].copy_(out, non_blocking=True)
-            h_out["gx"].copy_(gx, non_blocking=True)
-            h_out["gw"].copy_(gw, non_blocking=True)
-            h_out["gr"].copy_(gr, non_blocking=True)
+        def e2e_run(n):
+            done_comp, done_out = [], []
+            for k in range(n):
+                b = sets[k % 2]
+                if k >= 2:
+                    s_in.wait_event(done_comp[k - 2])   # set b's inputs were read by step k-2
+                with torch.cuda.stream(s_in):
+                    for key, v in pin.items():
+                        b[key].copy_(v, non_blocking=True)
+                ready = torch.cuda.Event()
+                ready.record(s_in)
+                s_comp.wait_event(ready)
+                if k >= 2:
+                    s_comp.wait_event(done_out[k - 2])  # set b's outputs were read back by step k-2
+                step(b=b, s=s_comp)
+                c = torch.cuda.Event()
+                c.record(s_comp)
+                done_comp.append(c)
+                s_out.wait_event(c)
+                with torch.cuda.stream(s_out):
+                    for key, v in h_out.items():
+                        v.copy_(b[key], non_blocking=True)
+                o = torch.cuda.Event()
+                o.record(s_out)
+                done_out.append(o)
+            return done_out[-1]
 
-        e2e_step()
+        e2e_run(2)
         torch.cuda.synchronize()
         replicas.barrier(world)
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        for _ in range(k_e2e):
-            e2e_step()
-        b.record(stream)
+        a, z = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(s_in)
+        last = e2e_run(k_e2e)
+        s_out.wait_event(last)
+        z.record(s_out)
         torch.cuda.synchronize()
-        e_ms = replicas.max_over_ranks(a.elapsed_time(b) / k_e2e, world, dev)
+        e_ms = replicas.max_over_ranks(a.elapsed_time(z) / k_e2e, world, dev)
         e2e = {"value": world * E / (e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-               "ms_per_step": e_ms, "steps": k_e2e}
+               "ms_per_step": e_ms, "steps": k_e2e,
+               "pipelining": "double-buffered: input copies, compute and output copies on three streams"}
 
     # kernels launched per step: the reverse CSR (one counting pass: counts, chunk scan, chunk-total scan,
     # scatter, edge rows; otherwise counts, scan, edge rows and 3 per 8-bit radix pass), frames, forward, backward
