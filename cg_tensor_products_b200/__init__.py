@@ -94,6 +94,7 @@ def _stream(stream):
 
 
 def _need_cuda(*ts):
+    dev = None
     for t in ts:
         if t is None:
             continue
@@ -101,6 +102,27 @@ def _need_cuda(*ts):
             raise ValueError("tensors must be CUDA tensors: this library has no CPU path")
         if not t.is_contiguous():
             raise ValueError("tensors must be contiguous")
+        if dev is None:
+            dev = t.device
+        elif t.device != dev:
+            raise ValueError(f"tensors on different devices ({dev}, {t.device})")
+
+
+def _expect(t, name: str, dtype: str, shape: tuple):
+    """Raise ValueError unless t (if given) has the dtype ('float32' / 'int32' / 'uint8') and the
+    shape (None entries match any size); checked before anything is launched."""
+    if t is None:
+        return
+    if str(t.dtype) != "torch." + dtype:
+        raise ValueError(f"{name}: expected {dtype}, got {t.dtype}")
+    if t.dim() != len(shape) or any(want is not None and got != want for got, want in zip(t.shape, shape)):
+        raise ValueError(f"{name}: expected shape {tuple('*' if v is None else v for v in shape)}, "
+                         f"got {tuple(t.shape)}")
+
+
+def _check_graph(row_ptr, src, N: int, E: int):
+    _expect(row_ptr, "row_ptr", "int32", (N + 1,))
+    _expect(src, "src", "int32", (E,))
 
 
 class Plan:
@@ -153,9 +175,11 @@ def edge_frames(plan: Plan, r, frames=None, stream=None):
     """Per-edge frame records [E][FRAME_FLOATS] for r (launches etp_edge_frames)."""
     import torch
 
+    _expect(r, "r", "float32", (None, 3))
     E = r.shape[0]
     if frames is None:
         frames = torch.empty((E, FRAME_FLOATS), device=r.device, dtype=torch.float32)
+    _expect(frames, "frames", "float32", (E, FRAME_FLOATS))
     _need_cuda(r, frames)
     _check(_load().etp_edge_frames(plan.handle, E, _ptr(r), _ptr(frames), _stream(stream)), "etp_edge_frames")
     return frames
@@ -167,8 +191,14 @@ def forward(plan: Plan, row_ptr, src, r, x, w, out=None, frames=None, stream=Non
     import torch
 
     N, E = row_ptr.numel() - 1, src.numel()
+    _check_graph(row_ptr, src, N, E)
+    _expect(r, "r", "float32", (E, 3))
+    _expect(frames, "frames", "float32", (E, FRAME_FLOATS))
+    _expect(x, "x", "float32", (N, plan.dim_in, plan.C))
+    _expect(w, "w", "float32", (E, plan.n_paths, plan.C))
     if out is None:
         out = torch.empty((N, plan.dim_out, plan.C), device=x.device, dtype=torch.float32)
+    _expect(out, "out", "float32", (N, plan.dim_out, plan.C))
     _need_cuda(row_ptr, src, r, frames, x, w, out)
     _check(_load().etp_forward(plan.handle, N, E, _ptr(row_ptr), _ptr(src), _ptr(r), _ptr(frames), _ptr(x), _ptr(w),
                                _ptr(out), _stream(stream)), "etp_forward")
@@ -181,6 +211,15 @@ def backward(plan: Plan, row_ptr, src, rev_ptr, rev_perm, dst, r, x, w, grad_out
     import torch
 
     N, E = row_ptr.numel() - 1, src.numel()
+    _check_graph(row_ptr, src, N, E)
+    _expect(rev_ptr, "rev_ptr", "int32", (N + 1,))
+    _expect(rev_perm, "rev_perm", "int32", (E,))
+    _expect(dst, "dst", "int32", (E,))
+    _expect(r, "r", "float32", (E, 3))
+    _expect(frames, "frames", "float32", (E, FRAME_FLOATS))
+    _expect(x, "x", "float32", (N, plan.dim_in, plan.C))
+    _expect(w, "w", "float32", (E, plan.n_paths, plan.C))
+    _expect(grad_out, "grad_out", "float32", (N, plan.dim_out, plan.C))
     dev = x.device
     if "x" in want and grad_x is None:
         grad_x = torch.empty((N, plan.dim_in, plan.C), device=dev, dtype=torch.float32)
@@ -188,6 +227,9 @@ def backward(plan: Plan, row_ptr, src, rev_ptr, rev_perm, dst, r, x, w, grad_out
         grad_w = torch.empty((E, plan.n_paths, plan.C), device=dev, dtype=torch.float32)
     if "r" in want and grad_r is None:
         grad_r = torch.empty((E, 3), device=dev, dtype=torch.float32)
+    _expect(grad_x, "grad_x", "float32", (N, plan.dim_in, plan.C))
+    _expect(grad_w, "grad_w", "float32", (E, plan.n_paths, plan.C))
+    _expect(grad_r, "grad_r", "float32", (E, 3))
     _need_cuda(row_ptr, src, rev_ptr, rev_perm, dst, r, frames, x, w, grad_out, grad_x, grad_w, grad_r)
     _check(_load().etp_backward(plan.handle, N, E, _ptr(row_ptr), _ptr(src), _ptr(rev_ptr), _ptr(rev_perm),
                                 _ptr(dst), _ptr(r), _ptr(frames), _ptr(x), _ptr(w), _ptr(grad_out), _ptr(grad_x),
@@ -200,12 +242,20 @@ def assemble_forces(N: int, row_ptr, rev_ptr, rev_perm, grad_r, r=None, forces=N
     The per-atom virial is computed when r is given."""
     import torch
 
+    _expect(grad_r, "grad_r", "float32", (None, 3))
     E = grad_r.shape[0]
+    _expect(row_ptr, "row_ptr", "int32", (N + 1,))
+    _expect(rev_ptr, "rev_ptr", "int32", (N + 1,))
+    _expect(rev_perm, "rev_perm", "int32", (E,))
+    _expect(r, "r", "float32", (E, 3))
     dev = grad_r.device
     if forces is None:
         forces = torch.empty((N, 3), device=dev, dtype=torch.float32)
     if r is not None and virial is None:
         virial = torch.empty((N, 3, 3), device=dev, dtype=torch.float32)
+    _expect(forces, "forces", "float32", (N, 3))
+    if virial is not None and (str(virial.dtype) != "torch.float32" or virial.numel() != 9 * N):
+        raise ValueError("virial: expected float32 with N*9 elements")
     _need_cuda(row_ptr, rev_ptr, rev_perm, grad_r, r, forces, virial)
     _check(_load().etp_assemble_forces(int(N), int(E), _ptr(row_ptr), _ptr(rev_ptr), _ptr(rev_perm), _ptr(r),
                                        _ptr(grad_r), _ptr(forces), _ptr(virial), _stream(stream)),
@@ -224,6 +274,7 @@ def build_reverse_csr(N: int, row_ptr, src, with_dst=True, workspace=None, strea
     import torch
 
     E = src.numel()
+    _check_graph(row_ptr, src, N, E)
     dev = row_ptr.device
     rev_ptr = torch.empty(N + 1, dtype=torch.int32, device=dev)
     rev_perm = torch.empty(E, dtype=torch.int32, device=dev)
@@ -231,6 +282,7 @@ def build_reverse_csr(N: int, row_ptr, src, with_dst=True, workspace=None, strea
     nbytes = reverse_csr_workspace_size(N, E)
     if workspace is None:
         workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=dev)
+    _expect(workspace, "workspace", "uint8", (None,))
     _need_cuda(row_ptr, src, rev_ptr, rev_perm, dst, workspace)
     _check(_load().etp_build_reverse_csr(N, E, _ptr(row_ptr), _ptr(src), _ptr(rev_ptr), _ptr(rev_perm), _ptr(dst),
                                          _ptr(workspace), workspace.numel(), _stream(stream)),
@@ -244,6 +296,7 @@ def build_reverse_csr_static(N: int, row_ptr, src, with_dst=True, stream=None):
     import torch
 
     E = src.numel()
+    _check_graph(row_ptr, src, N, E)
     dev = row_ptr.device
     rev_ptr = torch.empty(N + 1, dtype=torch.int32, device=dev)
     rev_perm = torch.empty(E, dtype=torch.int32, device=dev)
@@ -265,6 +318,7 @@ def validate_csr(N: int, row_ptr, src, stream=None) -> int:
     """The ETP_CSR_* bits of every problem found in the CSR (0 = valid). Synchronises the stream."""
     import torch
 
+    _check_graph(row_ptr, src, N, src.numel())
     flag = torch.empty(1, dtype=torch.int32, device=row_ptr.device)
     _need_cuda(row_ptr, src, flag)
     _check(_load().etp_validate_csr(N, src.numel(), _ptr(row_ptr), _ptr(src), _ptr(flag), _stream(stream)),

@@ -149,3 +149,28 @@ def test_binding_refuses_cpu_tensors(lib):
     with pytest.raises(ValueError):
         etp.forward(plan, row_ptr, torch.zeros(0, dtype=torch.int32), torch.zeros(0, 3),
                     torch.zeros(2, 4, 8), torch.zeros(0, 5, 8), out=torch.zeros(2, 4, 8))
+
+
+def test_binding_checks_dtypes_and_shapes(lib):
+    """Wrong dtypes or shapes are refused before anything reaches the library."""
+    import torch
+
+    plan = etp.Plan("0..1", 1, "0..1", 8)
+    N, E = 3, 4
+    row_ptr = torch.tensor([0, 1, 3, 4], dtype=torch.int32)
+    src = torch.zeros(E, dtype=torch.int32)
+    r, x, w = torch.zeros(E, 3), torch.zeros(N, 4, 8), torch.zeros(E, 5, 8)
+    out = torch.zeros(N, 4, 8)
+    cases = [dict(x=x.double()), dict(w=torch.zeros(E, 4, 8)), dict(r=torch.zeros(E, 2)),
+             dict(src=src.long()), dict(row_ptr=row_ptr[:3]), dict(out=torch.zeros(N, 4, 4))]
+    for bad in cases:
+        args = dict(row_ptr=row_ptr, src=src, r=r, x=x, w=w, out=out)
+        args.update(bad)
+        with pytest.raises(ValueError, match="expected"):
+            etp.forward(plan, args["row_ptr"], args["src"], args["r"], args["x"], args["w"], out=args["out"])
+    with pytest.raises(ValueError, match="expected"):
+        etp.edge_frames(plan, torch.zeros(E, 3, dtype=torch.float16))
+    with pytest.raises(ValueError, match="expected"):
+        etp.assemble_forces(N, row_ptr, row_ptr, src, torch.zeros(E, 3), forces=torch.zeros(N, 2))
+    with pytest.raises(ValueError, match="expected"):
+        etp.build_reverse_csr(N, row_ptr.long(), src)
