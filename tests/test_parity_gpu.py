@@ -330,3 +330,45 @@ def test_assembled_forces_match_oracle(name):
     F_own, V_own = oracle.assemble_forces(wl.N, wl.row_ptr, wl.src, wl.r, res["grad_r"].double().cpu().numpy())
     assert rel_err(F, F_own) <= 1e-5 and rel_err(V, V_own) <= 1e-5
     assert F.double().sum(0).abs().max().item() <= 1e-5 * res["grad_r"].double().abs().sum().item()
+
+
+def test_cuda_graph_capture_and_replay():
+    """The whole step (reverse CSR, frames, forward, VJP, forces) captured once into a
+    CUDA graph and replayed on new input values gives what eager calls give."""
+    rng = np.random.default_rng(31)
+    wl = workloads.random_graph(rng, 300, 9000, 3, 64, 34)
+    plan = etp.Plan(wl.irreps, wl.L, wl.irreps, wl.C)
+    t = to_dev(wl)
+    N, E = wl.N, wl.E
+    outs = dict(out=torch.empty(N, 16, 64, device="cuda"), gx=torch.empty(N, 16, 64, device="cuda"),
+                gw=torch.empty(E, 34, 64, device="cuda"), gr=torch.empty(E, 3, device="cuda"),
+                frames=torch.empty(E, etp.FRAME_FLOATS, device="cuda"), F=torch.empty(N, 3, device="cuda"),
+                ws=torch.empty(etp.reverse_csr_workspace_size(N, E), dtype=torch.uint8, device="cuda"))
+
+    def step():
+        rp, perm, dst = etp.build_reverse_csr(N, t["row_ptr"], t["src"], workspace=outs["ws"])
+        etp.edge_frames(plan, t["r"], frames=outs["frames"])
+        etp.forward(plan, t["row_ptr"], t["src"], None, t["x"], t["w"], out=outs["out"], frames=outs["frames"])
+        etp.backward(plan, t["row_ptr"], t["src"], rp, perm, dst, None, t["x"], t["w"], t["g"], grad_x=outs["gx"],
+                     grad_w=outs["gw"], grad_r=outs["gr"], frames=outs["frames"])
+        etp.assemble_forces(N, t["row_ptr"], rp, perm, outs["gr"], forces=outs["F"])
+
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        step()                        # warm-up outside capture (fills the launch-shape caches)
+    torch.cuda.current_stream().wait_stream(s)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        step()
+    for trial in range(2):
+        for k in ("r", "x", "w", "g"):
+            t[k].copy_(torch.randn_like(t[k]))
+        graph.replay()
+        torch.cuda.synchronize()
+        got = {k: outs[k].clone() for k in ("out", "gx", "gw", "gr", "F")}
+        step()
+        torch.cuda.synchronize()
+        assert etp.device_fault() == 0
+        for k, v in got.items():
+            assert rel_err(v, outs[k].double().cpu().numpy()) <= 1e-6, (trial, k)
