@@ -168,10 +168,15 @@ def measured_peaks():
 
 
 def kernel_source_hash():
+    """Hash of the kernel sources' code (line comments and blank lines dropped, so that documentation edits
+    keep a capture valid while any code change invalidates it)."""
     h = hashlib.sha256()
     for rel in KERNEL_SOURCES:
-        with open(os.path.join(ROOT, rel), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, rel), encoding="utf-8") as f:
+            for line in f:
+                code = line.split("//", 1)[0].rstrip()
+                if code:
+                    h.update(code.encode() + b"\n")
     return h.hexdigest()[:16]
 
 

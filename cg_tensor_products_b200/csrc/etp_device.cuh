@@ -1,6 +1,6 @@
-// Device building blocks shared by the forward and backward kernels: compile-time
-// path sets and coupling lists, a compile-time loop, and the real spherical
-// harmonics of an edge vector (values, and values with their r-derivative).
+// Device building blocks shared by the kernels: compile-time path sets, a
+// compile-time loop, the real spherical harmonics of a unit vector (used to fit
+// the Wigner matrices of each edge frame) and the L2 evict-first cache policy.
 #pragma once
 
 #include <cuda_runtime.h>
@@ -75,22 +75,10 @@ constexpr double sh_norm(int l, int m) {
     return csqrt((2.0 * l + 1.0) * cfact(l - m) / cfact(l + m)) * (m > 0 ? csqrt(2.0) : 1.0);
 }
 
-// Forward-mode dual number: a value and its derivative along the 3 edge-vector axes.
-struct Dual3 {
-    float v, d0, d1, d2;
-};
-__device__ __forceinline__ Dual3 operator+(Dual3 a, Dual3 b) { return {a.v + b.v, a.d0 + b.d0, a.d1 + b.d1, a.d2 + b.d2}; }
-__device__ __forceinline__ Dual3 operator-(Dual3 a, Dual3 b) { return {a.v - b.v, a.d0 - b.d0, a.d1 - b.d1, a.d2 - b.d2}; }
-__device__ __forceinline__ Dual3 operator*(Dual3 a, Dual3 b) {
-    return {a.v * b.v, a.d0 * b.v + a.v * b.d0, a.d1 * b.v + a.v * b.d1, a.d2 * b.v + a.v * b.d2};
-}
-__device__ __forceinline__ Dual3 operator*(float s, Dual3 a) { return {s * a.v, s * a.d0, s * a.d1, s * a.d2}; }
 template <class T>
 __device__ __forceinline__ T sh_const(float c);
 template <>
 __device__ __forceinline__ float sh_const<float>(float c) { return c; }
-template <>
-__device__ __forceinline__ Dual3 sh_const<Dual3>(float c) { return {c, 0.f, 0.f, 0.f}; }
 
 // Real spherical harmonics of a unit vector u, blocks l = 0..L, m = -l..l:
 //   Y_lm = K_lm * Pi_l^|m|(u_z) * {Re (u_x + i u_y)^m (m > 0), 1 (m = 0), Im (u_x + i u_y)^|m| (m < 0)}
@@ -136,66 +124,6 @@ __device__ __forceinline__ void sh_unit(T ux, T uy, T uz, T (&Y)[(L + 1) * (L + 
     });
 }
 
-// Y_lm(r / |r|) for all l <= L; |r| < 1e-12 gives Y_0 = 1 and the rest 0.
-template <int L>
-__device__ __forceinline__ void sh_eval(float rx, float ry, float rz, float (&Y)[(L + 1) * (L + 1)]) {
-    float n2 = rx * rx + ry * ry + rz * rz;
-    bool ok = n2 >= 1e-24f;
-    float inv = ok ? rsqrtf(n2) : 0.f;
-    sh_unit<L, float>(rx * inv, ry * inv, rz * inv, Y);
-    if (!ok) {
-#pragma unroll
-        for (int k = 1; k < (L + 1) * (L + 1); ++k) Y[k] = 0.f;
-    }
-}
-
-// dY_lm/dr (3 components each) for the unnormalised edge vector r: the
-// harmonics are evaluated on dual numbers seeded with du/dr = (I - u u^T)/|r|.
-template <int L>
-__device__ __forceinline__ void sh_eval_grad(float rx, float ry, float rz, float (&Y)[(L + 1) * (L + 1)],
-                                             float (&dY)[(L + 1) * (L + 1)][3]) {
-    constexpr int D = (L + 1) * (L + 1);
-    float n2 = rx * rx + ry * ry + rz * rz;
-    bool ok = n2 >= 1e-24f;
-    float inv = ok ? rsqrtf(n2) : 0.f;
-    float ux = rx * inv, uy = ry * inv, uz = rz * inv;
-    Dual3 dx{ux, (1.f - ux * ux) * inv, -ux * uy * inv, -ux * uz * inv};
-    Dual3 dy{uy, -uy * ux * inv, (1.f - uy * uy) * inv, -uy * uz * inv};
-    Dual3 dz{uz, -uz * ux * inv, -uz * uy * inv, (1.f - uz * uz) * inv};
-    Dual3 Yd[D];
-    sh_unit<L, Dual3>(dx, dy, dz, Yd);
-#pragma unroll
-    for (int k = 0; k < D; ++k) {
-        bool keep = ok || k == 0;
-        Y[k] = keep ? Yd[k].v : 0.f;
-        dY[k][0] = ok ? Yd[k].d0 : 0.f;
-        dY[k][1] = ok ? Yd[k].d1 : 0.f;
-        dY[k][2] = ok ? Yd[k].d2 : 0.f;
-    }
-}
-
-// ---------------------------------------------------------------------------
-// float4 helpers
-__device__ __forceinline__ float4 f4_zero() { return make_float4(0.f, 0.f, 0.f, 0.f); }
-__device__ __forceinline__ void f4_fma(float4& acc, float s, float4 v) {
-    acc.x = fmaf(s, v.x, acc.x);
-    acc.y = fmaf(s, v.y, acc.y);
-    acc.z = fmaf(s, v.z, acc.z);
-    acc.w = fmaf(s, v.w, acc.w);
-}
-__device__ __forceinline__ void f4_fma(float4& acc, float4 a, float4 b) {
-    acc.x = fmaf(a.x, b.x, acc.x);
-    acc.y = fmaf(a.y, b.y, acc.y);
-    acc.z = fmaf(a.z, b.z, acc.z);
-    acc.w = fmaf(a.w, b.w, acc.w);
-}
-__device__ __forceinline__ float4 f4_mul(float4 a, float4 b) {
-    return make_float4(a.x * b.x, a.y * b.y, a.z * b.z, a.w * b.w);
-}
-__device__ __forceinline__ float f4_dot(float4 a, float4 b) {
-    return fmaf(a.w, b.w, fmaf(a.z, b.z, fmaf(a.y, b.y, a.x * b.x)));
-}
-
 // L2 policy for data touched exactly once (per-edge weights and their
 // gradients): evict first, so that node features stay resident in L2.
 __device__ __forceinline__ uint64_t l2_evict_first_policy() {
@@ -203,19 +131,4 @@ __device__ __forceinline__ uint64_t l2_evict_first_policy() {
     asm("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
     return pol;
 }
-// Streaming load: no L1 allocation, L2 evict-first.
-__device__ __forceinline__ float4 ld_stream(const float4* p, uint64_t pol) {
-    float4 v;
-    asm("ld.global.nc.L1::no_allocate.L2::cache_hint.v4.f32 {%0, %1, %2, %3}, [%4], %5;"
-        : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
-        : "l"(p), "l"(pol));
-    return v;
-}
-// Streaming store: L2 evict-first.
-__device__ __forceinline__ void st_stream(float4* p, float4 v, uint64_t pol) {
-    asm volatile("st.global.L2::cache_hint.v4.f32 [%0], {%1, %2, %3, %4}, %5;" ::"l"(p), "f"(v.x), "f"(v.y),
-                 "f"(v.z), "f"(v.w), "l"(pol)
-                 : "memory");
-}
-
 }  // namespace etp

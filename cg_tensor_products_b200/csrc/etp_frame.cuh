@@ -23,13 +23,16 @@
 // The frame rotation itself is not described on the pages; it gives the same
 // result as the plain sparse contraction and is this library's choice.
 //
-// Work decomposition: a team of T lanes owns one node and a slice of 2T channels
-// (lane t holds channels 2(sT + t), 2(sT + t) + 1 as a float2). T = min(32, C/2);
-// with C = 128 a node has two slices, i.e. two warps of the same block. Each
-// team computes its edge's Wigner matrices cooperatively into its own shared
-// memory. Forward: teams walk the destination row (CSR), accumulate in
-// registers, store the node once. Backward: teams walk the source row (reverse
-// CSR) and store grad_x once; grad_w and grad_r are per edge. No atomics.
+// Work decomposition: a task is an equal contiguous range of edges (CSR order
+// forward, reverse-CSR order backward), whatever the degree distribution. A team
+// of T = min(32, C/2) lanes handles a slice of 2T channels of the task's edges
+// (lane t holds channels 2(sT + t), 2(sT + t) + 1 as a float2); with C = 128 a
+// task has two slices, the two warps of one block. Node sums accumulate in
+// registers and are stored once per row; a row cut by a task boundary is
+// combined with vector reductions onto the zeroed output. Per edge, one lane
+// bulk-copies the next edge's weights (and frame record, and in the forward the
+// source row) into the other of two shared-memory buffers; each team expands its
+// edge's Wigner matrices into shared memory, from the record or built from r.
 #pragma once
 
 #include "etp_device.cuh"
