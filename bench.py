@@ -524,7 +524,7 @@ def main():
     # kernels launched per step: the reverse CSR (one counting pass: counts, chunk scan, chunk-total scan,
     # scatter, edge rows; otherwise counts, scan, edge rows and 3 per 8-bit radix pass), frames, forward, backward
     n_tiles = (E + 1023) // 1024
-    if E > 0 and 1 <= N <= 2048 and (N + 1) * n_tiles <= (1 << 22):
+    if E > 0 and 1 <= N <= 8192 and (N + 1) * n_tiles <= (1 << 22):
         rc_launches = 5
     else:
         passes = 0

@@ -192,9 +192,10 @@ __global__ void __launch_bounds__(128) tile_scatter(const int32_t* __restrict__ 
 __device__ __forceinline__ int bucket_of(int j, int N) { return (unsigned)j < (unsigned)N ? j : N; }
 
 // table[b * n_tiles + t] = edges of tile t in bucket b, for b = 0..N.
+// (dynamic shared memory: N + 1 counters)
 __global__ void __launch_bounds__(256) tile_counts(const int32_t* __restrict__ src, int E, int N, int n_tiles,
                                                    int32_t* __restrict__ table) {
-    __shared__ int32_t h[kOnePassMaxNodes + 1];
+    extern __shared__ int32_t h[];
     for (int b = threadIdx.x; b <= N; b += 256) h[b] = 0;
     __syncthreads();
     const int t = blockIdx.x;
@@ -283,21 +284,24 @@ __global__ void __launch_bounds__(1024) scan_parts_rev_ptr(int32_t* __restrict__
 }
 
 // Stable scatter of one tile per block of 4 warps (as tile_scatter, with the
-// bucket of the full source id): rev_perm[pos] = edge id.
+// bucket of the full source id): rev_perm[pos] = edge id. Dynamic shared memory:
+// 4 x (N + 1) counters.
 __global__ void __launch_bounds__(128) tile_scatter_one_pass(const int32_t* __restrict__ src, int E, int N,
                                                              int n_tiles, const int32_t* __restrict__ table,
                                                              const int32_t* __restrict__ part,
                                                              int32_t* __restrict__ rev_perm) {
-    __shared__ int32_t cnt[4][kOnePassMaxNodes + 1];
+    extern __shared__ int32_t cnt[];  // [4][N + 1]
+    const int stride = N + 1;
     const int wid = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int t = blockIdx.x;
     constexpr int kQuarter = kTile / 4;
     const int lo = t * kTile + wid * kQuarter, hi = min(E, lo + kQuarter);
-    for (int b = lane; b <= N; b += 32) cnt[wid][b] = 0;
+    int32_t* base = cnt + wid * stride;
+    for (int b = lane; b <= N; b += 32) base[b] = 0;
     __syncwarp();
     for (int c = lo; c < hi; c += 32) {
         const int e = c + lane;
-        if (e < hi) atomicAdd(&cnt[wid][bucket_of(src[e], N)], 1);
+        if (e < hi) atomicAdd(&base[bucket_of(src[e], N)], 1);
     }
     __syncthreads();
     for (int b = threadIdx.x; b <= N; b += 128) {  // warp-exclusive prefix per bucket
@@ -305,18 +309,17 @@ __global__ void __launch_bounds__(128) tile_scatter_one_pass(const int32_t* __re
         int run = table[idx] + part[idx / kScanChunk];
 #pragma unroll
         for (int w = 0; w < 4; ++w) {
-            const int v = cnt[w][b];
-            cnt[w][b] = run;
+            const int v = cnt[w * stride + b];
+            cnt[w * stride + b] = run;
             run += v;
         }
     }
     __syncthreads();
-    int32_t* base = cnt[wid];
     const unsigned lt = (1u << lane) - 1u;
     for (int c = lo; c < hi; c += 32) {
         const int e = c + lane;
         const bool act = e < hi;
-        const int b = act ? bucket_of(src[e], N) : kOnePassMaxNodes + 1 + lane;  // inactive lanes match nobody
+        const int b = act ? bucket_of(src[e], N) : N + 1 + lane;  // inactive lanes match nobody
         const unsigned peers = __match_any_sync(0xffffffffu, b);
         if (act) rev_perm[base[b] + __popc(peers & lt)] = e;
         __syncwarp();
@@ -382,10 +385,16 @@ cudaError_t build_reverse_csr(int N, int E, const int32_t* row_ptr, const int32_
         const int nb = (int)((n + kScanChunk - 1) / kScanChunk);
         int32_t* table = static_cast<int32_t*>(ws);
         int32_t* part = reinterpret_cast<int32_t*>(static_cast<char*>(ws) + align16(sizeof(int32_t) * (size_t)n));
-        tile_counts<<<n_tiles, 256, 0, s>>>(src, E, N, n_tiles, table);
+        const size_t count_smem = sizeof(int32_t) * ((size_t)N + 1), scatter_smem = 4 * count_smem;
+        if (scatter_smem > 48 * 1024) {  // above the default limit: opt in (a host-side attribute; cheap)
+            cudaError_t e = cudaFuncSetAttribute(tile_scatter_one_pass, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 (int)scatter_smem);
+            if (e != cudaSuccess) return e;
+        }
+        tile_counts<<<n_tiles, 256, count_smem, s>>>(src, E, N, n_tiles, table);
         scan_chunks<<<nb, 1024, 0, s>>>(table, n, part);
         scan_parts_rev_ptr<<<1, 1024, 0, s>>>(part, nb, table, n_tiles, N, rev_ptr);
-        tile_scatter_one_pass<<<n_tiles, 128, 0, s>>>(src, E, N, n_tiles, table, part, rev_perm);
+        tile_scatter_one_pass<<<n_tiles, 128, scatter_smem, s>>>(src, E, N, n_tiles, table, part, rev_perm);
         if (dst) edge_rows<<<grid_for(E, 256), 256, 0, s>>>(row_ptr, N, E, dst);
         return cudaGetLastError();
     }

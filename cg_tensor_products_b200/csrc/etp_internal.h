@@ -76,7 +76,7 @@ cudaError_t launch_edge_frames(int E, const float* r, float* frames, cudaStream_
 // per-source counts, two key buffers, one value buffer and the digit-major table
 // of per-tile histograms (tiles of kRadixTile edges).
 constexpr int kRadixTile = 1024;
-constexpr int kOnePassMaxNodes = 2048;
+constexpr int kOnePassMaxNodes = 8192;
 constexpr long long kOnePassMaxEntries = 1ll << 22;
 constexpr int kScanChunk = 8192;  // table entries scanned per block
 constexpr size_t align16_bytes(size_t b) { return (b + 15) & ~size_t(15); }

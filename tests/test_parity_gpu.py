@@ -170,7 +170,8 @@ def test_bitwise_repeatable_when_rows_fit_a_task():
 
 @pytest.mark.parametrize("n,e", [(1, 0), (1, 50), (2, 7), (256, 5000), (257, 5000), (70000, 300000),
                                  (3, 10000), (2048, 200000), (2049, 200000), (1024, 131072),
-                                 (1500, 2_200_000)])
+                                 (1500, 2_200_000), (3072, 166518), (8192, 300000), (8193, 300000),
+                                 (4000, 1_000_000), (4000, 1_100_000)])
 def test_reverse_csr_bit_exact(n, e):
     rng = np.random.default_rng(n + e)
     dst = rng.integers(0, n, e)
