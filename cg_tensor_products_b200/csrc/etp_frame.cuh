@@ -821,7 +821,7 @@ __global__ void __launch_bounds__(frame::kThreads, 4) etp_fwd_frame_kernel(FwdAr
 // (cp.async) into lane-owned buffers, refilled for the next edge as soon as this
 // edge has read them. FR: frame records given, as in the forward.
 template <int L, bool O3, int C2T, bool FR>
-__global__ void __launch_bounds__(frame::kThreads, 4) etp_bwd_frame_kernel(BwdArgs a) {
+__global__ void __launch_bounds__(frame::kThreads, L <= 2 ? 6 : 4) etp_bwd_frame_kernel(BwdArgs a) {
     using namespace frame;
     constexpr int D = (L + 1) * (L + 1);
     constexpr int P = PathSet<L, O3>::P;
