@@ -55,6 +55,9 @@ def _load():
         "etp_forward": [vp, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp],
         "etp_backward": [vp, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp],
         "etp_assemble_forces": [i32, i32, vp, vp, vp, vp, vp, vp, vp, vp],
+        "etp_radial_workspace_size": [vp, i32, i32, i32, ctypes.POINTER(sz)],
+        "etp_radial_forward": [vp, i32, i32, i32, ctypes.c_float, vp, vp, vp, vp, vp, sz, vp],
+        "etp_radial_backward": [vp, i32, i32, i32, ctypes.c_float, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp],
         "etp_reverse_csr_workspace_size": [i32, i32, ctypes.POINTER(sz)],
         "etp_build_reverse_csr": [i32, i32, vp, vp, vp, vp, vp, vp, sz, vp],
         "etp_build_reverse_csr_static": [i32, i32, vp, vp, vp, vp, vp, vp],
@@ -261,6 +264,67 @@ def assemble_forces(N: int, row_ptr, rev_ptr, rev_perm, grad_r, r=None, forces=N
                                        _ptr(grad_r), _ptr(forces), _ptr(virial), _stream(stream)),
            "etp_assemble_forces")
     return forces, virial
+
+
+def radial_workspace_size(plan: Plan, E: int, n_basis: int, hidden: int) -> int:
+    b = ctypes.c_size_t()
+    _check(_load().etp_radial_workspace_size(plan.handle, int(E), int(n_basis), int(hidden), ctypes.byref(b)),
+           "etp_radial_workspace_size")
+    return b.value
+
+
+def _radial_ws(plan, E, W1, workspace):
+    import torch
+
+    nbytes = radial_workspace_size(plan, E, W1.shape[0], W1.shape[1])
+    if workspace is None:
+        workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=W1.device)
+    _expect(workspace, "workspace", "uint8", (None,))
+    return workspace
+
+
+def radial_forward(plan: Plan, r, W1, W2, r_cut: float, w=None, workspace=None, stream=None):
+    """w [E, P, C] = SiLU(bessel(|r|) W1) W2 (etp_radial_forward)."""
+    import torch
+
+    _expect(r, "r", "float32", (None, 3))
+    E = r.shape[0]
+    _expect(W1, "W1", "float32", (None, None))
+    _expect(W2, "W2", "float32", (W1.shape[1], plan.n_paths * plan.C))
+    if w is None:
+        w = torch.empty((E, plan.n_paths, plan.C), device=r.device, dtype=torch.float32)
+    _expect(w, "w", "float32", (E, plan.n_paths, plan.C))
+    workspace = _radial_ws(plan, E, W1, workspace)
+    _need_cuda(r, W1, W2, w, workspace)
+    _check(_load().etp_radial_forward(plan.handle, E, W1.shape[0], W1.shape[1], float(r_cut), _ptr(r), _ptr(W1),
+                                      _ptr(W2), _ptr(w), _ptr(workspace), workspace.numel(), _stream(stream)),
+           "etp_radial_forward")
+    return w
+
+
+def radial_backward(plan: Plan, r, W1, W2, r_cut: float, grad_w, grad_r, grad_W1=None, grad_W2=None,
+                    workspace=None, stream=None):
+    """(grad_W1, grad_W2); adds the derivative through |r| to grad_r in place (etp_radial_backward)."""
+    import torch
+
+    _expect(r, "r", "float32", (None, 3))
+    E = r.shape[0]
+    _expect(W1, "W1", "float32", (None, None))
+    _expect(W2, "W2", "float32", (W1.shape[1], plan.n_paths * plan.C))
+    _expect(grad_w, "grad_w", "float32", (E, plan.n_paths, plan.C))
+    _expect(grad_r, "grad_r", "float32", (E, 3))
+    if grad_W1 is None:
+        grad_W1 = torch.empty_like(W1)
+    if grad_W2 is None:
+        grad_W2 = torch.empty_like(W2)
+    _expect(grad_W1, "grad_W1", "float32", tuple(W1.shape))
+    _expect(grad_W2, "grad_W2", "float32", tuple(W2.shape))
+    workspace = _radial_ws(plan, E, W1, workspace)
+    _need_cuda(r, W1, W2, grad_w, grad_r, grad_W1, grad_W2, workspace)
+    _check(_load().etp_radial_backward(plan.handle, E, W1.shape[0], W1.shape[1], float(r_cut), _ptr(r), _ptr(W1),
+                                       _ptr(W2), _ptr(grad_w), _ptr(grad_W1), _ptr(grad_W2), _ptr(grad_r),
+                                       _ptr(workspace), workspace.numel(), _stream(stream)), "etp_radial_backward")
+    return grad_W1, grad_W2
 
 
 def reverse_csr_workspace_size(N: int, E: int) -> int:

@@ -308,6 +308,47 @@ etp_status etp_assemble_forces(int N, int E, const int32_t* row_ptr, const int32
                                             reinterpret_cast<cudaStream_t>(stream)));
 }
 
+namespace {
+bool radial_shape_ok(int n_basis, int hidden, float r_cut) {
+    return n_basis >= 1 && n_basis <= 32 && hidden >= 32 && hidden <= 256 && hidden % 32 == 0 && r_cut > 0.f;
+}
+}  // namespace
+
+etp_status etp_radial_workspace_size(etp_plan_t plan, int E, int n_basis, int hidden, size_t* bytes) {
+    if (!plan || E < 0 || !bytes || !radial_shape_ok(n_basis, hidden, 1.f)) return ETP_ERR_INVALID_ARG;
+    *bytes = etp::radial_workspace_bytes(E, n_basis, hidden, plan->P * plan->C);
+    return ETP_OK;
+}
+
+etp_status etp_radial_forward(etp_plan_t plan, int E, int n_basis, int hidden, float r_cut, const float* r,
+                              const float* W1, const float* W2, float* w, void* workspace, size_t workspace_bytes,
+                              etp_stream_t stream) {
+    if (!plan || E < 0 || !radial_shape_ok(n_basis, hidden, r_cut)) return ETP_ERR_INVALID_ARG;
+    if (E == 0) return ETP_OK;
+    if (!r || !W1 || !W2 || !w || !workspace || !aligned4(r) || !aligned4(W1) || !aligned4(W2) || !aligned16(w) ||
+        !aligned16(workspace))
+        return ETP_ERR_INVALID_ARG;
+    if (workspace_bytes < etp::radial_workspace_bytes(E, n_basis, hidden, plan->P * plan->C)) return ETP_ERR_WORKSPACE;
+    return cuda_status(etp::radial_forward(E, n_basis, hidden, plan->P * plan->C, r_cut, r, W1, W2, w, workspace,
+                                           reinterpret_cast<cudaStream_t>(stream)));
+}
+
+etp_status etp_radial_backward(etp_plan_t plan, int E, int n_basis, int hidden, float r_cut, const float* r,
+                               const float* W1, const float* W2, const float* grad_w, float* grad_W1, float* grad_W2,
+                               float* grad_r, void* workspace, size_t workspace_bytes, etp_stream_t stream) {
+    if (!plan || E < 0 || !radial_shape_ok(n_basis, hidden, r_cut)) return ETP_ERR_INVALID_ARG;
+    if (!W1 || !W2 || !grad_W1 || !grad_W2 || !aligned4(W1) || !aligned4(W2) || !aligned4(grad_W1) ||
+        !aligned4(grad_W2))
+        return ETP_ERR_INVALID_ARG;
+    if (E > 0 && (!r || !grad_w || !grad_r || !workspace || !aligned4(r) || !aligned4(grad_w) || !aligned4(grad_r) ||
+                  !aligned16(workspace)))
+        return ETP_ERR_INVALID_ARG;
+    if (E > 0 && workspace_bytes < etp::radial_workspace_bytes(E, n_basis, hidden, plan->P * plan->C))
+        return ETP_ERR_WORKSPACE;
+    return cuda_status(etp::radial_backward(E, n_basis, hidden, plan->P * plan->C, r_cut, r, W1, W2, grad_w, grad_W1,
+                                            grad_W2, grad_r, workspace, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 etp_status etp_reverse_csr_workspace_size(int N, int E, size_t* bytes) {
     if (N < 0 || E < 0 || !bytes) return ETP_ERR_INVALID_ARG;
     *bytes = etp::reverse_csr_workspace_bytes(N, E);

@@ -101,6 +101,12 @@ size_t reverse_csr_workspace_bytes(int N, int E);
 // radix_workspace_bytes_for).
 cudaError_t build_reverse_csr(int N, int E, const int32_t* row_ptr, const int32_t* src, int32_t* rev_ptr,
                               int32_t* rev_perm, int32_t* dst, void* ws, cudaStream_t s, bool one_pass = true);
+size_t radial_workspace_bytes(int E, int nb, int hidden, int PC);
+cudaError_t radial_forward(int E, int nb, int hidden, int PC, float rc, const float* r, const float* W1,
+                           const float* W2, float* w, void* ws, cudaStream_t s);
+cudaError_t radial_backward(int E, int nb, int hidden, int PC, float rc, const float* r, const float* W1,
+                            const float* W2, const float* grad_w, float* grad_W1, float* grad_W2, float* grad_r,
+                            void* ws, cudaStream_t s);
 cudaError_t assemble_forces(int N, int E, const int32_t* row_ptr, const int32_t* rev_ptr, const int32_t* rev_perm,
                             const float* r, const float* grad_r, float* forces, float* virial, cudaStream_t s);
 cudaError_t validate_csr(int N, int E, const int32_t* row_ptr, const int32_t* src, int32_t* flag, cudaStream_t s);

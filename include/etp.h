@@ -169,6 +169,33 @@ ETP_API etp_status etp_backward(etp_plan_t plan, int N, int E, const int32_t* ro
                         const float* grad_out, float* grad_x, float* grad_w, float* grad_r,
                         etp_stream_t stream);
 
+/* Radial weights: the tensor product's per-edge weights as a function of the edge
+ * length. The pages make these weights a learned function of |r| ("High-performance
+ * training and inference for deep equivariant interatomic potentials", section
+ * "제안 방법": the Allegro tensor product with per-edge weights; the water systems of
+ * section "주요 결과"); this library's plain reading, with d = |r_e|:
+ *   b_n(d) = sqrt(2/r_cut) sin(n pi d / r_cut) / d,  n = 1..n_basis  (b_n(0) = its limit)
+ *   w[e] = SiLU(b(d_e) W1) W2,   SiLU(z) = z / (1 + exp(-z)),   no biases, no envelope,
+ * W1: float32 [n_basis][hidden], W2: float32 [hidden][P*C] (row-major), w: float32
+ * [E][P][C] as etp_forward takes it. 1 <= n_basis <= 32; hidden a multiple of 32 in
+ * [32, 256]; r_cut > 0. The dense products run in FP32 (exact FMAs); every sum over
+ * edges is taken in a fixed order (results repeat bit for bit).
+ * workspace: device memory of etp_radial_workspace_size bytes, 16-byte aligned,
+ * owned by the caller. */
+ETP_API etp_status etp_radial_workspace_size(etp_plan_t plan, int E, int n_basis, int hidden, size_t* bytes);
+ETP_API etp_status etp_radial_forward(etp_plan_t plan, int E, int n_basis, int hidden, float r_cut,
+                                      const float* r, const float* W1, const float* W2, float* w,
+                                      void* workspace, size_t workspace_bytes, etp_stream_t stream);
+/* VJP of etp_radial_forward for grad_w = dL/dw [E][P][C]: overwrites grad_W1 [n_basis][hidden]
+ * and grad_W2 [hidden][P*C], and ADDS the derivative through the edge lengths,
+ * (dL/dd) r / |r|, to grad_r [E][3] (so that grad_r can first hold etp_backward's
+ * derivative through the harmonics; the sum is then the full dL/dr for
+ * etp_assemble_forces). */
+ETP_API etp_status etp_radial_backward(etp_plan_t plan, int E, int n_basis, int hidden, float r_cut,
+                                       const float* r, const float* W1, const float* W2, const float* grad_w,
+                                       float* grad_W1, float* grad_W2, float* grad_r, void* workspace,
+                                       size_t workspace_bytes, etp_stream_t stream);
+
 /* Atom forces and per-atom virials from per-edge energy derivatives.
  * The pages evaluate models on energies and forces ("FlashCart 如何让等变原子间势更快更准?",
  * section "560 万参数模型胜过 1.89 亿参数 transformer"); forces are minus the position

@@ -23,7 +23,7 @@ def lib():
 
 def test_exports_every_declared_symbol(lib):
     names = etp.declared_symbols()
-    assert len(names) == 14
+    assert len(names) == 17
     for n in names:
         assert hasattr(lib, n), n
 
@@ -118,6 +118,18 @@ def test_host_argument_checks(lib):
     assert A(4, 4, ok, ok, None, ok, ok, ok, None, None) == etp.ETP_ERR_INVALID_ARG     # rev_perm NULL
     assert A(4, 4, ok, ok, ok, None, ok, ok, ok, None) == etp.ETP_ERR_INVALID_ARG       # virial without r
     assert A(4, 4, ok, ok, ok, ok, ctypes.c_void_p(0x10002), ok, None, None) == etp.ETP_ERR_INVALID_ARG  # grad_r
+    rw = ctypes.c_size_t()
+    assert lib.etp_radial_workspace_size(h, 100, 8, 64, ctypes.byref(rw)) == etp.ETP_OK and rw.value > 0
+    assert lib.etp_radial_workspace_size(h, 100, 33, 64, ctypes.byref(rw)) == etp.ETP_ERR_INVALID_ARG  # n_basis
+    assert lib.etp_radial_workspace_size(h, 100, 8, 48, ctypes.byref(rw)) == etp.ETP_ERR_INVALID_ARG   # hidden
+    lib.etp_radial_workspace_size(h, 100, 8, 64, ctypes.byref(rw))
+    RF, RB = lib.etp_radial_forward, lib.etp_radial_backward
+    assert RF(h, 100, 8, 64, 0.0, ok, ok, ok, ok, ok, rw.value, None) == etp.ETP_ERR_INVALID_ARG       # r_cut
+    assert RF(h, 100, 8, 64, 5.0, ok, ok, ok, bad, ok, rw.value, None) == etp.ETP_ERR_INVALID_ARG      # w
+    assert RF(h, 100, 8, 64, 5.0, ok, ok, ok, ok, ok, rw.value - 1, None) == etp.ETP_ERR_WORKSPACE
+    assert RF(h, 0, 8, 64, 5.0, None, None, None, None, None, 0, None) == etp.ETP_OK                  # no edges
+    assert RB(h, 100, 8, 64, 5.0, ok, ok, ok, ok, None, ok, ok, ok, rw.value, None) == etp.ETP_ERR_INVALID_ARG
+    assert RB(h, 100, 8, 64, 5.0, ok, ok, ok, ok, ok, ok, ok, ok, rw.value - 1, None) == etp.ETP_ERR_WORKSPACE
     sz = ctypes.c_size_t()
     assert lib.etp_reverse_csr_workspace_size(10, 100, ctypes.byref(sz)) == 0 and sz.value > 0
     assert lib.etp_reverse_csr_workspace_size(-1, 100, ctypes.byref(sz)) == etp.ETP_ERR_INVALID_ARG
