@@ -52,6 +52,9 @@ def parse():
                     help="launch every step's kernels one by one (default: the step is captured once into a CUDA "
                          "graph and the timed region replays it; per-kernel times then come from eager steps run "
                          "outside the timed region)")
+    ap.add_argument("--radial", action="store_true",
+                    help="also time the radial weights (w from |r|: Bessel(8) -> 64 -> SiLU -> P*C) and their VJP, "
+                         "outside the step")
     ap.add_argument("--no-frames", action="store_true",
                     help="kernels build the edge frames themselves (no etp_edge_frames pass)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -455,6 +458,38 @@ def main():
     f_ms = fa.elapsed_time(fb) / 20
     kern["assemble_forces_ms"] = f_ms
     kern["assemble_forces_GBps"] = (40 * E + 48 * N + 8) / (f_ms * 1e6)
+
+    if args.radial:
+        rng = np.random.default_rng(99)
+        nb, hid, rc = 8, 64, 5.0
+        W1 = torch.from_numpy((rng.standard_normal((nb, hid)) / np.sqrt(nb)).astype(np.float32)).to(dev)
+        W2 = torch.from_numpy((rng.standard_normal((hid, plan.n_paths * wl.C)) / np.sqrt(hid)).astype(np.float32)).to(dev)
+        rws = torch.empty(max(etp.radial_workspace_size(plan, E, nb, hid), 16), dtype=torch.uint8, device=dev)
+        w_rad = torch.empty_like(d["w"])
+        gW1, gW2 = torch.empty_like(W1), torch.empty_like(W2)
+        gr_acc = torch.zeros_like(d["r"])
+
+        def rad_f():
+            etp._check(lib.etp_radial_forward(plan.handle, E, nb, hid, rc, P(d["r"]), P(W1), P(W2), P(w_rad), P(rws),
+                                              rws.numel(), sp), "radial forward")
+
+        def rad_b():
+            etp._check(lib.etp_radial_backward(plan.handle, E, nb, hid, rc, P(d["r"]), P(W1), P(W2), P(gw), P(gW1),
+                                               P(gW2), P(gr_acc), P(rws), rws.numel(), sp), "radial backward")
+
+        for fn, key in ((rad_f, "radial_forward_ms"), (rad_b, "radial_backward_ms")):
+            for _ in range(3):
+                fn()
+            ra, rb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            ra.record(stream)
+            for _ in range(10):
+                fn()
+            rb.record(stream)
+            torch.cuda.synchronize()
+            kern[key] = ra.elapsed_time(rb) / 10
+        pc = plan.n_paths * wl.C
+        kern["radial_forward_TFLOPs"] = 2.0 * E * hid * pc / (kern["radial_forward_ms"] * 1e9)
+        kern["radial_backward_TFLOPs"] = 4.0 * E * hid * pc / (kern["radial_backward_ms"] * 1e9)
 
     # the same kernel against the nominal FP32 rate at the clock seen under load (148 SMs x 128 FMA lanes x 2):
     # the method's sparse-CG FLOP count, which the edge-frame schedule undercuts (it executes fewer)
