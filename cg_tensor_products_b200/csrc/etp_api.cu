@@ -381,8 +381,9 @@ etp_status etp_device_fault(int* fault) {
     if (cudaDeviceSynchronize() != cudaSuccess) return ETP_ERR_CUDA;
     const int f0 = etp::read_and_clear_fault<0>(), f1 = etp::read_and_clear_fault<1>();
     const int f2 = etp::read_and_clear_fault<2>(), f3 = etp::read_and_clear_fault<3>();
-    if (f0 < 0 || f1 < 0 || f2 < 0 || f3 < 0) return ETP_ERR_CUDA;
-    *fault = f0 | f1 | f2 | f3;
+    const int f4 = etp::radial_tc_read_and_clear_fault();
+    if (f0 < 0 || f1 < 0 || f2 < 0 || f3 < 0 || f4 < 0) return ETP_ERR_CUDA;
+    *fault = f0 | f1 | f2 | f3 | f4;
     return ETP_OK;
 }
 

@@ -102,6 +102,12 @@ size_t reverse_csr_workspace_bytes(int N, int E);
 cudaError_t build_reverse_csr(int N, int E, const int32_t* row_ptr, const int32_t* src, int32_t* rev_ptr,
                               int32_t* rev_perm, int32_t* dst, void* ws, cudaStream_t s, bool one_pass = true);
 size_t radial_workspace_bytes(int E, int nb, int hidden, int PC);
+// Tensor-core path of the radial forward (hidden width 64, P*C a multiple of 16).
+bool radial_tc_supported(int nb, int hidden, int PC);
+size_t radial_tc_prepare_bytes(int PC);
+cudaError_t radial_tc_forward(int E, int nb, int PC, float rc, const float* r, const float* W1, const float* W2,
+                              float* w, void* ws, cudaStream_t s);
+int radial_tc_read_and_clear_fault();
 cudaError_t radial_forward(int E, int nb, int hidden, int PC, float rc, const float* r, const float* W1,
                            const float* W2, float* w, void* ws, cudaStream_t s);
 cudaError_t radial_backward(int E, int nb, int hidden, int PC, float rc, const float* r, const float* W1,

@@ -9,8 +9,9 @@
 // with SiLU, a linear output layer, no biases.)
 //
 // Layout (row-major): W1 [n_basis][hidden], W2 [hidden][P*C], w / grad_w [E][P*C],
-// hidden activations H [E][hidden]. The dense products run in FP32 on the SIMT
-// pipes (tiled, 64 x 64 outputs per block, exact fp32 FMAs); their reductions over
+// hidden activations H [E][hidden]. The forward with a hidden width of 64 runs on
+// the tensor cores (etp_radial_tc.cu); the other dense products run in FP32 on the
+// SIMT pipes (tiled, 64 x 64 outputs per block, exact fp32 FMAs); their reductions over
 // the edges are split across blocks into partial sums that a second kernel adds
 // in a fixed order, so every result repeats bit for bit.
 #include <cuda_runtime.h>
@@ -210,13 +211,16 @@ cudaError_t gemm(int M, int N, int K, const float* A, int lda, const float* B, i
 size_t radial_workspace_bytes(int E, int nb, int hidden, int PC) {
     const int s2 = edge_splits(E, ((hidden + kTile - 1) / kTile) * ((PC + kTile - 1) / kTile));
     const int s1 = edge_splits(E, ((nb + kTile - 1) / kTile) * ((hidden + kTile - 1) / kTile));
-    return 4 * a16(sizeof(float) * (size_t)E * hidden) + a16(sizeof(float) * (size_t)E * nb) +
-           a16(sizeof(float) * (size_t)s2 * hidden * PC) + a16(sizeof(float) * (size_t)s1 * nb * hidden);
+    const size_t bwd = 4 * a16(sizeof(float) * (size_t)E * hidden) + a16(sizeof(float) * (size_t)E * nb) +
+                       a16(sizeof(float) * (size_t)s2 * hidden * PC) + a16(sizeof(float) * (size_t)s1 * nb * hidden);
+    const size_t fwd_tc = radial_tc_supported(nb, hidden, PC) ? radial_tc_prepare_bytes(PC) : 0;
+    return bwd > fwd_tc ? bwd : fwd_tc;
 }
 
 cudaError_t radial_forward(int E, int nb, int hidden, int PC, float rc, const float* r, const float* W1,
                            const float* W2, float* w, void* ws, cudaStream_t s) {
     if (E == 0) return cudaSuccess;
+    if (radial_tc_supported(nb, hidden, PC)) return radial_tc_forward(E, nb, PC, rc, r, W1, W2, w, ws, s);
     float* H = static_cast<float*>(ws);
     radial_hidden<<<(E + kEdgesPerBlock - 1) / kEdgesPerBlock, 256, sizeof(float) * kEdgesPerBlock * nb, s>>>(
         E, r, W1, nb, hidden, rc, H, nullptr, nullptr);
