@@ -7,7 +7,7 @@
 // whose dropped term A_lo B_lo and rounding of the halves leave a relative error
 // near 2^-21 per product, below the 1e-5 tolerance of the forward.
 //
-// Per CTA (4 warps) and tile of 128 edges:
+// Per CTA (4 warps, one per SM: 225 KB of shared memory) and tile of 128 edges:
 //   1. each thread builds its edge's row of H (Bessel basis, first layer, SiLU),
 //      splits it into TF32 halves and stores both into shared memory in the
 //      tensor core's K-major layout without swizzle: 8-row x 16-byte core matrices,
@@ -100,30 +100,62 @@ __global__ void radial_tc_prepare(const float* __restrict__ W2, int PC, int n_ch
     }
 }
 
+// Shared memory: A halves (64 KB), two B slots of two halves (128 KB), the
+// epilogue stage (128 rows x 68 floats: 16-byte rows whose vector accesses hit
+// all 32 banks once per 8 threads), 4 mbarriers, the TMEM address.
+constexpr int kStageStride = 68;
+constexpr uint32_t kStageFloats = kRows * kStageStride;
+constexpr uint32_t kOffB = 2 * kTileBytes, kOffStage = 6 * kTileBytes;
+constexpr uint32_t kOffBars = kOffStage + kStageFloats * 4;
+constexpr uint32_t kSmemBytes = kOffBars + 64;
+static_assert(kOffBars % 16 == 0 && kSmemBytes <= 232448, "radial tensor-core kernel shared memory");
+
+__device__ __forceinline__ void load_b(const float* Bhi, const float* Blo, int c, unsigned char* slot_hi,
+                                       unsigned char* slot_lo, uint64_t* bar) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(2 * kTileBytes)
+                 : "memory");
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                     smem_u32(slot_hi)),
+                 "l"(Bhi + (size_t)c * (kTileBytes / 4)), "r"(kTileBytes), "r"(smem_u32(bar))
+                 : "memory");
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                     smem_u32(slot_lo)),
+                 "l"(Blo + (size_t)c * (kTileBytes / 4)), "r"(kTileBytes), "r"(smem_u32(bar))
+                 : "memory");
+}
+
+// Two-stage pipeline over the output chunks: while the tensor cores work on chunk
+// c (B slot c % 2, TMEM columns 128 (c % 2)), the warps write chunk c - 1 out and
+// the copy engine brings in chunk c + 1.
 __global__ void __launch_bounds__(kThreads, 1)
     radial_tc_forward(int E, int PC, int nb, float rc, const float* __restrict__ r, const float* __restrict__ W1,
                       const float* __restrict__ Bhi, const float* __restrict__ Blo, float* __restrict__ w) {
     extern __shared__ __align__(1024) unsigned char smem[];
-    // [A_hi 32 KB][A_lo 32 KB][B_hi 32 KB][B_lo 32 KB][2 mbarriers][TMEM address]
     unsigned char* a_hi = smem;
     unsigned char* a_lo = smem + kTileBytes;
-    unsigned char* b_hi = smem + 2 * kTileBytes;
-    unsigned char* b_lo = smem + 3 * kTileBytes;
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + 4 * kTileBytes);
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + 4 * kTileBytes + 16);
+    float* stage = reinterpret_cast<float*>(smem + kOffStage);
+    uint64_t* bar_b = reinterpret_cast<uint64_t*>(smem + kOffBars);       // [2] B slot filled
+    uint64_t* bar_m = bar_b + 2;                                            // [2] accumulator ready
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffBars + 32);
+    int* abort_flag = reinterpret_cast<int*>(smem + kOffBars + 36);
     const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
     const int m0 = blockIdx.x * kRows;
+    const int n_chunks = (PC + kChunk - 1) / kChunk;
+    auto slot_hi = [&](int s) { return smem + kOffB + (uint32_t)s * 2 * kTileBytes; };
+    auto slot_lo = [&](int s) { return smem + kOffB + (uint32_t)s * 2 * kTileBytes + kTileBytes; };
 
-    if (warp == 0) {  // 128 fp32 accumulator columns
+    if (warp == 0) {  // two accumulators of 128 fp32 columns
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
-                     "r"(128)
+                     "r"(256)
                      : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
     if (t == 0) {
-        mbar_init(&bars[0], 1);
-        mbar_init(&bars[1], 1);
+        for (int i = 0; i < 4; ++i) mbar_init(&bar_b[i], 1);
+        *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        load_b(Bhi, Blo, 0, slot_hi(0), slot_lo(0), &bar_b[0]);  // the first two chunks, behind H
+        if (n_chunks > 1) load_b(Bhi, Blo, 1, slot_hi(1), slot_lo(1), &bar_b[1]);
     }
 
     // 1. the tile's rows of H, split into TF32 halves
@@ -156,65 +188,50 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
     const uint32_t tmem = *tmem_slot;
+    int last_committed = -1;  // (thread 0) the last chunk whose MMAs were committed
 
-    const int n_chunks = (PC + kChunk - 1) / kChunk;
-    bool live = true;
-    for (int c = 0; c < n_chunks && live; ++c) {
-        const int n = min(kChunk, PC - c * kChunk);  // a multiple of 16
-        if (t == 0) {
-            asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(&bars[0])),
-                         "r"(2 * kTileBytes)
-                         : "memory");
-            asm volatile(
-                "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-                    smem_u32(b_hi)),
-                "l"(Bhi + (size_t)c * (kTileBytes / 4)), "r"(kTileBytes), "r"(smem_u32(&bars[0]))
-                : "memory");
-            asm volatile(
-                "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-                    smem_u32(b_lo)),
-                "l"(Blo + (size_t)c * (kTileBytes / 4)), "r"(kTileBytes), "r"(smem_u32(&bars[0]))
-                : "memory");
-            if (!mbar_wait(&bars[0], c & 1)) {
-                live = false;
-                mbar_wait(&bars[0], c & 1);  // give the copies in flight one more bounded wait before leaving
+    for (int c = 0; c <= n_chunks; ++c) {
+        // 2. the MMAs of chunk c
+        if (c < n_chunks && t == 0 && !*abort_flag) {
+            const int sb = c & 1;
+            if (!mbar_wait(&bar_b[sb], (c >> 1) & 1)) {
+                *abort_flag = 1;
             } else {
                 asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+                const int n = min(kChunk, PC - c * kChunk);  // a multiple of 16
                 const uint32_t idesc = instr_desc(n);
-                const unsigned char* A[3] = {a_hi, a_hi, a_lo};
-                const unsigned char* B[3] = {b_hi, b_lo, b_hi};
-                int issued = 0;
+                const uint32_t d_tmem = tmem + (uint32_t)sb * 128;
+                const uint32_t A[3] = {smem_u32(a_hi), smem_u32(a_hi), smem_u32(a_lo)};
+                const uint32_t B[3] = {smem_u32(slot_hi(sb)), smem_u32(slot_lo(sb)), smem_u32(slot_hi(sb))};
                 for (int s = 0; s < kHidden / 8; ++s) {
-                    for (int q = 0; q < 3; ++q, ++issued) {
-                        const uint64_t da = smem_desc(smem_u32(A[q]) + s * 2 * kLBO);
-                        const uint64_t db = smem_desc(smem_u32(B[q]) + s * 2 * kLBO);
-                        const uint32_t acc = issued > 0 ? 1u : 0u;
+                    for (int q = 0; q < 3; ++q) {
+                        const uint64_t da = smem_desc(A[q] + s * 2 * kLBO);
+                        const uint64_t db = smem_desc(B[q] + s * 2 * kLBO);
+                        const uint32_t acc = (s | q) ? 1u : 0u;
                         asm volatile(
                             "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
-                            " tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n}" ::"r"(tmem),
+                            " tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n}" ::"r"(d_tmem),
                             "l"(da), "l"(db), "r"(idesc), "r"(acc)
                             : "memory");
                     }
                 }
                 asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                                 smem_u32(&bars[1]))
+                                 smem_u32(&bar_m[sb]))
                              : "memory");
+                last_committed = c;
             }
         }
-        // everyone: the accumulator of this chunk
-        live = __syncthreads_and(live ? 1 : 0) != 0;
-        if (!live) break;
-        if (!mbar_wait(&bars[1], c & 1)) {
-            live = false;
-            mbar_wait(&bars[1], c & 1);  // the MMAs write TMEM: wait once more before it is freed
-        }
-        live = __syncthreads_and(live ? 1 : 0) != 0;
-        if (!live) break;
+        if (c == 0) continue;
+        // 3. chunk c - 1: wait for its accumulator, refill its B slot, write it out
+        const int cp = c - 1, sp = cp & 1;
+        __syncthreads();
+        if (*abort_flag) break;
+        if (!mbar_wait(&bar_m[sp], (cp >> 1) & 1)) atomicOr(abort_flag, 1);
+        __syncthreads();
+        if (*abort_flag) break;
+        if (t == 0 && cp + 2 < n_chunks) load_b(Bhi, Blo, cp + 2, slot_hi(sp), slot_lo(sp), &bar_b[sp]);
         asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-        // 3. epilogue through shared memory (the B buffers are free once the MMAs are
-        // done): each half of the chunk (64 columns) is staged row by row with a
-        // 65-float stride (conflict-free), then each warp stores whole row segments.
-        float* stage = reinterpret_cast<float*>(b_hi);
+        const int n = min(kChunk, PC - cp * kChunk);
         for (int h0 = 0; h0 < n; h0 += 64) {
             const int hn = min(64, n - h0);
             for (int j = 0; j < hn; j += 16) {
@@ -225,29 +242,37 @@ __global__ void __launch_bounds__(kThreads, 1)
                     : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
                       "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]),
                       "=r"(v[15])
-                    : "r"(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(h0 + j)));
+                    : "r"(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(sp * 128 + h0 + j)));
                 asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
-                for (int q = 0; q < 16; ++q) stage[t * 65 + j + q] = __uint_as_float(v[q]);
+                for (int q = 0; q < 4; ++q)
+                    *reinterpret_cast<float4*>(stage + t * kStageStride + j + 4 * q) =
+                        make_float4(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1]),
+                                    __uint_as_float(v[4 * q + 2]), __uint_as_float(v[4 * q + 3]));
             }
             __syncthreads();
-            for (int rr = 0; rr < 32; ++rr) {
-                const int row = warp * 32 + rr, e = m0 + row;
-                if (e < E && 2 * lane < hn) {
-                    const float2 val = make_float2(stage[row * 65 + 2 * lane], stage[row * 65 + 2 * lane + 1]);
-                    *reinterpret_cast<float2*>(w + (size_t)e * PC + c * kChunk + h0 + 2 * lane) = val;
-                }
+            // each half-warp stores one 64-float row segment per step: 16 lanes x 16 bytes
+            const int col = (lane & 15) * 4;
+            for (int rr = 0; rr < 32; rr += 2) {
+                const int row = warp * 32 + rr + (lane >> 4), e = m0 + row;
+                if (e < E && col < hn)
+                    *reinterpret_cast<float4*>(w + (size_t)e * PC + cp * kChunk + h0 + col) =
+                        *reinterpret_cast<const float4*>(stage + row * kStageStride + col);
             }
             __syncthreads();
         }
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // staging reads before the next bulk copy
-        asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-        __syncthreads();  // accumulator and B buffers free for the next chunk
+        asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");  // accumulator sp free for chunk c + 1
     }
-    if (!live && t == 0) atomicOr(&g_fault, 1);
+    __syncthreads();
+    if (t == 0 && *abort_flag) {
+        atomicOr(&g_fault, 1);
+        // leave nothing in flight on the freed TMEM and shared memory: one more bounded wait each
+        if (last_committed >= 0) mbar_wait(&bar_m[last_committed & 1], (last_committed >> 1) & 1);
+        for (int s2 = 0; s2 < 2 && s2 < n_chunks; ++s2) mbar_wait(&bar_b[s2], 0);
+    }
     __syncthreads();
     if (warp == 0)
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(128) : "memory");
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(256) : "memory");
 }
 
 }  // namespace rtc
@@ -266,7 +291,7 @@ cudaError_t radial_tc_forward(int E, int nb, int PC, float rc, const float* r, c
     float* hi = static_cast<float*>(ws);
     float* lo = hi + (size_t)n_chunks * (rtc::kTileBytes / 4);
     rtc::radial_tc_prepare<<<256, 256, 0, s>>>(W2, PC, n_chunks, hi, lo);
-    const size_t smem = 4 * (size_t)rtc::kTileBytes + 64;
+    const size_t smem = rtc::kSmemBytes;
     cudaError_t err = cudaFuncSetAttribute(rtc::radial_tc_forward, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                            (int)smem);
     if (err != cudaSuccess) return err;
