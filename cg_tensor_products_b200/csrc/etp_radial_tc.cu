@@ -30,6 +30,7 @@ namespace etp {
 namespace rtc {
 
 constexpr int kRows = 128;                    // edges per tile (MMA M)
+constexpr int kBasis = 8;                     // Bessel functions (compile-time: registers, unrolled)
 constexpr int kHidden = 64;                   // K of the product (the hidden width)
 constexpr int kChunk = 128;                   // output columns per MMA group (N)
 constexpr int kThreads = 128;
@@ -158,24 +159,32 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (n_chunks > 1) load_b(Bhi, Blo, 1, slot_hi(1), slot_lo(1), &bar_b[1]);
     }
 
-    // 1. the tile's rows of H, split into TF32 halves
+    // 1. the tile's rows of H, split into TF32 halves (W1 read from the epilogue
+    // stage, which is free until the first chunk is written out)
+    for (int i = t; i < kBasis * kHidden; i += kThreads) stage[i] = __ldg(W1 + i);
+    __syncthreads();
     {
         const int e = m0 + t;
-        float b[32];
+        float b[kBasis];
+#pragma unroll
+        for (int n = 0; n < kBasis; ++n) b[n] = 0.f;
         if (e < E) {
             const float x = __ldg(r + 3 * (size_t)e), y = __ldg(r + 3 * (size_t)e + 1), z = __ldg(r + 3 * (size_t)e + 2);
             const float d = sqrtf(x * x + y * y + z * z);
             const float c = sqrtf(2.f / rc);
-            for (int n = 0; n < nb; ++n) {
+#pragma unroll
+            for (int n = 0; n < kBasis; ++n) {
                 const float k = (float)(n + 1) * kPi / rc;
                 b[n] = d >= 1e-12f ? c * sinf(k * d) / d : c * k;
             }
         }
+#pragma unroll 4
         for (int k = 0; k < kHidden; ++k) {
             float h = 0.f;
             if (e < E) {
                 float zz = 0.f;
-                for (int n = 0; n < nb; ++n) zz = fmaf(b[n], __ldg(W1 + n * kHidden + k), zz);
+#pragma unroll
+                for (int n = 0; n < kBasis; ++n) zz = fmaf(b[n], stage[n * kHidden + k], zz);
                 h = zz / (1.f + expf(-zz));
             }
             const float hh = tf32_round(h);
@@ -234,22 +243,26 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int n = min(kChunk, PC - cp * kChunk);
         for (int h0 = 0; h0 < n; h0 += 64) {
             const int hn = min(64, n - h0);
-            for (int j = 0; j < hn; j += 16) {
-                uint32_t v[16];
-                asm volatile(
-                    "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, "
-                    "%13, %14, %15}, [%16];"
-                    : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
-                      "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]),
-                      "=r"(v[15])
-                    : "r"(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(sp * 128 + h0 + j)));
-                asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+            uint32_t v[64];  // this thread's row of the half-chunk: all loads in flight, one wait
 #pragma unroll
-                for (int q = 0; q < 4; ++q)
-                    *reinterpret_cast<float4*>(stage + t * kStageStride + j + 4 * q) =
+            for (int jj = 0; jj < 4; ++jj) {
+                if (jj * 16 < hn)
+                    asm volatile(
+                        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
+                        "%12, %13, %14, %15}, [%16];"
+                        : "=r"(v[16 * jj]), "=r"(v[16 * jj + 1]), "=r"(v[16 * jj + 2]), "=r"(v[16 * jj + 3]),
+                          "=r"(v[16 * jj + 4]), "=r"(v[16 * jj + 5]), "=r"(v[16 * jj + 6]), "=r"(v[16 * jj + 7]),
+                          "=r"(v[16 * jj + 8]), "=r"(v[16 * jj + 9]), "=r"(v[16 * jj + 10]), "=r"(v[16 * jj + 11]),
+                          "=r"(v[16 * jj + 12]), "=r"(v[16 * jj + 13]), "=r"(v[16 * jj + 14]), "=r"(v[16 * jj + 15])
+                        : "r"(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(sp * 128 + h0 + 16 * jj)));
+            }
+            asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+            for (int q = 0; q < 16; ++q)
+                if (q * 4 < hn)
+                    *reinterpret_cast<float4*>(stage + t * kStageStride + 4 * q) =
                         make_float4(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1]),
                                     __uint_as_float(v[4 * q + 2]), __uint_as_float(v[4 * q + 3]));
-            }
             __syncthreads();
             // each half-warp stores one 64-float row segment per step: 16 lanes x 16 bytes
             const int col = (lane & 15) * 4;
@@ -282,7 +295,9 @@ size_t radial_tc_prepare_bytes(int PC) {
     return 2 * (size_t)n_chunks * rtc::kTileBytes;
 }
 
-bool radial_tc_supported(int nb, int hidden, int PC) { return hidden == rtc::kHidden && nb <= 32 && PC % 16 == 0; }
+bool radial_tc_supported(int nb, int hidden, int PC) {
+    return hidden == rtc::kHidden && nb == rtc::kBasis && PC % 16 == 0;
+}
 
 cudaError_t radial_tc_forward(int E, int nb, int PC, float rc, const float* r, const float* W1, const float* W2,
                               float* w, void* ws, cudaStream_t s) {
