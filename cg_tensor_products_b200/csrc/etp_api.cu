@@ -340,7 +340,7 @@ etp_status etp_radial_backward(etp_plan_t plan, int E, int n_basis, int hidden, 
     if (!W1 || !W2 || !grad_W1 || !grad_W2 || !aligned4(W1) || !aligned4(W2) || !aligned4(grad_W1) ||
         !aligned4(grad_W2))
         return ETP_ERR_INVALID_ARG;
-    if (E > 0 && (!r || !grad_w || !grad_r || !workspace || !aligned4(r) || !aligned4(grad_w) || !aligned4(grad_r) ||
+    if (E > 0 && (!r || !grad_w || !grad_r || !workspace || !aligned4(r) || !aligned16(grad_w) || !aligned4(grad_r) ||
                   !aligned16(workspace)))
         return ETP_ERR_INVALID_ARG;
     if (E > 0 && workspace_bytes < etp::radial_workspace_bytes(E, n_basis, hidden, plan->P * plan->C))

@@ -107,6 +107,9 @@ bool radial_tc_supported(int nb, int hidden, int PC);
 size_t radial_tc_prepare_bytes(int PC);
 cudaError_t radial_tc_forward(int E, int nb, int PC, float rc, const float* r, const float* W1, const float* W2,
                               float* w, void* ws, cudaStream_t s);
+size_t radial_tc_backward_prepare_bytes(int PC);
+cudaError_t radial_tc_backward(int E, int PC, float rc, const float* r, const float* W1, const float* W2,
+                               const float* grad_w, float* gZ, float* grad_r, void* prep, cudaStream_t s);
 int radial_tc_read_and_clear_fault();
 cudaError_t radial_forward(int E, int nb, int hidden, int PC, float rc, const float* r, const float* W1,
                            const float* W2, float* w, void* ws, cudaStream_t s);

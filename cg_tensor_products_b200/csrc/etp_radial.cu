@@ -213,8 +213,10 @@ size_t radial_workspace_bytes(int E, int nb, int hidden, int PC) {
     const int s1 = edge_splits(E, ((nb + kTile - 1) / kTile) * ((hidden + kTile - 1) / kTile));
     const size_t bwd = 4 * a16(sizeof(float) * (size_t)E * hidden) + a16(sizeof(float) * (size_t)E * nb) +
                        a16(sizeof(float) * (size_t)s2 * hidden * PC) + a16(sizeof(float) * (size_t)s1 * nb * hidden);
-    const size_t fwd_tc = radial_tc_supported(nb, hidden, PC) ? radial_tc_prepare_bytes(PC) : 0;
-    return bwd > fwd_tc ? bwd : fwd_tc;
+    const bool tc = radial_tc_supported(nb, hidden, PC);
+    const size_t bwd_all = bwd + (tc ? a16(radial_tc_backward_prepare_bytes(PC)) : 0);
+    const size_t fwd_tc = tc ? radial_tc_prepare_bytes(PC) : 0;
+    return bwd_all > fwd_tc ? bwd_all : fwd_tc;
 }
 
 cudaError_t radial_forward(int E, int nb, int hidden, int PC, float rc, const float* r, const float* W1,
@@ -252,11 +254,17 @@ cudaError_t radial_backward(int E, int nb, int hidden, int PC, float rc, const f
         if ((err = cudaMemsetAsync(grad_W1, 0, sizeof(float) * nb * hidden, s)) != cudaSuccess) return err;
         return cudaMemsetAsync(grad_W2, 0, sizeof(float) * (size_t)hidden * PC, s);
     }
+    const bool tc = radial_tc_supported(nb, hidden, PC);
     radial_hidden<<<(E + kEdgesPerBlock - 1) / kEdgesPerBlock, 256, sizeof(float) * kEdgesPerBlock * nb, s>>>(
-        E, r, W1, nb, hidden, rc, H, Z, Bm);
-    // dL/dH [E][hidden] = grad_w [E][PC] W2^T
-    if ((err = gemm<false, true>(E, hidden, PC, grad_w, PC, W2, PC, gH, 1, s)) != cudaSuccess) return err;
-    radial_edge_backward<<<E, hidden, 0, s>>>(E, r, W1, nb, hidden, rc, Z, gH, gZ, grad_r);
+        E, r, W1, nb, hidden, rc, H, tc ? nullptr : Z, Bm);
+    if (tc) {  // dL/dH on the tensor cores, with dL/dz, dL/dd and grad_r fused into its epilogue
+        p += a16(sizeof(float) * (size_t)s1 * nb * hidden);
+        if ((err = radial_tc_backward(E, PC, rc, r, W1, W2, grad_w, gZ, grad_r, p, s)) != cudaSuccess) return err;
+    } else {
+        // dL/dH [E][hidden] = grad_w [E][PC] W2^T
+        if ((err = gemm<false, true>(E, hidden, PC, grad_w, PC, W2, PC, gH, 1, s)) != cudaSuccess) return err;
+        radial_edge_backward<<<E, hidden, 0, s>>>(E, r, W1, nb, hidden, rc, Z, gH, gZ, grad_r);
+    }
     // grad_W2 [hidden][PC] = H^T grad_w, grad_W1 [nb][hidden] = B^T dL/dz: reductions over the edges
     if ((err = gemm<true, false>(hidden, PC, E, H, hidden, grad_w, PC, part2, s2, s)) != cudaSuccess) return err;
     sum_splits<<<256, 256, 0, s>>>(part2, s2, (long long)hidden * PC, grad_W2);

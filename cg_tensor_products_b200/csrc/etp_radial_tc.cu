@@ -288,6 +288,220 @@ __global__ void __launch_bounds__(kThreads, 1)
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(256) : "memory");
 }
 
+// ---------------------------------------------------------------------------
+// Backward: dL/dH [E][64] = grad_w [E][PC] W2^T on the tensor cores (M = 128 edges,
+// N = 64 hidden units, K = PC in chunks of 64), with the per-edge rest of the VJP
+// fused into the epilogue: dL/dz = dL/dH * SiLU'(z) (written out for grad_W1),
+// dL/db = dL/dz W1^T, dL/dd = dL/db . db/dd and grad_r[e] += dL/dd r / |r|.
+// grad_w chunks are split into TF32 halves by the threads into one of two A slots
+// while the tensor cores multiply the other; W2 chunks (64 rows x 64 K, halves
+// pre-split) arrive by bulk copies into two B slots.
+constexpr int kKChunk = 64;
+constexpr uint32_t kBwTileB = 64 * kKChunk * 4;                 // 16 KB: one half of a W2 chunk
+constexpr uint32_t kBwOffB = 4 * kTileBytes;                    // after the two A slots (2 x 64 KB)
+constexpr uint32_t kBwOffW1 = kBwOffB + 4 * kBwTileB;           // after the two B slots (2 x 32 KB)
+constexpr uint32_t kBwOffBars = kBwOffW1 + kBasis * kHidden * 4;
+constexpr uint32_t kBwSmem = kBwOffBars + 64;
+static_assert(kBwSmem <= 232448 && kBwOffBars % 16 == 0, "radial backward shared memory");
+
+// W2 [64][PC] as K-major B chunks: chunk q holds rows h = 0..63, K = columns 64q..64q+63.
+__global__ void radial_tc_prepare_w2(const float* __restrict__ W2, int PC, int n_kc, float* __restrict__ hi,
+                                     float* __restrict__ lo) {
+    const long long total = (long long)n_kc * kHidden * kKChunk;
+    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total;
+         i += (long long)gridDim.x * blockDim.x) {
+        const int q = (int)(i / (kHidden * kKChunk)), rem = (int)(i % (kHidden * kKChunk));
+        const int h = rem / kKChunk, k = rem % kKChunk, col = q * kKChunk + k;
+        const float v = col < PC ? W2[(size_t)h * PC + col] : 0.f;
+        const float vh = tf32_round(v);
+        const size_t off = (size_t)q * (kBwTileB / 4) + tile_offset(h, k) / 4;
+        hi[off] = vh;
+        lo[off] = tf32_round(v - vh);
+    }
+}
+
+__device__ __forceinline__ void load_w2(const float* Bhi, const float* Blo, int q, unsigned char* dst_hi,
+                                        unsigned char* dst_lo, uint64_t* bar) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(2 * kBwTileB)
+                 : "memory");
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                     smem_u32(dst_hi)),
+                 "l"(Bhi + (size_t)q * (kBwTileB / 4)), "r"(kBwTileB), "r"(smem_u32(bar))
+                 : "memory");
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                     smem_u32(dst_lo)),
+                 "l"(Blo + (size_t)q * (kBwTileB / 4)), "r"(kBwTileB), "r"(smem_u32(bar))
+                 : "memory");
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    radial_tc_backward(int E, int PC, float rc, const float* __restrict__ r, const float* __restrict__ W1,
+                       const float* __restrict__ Bhi, const float* __restrict__ Blo,
+                       const float* __restrict__ grad_w, float* __restrict__ gZ, float* __restrict__ grad_r) {
+    extern __shared__ __align__(1024) unsigned char smem[];
+    float* w1s = reinterpret_cast<float*>(smem + kBwOffW1);
+    uint64_t* bar_b = reinterpret_cast<uint64_t*>(smem + kBwOffBars);  // [2] W2 chunk arrived
+    uint64_t* bar_m = bar_b + 2;                                         // [2] MMAs of a slot done
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kBwOffBars + 32);
+    int* abort_flag = reinterpret_cast<int*>(smem + kBwOffBars + 36);
+    const int t = threadIdx.x, warp = t >> 5;
+    const int m0 = blockIdx.x * kRows, e = m0 + t;
+    const int n_kc = (PC + kKChunk - 1) / kKChunk;
+    auto a_hi = [&](int s) { return smem + (uint32_t)s * 2 * kTileBytes; };
+    auto a_lo = [&](int s) { return smem + (uint32_t)s * 2 * kTileBytes + kTileBytes; };
+    auto b_hi = [&](int s) { return smem + kBwOffB + (uint32_t)s * 2 * kBwTileB; };
+    auto b_lo = [&](int s) { return smem + kBwOffB + (uint32_t)s * 2 * kBwTileB + kBwTileB; };
+
+    if (warp == 0) {  // 64 fp32 accumulator columns (dL/dH of the tile)
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                     "r"(64)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    for (int i = t; i < kBasis * kHidden; i += kThreads) w1s[i] = __ldg(W1 + i);
+    if (t == 0) {
+        for (int i = 0; i < 4; ++i) mbar_init(&bar_b[i], 1);
+        *abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        load_w2(Bhi, Blo, 0, b_hi(0), b_lo(0), &bar_b[0]);
+        if (n_kc > 1) load_w2(Bhi, Blo, 1, b_hi(1), b_lo(1), &bar_b[1]);
+    }
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+    __syncthreads();
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+    const uint32_t tmem = *tmem_slot;
+    int last = -1;
+
+    for (int q = 0; q < n_kc; ++q) {
+        const int sa = q & 1;
+        if (q >= 2) {  // slot sa was read by the MMAs of chunk q - 2
+            if (!mbar_wait(&bar_m[sa], ((q - 2) >> 1) & 1)) atomicOr(abort_flag, 1);
+            __syncthreads();
+            if (*abort_flag) break;
+            if (t == 0) load_w2(Bhi, Blo, q, b_hi(sa), b_lo(sa), &bar_b[sa]);
+        }
+        // this thread's edge row of the grad_w chunk, split into TF32 halves
+        const int c0 = q * kKChunk;
+#pragma unroll 4
+        for (int k4 = 0; k4 < kKChunk; k4 += 4) {
+            float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (e < E && c0 + k4 < PC) v = __ldg(reinterpret_cast<const float4*>(grad_w + (size_t)e * PC + c0 + k4));
+            const float vv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const float h = tf32_round(vv[j]);
+                *reinterpret_cast<float*>(a_hi(sa) + tile_offset(t, k4 + j)) = h;
+                *reinterpret_cast<float*>(a_lo(sa) + tile_offset(t, k4 + j)) = tf32_round(vv[j] - h);
+            }
+        }
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+        __syncthreads();
+        if (t == 0 && !*abort_flag) {
+            if (!mbar_wait(&bar_b[sa], (q >> 1) & 1)) {
+                *abort_flag = 1;
+            } else {
+                asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+                const uint32_t idesc = instr_desc(kHidden);  // N = 64
+                const uint32_t A[3] = {smem_u32(a_hi(sa)), smem_u32(a_hi(sa)), smem_u32(a_lo(sa))};
+                const uint32_t B[3] = {smem_u32(b_hi(sa)), smem_u32(b_lo(sa)), smem_u32(b_hi(sa))};
+                for (int s = 0; s < kKChunk / 8; ++s) {
+                    for (int p = 0; p < 3; ++p) {
+                        const uint64_t da = smem_desc(A[p] + s * 2 * kLBO);
+                        const uint64_t db = smem_desc(B[p] + s * 2 * kLBO);
+                        const uint32_t acc = (q | s | p) ? 1u : 0u;
+                        asm volatile(
+                            "{\n .reg .pred pp;\n setp.ne.b32 pp, %4, 0;\n"
+                            " tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, pp;\n}" ::"r"(tmem),
+                            "l"(da), "l"(db), "r"(idesc), "r"(acc)
+                            : "memory");
+                    }
+                }
+                asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                                 smem_u32(&bar_m[sa]))
+                             : "memory");
+                last = q;
+            }
+        }
+        __syncthreads();
+        if (*abort_flag) break;
+    }
+    // the accumulator is complete once the last chunk's MMAs are
+    if (!*abort_flag && n_kc > 0 && !mbar_wait(&bar_m[(n_kc - 1) & 1], ((n_kc - 1) >> 1) & 1)) atomicOr(abort_flag, 1);
+    __syncthreads();
+    if (!*abort_flag) {
+        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+        uint32_t g[64];
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj)
+            asm volatile(
+                "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
+                "%14, %15}, [%16];"
+                : "=r"(g[16 * jj]), "=r"(g[16 * jj + 1]), "=r"(g[16 * jj + 2]), "=r"(g[16 * jj + 3]),
+                  "=r"(g[16 * jj + 4]), "=r"(g[16 * jj + 5]), "=r"(g[16 * jj + 6]), "=r"(g[16 * jj + 7]),
+                  "=r"(g[16 * jj + 8]), "=r"(g[16 * jj + 9]), "=r"(g[16 * jj + 10]), "=r"(g[16 * jj + 11]),
+                  "=r"(g[16 * jj + 12]), "=r"(g[16 * jj + 13]), "=r"(g[16 * jj + 14]), "=r"(g[16 * jj + 15])
+                : "r"(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(16 * jj)));
+        asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+        if (e < E) {
+            const float x = __ldg(r + 3 * (size_t)e), y = __ldg(r + 3 * (size_t)e + 1), z = __ldg(r + 3 * (size_t)e + 2);
+            const float d = sqrtf(x * x + y * y + z * z);
+            const float c = sqrtf(2.f / rc);
+            float b[kBasis], db[kBasis], gb[kBasis];
+#pragma unroll
+            for (int n = 0; n < kBasis; ++n) {
+                const float kk = (float)(n + 1) * kPi / rc;
+                gb[n] = 0.f;
+                if (d >= 1e-12f) {
+                    float sn, cs;
+                    sincosf(kk * d, &sn, &cs);
+                    b[n] = c * sn / d;
+                    db[n] = c * (kk * cs / d - sn / (d * d));
+                } else {
+                    b[n] = c * kk;
+                    db[n] = 0.f;
+                }
+            }
+            float4* gz_row = reinterpret_cast<float4*>(gZ + (size_t)e * kHidden);
+#pragma unroll
+            for (int k4 = 0; k4 < kHidden; k4 += 4) {
+                float out[4];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const int k = k4 + j;
+                    float zz = 0.f;
+#pragma unroll
+                    for (int n = 0; n < kBasis; ++n) zz = fmaf(b[n], w1s[n * kHidden + k], zz);
+                    const float sg = 1.f / (1.f + expf(-zz));
+                    const float gz = __uint_as_float(g[k]) * (sg * (1.f + zz * (1.f - sg)));
+                    out[j] = gz;
+#pragma unroll
+                    for (int n = 0; n < kBasis; ++n) gb[n] = fmaf(gz, w1s[n * kHidden + k], gb[n]);
+                }
+                gz_row[k4 / 4] = make_float4(out[0], out[1], out[2], out[3]);
+            }
+            float dd = 0.f;
+#pragma unroll
+            for (int n = 0; n < kBasis; ++n) dd = fmaf(gb[n], db[n], dd);
+            if (d >= 1e-12f) {
+                const float f = dd / d;
+                grad_r[3 * (size_t)e] += f * x;
+                grad_r[3 * (size_t)e + 1] += f * y;
+                grad_r[3 * (size_t)e + 2] += f * z;
+            }
+        }
+    }
+    __syncthreads();
+    if (t == 0 && *abort_flag) {
+        atomicOr(&g_fault, 1);
+        if (last >= 0) mbar_wait(&bar_m[last & 1], (last >> 1) & 1);  // nothing left in flight on freed TMEM
+    }
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+    __syncthreads();
+    if (warp == 0)
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(64) : "memory");
+}
+
 }  // namespace rtc
 
 size_t radial_tc_prepare_bytes(int PC) {
@@ -312,6 +526,26 @@ cudaError_t radial_tc_forward(int E, int nb, int PC, float rc, const float* r, c
     if (err != cudaSuccess) return err;
     rtc::radial_tc_forward<<<(E + rtc::kRows - 1) / rtc::kRows, rtc::kThreads, smem, s>>>(E, PC, nb, rc, r, W1, hi, lo,
                                                                                          w);
+    return cudaGetLastError();
+}
+
+size_t radial_tc_backward_prepare_bytes(int PC) {
+    const int n_kc = (PC + rtc::kKChunk - 1) / rtc::kKChunk;
+    return 2 * (size_t)n_kc * rtc::kBwTileB;
+}
+
+cudaError_t radial_tc_backward(int E, int PC, float rc, const float* r, const float* W1, const float* W2,
+                               const float* grad_w, float* gZ, float* grad_r, void* prep, cudaStream_t s) {
+    if (E == 0) return cudaSuccess;
+    const int n_kc = (PC + rtc::kKChunk - 1) / rtc::kKChunk;
+    float* hi = static_cast<float*>(prep);
+    float* lo = hi + (size_t)n_kc * (rtc::kBwTileB / 4);
+    rtc::radial_tc_prepare_w2<<<256, 256, 0, s>>>(W2, PC, n_kc, hi, lo);
+    cudaError_t err = cudaFuncSetAttribute(rtc::radial_tc_backward, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           (int)rtc::kBwSmem);
+    if (err != cudaSuccess) return err;
+    rtc::radial_tc_backward<<<(E + rtc::kRows - 1) / rtc::kRows, rtc::kThreads, rtc::kBwSmem, s>>>(
+        E, PC, rc, r, W1, hi, lo, grad_w, gZ, grad_r);
     return cudaGetLastError();
 }
 

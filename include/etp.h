@@ -186,7 +186,7 @@ ETP_API etp_status etp_radial_workspace_size(etp_plan_t plan, int E, int n_basis
 ETP_API etp_status etp_radial_forward(etp_plan_t plan, int E, int n_basis, int hidden, float r_cut,
                                       const float* r, const float* W1, const float* W2, float* w,
                                       void* workspace, size_t workspace_bytes, etp_stream_t stream);
-/* VJP of etp_radial_forward for grad_w = dL/dw [E][P][C]: overwrites grad_W1 [n_basis][hidden]
+/* VJP of etp_radial_forward for grad_w = dL/dw [E][P][C] (16-byte aligned): overwrites grad_W1 [n_basis][hidden]
  * and grad_W2 [hidden][P*C], and ADDS the derivative through the edge lengths,
  * (dL/dd) r / |r|, to grad_r [E][3] (so that grad_r can first hold etp_backward's
  * derivative through the harmonics; the sum is then the full dL/dr for
