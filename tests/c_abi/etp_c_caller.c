@@ -5,8 +5,9 @@
  *   etp_c_caller run IN OUT         reads a problem from IN (binary, see read_problem),
  *                                   allocates device memory with the CUDA runtime, builds
  *                                   the reverse CSR and the edge frames, runs the forward
- *                                   and the VJP, and writes out, grad_x, grad_w, grad_r,
- *                                   rev_ptr and rev_perm to OUT.
+ *                                   and the VJP, assembles forces from grad_r, and writes
+ *                                   out, grad_x, grad_w, grad_r, rev_ptr, rev_perm and
+ *                                   forces to OUT.
  * Exit status 0 on success; a message on stderr otherwise. Test infrastructure. */
 #include <stdint.h>
 #include <stdio.h>
@@ -117,7 +118,7 @@ static int run(const char* in, const char* out_path) {
     float* d_w = dev_copy(pr.w, 4 * ew);
     float* d_g = dev_copy(pr.g, 4 * nd);
     CHECK(d_row_ptr && d_src && d_r && d_x && d_w && d_g, "device inputs");
-    float *d_out, *d_gx, *d_gw, *d_gr, *d_frames;
+    float *d_out, *d_gx, *d_gw, *d_gr, *d_frames, *d_forces;
     int32_t *d_rev_ptr, *d_rev_perm, *d_dst, *d_flag;
     void* d_ws;
     size_t ws_bytes = 0;
@@ -131,6 +132,7 @@ static int run(const char* in, const char* out_path) {
     CUDA(cudaMalloc((void**)&d_rev_perm, 4 * (size_t)E + 16));
     CUDA(cudaMalloc((void**)&d_dst, 4 * (size_t)E + 16));
     CUDA(cudaMalloc((void**)&d_flag, 4));
+    CUDA(cudaMalloc((void**)&d_forces, 12 * (size_t)N));
     CUDA(cudaMalloc(&d_ws, ws_bytes + 16));
     cudaStream_t s;
     CUDA(cudaStreamCreate(&s));
@@ -141,6 +143,7 @@ static int run(const char* in, const char* out_path) {
     ETP(etp_forward(plan, N, E, d_row_ptr, d_src, NULL, d_frames, d_x, d_w, d_out, es));
     ETP(etp_backward(plan, N, E, d_row_ptr, d_src, d_rev_ptr, d_rev_perm, d_dst, NULL, d_frames, d_x, d_w, d_g,
                      d_gx, d_gw, d_gr, es));
+    ETP(etp_assemble_forces(N, E, d_row_ptr, d_rev_ptr, d_rev_perm, NULL, d_gr, d_forces, NULL, es));
     CUDA(cudaStreamSynchronize(s));
     int flag = -1, fault = -1;
     CUDA(cudaMemcpy(&flag, d_flag, 4, cudaMemcpyDeviceToHost));
@@ -164,6 +167,8 @@ static int run(const char* in, const char* out_path) {
     fwrite(hi, 4, (size_t)N + 1, f);
     CUDA(cudaMemcpy(hi, d_rev_perm, 4 * (size_t)E, cudaMemcpyDeviceToHost));
     fwrite(hi, 4, (size_t)E, f);
+    CUDA(cudaMemcpy(h, d_forces, 12 * (size_t)N, cudaMemcpyDeviceToHost));
+    fwrite(h, 4, 3 * (size_t)N, f);
     fclose(f);
     cudaStreamDestroy(s);
     ETP(etp_plan_destroy(plan));

@@ -72,6 +72,7 @@ def test_c_caller_matches_oracle(caller, tmp_path, L, o3, C):
     gw = take(wl.E * P * C, np.float32).reshape(wl.E, P, C)
     gr = take(wl.E * 3, np.float32).reshape(wl.E, 3)
     rev_ptr, rev_perm = take(wl.N + 1, np.int32), take(wl.E, np.int32)
+    forces = take(wl.N * 3, np.float32).reshape(wl.N, 3)
     assert off == raw.size
     tp = oracle.OracleTP(irreps, L, irreps, C)
     ref_out = tp.forward(wl.row_ptr, wl.src, wl.r, wl.x, wl.w)
@@ -85,3 +86,5 @@ def test_c_caller_matches_oracle(caller, tmp_path, L, o3, C):
         assert rel(got, ref[key]) <= 1e-4, key
     o_rp, o_perm, _ = oracle.reverse_csr(wl.N, wl.row_ptr, wl.src)
     assert np.array_equal(rev_ptr, o_rp) and np.array_equal(rev_perm, o_perm)
+    F_ref, _ = oracle.assemble_forces(wl.N, wl.row_ptr, wl.src, wl.r, ref["grad_r"])
+    assert rel(forces, F_ref) <= 1e-4
