@@ -110,6 +110,10 @@ cudaError_t radial_tc_forward(int E, int nb, int PC, float rc, const float* r, c
 size_t radial_tc_backward_prepare_bytes(int PC);
 cudaError_t radial_tc_backward(int E, int PC, float rc, const float* r, const float* W1, const float* W2,
                                const float* grad_w, float* gZ, float* grad_r, void* prep, cudaStream_t s);
+// grad_W2 partial sums over `splits` edge splits on the tensor cores: part [splits][64][PC].
+int radial_tc_grad_w2_splits(int E, int PC);
+cudaError_t radial_tc_grad_w2(int E, int PC, const float* grad_w, const float* H, float* part, int splits,
+                              cudaStream_t s);
 int radial_tc_read_and_clear_fault();
 cudaError_t radial_forward(int E, int nb, int hidden, int PC, float rc, const float* r, const float* W1,
                            const float* W2, float* w, void* ws, cudaStream_t s);

@@ -9,8 +9,8 @@
 // with SiLU, a linear output layer, no biases.)
 //
 // Layout (row-major): W1 [n_basis][hidden], W2 [hidden][P*C], w / grad_w [E][P*C],
-// hidden activations H [E][hidden]. The forward with a hidden width of 64 runs on
-// the tensor cores (etp_radial_tc.cu); the other dense products run in FP32 on the
+// hidden activations H [E][hidden]. With a hidden width of 64 the forward, dL/dH and
+// grad_W2 run on the tensor cores (etp_radial_tc.cu); the other dense products run in FP32 on the
 // SIMT pipes (tiled, 64 x 64 outputs per block, exact fp32 FMAs); their reductions over
 // the edges are split across blocks into partial sums that a second kernel adds
 // in a fixed order, so every result repeats bit for bit.
@@ -186,6 +186,45 @@ __global__ void radial_edge_backward(int E, const float* __restrict__ r, const f
     }
 }
 
+// grad_W1 partial sums: part[split][n][k] = sum_e B[e][n] gZ[e][k] over this block's
+// split of the edges. 256 threads = (256 / hidden) edge lanes x hidden units; each
+// thread keeps its nb (<= 32) sums in registers, then the edge lanes are added in a
+// fixed order through shared memory.
+constexpr int kW1Threads = 256;
+__global__ void __launch_bounds__(kW1Threads) radial_grad_w1(int E, int nb, int hidden, int edges_per_split,
+                                                             const float* __restrict__ Bm, const float* __restrict__ gZ,
+                                                             float* __restrict__ part) {
+    extern __shared__ float red[];  // [lanes][nb][hidden]
+    const int lanes = kW1Threads / hidden, el = threadIdx.x / hidden, k = threadIdx.x % hidden;
+    const int e_begin = blockIdx.x * edges_per_split, e_end = min(E, e_begin + edges_per_split);
+    float acc[32];
+#pragma unroll
+    for (int n = 0; n < 32; ++n) acc[n] = 0.f;
+    if (el < lanes) {
+        for (int e = e_begin + el; e < e_end; e += lanes) {
+            const float g = __ldg(gZ + (size_t)e * hidden + k);
+#pragma unroll
+            for (int n = 0; n < 32; ++n)
+                if (n < nb) acc[n] = fmaf(__ldg(Bm + (size_t)e * nb + n), g, acc[n]);
+        }
+#pragma unroll
+        for (int n = 0; n < 32; ++n)
+            if (n < nb) red[(el * nb + n) * hidden + k] = acc[n];
+    }
+    __syncthreads();
+    for (int o = threadIdx.x; o < nb * hidden; o += kW1Threads) {
+        float v = 0.f;
+        for (int l = 0; l < lanes; ++l) v += red[l * nb * hidden + o];
+        part[(size_t)blockIdx.x * nb * hidden + o] = v;
+    }
+}
+
+// Edge splits of the grad_W1 reduction: two blocks per SM, at least 256 edges each.
+inline int grad_w1_splits(int E) {
+    int s = (E + 255) / 256;
+    return s > 296 ? 296 : (s < 1 ? 1 : s);
+}
+
 inline size_t a16(size_t b) { return (b + 15) & ~size_t(15); }
 
 // Splits of a K = E reduction: enough blocks to fill the GPU once, each split at
@@ -196,6 +235,12 @@ inline int edge_splits(int E, int tiles) {
     if (s > by_size) s = by_size;
     if (s > 64) s = 64;
     return s < 1 ? 1 : s;
+}
+
+// Edge splits of the grad_W2 reduction: the tensor-core kernel's when it runs.
+inline int grad_w2_splits(int E, int nb, int hidden, int PC) {
+    if (radial_tc_supported(nb, hidden, PC)) return radial_tc_grad_w2_splits(E, PC);
+    return edge_splits(E, ((hidden + kTile - 1) / kTile) * ((PC + kTile - 1) / kTile));
 }
 
 template <bool TA, bool TB>
@@ -209,8 +254,8 @@ cudaError_t gemm(int M, int N, int K, const float* A, int lda, const float* B, i
 }  // namespace
 
 size_t radial_workspace_bytes(int E, int nb, int hidden, int PC) {
-    const int s2 = edge_splits(E, ((hidden + kTile - 1) / kTile) * ((PC + kTile - 1) / kTile));
-    const int s1 = edge_splits(E, ((nb + kTile - 1) / kTile) * ((hidden + kTile - 1) / kTile));
+    const int s2 = grad_w2_splits(E, nb, hidden, PC);
+    const int s1 = grad_w1_splits(E);
     const size_t bwd = 4 * a16(sizeof(float) * (size_t)E * hidden) + a16(sizeof(float) * (size_t)E * nb) +
                        a16(sizeof(float) * (size_t)s2 * hidden * PC) + a16(sizeof(float) * (size_t)s1 * nb * hidden);
     const bool tc = radial_tc_supported(nb, hidden, PC);
@@ -245,10 +290,10 @@ cudaError_t radial_backward(int E, int nb, int hidden, int PC, float rc, const f
     float* Bm = reinterpret_cast<float*>(p);
     p += a16(sizeof(float) * (size_t)E * nb);
     float* part2 = reinterpret_cast<float*>(p);
-    const int s2 = edge_splits(E, ((hidden + kTile - 1) / kTile) * ((PC + kTile - 1) / kTile));
+    const int s2 = grad_w2_splits(E, nb, hidden, PC);
     p += a16(sizeof(float) * (size_t)s2 * hidden * PC);
     float* part1 = reinterpret_cast<float*>(p);
-    const int s1 = edge_splits(E, ((nb + kTile - 1) / kTile) * ((hidden + kTile - 1) / kTile));
+    const int s1 = grad_w1_splits(E);
     cudaError_t err;
     if (E == 0) {  // no edges: the parameter gradients are zero
         if ((err = cudaMemsetAsync(grad_W1, 0, sizeof(float) * nb * hidden, s)) != cudaSuccess) return err;
@@ -266,9 +311,15 @@ cudaError_t radial_backward(int E, int nb, int hidden, int PC, float rc, const f
         radial_edge_backward<<<E, hidden, 0, s>>>(E, r, W1, nb, hidden, rc, Z, gH, gZ, grad_r);
     }
     // grad_W2 [hidden][PC] = H^T grad_w, grad_W1 [nb][hidden] = B^T dL/dz: reductions over the edges
-    if ((err = gemm<true, false>(hidden, PC, E, H, hidden, grad_w, PC, part2, s2, s)) != cudaSuccess) return err;
+    if (tc)
+        err = radial_tc_grad_w2(E, PC, grad_w, H, part2, s2, s);
+    else
+        err = gemm<true, false>(hidden, PC, E, H, hidden, grad_w, PC, part2, s2, s);
+    if (err != cudaSuccess) return err;
     sum_splits<<<256, 256, 0, s>>>(part2, s2, (long long)hidden * PC, grad_W2);
-    if ((err = gemm<true, false>(nb, hidden, E, Bm, nb, gZ, hidden, part1, s1, s)) != cudaSuccess) return err;
+    const int per1 = (E + s1 - 1) / s1;
+    radial_grad_w1<<<s1, kW1Threads, sizeof(float) * (kW1Threads / hidden) * nb * hidden, s>>>(E, nb, hidden, per1,
+                                                                                               Bm, gZ, part1);
     sum_splits<<<16, 256, 0, s>>>(part1, s1, (long long)nb * hidden, grad_W1);
     return cudaGetLastError();
 }

@@ -502,7 +502,244 @@ __global__ void __launch_bounds__(kThreads, 1)
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(64) : "memory");
 }
 
+// ---------------------------------------------------------------------------
+// grad_W2 [64][PC] = H^T grad_w: a reduction over the edges, computed transposed on
+// the tensor cores as D [pc][h] = sum_e grad_w[e][pc] H[e][h] (M = 128 columns of w
+// per accumulator, N = 64 hidden units, K = edges). Both operands lie edge by edge in
+// memory, so they are transposed on the way into shared memory: each thread loads a
+// 4-edge x 4-column block as four float4 rows, transposes it in registers and stores
+// four 16-byte runs along K. The operands use the same K-major layout as above with
+// the 8 core matrices of a 32-edge chunk adjacent along K (LBO = 128 B) and row groups
+// kGwSBO = 1040 B apart: the pad of 16 B puts the 8 lanes of a 16-byte store phase
+// (two row groups per 4 lanes) on 8 distinct bank quads.
+//
+// Per CTA (8 warps, one per SM): 256 columns of w (two accumulators of 64 TMEM
+// columns) and one split of the edges, in chunks of 32 edges. Each thread holds
+// its part of the next chunk of grad_w and H in registers (loaded while the current
+// chunk is converted and multiplied), splits it into TF32 halves and stores them
+// into one of two operand slots; one thread issues 4 K-steps x 2 tiles x 3 products
+// per chunk and commits them to the slot's mbarrier. The split's partial sums are
+// written to part [split][64][PC]; the caller adds the splits in a fixed order.
+constexpr int kGwEdges = 32;                        // edges per chunk (4 K-steps)
+constexpr int kGwThreads = 256;
+constexpr int kGwCols = 256;                        // columns of w per CTA (2 x M = 128)
+constexpr uint32_t kGwSBO = kGwEdges * 4 * 8 + 16;  // one row group of a chunk, padded
+constexpr uint32_t kGwAHalf = 16 * kGwSBO;          // 128 columns x 32 edges, one TF32 half
+constexpr uint32_t kGwBHalf = 8 * kGwSBO;           // 64 hidden units x 32 edges
+constexpr uint32_t kGwOffB = 2 * 2 * 2 * kGwAHalf;  // [slot][half][tile] A, then [slot][half] B
+constexpr uint32_t kGwOffBars = kGwOffB + 2 * 2 * kGwBHalf;
+constexpr uint32_t kGwSmem = kGwOffBars + 64;
+static_assert(kGwSmem <= 232448 && kGwOffBars % 16 == 0 && kGwSBO % 128 == 16, "grad_W2 kernel shared memory");
+
+__device__ __forceinline__ uint64_t smem_desc_gw(uint32_t saddr) {
+    return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((kLBO >> 4) & 0x3FFFu) << 16) |
+           ((uint64_t)((kGwSBO >> 4) & 0x3FFFu) << 32) | ((uint64_t)1 << 46);
+}
+
+// grad_w is read once: stream it past L2 (evict first) and L1.
+__device__ __forceinline__ float4 ld_stream(const float* p, uint64_t policy) {
+    float4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.L2::cache_hint.v4.f32 {%0, %1, %2, %3}, [%4], %5;"
+                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                 : "l"(p), "l"(policy));
+    return v;
+}
+
+__device__ __forceinline__ void st_split(unsigned char* hi, unsigned char* lo, float a, float b, float c, float d) {
+    const float4 h = make_float4(tf32_round(a), tf32_round(b), tf32_round(c), tf32_round(d));
+    *reinterpret_cast<float4*>(hi) = h;
+    *reinterpret_cast<float4*>(lo) =
+        make_float4(tf32_round(a - h.x), tf32_round(b - h.y), tf32_round(c - h.z), tf32_round(d - h.w));
+}
+
+// Rows 4 e4 .. 4 e4 + 3 (edges) of a 4 x 4 block whose column j is row `row0 + j` of
+// the operand: column j goes to K-major position (row0 + j, 4 e4 .. 4 e4 + 3).
+__device__ __forceinline__ void st_block(unsigned char* hi, unsigned char* lo, int row0, int e4, const float4 (&v)[4]) {
+    const uint32_t base = (uint32_t)(row0 >> 3) * kGwSBO + (uint32_t)e4 * kLBO + (uint32_t)(row0 & 7) * 16;
+    st_split(hi + base, lo + base, v[0].x, v[1].x, v[2].x, v[3].x);
+    st_split(hi + base + 16, lo + base + 16, v[0].y, v[1].y, v[2].y, v[3].y);
+    st_split(hi + base + 32, lo + base + 32, v[0].z, v[1].z, v[2].z, v[3].z);
+    st_split(hi + base + 48, lo + base + 48, v[0].w, v[1].w, v[2].w, v[3].w);
+}
+
+__global__ void __launch_bounds__(kGwThreads, 1)
+    radial_tc_grad_w2(int E, int PC, int chunks_per_split, const float* __restrict__ grad_w,
+                      const float* __restrict__ H, float* __restrict__ part) {
+    extern __shared__ __align__(1024) unsigned char smem[];
+    uint64_t* bar_m = reinterpret_cast<uint64_t*>(smem + kGwOffBars);  // [2] MMAs of a slot done
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kGwOffBars + 16);
+    int* abort_flag = reinterpret_cast<int*>(smem + kGwOffBars + 20);
+    const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
+    const int pc0 = blockIdx.x * kGwCols;
+    const int n_tiles = PC - pc0 > kRows ? 2 : 1;
+    const int n_chunks = (E + kGwEdges - 1) / kGwEdges;
+    const int c_begin = blockIdx.y * chunks_per_split;
+    const int nq = max(0, min(n_chunks, c_begin + chunks_per_split) - c_begin);
+    auto a_half = [&](int slot, int lo, int mt) { return smem + (uint32_t)((slot * 2 + lo) * 2 + mt) * kGwAHalf; };
+    auto b_half = [&](int slot, int lo) { return smem + kGwOffB + (uint32_t)(slot * 2 + lo) * kGwBHalf; };
+    uint64_t policy;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(policy));
+
+    if (warp == 0) {  // two accumulators of 64 fp32 columns
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                     "r"(128)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    if (t == 0) {
+        mbar_init(&bar_m[0], 1);
+        mbar_init(&bar_m[1], 1);
+        *abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+    __syncthreads();
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+    const uint32_t tmem = *tmem_slot;
+
+    // this thread's share of a chunk: two 4 x 4 blocks of grad_w (edge quad i / 64,
+    // column group i % 64 for i = t + 256 j) and, for t < 128, one of H (edge quad
+    // t / 16, hidden group t % 16)
+    float4 g[2][2][4], hv[2][4];
+    auto load = [&](int b, int q) {
+        const int e0 = (c_begin + q) * kGwEdges;
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+            const int i = t + kGwThreads * j, pc = pc0 + 4 * (i & 63);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const int e = e0 + 4 * (i >> 6) + k;
+                g[b][j][k] = (e < E && pc < PC) ? ld_stream(grad_w + (size_t)e * PC + pc, policy)
+                                                : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+        }
+        if (t < 128) {
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const int e = e0 + 4 * (t >> 4) + k;
+                hv[b][k] = e < E ? __ldg(reinterpret_cast<const float4*>(H + (size_t)e * kHidden + 4 * (t & 15)))
+                                 : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+        }
+    };
+    if (nq > 0) load(0, 0);
+    if (nq > 1) load(1, 1);
+    int last = -1;
+    bool stop = false;
+    for (int q0 = 0; q0 < nq && !stop; q0 += 2) {
+#pragma unroll
+        for (int b = 0; b < 2; ++b) {
+            const int q = q0 + b;
+            if (q >= nq || stop) break;
+            if (q >= 2) {  // slot b was read by the MMAs of chunk q - 2
+                if (!mbar_wait(&bar_m[b], ((q - 2) >> 1) & 1)) atomicOr(abort_flag, 1);
+                __syncthreads();
+                if (*abort_flag) {
+                    stop = true;
+                    break;
+                }
+            }
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                const int i = t + kGwThreads * j, grp = i & 63;
+                st_block(a_half(b, 0, grp >> 5), a_half(b, 1, grp >> 5), 4 * (grp & 31), i >> 6, g[b][j]);
+            }
+            if (t < 128) st_block(b_half(b, 0), b_half(b, 1), 4 * (t & 15), t >> 4, hv[b]);
+            if (q + 2 < nq) load(b, q + 2);  // in flight while this chunk is multiplied
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+            __syncthreads();
+            if (t == 0) {
+                asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+                const uint32_t idesc = instr_desc(kHidden);  // M = 128, N = 64, both K-major
+                for (int s = 0; s < kGwEdges / 8; ++s) {
+                    for (int mt = 0; mt < n_tiles; ++mt) {
+                        // A_hi B_hi + A_hi B_lo + A_lo B_hi
+                        const uint32_t A[3] = {smem_u32(a_half(b, 0, mt)), smem_u32(a_half(b, 0, mt)),
+                                               smem_u32(a_half(b, 1, mt))};
+                        const uint32_t B[3] = {smem_u32(b_half(b, 0)), smem_u32(b_half(b, 1)),
+                                               smem_u32(b_half(b, 0))};
+                        for (int p = 0; p < 3; ++p) {
+                            const uint64_t da = smem_desc_gw(A[p] + s * 2 * kLBO);
+                            const uint64_t db = smem_desc_gw(B[p] + s * 2 * kLBO);
+                            const uint32_t acc = (q | s | p) ? 1u : 0u;
+                            asm volatile(
+                                "{\n .reg .pred pp;\n setp.ne.b32 pp, %4, 0;\n"
+                                " tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, pp;\n}" ::"r"(
+                                    tmem + (uint32_t)(mt * kHidden)),
+                                "l"(da), "l"(db), "r"(idesc), "r"(acc)
+                                : "memory");
+                        }
+                    }
+                }
+                asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                                 smem_u32(&bar_m[b]))
+                             : "memory");
+                last = q;
+            }
+        }
+    }
+    // all MMAs are complete once the last chunk's are
+    if (!*abort_flag && nq > 0 && !mbar_wait(&bar_m[(nq - 1) & 1], ((nq - 1) >> 1) & 1)) atomicOr(abort_flag, 1);
+    __syncthreads();
+    const int mt = warp >> 2, pc = pc0 + mt * kRows + (warp & 3) * 32 + lane;
+    if (!*abort_flag && mt < n_tiles) {
+        float* out = part + (size_t)blockIdx.y * kHidden * PC;
+        if (nq == 0) {  // an empty split contributes zeros
+            if (pc < PC)
+                for (int h = 0; h < kHidden; ++h) out[(size_t)h * PC + pc] = 0.f;
+        } else {
+            asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+            uint32_t v[64];
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj)
+                asm volatile(
+                    "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, "
+                    "%13, %14, %15}, [%16];"
+                    : "=r"(v[16 * jj]), "=r"(v[16 * jj + 1]), "=r"(v[16 * jj + 2]), "=r"(v[16 * jj + 3]),
+                      "=r"(v[16 * jj + 4]), "=r"(v[16 * jj + 5]), "=r"(v[16 * jj + 6]), "=r"(v[16 * jj + 7]),
+                      "=r"(v[16 * jj + 8]), "=r"(v[16 * jj + 9]), "=r"(v[16 * jj + 10]), "=r"(v[16 * jj + 11]),
+                      "=r"(v[16 * jj + 12]), "=r"(v[16 * jj + 13]), "=r"(v[16 * jj + 14]), "=r"(v[16 * jj + 15])
+                    : "r"(tmem + ((uint32_t)((warp & 3) * 32) << 16) + (uint32_t)(mt * kHidden + 16 * jj)));
+            asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+            if (pc < PC)
+#pragma unroll
+                for (int h = 0; h < kHidden; ++h) out[(size_t)h * PC + pc] = __uint_as_float(v[h]);
+        }
+    }
+    __syncthreads();
+    if (t == 0 && *abort_flag) {
+        atomicOr(&g_fault, 1);
+        if (last >= 0) mbar_wait(&bar_m[last & 1], (last >> 1) & 1);  // nothing left in flight on freed TMEM
+    }
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+    __syncthreads();
+    if (warp == 0)
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(128) : "memory");
+}
+
 }  // namespace rtc
+
+int radial_tc_grad_w2_splits(int E, int PC) {
+    const int n_cta = (PC + rtc::kGwCols - 1) / rtc::kGwCols;
+    const int n_chunks = (E + rtc::kGwEdges - 1) / rtc::kGwEdges;
+    int s = 148 / n_cta;                     // one wave of one CTA per SM
+    const int by_size = n_chunks / 8;        // at least 8 chunks (256 edges) per split
+    if (s > by_size) s = by_size;
+    return s < 1 ? 1 : s;
+}
+
+cudaError_t radial_tc_grad_w2(int E, int PC, const float* grad_w, const float* H, float* part, int splits,
+                              cudaStream_t s) {
+    const int n_chunks = (E + rtc::kGwEdges - 1) / rtc::kGwEdges;
+    const int per = (n_chunks + splits - 1) / splits;
+    cudaError_t err = cudaFuncSetAttribute(rtc::radial_tc_grad_w2, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           (int)rtc::kGwSmem);
+    if (err != cudaSuccess) return err;
+    dim3 grid((PC + rtc::kGwCols - 1) / rtc::kGwCols, splits);
+    rtc::radial_tc_grad_w2<<<grid, rtc::kGwThreads, rtc::kGwSmem, s>>>(E, PC, per, grad_w, H, part);
+    return cudaGetLastError();
+}
 
 size_t radial_tc_prepare_bytes(int PC) {
     const int n_chunks = (PC + rtc::kChunk - 1) / rtc::kChunk;
