@@ -289,20 +289,87 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ---------------------------------------------------------------------------
+// Shared by the two VJP kernels below: warp-specialised pipelines in which 8
+// producer warps split operand chunks into TF32 halves in shared memory and one
+// more warp issues the MMAs. A chunk's slot is handed over by mbarriers: `full`
+// (8 arrivals, one per producer warp, after each thread's proxy fence) and `empty`
+// (the tcgen05.commit of the chunk's MMAs). No block-wide barrier inside the loop.
+constexpr int kProducers = 256;               // 8 producer warps
+constexpr int kPipeThreads = kProducers + 32; // + the MMA warp
+
+// grad_w is read once: stream it past L2 (evict first) and L1.
+__device__ __forceinline__ float4 ld_stream(const float* p, uint64_t policy) {
+    float4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.L2::cache_hint.v4.f32 {%0, %1, %2, %3}, [%4], %5;"
+                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                 : "l"(p), "l"(policy));
+    return v;
+}
+
+__device__ __forceinline__ uint64_t evict_first_policy() {
+    uint64_t policy;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(policy));
+    return policy;
+}
+
+__device__ __forceinline__ void st_split(unsigned char* hi, unsigned char* lo, float a, float b, float c, float d) {
+    const float4 h = make_float4(tf32_round(a), tf32_round(b), tf32_round(c), tf32_round(d));
+    *reinterpret_cast<float4*>(hi) = h;
+    *reinterpret_cast<float4*>(lo) =
+        make_float4(tf32_round(a - h.x), tf32_round(b - h.y), tf32_round(c - h.z), tf32_round(d - h.w));
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+// A producer warp's hand-over of a filled slot: every thread's generic-proxy stores
+// are made visible to the tensor core's proxy, then one lane arrives.
+__device__ __forceinline__ void hand_over(uint64_t* full, int lane) {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    __syncwarp();
+    if (lane == 0) mbar_arrive(full);
+}
+
+__device__ __forceinline__ void mma_tf32(uint32_t d_tmem, uint64_t da, uint64_t db, uint32_t idesc, uint32_t acc) {
+    asm volatile(
+        "{\n .reg .pred pp;\n setp.ne.b32 pp, %4, 0;\n"
+        " tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, pp;\n}" ::"r"(d_tmem),
+        "l"(da), "l"(db), "r"(idesc), "r"(acc)
+        : "memory");
+}
+
+__device__ __forceinline__ void mma_commit(uint64_t* bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+                 : "memory");
+}
+
+// Shared-memory descriptor with explicit LBO / SBO (bytes), no swizzle.
+__device__ __forceinline__ uint64_t smem_desc_bo(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+    return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+           ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | ((uint64_t)1 << 46);
+}
+
+// ---------------------------------------------------------------------------
 // Backward: dL/dH [E][64] = grad_w [E][PC] W2^T on the tensor cores (M = 128 edges,
 // N = 64 hidden units, K = PC in chunks of 64), with the per-edge rest of the VJP
 // fused into the epilogue: dL/dz = dL/dH * SiLU'(z) (written out for grad_W1),
 // dL/db = dL/dz W1^T, dL/dd = dL/db . db/dd and grad_r[e] += dL/dd r / |r|.
-// grad_w chunks are split into TF32 halves by the threads into one of two A slots
-// while the tensor cores multiply the other; W2 chunks (64 rows x 64 K, halves
-// pre-split) arrive by bulk copies into two B slots.
+// The producers read the tile's grad_w chunk row segment by row segment (16 lanes x
+// 16 bytes per edge), keep the next chunk in flight in registers, and store the
+// TF32 halves K-major with LBO = 144 B between core matrices along K: the pad of
+// 16 B puts the 8 lanes of a store phase (consecutive K groups of one edge) on 8
+// distinct bank quads. W2 chunks (64 rows x 64 K, halves pre-split) arrive by bulk
+// copies into two B slots.
 constexpr int kKChunk = 64;
 constexpr uint32_t kBwTileB = 64 * kKChunk * 4;                 // 16 KB: one half of a W2 chunk
-constexpr uint32_t kBwOffB = 4 * kTileBytes;                    // after the two A slots (2 x 64 KB)
-constexpr uint32_t kBwOffW1 = kBwOffB + 4 * kBwTileB;           // after the two B slots (2 x 32 KB)
+constexpr uint32_t kBwLBO = 144, kBwSBO = 16 * kBwLBO;          // A: padded K-major, 64 K per row group
+constexpr uint32_t kBwAHalf = 16 * kBwSBO;                      // 128 edges x 64 K, one TF32 half
+constexpr uint32_t kBwOffB = 4 * kBwAHalf;                      // after the two A slots [slot][half]
+constexpr uint32_t kBwOffW1 = kBwOffB + 4 * kBwTileB;           // after the two B slots [slot][half]
 constexpr uint32_t kBwOffBars = kBwOffW1 + kBasis * kHidden * 4;
 constexpr uint32_t kBwSmem = kBwOffBars + 64;
-static_assert(kBwSmem <= 232448 && kBwOffBars % 16 == 0, "radial backward shared memory");
+static_assert(kBwSmem <= 232448 && kBwOffBars % 16 == 0 && kBwLBO % 128 == 16, "radial backward shared memory");
 
 // W2 [64][PC] as K-major B chunks: chunk q holds rows h = 0..63, K = columns 64q..64q+63.
 __global__ void radial_tc_prepare_w2(const float* __restrict__ W2, int PC, int n_kc, float* __restrict__ hi,
@@ -334,23 +401,22 @@ __device__ __forceinline__ void load_w2(const float* Bhi, const float* Blo, int 
                  : "memory");
 }
 
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kPipeThreads, 1)
     radial_tc_backward(int E, int PC, float rc, const float* __restrict__ r, const float* __restrict__ W1,
                        const float* __restrict__ Bhi, const float* __restrict__ Blo,
                        const float* __restrict__ grad_w, float* __restrict__ gZ, float* __restrict__ grad_r) {
     extern __shared__ __align__(1024) unsigned char smem[];
     float* w1s = reinterpret_cast<float*>(smem + kBwOffW1);
-    uint64_t* bar_b = reinterpret_cast<uint64_t*>(smem + kBwOffBars);  // [2] W2 chunk arrived
-    uint64_t* bar_m = bar_b + 2;                                         // [2] MMAs of a slot done
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kBwOffBars + 32);
-    int* abort_flag = reinterpret_cast<int*>(smem + kBwOffBars + 36);
-    const int t = threadIdx.x, warp = t >> 5;
-    const int m0 = blockIdx.x * kRows, e = m0 + t;
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + kBwOffBars);  // [2] A slot written
+    uint64_t* empty = full + 2;                                         // [2] MMAs of a slot done
+    uint64_t* bfull = full + 4;                                         // [2] W2 chunk arrived
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kBwOffBars + 48);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kBwOffBars + 52);
+    const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
+    const int m0 = blockIdx.x * kRows;
     const int n_kc = (PC + kKChunk - 1) / kKChunk;
-    auto a_hi = [&](int s) { return smem + (uint32_t)s * 2 * kTileBytes; };
-    auto a_lo = [&](int s) { return smem + (uint32_t)s * 2 * kTileBytes + kTileBytes; };
-    auto b_hi = [&](int s) { return smem + kBwOffB + (uint32_t)s * 2 * kBwTileB; };
-    auto b_lo = [&](int s) { return smem + kBwOffB + (uint32_t)s * 2 * kBwTileB + kBwTileB; };
+    auto a_half = [&](int s, int lo) { return smem + (uint32_t)(s * 2 + lo) * kBwAHalf; };
+    auto b_half = [&](int s, int lo) { return smem + kBwOffB + (uint32_t)(s * 2 + lo) * kBwTileB; };
 
     if (warp == 0) {  // 64 fp32 accumulator columns (dL/dH of the tile)
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
@@ -358,78 +424,99 @@ __global__ void __launch_bounds__(kThreads, 1)
                      : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
-    for (int i = t; i < kBasis * kHidden; i += kThreads) w1s[i] = __ldg(W1 + i);
+    for (int i = t; i < kBasis * kHidden; i += kPipeThreads) w1s[i] = __ldg(W1 + i);
+    int issued[2] = {-1, -1};  // (thread 0) the last W2 chunk copied into each B slot
     if (t == 0) {
-        for (int i = 0; i < 4; ++i) mbar_init(&bar_b[i], 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&full[i], kProducers / 32);
+            mbar_init(&empty[i], 1);
+            mbar_init(&bfull[i], 1);
+        }
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-        load_w2(Bhi, Blo, 0, b_hi(0), b_lo(0), &bar_b[0]);
-        if (n_kc > 1) load_w2(Bhi, Blo, 1, b_hi(1), b_lo(1), &bar_b[1]);
+        for (int q = 0; q < 2 && q < n_kc; ++q) {
+            load_w2(Bhi, Blo, q, b_half(q, 0), b_half(q, 1), &bfull[q]);
+            issued[q] = q;
+        }
     }
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
     __syncthreads();
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
     const uint32_t tmem = *tmem_slot;
-    int last = -1;
+    int last = -1;  // (MMA thread) the last chunk whose MMAs were committed
 
-    for (int q = 0; q < n_kc; ++q) {
-        const int sa = q & 1;
-        if (q >= 2) {  // slot sa was read by the MMAs of chunk q - 2
-            if (!mbar_wait(&bar_m[sa], ((q - 2) >> 1) & 1)) atomicOr(abort_flag, 1);
-            __syncthreads();
-            if (*abort_flag) break;
-            if (t == 0) load_w2(Bhi, Blo, q, b_hi(sa), b_lo(sa), &bar_b[sa]);
-        }
-        // this thread's edge row of the grad_w chunk, split into TF32 halves
-        const int c0 = q * kKChunk;
-#pragma unroll 4
-        for (int k4 = 0; k4 < kKChunk; k4 += 4) {
-            float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (e < E && c0 + k4 < PC) v = __ldg(reinterpret_cast<const float4*>(grad_w + (size_t)e * PC + c0 + k4));
-            const float vv[4] = {v.x, v.y, v.z, v.w};
+    if (warp < kProducers / 32) {
+        // this thread's share of a chunk: 8 float4, edge i / 16 of the tile and column
+        // group i % 16 of the chunk for i = t + 256 j
+        const uint64_t policy = evict_first_policy();
+        float4 g[2][8];
+        auto load = [&](int b, int q) {
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const float h = tf32_round(vv[j]);
-                *reinterpret_cast<float*>(a_hi(sa) + tile_offset(t, k4 + j)) = h;
-                *reinterpret_cast<float*>(a_lo(sa) + tile_offset(t, k4 + j)) = tf32_round(vv[j] - h);
+            for (int j = 0; j < 8; ++j) {
+                const int i = t + kProducers * j, e = m0 + (i >> 4), pc = q * kKChunk + 4 * (i & 15);
+                g[b][j] = (e < E && pc < PC) ? ld_stream(grad_w + (size_t)e * PC + pc, policy)
+                                             : make_float4(0.f, 0.f, 0.f, 0.f);
             }
-        }
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-        __syncthreads();
-        if (t == 0 && !*abort_flag) {
-            if (!mbar_wait(&bar_b[sa], (q >> 1) & 1)) {
-                *abort_flag = 1;
-            } else {
-                asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-                const uint32_t idesc = instr_desc(kHidden);  // N = 64
-                const uint32_t A[3] = {smem_u32(a_hi(sa)), smem_u32(a_hi(sa)), smem_u32(a_lo(sa))};
-                const uint32_t B[3] = {smem_u32(b_hi(sa)), smem_u32(b_lo(sa)), smem_u32(b_hi(sa))};
-                for (int s = 0; s < kKChunk / 8; ++s) {
-                    for (int p = 0; p < 3; ++p) {
-                        const uint64_t da = smem_desc(A[p] + s * 2 * kLBO);
-                        const uint64_t db = smem_desc(B[p] + s * 2 * kLBO);
-                        const uint32_t acc = (q | s | p) ? 1u : 0u;
-                        asm volatile(
-                            "{\n .reg .pred pp;\n setp.ne.b32 pp, %4, 0;\n"
-                            " tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, pp;\n}" ::"r"(tmem),
-                            "l"(da), "l"(db), "r"(idesc), "r"(acc)
-                            : "memory");
+        };
+        if (n_kc > 0) load(0, 0);
+        if (n_kc > 1) load(1, 1);
+        bool stop = false;
+        for (int q0 = 0; q0 < n_kc && !stop; q0 += 2) {
+#pragma unroll
+            for (int b = 0; b < 2; ++b) {
+                const int q = q0 + b;
+                // warp-uniform decisions: the hand-over below synchronises the warp
+                if (q >= n_kc || __any_sync(0xffffffffu, *abort_flag != 0)) {
+                    stop = true;
+                    break;
+                }
+                if (q >= 2) {  // slot b was read by the MMAs of chunk q - 2
+                    if (!__all_sync(0xffffffffu, mbar_wait(&empty[b], ((q - 2) >> 1) & 1))) {
+                        if (lane == 0) atomicOr((int*)abort_flag, 1);
+                        stop = true;
+                        break;
+                    }
+                    if (t == 0) {
+                        load_w2(Bhi, Blo, q, b_half(b, 0), b_half(b, 1), &bfull[b]);
+                        issued[b] = q;
                     }
                 }
-                asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                                 smem_u32(&bar_m[sa]))
-                             : "memory");
-                last = q;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const int i = t + kProducers * j, el = i >> 4;
+                    const uint32_t off = (uint32_t)(el >> 3) * kBwSBO + (uint32_t)(i & 15) * kBwLBO + (el & 7) * 16;
+                    st_split(a_half(b, 0) + off, a_half(b, 1) + off, g[b][j].x, g[b][j].y, g[b][j].z, g[b][j].w);
+                }
+                if (q + 2 < n_kc) load(b, q + 2);  // in flight while this chunk is multiplied
+                hand_over(&full[b], lane);
             }
         }
-        __syncthreads();
-        if (*abort_flag) break;
+    } else if (lane == 0) {  // the MMA warp
+        const uint32_t idesc = instr_desc(kHidden);  // N = 64
+        for (int q = 0; q < n_kc; ++q) {
+            const int b = q & 1;
+            if (*abort_flag) break;
+            if (!mbar_wait(&full[b], (q >> 1) & 1) || !mbar_wait(&bfull[b], (q >> 1) & 1)) {
+                atomicOr((int*)abort_flag, 1);
+                break;
+            }
+            asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+            const uint32_t A[3] = {smem_u32(a_half(b, 0)), smem_u32(a_half(b, 0)), smem_u32(a_half(b, 1))};
+            const uint32_t B[3] = {smem_u32(b_half(b, 0)), smem_u32(b_half(b, 1)), smem_u32(b_half(b, 0))};
+            for (int s = 0; s < kKChunk / 8; ++s)
+                for (int p = 0; p < 3; ++p)
+                    mma_tf32(tmem, smem_desc_bo(A[p] + s * 2 * kBwLBO, kBwLBO, kBwSBO),
+                             smem_desc_bo(B[p] + s * 2 * kLBO, kLBO, kSBO), idesc, (q | s | p) ? 1u : 0u);
+            mma_commit(&empty[b]);
+            last = q;
+        }
     }
     // the accumulator is complete once the last chunk's MMAs are
-    if (!*abort_flag && n_kc > 0 && !mbar_wait(&bar_m[(n_kc - 1) & 1], ((n_kc - 1) >> 1) & 1)) atomicOr(abort_flag, 1);
+    if (warp < 4 && !*abort_flag && n_kc > 0 && !mbar_wait(&empty[(n_kc - 1) & 1], ((n_kc - 1) >> 1) & 1))
+        atomicOr((int*)abort_flag, 1);
     __syncthreads();
-    if (!*abort_flag) {
+    const int e = m0 + t;
+    if (!*abort_flag && warp < 4) {
         asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
         uint32_t g[64];
 #pragma unroll
@@ -492,9 +579,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     }
     __syncthreads();
-    if (t == 0 && *abort_flag) {
-        atomicOr(&g_fault, 1);
-        if (last >= 0) mbar_wait(&bar_m[last & 1], (last >> 1) & 1);  // nothing left in flight on freed TMEM
+    if (*abort_flag) {  // leave nothing in flight on the freed TMEM and shared memory: one bounded wait each
+        if (t == 0) atomicOr(&g_fault, 1);
+        if (t == kProducers && last >= 0) mbar_wait(&empty[last & 1], (last >> 1) & 1);
+        if (t == 0)
+            for (int b = 0; b < 2; ++b)
+                if (issued[b] >= 0) mbar_wait(&bfull[b], (issued[b] >> 1) & 1);
     }
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
     __syncthreads();
@@ -506,22 +596,21 @@ __global__ void __launch_bounds__(kThreads, 1)
 // grad_W2 [64][PC] = H^T grad_w: a reduction over the edges, computed transposed on
 // the tensor cores as D [pc][h] = sum_e grad_w[e][pc] H[e][h] (M = 128 columns of w
 // per accumulator, N = 64 hidden units, K = edges). Both operands lie edge by edge in
-// memory, so they are transposed on the way into shared memory: each thread loads a
-// 4-edge x 4-column block as four float4 rows, transposes it in registers and stores
-// four 16-byte runs along K. The operands use the same K-major layout as above with
-// the 8 core matrices of a 32-edge chunk adjacent along K (LBO = 128 B) and row groups
-// kGwSBO = 1040 B apart: the pad of 16 B puts the 8 lanes of a 16-byte store phase
-// (two row groups per 4 lanes) on 8 distinct bank quads.
+// memory, so they are transposed on the way into shared memory: each producer thread
+// loads a 4-edge x 4-column block as four float4 rows, transposes it in registers and
+// stores four 16-byte runs along K. The operands are K-major with the 8 core matrices
+// of a 32-edge chunk adjacent along K (LBO = 128 B) and row groups kGwSBO = 1040 B
+// apart: the pad of 16 B puts the 8 lanes of a store phase (two row groups per 4
+// lanes) on 8 distinct bank quads.
 //
-// Per CTA (8 warps, one per SM): 256 columns of w (two accumulators of 64 TMEM
-// columns) and one split of the edges, in chunks of 32 edges. Each thread holds
-// its part of the next chunk of grad_w and H in registers (loaded while the current
-// chunk is converted and multiplied), splits it into TF32 halves and stores them
-// into one of two operand slots; one thread issues 4 K-steps x 2 tiles x 3 products
-// per chunk and commits them to the slot's mbarrier. The split's partial sums are
-// written to part [split][64][PC]; the caller adds the splits in a fixed order.
+// Per CTA (one per SM): 256 columns of w (two accumulators of 64 TMEM columns) and
+// one split of the edges, in chunks of 32 edges. Each producer thread holds its part
+// of the next chunk of grad_w and H in registers (loaded while the current chunk is
+// converted and multiplied), splits it into TF32 halves and stores them into one of
+// two operand slots; the MMA warp issues 4 K-steps x 2 tiles x 3 products per chunk.
+// The split's partial sums are written to part [split][64][PC]; the caller adds the
+// splits in a fixed order.
 constexpr int kGwEdges = 32;                        // edges per chunk (4 K-steps)
-constexpr int kGwThreads = 256;
 constexpr int kGwCols = 256;                        // columns of w per CTA (2 x M = 128)
 constexpr uint32_t kGwSBO = kGwEdges * 4 * 8 + 16;  // one row group of a chunk, padded
 constexpr uint32_t kGwAHalf = 16 * kGwSBO;          // 128 columns x 32 edges, one TF32 half
@@ -530,27 +619,6 @@ constexpr uint32_t kGwOffB = 2 * 2 * 2 * kGwAHalf;  // [slot][half][tile] A, the
 constexpr uint32_t kGwOffBars = kGwOffB + 2 * 2 * kGwBHalf;
 constexpr uint32_t kGwSmem = kGwOffBars + 64;
 static_assert(kGwSmem <= 232448 && kGwOffBars % 16 == 0 && kGwSBO % 128 == 16, "grad_W2 kernel shared memory");
-
-__device__ __forceinline__ uint64_t smem_desc_gw(uint32_t saddr) {
-    return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((kLBO >> 4) & 0x3FFFu) << 16) |
-           ((uint64_t)((kGwSBO >> 4) & 0x3FFFu) << 32) | ((uint64_t)1 << 46);
-}
-
-// grad_w is read once: stream it past L2 (evict first) and L1.
-__device__ __forceinline__ float4 ld_stream(const float* p, uint64_t policy) {
-    float4 v;
-    asm volatile("ld.global.nc.L1::no_allocate.L2::cache_hint.v4.f32 {%0, %1, %2, %3}, [%4], %5;"
-                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
-                 : "l"(p), "l"(policy));
-    return v;
-}
-
-__device__ __forceinline__ void st_split(unsigned char* hi, unsigned char* lo, float a, float b, float c, float d) {
-    const float4 h = make_float4(tf32_round(a), tf32_round(b), tf32_round(c), tf32_round(d));
-    *reinterpret_cast<float4*>(hi) = h;
-    *reinterpret_cast<float4*>(lo) =
-        make_float4(tf32_round(a - h.x), tf32_round(b - h.y), tf32_round(c - h.z), tf32_round(d - h.w));
-}
 
 // Rows 4 e4 .. 4 e4 + 3 (edges) of a 4 x 4 block whose column j is row `row0 + j` of
 // the operand: column j goes to K-major position (row0 + j, 4 e4 .. 4 e4 + 3).
@@ -562,13 +630,14 @@ __device__ __forceinline__ void st_block(unsigned char* hi, unsigned char* lo, i
     st_split(hi + base + 48, lo + base + 48, v[0].w, v[1].w, v[2].w, v[3].w);
 }
 
-__global__ void __launch_bounds__(kGwThreads, 1)
+__global__ void __launch_bounds__(kPipeThreads, 1)
     radial_tc_grad_w2(int E, int PC, int chunks_per_split, const float* __restrict__ grad_w,
                       const float* __restrict__ H, float* __restrict__ part) {
     extern __shared__ __align__(1024) unsigned char smem[];
-    uint64_t* bar_m = reinterpret_cast<uint64_t*>(smem + kGwOffBars);  // [2] MMAs of a slot done
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kGwOffBars + 16);
-    int* abort_flag = reinterpret_cast<int*>(smem + kGwOffBars + 20);
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + kGwOffBars);  // [2] slot written
+    uint64_t* empty = full + 2;                                         // [2] MMAs of a slot done
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kGwOffBars + 32);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kGwOffBars + 36);
     const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
     const int pc0 = blockIdx.x * kGwCols;
     const int n_tiles = PC - pc0 > kRows ? 2 : 1;
@@ -577,8 +646,6 @@ __global__ void __launch_bounds__(kGwThreads, 1)
     const int nq = max(0, min(n_chunks, c_begin + chunks_per_split) - c_begin);
     auto a_half = [&](int slot, int lo, int mt) { return smem + (uint32_t)((slot * 2 + lo) * 2 + mt) * kGwAHalf; };
     auto b_half = [&](int slot, int lo) { return smem + kGwOffB + (uint32_t)(slot * 2 + lo) * kGwBHalf; };
-    uint64_t policy;
-    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(policy));
 
     if (warp == 0) {  // two accumulators of 64 fp32 columns
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
@@ -587,8 +654,10 @@ __global__ void __launch_bounds__(kGwThreads, 1)
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
     if (t == 0) {
-        mbar_init(&bar_m[0], 1);
-        mbar_init(&bar_m[1], 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&full[i], kProducers / 32);
+            mbar_init(&empty[i], 1);
+        }
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -596,94 +665,92 @@ __global__ void __launch_bounds__(kGwThreads, 1)
     __syncthreads();
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
     const uint32_t tmem = *tmem_slot;
+    int last = -1;  // (MMA thread) the last chunk whose MMAs were committed
 
-    // this thread's share of a chunk: two 4 x 4 blocks of grad_w (edge quad i / 64,
-    // column group i % 64 for i = t + 256 j) and, for t < 128, one of H (edge quad
-    // t / 16, hidden group t % 16)
-    float4 g[2][2][4], hv[2][4];
-    auto load = [&](int b, int q) {
-        const int e0 = (c_begin + q) * kGwEdges;
+    if (warp < kProducers / 32) {
+        // this thread's share of a chunk: two 4 x 4 blocks of grad_w (edge quad i / 64,
+        // column group i % 64 for i = t + 256 j) and, for t < 128, one of H (edge quad
+        // t / 16, hidden group t % 16)
+        const uint64_t policy = evict_first_policy();
+        float4 g[2][2][4], hv[2][4];
+        auto load = [&](int b, int q) {
+            const int e0 = (c_begin + q) * kGwEdges;
 #pragma unroll
-        for (int j = 0; j < 2; ++j) {
-            const int i = t + kGwThreads * j, pc = pc0 + 4 * (i & 63);
+            for (int j = 0; j < 2; ++j) {
+                const int i = t + kProducers * j, pc = pc0 + 4 * (i & 63);
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const int e = e0 + 4 * (i >> 6) + k;
-                g[b][j][k] = (e < E && pc < PC) ? ld_stream(grad_w + (size_t)e * PC + pc, policy)
-                                                : make_float4(0.f, 0.f, 0.f, 0.f);
+                for (int k = 0; k < 4; ++k) {
+                    const int e = e0 + 4 * (i >> 6) + k;
+                    g[b][j][k] = (e < E && pc < PC) ? ld_stream(grad_w + (size_t)e * PC + pc, policy)
+                                                    : make_float4(0.f, 0.f, 0.f, 0.f);
+                }
             }
-        }
-        if (t < 128) {
+            if (t < 128) {
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const int e = e0 + 4 * (t >> 4) + k;
-                hv[b][k] = e < E ? __ldg(reinterpret_cast<const float4*>(H + (size_t)e * kHidden + 4 * (t & 15)))
-                                 : make_float4(0.f, 0.f, 0.f, 0.f);
+                for (int k = 0; k < 4; ++k) {
+                    const int e = e0 + 4 * (t >> 4) + k;
+                    hv[b][k] = e < E ? __ldg(reinterpret_cast<const float4*>(H + (size_t)e * kHidden + 4 * (t & 15)))
+                                     : make_float4(0.f, 0.f, 0.f, 0.f);
+                }
             }
-        }
-    };
-    if (nq > 0) load(0, 0);
-    if (nq > 1) load(1, 1);
-    int last = -1;
-    bool stop = false;
-    for (int q0 = 0; q0 < nq && !stop; q0 += 2) {
+        };
+        if (nq > 0) load(0, 0);
+        if (nq > 1) load(1, 1);
+        bool stop = false;
+        for (int q0 = 0; q0 < nq && !stop; q0 += 2) {
 #pragma unroll
-        for (int b = 0; b < 2; ++b) {
-            const int q = q0 + b;
-            if (q >= nq || stop) break;
-            if (q >= 2) {  // slot b was read by the MMAs of chunk q - 2
-                if (!mbar_wait(&bar_m[b], ((q - 2) >> 1) & 1)) atomicOr(abort_flag, 1);
-                __syncthreads();
-                if (*abort_flag) {
+            for (int b = 0; b < 2; ++b) {
+                const int q = q0 + b;
+                // warp-uniform decisions: the hand-over below synchronises the warp
+                if (q >= nq || __any_sync(0xffffffffu, *abort_flag != 0)) {
                     stop = true;
                     break;
                 }
-            }
-#pragma unroll
-            for (int j = 0; j < 2; ++j) {
-                const int i = t + kGwThreads * j, grp = i & 63;
-                st_block(a_half(b, 0, grp >> 5), a_half(b, 1, grp >> 5), 4 * (grp & 31), i >> 6, g[b][j]);
-            }
-            if (t < 128) st_block(b_half(b, 0), b_half(b, 1), 4 * (t & 15), t >> 4, hv[b]);
-            if (q + 2 < nq) load(b, q + 2);  // in flight while this chunk is multiplied
-            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-            asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-            __syncthreads();
-            if (t == 0) {
-                asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-                const uint32_t idesc = instr_desc(kHidden);  // M = 128, N = 64, both K-major
-                for (int s = 0; s < kGwEdges / 8; ++s) {
-                    for (int mt = 0; mt < n_tiles; ++mt) {
-                        // A_hi B_hi + A_hi B_lo + A_lo B_hi
-                        const uint32_t A[3] = {smem_u32(a_half(b, 0, mt)), smem_u32(a_half(b, 0, mt)),
-                                               smem_u32(a_half(b, 1, mt))};
-                        const uint32_t B[3] = {smem_u32(b_half(b, 0)), smem_u32(b_half(b, 1)),
-                                               smem_u32(b_half(b, 0))};
-                        for (int p = 0; p < 3; ++p) {
-                            const uint64_t da = smem_desc_gw(A[p] + s * 2 * kLBO);
-                            const uint64_t db = smem_desc_gw(B[p] + s * 2 * kLBO);
-                            const uint32_t acc = (q | s | p) ? 1u : 0u;
-                            asm volatile(
-                                "{\n .reg .pred pp;\n setp.ne.b32 pp, %4, 0;\n"
-                                " tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, pp;\n}" ::"r"(
-                                    tmem + (uint32_t)(mt * kHidden)),
-                                "l"(da), "l"(db), "r"(idesc), "r"(acc)
-                                : "memory");
-                        }
-                    }
+                if (q >= 2 && !__all_sync(0xffffffffu, mbar_wait(&empty[b], ((q - 2) >> 1) & 1))) {
+                    if (lane == 0) atomicOr((int*)abort_flag, 1);  // slot b still read by chunk q - 2
+                    stop = true;
+                    break;
                 }
-                asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                                 smem_u32(&bar_m[b]))
-                             : "memory");
-                last = q;
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    const int i = t + kProducers * j, grp = i & 63;
+                    st_block(a_half(b, 0, grp >> 5), a_half(b, 1, grp >> 5), 4 * (grp & 31), i >> 6, g[b][j]);
+                }
+                if (t < 128) st_block(b_half(b, 0), b_half(b, 1), 4 * (t & 15), t >> 4, hv[b]);
+                if (q + 2 < nq) load(b, q + 2);  // in flight while this chunk is multiplied
+                hand_over(&full[b], lane);
             }
+        }
+    } else if (lane == 0) {  // the MMA warp
+        const uint32_t idesc = instr_desc(kHidden);  // M = 128, N = 64, both K-major
+        for (int q = 0; q < nq; ++q) {
+            const int b = q & 1;
+            if (*abort_flag) break;
+            if (!mbar_wait(&full[b], (q >> 1) & 1)) {
+                atomicOr((int*)abort_flag, 1);
+                break;
+            }
+            asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+            for (int s = 0; s < kGwEdges / 8; ++s)
+                for (int mt = 0; mt < n_tiles; ++mt) {
+                    // A_hi B_hi + A_hi B_lo + A_lo B_hi
+                    const uint32_t A[3] = {smem_u32(a_half(b, 0, mt)), smem_u32(a_half(b, 0, mt)),
+                                           smem_u32(a_half(b, 1, mt))};
+                    const uint32_t B[3] = {smem_u32(b_half(b, 0)), smem_u32(b_half(b, 1)), smem_u32(b_half(b, 0))};
+                    for (int p = 0; p < 3; ++p)
+                        mma_tf32(tmem + (uint32_t)(mt * kHidden), smem_desc_bo(A[p] + s * 2 * kLBO, kLBO, kGwSBO),
+                                 smem_desc_bo(B[p] + s * 2 * kLBO, kLBO, kGwSBO), idesc, (q | s | p) ? 1u : 0u);
+                }
+            mma_commit(&empty[b]);
+            last = q;
         }
     }
     // all MMAs are complete once the last chunk's are
-    if (!*abort_flag && nq > 0 && !mbar_wait(&bar_m[(nq - 1) & 1], ((nq - 1) >> 1) & 1)) atomicOr(abort_flag, 1);
+    if (warp < kProducers / 32 && !*abort_flag && nq > 0 && !mbar_wait(&empty[(nq - 1) & 1], ((nq - 1) >> 1) & 1))
+        atomicOr((int*)abort_flag, 1);
     __syncthreads();
     const int mt = warp >> 2, pc = pc0 + mt * kRows + (warp & 3) * 32 + lane;
-    if (!*abort_flag && mt < n_tiles) {
+    if (!*abort_flag && warp < kProducers / 32 && mt < n_tiles) {
         float* out = part + (size_t)blockIdx.y * kHidden * PC;
         if (nq == 0) {  // an empty split contributes zeros
             if (pc < PC)
@@ -708,9 +775,9 @@ __global__ void __launch_bounds__(kGwThreads, 1)
         }
     }
     __syncthreads();
-    if (t == 0 && *abort_flag) {
-        atomicOr(&g_fault, 1);
-        if (last >= 0) mbar_wait(&bar_m[last & 1], (last >> 1) & 1);  // nothing left in flight on freed TMEM
+    if (*abort_flag) {
+        if (t == 0) atomicOr(&g_fault, 1);
+        if (t == kProducers && last >= 0) mbar_wait(&empty[last & 1], (last >> 1) & 1);  // nothing left in flight
     }
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
     __syncthreads();
@@ -737,7 +804,7 @@ cudaError_t radial_tc_grad_w2(int E, int PC, const float* grad_w, const float* H
                                            (int)rtc::kGwSmem);
     if (err != cudaSuccess) return err;
     dim3 grid((PC + rtc::kGwCols - 1) / rtc::kGwCols, splits);
-    rtc::radial_tc_grad_w2<<<grid, rtc::kGwThreads, rtc::kGwSmem, s>>>(E, PC, per, grad_w, H, part);
+    rtc::radial_tc_grad_w2<<<grid, rtc::kPipeThreads, rtc::kGwSmem, s>>>(E, PC, per, grad_w, H, part);
     return cudaGetLastError();
 }
 
@@ -781,7 +848,7 @@ cudaError_t radial_tc_backward(int E, int PC, float rc, const float* r, const fl
     cudaError_t err = cudaFuncSetAttribute(rtc::radial_tc_backward, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                            (int)rtc::kBwSmem);
     if (err != cudaSuccess) return err;
-    rtc::radial_tc_backward<<<(E + rtc::kRows - 1) / rtc::kRows, rtc::kThreads, rtc::kBwSmem, s>>>(
+    rtc::radial_tc_backward<<<(E + rtc::kRows - 1) / rtc::kRows, rtc::kPipeThreads, rtc::kBwSmem, s>>>(
         E, PC, rc, r, W1, hi, lo, grad_w, gZ, grad_r);
     return cudaGetLastError();
 }
