@@ -1,4 +1,5 @@
-"""FP64 CPU oracle for the edge-wise equivariant tensor product and its VJP.
+"""FP64 CPU oracle for the edge-wise equivariant tensor product, its VJP and the
+VJP of its VJP (double backward).
 
 TEST INFRASTRUCTURE ONLY. Only ``tests/``, ``__graft_entry__.smoke()`` and the
 CPU-baseline leg of ``bench.py`` may import, call, link or execute anything under
@@ -190,4 +191,86 @@ class OracleTP:
                 res["grad_w"] = gw
             if gr is not None:
                 res["grad_r"] = gr
+        return res
+
+
+    def double_backward(self, row_ptr, src, r, x, w, g, gg_x=None, gg_w=None, gg_r=None) -> dict:
+        """VJP of the VJP: the gradients of <gg_x, grad_x> + <gg_w, grad_w> + <gg_r, grad_r>
+        with respect to g, x, w and r, where (grad_x, grad_w, grad_r) = VJP(x, w, r; g).
+
+        Force-loss training differentiates the forces (built from grad_r) with respect to
+        the parameters, which takes this second-order product; FlashCart times it beside the
+        forward and the VJP ("FlashCart 如何让等变原子间势更快更准?", section
+        "生成内核在高阶下胜过球谐基线"). Written out from the definition: the tensor product
+        is linear in each of x, w, g and Y, so every term is one of the first-order loops
+        with one input replaced by its cotangent. With Ydot[e] = dY/dr[e] . gg_r[e] (the
+        directional derivative of the harmonics) and Hg[e] = d2Y/dr2[e] . gg_r[e]:
+
+            grad_g = fwd(x <- gg_x) + fwd(w <- gg_w) + fwd(Y <- Ydot)
+            grad_x = vjp_x(w <- gg_w) + vjp_x(Y <- Ydot)
+            grad_w = vjp_w(x <- gg_x) + vjp_w(Y <- Ydot)
+            grad_r = vjp_r(x <- gg_x) + vjp_r(w <- gg_w) + vjp_r(dY/dr <- Hg)
+
+        A cotangent given as None is zero. Everything in FP64; returns grad_g [N, d_out, C],
+        grad_x [N, d_in, C], grad_w [E, P, C], grad_r [E, 3].
+        """
+        lib = _load()
+        f64 = lambda a: np.ascontiguousarray(a, dtype=np.float64)
+        n = len(row_ptr) - 1
+        row_ptr = np.ascontiguousarray(row_ptr, dtype=np.int32)
+        src = np.ascontiguousarray(src, dtype=np.int32)
+        r, x, w, g = f64(r), f64(x), f64(w), f64(g)
+        self._check(n, row_ptr, src, r, x, w)
+        assert g.shape == (n, self.d_out, self.C)
+        E = len(src)
+        rev_ptr, rev_perm, dst = reverse_csr(n, row_ptr, src)
+        nodes = np.arange(n, dtype=np.int64)
+        edges = np.arange(E, dtype=np.int64)
+        Y = f64(sh_mod.sh(self.sh_lmax, r))
+        dY = f64(sh_mod.sh_grad(self.sh_lmax, r))
+        none = np.zeros((1,), dtype=np.float64)
+
+        def fwd(Ya, xa, wa):
+            out = np.zeros((n, self.d_out, self.C), dtype=np.float64)
+            lib.oracle_forward_f64(ctypes.c_int64(n), _p(nodes), _p(row_ptr), _p(src), *self._tables(),
+                                   _p(Ya), _p(xa), _p(wa), _p(out))
+            return out
+
+        def vjp_x(Ya, wa):
+            gx = np.zeros((n, self.d_in, self.C), dtype=np.float64)
+            lib.oracle_grad_x_f64(ctypes.c_int64(n), _p(nodes), _p(rev_ptr), _p(rev_perm), _p(dst), *self._tables(),
+                                  _p(Ya), _p(wa), _p(g), _p(gx))
+            return gx
+
+        def vjp_wr(Ya, dYa, xa, wa, want_w, want_r):
+            gw = np.zeros((E, self.P, self.C), dtype=np.float64) if want_w else None
+            gr = np.zeros((E, 3), dtype=np.float64) if want_r else None
+            lib.oracle_grad_wr_f64(ctypes.c_int64(E), _p(edges), _p(src), _p(dst), *self._tables(),
+                                   _p(Ya), _p(dYa if dYa is not None else none), _p(xa), _p(wa), _p(g), _p(gw), _p(gr))
+            return gw, gr
+
+        res = {"grad_g": np.zeros((n, self.d_out, self.C)), "grad_x": np.zeros((n, self.d_in, self.C)),
+               "grad_w": np.zeros((E, self.P, self.C)), "grad_r": np.zeros((E, 3))}
+        if gg_x is not None:
+            gg_x = f64(gg_x)
+            assert gg_x.shape == x.shape
+            res["grad_g"] += fwd(Y, gg_x, w)
+            gw, gr = vjp_wr(Y, dY, gg_x, w, True, True)
+            res["grad_w"] += gw
+            res["grad_r"] += gr
+        if gg_w is not None:
+            gg_w = f64(gg_w)
+            assert gg_w.shape == w.shape
+            res["grad_g"] += fwd(Y, x, gg_w)
+            res["grad_x"] += vjp_x(Y, gg_w)
+            res["grad_r"] += vjp_wr(Y, dY, x, gg_w, False, True)[1]
+        if gg_r is not None:
+            gg_r = f64(gg_r)
+            assert gg_r.shape == (E, 3)
+            Ydot = f64(np.einsum("eka,ea->ek", dY, gg_r))
+            Hg = f64(np.einsum("ekab,eb->eka", sh_mod.sh_hess(self.sh_lmax, r), gg_r))
+            res["grad_g"] += fwd(Ydot, x, w)
+            res["grad_x"] += vjp_x(Ydot, w)
+            res["grad_w"] += vjp_wr(Ydot, None, x, w, True, False)[0]
+            res["grad_r"] += vjp_wr(Y, Hg, x, w, False, True)[1]
         return res

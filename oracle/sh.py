@@ -105,6 +105,25 @@ def _eval_poly_grad(terms: dict, u: np.ndarray) -> np.ndarray:
     return g
 
 
+def _eval_poly_hess(terms: dict, u: np.ndarray) -> np.ndarray:
+    """Second derivatives of the polynomial in u, shape [..., 3, 3]."""
+    h = np.zeros(u.shape + (3,))
+    for p, c in terms.items():
+        for a in range(3):
+            for b in range(3):
+                q = list(p)
+                f = q[a]
+                q[a] -= 1
+                if f == 0 or q[a] < 0:
+                    continue
+                f2 = q[b]
+                q[b] -= 1
+                if f2 == 0 or q[b] < 0:
+                    continue
+                h[..., a, b] += c * f * f2 * u[..., 0] ** q[0] * u[..., 1] ** q[1] * u[..., 2] ** q[2]
+    return h
+
+
 def sh_block(l: int, r: np.ndarray) -> np.ndarray:
     """Y_l(r/|r|), shape [..., 2l+1]."""
     r = np.asarray(r, dtype=np.float64)
@@ -140,3 +159,34 @@ def sh_grad(lmax: int, r: np.ndarray) -> np.ndarray:
             d[~ok] = 0.0
             blocks.append(d)
     return np.stack(blocks, axis=-2)
+
+
+def sh_hess(lmax: int, r: np.ndarray) -> np.ndarray:
+    """d^2 Y_k / dr_a dr_b for the unnormalised vector r, shape [..., (lmax+1)^2, 3, 3].
+
+    With u = r/n, n = |r|, P = I - u u^T, g = grad_u p(u) and K = the polynomial's
+    second derivatives at u, the chain rule through u (du/dr = P / n) gives
+
+        H = ( P K P - (u . g) P - u (P g)^T - (P g) u^T ) / n^2,
+
+    symmetric in (a, b). Edges shorter than R_EPS give 0.
+    """
+    r = np.asarray(r, dtype=np.float64)
+    n = np.linalg.norm(r, axis=-1)
+    ok = n >= R_EPS
+    safe = np.where(ok, n, 1.0)
+    u = np.where(ok[..., None], r / safe[..., None], 0.0)
+    proj = np.eye(3) - u[..., :, None] * u[..., None, :]
+    blocks = []
+    for l in range(lmax + 1):
+        for t in sh_monomials(l):
+            g = _eval_poly_grad(t, u)
+            K = _eval_poly_hess(t, u)
+            pg = np.einsum("...ab,...b->...a", proj, g)
+            ug = np.einsum("...a,...a->...", u, g)
+            H = (np.einsum("...ac,...cd,...db->...ab", proj, K, proj) - ug[..., None, None] * proj
+                 - u[..., :, None] * pg[..., None, :] - pg[..., :, None] * u[..., None, :])
+            H = H / (safe**2)[..., None, None]
+            H[~ok] = 0.0
+            blocks.append(H)
+    return np.stack(blocks, axis=-3)
