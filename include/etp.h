@@ -178,8 +178,11 @@ ETP_API etp_status etp_backward(etp_plan_t plan, int N, int E, const int32_t* ro
  *   w[e] = SiLU(b(d_e) W1) W2,   SiLU(z) = z / (1 + exp(-z)),   no biases, no envelope,
  * W1: float32 [n_basis][hidden], W2: float32 [hidden][P*C] (row-major), w: float32
  * [E][P][C] as etp_forward takes it. 1 <= n_basis <= 32; hidden a multiple of 32 in
- * [32, 256]; r_cut > 0. The dense products run in FP32 (exact FMAs); every sum over
- * edges is taken in a fixed order (results repeat bit for bit).
+ * [32, 256]; r_cut > 0. With n_basis = 8, hidden = 64 and P*C a multiple of 16 the
+ * dense products run on the tensor cores, each FP32 product as three TF32 products
+ * (hi*hi + hi*lo + lo*hi of the operands' TF32 halves: relative error near 2^-21);
+ * otherwise as FP32 FMAs. Every sum over edges is taken in a fixed order (results
+ * repeat bit for bit).
  * workspace: device memory of etp_radial_workspace_size bytes, 16-byte aligned,
  * owned by the caller. */
 ETP_API etp_status etp_radial_workspace_size(etp_plan_t plan, int E, int n_basis, int hidden, size_t* bytes);
