@@ -19,6 +19,8 @@
 //   3. the 4 warps read the accumulator back (tcgen05.ld, warp w owns TMEM lanes
 //      32w..32w+31, i.e. edges), stage it in shared memory and store w in whole
 //      row segments.
+// The VJP's two dense products, dL/dH = grad_w W2^T and grad_W2 = H^T grad_w, follow
+// below as warp-specialised kernels with the same operand layout and split.
 // Every wait is bounded; on time-out the kernel raises its fault flag and leaves.
 #include <cuda_runtime.h>
 
