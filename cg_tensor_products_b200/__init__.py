@@ -89,14 +89,8 @@ def _ptr(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
-def _stream(stream):
-    import torch
-
-    s = stream if stream is not None else torch.cuda.current_stream()
-    return ctypes.c_void_p(s.cuda_stream)
-
-
 def _need_cuda(*ts):
+    """The one CUDA device all given tensors live on (None entries are skipped)."""
     dev = None
     for t in ts:
         if t is None:
@@ -109,6 +103,22 @@ def _need_cuda(*ts):
             dev = t.device
         elif t.device != dev:
             raise ValueError(f"tensors on different devices ({dev}, {t.device})")
+    return dev
+
+
+def _launch(dev, where: str, fn, *args, stream=None):
+    """Call library function `fn(*args, stream)` with the tensors' device current.
+
+    The library launches on the current device and on the stream it is given, so
+    both must be the tensors' device: torch's current stream of `dev`, or a
+    caller's stream, which must belong to `dev`."""
+    import torch
+
+    s = stream if stream is not None else torch.cuda.current_stream(dev)
+    if s.device != dev:
+        raise ValueError(f"{where}: stream on {s.device}, tensors on {dev}")
+    with torch.cuda.device(dev):
+        _check(fn(*args, ctypes.c_void_p(s.cuda_stream)), where)
 
 
 def _expect(t, name: str, dtype: str, shape: tuple):
@@ -183,8 +193,8 @@ def edge_frames(plan: Plan, r, frames=None, stream=None):
     if frames is None:
         frames = torch.empty((E, FRAME_FLOATS), device=r.device, dtype=torch.float32)
     _expect(frames, "frames", "float32", (E, FRAME_FLOATS))
-    _need_cuda(r, frames)
-    _check(_load().etp_edge_frames(plan.handle, E, _ptr(r), _ptr(frames), _stream(stream)), "etp_edge_frames")
+    dev = _need_cuda(r, frames)
+    _launch(dev, "etp_edge_frames", _load().etp_edge_frames, plan.handle, E, _ptr(r), _ptr(frames), stream=stream)
     return frames
 
 
@@ -202,9 +212,9 @@ def forward(plan: Plan, row_ptr, src, r, x, w, out=None, frames=None, stream=Non
     if out is None:
         out = torch.empty((N, plan.dim_out, plan.C), device=x.device, dtype=torch.float32)
     _expect(out, "out", "float32", (N, plan.dim_out, plan.C))
-    _need_cuda(row_ptr, src, r, frames, x, w, out)
-    _check(_load().etp_forward(plan.handle, N, E, _ptr(row_ptr), _ptr(src), _ptr(r), _ptr(frames), _ptr(x), _ptr(w),
-                               _ptr(out), _stream(stream)), "etp_forward")
+    dev = _need_cuda(row_ptr, src, r, frames, x, w, out)
+    _launch(dev, "etp_forward", _load().etp_forward, plan.handle, N, E, _ptr(row_ptr), _ptr(src), _ptr(r),
+            _ptr(frames), _ptr(x), _ptr(w), _ptr(out), stream=stream)
     return out
 
 
@@ -233,10 +243,10 @@ def backward(plan: Plan, row_ptr, src, rev_ptr, rev_perm, dst, r, x, w, grad_out
     _expect(grad_x, "grad_x", "float32", (N, plan.dim_in, plan.C))
     _expect(grad_w, "grad_w", "float32", (E, plan.n_paths, plan.C))
     _expect(grad_r, "grad_r", "float32", (E, 3))
-    _need_cuda(row_ptr, src, rev_ptr, rev_perm, dst, r, frames, x, w, grad_out, grad_x, grad_w, grad_r)
-    _check(_load().etp_backward(plan.handle, N, E, _ptr(row_ptr), _ptr(src), _ptr(rev_ptr), _ptr(rev_perm),
-                                _ptr(dst), _ptr(r), _ptr(frames), _ptr(x), _ptr(w), _ptr(grad_out), _ptr(grad_x),
-                                _ptr(grad_w), _ptr(grad_r), _stream(stream)), "etp_backward")
+    dev = _need_cuda(row_ptr, src, rev_ptr, rev_perm, dst, r, frames, x, w, grad_out, grad_x, grad_w, grad_r)
+    _launch(dev, "etp_backward", _load().etp_backward, plan.handle, N, E, _ptr(row_ptr), _ptr(src), _ptr(rev_ptr),
+            _ptr(rev_perm), _ptr(dst), _ptr(r), _ptr(frames), _ptr(x), _ptr(w), _ptr(grad_out), _ptr(grad_x),
+            _ptr(grad_w), _ptr(grad_r), stream=stream)
     return grad_x, grad_w, grad_r
 
 
@@ -259,10 +269,9 @@ def assemble_forces(N: int, row_ptr, rev_ptr, rev_perm, grad_r, r=None, forces=N
     _expect(forces, "forces", "float32", (N, 3))
     if virial is not None and (str(virial.dtype) != "torch.float32" or virial.numel() != 9 * N):
         raise ValueError("virial: expected float32 with N*9 elements")
-    _need_cuda(row_ptr, rev_ptr, rev_perm, grad_r, r, forces, virial)
-    _check(_load().etp_assemble_forces(int(N), int(E), _ptr(row_ptr), _ptr(rev_ptr), _ptr(rev_perm), _ptr(r),
-                                       _ptr(grad_r), _ptr(forces), _ptr(virial), _stream(stream)),
-           "etp_assemble_forces")
+    dev = _need_cuda(row_ptr, rev_ptr, rev_perm, grad_r, r, forces, virial)
+    _launch(dev, "etp_assemble_forces", _load().etp_assemble_forces, int(N), int(E), _ptr(row_ptr), _ptr(rev_ptr),
+            _ptr(rev_perm), _ptr(r), _ptr(grad_r), _ptr(forces), _ptr(virial), stream=stream)
     return forces, virial
 
 
@@ -295,10 +304,9 @@ def radial_forward(plan: Plan, r, W1, W2, r_cut: float, w=None, workspace=None, 
         w = torch.empty((E, plan.n_paths, plan.C), device=r.device, dtype=torch.float32)
     _expect(w, "w", "float32", (E, plan.n_paths, plan.C))
     workspace = _radial_ws(plan, E, W1, workspace)
-    _need_cuda(r, W1, W2, w, workspace)
-    _check(_load().etp_radial_forward(plan.handle, E, W1.shape[0], W1.shape[1], float(r_cut), _ptr(r), _ptr(W1),
-                                      _ptr(W2), _ptr(w), _ptr(workspace), workspace.numel(), _stream(stream)),
-           "etp_radial_forward")
+    dev = _need_cuda(r, W1, W2, w, workspace)
+    _launch(dev, "etp_radial_forward", _load().etp_radial_forward, plan.handle, E, W1.shape[0], W1.shape[1],
+            float(r_cut), _ptr(r), _ptr(W1), _ptr(W2), _ptr(w), _ptr(workspace), workspace.numel(), stream=stream)
     return w
 
 
@@ -320,10 +328,10 @@ def radial_backward(plan: Plan, r, W1, W2, r_cut: float, grad_w, grad_r, grad_W1
     _expect(grad_W1, "grad_W1", "float32", tuple(W1.shape))
     _expect(grad_W2, "grad_W2", "float32", tuple(W2.shape))
     workspace = _radial_ws(plan, E, W1, workspace)
-    _need_cuda(r, W1, W2, grad_w, grad_r, grad_W1, grad_W2, workspace)
-    _check(_load().etp_radial_backward(plan.handle, E, W1.shape[0], W1.shape[1], float(r_cut), _ptr(r), _ptr(W1),
-                                       _ptr(W2), _ptr(grad_w), _ptr(grad_W1), _ptr(grad_W2), _ptr(grad_r),
-                                       _ptr(workspace), workspace.numel(), _stream(stream)), "etp_radial_backward")
+    dev = _need_cuda(r, W1, W2, grad_w, grad_r, grad_W1, grad_W2, workspace)
+    _launch(dev, "etp_radial_backward", _load().etp_radial_backward, plan.handle, E, W1.shape[0], W1.shape[1],
+            float(r_cut), _ptr(r), _ptr(W1), _ptr(W2), _ptr(grad_w), _ptr(grad_W1), _ptr(grad_W2), _ptr(grad_r),
+            _ptr(workspace), workspace.numel(), stream=stream)
     return grad_W1, grad_W2
 
 
@@ -347,10 +355,9 @@ def build_reverse_csr(N: int, row_ptr, src, with_dst=True, workspace=None, strea
     if workspace is None:
         workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=dev)
     _expect(workspace, "workspace", "uint8", (None,))
-    _need_cuda(row_ptr, src, rev_ptr, rev_perm, dst, workspace)
-    _check(_load().etp_build_reverse_csr(N, E, _ptr(row_ptr), _ptr(src), _ptr(rev_ptr), _ptr(rev_perm), _ptr(dst),
-                                         _ptr(workspace), workspace.numel(), _stream(stream)),
-           "etp_build_reverse_csr")
+    dev = _need_cuda(row_ptr, src, rev_ptr, rev_perm, dst, workspace)
+    _launch(dev, "etp_build_reverse_csr", _load().etp_build_reverse_csr, N, E, _ptr(row_ptr), _ptr(src),
+            _ptr(rev_ptr), _ptr(rev_perm), _ptr(dst), _ptr(workspace), workspace.numel(), stream=stream)
     return rev_ptr, rev_perm, dst
 
 
@@ -365,9 +372,9 @@ def build_reverse_csr_static(N: int, row_ptr, src, with_dst=True, stream=None):
     rev_ptr = torch.empty(N + 1, dtype=torch.int32, device=dev)
     rev_perm = torch.empty(E, dtype=torch.int32, device=dev)
     dst = torch.empty(E, dtype=torch.int32, device=dev) if with_dst else None
-    _need_cuda(row_ptr, src, rev_ptr, rev_perm, dst)
-    _check(_load().etp_build_reverse_csr_static(N, E, _ptr(row_ptr), _ptr(src), _ptr(rev_ptr), _ptr(rev_perm),
-                                                _ptr(dst), _stream(stream)), "etp_build_reverse_csr_static")
+    dev = _need_cuda(row_ptr, src, rev_ptr, rev_perm, dst)
+    _launch(dev, "etp_build_reverse_csr_static", _load().etp_build_reverse_csr_static, N, E, _ptr(row_ptr),
+            _ptr(src), _ptr(rev_ptr), _ptr(rev_perm), _ptr(dst), stream=stream)
     return rev_ptr, rev_perm, dst
 
 
@@ -384,7 +391,7 @@ def validate_csr(N: int, row_ptr, src, stream=None) -> int:
 
     _check_graph(row_ptr, src, N, src.numel())
     flag = torch.empty(1, dtype=torch.int32, device=row_ptr.device)
-    _need_cuda(row_ptr, src, flag)
-    _check(_load().etp_validate_csr(N, src.numel(), _ptr(row_ptr), _ptr(src), _ptr(flag), _stream(stream)),
-           "etp_validate_csr")
+    dev = _need_cuda(row_ptr, src, flag)
+    _launch(dev, "etp_validate_csr", _load().etp_validate_csr, N, src.numel(), _ptr(row_ptr), _ptr(src),
+            _ptr(flag), stream=stream)
     return int(flag.item())

@@ -894,6 +894,9 @@ __global__ void __launch_bounds__(frame::kThreads, L <= 2 ? 6 : 4) etp_bwd_frame
 
     int row = segment_of(a.rev_ptr, a.N, k0);  // source node of position k0
     int row_lo = __ldg(a.rev_ptr + row), row_hi = __ldg(a.rev_ptr + row + 1);
+    // positions from rev_ptr[N] on hold the edges whose source is out of range (an
+    // invalid CSR): they contribute nothing and get zero grad_w and grad_r
+    const int pos_end = __ldg(a.rev_ptr + a.N);
     // the edge of the next position and the destination and vector of the next
     // edge are loaded an edge early (the position after next: two early)
     int e_cur = edge_at(k0);
@@ -938,7 +941,7 @@ __global__ void __launch_bounds__(frame::kThreads, L <= 2 ? 6 : 4) etp_bwd_frame
         const int e_after = q + 2 < k1 ? edge_at(q + 2) : 0;
         const int i_next = has_next ? dst_of(e_next) : 0;
         const float3 r_next = (!FR && has_next) ? load_r(a.r, valid_edge(e_next) ? e_next : 0) : r_cur;
-        const bool ok = valid_edge(e_cur) && (unsigned)i_cur < (unsigned)a.N;
+        const bool ok = valid_edge(e_cur) && (unsigned)i_cur < (unsigned)a.N && q < pos_end;
         Frame f;
         if constexpr (FR) {
             cp_async_wait_all();  // this edge's node rows (this lane's copies)
@@ -953,7 +956,7 @@ __global__ void __launch_bounds__(frame::kThreads, L <= 2 ? 6 : 4) etp_bwd_frame
             mbar_wait(&bar[slot], (it >> 1) & 1, live);
         }
         const float2* ws = reinterpret_cast<const float2*>(wbuf + slot * P * C) + cp;
-        float2* gwe = (want_w && ok) ? gw2 + (size_t)e_cur * P * C2 + cp : nullptr;
+        float2* gwe = (want_w && valid_edge(e_cur)) ? gw2 + (size_t)e_cur * P * C2 + cp : nullptr;
         float2 sx2 = f2_zero(), sy2 = f2_zero();  // dL/de_x, dL/de_y per channel of this lane
         if (ok && !f.degenerate) {
             float2 xp[D], gpa[D], z[D];
@@ -1054,6 +1057,8 @@ __global__ void __launch_bounds__(frame::kThreads, L <= 2 ? 6 : 4) etp_bwd_frame
                         if constexpr (pt.l2 > 0) st_stream2(gwe + p * C2, f2_zero(), pol_w);
                     });
                 }
+            } else if (gwe) {
+                static_for<0, P>([&](auto pc) { st_stream2(gwe + decltype(pc)::value * C2, f2_zero(), pol_w); });
             }
             if (has_next && row_next != row) copy_x(row_next);
             if (has_next) copy_g(i_next);
@@ -1072,7 +1077,7 @@ __global__ void __launch_bounds__(frame::kThreads, L <= 2 ? 6 : 4) etp_bwd_frame
             }
         }
         group_sync();  // weight buffer free for the edge after next; slice partials visible
-        if (want_r && ok && G.slice == 0 && G.tl == 0) {
+        if (want_r && valid_edge(e_cur) && G.slice == 0 && G.tl == 0) {  // zero when !ok (sx = sy = 0)
             if (G.S == 2) {
                 sx += comb[(it & 1) * 2];
                 sy += comb[(it & 1) * 2 + 1];

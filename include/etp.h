@@ -162,7 +162,8 @@ ETP_API etp_status etp_forward(etp_plan_t plan, int N, int E, const int32_t* row
  * is found by binary search in row_ptr). frames: as in etp_forward (with
  * frames, r is not read and may be NULL). Each of grad_x, grad_w, grad_r may be
  * NULL to skip it. All outputs are overwritten (sources without edges get zero
- * grad_x). */
+ * grad_x). An edge whose source or row is out of range (a CSR that
+ * etp_validate_csr flags) adds nothing to grad_x and gets zero grad_w and grad_r. */
 ETP_API etp_status etp_backward(etp_plan_t plan, int N, int E, const int32_t* row_ptr, const int32_t* src,
                         const int32_t* rev_ptr, const int32_t* rev_perm, const int32_t* dst_of_edge,
                         const float* r, const float* frames, const float* x, const float* w,
@@ -247,7 +248,9 @@ ETP_API etp_status etp_build_reverse_csr(int N, int E, const int32_t* row_ptr, c
  * E > ETP_STATIC_MAX_EDGES returns ETP_ERR_TOO_LARGE before any launch. The
  * first call on a device (the current device) looks up the array's device
  * address for that device; make that first call before any stream capture on
- * it. All calls share the one array: calls whose work overlaps on the GPU
+ * it. The address is kept for the life of the process: after cudaDeviceReset
+ * (or any other teardown of the device's primary context) this call must not be
+ * used on that device again. All calls share the one array: calls whose work overlaps on the GPU
  * (unordered streams or threads) race and give wrong results; calls ordered on
  * one stream are safe. */
 ETP_API etp_status etp_build_reverse_csr_static(int N, int E, const int32_t* row_ptr, const int32_t* src,

@@ -197,7 +197,8 @@ def test_validate_csr_flags():
 
 
 def test_out_of_range_sources_are_skipped_not_faulted():
-    """An invalid src (caught by validate_csr) must not make the kernels leave their buffers."""
+    """An invalid src (caught by validate_csr) must not make the kernels leave their buffers;
+    such edges contribute nothing, and their grad_w and grad_r are zero."""
     rng = np.random.default_rng(6)
     wl = workloads.random_graph(rng, 16, 100, 1, 8, 5)
     t = to_dev(wl)
@@ -212,8 +213,20 @@ def test_out_of_range_sources_are_skipped_not_faulted():
     # the same graph with those edges given zero weight is the reference
     w0 = wl.w.copy()
     w0[~keep] = 0
-    ref = oracle.OracleTP("0..1", 1, "0..1", 8).forward(wl.row_ptr, wl.src, wl.r, wl.x, w0)
+    tp = oracle.OracleTP("0..1", 1, "0..1", 8)
+    ref = tp.forward(wl.row_ptr, wl.src, wl.r, wl.x, w0)
     assert rel_err(out, ref) <= 1e-5
+    # the VJP: those edges add nothing to grad_x and get zero grad_w and grad_r
+    rev_ptr, rev_perm, dst = etp.build_reverse_csr(wl.N, t["row_ptr"], bad_src)
+    gx, gw, gr = etp.backward(plan, t["row_ptr"], bad_src, rev_ptr, rev_perm, dst, t["r"], t["x"], t["w"], t["g"])
+    torch.cuda.synchronize()
+    assert etp.device_fault() == 0
+    ref_b = tp.backward(wl.row_ptr, wl.src, wl.r, wl.x, w0, wl.g)
+    bad = torch.from_numpy(~keep).cuda()
+    assert torch.count_nonzero(gw[bad]) == 0 and torch.count_nonzero(gr[bad]) == 0
+    assert rel_err(gx, ref_b["grad_x"]) <= 1e-4
+    assert rel_err(gw[~bad], ref_b["grad_w"][keep]) <= 1e-4
+    assert rel_err(gr[~bad], ref_b["grad_r"][keep]) <= 1e-4
 
 
 @pytest.mark.parametrize("L", [0, 1, 2, 3])

@@ -67,6 +67,28 @@ def test_static_scratch_matches_workspace_version_twice(lib):
         assert torch.equal(a, b)
 
 
+@pytest.mark.parametrize("n,e,with_dst", [(1, 5, True), (7, 0, True), (300, 4000, False), (1, 1, False)])
+def test_static_scratch_small_and_degenerate_graphs(lib, n, e, with_dst):
+    """Cases only the fixed-scratch path reaches: one source (every edge has source 0,
+    no radix pass), no edges at all, and no dst output requested. Compared bit for bit
+    with the oracle's reverse CSR."""
+    import oracle
+
+    rng = np.random.default_rng(n * 131 + e)
+    row_ptr, src, _ = workloads.csr_from_pairs(n, rng.integers(0, n, e), rng.integers(0, n, e))
+    o_rp, o_perm, o_dst = oracle.reverse_csr(n, row_ptr, src)
+    d_rp, d_src = torch.from_numpy(row_ptr).cuda(), torch.from_numpy(src).cuda()
+    for _ in range(2):
+        rev_ptr, rev_perm, dst = etp.build_reverse_csr_static(n, d_rp, d_src, with_dst=with_dst)
+        torch.cuda.synchronize()
+        assert np.array_equal(rev_ptr.cpu().numpy(), o_rp)
+        assert np.array_equal(rev_perm.cpu().numpy(), o_perm)
+        if with_dst:
+            assert np.array_equal(dst.cpu().numpy(), o_dst)
+        else:
+            assert dst is None
+
+
 def test_static_scratch_refuses_sizes_above_its_limit(lib):
     big = etp.STATIC_MAX_EDGES + 1
     st = lib.etp_build_reverse_csr_static(10, big, None, None, None, None, None, None)
