@@ -58,6 +58,8 @@ def _load():
         "etp_radial_workspace_size": [vp, i32, i32, i32, ctypes.POINTER(sz)],
         "etp_radial_forward": [vp, i32, i32, i32, ctypes.c_float, vp, vp, vp, vp, vp, sz, vp],
         "etp_radial_backward": [vp, i32, i32, i32, ctypes.c_float, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp],
+        "etp_fused_workspace_size": [vp, i32, i32, i32, ctypes.POINTER(sz)],
+        "etp_fused_forward": [vp, i32, i32, vp, vp, vp, vp, i32, i32, ctypes.c_float, vp, vp, vp, vp, sz, vp],
         "etp_reverse_csr_workspace_size": [i32, i32, ctypes.POINTER(sz)],
         "etp_build_reverse_csr": [i32, i32, vp, vp, vp, vp, vp, vp, sz, vp],
         "etp_build_reverse_csr_static": [i32, i32, vp, vp, vp, vp, vp, vp],
@@ -333,6 +335,38 @@ def radial_backward(plan: Plan, r, W1, W2, r_cut: float, grad_w, grad_r, grad_W1
             float(r_cut), _ptr(r), _ptr(W1), _ptr(W2), _ptr(grad_w), _ptr(grad_W1), _ptr(grad_W2), _ptr(grad_r),
             _ptr(workspace), workspace.numel(), stream=stream)
     return grad_W1, grad_W2
+
+
+def fused_workspace_size(plan: Plan, E: int, n_basis: int = 8, hidden: int = 64) -> int:
+    b = ctypes.c_size_t()
+    _check(_load().etp_fused_workspace_size(plan.handle, int(E), int(n_basis), int(hidden), ctypes.byref(b)),
+           "etp_fused_workspace_size")
+    return b.value
+
+
+def fused_forward(plan: Plan, row_ptr, src, r, x, W1, W2, r_cut: float, out=None, workspace=None, stream=None):
+    """out [N, D, C] = forward(plan, ..., w = radial_forward(plan, r, W1, W2, r_cut)) without storing w
+    (launches etp_fused_forward)."""
+    import torch
+
+    N, E = row_ptr.numel() - 1, src.numel()
+    _check_graph(row_ptr, src, N, E)
+    _expect(r, "r", "float32", (E, 3))
+    _expect(x, "x", "float32", (N, plan.dim_in, plan.C))
+    _expect(W1, "W1", "float32", (None, None))
+    _expect(W2, "W2", "float32", (W1.shape[1], plan.n_paths * plan.C))
+    if out is None:
+        out = torch.empty((N, plan.dim_out, plan.C), device=x.device, dtype=torch.float32)
+    _expect(out, "out", "float32", (N, plan.dim_out, plan.C))
+    nbytes = fused_workspace_size(plan, E, W1.shape[0], W1.shape[1])
+    if workspace is None:
+        workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=x.device)
+    _expect(workspace, "workspace", "uint8", (None,))
+    dev = _need_cuda(row_ptr, src, r, x, W1, W2, out, workspace)
+    _launch(dev, "etp_fused_forward", _load().etp_fused_forward, plan.handle, N, E, _ptr(row_ptr), _ptr(src),
+            _ptr(r), _ptr(x), W1.shape[0], W1.shape[1], float(r_cut), _ptr(W1), _ptr(W2), _ptr(out),
+            _ptr(workspace), workspace.numel(), stream=stream)
+    return out
 
 
 def reverse_csr_workspace_size(N: int, E: int) -> int:

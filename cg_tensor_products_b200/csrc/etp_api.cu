@@ -349,6 +349,29 @@ etp_status etp_radial_backward(etp_plan_t plan, int E, int n_basis, int hidden, 
                                             grad_W2, grad_r, workspace, reinterpret_cast<cudaStream_t>(stream)));
 }
 
+etp_status etp_fused_workspace_size(etp_plan_t plan, int E, int n_basis, int hidden, size_t* bytes) {
+    if (!plan || E < 0 || !bytes) return ETP_ERR_INVALID_ARG;
+    if (!etp::fused_supported(n_basis, hidden)) return ETP_ERR_UNSUPPORTED;
+    *bytes = etp::fused_workspace_bytes(plan->L, plan->o3, plan->C, E);
+    return ETP_OK;
+}
+
+etp_status etp_fused_forward(etp_plan_t plan, int N, int E, const int32_t* row_ptr, const int32_t* src,
+                             const float* r, const float* x, int n_basis, int hidden, float r_cut, const float* W1,
+                             const float* W2, float* out, void* workspace, size_t workspace_bytes,
+                             etp_stream_t stream) {
+    if (!plan || N < 0 || E < 0 || !(r_cut > 0.f)) return ETP_ERR_INVALID_ARG;
+    if (!etp::fused_supported(n_basis, hidden)) return ETP_ERR_UNSUPPORTED;
+    if (N == 0) return E == 0 ? ETP_OK : ETP_ERR_INVALID_ARG;
+    if (!row_ptr || !x || !out || !W1 || !W2 || !workspace || !aligned4(row_ptr) || !aligned16(x) ||
+        !aligned16(out) || !aligned4(W1) || !aligned4(W2) || !aligned16(workspace))
+        return ETP_ERR_INVALID_ARG;
+    if (E > 0 && (!src || !r || !aligned4(src) || !aligned4(r))) return ETP_ERR_INVALID_ARG;
+    if (workspace_bytes < etp::fused_workspace_bytes(plan->L, plan->o3, plan->C, E)) return ETP_ERR_WORKSPACE;
+    return cuda_status(etp::fused_forward(plan->L, plan->o3, plan->C, N, E, row_ptr, src, r, x, W1, W2, r_cut, out,
+                                          workspace, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 etp_status etp_reverse_csr_workspace_size(int N, int E, size_t* bytes) {
     if (N < 0 || E < 0 || !bytes) return ETP_ERR_INVALID_ARG;
     *bytes = etp::reverse_csr_workspace_bytes(N, E);
@@ -381,9 +404,9 @@ etp_status etp_device_fault(int* fault) {
     if (cudaDeviceSynchronize() != cudaSuccess) return ETP_ERR_CUDA;
     const int f0 = etp::read_and_clear_fault<0>(), f1 = etp::read_and_clear_fault<1>();
     const int f2 = etp::read_and_clear_fault<2>(), f3 = etp::read_and_clear_fault<3>();
-    const int f4 = etp::radial_tc_read_and_clear_fault();
-    if (f0 < 0 || f1 < 0 || f2 < 0 || f3 < 0 || f4 < 0) return ETP_ERR_CUDA;
-    *fault = f0 | f1 | f2 | f3 | f4;
+    const int f4 = etp::radial_tc_read_and_clear_fault(), f5 = etp::fused_read_and_clear_fault();
+    if (f0 < 0 || f1 < 0 || f2 < 0 || f3 < 0 || f4 < 0 || f5 < 0) return ETP_ERR_CUDA;
+    *fault = f0 | f1 | f2 | f3 | f4 | f5;
     return ETP_OK;
 }
 

@@ -604,6 +604,45 @@ __device__ __forceinline__ void expand_wigner(const float* fb, int tl, int T, un
 }
 
 // ---------------------------------------------------------------------------
+// One thread's Wigner matrices D_2 (row-major 5 x 5) and D_3 (7 x 7) of the frame
+// f, fitted from the harmonics at the rotated fixed points (zero for a degenerate
+// frame, and not computed above L).
+template <int L>
+__device__ __forceinline__ void thread_wigner(const Frame& f, float (&d2)[25], float (&d3)[49]) {
+#pragma unroll
+    for (int i = 0; i < 25; ++i) d2[i] = 0.f;
+#pragma unroll
+    for (int i = 0; i < 49; ++i) d3[i] = 0.f;
+    if constexpr (L >= 2) {
+        if (!f.degenerate) {
+#pragma unroll
+            for (int k = 0; k < 2 * L + 1; ++k) {
+                const float px = c_fit.v[3 * k], py = c_fit.v[3 * k + 1], pz = c_fit.v[3 * k + 2];
+                const float qx = f.R[0] * px + f.R[1] * py + f.R[2] * pz;
+                const float qy = f.R[3] * px + f.R[4] * py + f.R[5] * pz;
+                const float qz = f.R[6] * px + f.R[7] * py + f.R[8] * pz;
+                float Y[(L + 1) * (L + 1)];
+                sh_unit<L, float>(qx, qy, qz, Y);
+                if (k < 5) {
+#pragma unroll
+                    for (int a = 0; a < 5; ++a)
+#pragma unroll
+                        for (int b = 0; b < 5; ++b)
+                            d2[a * 5 + b] = fmaf(Y[4 + a], c_fit.v[24 + k * 7 + b], d2[a * 5 + b]);
+                }
+                if constexpr (L >= 3) {
+#pragma unroll
+                    for (int a = 0; a < 7; ++a)
+#pragma unroll
+                        for (int b = 0; b < 7; ++b)
+                            d3[a * 7 + b] = fmaf(Y[9 + a], c_fit.v[73 + k * 7 + b], d3[a * 7 + b]);
+                }
+            }
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
 // Edge frames: one thread per edge builds the edge's record (R, 1/|r|, the
 // zero-length flag, and D_2, D_3 of R fitted from the harmonics at the fixed
 // points, in the same operation order as the in-kernel build); the block's
@@ -619,37 +658,7 @@ __global__ void __launch_bounds__(kFrameBlock) etp_edge_frames_kernel(int E, con
         const float3 rv = load_r(r, e);
         const Frame f = make_frame(rv.x, rv.y, rv.z);
         float d2[25], d3[49];
-#pragma unroll
-        for (int i = 0; i < 25; ++i) d2[i] = 0.f;
-#pragma unroll
-        for (int i = 0; i < 49; ++i) d3[i] = 0.f;
-        if constexpr (L >= 2) {
-            if (!f.degenerate) {
-#pragma unroll
-                for (int k = 0; k < 2 * L + 1; ++k) {
-                    const float px = c_fit.v[3 * k], py = c_fit.v[3 * k + 1], pz = c_fit.v[3 * k + 2];
-                    const float qx = f.R[0] * px + f.R[1] * py + f.R[2] * pz;
-                    const float qy = f.R[3] * px + f.R[4] * py + f.R[5] * pz;
-                    const float qz = f.R[6] * px + f.R[7] * py + f.R[8] * pz;
-                    float Y[(L + 1) * (L + 1)];
-                    sh_unit<L, float>(qx, qy, qz, Y);
-                    if (k < 5) {
-#pragma unroll
-                        for (int a = 0; a < 5; ++a)
-#pragma unroll
-                            for (int b = 0; b < 5; ++b)
-                                d2[a * 5 + b] = fmaf(Y[4 + a], c_fit.v[24 + k * 7 + b], d2[a * 5 + b]);
-                    }
-                    if constexpr (L >= 3) {
-#pragma unroll
-                        for (int a = 0; a < 7; ++a)
-#pragma unroll
-                            for (int b = 0; b < 7; ++b)
-                                d3[a * 7 + b] = fmaf(Y[9 + a], c_fit.v[73 + k * 7 + b], d3[a * 7 + b]);
-                    }
-                }
-            }
-        }
+        thread_wigner<L>(f, d2, d3);
         float4* rec = reinterpret_cast<float4*>(stage + threadIdx.x * kFrameFloats);
         float v[kFrameFloats];
 #pragma unroll

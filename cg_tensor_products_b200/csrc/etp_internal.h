@@ -120,6 +120,14 @@ cudaError_t radial_forward(int E, int nb, int hidden, int PC, float rc, const fl
 cudaError_t radial_backward(int E, int nb, int hidden, int PC, float rc, const float* r, const float* W1,
                             const float* W2, const float* grad_w, float* grad_W1, float* grad_W2, float* grad_r,
                             void* ws, cudaStream_t s);
+// Radial weights fused into the tensor product (etp_fused.cu): n_basis 8, hidden 64.
+bool fused_supported(int nb, int hidden);
+size_t fused_workspace_bytes(int L, bool o3, int C, int E);
+size_t fused_smem_bytes(int L, bool o3, int C);
+cudaError_t fused_forward(int L, bool o3, int C, int N, int E, const int32_t* row_ptr, const int32_t* src,
+                          const float* r, const float* x, const float* W1, const float* W2, float rc, float* out,
+                          void* ws, cudaStream_t s);
+int fused_read_and_clear_fault();
 cudaError_t assemble_forces(int N, int E, const int32_t* row_ptr, const int32_t* rev_ptr, const int32_t* rev_perm,
                             const float* r, const float* grad_r, float* forces, float* virial, cudaStream_t s);
 cudaError_t validate_csr(int N, int E, const int32_t* row_ptr, const int32_t* src, int32_t* flag, cudaStream_t s);

@@ -200,6 +200,30 @@ ETP_API etp_status etp_radial_backward(etp_plan_t plan, int E, int n_basis, int 
                                        float* grad_W1, float* grad_W2, float* grad_r, void* workspace,
                                        size_t workspace_bytes, etp_stream_t stream);
 
+/* Radial weights fused into the tensor product, forward: the same result as
+ * etp_radial_forward followed by etp_forward,
+ *   out[i] = sum_{e in row i} sum_p w[e,p,:] (coupling of x[src e] with Y(r_e))_p,
+ *   w[e] = SiLU(b(|r_e|) W1) W2   (as etp_radial_forward),
+ * without the per-edge weights ever being stored: they are produced on the tensor
+ * cores 128 edges at a time (each FP32 product as three TF32 products) and read by
+ * the tensor product straight from tensor memory. ("High-performance training and
+ * inference for deep equivariant interatomic potentials", section "제안 방법": a
+ * fused tensor-product kernel without materialised intermediates, whose per-edge
+ * weights are a learned function of the edge length.)
+ * n_basis = 8 and hidden = 64 only (ETP_ERR_UNSUPPORTED otherwise); W1 [8][64],
+ * W2 [64][P*C] row-major as in etp_radial_forward; r [E][3], x [N][D][C], out
+ * [N][D][C]. workspace: device memory of etp_fused_workspace_size bytes, 16-byte
+ * aligned, owned by the caller (the rearranged W2 and per-warp carry rows),
+ * reusable once the stream has passed the call. Node sums are taken in a fixed
+ * order; a row shared by two CTAs is completed by a reduction of its two parts
+ * onto the zeroed output (bitwise repeatable while no row is longer than a CTA's
+ * range of edges, about E / number of SMs). */
+ETP_API etp_status etp_fused_workspace_size(etp_plan_t plan, int E, int n_basis, int hidden, size_t* bytes);
+ETP_API etp_status etp_fused_forward(etp_plan_t plan, int N, int E, const int32_t* row_ptr, const int32_t* src,
+                                     const float* r, const float* x, int n_basis, int hidden, float r_cut,
+                                     const float* W1, const float* W2, float* out, void* workspace,
+                                     size_t workspace_bytes, etp_stream_t stream);
+
 /* Atom forces and per-atom virials from per-edge energy derivatives.
  * The pages evaluate models on energies and forces ("FlashCart 如何让等变原子间势更快更准?",
  * section "560 万参数模型胜过 1.89 亿参数 transformer"); forces are minus the position

@@ -23,7 +23,7 @@ def lib():
 
 def test_exports_every_declared_symbol(lib):
     names = etp.declared_symbols()
-    assert len(names) == 17
+    assert len(names) == 19
     for n in names:
         assert hasattr(lib, n), n
 
@@ -186,3 +186,15 @@ def test_binding_checks_dtypes_and_shapes(lib):
         etp.assemble_forces(N, row_ptr, row_ptr, src, torch.zeros(E, 3), forces=torch.zeros(N, 2))
     with pytest.raises(ValueError, match="expected"):
         etp.build_reverse_csr(N, row_ptr.long(), src)
+
+
+def test_fused_workspace_size_and_refusals(lib):
+    """The fused radial tensor product takes the tensor-core MLP shape only (8 Bessel
+    functions, hidden 64); its workspace size is answered on the host."""
+    plan = etp.Plan("0..3", 3, "0..3", 128)
+    assert etp.fused_workspace_size(plan, 131072) > 0
+    with pytest.raises(etp.EtpError) as e:
+        etp.fused_workspace_size(plan, 100, n_basis=6, hidden=64)
+    assert e.value.status == etp.ETP_ERR_UNSUPPORTED
+    with pytest.raises(etp.EtpError):
+        etp.fused_workspace_size(plan, 100, n_basis=8, hidden=128)

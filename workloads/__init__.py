@@ -55,6 +55,10 @@ class Workload:
     x: np.ndarray         # float32 [N, (L+1)^2, C]
     w: np.ndarray         # float32 [E, P, C]
     g: np.ndarray         # float32 [N, (L+1)^2, C]
+    # the radial MLP that produced w (water only): W1 [8, 64], W2 [64, P*C] float32, cutoff
+    W1: np.ndarray | None = None
+    W2: np.ndarray | None = None
+    r_cut: float | None = None
 
     @property
     def N(self) -> int:
@@ -190,8 +194,9 @@ def _geometry_large(rng, rc=4.5, n=32768):
 
 
 def radial_mlp_weights(rng, r: np.ndarray, rc: float, P: int, C: int,
-                       n_basis: int = 8, hidden: int = 64) -> np.ndarray:
-    """w[e] = Linear(64 -> P*C)(SiLU(Linear(8 -> 64)(bessel(|r_e|)))) in FP64, cast to fp32.
+                       n_basis: int = 8, hidden: int = 64):
+    """(w, W1, W2): w[e] = Linear(64 -> P*C)(SiLU(Linear(8 -> 64)(bessel(|r_e|)))) in FP64, cast to
+    fp32, and the MLP's weights W1 [8, 64], W2 [64, P*C] cast to fp32.
 
     Bessel basis b_n(d) = sqrt(2/rc) sin(n pi d / rc) / d, n = 1..8, no envelope;
     weights N(0, 1/fan_in), no biases.
@@ -207,7 +212,7 @@ def radial_mlp_weights(rng, r: np.ndarray, rc: float, P: int, C: int,
     step = 16384
     for s in range(0, len(d), step):
         out[s:s + step] = (h[s:s + step] @ W2).astype(np.float32)
-    return out.reshape(len(d), P, C)
+    return out.reshape(len(d), P, C), W1.astype(np.float32), W2.astype(np.float32)
 
 
 def make(name: str, seed: int = 0, n_nodes: int | None = None) -> Workload:
@@ -235,12 +240,14 @@ def make(name: str, seed: int = 0, n_nodes: int | None = None) -> Workload:
         raise KeyError(name)
     N, E = len(row_ptr) - 1, len(src)
     x = _normal(rng, (N, D, C))
+    mlp = {}
     if name == "water":
-        w = radial_mlp_weights(rng, r64, rc, P, C)
+        w, W1, W2 = radial_mlp_weights(rng, r64, rc, P, C)
+        mlp = dict(W1=W1, W2=W2, r_cut=rc)
     else:
         w = _normal(rng, (E, P, C), 1.0 / np.sqrt(P))
     g = _normal(rng, (N, D, C))
-    return Workload(name, L, C, P, row_ptr, src.astype(np.int32), np.ascontiguousarray(r), x, w, g)
+    return Workload(name, L, C, P, row_ptr, src.astype(np.int32), np.ascontiguousarray(r), x, w, g, **mlp)
 
 
 def random_graph(rng, n: int, e: int, L: int, C: int, P: int, empty_rows=True) -> Workload:
