@@ -54,6 +54,9 @@ def _load():
         "etp_edge_frames": [vp, i32, vp, vp, vp],
         "etp_forward": [vp, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp],
         "etp_backward": [vp, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp],
+        "etp_double_backward": [vp, i32, i32] + [vp] * 17,
+        "etp_cart_forward": [vp, i32, i32, vp, vp, vp, vp, vp, vp, vp],
+        "etp_cart_backward": [vp, i32, i32] + [vp] * 13,
         "etp_assemble_forces": [i32, i32, vp, vp, vp, vp, vp, vp, vp, vp],
         "etp_radial_workspace_size": [vp, i32, i32, i32, ctypes.POINTER(sz)],
         "etp_radial_forward": [vp, i32, i32, i32, ctypes.c_float, vp, vp, vp, vp, vp, sz, vp],
@@ -250,6 +253,83 @@ def backward(plan: Plan, row_ptr, src, rev_ptr, rev_perm, dst, r, x, w, grad_out
             _ptr(rev_perm), _ptr(dst), _ptr(r), _ptr(frames), _ptr(x), _ptr(w), _ptr(grad_out), _ptr(grad_x),
             _ptr(grad_w), _ptr(grad_r), stream=stream)
     return grad_x, grad_w, grad_r
+
+
+def cart_forward(plan: Plan, row_ptr, src, r, x, w, out=None, stream=None):
+    """Cartesian edge convolution (launches etp_cart_forward): x and out in independent STF components."""
+    import torch
+
+    N, E = row_ptr.numel() - 1, src.numel()
+    _check_graph(row_ptr, src, N, E)
+    _expect(r, "r", "float32", (E, 3))
+    _expect(x, "x", "float32", (N, plan.dim_in, plan.C))
+    _expect(w, "w", "float32", (E, plan.n_paths, plan.C))
+    if out is None:
+        out = torch.empty((N, plan.dim_out, plan.C), device=x.device, dtype=torch.float32)
+    _expect(out, "out", "float32", (N, plan.dim_out, plan.C))
+    dev = _need_cuda(row_ptr, src, r, x, w, out)
+    _launch(dev, "etp_cart_forward", _load().etp_cart_forward, plan.handle, N, E, _ptr(row_ptr), _ptr(src), _ptr(r),
+            _ptr(x), _ptr(w), _ptr(out), stream=stream)
+    return out
+
+
+def cart_backward(plan: Plan, row_ptr, src, rev_ptr, rev_perm, dst, r, x, w, grad_out, want=("x", "w", "r"),
+                  stream=None):
+    """VJP of cart_forward (launches etp_cart_backward): (grad_x, grad_w, grad_r), unwanted ones None."""
+    import torch
+
+    N, E = row_ptr.numel() - 1, src.numel()
+    _check_graph(row_ptr, src, N, E)
+    _expect(rev_ptr, "rev_ptr", "int32", (N + 1,))
+    _expect(rev_perm, "rev_perm", "int32", (E,))
+    _expect(dst, "dst", "int32", (E,))
+    _expect(r, "r", "float32", (E, 3))
+    _expect(x, "x", "float32", (N, plan.dim_in, plan.C))
+    _expect(w, "w", "float32", (E, plan.n_paths, plan.C))
+    _expect(grad_out, "grad_out", "float32", (N, plan.dim_out, plan.C))
+    dev = x.device
+    gx = torch.empty((N, plan.dim_in, plan.C), device=dev, dtype=torch.float32) if "x" in want else None
+    gw = torch.empty((E, plan.n_paths, plan.C), device=dev, dtype=torch.float32) if "w" in want else None
+    gr = torch.empty((E, 3), device=dev, dtype=torch.float32) if "r" in want else None
+    dev = _need_cuda(row_ptr, src, rev_ptr, rev_perm, dst, r, x, w, grad_out, gx, gw, gr)
+    _launch(dev, "etp_cart_backward", _load().etp_cart_backward, plan.handle, N, E, _ptr(row_ptr), _ptr(src),
+            _ptr(rev_ptr), _ptr(rev_perm), _ptr(dst), _ptr(r), _ptr(x), _ptr(w), _ptr(grad_out), _ptr(gx), _ptr(gw),
+            _ptr(gr), stream=stream)
+    return gx, gw, gr
+
+
+def double_backward(plan: Plan, row_ptr, src, rev_ptr, rev_perm, dst, r, x, w, grad_out, gg_x=None, gg_w=None,
+                    gg_r=None, want=("g", "x", "w", "r"), out=None, stream=None):
+    """VJP of the VJP (launches etp_double_backward): dict with 'grad_g', 'grad_x', 'grad_w', 'grad_r'
+    (the wanted ones) of <gg_x, grad_x> + <gg_w, grad_w> + <gg_r, grad_r>; None cotangents are zero."""
+    import torch
+
+    N, E = row_ptr.numel() - 1, src.numel()
+    _check_graph(row_ptr, src, N, E)
+    _expect(rev_ptr, "rev_ptr", "int32", (N + 1,))
+    _expect(rev_perm, "rev_perm", "int32", (E,))
+    _expect(dst, "dst", "int32", (E,))
+    _expect(r, "r", "float32", (E, 3))
+    for t, name in ((x, "x"), (gg_x, "gg_x")):
+        _expect(t, name, "float32", (N, plan.dim_in, plan.C))
+    for t, name in ((w, "w"), (gg_w, "gg_w")):
+        _expect(t, name, "float32", (E, plan.n_paths, plan.C))
+    _expect(grad_out, "grad_out", "float32", (N, plan.dim_out, plan.C))
+    _expect(gg_r, "gg_r", "float32", (E, 3))
+    shapes = {"g": (N, plan.dim_out, plan.C), "x": (N, plan.dim_in, plan.C), "w": (E, plan.n_paths, plan.C),
+              "r": (E, 3)}
+    out = dict(out or {})
+    for k in "gxwr":
+        key = "grad_" + k
+        if k in want and out.get(key) is None:
+            out[key] = torch.empty(shapes[k], device=x.device, dtype=torch.float32)
+        _expect(out.get(key), key, "float32", shapes[k])
+    dev = _need_cuda(row_ptr, src, rev_ptr, rev_perm, dst, r, x, w, grad_out, gg_x, gg_w, gg_r, *out.values())
+    _launch(dev, "etp_double_backward", _load().etp_double_backward, plan.handle, N, E, _ptr(row_ptr), _ptr(src),
+            _ptr(rev_ptr), _ptr(rev_perm), _ptr(dst), _ptr(r), _ptr(x), _ptr(w), _ptr(grad_out), _ptr(gg_x),
+            _ptr(gg_w), _ptr(gg_r), _ptr(out.get("grad_g")), _ptr(out.get("grad_x")), _ptr(out.get("grad_w")),
+            _ptr(out.get("grad_r")), stream=stream)
+    return out
 
 
 def assemble_forces(N: int, row_ptr, rev_ptr, rev_perm, grad_r, r=None, forces=None, virial=None, stream=None):

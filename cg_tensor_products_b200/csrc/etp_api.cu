@@ -295,6 +295,70 @@ etp_status etp_backward(etp_plan_t plan, int N, int E, const int32_t* row_ptr, c
     return cuda_status(err);
 }
 
+etp_status etp_double_backward(etp_plan_t plan, int N, int E, const int32_t* row_ptr, const int32_t* src,
+                               const int32_t* rev_ptr, const int32_t* rev_perm, const int32_t* dst_of_edge,
+                               const float* r, const float* x, const float* w, const float* grad_out,
+                               const float* gg_x, const float* gg_w, const float* gg_r, float* grad_grad_out,
+                               float* grad_x, float* grad_w, float* grad_r, etp_stream_t stream) {
+    if (!plan || N < 0 || E < 0) return ETP_ERR_INVALID_ARG;
+    if (N == 0) return E == 0 ? ETP_OK : ETP_ERR_INVALID_ARG;
+    if (!row_ptr || !rev_ptr || !x || !grad_out || !aligned4(row_ptr) || !aligned4(rev_ptr) || !aligned16(x) ||
+        !aligned16(grad_out))
+        return ETP_ERR_INVALID_ARG;
+    if ((gg_x && !aligned16(gg_x)) || (grad_grad_out && !aligned16(grad_grad_out)) || (grad_x && !aligned16(grad_x)))
+        return ETP_ERR_INVALID_ARG;
+    if (E > 0) {
+        if (!src || !rev_perm || !w || !r || !aligned4(src) || !aligned4(rev_perm) || !aligned16(w) || !aligned4(r))
+            return ETP_ERR_INVALID_ARG;
+        if ((gg_w && !aligned16(gg_w)) || (gg_r && !aligned4(gg_r)) || (grad_w && !aligned16(grad_w)) ||
+            (grad_r && !aligned4(grad_r)) || (dst_of_edge && !aligned4(dst_of_edge)))
+            return ETP_ERR_INVALID_ARG;
+    } else {
+        grad_w = nullptr;
+        grad_r = nullptr;
+    }
+    if (!grad_grad_out && !grad_x && !grad_w && !grad_r) return ETP_OK;
+    return cuda_status(etp::double_backward(plan->L, plan->o3, plan->C, N, E, row_ptr, src, rev_ptr, rev_perm,
+                                            dst_of_edge, r, x, w, grad_out, gg_x, gg_w, gg_r, grad_grad_out, grad_x,
+                                            grad_w, grad_r, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+etp_status etp_cart_forward(etp_plan_t plan, int N, int E, const int32_t* row_ptr, const int32_t* src, const float* r,
+                            const float* x, const float* w, float* out, etp_stream_t stream) {
+    if (!plan || N < 0 || E < 0) return ETP_ERR_INVALID_ARG;
+    if (N == 0) return E == 0 ? ETP_OK : ETP_ERR_INVALID_ARG;
+    if (!row_ptr || !x || !out || !aligned4(row_ptr) || !aligned16(x) || !aligned16(out)) return ETP_ERR_INVALID_ARG;
+    if (E > 0 && (!src || !w || !r || !aligned4(src) || !aligned16(w) || !aligned4(r))) return ETP_ERR_INVALID_ARG;
+    return cuda_status(etp::cart_forward(plan->L, plan->o3, plan->C, N, E, row_ptr, src, r, x, w, out,
+                                         reinterpret_cast<cudaStream_t>(stream)));
+}
+
+etp_status etp_cart_backward(etp_plan_t plan, int N, int E, const int32_t* row_ptr, const int32_t* src,
+                             const int32_t* rev_ptr, const int32_t* rev_perm, const int32_t* dst_of_edge,
+                             const float* r, const float* x, const float* w, const float* grad_out, float* grad_x,
+                             float* grad_w, float* grad_r, etp_stream_t stream) {
+    if (!plan || N < 0 || E < 0) return ETP_ERR_INVALID_ARG;
+    if (N == 0) return E == 0 ? ETP_OK : ETP_ERR_INVALID_ARG;
+    if (!row_ptr || !rev_ptr || !x || !grad_out || !aligned4(row_ptr) || !aligned4(rev_ptr) || !aligned16(x) ||
+        !aligned16(grad_out))
+        return ETP_ERR_INVALID_ARG;
+    if (grad_x && !aligned16(grad_x)) return ETP_ERR_INVALID_ARG;
+    if (E > 0) {
+        if (!src || !rev_perm || !w || !r || !aligned4(src) || !aligned4(rev_perm) || !aligned16(w) || !aligned4(r))
+            return ETP_ERR_INVALID_ARG;
+        if ((grad_w && !aligned16(grad_w)) || (grad_r && !aligned4(grad_r)) ||
+            (dst_of_edge && !aligned4(dst_of_edge)))
+            return ETP_ERR_INVALID_ARG;
+    } else {
+        grad_w = nullptr;
+        grad_r = nullptr;
+    }
+    if (!grad_x && !grad_w && !grad_r) return ETP_OK;
+    return cuda_status(etp::cart_backward(plan->L, plan->o3, plan->C, N, E, row_ptr, rev_ptr, rev_perm, dst_of_edge,
+                                          r, x, w, grad_out, grad_x, grad_w, grad_r,
+                                          reinterpret_cast<cudaStream_t>(stream)));
+}
+
 etp_status etp_assemble_forces(int N, int E, const int32_t* row_ptr, const int32_t* rev_ptr, const int32_t* rev_perm,
                                const float* r, const float* grad_r, float* forces, float* virial, etp_stream_t stream) {
     if (N < 0 || E < 0) return ETP_ERR_INVALID_ARG;

@@ -46,8 +46,6 @@ namespace fused {
 constexpr int kRows = 128;                    // edges per tile (MMA M)
 constexpr int kBasis = 8;                     // Bessel functions
 constexpr int kHidden = 64;                   // hidden width (MMA K)
-constexpr int kConsumers = 128;               // warps 0-3
-constexpr int kThreads = kConsumers + 32;     // + warp 4: TMEM owner, bulk copies and MMAs
 constexpr int kAccBufs = 3;                   // TMEM accumulators in flight
 constexpr uint32_t kLBO = 128, kSBO = 2048;   // K-major operand: K = 64 per 8-row group
 constexpr uint32_t kAHalf = kRows * kHidden * 4;  // 32 KB
@@ -171,39 +169,48 @@ __device__ __forceinline__ void red_add(float* p, float v) {
 }
 
 // Shared memory: A (two TF32 halves, 64 KB), two B slots of 2 x Npad x 256 B, the
-// consumers' transpose stage (4 x 32 rows of 2D + 1 floats), the mbarriers and the
-// TMEM address.
+// consumers' transpose stage (NW warps x 32 rows of 2D + 1 floats), W1, the
+// mbarriers and the TMEM address.
 struct Smem {
-    uint32_t slot_bytes, off_b, off_stage, off_bars, total;
+    uint32_t slot_bytes, off_b, off_stage, off_w1, off_bars, total;
 };
-__host__ __device__ constexpr Smem smem_layout(int Npad, int D) {
+__host__ __device__ constexpr Smem smem_layout(int Npad, int D, int NW) {
     Smem s{};
     s.slot_bytes = 2u * (uint32_t)Npad * (kHidden * 4);
     s.off_b = 2 * kAHalf;
     s.off_stage = s.off_b + 2 * s.slot_bytes;
-    s.off_bars = s.off_stage + (uint32_t)((4 * 32 * (2 * D + 1) * 4 + 15) / 16 * 16);
+    s.off_w1 = s.off_stage + (uint32_t)((NW * 32 * (2 * D + 1) * 4 + 15) / 16 * 16);
+    s.off_bars = s.off_w1 + kBasis * kHidden * 4;
     s.total = s.off_bars + 16 * 8;
     return s;
 }
+// Consumer warps: eight (two per TMEM lane quarter, splitting the channel pairs)
+// where the stage fits in shared memory, else four.
+template <int L>
+constexpr int consumer_warps() { return L <= 2 ? 8 : 4; }
 
 template <int L, bool O3>
-__global__ void __launch_bounds__(kThreads, 1) etp_fused_fwd_kernel(FwdArgs a) {
+__global__ void __launch_bounds__(consumer_warps<L>() * 32 + 32, 1) etp_fused_fwd_kernel(FwdArgs a) {
     using namespace frame;
     using O = L3Order<L, O3>;
     constexpr int D = (L + 1) * (L + 1);
     constexpr int P = PathSet<L, O3>::P;
     constexpr int STR = 2 * D + 1;
+    constexpr int NW = consumer_warps<L>();  // consumer warps
+    constexpr int NH = NW / 4;               // consumer warps per TMEM lane quarter
+    constexpr int kConsumers = NW * 32;
+    constexpr bool kPrefetchX = L <= 2;      // registers for the next pair's x
     extern __shared__ __align__(1024) unsigned char smem[];
-    const Smem lay = smem_layout(a.Npad, D);
+    const Smem lay = smem_layout(a.Npad, D, NW);
     unsigned char* A_hi = smem;
     unsigned char* A_lo = smem + kAHalf;
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + lay.off_bars);
-    uint64_t* a_full = bars + 0;       // consumers wrote A (128 arrivals)
+    uint64_t* a_full = bars + 0;       // consumers wrote A (one arrival per consumer thread)
     uint64_t* a_empty = bars + 1;      // the tile's MMAs are done (commit)
     uint64_t* b_full = bars + 2;       // [2] slice operand arrived (bulk copy)
     uint64_t* b_empty = bars + 4;      // [2] slice MMAs done (commit)
     uint64_t* acc_full = bars + 6;     // [3] accumulator ready (commit)
-    uint64_t* acc_empty = bars + 9;    // [3] consumers done with it (4 arrivals)
+    uint64_t* acc_empty = bars + 9;    // [3] consumers done with it (one arrival per consumer warp)
     uint64_t* done_bar = bars + 12;    // every MMA done (commit, once)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 13);
     const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
@@ -218,12 +225,14 @@ __global__ void __launch_bounds__(kThreads, 1) etp_fused_fwd_kernel(FwdArgs a) {
     const int S = a.S;
     const int G = ntiles * S;
 
-    if (warp == 4) tc::tmem_alloc(tmem_slot, 512);
+    float* w1s = reinterpret_cast<float*>(smem + lay.off_w1);
+    for (int k = t; k < kBasis * kHidden; k += kConsumers + 32) w1s[k] = __ldg(a.W1 + k);
+    if (warp == NW) tc::tmem_alloc(tmem_slot, 512);
     if (t == kConsumers) {
         tc::mbar_init(a_full, kConsumers);
         tc::mbar_init(a_empty, 1);
         for (int i = 0; i < 2; ++i) tc::mbar_init(&b_full[i], 1), tc::mbar_init(&b_empty[i], 1);
-        for (int i = 0; i < kAccBufs; ++i) tc::mbar_init(&acc_full[i], 1), tc::mbar_init(&acc_empty[i], 4);
+        for (int i = 0; i < kAccBufs; ++i) tc::mbar_init(&acc_full[i], 1), tc::mbar_init(&acc_empty[i], NW);
         tc::mbar_init(done_bar, 1);
         tc::mbar_fence_init();
     }
@@ -233,7 +242,7 @@ __global__ void __launch_bounds__(kThreads, 1) etp_fused_fwd_kernel(FwdArgs a) {
     const uint32_t tmem = *tmem_slot;
     bool live = true;
 
-    if (warp == 4) {
+    if (warp == NW) {
         // ---------------- bulk copies of the slice operands and the MMAs ----------------
         if (lane == 0 && G > 0) {
             auto load = [&](int g) {
@@ -287,16 +296,22 @@ __global__ void __launch_bounds__(kThreads, 1) etp_fused_fwd_kernel(FwdArgs a) {
         }
     } else {
         // ---------------- consumers: one edge per thread ----------------
-        const int ra = k0 + (int)(len * warp / 4), rb = k0 + (int)(len * (warp + 1) / 4);
+        // warp = quarter + 4 half: the quarter fixes the TMEM lanes (edges), the half
+        // the channel pairs of each slice (pairs q with q % NH == half)
+        const int quarter = warp & 3, half = warp >> 2;
+        const int ra = k0 + (int)(len * quarter / 4), rb = k0 + (int)(len * (quarter + 1) / 4);
         const float2* x2 = reinterpret_cast<const float2*>(a.x);
         const int C2 = a.C / 2, pairs = a.cs / 2;
         float* stage = reinterpret_cast<float*>(smem + lay.off_stage) + warp * 32 * STR;
-        float* carry = a.carry + ((size_t)(task * 4 + warp) * C2) * 32 + lane;
-        const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
+        float* carry = a.carry + ((size_t)(task * 4 + quarter) * C2) * 32 + lane;
+        const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
         int cur_row = ra < rb ? segment_of(a.row_ptr, a.N, ra) : 0;
         bool carried = false;  // warp-uniform: this chunk's first row continues the previous chunk's last
-        unsigned char* arow_hi = A_hi + tc::kmajor_offset(warp * 32 + lane, 0, kLBO, kSBO);
-        unsigned char* arow_lo = A_lo + tc::kmajor_offset(warp * 32 + lane, 0, kLBO, kSBO);
+        unsigned char* arow_hi = A_hi + tc::kmajor_offset(quarter * 32 + lane, 0, kLBO, kSBO);
+        unsigned char* arow_lo = A_lo + tc::kmajor_offset(quarter * 32 + lane, 0, kLBO, kSBO);
+        const int kh0 = half * (kHidden / NH), kh1 = kh0 + kHidden / NH;  // this warp's hidden units of A
+        const int my_pairs = (pairs - half + NH - 1) / NH;                   // pairs q = half, half + NH, ...
+        const int n_my = S * my_pairs;                                       // this warp's pairs per tile
 
         for (int i = 0; i < ntiles; ++i) {
             const int cb = ra + 32 * i, ce = min(cb + 32, rb);
@@ -326,7 +341,9 @@ __global__ void __launch_bounds__(kThreads, 1) etp_fused_fwd_kernel(FwdArgs a) {
             const unsigned cont_mask = __ballot_sync(0xffffffffu, is_end && lane == nrows - 1 && re > ce && ce < rb);
             // the row lies wholly in this warp range: stored once, else reduced onto the output
             const unsigned whole_mask = __ballot_sync(0xffffffffu, has && rs >= ra && re <= rb);
+            const bool one_segment = nrows > 0 && end_mask == (1u << (nrows - 1));
             if (nrows > 0) cur_row = __shfl_sync(0xffffffffu, d, nrows - 1);
+            const float2* xrow = x2 + (size_t)(valid ? j : 0) * D * C2;
 
             // frame and Wigner matrices of the edge
             const float3 rv = has ? load_r(a.r, e) : make_float3(0.f, 0.f, 1.f);
@@ -334,7 +351,7 @@ __global__ void __launch_bounds__(kThreads, 1) etp_fused_fwd_kernel(FwdArgs a) {
             float d2[25], d3[49];
             thread_wigner<L>(f, d2, d3);
 
-            // hidden layer of the edge into the A operand (once the previous tile's MMAs are done)
+            // this warp's share of the hidden layer into the A operand (once the previous tile's MMAs are done)
             {
                 float b[kBasis];
                 const float dist = sqrtf(rv.x * rv.x + rv.y * rv.y + rv.z * rv.z);
@@ -346,15 +363,16 @@ __global__ void __launch_bounds__(kThreads, 1) etp_fused_fwd_kernel(FwdArgs a) {
                 }
                 if (i > 0) wait_live(a_empty, (i - 1) & 1, live);
 #pragma unroll 2
-                for (int k4 = 0; k4 < kHidden; k4 += 4) {
-                    float h[4];
+                for (int k4 = kh0; k4 < kh1; k4 += 4) {
+                    float h[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        float z = 0.f;
-#pragma unroll
-                        for (int n = 0; n < kBasis; ++n) z = fmaf(b[n], __ldg(a.W1 + n * kHidden + k4 + u), z);
-                        h[u] = has ? z / (1.f + expf(-z)) : 0.f;
+                    for (int n = 0; n < kBasis; ++n) {
+                        const float4 wv = *reinterpret_cast<const float4*>(w1s + n * kHidden + k4);
+                        h[0] = fmaf(b[n], wv.x, h[0]), h[1] = fmaf(b[n], wv.y, h[1]);
+                        h[2] = fmaf(b[n], wv.z, h[2]), h[3] = fmaf(b[n], wv.w, h[3]);
                     }
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) h[u] = has ? h[u] / (1.f + expf(-h[u])) : 0.f;
                     float4 hh, hl;
                     hh.x = tc::tf32_round(h[0]), hh.y = tc::tf32_round(h[1]);
                     hh.z = tc::tf32_round(h[2]), hh.w = tc::tf32_round(h[3]);
@@ -367,21 +385,32 @@ __global__ void __launch_bounds__(kThreads, 1) etp_fused_fwd_kernel(FwdArgs a) {
                 tc::mbar_arrive(a_full);
             }
 
+            // x of the source for a channel pair (zero for an invalid source)
+            auto load_x = [&](int gp, float2 (&xv)[D]) {
+#pragma unroll
+                for (int k = 0; k < D; ++k) xv[k] = valid ? __ldg(xrow + (size_t)k * C2 + gp) : f2_zero();
+            };
+            float2 xn[D];
+            if constexpr (kPrefetchX) load_x(half, xn);
+
             for (int s = 0; s < S; ++s) {
                 const int g = i * S + s, buf = g % kAccBufs;
                 wait_live(&acc_full[buf], (g / kAccBufs) & 1, live);
                 tc::fence_after_sync();
-                for (int q = 0; q < pairs; ++q) {
+                for (int q = half; q < pairs; q += NH) {
                     const int gp = s * pairs + q;  // channel pair index: channels 2 gp, 2 gp + 1
                     const uint32_t colq = lane_base + (uint32_t)(buf * a.Npad + q * 2 * P);
                     float2 xv[D];
-                    if (valid) {
-                        const float2* xs = x2 + (size_t)j * D * C2 + gp;
+                    if constexpr (kPrefetchX) {
 #pragma unroll
-                        for (int k = 0; k < D; ++k) xv[k] = __ldg(xs + (size_t)k * C2);
+                        for (int k = 0; k < D; ++k) xv[k] = xn[k];
+                        const int nxt = (s * my_pairs + (q - half) / NH) + 1;  // this warp's next pair in the tile
+                        if (nxt < n_my) {
+                            const int sn = nxt / my_pairs, qn = half + (nxt - sn * my_pairs) * NH;
+                            load_x(sn * pairs + qn, xn);
+                        }
                     } else {
-#pragma unroll
-                        for (int k = 0; k < D; ++k) xv[k] = f2_zero();
+                        load_x(gp, xv);
                     }
                     float2 xp[D];
                     static_for<0, L + 1>([&](auto lc) {
@@ -389,12 +418,32 @@ __global__ void __launch_bounds__(kThreads, 1) etp_fused_fwd_kernel(FwdArgs a) {
                         rot_reg<l, false>(f, d2, d3, xv + l * l, xp + l * l);
                     });
                     float* srow = stage + lane * STR;
+                    // the pair's weights, one TMEM load per l3 group: all in flight together
+                    // (L <= 2), or group by group (L = 3: registers)
+                    constexpr int kAll = O::cols_pow2(0) + (L >= 1 ? O::cols_pow2(1) : 0) +
+                                         (L >= 2 ? O::cols_pow2(2) : 0);
+                    float vall[L <= 2 ? kAll : 1];
+                    if constexpr (L <= 2) {
+                        static_for<0, L + 1>([&](auto l3c) {
+                            constexpr int l3 = decltype(l3c)::value;
+                            constexpr int off = l3 == 0 ? 0 : (l3 == 1 ? O::cols_pow2(0) : O::cols_pow2(0) + O::cols_pow2(1));
+                            tc::tmem_ld<O::cols_pow2(l3)>(colq + 2 * O::start(l3),
+                                                          *reinterpret_cast<float(*)[O::cols_pow2(l3)]>(vall + off));
+                        });
+                        tc::tmem_wait_ld(vall);
+                    }
                     static_for<0, L + 1>([&](auto l3c) {
                         constexpr int l3 = decltype(l3c)::value;
                         constexpr int NC = O::cols_pow2(l3);
                         float v[NC];
-                        tc::tmem_ld<NC>(colq + 2 * O::start(l3), v);
-                        tc::tmem_wait_ld(v);
+                        if constexpr (L <= 2) {
+                            constexpr int off = l3 == 0 ? 0 : (l3 == 1 ? O::cols_pow2(0) : O::cols_pow2(0) + O::cols_pow2(1));
+#pragma unroll
+                            for (int u = 0; u < NC; ++u) v[u] = vall[off + u];
+                        } else {
+                            tc::tmem_ld<NC>(colq + 2 * O::start(l3), v);
+                            tc::tmem_wait_ld(v);
+                        }
                         float2 y[2 * l3 + 1], msg[2 * l3 + 1];
 #pragma unroll
                         for (int m = 0; m < 2 * l3 + 1; ++m) y[m] = f2_zero();
@@ -423,28 +472,45 @@ __global__ void __launch_bounds__(kThreads, 1) etp_fused_fwd_kernel(FwdArgs a) {
                     });
                     __syncwarp();
                     // sum the rows of equal destination, in row order; lane k < 2D owns column k
-                    // (component k / 2, channel 2 gp + k % 2)
+                    // (component k / 2, channel 2 gp + k % 2); rows without an edge hold zeros
                     const bool col = lane < 2 * D;
-                    float acc = (carried && col) ? carry[(size_t)gp * 32] : 0.f;
-                    for (int row = 0; row < nrows; ++row) {
-                        acc += col ? stage[row * STR + lane] : 0.f;
-                        if ((end_mask >> row) & 1u) {
-                            const int dd = __shfl_sync(0xffffffffu, d, row);
-                            if (col) {
-                                if ((cont_mask >> row) & 1u) {
-                                    carry[(size_t)gp * 32] = acc;
-                                } else {
-                                    float* o = a.out + ((size_t)dd * D + (lane >> 1)) * a.C + 2 * gp + (lane & 1);
-                                    if ((whole_mask >> row) & 1u)
-                                        *o = acc;
-                                    else
-                                        red_add(o, acc);
-                                }
+                    float vr[32];
+#pragma unroll
+                    for (int rr = 0; rr < 32; ++rr) vr[rr] = stage[rr * STR + (col ? lane : 0)];
+                    __syncwarp();  // the stage is rewritten by the next pair
+                    float* optr = a.out + (size_t)(lane >> 1) * a.C + 2 * gp + (lane & 1);
+                    auto finish = [&](int rr, float acc) {  // the segment that ends at row rr
+                        const int dd = __shfl_sync(0xffffffffu, d, rr);
+                        if (col) {
+                            if ((cont_mask >> rr) & 1u) {
+                                carry[(size_t)gp * 32] = acc;
+                            } else {
+                                float* o = optr + (size_t)dd * D * a.C;
+                                if ((whole_mask >> rr) & 1u)
+                                    *o = acc;
+                                else
+                                    red_add(o, acc);
                             }
-                            acc = 0.f;
+                        }
+                    };
+                    const float cin = (carried && col) ? carry[(size_t)gp * 32] : 0.f;
+                    if (one_segment) {
+#pragma unroll
+                        for (int w = 16; w >= 1; w >>= 1)
+#pragma unroll
+                            for (int rr = 0; rr < w; ++rr) vr[rr] += vr[rr + w];
+                        finish(nrows - 1, cin + vr[0]);
+                    } else if (nrows > 0) {
+                        float acc = cin;
+#pragma unroll
+                        for (int rr = 0; rr < 32; ++rr) {
+                            acc += vr[rr];
+                            if ((end_mask >> rr) & 1u) {
+                                finish(rr, acc);
+                                acc = 0.f;
+                            }
                         }
                     }
-                    __syncwarp();  // the stage is rewritten by the next pair
                 }
                 tc::fence_before_sync();
                 __syncwarp();
@@ -455,7 +521,7 @@ __global__ void __launch_bounds__(kThreads, 1) etp_fused_fwd_kernel(FwdArgs a) {
     }
     tc::fence_before_sync();
     __syncthreads();
-    if (warp == 4) {
+    if (warp == NW) {
         __syncwarp();
         tc::fence_after_sync();
         tc::tmem_dealloc(tmem, 512);
@@ -537,7 +603,7 @@ FusedGeometry fused_geometry(int L, bool o3, int C, int E) {
         default: g.P = FusedSpec<3, true>::P; break;
     }
     g.Npad = (g.P * g.cs + 15) / 16 * 16;
-    const fused::Smem lay = fused::smem_layout(g.Npad, g.D);
+    const fused::Smem lay = fused::smem_layout(g.Npad, g.D, 4);
     g.w2_bytes = (size_t)g.S * lay.slot_bytes;
     long long tasks = ((long long)E + fused::kRows - 1) / fused::kRows;
     if (tasks > kMaxFusedTasks) tasks = kMaxFusedTasks;
@@ -572,12 +638,13 @@ cudaError_t launch_fused(const FusedGeometry& g, int C, int N, int E, const int3
     if (ntasks > sms) ntasks = sms;
     if (ntasks > kMaxFusedTasks) ntasks = kMaxFusedTasks;
     fused::FwdArgs a{N, E, row_ptr, src, r, x, W1, w2s, out, carry, rc, C, g.cs, g.S, g.Npad, (int)ntasks};
-    const fused::Smem lay = fused::smem_layout(g.Npad, g.D);
+    constexpr int NW = fused::consumer_warps<L>();
+    const fused::Smem lay = fused::smem_layout(g.Npad, g.D, NW);
     const void* k = (const void*)fused::etp_fused_fwd_kernel<L, O3>;
     if ((err = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)lay.total)) != cudaSuccess)
         return err;
     void* args[] = {&a};
-    return cudaLaunchKernel(k, dim3((unsigned)ntasks), dim3(fused::kThreads), args, lay.total, s);
+    return cudaLaunchKernel(k, dim3((unsigned)ntasks), dim3(NW * 32 + 32), args, lay.total, s);
 }
 
 }  // namespace
@@ -591,7 +658,7 @@ size_t fused_workspace_bytes(int L, bool o3, int C, int E) {
 
 size_t fused_smem_bytes(int L, bool o3, int C) {
     const FusedGeometry g = fused_geometry(L, o3, C, 1);
-    return fused::smem_layout(g.Npad, g.D).total;
+    return fused::smem_layout(g.Npad, g.D, L <= 2 ? fused::consumer_warps<2>() : fused::consumer_warps<3>()).total;
 }
 
 cudaError_t fused_forward(int L, bool o3, int C, int N, int E, const int32_t* row_ptr, const int32_t* src,

@@ -128,6 +128,18 @@ cudaError_t fused_forward(int L, bool o3, int C, int N, int E, const int32_t* ro
                           const float* r, const float* x, const float* W1, const float* W2, float rc, float* out,
                           void* ws, cudaStream_t s);
 int fused_read_and_clear_fault();
+// VJP of the VJP (etp_double.cu).
+cudaError_t double_backward(int L, bool o3, int C, int N, int E, const int32_t* row_ptr, const int32_t* src,
+                            const int32_t* rev_ptr, const int32_t* rev_perm, const int32_t* dst, const float* r,
+                            const float* x, const float* w, const float* g, const float* gg_x, const float* gg_w,
+                            const float* gg_r, float* grad_g, float* grad_x, float* grad_w, float* grad_r,
+                            cudaStream_t s);
+// Cartesian edge convolution (etp_cart.cu): features in independent STF components.
+cudaError_t cart_forward(int L, bool o3, int C, int N, int E, const int32_t* row_ptr, const int32_t* src,
+                         const float* r, const float* x, const float* w, float* out, cudaStream_t s);
+cudaError_t cart_backward(int L, bool o3, int C, int N, int E, const int32_t* row_ptr, const int32_t* rev_ptr,
+                          const int32_t* rev_perm, const int32_t* dst, const float* r, const float* x, const float* w,
+                          const float* g, float* grad_x, float* grad_w, float* grad_r, cudaStream_t s);
 cudaError_t assemble_forces(int N, int E, const int32_t* row_ptr, const int32_t* rev_ptr, const int32_t* rev_perm,
                             const float* r, const float* grad_r, float* forces, float* virial, cudaStream_t s);
 cudaError_t validate_csr(int N, int E, const int32_t* row_ptr, const int32_t* src, int32_t* flag, cudaStream_t s);

@@ -44,6 +44,8 @@
 #include <complex>
 #include <cstdio>
 #include <cstdlib>
+#include <algorithm>
+#include <functional>
 #include <vector>
 
 namespace {
@@ -259,6 +261,169 @@ std::vector<ld> real_generator(int l, int axis) {
     return J;
 }
 
+// ---------------------------------------------------------------------------
+// Cartesian couplings in independent components. A symmetric traceless (STF)
+// tensor of rank l is held by its 2l + 1 entries with at most one z index,
+// ordered (x^l, x^(l-1) y, .., y^l, x^(l-1) z, .., y^(l-1) z) by the counts (a, b, c)
+// of x, y, z indices; the other entries follow from tracelessness,
+// T(a, b, c) = -T(a + 2, b, c - 2) - T(a, b + 2, c - 2). The path (l1, l2 -> l3)
+// contracts the last k indices of the first operand with the first k of the
+// second, k = (l1 + l2 - l3 - odd) / 2 with odd = (l1 + l2 + l3) mod 2; when odd,
+// the first operand's last free index and the second's first free index go
+// through the Levi-Civita symbol into a new last index; the STF part of the l3
+// remaining indices is the result, with no normalisation constant. In
+// independent components the coupling is a sparse tensor Cc[i1][i2][i3].
+struct Cnt3 {
+    int a, b, c;
+};
+std::vector<Cnt3> compact_counts(int l) {
+    std::vector<Cnt3> v;
+    for (int b = 0; b <= l; ++b) v.push_back({l - b, b, 0});
+    for (int b = 0; b + 1 <= l; ++b) v.push_back({l - 1 - b, b, 1});
+    return v;
+}
+int ipow3(int l) {
+    int n = 1;
+    for (int k = 0; k < l; ++k) n *= 3;
+    return n;
+}
+// digits of full index t (rank l, first index most significant)
+std::vector<int> digits(int t, int l) {
+    std::vector<int> d(l);
+    for (int k = l - 1; k >= 0; --k) {
+        d[k] = t % 3;
+        t /= 3;
+    }
+    return d;
+}
+Cnt3 counts_of(const std::vector<int>& d) {
+    Cnt3 c{0, 0, 0};
+    for (int v : d) (v == 0 ? c.a : (v == 1 ? c.b : c.c))++;
+    return c;
+}
+// full STF tensor of rank l from independent components
+std::vector<ld> stf_expand(int l, const std::vector<ld>& comp) {
+    auto cc = compact_counts(l);
+    std::function<ld(int, int, int)> T = [&](int a, int b, int c) -> ld {
+        if (c <= 1) {
+            for (size_t i = 0; i < cc.size(); ++i)
+                if (cc[i].a == a && cc[i].b == b && cc[i].c == c) return comp[i];
+            return 0;
+        }
+        return -T(a + 2, b, c - 2) - T(a, b + 2, c - 2);
+    };
+    std::vector<ld> full(ipow3(l));
+    for (int t = 0; t < ipow3(l); ++t) {
+        Cnt3 c = counts_of(digits(t, l));
+        full[t] = l == 0 ? comp[0] : T(c.a, c.b, c.c);
+    }
+    return full;
+}
+// STF projection of a rank-l tensor (l <= 3)
+std::vector<ld> stf_project(int l, const std::vector<ld>& T) {
+    if (l <= 1) return T;
+    const int n = ipow3(l);
+    std::vector<ld> S(n, 0);
+    for (int t = 0; t < n; ++t) {  // symmetrise: average over index permutations
+        auto d = digits(t, l);
+        std::vector<int> perm(l);
+        for (int k = 0; k < l; ++k) perm[k] = k;
+        int np = 0;
+        ld acc = 0;
+        do {
+            int u = 0;
+            for (int k = 0; k < l; ++k) u = u * 3 + d[perm[k]];
+            acc += T[u];
+            ++np;
+        } while (std::next_permutation(perm.begin(), perm.end()));
+        S[t] = acc / np;
+    }
+    std::vector<ld> out(S);
+    if (l == 2) {
+        const ld tr = (S[0] + S[4] + S[8]) / 3;
+        for (int i = 0; i < 3; ++i) out[i * 3 + i] -= tr;
+    } else {  // l == 3: S_ijk - (delta_ij t_k + delta_ik t_j + delta_jk t_i) / 5, t_k = S_llk
+        ld tv[3];
+        for (int k = 0; k < 3; ++k) tv[k] = S[(0 * 3 + 0) * 3 + k] + S[(1 * 3 + 1) * 3 + k] + S[(2 * 3 + 2) * 3 + k];
+        for (int i = 0; i < 3; ++i)
+            for (int j = 0; j < 3; ++j)
+                for (int k = 0; k < 3; ++k) {
+                    ld v = 0;
+                    if (i == j) v += tv[k];
+                    if (i == k) v += tv[j];
+                    if (j == k) v += tv[i];
+                    out[(i * 3 + j) * 3 + k] -= v / 5;
+                }
+    }
+    return out;
+}
+ld levi(int a, int b, int c) {
+    if (a == b || b == c || a == c) return 0;
+    return ((a + 1) % 3 == b) ? 1 : -1;  // cyclic (0 1 2), (1 2 0), (2 0 1): +1
+}
+// the path's contraction of full tensors A (rank l1) and B (rank l2), before STF
+std::vector<ld> cart_contract(int l1, int l2, int l3, const std::vector<ld>& A, const std::vector<ld>& B) {
+    const int odd = (l1 + l2 + l3) % 2, k = (l1 + l2 - l3 - odd) / 2;
+    std::vector<ld> out(ipow3(l3), 0);
+    for (int ta = 0; ta < ipow3(l1); ++ta) {
+        if (A[ta] == 0) continue;
+        auto da = digits(ta, l1);
+        for (int tb = 0; tb < ipow3(l2); ++tb) {
+            if (B[tb] == 0) continue;
+            auto db = digits(tb, l2);
+            bool match = true;
+            for (int t = 0; t < k && match; ++t) match = da[l1 - k + t] == db[t];
+            if (!match) continue;
+            std::vector<int> fa(da.begin(), da.begin() + (l1 - k)), fb(db.begin() + k, db.end());
+            const ld ab = A[ta] * B[tb];
+            if (!odd) {
+                int u = 0;
+                for (int v : fa) u = u * 3 + v;
+                for (int v : fb) u = u * 3 + v;
+                out[u] += ab;
+            } else {
+                for (int n = 0; n < 3; ++n) {
+                    const ld e = levi(fa.back(), fb.front(), n);
+                    if (e == 0) continue;
+                    int u = 0;
+                    for (size_t q = 0; q + 1 < fa.size(); ++q) u = u * 3 + fa[q];
+                    for (size_t q = 1; q < fb.size(); ++q) u = u * 3 + fb[q];
+                    u = u * 3 + n;
+                    out[u] += e * ab;
+                }
+            }
+        }
+    }
+    return out;
+}
+std::vector<Nz> cart_coupling(int l1, int l2, int l3) {
+    std::vector<Nz> out;
+    if (l3 < std::abs(l1 - l2) || l3 > l1 + l2) return out;
+    const int d1 = 2 * l1 + 1, d2 = 2 * l2 + 1;
+    auto c3 = compact_counts(l3);
+    for (int i1 = 0; i1 < d1; ++i1)
+        for (int i2 = 0; i2 < d2; ++i2) {
+            std::vector<ld> e1(d1, 0), e2(d2, 0);
+            e1[i1] = 1;
+            e2[i2] = 1;
+            auto R = stf_project(l3, cart_contract(l1, l2, l3, stf_expand(l1, e1), stf_expand(l2, e2)));
+            for (int i3 = 0; i3 < 2 * l3 + 1; ++i3) {
+                ld v;
+                if (l3 == 0) {
+                    v = R[0];
+                } else {
+                    int u = 0;
+                    for (int q = 0; q < c3[i3].a; ++q) u = u * 3 + 0;
+                    for (int q = 0; q < c3[i3].b; ++q) u = u * 3 + 1;
+                    for (int q = 0; q < c3[i3].c; ++q) u = u * 3 + 2;
+                    v = R[u];
+                }
+                if (std::fabs(v) > 1e-15L) out.push_back({i1, i2, i3, v});
+            }
+        }
+    return out;
+}
+
 }  // namespace
 
 int main(int argc, char** argv) {
@@ -430,6 +595,40 @@ int main(int argc, char** argv) {
             std::fprintf(f, "},\n");
         }
         std::fprintf(f, "};\n\n");
+    }
+    // --- Cartesian couplings in independent STF components ------------------
+    {
+        int coff[kLmax + 1][kLmax + 1][kLmax + 1], ccnt[kLmax + 1][kLmax + 1][kLmax + 1];
+        std::vector<Nz> call;
+        for (int a = 0; a <= kLmax; ++a)
+            for (int b = 0; b <= kLmax; ++b)
+                for (int c = 0; c <= kLmax; ++c) {
+                    auto v = cart_coupling(a, b, c);
+                    coff[a][b][c] = (int)call.size();
+                    ccnt[a][b][c] = (int)v.size();
+                    call.insert(call.end(), v.begin(), v.end());
+                }
+        std::fprintf(f, "// Cartesian couplings Cc[i1][i2][i3] in independent STF components (counts of x, y, z\n");
+        std::fprintf(f, "// indices: c = 0 entries by ascending y count, then c = 1 entries); see gen_tables.cpp.\n");
+        std::fprintf(f, "constexpr int kCartTotal = %d;\n", (int)call.size());
+        std::fprintf(f, "constexpr CgNz kCart[kCartTotal] = {\n");
+        for (auto& z : call) std::fprintf(f, "    {%d, %d, %d, %.21Lg},\n", z.m1, z.m2, z.m3, z.v);
+        std::fprintf(f, "};\n\n");
+        for (int pass = 0; pass < 2; ++pass) {
+            std::fprintf(f, "constexpr int %s[%d][%d][%d] = {\n", pass ? "kCartCnt" : "kCartOff", kLmax + 1, kLmax + 1,
+                         kLmax + 1);
+            for (int a = 0; a <= kLmax; ++a) {
+                std::fprintf(f, "    {");
+                for (int b = 0; b <= kLmax; ++b) {
+                    std::fprintf(f, "{");
+                    for (int c = 0; c <= kLmax; ++c)
+                        std::fprintf(f, "%d%s", pass ? ccnt[a][b][c] : coff[a][b][c], c < kLmax ? ", " : "");
+                    std::fprintf(f, "}%s", b < kLmax ? ", " : "");
+                }
+                std::fprintf(f, "},\n");
+            }
+            std::fprintf(f, "};\n\n");
+        }
     }
     std::fprintf(f, "}  // namespace etp_gen\n");
     std::fclose(f);

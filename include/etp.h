@@ -170,6 +170,57 @@ ETP_API etp_status etp_backward(etp_plan_t plan, int N, int E, const int32_t* ro
                         const float* grad_out, float* grad_x, float* grad_w, float* grad_r,
                         etp_stream_t stream);
 
+/* VJP of the VJP (double backward). With (grad_x, grad_w, grad_r) = etp_backward's
+ * outputs for (x, w, r; grad_out) and cotangents gg_x [N][D][C], gg_w [E][P][C],
+ * gg_r [E][3] of those outputs, computes the gradients of
+ *     <gg_x, grad_x> + <gg_w, grad_w> + <gg_r, grad_r>
+ * with respect to grad_out (grad_grad_out [N][D][C]), x (grad_x [N][D][C]), w
+ * (grad_w [E][P][C]) and r (grad_r [E][3]). Force-loss training differentiates the
+ * forces, built from grad_r, with respect to the parameters, which takes this
+ * product ("FlashCart 如何让等变原子间势更快更准?", section "生成内核在高阶下胜过球谐
+ * 基线": the VJP of the VJP is timed beside the forward and the VJP). It includes
+ * the term through the Hessian of the harmonics (through gg_r). Each of gg_x,
+ * gg_w, gg_r may be NULL (zero); each output may be NULL (skipped); outputs are
+ * overwritten (nodes without edges get zeros). Graph arguments as in etp_backward
+ * (rev_ptr, rev_perm from etp_build_reverse_csr; dst_of_edge may be NULL). r is
+ * always read. Edges shorter than 1e-12 have no direction: only the (l, 0, l)
+ * paths act and every derivative in r is zero there. Allocates nothing; node sums
+ * in a fixed order, except rows cut by a task boundary (added onto the zeroed
+ * output) and, for C = 128, grad_r (two channel halves added onto zeros). */
+ETP_API etp_status etp_double_backward(etp_plan_t plan, int N, int E, const int32_t* row_ptr, const int32_t* src,
+                                       const int32_t* rev_ptr, const int32_t* rev_perm, const int32_t* dst_of_edge,
+                                       const float* r, const float* x, const float* w, const float* grad_out,
+                                       const float* gg_x, const float* gg_w, const float* gg_r,
+                                       float* grad_grad_out, float* grad_x, float* grad_w, float* grad_r,
+                                       etp_stream_t stream);
+
+/* Cartesian edge convolution: the same edge tensor product with Cartesian
+ * couplings ("FlashCart 如何让等变原子间势更快更准?", sections "FlashCart 用笛卡尔内核替
+ * 代球谐耦合" and "生成内核在高阶下胜过球谐基线": Cartesian kernels in place of
+ * spherical-harmonic couplings, compared at equal rank). A rank-l feature is a
+ * symmetric traceless (STF) tensor held by its 2l + 1 entries with at most one z
+ * index, in the order x^l, x^(l-1) y, .., y^l, x^(l-1) z, .., y^(l-1) z (rank 1:
+ * x, y, z); x, out, grad_out, grad_x are [N][(L+1)^2][C] with these blocks for
+ * l = 0..L. The edge attribute of rank l is the STF part of u (x) .. (x) u,
+ * u = r_e / |r_e| (zero for l >= 1 when |r_e| < 1e-12). Path (l1, l2 -> l3), in the
+ * plan's path order: k = (l1 + l2 - l3 - odd) / 2 index pairs contracted, the
+ * first operand's last k indices with the second's first k; for l1 + l2 + l3 odd
+ * (odd = 1) the first operand's last free index and the second's first free index
+ * go through the Levi-Civita symbol into a new last index; the STF part of the
+ * result; no normalisation constant. Then
+ *   out[i] = sum over row i of sum_p w[e,p,:] coupling_p(x[src e], attribute_l2(r_e)).
+ * The couplings are compile-time sparse tables of explicit sums; the pages give no
+ * formula, so these are this library's reading. Arguments, layouts, ownership and
+ * errors as etp_forward / etp_backward (no frame records); the VJP writes grad_x
+ * (sources without edges: zero), grad_w and grad_r (derivative through the edge
+ * attribute), each optional. */
+ETP_API etp_status etp_cart_forward(etp_plan_t plan, int N, int E, const int32_t* row_ptr, const int32_t* src,
+                                    const float* r, const float* x, const float* w, float* out, etp_stream_t stream);
+ETP_API etp_status etp_cart_backward(etp_plan_t plan, int N, int E, const int32_t* row_ptr, const int32_t* src,
+                                     const int32_t* rev_ptr, const int32_t* rev_perm, const int32_t* dst_of_edge,
+                                     const float* r, const float* x, const float* w, const float* grad_out,
+                                     float* grad_x, float* grad_w, float* grad_r, etp_stream_t stream);
+
 /* Radial weights: the tensor product's per-edge weights as a function of the edge
  * length. The pages make these weights a learned function of |r| ("High-performance
  * training and inference for deep equivariant interatomic potentials", section

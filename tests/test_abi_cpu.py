@@ -23,7 +23,7 @@ def lib():
 
 def test_exports_every_declared_symbol(lib):
     names = etp.declared_symbols()
-    assert len(names) == 19
+    assert len(names) == 22
     for n in names:
         assert hasattr(lib, n), n
 
