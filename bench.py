@@ -55,8 +55,12 @@ def parse():
     ap.add_argument("--radial", action="store_true",
                     help="also time the radial weights (w from |r|: Bessel(8) -> 64 -> SiLU -> P*C) and their VJP, "
                          "outside the step")
-    ap.add_argument("--no-frames", action="store_true",
-                    help="kernels build the edge frames themselves (no etp_edge_frames pass)")
+    ap.add_argument("--frames", choices=["auto", "on", "off"], default="auto",
+                    help="edge frame records: as the plan advises (auto), always, or never (the kernels build "
+                         "the frames themselves)")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="skip the timings beside the step: the fused radial-weights forward, the VJP of the VJP "
+                         "and the Cartesian edge convolution")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU seconds of the oracle baseline")
     return ap.parse_args()
@@ -301,6 +305,125 @@ def reference_arm(args):
 
 
 # ---------------------------------------------------------------------------
+def _time_ms(fn, stream, reps=10, warm=3):
+    import torch
+
+    for _ in range(warm):
+        fn()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(reps):
+        fn()
+    b.record(stream)
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / reps
+
+
+def measured_bf16():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured"
+    except Exception:
+        return 1590.0, "fallback"
+
+
+def extra_timings(etp, lib, plan, wl, d, rev_ptr, rev_perm, dst, gw, stream, dev, nnz_total):
+    """Kernels beside the step, each timed alone (CUDA events, 10 calls after 3 warm-up calls) on the same
+    workload, each with its roofline:
+      - the fused radial-weights tensor product (w = SiLU(bessel(|r|) W1) W2 produced on the tensor cores and
+        consumed in the kernel) against the unfused radial_forward + forward; bound by the tensor cores
+        (3 TF32 products per FP32 product of the dense layer, TF32 peak = measured bf16 x 1/2);
+      - the VJP of the VJP (all three cotangents), against its algorithmic bytes (HBM);
+      - the Cartesian edge convolution (forward and VJP) beside the spherical kernels at equal rank, against
+        the same algorithmic bytes (HBM)."""
+    import numpy as np
+    import torch
+
+    P = etp._ptr
+    sp = etp._stream(stream)
+    N, E, C, Pn = wl.N, wl.E, wl.C, plan.n_paths
+    D = (wl.L + 1) ** 2
+    node = N * D * C * 4
+    hbm, hbm_kind = measured_peaks()
+    bf16, bf16_kind = measured_bf16()
+    out = {}
+    # fused radial weights -> tensor product
+    rng = np.random.default_rng(7)
+    W1 = wl.W1 if wl.W1 is not None else (rng.standard_normal((8, 64)) / np.sqrt(8)).astype(np.float32)
+    W2 = wl.W2 if wl.W2 is not None else (rng.standard_normal((64, Pn * C)) / 8.0).astype(np.float32)
+    rc = wl.r_cut or 5.0
+    W1d, W2d = torch.from_numpy(W1).to(dev), torch.from_numpy(W2).to(dev)
+    fws = torch.empty(max(etp.fused_workspace_size(plan, E), 16), dtype=torch.uint8, device=dev)
+    fout = torch.empty((N, D, C), device=dev)
+    t_fused = _time_ms(lambda: etp._check(lib.etp_fused_forward(
+        plan.handle, N, E, P(d["row_ptr"]), P(d["src"]), P(d["r"]), P(d["x"]), 8, 64, rc, P(W1d), P(W2d), P(fout),
+        P(fws), fws.numel(), sp), "fused forward"), stream)
+    rws = torch.empty(max(etp.radial_workspace_size(plan, E, 8, 64), 16), dtype=torch.uint8, device=dev)
+    w_rad = torch.empty((E, Pn, C), device=dev)
+    t_rad = _time_ms(lambda: etp._check(lib.etp_radial_forward(
+        plan.handle, E, 8, 64, rc, P(d["r"]), P(W1d), P(W2d), P(w_rad), P(rws), rws.numel(), sp), "radial"), stream)
+    out2 = torch.empty_like(fout)
+    t_tp = _time_ms(lambda: etp._check(lib.etp_forward(
+        plan.handle, N, E, P(d["row_ptr"]), P(d["src"]), P(d["r"]), None, P(d["x"]), P(w_rad), P(out2), sp),
+        "forward"), stream)
+    tflop = 3 * 2.0 * E * 64 * Pn * C
+    del w_rad, rws
+    out["fused_radial_forward"] = {
+        "ms": t_fused, "unfused_ms": t_rad + t_tp, "unfused_radial_forward_ms": t_rad, "unfused_forward_ms": t_tp,
+        "speedup_over_unfused": (t_rad + t_tp) / t_fused,
+        "roofline": {"bound": "tensor", "achieved": tflop / (t_fused * 1e9), "peak": bf16 / 2, "unit": "TFLOP/s",
+                     "frac": tflop / (t_fused * 1e9) / (bf16 / 2),
+                     "peak_source": f"{bf16_kind} bf16 x 1/2 (TF32 nominal ratio)",
+                     "work": "3 TF32 products x 2 x E x 64 x P x C (the dense layer; the tensor product on the "
+                             "FP32 pipes besides)"},
+        "hbm_bytes_per_launch": E * 16 + 2 * node + 4 * (N + 1) + 4 * 64 * (8 + Pn * C)}
+    # VJP of the VJP
+    ggx = torch.randn((N, D, C), device=dev, generator=torch.Generator(device=dev).manual_seed(1))
+    ggw = torch.randn((E, Pn, C), device=dev, generator=torch.Generator(device=dev).manual_seed(2)) / Pn ** 0.5
+    ggr = torch.randn((E, 3), device=dev, generator=torch.Generator(device=dev).manual_seed(3))
+    o = {k: torch.empty_like(v) for k, v in (("g", d["g"]), ("x", d["x"]), ("r", d["r"]))}
+    t_dd = _time_ms(lambda: etp._check(lib.etp_double_backward(
+        plan.handle, N, E, P(d["row_ptr"]), P(d["src"]), P(rev_ptr), P(rev_perm), P(dst), P(d["r"]), P(d["x"]),
+        P(d["w"]), P(d["g"]), P(ggx), P(ggw), P(ggr), P(o["g"]), P(o["x"]), P(gw), P(o["r"]), sp), "double"),
+        stream)
+    dd_bytes = E * (3 * 4 * Pn * C + 12 * 3 + 4 * 3) + 5 * node + 4 * 2 * (N + 1)
+    mem = torch.cuda.max_memory_allocated(dev)
+    out["double_backward"] = {
+        "ms": t_dd, "bytes_per_launch": dd_bytes, "GBps": dd_bytes / (t_dd * 1e6),
+        "roofline": {"bound": "hbm", "achieved": dd_bytes / (t_dd * 1e6), "peak": hbm, "unit": "GB/s",
+                     "frac": dd_bytes / (t_dd * 1e6) / hbm, "peak_source": f"{hbm_kind} (hbm_gbs)"},
+        "bytes_note": "w and gg_w read, grad_w written (3 x 4PC per edge), r, gg_r, grad_r and three index "
+                      "arrays per edge, x, gg_x, g read and grad_g, grad_x written once per node",
+        "device_memory_peak_GB": mem / 1e9}
+    del ggx, ggw, ggr, o
+    # Cartesian edge convolution at equal rank
+    cout = torch.empty_like(fout)
+    cgx = torch.empty_like(d["x"])
+    cgr = torch.empty_like(d["r"])
+    t_cf = _time_ms(lambda: etp._check(lib.etp_cart_forward(
+        plan.handle, N, E, P(d["row_ptr"]), P(d["src"]), P(d["r"]), P(d["x"]), P(d["w"]), P(cout), sp), "cart"),
+        stream)
+    t_cb = _time_ms(lambda: etp._check(lib.etp_cart_backward(
+        plan.handle, N, E, P(d["row_ptr"]), P(d["src"]), P(rev_ptr), P(rev_perm), P(dst), P(d["r"]), P(d["x"]),
+        P(d["w"]), P(d["g"]), P(cgx), P(gw), P(cgr), sp), "cart backward"), stream)
+    t_sf = _time_ms(lambda: etp._check(lib.etp_forward(
+        plan.handle, N, E, P(d["row_ptr"]), P(d["src"]), P(d["r"]), None, P(d["x"]), P(d["w"]), P(out2), sp),
+        "forward"), stream)
+    t_sb = _time_ms(lambda: etp._check(lib.etp_backward(
+        plan.handle, N, E, P(d["row_ptr"]), P(d["src"]), P(rev_ptr), P(rev_perm), P(dst), P(d["r"]), None,
+        P(d["x"]), P(d["w"]), P(d["g"]), P(cgx), P(gw), P(cgr), sp), "backward"), stream)
+    alg = algorithmic(wl, Pn, nnz_total)
+    cart = {}
+    for key, t, nb in (("cartesian_forward", t_cf, alg["fwd_bytes"]), ("cartesian_backward", t_cb, alg["bwd_bytes"]),
+                       ("spherical_forward", t_sf, alg["fwd_bytes"]), ("spherical_backward", t_sb, alg["bwd_bytes"])):
+        cart[key] = {"ms": t, "GBps": nb / (t * 1e6), "frac_of_hbm_peak": nb / (t * 1e6) / hbm}
+    cart["note"] = ("equal rank: the same graph, weights and path list; both read the edge vectors (no frame "
+                    "records); algorithmic bytes of the spherical step for both")
+    out["cartesian_vs_spherical"] = cart
+    return out
+
+
+# ---------------------------------------------------------------------------
 def main():
     args = parse()
     if args.impl == "reference":
@@ -341,7 +464,7 @@ def main():
     rev_perm = torch.empty(E, dtype=torch.int32, device=dev)
     dst = torch.empty(E, dtype=torch.int32, device=dev)
     ws = torch.empty(max(etp.reverse_csr_workspace_size(N, E), 16), dtype=torch.uint8, device=dev)
-    framed = not args.no_frames
+    framed = plan.frames_advised(E) if args.frames == "auto" else args.frames == "on"
     frames = torch.empty((E, etp.FRAME_FLOATS), device=dev) if framed else None
     lib = etp._load()
     stream = torch.cuda.current_stream()
@@ -497,8 +620,18 @@ def main():
     mhz = (clocks or {}).get("sm_mhz") or (clocks or {}).get("sm_max_mhz") or 1965.0
     fp32_peak = sms * 128 * 2 * mhz * 1e6 / 1e12
     eq = kern[f"{dom}_equiv_TFLOPs"]
-    fp32 = {"kernel": kname, "equiv_tflops": eq, "nominal_peak_tflops": fp32_peak, "frac": eq / fp32_peak,
-            "note": f"nominal = {sms} SMs x 128 lanes x 2 flop x {mhz:.0f} MHz; flop = the method's sparse-CG count"}
+    sparse_cg = {"kernel": kname, "equiv_tflops": eq, "nominal_fp32_peak_tflops": fp32_peak,
+                 "equiv_over_nominal_peak": eq / fp32_peak,
+                 "note": f"NOT an FP32 roofline: the method's plain sparse-CG FLOP count over the kernel time, "
+                         f"which the edge-frame schedule undercuts (it executes fewer FLOPs); nominal = {sms} SMs x "
+                         f"128 lanes x 2 flop x {mhz:.0f} MHz"}
+
+    extra = None
+    if not args.no_extra:
+        try:
+            extra = extra_timings(etp, lib, plan, wl, d, rev_ptr, rev_perm, dst, gw, stream, dev, nnz_total)
+        except Exception as exc:  # reported, not fatal: the step's line stands on its own
+            extra = {"error": f"{type(exc).__name__}: {exc}"}
 
     # end to end through the public API with host buffers (pinned): every step copies its inputs host -> device,
     # runs the path and copies its outputs device -> host, all inside the timed region. Steps are pipelined the
@@ -587,7 +720,7 @@ def main():
                    "l2": f"inputs larger than L2 (w = {wl.w.nbytes / 1e9:.2f} GB streamed per pass)",
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                    "launch": "stream launches" if args.eager else "one CUDA graph replay per step"},
-        "roofline": roofline, "fp32": fp32, "kernels": kern, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches,
+        "roofline": roofline, "sparse_cg_equiv": sparse_cg, "kernels": kern, "beside_the_step": extra, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches,
         "clocks": clocks,
     }), flush=True)
 

@@ -51,6 +51,7 @@ def _load():
         "etp_plan_info": [vp, vp, vp, vp, vp, vp],
         "etp_plan_couplings": [vp, vp, vp, vp, vp, vp, vp],
         "etp_plan_destroy": [vp],
+        "etp_plan_frames_advised": [vp, i32, ctypes.POINTER(i32)],
         "etp_edge_frames": [vp, i32, vp, vp, vp],
         "etp_forward": [vp, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp],
         "etp_backward": [vp, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp],
@@ -176,6 +177,12 @@ class Plan:
         val = (ctypes.c_double * n)()
         _check(lib.etp_plan_couplings(self._h, ctypes.byref(nnz), off, m1, m2, m3, val), "couplings")
         return list(off), list(m1), list(m2), list(m3), list(val)
+
+    def frames_advised(self, E: int) -> bool:
+        """Whether precomputed edge frame records pay for E edges (etp_plan_frames_advised)."""
+        v = ctypes.c_int()
+        _check(_load().etp_plan_frames_advised(self._h, int(E), ctypes.byref(v)), "etp_plan_frames_advised")
+        return bool(v.value)
 
     def close(self):
         if getattr(self, "_h", None) and _lib is not None:

@@ -205,6 +205,14 @@ etp_status etp_edge_frames(etp_plan_t plan, int E, const float* r, float* frames
     return cuda_status(err);
 }
 
+etp_status etp_plan_frames_advised(etp_plan_t plan, int E, int* use_records) {
+    if (!plan || E < 0 || !use_records) return ETP_ERR_INVALID_ARG;
+    const size_t bytes = (size_t)E * ETP_FRAME_FLOATS * sizeof(float);
+    // L <= 1 kernels use no Wigner matrices beyond the rotation itself: records never pay
+    *use_records = (plan->L >= 2 && bytes <= (size_t)64 << 20) ? 1 : 0;
+    return ETP_OK;
+}
+
 etp_status etp_forward(etp_plan_t plan, int N, int E, const int32_t* row_ptr, const int32_t* src, const float* r,
                        const float* frames, const float* x, const float* w, float* out, etp_stream_t stream) {
     if (!plan || N < 0 || E < 0) return ETP_ERR_INVALID_ARG;

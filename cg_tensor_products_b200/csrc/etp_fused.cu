@@ -186,6 +186,8 @@ __host__ __device__ constexpr Smem smem_layout(int Npad, int D, int NW) {
 }
 // Consumer warps: eight (two per TMEM lane quarter, splitting the channel pairs)
 // where the stage fits in shared memory, else four.
+// (Nine warps put three on one scheduler, whose register file then allows 168 per
+// thread: enough for L <= 2, not for the L = 3 Wigner matrices.)
 template <int L>
 constexpr int consumer_warps() { return L <= 2 ? 8 : 4; }
 
@@ -310,8 +312,7 @@ __global__ void __launch_bounds__(consumer_warps<L>() * 32 + 32, 1) etp_fused_fw
         unsigned char* arow_hi = A_hi + tc::kmajor_offset(quarter * 32 + lane, 0, kLBO, kSBO);
         unsigned char* arow_lo = A_lo + tc::kmajor_offset(quarter * 32 + lane, 0, kLBO, kSBO);
         const int kh0 = half * (kHidden / NH), kh1 = kh0 + kHidden / NH;  // this warp's hidden units of A
-        const int my_pairs = (pairs - half + NH - 1) / NH;                   // pairs q = half, half + NH, ...
-        const int n_my = S * my_pairs;                                       // this warp's pairs per tile
+        // this warp's channel pairs: gp = s * pairs + q with gp % NH == half
 
         for (int i = 0; i < ntiles; ++i) {
             const int cb = ra + 32 * i, ce = min(cb + 32, rb);
@@ -392,23 +393,21 @@ __global__ void __launch_bounds__(consumer_warps<L>() * 32 + 32, 1) etp_fused_fw
             };
             float2 xn[D];
             if constexpr (kPrefetchX) load_x(half, xn);
+            const int npairs = S * pairs;
 
             for (int s = 0; s < S; ++s) {
                 const int g = i * S + s, buf = g % kAccBufs;
                 wait_live(&acc_full[buf], (g / kAccBufs) & 1, live);
                 tc::fence_after_sync();
-                for (int q = half; q < pairs; q += NH) {
-                    const int gp = s * pairs + q;  // channel pair index: channels 2 gp, 2 gp + 1
+                for (int gp = s * pairs + ((half - s * pairs) % NH + NH) % NH; gp < (s + 1) * pairs; gp += NH) {
+                    // channel pair gp: channels 2 gp, 2 gp + 1, TMEM pair block q of the slice
+                    const int q = gp - s * pairs;
                     const uint32_t colq = lane_base + (uint32_t)(buf * a.Npad + q * 2 * P);
                     float2 xv[D];
                     if constexpr (kPrefetchX) {
 #pragma unroll
                         for (int k = 0; k < D; ++k) xv[k] = xn[k];
-                        const int nxt = (s * my_pairs + (q - half) / NH) + 1;  // this warp's next pair in the tile
-                        if (nxt < n_my) {
-                            const int sn = nxt / my_pairs, qn = half + (nxt - sn * my_pairs) * NH;
-                            load_x(sn * pairs + qn, xn);
-                        }
+                        if (gp + NH < npairs) load_x(gp + NH, xn);  // this warp's next pair in the tile
                     } else {
                         load_x(gp, xv);
                     }

@@ -143,6 +143,13 @@ ETP_API etp_status etp_plan_destroy(etp_plan_t plan);
  * caller; r: [E][3]. E = 0 launches nothing. */
 ETP_API etp_status etp_edge_frames(etp_plan_t plan, int E, const float* r, float* frames, etp_stream_t stream);
 
+/* Whether precomputed frame records pay for this plan and edge count: 1 when the
+ * records (E x ETP_FRAME_FLOATS x 4 bytes) stay small enough to be read back from
+ * L2 by both kernels (at most 64 MB; the 1024-node micro-benchmark graph: 46 MB),
+ * else 0 (then the kernels build the frames themselves, cheaper than streaming the
+ * records from HBM: 440 MB at 1.25 M edges). Host only. */
+ETP_API etp_status etp_plan_frames_advised(etp_plan_t plan, int E, int* use_records);
+
 /* Forward: out[i] = sum_{e in row i} msg_e (see above), for all N rows.
  * x: [N][D][C], w: [E][P][C], r: [E][3], out: [N][D][C] device pointers.
  * frames: NULL (the kernel builds each edge's frame from r), or the records

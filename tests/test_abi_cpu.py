@@ -23,7 +23,7 @@ def lib():
 
 def test_exports_every_declared_symbol(lib):
     names = etp.declared_symbols()
-    assert len(names) == 22
+    assert len(names) == 23
     for n in names:
         assert hasattr(lib, n), n
 
@@ -198,3 +198,10 @@ def test_fused_workspace_size_and_refusals(lib):
     assert e.value.status == etp.ETP_ERR_UNSUPPORTED
     with pytest.raises(etp.EtpError):
         etp.fused_workspace_size(plan, 100, n_basis=8, hidden=128)
+
+
+def test_frames_advised_by_size(lib):
+    """Frame records pay while they stay small enough for L2; never at L <= 1."""
+    assert etp.Plan("0..3", 3, "0..3", 128).frames_advised(131072)          # 46 MB of records
+    assert not etp.Plan("0..3", 3, "0..3", 64).frames_advised(1250256)     # 440 MB
+    assert not etp.Plan("0..1", 1, "0..1", 8).frames_advised(256)

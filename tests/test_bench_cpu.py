@@ -41,5 +41,5 @@ def test_default_timing_settings(monkeypatch):
     monkeypatch.setattr(sys, "argv", ["bench.py"])
     args = bench.parse()
     assert args.gpus == 1 and args.warmup >= 3 and args.steps >= 1 and args.workload == "micro_l3"
-    assert not args.eager and not args.no_frames and args.impl == "ours"
+    assert not args.eager and args.frames == "auto" and args.impl == "ours"
     assert args.workload in bench.DESCR and set(bench.DESCR) == set(workloads.SPECS)
