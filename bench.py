@@ -305,6 +305,13 @@ def reference_arm(args):
 
 
 # ---------------------------------------------------------------------------
+def stream_ptr(stream):
+    """A torch stream as the C ABI's stream argument."""
+    import ctypes
+
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
 def _time_ms(fn, stream, reps=10, warm=3):
     import torch
 
@@ -340,7 +347,7 @@ def extra_timings(etp, lib, plan, wl, d, rev_ptr, rev_perm, dst, gw, stream, dev
     import torch
 
     P = etp._ptr
-    sp = etp._stream(stream)
+    sp = stream_ptr(stream)
     N, E, C, Pn = wl.N, wl.E, wl.C, plan.n_paths
     D = (wl.L + 1) ** 2
     node = N * D * C * 4
@@ -468,7 +475,7 @@ def main():
     frames = torch.empty((E, etp.FRAME_FLOATS), device=dev) if framed else None
     lib = etp._load()
     stream = torch.cuda.current_stream()
-    sp = etp._stream(stream)
+    sp = stream_ptr(stream)
     P = etp._ptr
 
     def step(ev=None, b=None, s=None):
@@ -476,7 +483,7 @@ def main():
         CSR, frames and workspace are shared scratch (every use is ordered on the one compute stream)."""
         b = d if b is None else b
         s = stream if s is None else s
-        spp = etp._stream(s)
+        spp = stream_ptr(s)
         if ev:
             ev[0].record(s)
         etp._check(lib.etp_build_reverse_csr(N, E, P(b["row_ptr"]), P(b["src"]), P(rev_ptr), P(rev_perm), P(dst),

@@ -403,6 +403,9 @@ __global__ void __launch_bounds__(consumer_warps<L>() * 32 + 32, 1) etp_fused_fw
                     // channel pair gp: channels 2 gp, 2 gp + 1, TMEM pair block q of the slice
                     const int q = gp - s * pairs;
                     const uint32_t colq = lane_base + (uint32_t)(buf * a.Npad + q * 2 * P);
+                    const bool col = lane < 2 * D;
+                    // the row carried in from the previous chunk: loaded now, used after the pair's compute
+                    const float cin = (carried && col) ? carry[(size_t)gp * 32] : 0.f;
                     float2 xv[D];
                     if constexpr (kPrefetchX) {
 #pragma unroll
@@ -472,7 +475,6 @@ __global__ void __launch_bounds__(consumer_warps<L>() * 32 + 32, 1) etp_fused_fw
                     __syncwarp();
                     // sum the rows of equal destination, in row order; lane k < 2D owns column k
                     // (component k / 2, channel 2 gp + k % 2); rows without an edge hold zeros
-                    const bool col = lane < 2 * D;
                     float vr[32];
 #pragma unroll
                     for (int rr = 0; rr < 32; ++rr) vr[rr] = stage[rr * STR + (col ? lane : 0)];
@@ -492,7 +494,6 @@ __global__ void __launch_bounds__(consumer_warps<L>() * 32 + 32, 1) etp_fused_fw
                             }
                         }
                     };
-                    const float cin = (carried && col) ? carry[(size_t)gp * 32] : 0.f;
                     if (one_segment) {
 #pragma unroll
                         for (int w = 16; w >= 1; w >>= 1)
