@@ -31,8 +31,8 @@
 // summed in registers and stored once (a row cut by a task boundary is added by
 // vector reduction onto the zeroed output):
 //   dd_dst: CSR order, grad_g;
-//   dd_src: reverse-CSR order, grad_x, and per edge grad_w and grad_r. Its frame
-//           vectors (x', gg_x', g', K_w x', K_w g') sit in lane-owned shared memory.
+//   dd_src: reverse-CSR order, grad_x, and per edge grad_w and grad_r.
+// The frame vectors of an edge sit in lane-owned shared memory (registers).
 // Per-edge weights and cotangents are read straight from global memory (coalesced
 // over the team's channels).
 #include <cuda_runtime.h>
@@ -183,6 +183,18 @@ __device__ __forceinline__ void load_fit(float* fit) {
     __syncthreads();
 }
 
+// Per team in shared memory: the Wigner buffers, then lane-owned frame vectors
+// [v][k] float2 (the destination kernel: x', ggx' + K_w x'; the source kernel:
+// x', ggx', g', K_w x', K_w g').
+template <int L>
+constexpr int dst_team_floats(int T) {
+    return frame::kTeamFloats + 2 * (L + 1) * (L + 1) * T * 2;
+}
+template <int L>
+constexpr int src_team_floats(int T) {
+    return frame::kTeamFloats + 5 * (L + 1) * (L + 1) * T * 2;
+}
+
 // ---------------------------------------------------------------------------
 // grad_g: destination order.
 template <int L, bool O3>
@@ -196,9 +208,11 @@ __global__ void __launch_bounds__(kThreads) etp_dd_dst_kernel(Args a) {
     int k0, k1;
     task_range(a.E, tm.task, a.ntasks, k0, k1);
     if (k0 >= k1) return;
-    const int C2 = a.C2;
-    float* ybuf = smem + kFitStride + tm.tb * kTeamFloats;
+    const int C2 = a.C2, T = tm.T;
+    float* ybuf = smem + kFitStride + tm.tb * dst_team_floats<L>(T);
     float* dbuf = ybuf + kYbufFloats;
+    float2* vec = reinterpret_cast<float2*>(ybuf + kTeamFloats) + tm.tl;  // [v][k] at (v * D + k) * T
+    auto V = [&](int v, int k) -> float2& { return vec[(v * D + k) * T]; };
     int row = segment_of(a.row_ptr, a.N, k0);
     int row_lo = __ldg(a.row_ptr + row), row_hi = __ldg(a.row_ptr + row + 1);
     float2 acc[D];
@@ -223,12 +237,6 @@ __global__ void __launch_bounds__(kThreads) etp_dd_dst_kernel(Args a) {
         const float2* gxs = a.ggx ? a.ggx + (size_t)j * D * C2 + tm.cp : nullptr;
         const float2* wrow = a.w + (size_t)e * PathSet<L, O3>::P * C2 + tm.cp;
         const float2* gwrow = a.ggw ? a.ggw + (size_t)e * PathSet<L, O3>::P * C2 + tm.cp : nullptr;
-        float2 xv[D], gxv[D];
-#pragma unroll
-        for (int k = 0; k < D; ++k) {
-            xv[k] = __ldg(xs + k * C2);
-            gxv[k] = gxs ? __ldg(gxs + k * C2) : f2_zero();
-        }
         if (!f.degenerate) {
             team_wigner<L>(f, tm.tl, tm.T, tm.tmask, ybuf, dbuf, smem);
             float wx = 0.f, wy = 0.f;
@@ -240,15 +248,26 @@ __global__ void __launch_bounds__(kThreads) etp_dd_dst_kernel(Args a) {
                 wx = vy;
                 wy = -vx;
             }
-            float2 xp[D], sum[D];
-            rotate_all2<L>(f, dbuf, xv, gxv, xp, sum);  // sum = ggx' (+ K_w x' below)
-            static_for<0, L + 1>([&](auto lc) {
-                constexpr int l = decltype(lc)::value;
-                float2 t[2 * l + 1];
-                gen_apply<l>(wx, wy, xp + l * l, t);
+            {  // x' (vector 0) and ggx' + K_w x' (vector 1) into this lane's shared-memory rows
+                float2 v[D], u[D];
 #pragma unroll
-                for (int m = 0; m < 2 * l + 1; ++m) sum[l * l + m] = f2_add(sum[l * l + m], t[m]);
-            });
+                for (int k = 0; k < D; ++k) v[k] = __ldg(xs + k * C2);
+                rotate_all<L>(f, dbuf, v, u);
+#pragma unroll
+                for (int k = 0; k < D; ++k) {
+                    V(0, k) = u[k];
+                    v[k] = gxs ? __ldg(gxs + k * C2) : f2_zero();
+                }
+                float2 gp[D];
+                rotate_all<L>(f, dbuf, v, gp);
+                static_for<0, L + 1>([&](auto lc) {
+                    constexpr int l = decltype(lc)::value;
+                    float2 t[2 * l + 1];
+                    gen_apply<l>(wx, wy, u + l * l, t);
+#pragma unroll
+                    for (int m = 0; m < 2 * l + 1; ++m) V(1, l * l + m) = f2_add(gp[l * l + m], t[m]);
+                });
+            }
             static_for<0, L + 1>([&](auto l3c) {
                 constexpr int l3 = decltype(l3c)::value;
                 constexpr int d3 = 2 * l3 + 1;
@@ -258,13 +277,19 @@ __global__ void __launch_bounds__(kThreads) etp_dd_dst_kernel(Args a) {
                 static_for<0, L + 1>([&](auto l1c) {
                     constexpr int l1 = decltype(l1c)::value;
                     if constexpr (has_type<L, O3>(l1, l3, 0) || has_type<L, O3>(l1, l3, 1)) {
+                        float2 xp[2 * l1 + 1], sum[2 * l1 + 1];
+#pragma unroll
+                        for (int m = 0; m < 2 * l1 + 1; ++m) {
+                            xp[m] = V(0, l1 * l1 + m);
+                            sum[m] = V(1, l1 * l1 + m);
+                        }
                         float2 We[4], Wo[4];
                         group_weights_g<L, O3, l1, l3>(wrow, C2, We, Wo);
-                        apply_M<L, O3, l1, l3>(We, Wo, sum + l1 * l1, y);
-                        apply_M<L, O3, l1, l3>(We, Wo, xp + l1 * l1, y3);
+                        apply_M<L, O3, l1, l3>(We, Wo, sum, y);
+                        apply_M<L, O3, l1, l3>(We, Wo, xp, y3);
                         if (gwrow) {
                             group_weights_g<L, O3, l1, l3>(gwrow, C2, We, Wo);
-                            apply_M<L, O3, l1, l3>(We, Wo, xp + l1 * l1, y);
+                            apply_M<L, O3, l1, l3>(We, Wo, xp, y);
                         }
                     }
                 });
@@ -283,8 +308,8 @@ __global__ void __launch_bounds__(kThreads) etp_dd_dst_kernel(Args a) {
                 const float2 gw0 = gwrow ? __ldg(gwrow + p0 * C2) : f2_zero();
 #pragma unroll
                 for (int m = 0; m < 2 * l + 1; ++m) {
-                    f2_fma(acc[l * l + m], w0, gxv[l * l + m]);
-                    f2_fma(acc[l * l + m], gw0, xv[l * l + m]);
+                    if (gxs) f2_fma(acc[l * l + m], w0, __ldg(gxs + (l * l + m) * C2));
+                    f2_fma(acc[l * l + m], gw0, __ldg(xs + (l * l + m) * C2));
                 }
             });
         }
@@ -292,14 +317,6 @@ __global__ void __launch_bounds__(kThreads) etp_dd_dst_kernel(Args a) {
     if (a.grad_g) flush_row<D>(a.grad_g + (size_t)row * D * C2 + tm.cp, C2, acc, row_lo >= k0 && row_hi <= k1);
 }
 
-// ---------------------------------------------------------------------------
-// grad_x (source order), grad_w and grad_r (per edge).
-// Lane-owned frame vectors in shared memory: [5][D] float2 per lane.
-constexpr int kVecs = 5;
-template <int L>
-constexpr int src_team_floats(int T) {
-    return frame::kTeamFloats + kVecs * (L + 1) * (L + 1) * T * 2;
-}
 
 template <int L, bool O3>
 __global__ void __launch_bounds__(kThreads) etp_dd_src_kernel(Args a) {
@@ -560,7 +577,7 @@ __global__ void __launch_bounds__(kThreads) etp_dd_src_kernel(Args a) {
 template <int L, bool O3>
 size_t smem_for(bool src_side, int T) {
     const int teams = kThreads / T;
-    return sizeof(float) * (size_t)(frame::kFitStride + teams * (src_side ? src_team_floats<L>(T) : frame::kTeamFloats));
+    return sizeof(float) * (size_t)(frame::kFitStride + teams * (src_side ? src_team_floats<L>(T) : dst_team_floats<L>(T)));
 }
 
 }  // namespace dd
@@ -577,6 +594,8 @@ cudaError_t launch_dd(dd::Args a, cudaStream_t s) {
     const void* ks = (const void*)dd::etp_dd_src_kernel<L, O3>;
     cudaError_t err;
     if ((err = cudaFuncSetAttribute(ks, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_src)) != cudaSuccess)
+        return err;
+    if ((err = cudaFuncSetAttribute(kd, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_dst)) != cudaSuccess)
         return err;
     int dev = 0, sms = 1, bps_d = 1, bps_s = 1;
     if ((err = cudaGetDevice(&dev)) != cudaSuccess) return err;
