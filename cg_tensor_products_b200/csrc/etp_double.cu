@@ -32,9 +32,9 @@
 // vector reduction onto the zeroed output):
 //   dd_dst: CSR order, grad_g;
 //   dd_src: reverse-CSR order, grad_x, and per edge grad_w and grad_r.
-// The frame vectors of an edge sit in lane-owned shared memory (registers).
-// Per-edge weights and cotangents are read straight from global memory (coalesced
-// over the team's channels).
+// The frame vectors of an edge sit in lane-owned shared memory (registers), and so
+// do the edge's weight and cotangent-weight rows, copied in asynchronously at the
+// start of the edge (their latency hides behind the frame work).
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -186,13 +186,29 @@ __device__ __forceinline__ void load_fit(float* fit) {
 // Per team in shared memory: the Wigner buffers, then lane-owned frame vectors
 // [v][k] float2 (the destination kernel: x', ggx' + K_w x'; the source kernel:
 // x', ggx', g', K_w x', K_w g').
-template <int L>
+// After those, lane-owned rows of the edge's weights and cotangent weights
+// ([p][lane] float2 each), filled by per-lane asynchronous copies at the start of
+// the edge so that the frame work hides their latency; in the source kernel the
+// destination's g row arrives the same way, in the slot of its frame vector.
+template <int L, bool O3>
 constexpr int dst_team_floats(int T) {
-    return frame::kTeamFloats + 2 * (L + 1) * (L + 1) * T * 2;
+    return frame::kTeamFloats + (2 * (L + 1) * (L + 1) + 2 * PathSet<L, O3>::P) * T * 2;
 }
-template <int L>
+template <int L, bool O3>
 constexpr int src_team_floats(int T) {
-    return frame::kTeamFloats + 5 * (L + 1) * (L + 1) * T * 2;
+    return frame::kTeamFloats + (3 * (L + 1) * (L + 1) + 2 * PathSet<L, O3>::P) * T * 2;
+}
+
+// This lane's channel pair of every path of two weight rows, into lane-owned
+// shared memory (rows at p * T), by 8-byte asynchronous copies; one commit group.
+template <int P>
+__device__ __forceinline__ void copy_weight_rows(float2* wbuf, float2* gwbuf, const float2* wrow, const float2* gwrow,
+                                                 int C2, int T) {
+#pragma unroll
+    for (int p = 0; p < P; ++p) {
+        frame::cp_async8(wbuf + p * T, wrow + p * C2);
+        if (gwrow) frame::cp_async8(gwbuf + p * T, gwrow + p * C2);
+    }
 }
 
 // ---------------------------------------------------------------------------
@@ -208,11 +224,14 @@ __global__ void __launch_bounds__(kThreads) etp_dd_dst_kernel(Args a) {
     int k0, k1;
     task_range(a.E, tm.task, a.ntasks, k0, k1);
     if (k0 >= k1) return;
+    constexpr int P = PathSet<L, O3>::P;
     const int C2 = a.C2, T = tm.T;
-    float* ybuf = smem + kFitStride + tm.tb * dst_team_floats<L>(T);
+    float* ybuf = smem + kFitStride + tm.tb * dst_team_floats<L, O3>(T);
     float* dbuf = ybuf + kYbufFloats;
     float2* vec = reinterpret_cast<float2*>(ybuf + kTeamFloats) + tm.tl;  // [v][k] at (v * D + k) * T
     auto V = [&](int v, int k) -> float2& { return vec[(v * D + k) * T]; };
+    float2* wbuf = vec + 2 * D * T;  // [p] at p * T
+    float2* gwbuf = wbuf + P * T;
     int row = segment_of(a.row_ptr, a.N, k0);
     int row_lo = __ldg(a.row_ptr + row), row_hi = __ldg(a.row_ptr + row + 1);
     float2 acc[D];
@@ -235,8 +254,10 @@ __global__ void __launch_bounds__(kThreads) etp_dd_dst_kernel(Args a) {
         const Frame f = make_frame(rv.x, rv.y, rv.z);
         const float2* xs = a.x + (size_t)j * D * C2 + tm.cp;
         const float2* gxs = a.ggx ? a.ggx + (size_t)j * D * C2 + tm.cp : nullptr;
-        const float2* wrow = a.w + (size_t)e * PathSet<L, O3>::P * C2 + tm.cp;
-        const float2* gwrow = a.ggw ? a.ggw + (size_t)e * PathSet<L, O3>::P * C2 + tm.cp : nullptr;
+        const float2* wrow = a.w + (size_t)e * P * C2 + tm.cp;
+        const float2* gwrow = a.ggw ? a.ggw + (size_t)e * P * C2 + tm.cp : nullptr;
+        copy_weight_rows<P>(wbuf, gwbuf, wrow, gwrow, C2, T);
+        cp_async_commit();
         if (!f.degenerate) {
             team_wigner<L>(f, tm.tl, tm.T, tm.tmask, ybuf, dbuf, smem);
             float wx = 0.f, wy = 0.f;
@@ -268,6 +289,7 @@ __global__ void __launch_bounds__(kThreads) etp_dd_dst_kernel(Args a) {
                     for (int m = 0; m < 2 * l + 1; ++m) V(1, l * l + m) = f2_add(gp[l * l + m], t[m]);
                 });
             }
+            cp_async_wait_all();  // this lane's weight rows
             static_for<0, L + 1>([&](auto l3c) {
                 constexpr int l3 = decltype(l3c)::value;
                 constexpr int d3 = 2 * l3 + 1;
@@ -284,11 +306,11 @@ __global__ void __launch_bounds__(kThreads) etp_dd_dst_kernel(Args a) {
                             sum[m] = V(1, l1 * l1 + m);
                         }
                         float2 We[4], Wo[4];
-                        group_weights_g<L, O3, l1, l3>(wrow, C2, We, Wo);
+                        group_weights<L, O3, l1, l3>(wbuf, T, We, Wo);
                         apply_M<L, O3, l1, l3>(We, Wo, sum, y);
                         apply_M<L, O3, l1, l3>(We, Wo, xp, y3);
                         if (gwrow) {
-                            group_weights_g<L, O3, l1, l3>(gwrow, C2, We, Wo);
+                            group_weights<L, O3, l1, l3>(gwbuf, T, We, Wo);
                             apply_M<L, O3, l1, l3>(We, Wo, xp, y);
                         }
                     }
@@ -301,6 +323,7 @@ __global__ void __launch_bounds__(kThreads) etp_dd_dst_kernel(Args a) {
             });
         } else {
             // no direction: only the paths (l, 0, l) act, each as the identity; no derivative in r
+            cp_async_wait_all();
             static_for<0, L + 1>([&](auto lc) {
                 constexpr int l = decltype(lc)::value;
                 constexpr int p0 = path_index<L, O3>(l, 0, l);
@@ -331,11 +354,13 @@ __global__ void __launch_bounds__(kThreads) etp_dd_src_kernel(Args a) {
     task_range(a.E, tm.task, a.ntasks, k0, k1);
     if (k0 >= k1) return;
     const int C2 = a.C2, T = tm.T;
-    float* ybuf = smem + kFitStride + tm.tb * src_team_floats<L>(T);
+    float* ybuf = smem + kFitStride + tm.tb * src_team_floats<L, O3>(T);
     float* dbuf = ybuf + kYbufFloats;
     float2* vec = reinterpret_cast<float2*>(ybuf + kTeamFloats) + tm.tl;  // [v][k] at (v * D + k) * T
     auto V = [&](int v, int k) -> float2& { return vec[(v * D + k) * T]; };
-    enum { XP = 0, GXP = 1, GP = 2, XT = 3, GT = 4 };
+    enum { XP = 0, GXP = 1, GP = 2 };  // x', ggx', g' (the g row is copied into the g' slot, then rotated)
+    float2* wbuf = vec + 3 * D * T;  // [p] at p * T
+    float2* gwbuf = wbuf + P * T;
 
     int row = segment_of(a.rev_ptr, a.N, k0);
     int row_lo = __ldg(a.rev_ptr + row), row_hi = __ldg(a.rev_ptr + row + 1);
@@ -397,6 +422,11 @@ __global__ void __launch_bounds__(kThreads) etp_dd_src_kernel(Args a) {
             if (write_r && tm.slice == 0) a.grad_r[3 * (size_t)e] = a.grad_r[3 * (size_t)e + 1] = a.grad_r[3 * (size_t)e + 2] = 0.f;
             continue;
         }
+        // this edge's weight rows and g row, in flight while the frame is built
+        copy_weight_rows<P>(wbuf, gwbuf, wrow, gwrow, C2, T);
+#pragma unroll
+        for (int k = 0; k < D; ++k) cp_async8(&V(GP, k), gs + k * C2);
+        cp_async_commit();
         team_wigner<L>(f, tm.tl, T, tm.tmask, ybuf, dbuf, smem);
         float wx = 0.f, wy = 0.f, vz = 0.f;
         if (a.ggr) {
@@ -408,7 +438,7 @@ __global__ void __launch_bounds__(kThreads) etp_dd_src_kernel(Args a) {
             wx = vy;
             wy = -vx;
         }
-        // frame vectors: x', ggx', g', K_w x', K_w g'
+        // frame vectors x', ggx', g' (K_w x' and K_w g' are formed block by block where used)
         {
             float2 u[D], v[D], up[D], vp[D];
 #pragma unroll
@@ -417,25 +447,16 @@ __global__ void __launch_bounds__(kThreads) etp_dd_src_kernel(Args a) {
                 v[k] = gxs ? __ldg(gxs + k * C2) : f2_zero();
             }
             rotate_all2<L>(f, dbuf, u, v, up, vp);
+            cp_async_wait_all();  // this lane's weight rows and g row
 #pragma unroll
             for (int k = 0; k < D; ++k) {
                 V(XP, k) = up[k];
                 V(GXP, k) = vp[k];
-                u[k] = __ldg(gs + k * C2);
+                u[k] = V(GP, k);
             }
             rotate_all<L>(f, dbuf, u, v);
-            static_for<0, L + 1>([&](auto lc) {
-                constexpr int l = decltype(lc)::value;
-                float2 t1[2 * l + 1], t2[2 * l + 1];
-                gen_apply<l>(wx, wy, up + l * l, t1);
-                gen_apply<l>(wx, wy, v + l * l, t2);
 #pragma unroll
-                for (int m = 0; m < 2 * l + 1; ++m) {
-                    V(GP, l * l + m) = v[l * l + m];
-                    V(XT, l * l + m) = t1[m];
-                    V(GT, l * l + m) = t2[m];
-                }
-            });
+            for (int k = 0; k < D; ++k) V(GP, k) = v[k];
         }
         float2 c0 = f2_zero(), c1 = f2_zero(), c2 = f2_zero();
         // (1) blocks l1: z = M^T g', zt = M^T K_w g', z2 = M(gg_w)^T g'; grad_x; the x-side forms
@@ -449,16 +470,14 @@ __global__ void __launch_bounds__(kThreads) etp_dd_src_kernel(Args a) {
                 constexpr int l3 = decltype(l3c)::value;
                 if constexpr (has_type<L, O3>(l1, l3, 0) || has_type<L, O3>(l1, l3, 1)) {
 #pragma unroll
-                    for (int m = 0; m < 2 * l3 + 1; ++m) {
-                        gp3[m] = V(GP, l3 * l3 + m);
-                        gt3[m] = V(GT, l3 * l3 + m);
-                    }
+                    for (int m = 0; m < 2 * l3 + 1; ++m) gp3[m] = V(GP, l3 * l3 + m);
+                    gen_apply<l3>(wx, wy, gp3, gt3);
                     float2 We[4], Wo[4];
-                    group_weights_g<L, O3, l1, l3>(wrow, C2, We, Wo);
+                    group_weights<L, O3, l1, l3>(wbuf, T, We, Wo);
                     apply_MT<L, O3, l1, l3>(We, Wo, gp3, z);
                     apply_MT<L, O3, l1, l3>(We, Wo, gt3, zt);
                     if (gwrow) {
-                        group_weights_g<L, O3, l1, l3>(gwrow, C2, We, Wo);
+                        group_weights<L, O3, l1, l3>(gwbuf, T, We, Wo);
                         apply_MT<L, O3, l1, l3>(We, Wo, gp3, z2);
                     }
                 }
@@ -492,8 +511,8 @@ __global__ void __launch_bounds__(kThreads) etp_dd_src_kernel(Args a) {
             for (int m = 0; m < d3; ++m) {
                 y[m] = yt[m] = y56[m] = f2_zero();
                 gp3[m] = V(GP, l3 * l3 + m);
-                gt3[m] = V(GT, l3 * l3 + m);
             }
+            gen_apply<l3>(wx, wy, gp3, gt3);
             static_for<0, L + 1>([&](auto l1c) {
                 constexpr int l1 = decltype(l1c)::value;
                 if constexpr (has_type<L, O3>(l1, l3, 0) || has_type<L, O3>(l1, l3, 1)) {
@@ -502,16 +521,16 @@ __global__ void __launch_bounds__(kThreads) etp_dd_src_kernel(Args a) {
 #pragma unroll
                     for (int m = 0; m < d1; ++m) {
                         xp1[m] = V(XP, l1 * l1 + m);
-                        xt1[m] = V(XT, l1 * l1 + m);
                         gxp1[m] = V(GXP, l1 * l1 + m);
                     }
+                    gen_apply<l1>(wx, wy, xp1, xt1);
                     float2 We[4], Wo[4];
-                    group_weights_g<L, O3, l1, l3>(wrow, C2, We, Wo);
+                    group_weights<L, O3, l1, l3>(wbuf, T, We, Wo);
                     apply_M<L, O3, l1, l3>(We, Wo, xp1, y);
                     apply_M<L, O3, l1, l3>(We, Wo, xt1, yt);
                     apply_M<L, O3, l1, l3>(We, Wo, gxp1, y56);
                     if (gwrow) {
-                        group_weights_g<L, O3, l1, l3>(gwrow, C2, We, Wo);
+                        group_weights<L, O3, l1, l3>(gwbuf, T, We, Wo);
                         apply_M<L, O3, l1, l3>(We, Wo, xp1, y56);
                     }
                     if (gwe) {
@@ -577,7 +596,8 @@ __global__ void __launch_bounds__(kThreads) etp_dd_src_kernel(Args a) {
 template <int L, bool O3>
 size_t smem_for(bool src_side, int T) {
     const int teams = kThreads / T;
-    return sizeof(float) * (size_t)(frame::kFitStride + teams * (src_side ? src_team_floats<L>(T) : dst_team_floats<L>(T)));
+    return sizeof(float) *
+           (size_t)(frame::kFitStride + teams * (src_side ? src_team_floats<L, O3>(T) : dst_team_floats<L, O3>(T)));
 }
 
 }  // namespace dd
