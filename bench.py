@@ -58,6 +58,9 @@ def parse():
     ap.add_argument("--frames", choices=["auto", "on", "off"], default="auto",
                     help="edge frame records: as the plan advises (auto), always, or never (the kernels build "
                          "the frames themselves)")
+    ap.add_argument("--schedule", choices=["auto", "on", "off"], default="auto",
+                    help="locality schedule (rows in the Morton order of the atom positions, several waves of "
+                         "tasks): auto = on for workloads with positions whose node features exceed half of L2")
     ap.add_argument("--no-extra", action="store_true",
                     help="skip the timings beside the step: the fused radial-weights forward, the VJP of the VJP "
                          "and the Cartesian edge convolution")
@@ -187,12 +190,13 @@ def kernel_source_hash():
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(kernel, framed, workload, n_nodes):
+def recorded_traffic(kernel, framed, workload, n_nodes, scheduled=False):
     """DRAM bytes (read + write) per launch from a committed ncu capture of the same
     kernel source and launch, else None. The summaries under profiles/ carry lines
-    `traffic: <kernel> framed=<0|1> workload=<name> nodes=<N> source=<hash> bytes=<B>`."""
+    `traffic: <kernel> framed=<0|1> workload=<name> nodes=<N> source=<hash> bytes=<B>`
+    (with `schedule=1` for a launch on a locality schedule)."""
     want = {"kernel": kernel, "framed": str(int(framed)), "workload": workload, "nodes": str(n_nodes),
-            "source": kernel_source_hash()}
+            "source": kernel_source_hash(), "schedule": "1" if scheduled else None}
     pdir = os.path.join(ROOT, "profiles")
     try:
         names = sorted(os.listdir(pdir))
@@ -459,6 +463,12 @@ def main():
     nnz_total = len(plan.couplings()[1])
     N, E = wl.N, wl.E
     host = {k: torch.from_numpy(np.ascontiguousarray(getattr(wl, k))) for k in ("row_ptr", "src", "r", "x", "w", "g")}
+    big_nodes = wl.x.nbytes > 64e6  # node features above half of L2: their gathers miss L2 in id order
+    scheduled = (wl.pos is not None and big_nodes) if args.schedule == "auto" else args.schedule == "on"
+    if scheduled:
+        if wl.pos is None:
+            raise SystemExit(f"--schedule on: workload {args.workload} has no atom positions")
+        host["pos"] = torch.from_numpy(np.ascontiguousarray(wl.pos))
 
     def io_buffers():
         """A step's inputs (a device copy of `host`) and outputs."""
@@ -474,7 +484,13 @@ def main():
     rev_ptr = torch.empty(N + 1, dtype=torch.int32, device=dev)
     rev_perm = torch.empty(E, dtype=torch.int32, device=dev)
     dst = torch.empty(E, dtype=torch.int32, device=dev)
-    ws = torch.empty(max(etp.reverse_csr_workspace_size(N, E), 16), dtype=torch.uint8, device=dev)
+    ws_bytes = etp.reverse_csr_workspace_size(N, E)
+    if scheduled:
+        ws_bytes = max(ws_bytes, etp.locality_schedule_workspace_size(N, E))
+        sched = etp.Schedule(N, E, torch.empty(N, dtype=torch.int32, device=dev),
+                             torch.empty(N + 1, dtype=torch.int32, device=dev),
+                             torch.empty(E, dtype=torch.int32, device=dev), rev_ptr, rev_perm, dst)
+    ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
     framed = plan.frames_advised(E) if args.frames == "auto" else args.frames == "on"
     frames = torch.empty((E, etp.FRAME_FLOATS), device=dev) if framed else None
     lib = etp._load()
@@ -490,21 +506,36 @@ def main():
         spp = stream_ptr(s)
         if ev:
             ev[0].record(s)
-        etp._check(lib.etp_build_reverse_csr(N, E, P(b["row_ptr"]), P(b["src"]), P(rev_ptr), P(rev_perm), P(dst),
-                                             P(ws), ws.numel(), spp), "reverse csr")
+        if scheduled:
+            etp._check(lib.etp_build_locality_schedule(N, E, P(b["row_ptr"]), P(b["src"]), P(b["pos"]),
+                                                       float(wl.graph_cutoff), *[P(t) for t in sched.tensors()],
+                                                       P(ws), ws.numel(), spp), "locality schedule")
+        else:
+            etp._check(lib.etp_build_reverse_csr(N, E, P(b["row_ptr"]), P(b["src"]), P(rev_ptr), P(rev_perm),
+                                                 P(dst), P(ws), ws.numel(), spp), "reverse csr")
         if ev:
             ev[1].record(s)
         if framed:
             etp._check(lib.etp_edge_frames(plan.handle, E, P(b["r"]), P(frames), spp), "edge frames")
         if ev:
             ev[2].record(s)
-        etp._check(lib.etp_forward(plan.handle, N, E, P(b["row_ptr"]), P(b["src"]), P(b["r"]), P(frames), P(b["x"]),
-                                   P(b["w"]), P(b["out"]), spp), "forward")
+        if scheduled:
+            etp._check(lib.etp_forward_ordered(plan.handle, N, E, P(sched.order), P(sched.ord_ptr),
+                                               P(sched.ord_edge), P(b["src"]), P(b["r"]), P(frames), P(b["x"]),
+                                               P(b["w"]), P(b["out"]), spp), "forward (scheduled)")
+        else:
+            etp._check(lib.etp_forward(plan.handle, N, E, P(b["row_ptr"]), P(b["src"]), P(b["r"]), P(frames),
+                                       P(b["x"]), P(b["w"]), P(b["out"]), spp), "forward")
         if ev:
             ev[3].record(s)
-        etp._check(lib.etp_backward(plan.handle, N, E, P(b["row_ptr"]), P(b["src"]), P(rev_ptr), P(rev_perm), P(dst),
-                                    P(b["r"]), P(frames), P(b["x"]), P(b["w"]), P(b["g"]), P(b["gx"]), P(b["gw"]),
-                                    P(b["gr"]), spp), "backward")
+        if scheduled:
+            etp._check(lib.etp_backward_ordered(plan.handle, N, E, P(sched.order), P(rev_ptr), P(rev_perm), P(dst),
+                                                P(b["r"]), P(frames), P(b["x"]), P(b["w"]), P(b["g"]), P(b["gx"]),
+                                                P(b["gw"]), P(b["gr"]), spp), "backward (scheduled)")
+        else:
+            etp._check(lib.etp_backward(plan.handle, N, E, P(b["row_ptr"]), P(b["src"]), P(rev_ptr), P(rev_perm),
+                                        P(dst), P(b["r"]), P(frames), P(b["x"]), P(b["w"]), P(b["g"]), P(b["gx"]),
+                                        P(b["gw"]), P(b["gr"]), spp), "backward")
         if ev:
             ev[4].record(s)
 
@@ -559,7 +590,9 @@ def main():
     alg = algorithmic(wl, plan.n_paths, nnz_total)
     peak, peak_kind = measured_peaks()
     fl_fwd, fl_bwd = flops(wl.L, plan.paths, nnz_total, wl.C, E)
-    kern = {"reverse_csr_ms": rc_ms, "edge_frames_ms": fr_ms if framed else None,
+    kern = {"graph_prep": "locality schedule" if scheduled else "reverse CSR",
+            "reverse_csr_ms" if not scheduled else "locality_schedule_ms": rc_ms,
+            "edge_frames_ms": fr_ms if framed else None,
             "forward_ms": fwd_ms, "backward_ms": bwd_ms,
             "forward_GBps": alg["fwd_bytes"] / (fwd_ms * 1e6), "backward_GBps": alg["bwd_bytes"] / (bwd_ms * 1e6),
             "forward_equiv_TFLOPs": fl_fwd / (fwd_ms * 1e9), "backward_equiv_TFLOPs": fl_bwd / (bwd_ms * 1e9),
@@ -571,7 +604,10 @@ def main():
     roofline = {"bound": "hbm", "kernel": f"{kname} ({'frames given' if framed else 'frames built in the kernel'})",
                 "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                 "peak_source": f"{peak_kind} (hbm_gbs, burst copy)",
-                "traffic": recorded_traffic(kname, framed, args.workload, N)}
+                "traffic": recorded_traffic(kname, framed, args.workload, N, scheduled)}
+    if scheduled:  # the calls below take the reverse CSR in source-id order
+        etp._check(lib.etp_build_reverse_csr(N, E, P(d["row_ptr"]), P(d["src"]), P(rev_ptr), P(rev_perm), P(dst),
+                                             P(ws), ws.numel(), sp), "reverse csr")
 
     # force assembly from grad_r (a separate call, not part of the step): forces and per-atom virials
     forces_t = torch.empty((N, 3), device=dev)
@@ -710,6 +746,9 @@ def main():
         while (1 << (8 * passes)) < N and passes < 4:
             passes += 1
         rc_launches = (1 if E > 0 else 0) + 1 + (1 if E > 0 else 0) + ((1 if passes == 0 else 3 * passes) if E > 0 else 0)
+    if scheduled:  # bounding box (2), Morton keys, 4 radix passes of 3; rank, degrees, scan (3); edge rows,
+        # positions, source ranks (3 with edges); then the reverse CSR over the ranks
+        rc_launches = 3 + 12 + 3 + ((3 + rc_launches - 1) if E > 0 else 0)  # (its own edge-rows launch is skipped)
     launches = K * (rc_launches + 2 + (1 if framed and E > 0 else 0))  # in the timed steps
 
     cpu = None
@@ -726,7 +765,8 @@ def main():
         "config": {"workload": f"{args.workload}: {DESCR[args.workload]}" + (f" (reduced to {N} nodes)" if args.nodes else ""),
                    "N": N, "E": E, "L": wl.L, "C": wl.C,
                    "P": plan.n_paths, "cg_nnz": nnz_total,
-                   "step": ("reverse CSR + " + ("edge frames + " if framed else "") +
+                   "step": (("locality schedule (Morton order of the positions, ordered CSRs) + " if scheduled
+                             else "reverse CSR + ") + ("edge frames + " if framed else "") +
                             "forward + VJP (grad_x, grad_w, grad_r), inputs resident in HBM"),
                    "l2": f"inputs larger than L2 (w = {wl.w.nbytes / 1e9:.2f} GB streamed per pass)",
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",

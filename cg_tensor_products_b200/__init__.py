@@ -68,6 +68,10 @@ def _load():
         "etp_build_reverse_csr": [i32, i32, vp, vp, vp, vp, vp, vp, sz, vp],
         "etp_build_reverse_csr_static": [i32, i32, vp, vp, vp, vp, vp, vp],
         "etp_validate_csr": [i32, i32, vp, vp, vp, vp],
+        "etp_locality_schedule_workspace_size": [i32, i32, ctypes.POINTER(sz)],
+        "etp_build_locality_schedule": [i32, i32, vp, vp, vp, ctypes.c_float, vp, vp, vp, vp, vp, vp, vp, sz, vp],
+        "etp_forward_ordered": [vp, i32, i32] + [vp] * 10,
+        "etp_backward_ordered": [vp, i32, i32] + [vp] * 13,
         "etp_device_fault": [vp],
         "etp_status_string": [i32],
     }
@@ -497,6 +501,101 @@ def build_reverse_csr_static(N: int, row_ptr, src, with_dst=True, stream=None):
     _launch(dev, "etp_build_reverse_csr_static", _load().etp_build_reverse_csr_static, N, E, _ptr(row_ptr),
             _ptr(src), _ptr(rev_ptr), _ptr(rev_perm), _ptr(dst), stream=stream)
     return rev_ptr, rev_perm, dst
+
+
+class Schedule:
+    """Locality schedule of a CSR graph (etp_build_locality_schedule): node order, the
+    forward CSR over that order (ord_ptr, ord_edge), the reverse CSR over that order
+    (rev_ptr, rev_perm) and the destination of every edge, all int32 on the device."""
+
+    def __init__(self, N, E, order, ord_ptr, ord_edge, rev_ptr, rev_perm, dst):
+        self.N, self.E = N, E
+        self.order, self.ord_ptr, self.ord_edge = order, ord_ptr, ord_edge
+        self.rev_ptr, self.rev_perm, self.dst = rev_ptr, rev_perm, dst
+
+    def tensors(self):
+        return self.order, self.ord_ptr, self.ord_edge, self.rev_ptr, self.rev_perm, self.dst
+
+
+def locality_schedule_workspace_size(N: int, E: int) -> int:
+    b = ctypes.c_size_t()
+    _check(_load().etp_locality_schedule_workspace_size(int(N), int(E), ctypes.byref(b)), "workspace_size")
+    return b.value
+
+
+def locality_schedule(N: int, row_ptr, src, pos, cell: float, out: Schedule = None, workspace=None, stream=None):
+    """Schedule whose rows follow the Morton order of the nodes' cells (side `cell`) of pos [N, 3]
+    (etp_build_locality_schedule). out: a Schedule of the same sizes to overwrite."""
+    import torch
+
+    E = src.numel()
+    _check_graph(row_ptr, src, N, E)
+    _expect(pos, "pos", "float32", (N, 3))
+    dev = row_ptr.device
+    if out is None:
+        i32 = dict(dtype=torch.int32, device=dev)
+        out = Schedule(N, E, torch.empty(N, **i32), torch.empty(N + 1, **i32), torch.empty(E, **i32),
+                       torch.empty(N + 1, **i32), torch.empty(E, **i32), torch.empty(E, **i32))
+    if (out.N, out.E) != (N, E):
+        raise ValueError(f"schedule for (N, E) = {(out.N, out.E)}, graph has {(N, E)}")
+    nbytes = locality_schedule_workspace_size(N, E)
+    if workspace is None:
+        workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=dev)
+    _expect(workspace, "workspace", "uint8", (None,))
+    dev = _need_cuda(row_ptr, src, pos, workspace, *out.tensors())
+    _launch(dev, "etp_build_locality_schedule", _load().etp_build_locality_schedule, N, E, _ptr(row_ptr), _ptr(src),
+            _ptr(pos), float(cell), *[_ptr(t) for t in out.tensors()], _ptr(workspace), workspace.numel(),
+            stream=stream)
+    return out
+
+
+def forward_ordered(plan: Plan, sched: Schedule, src, r, x, w, out=None, frames=None, stream=None):
+    """forward() on a locality schedule (etp_forward_ordered): the same out, rows visited in schedule order."""
+    import torch
+
+    N, E = sched.N, sched.E
+    _expect(src, "src", "int32", (E,))
+    _expect(r, "r", "float32", (E, 3))
+    _expect(frames, "frames", "float32", (E, FRAME_FLOATS))
+    _expect(x, "x", "float32", (N, plan.dim_in, plan.C))
+    _expect(w, "w", "float32", (E, plan.n_paths, plan.C))
+    if out is None:
+        out = torch.empty((N, plan.dim_out, plan.C), device=x.device, dtype=torch.float32)
+    _expect(out, "out", "float32", (N, plan.dim_out, plan.C))
+    dev = _need_cuda(sched.order, sched.ord_ptr, sched.ord_edge, src, r, frames, x, w, out)
+    _launch(dev, "etp_forward_ordered", _load().etp_forward_ordered, plan.handle, N, E, _ptr(sched.order),
+            _ptr(sched.ord_ptr), _ptr(sched.ord_edge), _ptr(src), _ptr(r), _ptr(frames), _ptr(x), _ptr(w),
+            _ptr(out), stream=stream)
+    return out
+
+
+def backward_ordered(plan: Plan, sched: Schedule, r, x, w, grad_out, want=("x", "w", "r"), grad_x=None,
+                     grad_w=None, grad_r=None, frames=None, stream=None):
+    """backward() on a locality schedule (etp_backward_ordered): the same (grad_x, grad_w, grad_r)."""
+    import torch
+
+    N, E = sched.N, sched.E
+    _expect(r, "r", "float32", (E, 3))
+    _expect(frames, "frames", "float32", (E, FRAME_FLOATS))
+    _expect(x, "x", "float32", (N, plan.dim_in, plan.C))
+    _expect(w, "w", "float32", (E, plan.n_paths, plan.C))
+    _expect(grad_out, "grad_out", "float32", (N, plan.dim_out, plan.C))
+    dev = x.device
+    if "x" in want and grad_x is None:
+        grad_x = torch.empty((N, plan.dim_in, plan.C), device=dev, dtype=torch.float32)
+    if "w" in want and grad_w is None:
+        grad_w = torch.empty((E, plan.n_paths, plan.C), device=dev, dtype=torch.float32)
+    if "r" in want and grad_r is None:
+        grad_r = torch.empty((E, 3), device=dev, dtype=torch.float32)
+    _expect(grad_x, "grad_x", "float32", (N, plan.dim_in, plan.C))
+    _expect(grad_w, "grad_w", "float32", (E, plan.n_paths, plan.C))
+    _expect(grad_r, "grad_r", "float32", (E, 3))
+    dev = _need_cuda(sched.order, sched.rev_ptr, sched.rev_perm, sched.dst, r, frames, x, w, grad_out, grad_x,
+                     grad_w, grad_r)
+    _launch(dev, "etp_backward_ordered", _load().etp_backward_ordered, plan.handle, N, E, _ptr(sched.order),
+            _ptr(sched.rev_ptr), _ptr(sched.rev_perm), _ptr(sched.dst), _ptr(r), _ptr(frames), _ptr(x), _ptr(w),
+            _ptr(grad_out), _ptr(grad_x), _ptr(grad_w), _ptr(grad_r), stream=stream)
+    return grad_x, grad_w, grad_r
 
 
 def device_fault() -> int:

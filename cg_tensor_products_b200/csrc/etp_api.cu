@@ -3,6 +3,7 @@
 #include <cuda_runtime.h>
 
 #include <cctype>
+#include <cmath>
 #include <cstdint>
 #include <cstring>
 #include <new>
@@ -213,18 +214,27 @@ etp_status etp_plan_frames_advised(etp_plan_t plan, int E, int* use_records) {
     return ETP_OK;
 }
 
-etp_status etp_forward(etp_plan_t plan, int N, int E, const int32_t* row_ptr, const int32_t* src, const float* r,
-                       const float* frames, const float* x, const float* w, float* out, etp_stream_t stream) {
+namespace {
+
+// Waves of tasks of a locality schedule: the tasks in flight hold about
+// 1/waves of the rows, in the schedule's order.
+constexpr int kOrderedWaves = 8;
+
+etp_status forward_impl(etp_plan_t plan, int N, int E, const int32_t* row_ptr, const int32_t* src, const float* r,
+                        const float* frames, const float* x, const float* w, float* out, const int32_t* order,
+                        const int32_t* pos_edge, etp_stream_t stream) {
     if (!plan || N < 0 || E < 0) return ETP_ERR_INVALID_ARG;
     if (N == 0) return E == 0 ? ETP_OK : ETP_ERR_INVALID_ARG;
     if (!row_ptr || !x || !out || !aligned4(row_ptr) || !aligned16(x) || !aligned16(out)) return ETP_ERR_INVALID_ARG;
     if (E > 0 && (!src || !w || !aligned4(src) || !aligned16(w))) return ETP_ERR_INVALID_ARG;
     if (E > 0 && (frames ? !aligned16(frames) : (!r || !aligned4(r)))) return ETP_ERR_INVALID_ARG;
+    if ((order && !aligned4(order)) || (pos_edge && !aligned4(pos_edge))) return ETP_ERR_INVALID_ARG;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     // rows cut by a task boundary are reduced onto zeros; empty rows stay zero
     cudaError_t err = cudaMemsetAsync(out, 0, sizeof(float) * (size_t)N * plan->D * plan->C, s);
     if (err != cudaSuccess || E == 0) return cuda_status(err);
-    const etp::LaunchShape sh = etp::launch_shape(plan->C, plan->L, plan->o3, false, frames != nullptr, E, N);
+    const etp::LaunchShape sh = etp::launch_shape(plan->C, plan->L, plan->o3, false, frames != nullptr, E, N,
+                                                  order ? kOrderedWaves : 1);
     etp::FwdArgs a{N,
                    E,
                    row_ptr,
@@ -237,7 +247,9 @@ etp_status etp_forward(etp_plan_t plan, int N, int E, const int32_t* row_ptr, co
                    plan->C / 4,
                    sh.team,
                    sh.slices,
-                   sh.ntasks};
+                   sh.ntasks,
+                   order,
+                   pos_edge};
     switch (plan->L) {
         case 0: err = etp::launch_forward<0>(plan->o3, a, sh.grid, sh.smem_bytes, s); break;
         case 1: err = etp::launch_forward<1>(plan->o3, a, sh.grid, sh.smem_bytes, s); break;
@@ -247,19 +259,20 @@ etp_status etp_forward(etp_plan_t plan, int N, int E, const int32_t* row_ptr, co
     return cuda_status(err);
 }
 
-etp_status etp_backward(etp_plan_t plan, int N, int E, const int32_t* row_ptr, const int32_t* src,
-                        const int32_t* rev_ptr, const int32_t* rev_perm, const int32_t* dst_of_edge, const float* r,
-                        const float* frames, const float* x, const float* w, const float* grad_out, float* grad_x,
-                        float* grad_w, float* grad_r, etp_stream_t stream) {
+etp_status backward_impl(etp_plan_t plan, int N, int E, const int32_t* row_ptr, const int32_t* src,
+                         const int32_t* rev_ptr, const int32_t* rev_perm, const int32_t* dst_of_edge, const float* r,
+                         const float* frames, const float* x, const float* w, const float* grad_out, float* grad_x,
+                         float* grad_w, float* grad_r, const int32_t* order, etp_stream_t stream) {
     if (!plan || N < 0 || E < 0) return ETP_ERR_INVALID_ARG;
     if (N == 0) return E == 0 ? ETP_OK : ETP_ERR_INVALID_ARG;
-    if (!row_ptr || !rev_ptr || !x || !grad_out || !aligned4(row_ptr) || !aligned4(rev_ptr) || !aligned16(x) ||
-        !aligned16(grad_out))
+    if (!rev_ptr || !x || !grad_out || !aligned4(rev_ptr) || !aligned16(x) || !aligned16(grad_out))
         return ETP_ERR_INVALID_ARG;
+    if (row_ptr ? !aligned4(row_ptr) : !dst_of_edge) return ETP_ERR_INVALID_ARG;  // one of them finds the rows
+    if (order && !aligned4(order)) return ETP_ERR_INVALID_ARG;
     if (grad_x && !aligned16(grad_x)) return ETP_ERR_INVALID_ARG;
     if (E > 0) {
-        if (!src || !rev_perm || !w || !aligned4(src) || !aligned4(rev_perm) || !aligned16(w))
-            return ETP_ERR_INVALID_ARG;
+        if (!rev_perm || !w || !aligned4(rev_perm) || !aligned16(w)) return ETP_ERR_INVALID_ARG;
+        if (src && !aligned4(src)) return ETP_ERR_INVALID_ARG;
         if (frames ? !aligned16(frames) : (!r || !aligned4(r))) return ETP_ERR_INVALID_ARG;
         if ((grad_w && !aligned16(grad_w)) || (grad_r && !aligned4(grad_r)) ||
             (dst_of_edge && !aligned4(dst_of_edge)))
@@ -274,7 +287,8 @@ etp_status etp_backward(etp_plan_t plan, int N, int E, const int32_t* row_ptr, c
     // source rows cut by a task boundary are reduced onto zeros; sources without edges stay zero
     if (grad_x) err = cudaMemsetAsync(grad_x, 0, sizeof(float) * (size_t)N * plan->D * plan->C, s);
     if (err != cudaSuccess || E == 0) return cuda_status(err);
-    const etp::LaunchShape sh = etp::launch_shape(plan->C, plan->L, plan->o3, true, frames != nullptr, E, N);
+    const etp::LaunchShape sh = etp::launch_shape(plan->C, plan->L, plan->o3, true, frames != nullptr, E, N,
+                                                  order ? kOrderedWaves : 1);
     etp::BwdArgs a{N,
                    E,
                    row_ptr,
@@ -293,7 +307,8 @@ etp_status etp_backward(etp_plan_t plan, int N, int E, const int32_t* row_ptr, c
                    plan->C / 4,
                    sh.team,
                    sh.slices,
-                   sh.ntasks};
+                   sh.ntasks,
+                   order};
     switch (plan->L) {
         case 0: err = etp::launch_backward<0>(plan->o3, a, sh.grid, sh.smem_bytes, s); break;
         case 1: err = etp::launch_backward<1>(plan->o3, a, sh.grid, sh.smem_bytes, s); break;
@@ -301,6 +316,38 @@ etp_status etp_backward(etp_plan_t plan, int N, int E, const int32_t* row_ptr, c
         default: err = etp::launch_backward<3>(plan->o3, a, sh.grid, sh.smem_bytes, s); break;
     }
     return cuda_status(err);
+}
+
+}  // namespace
+
+etp_status etp_forward(etp_plan_t plan, int N, int E, const int32_t* row_ptr, const int32_t* src, const float* r,
+                       const float* frames, const float* x, const float* w, float* out, etp_stream_t stream) {
+    return forward_impl(plan, N, E, row_ptr, src, r, frames, x, w, out, nullptr, nullptr, stream);
+}
+
+etp_status etp_forward_ordered(etp_plan_t plan, int N, int E, const int32_t* order, const int32_t* ord_ptr,
+                               const int32_t* ord_edge, const int32_t* src, const float* r, const float* frames,
+                               const float* x, const float* w, float* out, etp_stream_t stream) {
+    if (N > 0 && (!order || (E > 0 && !ord_edge))) return ETP_ERR_INVALID_ARG;
+    return forward_impl(plan, N, E, ord_ptr, src, r, frames, x, w, out, order, ord_edge, stream);
+}
+
+etp_status etp_backward(etp_plan_t plan, int N, int E, const int32_t* row_ptr, const int32_t* src,
+                        const int32_t* rev_ptr, const int32_t* rev_perm, const int32_t* dst_of_edge, const float* r,
+                        const float* frames, const float* x, const float* w, const float* grad_out, float* grad_x,
+                        float* grad_w, float* grad_r, etp_stream_t stream) {
+    if (!row_ptr || (E > 0 && !src)) return ETP_ERR_INVALID_ARG;
+    return backward_impl(plan, N, E, row_ptr, src, rev_ptr, rev_perm, dst_of_edge, r, frames, x, w, grad_out, grad_x,
+                         grad_w, grad_r, nullptr, stream);
+}
+
+etp_status etp_backward_ordered(etp_plan_t plan, int N, int E, const int32_t* order, const int32_t* rev_ptr,
+                                const int32_t* rev_perm, const int32_t* dst_of_edge, const float* r,
+                                const float* frames, const float* x, const float* w, const float* grad_out,
+                                float* grad_x, float* grad_w, float* grad_r, etp_stream_t stream) {
+    if (N > 0 && (!order || (E > 0 && !dst_of_edge))) return ETP_ERR_INVALID_ARG;
+    return backward_impl(plan, N, E, nullptr, nullptr, rev_ptr, rev_perm, dst_of_edge, r, frames, x, w, grad_out,
+                         grad_x, grad_w, grad_r, order, stream);
 }
 
 etp_status etp_double_backward(etp_plan_t plan, int N, int E, const int32_t* row_ptr, const int32_t* src,
@@ -462,6 +509,36 @@ etp_status etp_build_reverse_csr(int N, int E, const int32_t* row_ptr, const int
     if (workspace_bytes < etp::reverse_csr_workspace_bytes(N, E)) return ETP_ERR_WORKSPACE;
     return cuda_status(etp::build_reverse_csr(N, E, row_ptr, src, rev_ptr, rev_perm, dst_of_edge, workspace,
                                               reinterpret_cast<cudaStream_t>(stream)));
+}
+
+etp_status etp_locality_schedule_workspace_size(int N, int E, size_t* bytes) {
+    if (N < 0 || E < 0 || !bytes) return ETP_ERR_INVALID_ARG;
+    const size_t a = etp::spatial_order_workspace_bytes(N), b = etp::ordered_csr_workspace_bytes(N, E);
+    *bytes = a > b ? a : b;
+    return ETP_OK;
+}
+
+etp_status etp_build_locality_schedule(int N, int E, const int32_t* row_ptr, const int32_t* src, const float* pos,
+                                       float cell, int32_t* order, int32_t* ord_ptr, int32_t* ord_edge,
+                                       int32_t* rev_ptr, int32_t* rev_perm, int32_t* dst_of_edge, void* workspace,
+                                       size_t workspace_bytes, etp_stream_t stream) {
+    if (N < 0 || E < 0 || !(cell > 0.f) || !std::isfinite(cell)) return ETP_ERR_INVALID_ARG;
+    if (N == 0) return E == 0 ? ETP_OK : ETP_ERR_INVALID_ARG;
+    if (!row_ptr || !pos || !order || !ord_ptr || !rev_ptr || !workspace) return ETP_ERR_INVALID_ARG;
+    if (!aligned4(row_ptr) || !aligned4(pos) || !aligned4(order) || !aligned4(ord_ptr) || !aligned4(rev_ptr) ||
+        !aligned16(workspace))
+        return ETP_ERR_INVALID_ARG;
+    if (E > 0 && (!src || !ord_edge || !rev_perm || !dst_of_edge || !aligned4(src) || !aligned4(ord_edge) ||
+                  !aligned4(rev_perm) || !aligned4(dst_of_edge)))
+        return ETP_ERR_INVALID_ARG;
+    size_t need = 0;
+    etp_locality_schedule_workspace_size(N, E, &need);
+    if (workspace_bytes < need) return ETP_ERR_WORKSPACE;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t err = etp::spatial_order(N, pos, cell, order, workspace, s);
+    if (err != cudaSuccess) return cuda_status(err);
+    return cuda_status(etp::build_ordered_csr(N, E, row_ptr, src, order, ord_ptr, ord_edge, rev_ptr, rev_perm,
+                                              dst_of_edge, workspace, s));
 }
 
 etp_status etp_validate_csr(int N, int E, const int32_t* row_ptr, const int32_t* src, int32_t* d_flag,

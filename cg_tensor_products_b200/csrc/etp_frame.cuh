@@ -724,7 +724,14 @@ __global__ void __launch_bounds__(frame::kThreads, 4) etp_fwd_frame_kernel(FwdAr
     };
     const unsigned wbytes = 4u * P * C, xbytes = 4u * D * C, fbytes = FR ? 4u * kFrameFloats : 0u;
     const uint64_t pol_w = l2_evict_first_policy();
+    // position q -> edge, and row rank -> node: the identity, or a locality order
+    // (rows taken in the order's sequence, each row's edges contiguous)
+    // (an out-of-range edge of the map counts as an edge with an invalid source)
+    auto edge_at = [&](int q) -> int { return a.pos_edge ? __ldg(a.pos_edge + q) : q; };
+    auto node_of = [&](int rank) -> int { return a.order ? __ldg(a.order + rank) : rank; };
+    auto src_of = [&](int e) -> int { return (unsigned)e < (unsigned)a.E ? __ldg(a.src + e) : -1; };
     auto issue = [&](int e, int j, int slot) {
+        e = (unsigned)e < (unsigned)a.E ? e : 0;
         j = (unsigned)j < (unsigned)a.N ? j : 0;
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         mbar_expect_tx(&bar[slot], wbytes + xbytes + fbytes);
@@ -740,35 +747,43 @@ __global__ void __launch_bounds__(frame::kThreads, 4) etp_fwd_frame_kernel(FwdAr
         mbar_fence_init();
     }
     group_sync();
-    // source indices one and two edges ahead and the next edge vector are loaded
-    // an edge early, so their latency hides behind an edge of compute
-    int j_cur = __ldg(a.src + k0);
-    int j_next = k0 + 1 < k1 ? __ldg(a.src + k0 + 1) : 0;
-    float3 r_cur = FR ? make_float3(0.f, 0.f, 1.f) : load_r(a.r, k0);
-    if (producer) issue(k0, j_cur, 0);
+    // edges one to three positions ahead, source indices one and two ahead and the
+    // next edge vector are loaded an edge early, so their latency (and that of the
+    // position -> edge map before them) hides behind an edge of compute
+    const int e0 = edge_at(k0);
+    int e_next = k0 + 1 < k1 ? edge_at(k0 + 1) : 0;
+    int e_next2 = k0 + 2 < k1 ? edge_at(k0 + 2) : 0;
+    int j_cur = src_of(e0);
+    int j_next = k0 + 1 < k1 ? src_of(e_next) : 0;
+    float3 r_cur = FR ? make_float3(0.f, 0.f, 1.f) : load_r(a.r, (unsigned)e0 < (unsigned)a.E ? e0 : 0);
+    if (producer) issue(e0, j_cur, 0);
     bool live = true;
 
     int row = segment_of(a.row_ptr, a.N, k0);
     int row_lo = __ldg(a.row_ptr + row), row_hi = __ldg(a.row_ptr + row + 1);
+    int node = node_of(row);  // loaded a row early: used when the row is stored
     float2 acc[D];
 #pragma unroll
     for (int k = 0; k < D; ++k) acc[k] = f2_zero();
 
-    for (int e = k0, it = 0; e < k1; ++e, ++it) {
-        while (e >= row_hi && row < a.N - 1) {  // the edge opens a later row: store the finished one
+    for (int q = k0, it = 0; q < k1; ++q, ++it) {
+        while (q >= row_hi && row < a.N - 1) {  // the edge opens a later row: store the finished one
             if (row_hi > max(row_lo, k0)) {
-                flush_row<D>(out2 + (size_t)row * D * C2 + cp, C2, acc, row_lo >= k0);
+                flush_row<D>(out2 + (size_t)node * D * C2 + cp, C2, acc, row_lo >= k0);
 #pragma unroll
                 for (int k = 0; k < D; ++k) acc[k] = f2_zero();
             }
             ++row;
             row_lo = row_hi;
             row_hi = __ldg(a.row_ptr + row + 1);
+            node = node_of(row);
         }
         const int slot = it & 1;
-        if (producer && e + 1 < k1) issue(e + 1, j_next, slot ^ 1);
-        const int j_after = e + 2 < k1 ? __ldg(a.src + e + 2) : 0;
-        const float3 r_next = (!FR && e + 1 < k1) ? load_r(a.r, e + 1) : r_cur;
+        if (producer && q + 1 < k1) issue(e_next, j_next, slot ^ 1);
+        const int e_next3 = q + 3 < k1 ? edge_at(q + 3) : 0;
+        const int j_after = q + 2 < k1 ? src_of(e_next2) : 0;
+        const float3 r_next =
+            (!FR && q + 1 < k1) ? load_r(a.r, (unsigned)e_next < (unsigned)a.E ? e_next : 0) : r_cur;
         const bool valid = (unsigned)j_cur < (unsigned)a.N;  // an invalid source contributes nothing
         Frame f;
         if constexpr (FR) {
@@ -818,9 +833,11 @@ __global__ void __launch_bounds__(frame::kThreads, 4) etp_fwd_frame_kernel(FwdAr
         group_sync();  // this slot's buffers are free for the edge after next
         j_cur = j_next;
         j_next = j_after;
+        e_next = e_next2;
+        e_next2 = e_next3;
         r_cur = r_next;
     }
-    flush_row<D>(out2 + (size_t)row * D * C2 + cp, C2, acc, row_lo >= k0 && row_hi <= k1);
+    flush_row<D>(out2 + (size_t)node * D * C2 + cp, C2, acc, row_lo >= k0 && row_hi <= k1);
 }
 
 // ===========================================================================
@@ -871,6 +888,7 @@ __global__ void __launch_bounds__(frame::kThreads, L <= 2 ? 6 : 4) etp_bwd_frame
     // position q of the reverse order -> edge; out-of-range edges and rows map to
     // valid addresses and are marked invalid (they contribute and store nothing)
     auto edge_at = [&](int q) -> int { return __ldg(a.rev_perm + q); };
+    auto node_of = [&](int rank) -> int { return a.order ? __ldg(a.order + rank) : rank; };  // source row -> node
     auto valid_edge = [&](int e) { return (unsigned)e < (unsigned)a.E; };
     auto dst_of = [&](int e) -> int {
         if (!valid_edge(e)) return -1;
@@ -888,8 +906,8 @@ __global__ void __launch_bounds__(frame::kThreads, L <= 2 ? 6 : 4) etp_bwd_frame
     };
     const float2* x2 = reinterpret_cast<const float2*>(a.x);
     const float2* g2 = reinterpret_cast<const float2*>(a.g);
-    auto copy_x = [&](int j) {
-        const float2* xs = x2 + (size_t)j * D * C2 + cp;
+    auto copy_x = [&](int node) {
+        const float2* xs = x2 + (size_t)node * D * C2 + cp;
 #pragma unroll
         for (int k = 0; k < D; ++k) cp_async8(xrow + k * G.T + G.tl, xs + k * C2);
         cp_async_commit();
@@ -901,8 +919,10 @@ __global__ void __launch_bounds__(frame::kThreads, L <= 2 ? 6 : 4) etp_bwd_frame
         cp_async_commit();
     };
 
-    int row = segment_of(a.rev_ptr, a.N, k0);  // source node of position k0
+    int row = segment_of(a.rev_ptr, a.N, k0);  // source row of position k0
     int row_lo = __ldg(a.rev_ptr + row), row_hi = __ldg(a.rev_ptr + row + 1);
+    // the nodes of this source row and the next, loaded a row early
+    int node = node_of(row), node_nx = row + 1 < a.N ? node_of(row + 1) : 0;
     // positions from rev_ptr[N] on hold the edges whose source is out of range (an
     // invalid CSR): they contribute nothing and get zero grad_w and grad_r
     const int pos_end = __ldg(a.rev_ptr + a.N);
@@ -919,7 +939,7 @@ __global__ void __launch_bounds__(frame::kThreads, L <= 2 ? 6 : 4) etp_bwd_frame
     }
     group_sync();
     if (producer) issue_w(e_cur, 0);
-    copy_x(row);
+    copy_x(node);
     copy_g(i_cur);
     bool live = true;
 
@@ -930,13 +950,15 @@ __global__ void __launch_bounds__(frame::kThreads, L <= 2 ? 6 : 4) etp_bwd_frame
     for (int q = k0, it = 0; q < k1; ++q, ++it) {
         while (q >= row_hi && row < a.N - 1) {  // the position opens a later source row: store the finished one
             if (row_hi > max(row_lo, k0)) {
-                if (gx2) flush_row<D>(gx2 + (size_t)row * D * C2 + cp, C2, gx, row_lo >= k0);
+                if (gx2) flush_row<D>(gx2 + (size_t)node * D * C2 + cp, C2, gx, row_lo >= k0);
 #pragma unroll
                 for (int k = 0; k < D; ++k) gx[k] = f2_zero();
             }
             ++row;
             row_lo = row_hi;
             row_hi = __ldg(a.rev_ptr + row + 1);
+            node = node_nx;
+            node_nx = row + 1 < a.N ? node_of(row + 1) : 0;
         }
         // the next position's source row, edge and destination (for the prefetches)
         const bool has_next = q + 1 < k1;
@@ -977,7 +999,8 @@ __global__ void __launch_bounds__(frame::kThreads, L <= 2 ? 6 : 4) etp_bwd_frame
                 for (int k = 0; k < D; ++k) u[k] = lds2(grow + k * G.T + G.tl);
                 rotate_all2<L>(f, dbuf, v, u, xp, gpa);
             }
-            if (has_next && row_next != row) copy_x(row_next);  // next source's x row, behind this edge's reads
+            // next source's x row, behind this edge's reads
+            if (has_next && row_next != row) copy_x(row_next == row + 1 ? node_nx : node_of(row_next));
             if (has_next) copy_g(i_next);
 #pragma unroll
             for (int k = 0; k < D; ++k) z[k] = f2_zero();
@@ -1069,7 +1092,7 @@ __global__ void __launch_bounds__(frame::kThreads, L <= 2 ? 6 : 4) etp_bwd_frame
             } else if (gwe) {
                 static_for<0, P>([&](auto pc) { st_stream2(gwe + decltype(pc)::value * C2, f2_zero(), pol_w); });
             }
-            if (has_next && row_next != row) copy_x(row_next);
+            if (has_next && row_next != row) copy_x(row_next == row + 1 ? node_nx : node_of(row_next));
             if (has_next) copy_g(i_next);
         }
         // sum dL/de over the lane's channels and the team's lanes; the second
@@ -1104,7 +1127,7 @@ __global__ void __launch_bounds__(frame::kThreads, L <= 2 ? 6 : 4) etp_bwd_frame
         r_cur = r_next;
     }
     cp_async_wait_all();
-    if (gx2) flush_row<D>(gx2 + (size_t)row * D * C2 + cp, C2, gx, row_lo >= k0 && row_hi <= k1);
+    if (gx2) flush_row<D>(gx2 + (size_t)node * D * C2 + cp, C2, gx, row_lo >= k0 && row_hi <= k1);
 }
 
 namespace frame {

@@ -1,5 +1,7 @@
 // Graph preprocessing on the device: the reverse CSR (edges grouped by source,
-// stable in edge id), the destination of every edge, and a CSR validator.
+// stable in edge id), the destination of every edge, a CSR validator, and the
+// locality schedule (a spatial order of the nodes and the forward and reverse
+// CSRs taken in that order).
 //
 // Up to kOnePassMaxNodes sources the grouping is one stable counting pass: the
 // count of every (source, tile of kTile edges) pair in a source-major table, one
@@ -360,6 +362,120 @@ __global__ void validate(const int32_t* __restrict__ row_ptr, const int32_t* __r
     if (bits) atomicOr(flag, bits);
 }
 
+// ---------------------------------------------------------------------------
+// Spatial order. The bounding box is reduced on order-preserving unsigned codes of
+// the coordinates (a float's bits with the sign flipped, or all bits flipped when
+// negative: unsigned order = float order), with atomicMin / atomicMax.
+__device__ __forceinline__ unsigned float_code(float f) {
+    const unsigned u = __float_as_uint(f);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float code_float(unsigned c) {
+    return __uint_as_float((c & 0x80000000u) ? (c & 0x7fffffffu) : ~c);
+}
+
+__global__ void bbox_init(unsigned* box) {
+    if (threadIdx.x < 3) box[threadIdx.x] = 0xffffffffu;  // min codes
+    else if (threadIdx.x < 6) box[threadIdx.x] = 0u;      // max codes
+}
+
+// NaN coordinates are skipped (their nodes land in cell 0 on that axis).
+__global__ void __launch_bounds__(256) bbox_reduce(const float* __restrict__ pos, int N, unsigned* __restrict__ box) {
+    unsigned lo[3] = {0xffffffffu, 0xffffffffu, 0xffffffffu}, hi[3] = {0u, 0u, 0u};
+    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < N; i += gridDim.x * blockDim.x) {
+#pragma unroll
+        for (int a = 0; a < 3; ++a) {
+            const float v = pos[3 * (size_t)i + a];
+            if (v == v) {
+                const unsigned c = float_code(v);
+                lo[a] = min(lo[a], c);
+                hi[a] = max(hi[a], c);
+            }
+        }
+    }
+#pragma unroll
+    for (int a = 0; a < 3; ++a) {
+#pragma unroll
+        for (int o = 16; o; o >>= 1) {
+            lo[a] = min(lo[a], __shfl_xor_sync(0xffffffffu, lo[a], o));
+            hi[a] = max(hi[a], __shfl_xor_sync(0xffffffffu, hi[a], o));
+        }
+    }
+    if ((threadIdx.x & 31) == 0) {
+#pragma unroll
+        for (int a = 0; a < 3; ++a) {
+            atomicMin(box + a, lo[a]);
+            atomicMax(box + 3 + a, hi[a]);
+        }
+    }
+}
+
+// 10 bits spread to every third bit (bit k -> bit 3k).
+__device__ __forceinline__ unsigned spread3(unsigned v) {
+    v &= 0x3ffu;
+    v = (v | (v << 16)) & 0x030000ffu;
+    v = (v | (v << 8)) & 0x0300f00fu;
+    v = (v | (v << 4)) & 0x030c30c3u;
+    v = (v | (v << 2)) & 0x09249249u;
+    return v;
+}
+
+// Morton code of the node's cell: cells of side max(cell, largest extent / 1024)
+// from the box's low corner, 10 bits per axis (x in the lowest bit of each triple).
+__global__ void morton_keys(const float* __restrict__ pos, int N, const unsigned* __restrict__ box, float cell,
+                            int32_t* __restrict__ keys) {
+    const float lx = code_float(box[0]), ly = code_float(box[1]), lz = code_float(box[2]);
+    const float ext = fmaxf(fmaxf(code_float(box[3]) - lx, code_float(box[4]) - ly), code_float(box[5]) - lz);
+    const float side = fmaxf(cell, ext * (1.0f / 1023.0f));
+    const float inv = side > 0.f ? 1.0f / side : 0.f;
+    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < N; i += gridDim.x * blockDim.x) {
+        const float lo3[3] = {lx, ly, lz};
+        unsigned c[3];
+#pragma unroll
+        for (int a = 0; a < 3; ++a) {
+            const float t = (pos[3 * (size_t)i + a] - lo3[a]) * inv;  // NaN fails both tests below: cell 0
+            c[a] = t >= 1023.f ? 1023u : (t > 0.f ? (unsigned)t : 0u);
+        }
+        keys[i] = (int32_t)(spread3(c[0]) | (spread3(c[1]) << 1) | (spread3(c[2]) << 2));
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Locality schedule from an order of the nodes.
+__global__ void invert_order(const int32_t* __restrict__ order, int N, int32_t* __restrict__ rank) {
+    for (int j = blockIdx.x * blockDim.x + threadIdx.x; j < N; j += gridDim.x * blockDim.x) rank[order[j]] = j;
+}
+
+// deg[j] = in-degree of the node of rank j
+__global__ void ordered_degrees(const int32_t* __restrict__ row_ptr, const int32_t* __restrict__ order, int N,
+                                int32_t* __restrict__ deg) {
+    for (int j = blockIdx.x * blockDim.x + threadIdx.x; j < N; j += gridDim.x * blockDim.x) {
+        const int i = order[j];
+        deg[j] = row_ptr[i + 1] - row_ptr[i];
+    }
+}
+
+// The position of edge e in the ordered forward CSR: its row's start there plus
+// its offset inside the row (rows keep their edges in CSR order).
+__global__ void ordered_positions(const int32_t* __restrict__ row_ptr, const int32_t* __restrict__ dst,
+                                  const int32_t* __restrict__ rank, const int32_t* __restrict__ ord_ptr, int E,
+                                  int32_t* __restrict__ ord_edge) {
+    for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < E; e += gridDim.x * blockDim.x) {
+        const int i = dst[e];
+        ord_edge[ord_ptr[rank[i]] + (e - row_ptr[i])] = e;
+    }
+}
+
+// Source keys of the ordered reverse CSR: the source's rank; an out-of-range
+// source keeps its value, so it is grouped after every valid one as before.
+__global__ void source_ranks(const int32_t* __restrict__ src, const int32_t* __restrict__ rank, int N, int E,
+                             int32_t* __restrict__ keys) {
+    for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < E; e += gridDim.x * blockDim.x) {
+        const int j = src[e];
+        keys[e] = (unsigned)j < (unsigned)N ? rank[j] : j;
+    }
+}
+
 inline size_t align16(size_t b) { return (b + 15) & ~size_t(15); }
 inline int grid_for(long long n, int threads) {
     long long b = (n + threads - 1) / threads;
@@ -371,6 +487,29 @@ inline int radix_passes(int N) {
     int bits = 0;
     while (bits < 31 && (1ll << bits) < (long long)N) ++bits;  // keys are in [0, N)
     return (bits + 7) / 8;
+}
+
+// Stable LSD radix sort of the ids 0..n-1 by keys (8 bits per pass, `passes`
+// passes from the lowest digit); the sorted ids end in out. keys_a, keys_b,
+// vals_spare: n entries each; hist: 256 * tiles + 1.
+void radix_sort_ids(const int32_t* keys, int n, int passes, int32_t* keys_a, int32_t* keys_b, int32_t* vals_spare,
+                    int32_t* hist, int32_t* out, cudaStream_t s) {
+    const int n_tiles = (n + kTile - 1) / kTile;
+    // values ping-pong between vals_spare and out, ending in out
+    int32_t* vbuf[2] = {passes % 2 ? out : vals_spare, passes % 2 ? vals_spare : out};
+    int32_t* kbuf[2] = {keys_a, keys_b};
+    const int32_t* kin = keys;
+    const int32_t* vin = nullptr;
+    for (int pass = 0; pass < passes; ++pass) {
+        const int shift = 8 * pass;
+        tile_histogram<<<n_tiles, 256, 0, s>>>(kin, n, shift, hist);
+        scan_digit_columns<<<1, 256, 0, s>>>(hist, n_tiles);
+        int32_t* kout = kbuf[pass & 1];
+        int32_t* vout = vbuf[pass & 1];
+        tile_scatter<<<n_tiles, 128, 0, s>>>(kin, vin, n, shift, hist, kout, vout);
+        kin = kout;
+        vin = vout;
+    }
 }
 
 }  // namespace
@@ -423,23 +562,61 @@ cudaError_t build_reverse_csr(int N, int E, const int32_t* row_ptr, const int32_
         iota<<<grid_for(E, 256), 256, 0, s>>>(rev_perm, E);
         return cudaGetLastError();
     }
-    const int n_tiles = (E + kTile - 1) / kTile;
-    // values ping-pong between vals_spare and rev_perm, ending in rev_perm
-    int32_t* vbuf[2] = {passes % 2 ? rev_perm : vals_spare, passes % 2 ? vals_spare : rev_perm};
-    int32_t* kbuf[2] = {keys_a, keys_b};
-    const int32_t* kin = src;
-    const int32_t* vin = nullptr;
-    for (int pass = 0; pass < passes; ++pass) {
-        const int shift = 8 * pass;
-        tile_histogram<<<n_tiles, 256, 0, s>>>(kin, E, shift, hist);
-        scan_digit_columns<<<1, 256, 0, s>>>(hist, n_tiles);
-        int32_t* kout = kbuf[pass & 1];
-        int32_t* vout = vbuf[pass & 1];
-        tile_scatter<<<n_tiles, 128, 0, s>>>(kin, vin, E, shift, hist, kout, vout);
-        kin = kout;
-        vin = vout;
-    }
+    radix_sort_ids(src, E, passes, keys_a, keys_b, vals_spare, hist, rev_perm, s);
     return cudaGetLastError();
+}
+
+size_t spatial_order_workspace_bytes(int N) {
+    return align16(8 * sizeof(unsigned)) + 4 * align16(sizeof(int32_t) * (size_t)N) +
+           align16(sizeof(int32_t) * (256 * (size_t)radix_tiles(N) + 1));
+}
+
+cudaError_t spatial_order(int N, const float* pos, float cell, int32_t* order, void* ws, cudaStream_t s) {
+    char* p = static_cast<char*>(ws);
+    unsigned* box = reinterpret_cast<unsigned*>(p);
+    p += align16(8 * sizeof(unsigned));
+    int32_t* keys = reinterpret_cast<int32_t*>(p);
+    p += align16(sizeof(int32_t) * (size_t)N);
+    int32_t* keys_a = reinterpret_cast<int32_t*>(p);
+    p += align16(sizeof(int32_t) * (size_t)N);
+    int32_t* keys_b = reinterpret_cast<int32_t*>(p);
+    p += align16(sizeof(int32_t) * (size_t)N);
+    int32_t* spare = reinterpret_cast<int32_t*>(p);
+    p += align16(sizeof(int32_t) * (size_t)N);
+    int32_t* hist = reinterpret_cast<int32_t*>(p);
+    bbox_init<<<1, 32, 0, s>>>(box);
+    bbox_reduce<<<grid_for(N, 256), 256, 0, s>>>(pos, N, box);
+    morton_keys<<<grid_for(N, 256), 256, 0, s>>>(pos, N, box, cell, keys);
+    radix_sort_ids(keys, N, 4, keys_a, keys_b, spare, hist, order, s);  // 30-bit keys
+    return cudaGetLastError();
+}
+
+size_t ordered_csr_workspace_bytes(int N, int E) {
+    return align16(sizeof(int32_t) * (size_t)N) + align16(sizeof(int32_t) * (size_t)E) +
+           reverse_csr_workspace_bytes_for(N, E);
+}
+
+cudaError_t build_ordered_csr(int N, int E, const int32_t* row_ptr, const int32_t* src, const int32_t* order,
+                              int32_t* ord_ptr, int32_t* ord_edge, int32_t* rev_ptr, int32_t* rev_perm, int32_t* dst,
+                              void* ws, cudaStream_t s) {
+    char* p = static_cast<char*>(ws);
+    int32_t* rank = reinterpret_cast<int32_t*>(p);
+    p += align16(sizeof(int32_t) * (size_t)N);
+    int32_t* keys = reinterpret_cast<int32_t*>(p);
+    p += align16(sizeof(int32_t) * (size_t)E);
+    invert_order<<<grid_for(N, 256), 256, 0, s>>>(order, N, rank);
+    ordered_degrees<<<grid_for(N, 256), 256, 0, s>>>(row_ptr, order, N, ord_ptr);
+    scan_exclusive<<<1, kScanThreads, 0, s>>>(ord_ptr, ord_ptr, N);
+    cudaError_t err = cudaGetLastError();
+    if (err != cudaSuccess || E == 0) {
+        if (err == cudaSuccess) err = cudaMemsetAsync(rev_ptr, 0, sizeof(int32_t) * ((size_t)N + 1), s);
+        return err;
+    }
+    edge_rows<<<grid_for(E, 256), 256, 0, s>>>(row_ptr, N, E, dst);
+    ordered_positions<<<grid_for(E, 256), 256, 0, s>>>(row_ptr, dst, rank, ord_ptr, E, ord_edge);
+    source_ranks<<<grid_for(E, 256), 256, 0, s>>>(src, rank, N, E, keys);
+    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    return build_reverse_csr(N, E, row_ptr, keys, rev_ptr, rev_perm, nullptr, p, s);
 }
 
 cudaError_t validate_csr(int N, int E, const int32_t* row_ptr, const int32_t* src, int32_t* flag,

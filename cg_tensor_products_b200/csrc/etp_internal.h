@@ -12,7 +12,7 @@ constexpr int kThreadsPerBlock = 64;  // 2 warps; forward and backward kernels
 
 struct FwdArgs {
     int N, E;
-    const int32_t* row_ptr;
+    const int32_t* row_ptr;  // over row ranks when `order` is given
     const int32_t* src;
     const float* r;
     const float* frames;  // may be null: frames built in the kernel
@@ -22,7 +22,9 @@ struct FwdArgs {
     int C4;      // C / 4
     int team;    // lanes per team = min(32, C/2), a power of two
     int slices;  // teams per task = C / (2 team): 1, or 2 when C = 128
-    int ntasks;  // equal contiguous edge ranges
+    int ntasks;  // equal contiguous ranges of positions
+    const int32_t* order;     // may be null: row rank -> destination node (locality order)
+    const int32_t* pos_edge;  // may be null: position -> edge (the ranks' rows in sequence)
 };
 
 struct BwdArgs {
@@ -44,6 +46,7 @@ struct BwdArgs {
     int team;
     int slices;
     int ntasks;
+    const int32_t* order;  // may be null: source row rank -> node (rev_ptr is then over ranks)
 };
 
 // Launch geometry shared by the forward and backward kernels: teams of
@@ -54,7 +57,7 @@ struct LaunchShape {
     size_t smem_bytes;
     dim3 grid;
 };
-LaunchShape launch_shape(int C, int L, bool o3, bool backward, bool framed, int E, int N);
+LaunchShape launch_shape(int C, int L, bool o3, bool backward, bool framed, int E, int N, int waves = 1);
 
 template <int L>
 size_t smem_bytes(bool o3, int C, int T, bool backward, bool framed);
@@ -101,6 +104,15 @@ size_t reverse_csr_workspace_bytes(int N, int E);
 // radix_workspace_bytes_for).
 cudaError_t build_reverse_csr(int N, int E, const int32_t* row_ptr, const int32_t* src, int32_t* rev_ptr,
                               int32_t* rev_perm, int32_t* dst, void* ws, cudaStream_t s, bool one_pass = true);
+// Locality schedule: nodes sorted stably by the Morton code of their cell
+// (spatial_order), and the forward and reverse CSRs with rows in a given node
+// order (build_ordered_csr; dst = destination of every edge).
+size_t spatial_order_workspace_bytes(int N);
+cudaError_t spatial_order(int N, const float* pos, float cell, int32_t* order, void* ws, cudaStream_t s);
+size_t ordered_csr_workspace_bytes(int N, int E);
+cudaError_t build_ordered_csr(int N, int E, const int32_t* row_ptr, const int32_t* src, const int32_t* order,
+                              int32_t* ord_ptr, int32_t* ord_edge, int32_t* rev_ptr, int32_t* rev_perm, int32_t* dst,
+                              void* ws, cudaStream_t s);
 size_t radial_workspace_bytes(int E, int nb, int hidden, int PC);
 // Tensor-core path of the radial forward (hidden width 64, P*C a multiple of 16).
 bool radial_tc_supported(int nb, int hidden, int PC);

@@ -18,7 +18,7 @@ int log2i(int t) {
 
 }  // namespace
 
-LaunchShape launch_shape(int C, int L, bool o3, bool backward, bool framed, int E, int N) {
+LaunchShape launch_shape(int C, int L, bool o3, bool backward, bool framed, int E, int N, int waves) {
     LaunchShape s;
     s.team = C / 2 < 32 ? C / 2 : 32;
     s.slices = C / (2 * s.team);
@@ -47,10 +47,11 @@ LaunchShape launch_shape(int C, int L, bool o3, bool backward, bool framed, int 
         }
         occ.store(bps);
     }
-    // One wave of tasks, at least 16 edges each and no more tasks than rows: a
-    // row longer than a task is cut more than once, and its pieces are then
-    // summed in a run-dependent order (still correct, not bitwise repeatable).
-    long long cap = (long long)sms * bps * s.tasks_per_block;
+    // `waves` waves of tasks (one, unless a locality schedule asks for more), at
+    // least 16 edges each and no more tasks than rows: a row longer than a task
+    // is cut more than once, and its pieces are then summed in a run-dependent
+    // order (still correct, not bitwise repeatable).
+    long long cap = (long long)sms * bps * s.tasks_per_block * (waves < 1 ? 1 : waves);
     long long want = ((long long)E + 15) / 16;
     if (want > N) want = N;
     long long nt = want < cap ? want : cap;

@@ -313,6 +313,62 @@ ETP_API etp_status etp_build_reverse_csr(int N, int E, const int32_t* row_ptr, c
                                  int32_t* rev_ptr, int32_t* rev_perm, int32_t* dst_of_edge,
                                  void* workspace, size_t workspace_bytes, etp_stream_t stream);
 
+/* Locality schedule. With node features larger than L2 and node ids in no spatial
+ * order, the per-edge gathers of x[src] (forward) and grad_out[dst] (backward)
+ * miss L2 often. A locality schedule takes the rows in a spatial order of the
+ * nodes and splits the work into several waves of tasks, so that the tasks in
+ * flight at any time hold nearby rows and share their neighbours' rows in L2.
+ * Results are the same as etp_forward's and etp_backward's up to the rounding of
+ * rows cut by a task boundary. The pages measure on spatially coherent systems
+ * ("FlashCart 如何让等变原子间势更快更准?", section "FlashCart 用笛卡尔内核替代球谐耦合":
+ * the speed comes from memory access and the aggregation of edge contributions);
+ * the schedule is this library's way to keep those accesses local when the ids
+ * are not. */
+
+/* Bytes of device workspace etp_build_locality_schedule needs for (N, E). */
+ETP_API etp_status etp_locality_schedule_workspace_size(int N, int E, size_t* bytes);
+
+/* Build the locality schedule of a CSR graph from node positions:
+ *   order [N]: the node ids sorted stably by the Morton (Z-order) code of their
+ *     cell: cubic cells of side max(cell, largest bounding-box extent / 1023),
+ *     10 bits per axis (ties keep increasing id; NaN coordinates fall in cell 0);
+ *   ord_ptr [N+1], ord_edge [E]: the forward CSR with its rows taken in that
+ *     order: positions ord_ptr[k]..ord_ptr[k+1] hold the edges of row order[k],
+ *     in CSR order;
+ *   rev_ptr [N+1], rev_perm [E]: the reverse CSR with its sources taken in that
+ *     order (positions rev_ptr[k]..rev_ptr[k+1]: the edges whose source is
+ *     order[k], in increasing edge id; edges with an out-of-range source last);
+ *   dst_of_edge [E]: the CSR row of every edge.
+ * pos: device float32 [N][3]; cell > 0 and finite (the radial cutoff is a good
+ * choice). workspace: at least etp_locality_schedule_workspace_size bytes, 16-byte
+ * aligned, owned by the caller. Deterministic (counting and radix sorts). Needs a
+ * valid CSR (see etp_validate_csr). N = 0 launches nothing. */
+ETP_API etp_status etp_build_locality_schedule(int N, int E, const int32_t* row_ptr, const int32_t* src,
+                                               const float* pos, float cell, int32_t* order, int32_t* ord_ptr,
+                                               int32_t* ord_edge, int32_t* rev_ptr, int32_t* rev_perm,
+                                               int32_t* dst_of_edge, void* workspace, size_t workspace_bytes,
+                                               etp_stream_t stream);
+
+/* etp_forward on a locality schedule: the same result, out[i] = sum over the
+ * edges of row i, with the rows visited in the schedule's order. order, ord_ptr,
+ * ord_edge: as written by etp_build_locality_schedule for this graph (an entry of
+ * ord_edge out of [0, E) counts as an edge with an invalid source). src, r,
+ * frames, x, w, out: as in etp_forward (indexed by edge and node id, unchanged). */
+ETP_API etp_status etp_forward_ordered(etp_plan_t plan, int N, int E, const int32_t* order, const int32_t* ord_ptr,
+                                       const int32_t* ord_edge, const int32_t* src, const float* r,
+                                       const float* frames, const float* x, const float* w, float* out,
+                                       etp_stream_t stream);
+
+/* etp_backward on a locality schedule: the same outputs, with the sources visited
+ * in the schedule's order. order, rev_ptr, rev_perm, dst_of_edge: as written by
+ * etp_build_locality_schedule (dst_of_edge is required). The other arguments as
+ * in etp_backward. */
+ETP_API etp_status etp_backward_ordered(etp_plan_t plan, int N, int E, const int32_t* order,
+                                        const int32_t* rev_ptr, const int32_t* rev_perm,
+                                        const int32_t* dst_of_edge, const float* r, const float* frames,
+                                        const float* x, const float* w, const float* grad_out, float* grad_x,
+                                        float* grad_w, float* grad_r, etp_stream_t stream);
+
 /* Limits of etp_build_reverse_csr_static and the size of its scratch array. */
 #define ETP_STATIC_MAX_NODES (1 << 18)
 #define ETP_STATIC_MAX_EDGES (1 << 18)

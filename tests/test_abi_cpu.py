@@ -23,7 +23,7 @@ def lib():
 
 def test_exports_every_declared_symbol(lib):
     names = etp.declared_symbols()
-    assert len(names) == 23
+    assert len(names) == 27
     for n in names:
         assert hasattr(lib, n), n
 
@@ -142,6 +142,28 @@ def test_host_argument_checks(lib):
     assert S((1 << 18) + 1, 10, ok, ok, ok, ok, ok, None) == etp.ETP_ERR_TOO_LARGE
     assert S(10, 100, ok, ok, ctypes.c_void_p(0x10002), ok, ok, None) == etp.ETP_ERR_INVALID_ARG  # rev_ptr
     assert S(-1, 100, ok, ok, ok, ok, ok, None) == etp.ETP_ERR_INVALID_ARG
+    ls = ctypes.c_size_t()
+    assert lib.etp_locality_schedule_workspace_size(10, 100, ctypes.byref(ls)) == 0 and ls.value > 0
+    assert lib.etp_locality_schedule_workspace_size(10, -1, ctypes.byref(ls)) == etp.ETP_ERR_INVALID_ARG
+    LS = lib.etp_build_locality_schedule
+    full = [ok] * 6
+    assert LS(10, 100, ok, ok, ok, 4.5, *full, ok, ls.value - 1, None) == etp.ETP_ERR_WORKSPACE
+    assert LS(10, 100, ok, ok, ok, 0.0, *full, ok, ls.value, None) == etp.ETP_ERR_INVALID_ARG      # cell
+    assert LS(10, 100, ok, ok, ok, float("nan"), *full, ok, ls.value, None) == etp.ETP_ERR_INVALID_ARG
+    assert LS(10, 100, ok, ok, ok, float("inf"), *full, ok, ls.value, None) == etp.ETP_ERR_INVALID_ARG
+    assert LS(10, 100, ok, ok, None, 4.5, *full, ok, ls.value, None) == etp.ETP_ERR_INVALID_ARG    # pos
+    assert LS(10, 100, ok, ok, ok, 4.5, ok, ok, ok, ok, ok, None, ok, ls.value, None) == etp.ETP_ERR_INVALID_ARG
+    assert LS(10, 100, ok, ok, ok, 4.5, *full, ctypes.c_void_p(0x10004), ls.value, None) == etp.ETP_ERR_INVALID_ARG
+    assert LS(0, 0, None, None, None, 4.5, *([None] * 6), None, 0, None) == etp.ETP_OK            # nothing to do
+    FO, BO = lib.etp_forward_ordered, lib.etp_backward_ordered
+    assert FO(h, 4, 4, None, ok, ok, ok, ok, None, ok, ok, ok, None) == etp.ETP_ERR_INVALID_ARG    # order NULL
+    assert FO(h, 4, 4, ok, ok, None, ok, ok, None, ok, ok, ok, None) == etp.ETP_ERR_INVALID_ARG    # ord_edge NULL
+    assert FO(h, 4, 4, ok, None, ok, ok, ok, None, ok, ok, ok, None) == etp.ETP_ERR_INVALID_ARG    # ord_ptr NULL
+    assert FO(h, 4, 4, ok, ok, ok, ok, ok, None, ok, ok, bad, None) == etp.ETP_ERR_INVALID_ARG     # out
+    assert BO(h, 4, 4, ok, ok, ok, None, ok, None, ok, ok, ok, ok, ok, ok, None) == etp.ETP_ERR_INVALID_ARG  # dst
+    assert BO(h, 4, 4, None, ok, ok, ok, ok, None, ok, ok, ok, ok, ok, ok, None) == etp.ETP_ERR_INVALID_ARG  # order
+    assert BO(h, 4, 4, ok, ok, ok, ok, ok, None, ok, ok, bad, ok, ok, ok, None) == etp.ETP_ERR_INVALID_ARG   # grad_out
+    assert BO(h, 4, 4, ok, ok, ok, ok, ok, None, ok, ok, ok, None, None, None, None) == etp.ETP_OK          # nothing
     V = lib.etp_validate_csr
     assert V(10, 100, None, ok, ok, None) == etp.ETP_ERR_INVALID_ARG
     assert V(10, 100, ok, ok, None, None) == etp.ETP_ERR_INVALID_ARG

@@ -59,6 +59,9 @@ class Workload:
     W1: np.ndarray | None = None
     W2: np.ndarray | None = None
     r_cut: float | None = None
+    # atom positions in the periodic box, float32 [N, 3], and the radius-graph cutoff (water, large)
+    pos: np.ndarray | None = None
+    graph_cutoff: float | None = None
 
     @property
     def N(self) -> int:
@@ -178,7 +181,7 @@ def _geometry_water(rng, rc=5.0):
     dst, src = radius_pairs(pos, box, rc)
     row_ptr, src_sorted, order = csr_from_pairs(n, dst, src)
     r = min_image(pos[src_sorted] - pos[dst[order]], box)
-    return row_ptr, src_sorted, r, rc
+    return row_ptr, src_sorted, r, rc, pos
 
 
 def _geometry_large(rng, rc=4.5, n=32768):
@@ -190,7 +193,9 @@ def _geometry_large(rng, rc=4.5, n=32768):
     perm = rng.permutation(n)             # old id -> new id
     dst, src = perm[dst], perm[src]
     row_ptr, src_sorted, order = csr_from_pairs(n, dst, src)
-    return row_ptr, src_sorted, rvec[order]
+    pos_new = np.empty_like(pos)
+    pos_new[perm] = pos
+    return row_ptr, src_sorted, rvec[order], rc, pos_new
 
 
 def radial_mlp_weights(rng, r: np.ndarray, rc: float, P: int, C: int,
@@ -231,10 +236,10 @@ def make(name: str, seed: int = 0, n_nodes: int | None = None) -> Workload:
     elif name in ("micro_l2", "micro_l3"):
         row_ptr, src, r = _geometry_micro(rng, n_nodes or 1024)
     elif name == "water":
-        row_ptr, src, r64, rc = _geometry_water(rng)
+        row_ptr, src, r64, rc, pos = _geometry_water(rng)
         r = r64.astype(np.float32)
     elif name == "large":
-        row_ptr, src, r64 = _geometry_large(rng, n=n_nodes or 32768)
+        row_ptr, src, r64, rc, pos = _geometry_large(rng, n=n_nodes or 32768)
         r = r64.astype(np.float32)
     else:
         raise KeyError(name)
@@ -247,7 +252,8 @@ def make(name: str, seed: int = 0, n_nodes: int | None = None) -> Workload:
     else:
         w = _normal(rng, (E, P, C), 1.0 / np.sqrt(P))
     g = _normal(rng, (N, D, C))
-    return Workload(name, L, C, P, row_ptr, src.astype(np.int32), np.ascontiguousarray(r), x, w, g, **mlp)
+    geo = dict(pos=pos.astype(np.float32), graph_cutoff=rc) if name in ("water", "large") else {}
+    return Workload(name, L, C, P, row_ptr, src.astype(np.int32), np.ascontiguousarray(r), x, w, g, **mlp, **geo)
 
 
 def random_graph(rng, n: int, e: int, L: int, C: int, P: int, empty_rows=True) -> Workload:
