@@ -351,6 +351,7 @@ def extra_timings(etp, lib, plan, wl, d, rev_ptr, rev_perm, dst, gw, stream, dev
     import torch
 
     P = etp._ptr
+    tws = torch.empty(max(etp.tp_workspace_size(plan, wl.N, wl.E, False, dev), 16), dtype=torch.uint8, device=dev)
     sp = stream_ptr(stream)
     N, E, C, Pn = wl.N, wl.E, wl.C, plan.n_paths
     D = (wl.L + 1) ** 2
@@ -375,8 +376,8 @@ def extra_timings(etp, lib, plan, wl, d, rev_ptr, rev_perm, dst, gw, stream, dev
         plan.handle, E, 8, 64, rc, P(d["r"]), P(W1d), P(W2d), P(w_rad), P(rws), rws.numel(), sp), "radial"), stream)
     out2 = torch.empty_like(fout)
     t_tp = _time_ms(lambda: etp._check(lib.etp_forward(
-        plan.handle, N, E, P(d["row_ptr"]), P(d["src"]), P(d["r"]), None, P(d["x"]), P(w_rad), P(out2), sp),
-        "forward"), stream)
+        plan.handle, N, E, P(d["row_ptr"]), P(d["src"]), P(d["r"]), None, P(d["x"]), P(w_rad), P(out2), P(tws),
+        tws.numel(), sp), "forward"), stream)
     tflop = 3 * 2.0 * E * 64 * Pn * C
     del w_rad, rws
     out["fused_radial_forward"] = {
@@ -395,12 +396,12 @@ def extra_timings(etp, lib, plan, wl, d, rev_ptr, rev_perm, dst, gw, stream, dev
     o = {k: torch.empty_like(v) for k, v in (("g", d["g"]), ("x", d["x"]), ("r", d["r"]))}
     t_dd = _time_ms(lambda: etp._check(lib.etp_double_backward(
         plan.handle, N, E, P(d["row_ptr"]), P(d["src"]), P(rev_ptr), P(rev_perm), P(dst), P(d["r"]), P(d["x"]),
-        P(d["w"]), P(d["g"]), P(ggx), P(ggw), P(ggr), P(o["g"]), P(o["x"]), P(gw), P(o["r"]), sp), "double"),
-        stream)
+        P(d["w"]), P(d["g"]), P(ggx), P(ggw), P(ggr), P(o["g"]), P(o["x"]), P(gw), P(o["r"]), P(tws), tws.numel(),
+        sp), "double"), stream)
     dd_bytes = E * (3 * 4 * Pn * C + 12 * 3 + 4 * 3) + 5 * node + 4 * 2 * (N + 1)
     # the call allocates nothing: its device memory is its arguments (inputs, cotangents, outputs, graph)
     mem = sum(t.numel() * t.element_size() for t in (d["x"], d["w"], d["g"], d["r"], ggx, ggw, ggr, o["g"], o["x"],
-                                                     gw, o["r"], d["row_ptr"], d["src"], rev_ptr, rev_perm, dst))
+                                                     gw, o["r"], d["row_ptr"], d["src"], rev_ptr, rev_perm, dst, tws))
     out["double_backward"] = {
         "ms": t_dd, "bytes_per_launch": dd_bytes, "GBps": dd_bytes / (t_dd * 1e6),
         "roofline": {"bound": "hbm", "achieved": dd_bytes / (t_dd * 1e6), "peak": hbm, "unit": "GB/s",
@@ -408,25 +409,25 @@ def extra_timings(etp, lib, plan, wl, d, rev_ptr, rev_perm, dst, gw, stream, dev
         "bytes_note": "w and gg_w read, grad_w written (3 x 4PC per edge), r, gg_r, grad_r and three index "
                       "arrays per edge, x, gg_x, g read and grad_g, grad_x written once per node",
         "device_memory_GB": mem / 1e9,
-        "device_memory_note": "the call's arguments; it allocates no workspace and keeps no [E, P, C] "
-                              "intermediate besides grad_w"}
+        "device_memory_note": "the call's arguments, its partial-row workspace included; it allocates nothing "
+                              "and keeps no [E, P, C] intermediate besides grad_w"}
     del ggx, ggw, ggr, o
     # Cartesian edge convolution at equal rank
     cout = torch.empty_like(fout)
     cgx = torch.empty_like(d["x"])
     cgr = torch.empty_like(d["r"])
     t_cf = _time_ms(lambda: etp._check(lib.etp_cart_forward(
-        plan.handle, N, E, P(d["row_ptr"]), P(d["src"]), P(d["r"]), P(d["x"]), P(d["w"]), P(cout), sp), "cart"),
-        stream)
+        plan.handle, N, E, P(d["row_ptr"]), P(d["src"]), P(d["r"]), P(d["x"]), P(d["w"]), P(cout), P(tws),
+        tws.numel(), sp), "cart"), stream)
     t_cb = _time_ms(lambda: etp._check(lib.etp_cart_backward(
         plan.handle, N, E, P(d["row_ptr"]), P(d["src"]), P(rev_ptr), P(rev_perm), P(dst), P(d["r"]), P(d["x"]),
-        P(d["w"]), P(d["g"]), P(cgx), P(gw), P(cgr), sp), "cart backward"), stream)
+        P(d["w"]), P(d["g"]), P(cgx), P(gw), P(cgr), P(tws), tws.numel(), sp), "cart backward"), stream)
     t_sf = _time_ms(lambda: etp._check(lib.etp_forward(
-        plan.handle, N, E, P(d["row_ptr"]), P(d["src"]), P(d["r"]), None, P(d["x"]), P(d["w"]), P(out2), sp),
-        "forward"), stream)
+        plan.handle, N, E, P(d["row_ptr"]), P(d["src"]), P(d["r"]), None, P(d["x"]), P(d["w"]), P(out2), P(tws),
+        tws.numel(), sp), "forward"), stream)
     t_sb = _time_ms(lambda: etp._check(lib.etp_backward(
         plan.handle, N, E, P(d["row_ptr"]), P(d["src"]), P(rev_ptr), P(rev_perm), P(dst), P(d["r"]), None,
-        P(d["x"]), P(d["w"]), P(d["g"]), P(cgx), P(gw), P(cgr), sp), "backward"), stream)
+        P(d["x"]), P(d["w"]), P(d["g"]), P(cgx), P(gw), P(cgr), P(tws), tws.numel(), sp), "backward"), stream)
     alg = algorithmic(wl, Pn, nnz_total)
     cart = {}
     for key, t, nb in (("cartesian_forward", t_cf, alg["fwd_bytes"]), ("cartesian_backward", t_cb, alg["bwd_bytes"]),
@@ -484,7 +485,8 @@ def main():
     rev_ptr = torch.empty(N + 1, dtype=torch.int32, device=dev)
     rev_perm = torch.empty(E, dtype=torch.int32, device=dev)
     dst = torch.empty(E, dtype=torch.int32, device=dev)
-    ws_bytes = etp.reverse_csr_workspace_size(N, E)
+    # one scratch for the graph preprocessing and the partial rows of the segment sums (used in turn on one stream)
+    ws_bytes = max(etp.reverse_csr_workspace_size(N, E), etp.tp_workspace_size(plan, N, E, scheduled, dev))
     if scheduled:
         ws_bytes = max(ws_bytes, etp.locality_schedule_workspace_size(N, E))
         sched = etp.Schedule(N, E, torch.empty(N, dtype=torch.int32, device=dev),
@@ -522,20 +524,20 @@ def main():
         if scheduled:
             etp._check(lib.etp_forward_ordered(plan.handle, N, E, P(sched.order), P(sched.ord_ptr),
                                                P(sched.ord_edge), P(b["src"]), P(b["r"]), P(frames), P(b["x"]),
-                                               P(b["w"]), P(b["out"]), spp), "forward (scheduled)")
+                                               P(b["w"]), P(b["out"]), P(ws), ws.numel(), spp), "forward (scheduled)")
         else:
             etp._check(lib.etp_forward(plan.handle, N, E, P(b["row_ptr"]), P(b["src"]), P(b["r"]), P(frames),
-                                       P(b["x"]), P(b["w"]), P(b["out"]), spp), "forward")
+                                       P(b["x"]), P(b["w"]), P(b["out"]), P(ws), ws.numel(), spp), "forward")
         if ev:
             ev[3].record(s)
         if scheduled:
             etp._check(lib.etp_backward_ordered(plan.handle, N, E, P(sched.order), P(rev_ptr), P(rev_perm), P(dst),
                                                 P(b["r"]), P(frames), P(b["x"]), P(b["w"]), P(b["g"]), P(b["gx"]),
-                                                P(b["gw"]), P(b["gr"]), spp), "backward (scheduled)")
+                                                P(b["gw"]), P(b["gr"]), P(ws), ws.numel(), spp), "backward (scheduled)")
         else:
             etp._check(lib.etp_backward(plan.handle, N, E, P(b["row_ptr"]), P(b["src"]), P(rev_ptr), P(rev_perm),
                                         P(dst), P(b["r"]), P(frames), P(b["x"]), P(b["w"]), P(b["g"]), P(b["gx"]),
-                                        P(b["gw"]), P(b["gr"]), spp), "backward")
+                                        P(b["gw"]), P(b["gr"]), P(ws), ws.numel(), spp), "backward")
         if ev:
             ev[4].record(s)
 

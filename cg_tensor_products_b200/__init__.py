@@ -53,11 +53,12 @@ def _load():
         "etp_plan_destroy": [vp],
         "etp_plan_frames_advised": [vp, i32, ctypes.POINTER(i32)],
         "etp_edge_frames": [vp, i32, vp, vp, vp],
-        "etp_forward": [vp, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp],
-        "etp_backward": [vp, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp],
-        "etp_double_backward": [vp, i32, i32] + [vp] * 17,
-        "etp_cart_forward": [vp, i32, i32, vp, vp, vp, vp, vp, vp, vp],
-        "etp_cart_backward": [vp, i32, i32] + [vp] * 13,
+        "etp_tp_workspace_size": [vp, i32, i32, i32, ctypes.POINTER(sz)],
+        "etp_forward": [vp, i32, i32] + [vp] * 7 + [vp, sz, vp],
+        "etp_backward": [vp, i32, i32] + [vp] * 13 + [vp, sz, vp],
+        "etp_double_backward": [vp, i32, i32] + [vp] * 16 + [vp, sz, vp],
+        "etp_cart_forward": [vp, i32, i32, vp, vp, vp, vp, vp, vp, vp, sz, vp],
+        "etp_cart_backward": [vp, i32, i32] + [vp] * 12 + [vp, sz, vp],
         "etp_assemble_forces": [i32, i32, vp, vp, vp, vp, vp, vp, vp, vp],
         "etp_radial_workspace_size": [vp, i32, i32, i32, ctypes.POINTER(sz)],
         "etp_radial_forward": [vp, i32, i32, i32, ctypes.c_float, vp, vp, vp, vp, vp, sz, vp],
@@ -70,8 +71,8 @@ def _load():
         "etp_validate_csr": [i32, i32, vp, vp, vp, vp],
         "etp_locality_schedule_workspace_size": [i32, i32, ctypes.POINTER(sz)],
         "etp_build_locality_schedule": [i32, i32, vp, vp, vp, ctypes.c_float, vp, vp, vp, vp, vp, vp, vp, sz, vp],
-        "etp_forward_ordered": [vp, i32, i32] + [vp] * 10,
-        "etp_backward_ordered": [vp, i32, i32] + [vp] * 13,
+        "etp_forward_ordered": [vp, i32, i32] + [vp] * 10 + [sz, vp],
+        "etp_backward_ordered": [vp, i32, i32] + [vp] * 13 + [sz, vp],
         "etp_device_fault": [vp],
         "etp_status_string": [i32],
     }
@@ -214,9 +215,33 @@ def edge_frames(plan: Plan, r, frames=None, stream=None):
     return frames
 
 
-def forward(plan: Plan, row_ptr, src, r, x, w, out=None, frames=None, stream=None):
+def tp_workspace_size(plan: Plan, N: int, E: int, ordered: bool = False, device=None) -> int:
+    """Bytes of partial-row workspace forward/backward (ordered: their schedule variants) need
+    (etp_tp_workspace_size, answered for `device`, default the current one)."""
+    import torch
+
+    b = ctypes.c_size_t()
+    with torch.cuda.device(device if device is not None else torch.cuda.current_device()):
+        _check(_load().etp_tp_workspace_size(plan.handle, int(N), int(E), int(bool(ordered)), ctypes.byref(b)),
+               "tp_workspace_size")
+    return b.value
+
+
+def _tp_workspace(plan, N, E, ordered, workspace, dev):
+    """The caller's workspace (checked), or a new one of the needed size on dev."""
+    import torch
+
+    if workspace is None:
+        n = tp_workspace_size(plan, N, E, ordered, dev)
+        workspace = torch.empty(max(n, 16), dtype=torch.uint8, device=dev)
+    _expect(workspace, "workspace", "uint8", (None,))
+    return workspace
+
+
+def forward(plan: Plan, row_ptr, src, r, x, w, out=None, frames=None, workspace=None, stream=None):
     """out[i] = sum over row i of the weighted tensor products (launches etp_forward).
-    frames: None, or edge_frames(plan, r) (then the kernel reads those instead of building them)."""
+    frames: None, or edge_frames(plan, r) (then the kernel reads those instead of building them).
+    workspace: uint8 device tensor of tp_workspace_size bytes (allocated when None)."""
     import torch
 
     N, E = row_ptr.numel() - 1, src.numel()
@@ -229,13 +254,15 @@ def forward(plan: Plan, row_ptr, src, r, x, w, out=None, frames=None, stream=Non
         out = torch.empty((N, plan.dim_out, plan.C), device=x.device, dtype=torch.float32)
     _expect(out, "out", "float32", (N, plan.dim_out, plan.C))
     dev = _need_cuda(row_ptr, src, r, frames, x, w, out)
+    workspace = _tp_workspace(plan, N, E, False, workspace, dev)
+    _need_cuda(out, workspace)
     _launch(dev, "etp_forward", _load().etp_forward, plan.handle, N, E, _ptr(row_ptr), _ptr(src), _ptr(r),
-            _ptr(frames), _ptr(x), _ptr(w), _ptr(out), stream=stream)
+            _ptr(frames), _ptr(x), _ptr(w), _ptr(out), _ptr(workspace), workspace.numel(), stream=stream)
     return out
 
 
 def backward(plan: Plan, row_ptr, src, rev_ptr, rev_perm, dst, r, x, w, grad_out,
-             want=("x", "w", "r"), grad_x=None, grad_w=None, grad_r=None, frames=None, stream=None):
+             want=("x", "w", "r"), grad_x=None, grad_w=None, grad_r=None, frames=None, workspace=None, stream=None):
     """(grad_x, grad_w, grad_r) for the cotangent grad_out (launches etp_backward); unwanted ones are None."""
     import torch
 
@@ -260,13 +287,15 @@ def backward(plan: Plan, row_ptr, src, rev_ptr, rev_perm, dst, r, x, w, grad_out
     _expect(grad_w, "grad_w", "float32", (E, plan.n_paths, plan.C))
     _expect(grad_r, "grad_r", "float32", (E, 3))
     dev = _need_cuda(row_ptr, src, rev_ptr, rev_perm, dst, r, frames, x, w, grad_out, grad_x, grad_w, grad_r)
+    workspace = _tp_workspace(plan, N, E, False, workspace, dev)
+    _need_cuda(x, workspace)
     _launch(dev, "etp_backward", _load().etp_backward, plan.handle, N, E, _ptr(row_ptr), _ptr(src), _ptr(rev_ptr),
             _ptr(rev_perm), _ptr(dst), _ptr(r), _ptr(frames), _ptr(x), _ptr(w), _ptr(grad_out), _ptr(grad_x),
-            _ptr(grad_w), _ptr(grad_r), stream=stream)
+            _ptr(grad_w), _ptr(grad_r), _ptr(workspace), workspace.numel(), stream=stream)
     return grad_x, grad_w, grad_r
 
 
-def cart_forward(plan: Plan, row_ptr, src, r, x, w, out=None, stream=None):
+def cart_forward(plan: Plan, row_ptr, src, r, x, w, out=None, workspace=None, stream=None):
     """Cartesian edge convolution (launches etp_cart_forward): x and out in independent STF components."""
     import torch
 
@@ -279,13 +308,15 @@ def cart_forward(plan: Plan, row_ptr, src, r, x, w, out=None, stream=None):
         out = torch.empty((N, plan.dim_out, plan.C), device=x.device, dtype=torch.float32)
     _expect(out, "out", "float32", (N, plan.dim_out, plan.C))
     dev = _need_cuda(row_ptr, src, r, x, w, out)
+    workspace = _tp_workspace(plan, N, E, False, workspace, dev)
+    _need_cuda(out, workspace)
     _launch(dev, "etp_cart_forward", _load().etp_cart_forward, plan.handle, N, E, _ptr(row_ptr), _ptr(src), _ptr(r),
-            _ptr(x), _ptr(w), _ptr(out), stream=stream)
+            _ptr(x), _ptr(w), _ptr(out), _ptr(workspace), workspace.numel(), stream=stream)
     return out
 
 
 def cart_backward(plan: Plan, row_ptr, src, rev_ptr, rev_perm, dst, r, x, w, grad_out, want=("x", "w", "r"),
-                  stream=None):
+                  workspace=None, stream=None):
     """VJP of cart_forward (launches etp_cart_backward): (grad_x, grad_w, grad_r), unwanted ones None."""
     import torch
 
@@ -303,14 +334,16 @@ def cart_backward(plan: Plan, row_ptr, src, rev_ptr, rev_perm, dst, r, x, w, gra
     gw = torch.empty((E, plan.n_paths, plan.C), device=dev, dtype=torch.float32) if "w" in want else None
     gr = torch.empty((E, 3), device=dev, dtype=torch.float32) if "r" in want else None
     dev = _need_cuda(row_ptr, src, rev_ptr, rev_perm, dst, r, x, w, grad_out, gx, gw, gr)
+    workspace = _tp_workspace(plan, N, E, False, workspace, dev)
+    _need_cuda(x, workspace)
     _launch(dev, "etp_cart_backward", _load().etp_cart_backward, plan.handle, N, E, _ptr(row_ptr), _ptr(src),
             _ptr(rev_ptr), _ptr(rev_perm), _ptr(dst), _ptr(r), _ptr(x), _ptr(w), _ptr(grad_out), _ptr(gx), _ptr(gw),
-            _ptr(gr), stream=stream)
+            _ptr(gr), _ptr(workspace), workspace.numel(), stream=stream)
     return gx, gw, gr
 
 
 def double_backward(plan: Plan, row_ptr, src, rev_ptr, rev_perm, dst, r, x, w, grad_out, gg_x=None, gg_w=None,
-                    gg_r=None, want=("g", "x", "w", "r"), out=None, stream=None):
+                    gg_r=None, want=("g", "x", "w", "r"), out=None, workspace=None, stream=None):
     """VJP of the VJP (launches etp_double_backward): dict with 'grad_g', 'grad_x', 'grad_w', 'grad_r'
     (the wanted ones) of <gg_x, grad_x> + <gg_w, grad_w> + <gg_r, grad_r>; None cotangents are zero."""
     import torch
@@ -336,10 +369,12 @@ def double_backward(plan: Plan, row_ptr, src, rev_ptr, rev_perm, dst, r, x, w, g
             out[key] = torch.empty(shapes[k], device=x.device, dtype=torch.float32)
         _expect(out.get(key), key, "float32", shapes[k])
     dev = _need_cuda(row_ptr, src, rev_ptr, rev_perm, dst, r, x, w, grad_out, gg_x, gg_w, gg_r, *out.values())
+    workspace = _tp_workspace(plan, N, E, False, workspace, dev)
+    _need_cuda(x, workspace)
     _launch(dev, "etp_double_backward", _load().etp_double_backward, plan.handle, N, E, _ptr(row_ptr), _ptr(src),
             _ptr(rev_ptr), _ptr(rev_perm), _ptr(dst), _ptr(r), _ptr(x), _ptr(w), _ptr(grad_out), _ptr(gg_x),
             _ptr(gg_w), _ptr(gg_r), _ptr(out.get("grad_g")), _ptr(out.get("grad_x")), _ptr(out.get("grad_w")),
-            _ptr(out.get("grad_r")), stream=stream)
+            _ptr(out.get("grad_r")), _ptr(workspace), workspace.numel(), stream=stream)
     return out
 
 
@@ -549,7 +584,7 @@ def locality_schedule(N: int, row_ptr, src, pos, cell: float, out: Schedule = No
     return out
 
 
-def forward_ordered(plan: Plan, sched: Schedule, src, r, x, w, out=None, frames=None, stream=None):
+def forward_ordered(plan: Plan, sched: Schedule, src, r, x, w, out=None, frames=None, workspace=None, stream=None):
     """forward() on a locality schedule (etp_forward_ordered): the same out, rows visited in schedule order."""
     import torch
 
@@ -563,14 +598,16 @@ def forward_ordered(plan: Plan, sched: Schedule, src, r, x, w, out=None, frames=
         out = torch.empty((N, plan.dim_out, plan.C), device=x.device, dtype=torch.float32)
     _expect(out, "out", "float32", (N, plan.dim_out, plan.C))
     dev = _need_cuda(sched.order, sched.ord_ptr, sched.ord_edge, src, r, frames, x, w, out)
+    workspace = _tp_workspace(plan, N, E, True, workspace, dev)
+    _need_cuda(out, workspace)
     _launch(dev, "etp_forward_ordered", _load().etp_forward_ordered, plan.handle, N, E, _ptr(sched.order),
             _ptr(sched.ord_ptr), _ptr(sched.ord_edge), _ptr(src), _ptr(r), _ptr(frames), _ptr(x), _ptr(w),
-            _ptr(out), stream=stream)
+            _ptr(out), _ptr(workspace), workspace.numel(), stream=stream)
     return out
 
 
 def backward_ordered(plan: Plan, sched: Schedule, r, x, w, grad_out, want=("x", "w", "r"), grad_x=None,
-                     grad_w=None, grad_r=None, frames=None, stream=None):
+                     grad_w=None, grad_r=None, frames=None, workspace=None, stream=None):
     """backward() on a locality schedule (etp_backward_ordered): the same (grad_x, grad_w, grad_r)."""
     import torch
 
@@ -592,9 +629,12 @@ def backward_ordered(plan: Plan, sched: Schedule, r, x, w, grad_out, want=("x", 
     _expect(grad_r, "grad_r", "float32", (E, 3))
     dev = _need_cuda(sched.order, sched.rev_ptr, sched.rev_perm, sched.dst, r, frames, x, w, grad_out, grad_x,
                      grad_w, grad_r)
+    workspace = _tp_workspace(plan, N, E, True, workspace, dev)
+    _need_cuda(x, workspace)
     _launch(dev, "etp_backward_ordered", _load().etp_backward_ordered, plan.handle, N, E, _ptr(sched.order),
             _ptr(sched.rev_ptr), _ptr(sched.rev_perm), _ptr(sched.dst), _ptr(r), _ptr(frames), _ptr(x), _ptr(w),
-            _ptr(grad_out), _ptr(grad_x), _ptr(grad_w), _ptr(grad_r), stream=stream)
+            _ptr(grad_out), _ptr(grad_x), _ptr(grad_w), _ptr(grad_r), _ptr(workspace), workspace.numel(),
+            stream=stream)
     return grad_x, grad_w, grad_r
 
 

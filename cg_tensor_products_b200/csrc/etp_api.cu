@@ -220,9 +220,23 @@ namespace {
 // 1/waves of the rows, in the schedule's order.
 constexpr int kOrderedWaves = 8;
 
+// Bytes of partial rows the forward (backward) of this plan, graph size and
+// schedule needs, the larger of the two frame variants.
+size_t partial_bytes(etp_plan_t plan, int N, int E, bool backward, bool ordered) {
+    if (E <= 0 || N <= 0) return 0;
+    size_t b = 0;
+    for (int framed = 0; framed < 2; ++framed) {
+        const etp::LaunchShape sh =
+            etp::launch_shape(plan->C, plan->L, plan->o3, backward, framed != 0, E, N, ordered ? kOrderedWaves : 1);
+        const size_t v = etp::partial_rows_bytes(sh.ntasks, plan->D, plan->C);
+        b = v > b ? v : b;
+    }
+    return b;
+}
+
 etp_status forward_impl(etp_plan_t plan, int N, int E, const int32_t* row_ptr, const int32_t* src, const float* r,
                         const float* frames, const float* x, const float* w, float* out, const int32_t* order,
-                        const int32_t* pos_edge, etp_stream_t stream) {
+                        const int32_t* pos_edge, void* workspace, size_t workspace_bytes, etp_stream_t stream) {
     if (!plan || N < 0 || E < 0) return ETP_ERR_INVALID_ARG;
     if (N == 0) return E == 0 ? ETP_OK : ETP_ERR_INVALID_ARG;
     if (!row_ptr || !x || !out || !aligned4(row_ptr) || !aligned16(x) || !aligned16(out)) return ETP_ERR_INVALID_ARG;
@@ -230,11 +244,12 @@ etp_status forward_impl(etp_plan_t plan, int N, int E, const int32_t* row_ptr, c
     if (E > 0 && (frames ? !aligned16(frames) : (!r || !aligned4(r)))) return ETP_ERR_INVALID_ARG;
     if ((order && !aligned4(order)) || (pos_edge && !aligned4(pos_edge))) return ETP_ERR_INVALID_ARG;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    // rows cut by a task boundary are reduced onto zeros; empty rows stay zero
-    cudaError_t err = cudaMemsetAsync(out, 0, sizeof(float) * (size_t)N * plan->D * plan->C, s);
-    if (err != cudaSuccess || E == 0) return cuda_status(err);
+    if (E == 0) return cuda_status(cudaMemsetAsync(out, 0, sizeof(float) * (size_t)N * plan->D * plan->C, s));
     const etp::LaunchShape sh = etp::launch_shape(plan->C, plan->L, plan->o3, false, frames != nullptr, E, N,
                                                   order ? kOrderedWaves : 1);
+    if (!workspace || !aligned16(workspace)) return ETP_ERR_INVALID_ARG;
+    if (workspace_bytes < etp::partial_rows_bytes(sh.ntasks, plan->D, plan->C)) return ETP_ERR_WORKSPACE;
+    cudaError_t err;
     etp::FwdArgs a{N,
                    E,
                    row_ptr,
@@ -249,20 +264,25 @@ etp_status forward_impl(etp_plan_t plan, int N, int E, const int32_t* row_ptr, c
                    sh.slices,
                    sh.ntasks,
                    order,
-                   pos_edge};
+                   pos_edge,
+                   static_cast<float4*>(workspace)};
     switch (plan->L) {
         case 0: err = etp::launch_forward<0>(plan->o3, a, sh.grid, sh.smem_bytes, s); break;
         case 1: err = etp::launch_forward<1>(plan->o3, a, sh.grid, sh.smem_bytes, s); break;
         case 2: err = etp::launch_forward<2>(plan->o3, a, sh.grid, sh.smem_bytes, s); break;
         default: err = etp::launch_forward<3>(plan->o3, a, sh.grid, sh.smem_bytes, s); break;
     }
-    return cuda_status(err);
+    if (err != cudaSuccess) return cuda_status(err);
+    return cuda_status(etp::launch_combine_rows(row_ptr, order, N, E, sh.ntasks, plan->D * plan->C / 4,
+                                                static_cast<const float4*>(workspace), reinterpret_cast<float4*>(out),
+                                                s));
 }
 
 etp_status backward_impl(etp_plan_t plan, int N, int E, const int32_t* row_ptr, const int32_t* src,
                          const int32_t* rev_ptr, const int32_t* rev_perm, const int32_t* dst_of_edge, const float* r,
                          const float* frames, const float* x, const float* w, const float* grad_out, float* grad_x,
-                         float* grad_w, float* grad_r, const int32_t* order, etp_stream_t stream) {
+                         float* grad_w, float* grad_r, const int32_t* order, void* workspace,
+                         size_t workspace_bytes, etp_stream_t stream) {
     if (!plan || N < 0 || E < 0) return ETP_ERR_INVALID_ARG;
     if (N == 0) return E == 0 ? ETP_OK : ETP_ERR_INVALID_ARG;
     if (!rev_ptr || !x || !grad_out || !aligned4(rev_ptr) || !aligned16(x) || !aligned16(grad_out))
@@ -283,12 +303,16 @@ etp_status backward_impl(etp_plan_t plan, int N, int E, const int32_t* row_ptr, 
     }
     if (!grad_x && !grad_w && !grad_r) return ETP_OK;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    cudaError_t err = cudaSuccess;
-    // source rows cut by a task boundary are reduced onto zeros; sources without edges stay zero
-    if (grad_x) err = cudaMemsetAsync(grad_x, 0, sizeof(float) * (size_t)N * plan->D * plan->C, s);
-    if (err != cudaSuccess || E == 0) return cuda_status(err);
+    if (E == 0)
+        return grad_x ? cuda_status(cudaMemsetAsync(grad_x, 0, sizeof(float) * (size_t)N * plan->D * plan->C, s))
+                      : ETP_OK;
     const etp::LaunchShape sh = etp::launch_shape(plan->C, plan->L, plan->o3, true, frames != nullptr, E, N,
                                                   order ? kOrderedWaves : 1);
+    if (grad_x) {
+        if (!workspace || !aligned16(workspace)) return ETP_ERR_INVALID_ARG;
+        if (workspace_bytes < etp::partial_rows_bytes(sh.ntasks, plan->D, plan->C)) return ETP_ERR_WORKSPACE;
+    }
+    cudaError_t err;
     etp::BwdArgs a{N,
                    E,
                    row_ptr,
@@ -308,53 +332,74 @@ etp_status backward_impl(etp_plan_t plan, int N, int E, const int32_t* row_ptr, 
                    sh.team,
                    sh.slices,
                    sh.ntasks,
-                   order};
+                   order,
+                   grad_x ? static_cast<float4*>(workspace) : nullptr};
     switch (plan->L) {
         case 0: err = etp::launch_backward<0>(plan->o3, a, sh.grid, sh.smem_bytes, s); break;
         case 1: err = etp::launch_backward<1>(plan->o3, a, sh.grid, sh.smem_bytes, s); break;
         case 2: err = etp::launch_backward<2>(plan->o3, a, sh.grid, sh.smem_bytes, s); break;
         default: err = etp::launch_backward<3>(plan->o3, a, sh.grid, sh.smem_bytes, s); break;
     }
-    return cuda_status(err);
+    if (err != cudaSuccess || !grad_x) return cuda_status(err);
+    return cuda_status(etp::launch_combine_rows(rev_ptr, order, N, E, sh.ntasks, plan->D * plan->C / 4,
+                                                static_cast<const float4*>(workspace),
+                                                reinterpret_cast<float4*>(grad_x), s));
 }
 
 }  // namespace
 
+etp_status etp_tp_workspace_size(etp_plan_t plan, int N, int E, int ordered, size_t* bytes) {
+    if (!plan || N < 0 || E < 0 || !bytes) return ETP_ERR_INVALID_ARG;
+    size_t m = partial_bytes(plan, N, E, false, ordered != 0);
+    const size_t more[] = {partial_bytes(plan, N, E, true, ordered != 0),
+                           etp::double_backward_partial_bytes(plan->L, plan->o3, plan->C, N, E),
+                           etp::cart_partial_bytes(plan->L, plan->o3, plan->C, N, E)};
+    for (size_t v : more) m = v > m ? v : m;
+    *bytes = m;
+    return ETP_OK;
+}
+
 etp_status etp_forward(etp_plan_t plan, int N, int E, const int32_t* row_ptr, const int32_t* src, const float* r,
-                       const float* frames, const float* x, const float* w, float* out, etp_stream_t stream) {
-    return forward_impl(plan, N, E, row_ptr, src, r, frames, x, w, out, nullptr, nullptr, stream);
+                       const float* frames, const float* x, const float* w, float* out, void* workspace,
+                       size_t workspace_bytes, etp_stream_t stream) {
+    return forward_impl(plan, N, E, row_ptr, src, r, frames, x, w, out, nullptr, nullptr, workspace, workspace_bytes,
+                        stream);
 }
 
 etp_status etp_forward_ordered(etp_plan_t plan, int N, int E, const int32_t* order, const int32_t* ord_ptr,
                                const int32_t* ord_edge, const int32_t* src, const float* r, const float* frames,
-                               const float* x, const float* w, float* out, etp_stream_t stream) {
+                               const float* x, const float* w, float* out, void* workspace,
+                               size_t workspace_bytes, etp_stream_t stream) {
     if (N > 0 && (!order || (E > 0 && !ord_edge))) return ETP_ERR_INVALID_ARG;
-    return forward_impl(plan, N, E, ord_ptr, src, r, frames, x, w, out, order, ord_edge, stream);
+    return forward_impl(plan, N, E, ord_ptr, src, r, frames, x, w, out, order, ord_edge, workspace, workspace_bytes,
+                        stream);
 }
 
 etp_status etp_backward(etp_plan_t plan, int N, int E, const int32_t* row_ptr, const int32_t* src,
                         const int32_t* rev_ptr, const int32_t* rev_perm, const int32_t* dst_of_edge, const float* r,
                         const float* frames, const float* x, const float* w, const float* grad_out, float* grad_x,
-                        float* grad_w, float* grad_r, etp_stream_t stream) {
+                        float* grad_w, float* grad_r, void* workspace, size_t workspace_bytes, etp_stream_t stream) {
     if (!row_ptr || (E > 0 && !src)) return ETP_ERR_INVALID_ARG;
     return backward_impl(plan, N, E, row_ptr, src, rev_ptr, rev_perm, dst_of_edge, r, frames, x, w, grad_out, grad_x,
-                         grad_w, grad_r, nullptr, stream);
+                         grad_w, grad_r, nullptr, workspace, workspace_bytes, stream);
 }
 
 etp_status etp_backward_ordered(etp_plan_t plan, int N, int E, const int32_t* order, const int32_t* rev_ptr,
                                 const int32_t* rev_perm, const int32_t* dst_of_edge, const float* r,
                                 const float* frames, const float* x, const float* w, const float* grad_out,
-                                float* grad_x, float* grad_w, float* grad_r, etp_stream_t stream) {
+                                float* grad_x, float* grad_w, float* grad_r, void* workspace,
+                                size_t workspace_bytes, etp_stream_t stream) {
     if (N > 0 && (!order || (E > 0 && !dst_of_edge))) return ETP_ERR_INVALID_ARG;
     return backward_impl(plan, N, E, nullptr, nullptr, rev_ptr, rev_perm, dst_of_edge, r, frames, x, w, grad_out,
-                         grad_x, grad_w, grad_r, order, stream);
+                         grad_x, grad_w, grad_r, order, workspace, workspace_bytes, stream);
 }
 
 etp_status etp_double_backward(etp_plan_t plan, int N, int E, const int32_t* row_ptr, const int32_t* src,
                                const int32_t* rev_ptr, const int32_t* rev_perm, const int32_t* dst_of_edge,
                                const float* r, const float* x, const float* w, const float* grad_out,
                                const float* gg_x, const float* gg_w, const float* gg_r, float* grad_grad_out,
-                               float* grad_x, float* grad_w, float* grad_r, etp_stream_t stream) {
+                               float* grad_x, float* grad_w, float* grad_r, void* workspace,
+                               size_t workspace_bytes, etp_stream_t stream) {
     if (!plan || N < 0 || E < 0) return ETP_ERR_INVALID_ARG;
     if (N == 0) return E == 0 ? ETP_OK : ETP_ERR_INVALID_ARG;
     if (!row_ptr || !rev_ptr || !x || !grad_out || !aligned4(row_ptr) || !aligned4(rev_ptr) || !aligned16(x) ||
@@ -373,25 +418,37 @@ etp_status etp_double_backward(etp_plan_t plan, int N, int E, const int32_t* row
         grad_r = nullptr;
     }
     if (!grad_grad_out && !grad_x && !grad_w && !grad_r) return ETP_OK;
+    if (E > 0 && (grad_grad_out || grad_x)) {
+        if (!workspace || !aligned16(workspace)) return ETP_ERR_INVALID_ARG;
+        if (workspace_bytes < etp::double_backward_partial_bytes(plan->L, plan->o3, plan->C, N, E))
+            return ETP_ERR_WORKSPACE;
+    }
     return cuda_status(etp::double_backward(plan->L, plan->o3, plan->C, N, E, row_ptr, src, rev_ptr, rev_perm,
                                             dst_of_edge, r, x, w, grad_out, gg_x, gg_w, gg_r, grad_grad_out, grad_x,
-                                            grad_w, grad_r, reinterpret_cast<cudaStream_t>(stream)));
+                                            grad_w, grad_r, workspace, workspace_bytes,
+                                            reinterpret_cast<cudaStream_t>(stream)));
 }
 
 etp_status etp_cart_forward(etp_plan_t plan, int N, int E, const int32_t* row_ptr, const int32_t* src, const float* r,
-                            const float* x, const float* w, float* out, etp_stream_t stream) {
+                            const float* x, const float* w, float* out, void* workspace, size_t workspace_bytes,
+                            etp_stream_t stream) {
     if (!plan || N < 0 || E < 0) return ETP_ERR_INVALID_ARG;
     if (N == 0) return E == 0 ? ETP_OK : ETP_ERR_INVALID_ARG;
     if (!row_ptr || !x || !out || !aligned4(row_ptr) || !aligned16(x) || !aligned16(out)) return ETP_ERR_INVALID_ARG;
     if (E > 0 && (!src || !w || !r || !aligned4(src) || !aligned16(w) || !aligned4(r))) return ETP_ERR_INVALID_ARG;
-    return cuda_status(etp::cart_forward(plan->L, plan->o3, plan->C, N, E, row_ptr, src, r, x, w, out,
-                                         reinterpret_cast<cudaStream_t>(stream)));
+    if (E > 0) {
+        if (!workspace || !aligned16(workspace)) return ETP_ERR_INVALID_ARG;
+        if (workspace_bytes < etp::cart_partial_bytes(plan->L, plan->o3, plan->C, N, E)) return ETP_ERR_WORKSPACE;
+    }
+    return cuda_status(etp::cart_forward(plan->L, plan->o3, plan->C, N, E, row_ptr, src, r, x, w, out, workspace,
+                                         workspace_bytes, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 etp_status etp_cart_backward(etp_plan_t plan, int N, int E, const int32_t* row_ptr, const int32_t* src,
                              const int32_t* rev_ptr, const int32_t* rev_perm, const int32_t* dst_of_edge,
                              const float* r, const float* x, const float* w, const float* grad_out, float* grad_x,
-                             float* grad_w, float* grad_r, etp_stream_t stream) {
+                             float* grad_w, float* grad_r, void* workspace, size_t workspace_bytes,
+                             etp_stream_t stream) {
     if (!plan || N < 0 || E < 0) return ETP_ERR_INVALID_ARG;
     if (N == 0) return E == 0 ? ETP_OK : ETP_ERR_INVALID_ARG;
     if (!row_ptr || !rev_ptr || !x || !grad_out || !aligned4(row_ptr) || !aligned4(rev_ptr) || !aligned16(x) ||
@@ -409,8 +466,12 @@ etp_status etp_cart_backward(etp_plan_t plan, int N, int E, const int32_t* row_p
         grad_r = nullptr;
     }
     if (!grad_x && !grad_w && !grad_r) return ETP_OK;
+    if (E > 0 && grad_x) {
+        if (!workspace || !aligned16(workspace)) return ETP_ERR_INVALID_ARG;
+        if (workspace_bytes < etp::cart_partial_bytes(plan->L, plan->o3, plan->C, N, E)) return ETP_ERR_WORKSPACE;
+    }
     return cuda_status(etp::cart_backward(plan->L, plan->o3, plan->C, N, E, row_ptr, rev_ptr, rev_perm, dst_of_edge,
-                                          r, x, w, grad_out, grad_x, grad_w, grad_r,
+                                          r, x, w, grad_out, grad_x, grad_w, grad_r, workspace, workspace_bytes,
                                           reinterpret_cast<cudaStream_t>(stream)));
 }
 

@@ -55,6 +55,7 @@ struct Args {
     float2* grad_w;  // may be null
     float* grad_r;   // may be null
     int C2, team, slices, ntasks;
+    float2* part;    // partial rows [ntasks][2][D][C] of rows cut by task boundaries
 };
 
 // Edge attribute (independent STF components, blocks l = 0..L) of the unit vector
@@ -159,7 +160,7 @@ __global__ void __launch_bounds__(kThreads) etp_cart_fwd_kernel(Args a) {
     for (int e = k0; e < k1; ++e) {
         while (e >= row_hi && row < a.N - 1) {
             if (row_hi > max(row_lo, k0)) {
-                flush_row<D>(a.out + (size_t)row * D * C2 + tm.cp, C2, acc, row_lo >= k0);
+                store_row<D>(row_slot(a.out, a.part, row, row_lo, row_hi, k0, k1, tm.task, D * C2, tm.cp), C2, acc);
 #pragma unroll
                 for (int k = 0; k < D; ++k) acc[k] = f2_zero();
             }
@@ -194,7 +195,7 @@ __global__ void __launch_bounds__(kThreads) etp_cart_fwd_kernel(Args a) {
             for (int m = 0; m < 2 * pt.l3 + 1; ++m) acc[pt.l3 * pt.l3 + m] = __ffma2_rn(wp, t[m], acc[pt.l3 * pt.l3 + m]);
         });
     }
-    flush_row<D>(a.out + (size_t)row * D * C2 + tm.cp, C2, acc, row_lo >= k0 && row_hi <= k1);
+    store_row<D>(row_slot(a.out, a.part, row, row_lo, row_hi, k0, k1, tm.task, D * C2, tm.cp), C2, acc);
 }
 
 template <int L, bool O3>
@@ -217,7 +218,9 @@ __global__ void __launch_bounds__(kThreads) etp_cart_bwd_kernel(Args a) {
     for (int q = k0; q < k1; ++q) {
         while (q >= row_hi && row < a.N - 1) {
             if (row_hi > max(row_lo, k0)) {
-                if (a.grad_x) flush_row<D>(a.grad_x + (size_t)row * D * C2 + tm.cp, C2, gx, row_lo >= k0);
+                if (a.grad_x)
+                    store_row<D>(row_slot(a.grad_x, a.part, row, row_lo, row_hi, k0, k1, tm.task, D * C2, tm.cp), C2,
+                                 gx);
 #pragma unroll
                 for (int k = 0; k < D; ++k) gx[k] = f2_zero();
             }
@@ -302,7 +305,8 @@ __global__ void __launch_bounds__(kThreads) etp_cart_bwd_kernel(Args a) {
             }
         }
     }
-    if (a.grad_x) flush_row<D>(a.grad_x + (size_t)row * D * C2 + tm.cp, C2, gx, row_lo >= k0 && row_hi <= k1);
+    if (a.grad_x)
+        store_row<D>(row_slot(a.grad_x, a.part, row, row_lo, row_hi, k0, k1, tm.task, D * C2, tm.cp), C2, gx);
 }
 
 }  // namespace cart
@@ -310,67 +314,103 @@ __global__ void __launch_bounds__(kThreads) etp_cart_bwd_kernel(Args a) {
 // ---------------------------------------------------------------------------
 namespace {
 
+// Tasks of the forward or backward kernel: one wave, at least 16 edges each, no
+// more tasks than rows.
 template <int L, bool O3>
-cudaError_t launch_cart(cart::Args a, bool backward, cudaStream_t s) {
+int cart_tasks(int C, int N, int E, bool backward) {
     const void* k = backward ? (const void*)cart::etp_cart_bwd_kernel<L, O3> : (const void*)cart::etp_cart_fwd_kernel<L, O3>;
-    cudaError_t err;
+    const int T = C / 2 < 32 ? C / 2 : 32, slices = C / (2 * T);
     int dev = 0, sms = 1, bps = 1;
-    if ((err = cudaGetDevice(&dev)) != cudaSuccess) return err;
-    if ((err = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return err;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) !=
+                                                   cudaSuccess || sms < 1)
+        sms = 1;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&bps, k, cart::kThreads, 0) != cudaSuccess || bps < 1) bps = 1;
+    const long long cap = (long long)sms * bps * (cart::kThreads / T) / slices;
+    long long want = ((long long)E + 15) / 16;
+    if (want > N) want = N;
+    const long long nt = want < cap ? want : cap;
+    return (int)(nt < 1 ? 1 : nt);
+}
+
+template <int L, bool O3>
+cudaError_t launch_cart(cart::Args a, bool backward, size_t part_bytes, cudaStream_t s) {
+    const void* k = backward ? (const void*)cart::etp_cart_bwd_kernel<L, O3> : (const void*)cart::etp_cart_fwd_kernel<L, O3>;
+    const int C = 2 * a.C2, D = (L + 1) * (L + 1);
+    a.ntasks = cart_tasks<L, O3>(C, a.N, a.E, backward);
+    float2* rows = backward ? a.grad_x : a.out;
+    if (rows && part_bytes < partial_rows_bytes(a.ntasks, D, C)) return cudaErrorInvalidValue;
     const int teams_per_block = cart::kThreads / a.team;
-    long long cap = (long long)sms * bps * teams_per_block / a.slices;
-    long long want = ((long long)a.E + 15) / 16;
-    if (want > a.N) want = a.N;
-    long long nt = want < cap ? want : cap;
-    a.ntasks = (int)(nt < 1 ? 1 : nt);
     const long long teams = (long long)a.ntasks * a.slices;
     const unsigned blocks = (unsigned)((teams + teams_per_block - 1) / teams_per_block);
     void* args[] = {&a};
-    return cudaLaunchKernel(k, dim3(blocks), dim3(cart::kThreads), args, 0, s);
+    cudaError_t err = cudaLaunchKernel(k, dim3(blocks), dim3(cart::kThreads), args, 0, s);
+    if (err != cudaSuccess || !rows) return err;
+    return launch_combine_rows(backward ? a.rev_ptr : a.row_ptr, nullptr, a.N, a.E, a.ntasks, D * C / 4,
+                               reinterpret_cast<const float4*>(a.part), reinterpret_cast<float4*>(rows), s);
 }
 
-cudaError_t dispatch_cart(int L, bool o3, const cart::Args& a, bool backward, cudaStream_t s) {
+cudaError_t dispatch_cart(int L, bool o3, const cart::Args& a, bool backward, size_t part_bytes, cudaStream_t s) {
     switch (L * 2 + (o3 ? 1 : 0)) {
-        case 0: return launch_cart<0, false>(a, backward, s);
-        case 1: return launch_cart<0, true>(a, backward, s);
-        case 2: return launch_cart<1, false>(a, backward, s);
-        case 3: return launch_cart<1, true>(a, backward, s);
-        case 4: return launch_cart<2, false>(a, backward, s);
-        case 5: return launch_cart<2, true>(a, backward, s);
-        case 6: return launch_cart<3, false>(a, backward, s);
-        default: return launch_cart<3, true>(a, backward, s);
+        case 0: return launch_cart<0, false>(a, backward, part_bytes, s);
+        case 1: return launch_cart<0, true>(a, backward, part_bytes, s);
+        case 2: return launch_cart<1, false>(a, backward, part_bytes, s);
+        case 3: return launch_cart<1, true>(a, backward, part_bytes, s);
+        case 4: return launch_cart<2, false>(a, backward, part_bytes, s);
+        case 5: return launch_cart<2, true>(a, backward, part_bytes, s);
+        case 6: return launch_cart<3, false>(a, backward, part_bytes, s);
+        default: return launch_cart<3, true>(a, backward, part_bytes, s);
+    }
+}
+
+int cart_tasks_for(int L, bool o3, int C, int N, int E, bool backward) {
+    switch (L * 2 + (o3 ? 1 : 0)) {
+        case 0: return cart_tasks<0, false>(C, N, E, backward);
+        case 1: return cart_tasks<0, true>(C, N, E, backward);
+        case 2: return cart_tasks<1, false>(C, N, E, backward);
+        case 3: return cart_tasks<1, true>(C, N, E, backward);
+        case 4: return cart_tasks<2, false>(C, N, E, backward);
+        case 5: return cart_tasks<2, true>(C, N, E, backward);
+        case 6: return cart_tasks<3, false>(C, N, E, backward);
+        default: return cart_tasks<3, true>(C, N, E, backward);
     }
 }
 
 }  // namespace
 
+size_t cart_partial_bytes(int L, bool o3, int C, int N, int E) {
+    if (E <= 0 || N <= 0) return 0;
+    const int a = cart_tasks_for(L, o3, C, N, E, false), b = cart_tasks_for(L, o3, C, N, E, true);
+    return partial_rows_bytes(a > b ? a : b, (L + 1) * (L + 1), C);
+}
+
 cudaError_t cart_forward(int L, bool o3, int C, int N, int E, const int32_t* row_ptr, const int32_t* src,
-                         const float* r, const float* x, const float* w, float* out, cudaStream_t s) {
+                         const float* r, const float* x, const float* w, float* out, void* part, size_t part_bytes,
+                         cudaStream_t s) {
     const int D = (L + 1) * (L + 1);
-    cudaError_t err = cudaMemsetAsync(out, 0, sizeof(float) * (size_t)N * D * C, s);
-    if (err != cudaSuccess || E == 0) return err;
+    if (E == 0) return cudaMemsetAsync(out, 0, sizeof(float) * (size_t)N * D * C, s);
     const int team = C / 2 < 32 ? C / 2 : 32;
     cart::Args a{N, E, row_ptr, src, nullptr, nullptr, nullptr, r, reinterpret_cast<const float2*>(x),
                  reinterpret_cast<const float2*>(w), nullptr, reinterpret_cast<float2*>(out), nullptr, nullptr,
-                 nullptr, C / 2, team, C / (2 * team), 1};
-    return dispatch_cart(L, o3, a, false, s);
+                 nullptr, C / 2, team, C / (2 * team), 1, static_cast<float2*>(part)};
+    return dispatch_cart(L, o3, a, false, part_bytes, s);
 }
 
 cudaError_t cart_backward(int L, bool o3, int C, int N, int E, const int32_t* row_ptr, const int32_t* rev_ptr,
                           const int32_t* rev_perm, const int32_t* dst, const float* r, const float* x, const float* w,
-                          const float* g, float* grad_x, float* grad_w, float* grad_r, cudaStream_t s) {
+                          const float* g, float* grad_x, float* grad_w, float* grad_r, void* part,
+                          size_t part_bytes, cudaStream_t s) {
     const int D = (L + 1) * (L + 1);
     const int team = C / 2 < 32 ? C / 2 : 32, slices = C / (2 * team);
     cudaError_t err;
-    if (grad_x && (err = cudaMemsetAsync(grad_x, 0, sizeof(float) * (size_t)N * D * C, s)) != cudaSuccess) return err;
+    // with two channel slices, grad_r is the sum of the slices' two terms (added onto zero: order-free)
     if (grad_r && slices > 1 && (err = cudaMemsetAsync(grad_r, 0, sizeof(float) * 3 * (size_t)E, s)) != cudaSuccess)
         return err;
-    if (E == 0) return cudaSuccess;
+    if (E == 0) return grad_x ? cudaMemsetAsync(grad_x, 0, sizeof(float) * (size_t)N * D * C, s) : cudaSuccess;
     cart::Args a{N, E, row_ptr, nullptr, rev_ptr, rev_perm, dst, r, reinterpret_cast<const float2*>(x),
                  reinterpret_cast<const float2*>(w), reinterpret_cast<const float2*>(g), nullptr,
-                 reinterpret_cast<float2*>(grad_x), reinterpret_cast<float2*>(grad_w), grad_r, C / 2, team, slices, 1};
-    return dispatch_cart(L, o3, a, true, s);
+                 reinterpret_cast<float2*>(grad_x), reinterpret_cast<float2*>(grad_w), grad_r, C / 2, team, slices, 1,
+                 static_cast<float2*>(part)};
+    return dispatch_cart(L, o3, a, true, part_bytes, s);
 }
 
 }  // namespace etp

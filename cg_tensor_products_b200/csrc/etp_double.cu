@@ -73,6 +73,7 @@ struct Args {
     float* grad_r;      // may be null
     int C2;             // channel pairs
     int team, slices, ntasks;
+    float2* part;       // partial rows [ntasks][2][D][C] of rows cut by task boundaries
 };
 
 __device__ __forceinline__ float2 f2_sub(float2 a, float2 b) { return make_float2(a.x - b.x, a.y - b.y); }
@@ -240,7 +241,9 @@ __global__ void __launch_bounds__(kThreads) etp_dd_dst_kernel(Args a) {
     for (int e = k0; e < k1; ++e) {
         while (e >= row_hi && row < a.N - 1) {
             if (row_hi > max(row_lo, k0)) {
-                if (a.grad_g) flush_row<D>(a.grad_g + (size_t)row * D * C2 + tm.cp, C2, acc, row_lo >= k0);
+                if (a.grad_g)
+                    store_row<D>(row_slot(a.grad_g, a.part, row, row_lo, row_hi, k0, k1, tm.task, D * C2, tm.cp), C2,
+                                 acc);
 #pragma unroll
                 for (int k = 0; k < D; ++k) acc[k] = f2_zero();
             }
@@ -337,7 +340,8 @@ __global__ void __launch_bounds__(kThreads) etp_dd_dst_kernel(Args a) {
             });
         }
     }
-    if (a.grad_g) flush_row<D>(a.grad_g + (size_t)row * D * C2 + tm.cp, C2, acc, row_lo >= k0 && row_hi <= k1);
+    if (a.grad_g)
+        store_row<D>(row_slot(a.grad_g, a.part, row, row_lo, row_hi, k0, k1, tm.task, D * C2, tm.cp), C2, acc);
 }
 
 
@@ -371,7 +375,9 @@ __global__ void __launch_bounds__(kThreads) etp_dd_src_kernel(Args a) {
     for (int q = k0; q < k1; ++q) {
         while (q >= row_hi && row < a.N - 1) {
             if (row_hi > max(row_lo, k0)) {
-                if (a.grad_x) flush_row<D>(a.grad_x + (size_t)row * D * C2 + tm.cp, C2, gx, row_lo >= k0);
+                if (a.grad_x)
+                    store_row<D>(row_slot(a.grad_x, a.part, row, row_lo, row_hi, k0, k1, tm.task, D * C2, tm.cp), C2,
+                                 gx);
 #pragma unroll
                 for (int k = 0; k < D; ++k) gx[k] = f2_zero();
             }
@@ -590,7 +596,8 @@ __global__ void __launch_bounds__(kThreads) etp_dd_src_kernel(Args a) {
             }
         }
     }
-    if (a.grad_x) flush_row<D>(a.grad_x + (size_t)row * D * C2 + tm.cp, C2, gx, row_lo >= k0 && row_hi <= k1);
+    if (a.grad_x)
+        store_row<D>(row_slot(a.grad_x, a.part, row, row_lo, row_hi, k0, k1, tm.task, D * C2, tm.cp), C2, gx);
 }
 
 template <int L, bool O3>
@@ -606,44 +613,49 @@ size_t smem_for(bool src_side, int T) {
 // host side
 namespace {
 
+// Tasks of the destination-side (src_side false) or source-side kernel: one wave,
+// at least 16 edges each, no more tasks than rows (as in the first-order kernels).
 template <int L, bool O3>
-cudaError_t launch_dd(dd::Args a, cudaStream_t s) {
-    const int T = a.team;
-    const size_t sm_dst = dd::smem_for<L, O3>(false, T), sm_src = dd::smem_for<L, O3>(true, T);
-    const void* kd = (const void*)dd::etp_dd_dst_kernel<L, O3>;
-    const void* ks = (const void*)dd::etp_dd_src_kernel<L, O3>;
-    cudaError_t err;
-    if ((err = cudaFuncSetAttribute(ks, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_src)) != cudaSuccess)
-        return err;
-    if ((err = cudaFuncSetAttribute(kd, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_dst)) != cudaSuccess)
-        return err;
-    int dev = 0, sms = 1, bps_d = 1, bps_s = 1;
-    if ((err = cudaGetDevice(&dev)) != cudaSuccess) return err;
-    if ((err = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return err;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&bps_d, kd, dd::kThreads, sm_dst) != cudaSuccess || bps_d < 1)
-        bps_d = 1;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&bps_s, ks, dd::kThreads, sm_src) != cudaSuccess || bps_s < 1)
-        bps_s = 1;
+int dd_tasks(int C, int N, int E, bool src_side) {
+    const int T = C / 2 < 32 ? C / 2 : 32, slices = C / (2 * T);
+    const size_t sm = dd::smem_for<L, O3>(src_side, T);
+    const void* k = src_side ? (const void*)dd::etp_dd_src_kernel<L, O3> : (const void*)dd::etp_dd_dst_kernel<L, O3>;
+    cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    int dev = 0, sms = 1, bps = 1;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) !=
+                                                   cudaSuccess || sms < 1)
+        sms = 1;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&bps, k, dd::kThreads, sm) != cudaSuccess || bps < 1) bps = 1;
+    const long long cap = (long long)sms * bps * (dd::kThreads / T) / slices;
+    long long want = ((long long)E + 15) / 16;
+    if (want > N) want = N;
+    const long long nt = want < cap ? want : cap;
+    return (int)(nt < 1 ? 1 : nt);
+}
+
+template <int L, bool O3>
+cudaError_t launch_dd(dd::Args a, size_t part_bytes, cudaStream_t s) {
+    const int T = a.team, C = 2 * a.C2, D = (L + 1) * (L + 1);
     const int teams_per_block = dd::kThreads / T;
-    auto tasks_for = [&](int bps) {
-        long long cap = (long long)sms * bps * teams_per_block / a.slices;
-        long long want = ((long long)a.E + 15) / 16;
-        if (want > a.N) want = a.N;
-        long long nt = want < cap ? want : cap;
-        return (int)(nt < 1 ? 1 : nt);
-    };
+    cudaError_t err;
     void* args[] = {&a};
-    if (a.grad_g) {
-        a.ntasks = tasks_for(bps_d);
+    for (int side = 0; side < 2; ++side) {
+        float2* rows = side ? a.grad_x : a.grad_g;
+        if (side ? !(a.grad_x || a.grad_w || a.grad_r) : !a.grad_g) continue;
+        a.ntasks = dd_tasks<L, O3>(C, a.N, a.E, side != 0);
+        if (rows && part_bytes < partial_rows_bytes(a.ntasks, D, C)) return cudaErrorInvalidValue;
+        const size_t sm = dd::smem_for<L, O3>(side != 0, T);
+        const void* k = side ? (const void*)dd::etp_dd_src_kernel<L, O3> : (const void*)dd::etp_dd_dst_kernel<L, O3>;
+        if ((err = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm)) != cudaSuccess)
+            return err;
         const long long teams = (long long)a.ntasks * a.slices;
         const unsigned blocks = (unsigned)((teams + teams_per_block - 1) / teams_per_block);
-        if ((err = cudaLaunchKernel(kd, dim3(blocks), dim3(dd::kThreads), args, sm_dst, s)) != cudaSuccess) return err;
-    }
-    if (a.grad_x || a.grad_w || a.grad_r) {
-        a.ntasks = tasks_for(bps_s);
-        const long long teams = (long long)a.ntasks * a.slices;
-        const unsigned blocks = (unsigned)((teams + teams_per_block - 1) / teams_per_block);
-        if ((err = cudaLaunchKernel(ks, dim3(blocks), dim3(dd::kThreads), args, sm_src, s)) != cudaSuccess) return err;
+        if ((err = cudaLaunchKernel(k, dim3(blocks), dim3(dd::kThreads), args, sm, s)) != cudaSuccess) return err;
+        if (rows &&
+            (err = launch_combine_rows(side ? a.rev_ptr : a.row_ptr, nullptr, a.N, a.E, a.ntasks, D * C / 4,
+                                       reinterpret_cast<const float4*>(a.part), reinterpret_cast<float4*>(rows), s)) !=
+                cudaSuccess)
+            return err;
     }
     return cudaSuccess;
 }
@@ -654,16 +666,20 @@ cudaError_t double_backward(int L, bool o3, int C, int N, int E, const int32_t* 
                             const int32_t* rev_ptr, const int32_t* rev_perm, const int32_t* dst, const float* r,
                             const float* x, const float* w, const float* g, const float* gg_x, const float* gg_w,
                             const float* gg_r, float* grad_g, float* grad_x, float* grad_w, float* grad_r,
-                            cudaStream_t s) {
+                            void* part, size_t part_bytes, cudaStream_t s) {
     const int D = (L + 1) * (L + 1);
     cudaError_t err;
-    // rows cut by a task boundary (and, with two channel slices, grad_r) are added onto zeros
-    if (grad_g && (err = cudaMemsetAsync(grad_g, 0, sizeof(float) * (size_t)N * D * C, s)) != cudaSuccess) return err;
-    if (grad_x && (err = cudaMemsetAsync(grad_x, 0, sizeof(float) * (size_t)N * D * C, s)) != cudaSuccess) return err;
     const int team = C / 2 < 32 ? C / 2 : 32, slices = C / (2 * team);
+    // with two channel slices, grad_r is the sum of the slices' two terms (added onto zero: order-free)
     if (grad_r && slices > 1 && (err = cudaMemsetAsync(grad_r, 0, sizeof(float) * 3 * (size_t)E, s)) != cudaSuccess)
         return err;
-    if (E == 0) return cudaSuccess;
+    if (E == 0) {
+        if (grad_g && (err = cudaMemsetAsync(grad_g, 0, sizeof(float) * (size_t)N * D * C, s)) != cudaSuccess)
+            return err;
+        if (grad_x && (err = cudaMemsetAsync(grad_x, 0, sizeof(float) * (size_t)N * D * C, s)) != cudaSuccess)
+            return err;
+        return cudaSuccess;
+    }
     dd::Args a{N,
                E,
                row_ptr,
@@ -685,17 +701,34 @@ cudaError_t double_backward(int L, bool o3, int C, int N, int E, const int32_t* 
                C / 2,
                team,
                slices,
-               1};
+               1,
+               static_cast<float2*>(part)};
     switch (L * 2 + (o3 ? 1 : 0)) {
-        case 0: return launch_dd<0, false>(a, s);
-        case 1: return launch_dd<0, true>(a, s);
-        case 2: return launch_dd<1, false>(a, s);
-        case 3: return launch_dd<1, true>(a, s);
-        case 4: return launch_dd<2, false>(a, s);
-        case 5: return launch_dd<2, true>(a, s);
-        case 6: return launch_dd<3, false>(a, s);
-        default: return launch_dd<3, true>(a, s);
+        case 0: return launch_dd<0, false>(a, part_bytes, s);
+        case 1: return launch_dd<0, true>(a, part_bytes, s);
+        case 2: return launch_dd<1, false>(a, part_bytes, s);
+        case 3: return launch_dd<1, true>(a, part_bytes, s);
+        case 4: return launch_dd<2, false>(a, part_bytes, s);
+        case 5: return launch_dd<2, true>(a, part_bytes, s);
+        case 6: return launch_dd<3, false>(a, part_bytes, s);
+        default: return launch_dd<3, true>(a, part_bytes, s);
     }
+}
+
+size_t double_backward_partial_bytes(int L, bool o3, int C, int N, int E) {
+    if (E <= 0 || N <= 0) return 0;
+    int nd = 1, ns = 1;
+    switch (L * 2 + (o3 ? 1 : 0)) {
+        case 0: nd = dd_tasks<0, false>(C, N, E, false), ns = dd_tasks<0, false>(C, N, E, true); break;
+        case 1: nd = dd_tasks<0, true>(C, N, E, false), ns = dd_tasks<0, true>(C, N, E, true); break;
+        case 2: nd = dd_tasks<1, false>(C, N, E, false), ns = dd_tasks<1, false>(C, N, E, true); break;
+        case 3: nd = dd_tasks<1, true>(C, N, E, false), ns = dd_tasks<1, true>(C, N, E, true); break;
+        case 4: nd = dd_tasks<2, false>(C, N, E, false), ns = dd_tasks<2, false>(C, N, E, true); break;
+        case 5: nd = dd_tasks<2, true>(C, N, E, false), ns = dd_tasks<2, true>(C, N, E, true); break;
+        case 6: nd = dd_tasks<3, false>(C, N, E, false), ns = dd_tasks<3, false>(C, N, E, true); break;
+        default: nd = dd_tasks<3, true>(C, N, E, false), ns = dd_tasks<3, true>(C, N, E, true); break;
+    }
+    return partial_rows_bytes(nd > ns ? nd : ns, (L + 1) * (L + 1), C);
 }
 
 }  // namespace etp

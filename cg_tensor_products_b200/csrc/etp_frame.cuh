@@ -525,21 +525,23 @@ __device__ __forceinline__ int segment_of(const int32_t* __restrict__ ptr, int n
     return lo;
 }
 
-__device__ __forceinline__ void red_add2(float2* p, float2 v) {
-    asm volatile("red.global.add.v2.f32 [%0], {%1, %2};" ::"l"(p), "f"(v.x), "f"(v.y) : "memory");
+
+// One finished row of a task, stored with plain stores: into the output when the
+// task holds all of the row's positions, else into the task's slot of the
+// partial-row buffer (slot 0: the row began before the task; slot 1: it goes on
+// past it). etp_combine_rows_kernel then sums each cut row's pieces in task order.
+template <int D>
+__device__ __forceinline__ void store_row(float2* dst, int C2, const float2 (&acc)[D]) {
+#pragma unroll
+    for (int k = 0; k < D; ++k) dst[k * C2] = acc[k];
 }
 
-// Store a row accumulator: plainly when the task owns the whole row, else by
-// vector reduction onto the zeroed output.
-template <int D>
-__device__ __forceinline__ void flush_row(float2* row, int C2, const float2 (&acc)[D], bool whole) {
-#pragma unroll
-    for (int k = 0; k < D; ++k) {
-        if (whole)
-            row[k * C2] = acc[k];
-        else
-            red_add2(row + k * C2, acc[k]);
-    }
+// Where a task's finished row [lo, hi) of positions goes (this lane's channel
+// pair): the output row, or the task's partial slot.
+__device__ __forceinline__ float2* row_slot(float2* rows, float2* part, int node, int lo, int hi, int k0, int k1,
+                                            int task, int DC2, int cp) {
+    if (lo >= k0 && hi <= k1) return rows + (size_t)node * DC2 + cp;
+    return part + ((size_t)task * 2 + (lo < k0 ? 0 : 1)) * DC2 + cp;
 }
 
 // The fitting points and inverses as one constant-memory table, built at
@@ -716,6 +718,7 @@ __global__ void __launch_bounds__(frame::kThreads, 4) etp_fwd_frame_kernel(FwdAr
     const bool producer = G.slice == 0 && G.tl == 0;
     const int cp = G.slice * G.T + G.tl;
     float2* out2 = reinterpret_cast<float2*>(a.out);
+    float2* part2 = reinterpret_cast<float2*>(a.part);
     auto group_sync = [&] {
         if (G.S == 2)
             __syncthreads();  // the block is exactly this task's two warps
@@ -769,7 +772,7 @@ __global__ void __launch_bounds__(frame::kThreads, 4) etp_fwd_frame_kernel(FwdAr
     for (int q = k0, it = 0; q < k1; ++q, ++it) {
         while (q >= row_hi && row < a.N - 1) {  // the edge opens a later row: store the finished one
             if (row_hi > max(row_lo, k0)) {
-                flush_row<D>(out2 + (size_t)node * D * C2 + cp, C2, acc, row_lo >= k0);
+                store_row<D>(row_slot(out2, part2, node, row_lo, row_hi, k0, k1, G.task, D * C2, cp), C2, acc);
 #pragma unroll
                 for (int k = 0; k < D; ++k) acc[k] = f2_zero();
             }
@@ -837,7 +840,7 @@ __global__ void __launch_bounds__(frame::kThreads, 4) etp_fwd_frame_kernel(FwdAr
         e_next2 = e_next3;
         r_cur = r_next;
     }
-    flush_row<D>(out2 + (size_t)node * D * C2 + cp, C2, acc, row_lo >= k0 && row_hi <= k1);
+    store_row<D>(row_slot(out2, part2, node, row_lo, row_hi, k0, k1, G.task, D * C2, cp), C2, acc);
 }
 
 // ===========================================================================
@@ -876,6 +879,7 @@ __global__ void __launch_bounds__(frame::kThreads, L <= 2 ? 6 : 4) etp_bwd_frame
     const uint64_t pol_w = l2_evict_first_policy();
     float2* gw2 = reinterpret_cast<float2*>(a.grad_w);
     float2* gx2 = reinterpret_cast<float2*>(a.grad_x);
+    float2* part2 = reinterpret_cast<float2*>(a.part);
     const bool want_w = a.grad_w != nullptr;
     const bool want_r = a.grad_r != nullptr;
     auto group_sync = [&] {
@@ -950,7 +954,7 @@ __global__ void __launch_bounds__(frame::kThreads, L <= 2 ? 6 : 4) etp_bwd_frame
     for (int q = k0, it = 0; q < k1; ++q, ++it) {
         while (q >= row_hi && row < a.N - 1) {  // the position opens a later source row: store the finished one
             if (row_hi > max(row_lo, k0)) {
-                if (gx2) flush_row<D>(gx2 + (size_t)node * D * C2 + cp, C2, gx, row_lo >= k0);
+                if (gx2) store_row<D>(row_slot(gx2, part2, node, row_lo, row_hi, k0, k1, G.task, D * C2, cp), C2, gx);
 #pragma unroll
                 for (int k = 0; k < D; ++k) gx[k] = f2_zero();
             }
@@ -1127,7 +1131,7 @@ __global__ void __launch_bounds__(frame::kThreads, L <= 2 ? 6 : 4) etp_bwd_frame
         r_cur = r_next;
     }
     cp_async_wait_all();
-    if (gx2) flush_row<D>(gx2 + (size_t)node * D * C2 + cp, C2, gx, row_lo >= k0 && row_hi <= k1);
+    if (gx2) store_row<D>(row_slot(gx2, part2, node, row_lo, row_hi, k0, k1, G.task, D * C2, cp), C2, gx);
 }
 
 namespace frame {

@@ -25,6 +25,7 @@ struct FwdArgs {
     int ntasks;  // equal contiguous ranges of positions
     const int32_t* order;     // may be null: row rank -> destination node (locality order)
     const int32_t* pos_edge;  // may be null: position -> edge (the ranks' rows in sequence)
+    float4* part;             // partial rows [ntasks][2][D][C] of rows cut by task boundaries
 };
 
 struct BwdArgs {
@@ -47,6 +48,7 @@ struct BwdArgs {
     int slices;
     int ntasks;
     const int32_t* order;  // may be null: source row rank -> node (rev_ptr is then over ranks)
+    float4* part;          // partial rows [ntasks][2][D][C] of grad_x rows cut by task boundaries
 };
 
 // Launch geometry shared by the forward and backward kernels: teams of
@@ -72,6 +74,12 @@ template <int L>
 cudaError_t launch_backward(bool o3, const BwdArgs& a, dim3 grid, size_t smem, cudaStream_t s);
 template <int L>
 cudaError_t launch_edge_frames(int E, const float* r, float* frames, cudaStream_t s);
+// The second pass of the segment sums (rows cut by task boundaries, rows without
+// positions) over rows of row4 float4s; ptr: the CSR pointer the tasks ran over.
+cudaError_t launch_combine_rows(const int32_t* ptr, const int32_t* order, int N, int E, int ntasks, int row4,
+                                const float4* part, float4* rows, cudaStream_t s);
+// Bytes of the partial-row buffer of one launch shape.
+inline size_t partial_rows_bytes(int ntasks, int D, int C) { return 2 * (size_t)ntasks * D * C * sizeof(float); }
 
 // Reverse CSR workspace. Up to kOnePassMaxNodes sources (and a bounded table)
 // the grouping is one stable counting pass over a (source, tile) count table;
@@ -145,13 +153,17 @@ cudaError_t double_backward(int L, bool o3, int C, int N, int E, const int32_t* 
                             const int32_t* rev_ptr, const int32_t* rev_perm, const int32_t* dst, const float* r,
                             const float* x, const float* w, const float* g, const float* gg_x, const float* gg_w,
                             const float* gg_r, float* grad_g, float* grad_x, float* grad_w, float* grad_r,
-                            cudaStream_t s);
+                            void* part, size_t part_bytes, cudaStream_t s);
+size_t double_backward_partial_bytes(int L, bool o3, int C, int N, int E);
 // Cartesian edge convolution (etp_cart.cu): features in independent STF components.
 cudaError_t cart_forward(int L, bool o3, int C, int N, int E, const int32_t* row_ptr, const int32_t* src,
-                         const float* r, const float* x, const float* w, float* out, cudaStream_t s);
+                         const float* r, const float* x, const float* w, float* out, void* part, size_t part_bytes,
+                         cudaStream_t s);
 cudaError_t cart_backward(int L, bool o3, int C, int N, int E, const int32_t* row_ptr, const int32_t* rev_ptr,
                           const int32_t* rev_perm, const int32_t* dst, const float* r, const float* x, const float* w,
-                          const float* g, float* grad_x, float* grad_w, float* grad_r, cudaStream_t s);
+                          const float* g, float* grad_x, float* grad_w, float* grad_r, void* part, size_t part_bytes,
+                          cudaStream_t s);
+size_t cart_partial_bytes(int L, bool o3, int C, int N, int E);
 cudaError_t assemble_forces(int N, int E, const int32_t* row_ptr, const int32_t* rev_ptr, const int32_t* rev_perm,
                             const float* r, const float* grad_r, float* forces, float* virial, cudaStream_t s);
 cudaError_t validate_csr(int N, int E, const int32_t* row_ptr, const int32_t* src, int32_t* flag, cudaStream_t s);

@@ -16,6 +16,51 @@ int log2i(int t) {
     return k;
 }
 
+// Second pass of the segment sums, after the forward or backward kernel on the
+// same stream. (1) A row cut by task boundaries is stored by the block of the
+// task where it begins: the sum, in task order, of that task's slot 1 and the
+// slot 0 of each following task up to the one where the row ends. (2) Rows
+// without positions are zeroed, one warp per row. Every output row is thus
+// written exactly once, in a fixed order: no atomics, bitwise repeatable.
+__global__ void __launch_bounds__(256) etp_combine_rows_kernel(const int32_t* __restrict__ ptr,
+                                                               const int32_t* __restrict__ order, int N, int E,
+                                                               int ntasks, int row4, const float4* __restrict__ part,
+                                                               float4* __restrict__ rows) {
+    for (int t = blockIdx.x; t < ntasks; t += gridDim.x) {
+        int k0, k1;
+        frame::task_range(E, t, ntasks, k0, k1);
+        if (k0 >= k1) continue;
+        const int R = frame::segment_of(ptr, N, k1 - 1);
+        const int lo = __ldg(ptr + R), hi = __ldg(ptr + R + 1);
+        if (!(hi > k1 && lo >= k0)) continue;  // the task's last row ends in it, or began before it
+        const int node = order ? __ldg(order + R) : R;
+        for (int f = threadIdx.x; f < row4; f += blockDim.x) {
+            float4 acc = part[((size_t)t * 2 + 1) * row4 + f];
+            for (int u = t + 1; u < ntasks; ++u) {
+                int u0, u1;
+                frame::task_range(E, u, ntasks, u0, u1);
+                if (u0 >= hi) break;
+                if (u0 < u1) {
+                    const float4 v = part[(size_t)u * 2 * row4 + f];
+                    acc.x += v.x;
+                    acc.y += v.y;
+                    acc.z += v.z;
+                    acc.w += v.w;
+                }
+                if (u1 >= hi) break;
+            }
+            rows[(size_t)node * row4 + f] = acc;
+        }
+    }
+    const int lane = threadIdx.x & 31;
+    const int warps = gridDim.x * (blockDim.x >> 5);
+    for (int j = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); j < N; j += warps) {
+        if (__ldg(ptr + j + 1) > __ldg(ptr + j)) continue;
+        float4* dst = rows + (size_t)(order ? __ldg(order + j) : j) * row4;
+        for (int f = lane; f < row4; f += 32) dst[f] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+}
+
 }  // namespace
 
 LaunchShape launch_shape(int C, int L, bool o3, bool backward, bool framed, int E, int N, int waves) {
@@ -58,6 +103,16 @@ LaunchShape launch_shape(int C, int L, bool o3, bool backward, bool framed, int 
     s.ntasks = (int)(nt < 1 ? 1 : nt);
     s.grid = dim3((unsigned)((s.ntasks + s.tasks_per_block - 1) / s.tasks_per_block), 1, 1);
     return s;
+}
+
+cudaError_t launch_combine_rows(const int32_t* ptr, const int32_t* order, int N, int E, int ntasks, int row4,
+                                const float4* part, float4* rows, cudaStream_t s) {
+    int blocks = ntasks;
+    const int row_blocks = (N + 7) / 8;  // eight warps per block, one row each
+    if (blocks < row_blocks) blocks = row_blocks < 4 * 148 ? row_blocks : 4 * 148;
+    if (blocks < 1) blocks = 1;
+    etp_combine_rows_kernel<<<blocks, 256, 0, s>>>(ptr, order, N, E, ntasks, row4, part, rows);
+    return cudaGetLastError();
 }
 
 }  // namespace etp

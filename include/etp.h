@@ -150,15 +150,30 @@ ETP_API etp_status etp_edge_frames(etp_plan_t plan, int E, const float* r, float
  * records from HBM: 440 MB at 1.25 M edges). Host only. */
 ETP_API etp_status etp_plan_frames_advised(etp_plan_t plan, int E, int* use_records);
 
+/* Bytes of device workspace the tensor-product calls need for this plan and graph
+ * size: etp_forward, etp_backward, etp_double_backward, etp_cart_forward and
+ * etp_cart_backward (ordered = 0), and with ordered = 1 also etp_forward_ordered
+ * and etp_backward_ordered; with or without frame records. Host only; it reads
+ * the current device's multiprocessor count and the kernels' occupancy. 0 when
+ * E = 0. */
+ETP_API etp_status etp_tp_workspace_size(etp_plan_t plan, int N, int E, int ordered, size_t* bytes);
+
 /* Forward: out[i] = sum_{e in row i} msg_e (see above), for all N rows.
  * x: [N][D][C], w: [E][P][C], r: [E][3], out: [N][D][C] device pointers.
  * frames: NULL (the kernel builds each edge's frame from r), or the records
  * etp_edge_frames wrote for this r and plan's L (then r is not read and may be
  * NULL). N >= 0, E >= 0; with N = 0 nothing is launched; with E = 0 out is
- * zeroed. */
+ * zeroed.
+ * Segment sums without atomics: the edges are split into equal contiguous tasks;
+ * each row is summed in registers in edge order and stored once. A row cut by task
+ * boundaries leaves one partial row per task in `workspace` (at least
+ * etp_tp_workspace_size bytes, 16-byte aligned, owned by the caller; may be NULL
+ * when E = 0), and a second launch on the same stream adds them up in task order
+ * and zeroes the rows without edges. Every output is written once, in a fixed
+ * order: results repeat bit for bit. */
 ETP_API etp_status etp_forward(etp_plan_t plan, int N, int E, const int32_t* row_ptr, const int32_t* src,
                        const float* r, const float* frames, const float* x, const float* w, float* out,
-                       etp_stream_t stream);
+                       void* workspace, size_t workspace_bytes, etp_stream_t stream);
 
 /* Vector-Jacobian product for the cotangent grad_out = dLoss/d(out), [N][D][C]:
  *   grad_x[j, l1 m1, c] = sum_{e: src e = j} sum_p w[e,p,c] sum_{m2,m3} CG_p Y_{l2 m2}(r_e) grad_out[dst e, l3 m3, c]
@@ -170,12 +185,15 @@ ETP_API etp_status etp_forward(etp_plan_t plan, int N, int E, const int32_t* row
  * frames, r is not read and may be NULL). Each of grad_x, grad_w, grad_r may be
  * NULL to skip it. All outputs are overwritten (sources without edges get zero
  * grad_x). An edge whose source or row is out of range (a CSR that
- * etp_validate_csr flags) adds nothing to grad_x and gets zero grad_w and grad_r. */
+ * etp_validate_csr flags) adds nothing to grad_x and gets zero grad_w and grad_r.
+ * workspace: as in etp_forward, for the source rows of grad_x (may be NULL when
+ * grad_x is NULL or E = 0); grad_x is summed without atomics and repeats bit for
+ * bit, like out. */
 ETP_API etp_status etp_backward(etp_plan_t plan, int N, int E, const int32_t* row_ptr, const int32_t* src,
                         const int32_t* rev_ptr, const int32_t* rev_perm, const int32_t* dst_of_edge,
                         const float* r, const float* frames, const float* x, const float* w,
                         const float* grad_out, float* grad_x, float* grad_w, float* grad_r,
-                        etp_stream_t stream);
+                        void* workspace, size_t workspace_bytes, etp_stream_t stream);
 
 /* VJP of the VJP (double backward). With (grad_x, grad_w, grad_r) = etp_backward's
  * outputs for (x, w, r; grad_out) and cotangents gg_x [N][D][C], gg_w [E][P][C],
@@ -191,15 +209,18 @@ ETP_API etp_status etp_backward(etp_plan_t plan, int N, int E, const int32_t* ro
  * overwritten (nodes without edges get zeros). Graph arguments as in etp_backward
  * (rev_ptr, rev_perm from etp_build_reverse_csr; dst_of_edge may be NULL). r is
  * always read. Edges shorter than 1e-12 have no direction: only the (l, 0, l)
- * paths act and every derivative in r is zero there. Allocates nothing; node sums
- * in a fixed order, except rows cut by a task boundary (added onto the zeroed
- * output) and, for C = 128, grad_r (two channel halves added onto zeros). */
+ * paths act and every derivative in r is zero there. Allocates nothing. Node sums
+ * as in etp_forward: rows cut by a task boundary leave partial rows in `workspace`
+ * (etp_tp_workspace_size bytes; may be NULL when neither grad_grad_out nor grad_x
+ * is wanted, or E = 0), summed in task order by a second launch; for C = 128,
+ * grad_r is the sum of two channel halves added onto zero (exact in either order).
+ * Results repeat bit for bit. */
 ETP_API etp_status etp_double_backward(etp_plan_t plan, int N, int E, const int32_t* row_ptr, const int32_t* src,
                                        const int32_t* rev_ptr, const int32_t* rev_perm, const int32_t* dst_of_edge,
                                        const float* r, const float* x, const float* w, const float* grad_out,
                                        const float* gg_x, const float* gg_w, const float* gg_r,
                                        float* grad_grad_out, float* grad_x, float* grad_w, float* grad_r,
-                                       etp_stream_t stream);
+                                       void* workspace, size_t workspace_bytes, etp_stream_t stream);
 
 /* Cartesian edge convolution: the same edge tensor product with Cartesian
  * couplings ("FlashCart 如何让等变原子间势更快更准?", sections "FlashCart 用笛卡尔内核替
@@ -218,15 +239,17 @@ ETP_API etp_status etp_double_backward(etp_plan_t plan, int N, int E, const int3
  *   out[i] = sum over row i of sum_p w[e,p,:] coupling_p(x[src e], attribute_l2(r_e)).
  * The couplings are compile-time sparse tables of explicit sums; the pages give no
  * formula, so these are this library's reading. Arguments, layouts, ownership and
- * errors as etp_forward / etp_backward (no frame records); the VJP writes grad_x
- * (sources without edges: zero), grad_w and grad_r (derivative through the edge
- * attribute), each optional. */
+ * errors as etp_forward / etp_backward (no frame records; the same workspace); the
+ * VJP writes grad_x (sources without edges: zero), grad_w and grad_r (derivative
+ * through the edge attribute), each optional. */
 ETP_API etp_status etp_cart_forward(etp_plan_t plan, int N, int E, const int32_t* row_ptr, const int32_t* src,
-                                    const float* r, const float* x, const float* w, float* out, etp_stream_t stream);
+                                    const float* r, const float* x, const float* w, float* out, void* workspace,
+                                    size_t workspace_bytes, etp_stream_t stream);
 ETP_API etp_status etp_cart_backward(etp_plan_t plan, int N, int E, const int32_t* row_ptr, const int32_t* src,
                                      const int32_t* rev_ptr, const int32_t* rev_perm, const int32_t* dst_of_edge,
                                      const float* r, const float* x, const float* w, const float* grad_out,
-                                     float* grad_x, float* grad_w, float* grad_r, etp_stream_t stream);
+                                     float* grad_x, float* grad_w, float* grad_r, void* workspace,
+                                     size_t workspace_bytes, etp_stream_t stream);
 
 /* Radial weights: the tensor product's per-edge weights as a function of the edge
  * length. The pages make these weights a learned function of |r| ("High-performance
@@ -319,7 +342,8 @@ ETP_API etp_status etp_build_reverse_csr(int N, int E, const int32_t* row_ptr, c
  * nodes and splits the work into several waves of tasks, so that the tasks in
  * flight at any time hold nearby rows and share their neighbours' rows in L2.
  * Results are the same as etp_forward's and etp_backward's up to the rounding of
- * rows cut by a task boundary. The pages measure on spatially coherent systems
+ * rows cut by a task boundary (the two split the edges differently); each repeats
+ * bit for bit. The pages measure on spatially coherent systems
  * ("FlashCart 如何让等变原子间势更快更准?", section "FlashCart 用笛卡尔内核替代球谐耦合":
  * the speed comes from memory access and the aggregation of edge contributions);
  * the schedule is this library's way to keep those accesses local when the ids
@@ -357,7 +381,7 @@ ETP_API etp_status etp_build_locality_schedule(int N, int E, const int32_t* row_
 ETP_API etp_status etp_forward_ordered(etp_plan_t plan, int N, int E, const int32_t* order, const int32_t* ord_ptr,
                                        const int32_t* ord_edge, const int32_t* src, const float* r,
                                        const float* frames, const float* x, const float* w, float* out,
-                                       etp_stream_t stream);
+                                       void* workspace, size_t workspace_bytes, etp_stream_t stream);
 
 /* etp_backward on a locality schedule: the same outputs, with the sources visited
  * in the schedule's order. order, rev_ptr, rev_perm, dst_of_edge: as written by
@@ -367,7 +391,8 @@ ETP_API etp_status etp_backward_ordered(etp_plan_t plan, int N, int E, const int
                                         const int32_t* rev_ptr, const int32_t* rev_perm,
                                         const int32_t* dst_of_edge, const float* r, const float* frames,
                                         const float* x, const float* w, const float* grad_out, float* grad_x,
-                                        float* grad_w, float* grad_r, etp_stream_t stream);
+                                        float* grad_w, float* grad_r, void* workspace, size_t workspace_bytes,
+                                        etp_stream_t stream);
 
 /* Limits of etp_build_reverse_csr_static and the size of its scratch array. */
 #define ETP_STATIC_MAX_NODES (1 << 18)

@@ -36,7 +36,7 @@ static int host_checks(void) {
     CHECK(P == 34 && din == 16 && dsh == 16 && dout == 16, "plan shape");
     ETP(etp_plan_couplings(plan, &nnz, NULL, NULL, NULL, NULL, NULL));
     CHECK(nnz > 0, "coupling count");
-    CHECK(etp_forward(plan, -1, 0, NULL, NULL, NULL, NULL, NULL, NULL, NULL, NULL) == ETP_ERR_INVALID_ARG,
+    CHECK(etp_forward(plan, -1, 0, NULL, NULL, NULL, NULL, NULL, NULL, NULL, NULL, 0, NULL) == ETP_ERR_INVALID_ARG,
           "negative N rejected");
     CHECK(etp_edge_frames(NULL, 4, NULL, NULL, NULL) == ETP_ERR_INVALID_ARG, "NULL plan rejected");
     etp_plan_t bad = NULL;
@@ -123,6 +123,9 @@ static int run(const char* in, const char* out_path) {
     void* d_ws;
     size_t ws_bytes = 0;
     ETP(etp_reverse_csr_workspace_size(N, E, &ws_bytes));
+    size_t tp_bytes = 0;
+    ETP(etp_tp_workspace_size(plan, N, E, 0, &tp_bytes));
+    if (tp_bytes > ws_bytes) ws_bytes = tp_bytes; /* one workspace, used by one call at a time on one stream */
     CUDA(cudaMalloc((void**)&d_out, 4 * nd));
     CUDA(cudaMalloc((void**)&d_gx, 4 * nd));
     CUDA(cudaMalloc((void**)&d_gw, 4 * ew + 16));
@@ -140,9 +143,9 @@ static int run(const char* in, const char* out_path) {
     ETP(etp_validate_csr(N, E, d_row_ptr, d_src, d_flag, es));
     ETP(etp_build_reverse_csr(N, E, d_row_ptr, d_src, d_rev_ptr, d_rev_perm, d_dst, d_ws, ws_bytes, es));
     ETP(etp_edge_frames(plan, E, d_r, d_frames, es));
-    ETP(etp_forward(plan, N, E, d_row_ptr, d_src, NULL, d_frames, d_x, d_w, d_out, es));
+    ETP(etp_forward(plan, N, E, d_row_ptr, d_src, NULL, d_frames, d_x, d_w, d_out, d_ws, ws_bytes, es));
     ETP(etp_backward(plan, N, E, d_row_ptr, d_src, d_rev_ptr, d_rev_perm, d_dst, NULL, d_frames, d_x, d_w, d_g,
-                     d_gx, d_gw, d_gr, es));
+                     d_gx, d_gw, d_gr, d_ws, ws_bytes, es));
     ETP(etp_assemble_forces(N, E, d_row_ptr, d_rev_ptr, d_rev_perm, NULL, d_gr, d_forces, NULL, es));
     CUDA(cudaStreamSynchronize(s));
     int flag = -1, fault = -1;

@@ -89,3 +89,18 @@ def check_reverse_csr(wl, res):
     assert np.array_equal(res["rev_perm"].cpu().numpy(), o_perm)
     if res["dst"] is not None:
         assert np.array_equal(res["dst"].cpu().numpy(), o_dst)
+
+
+def hub_workload(rng, L, C, P, n=64, hub=20000, rest=3000):
+    """A destination with `hub` edges and a source with `hub` edges among n nodes: with
+    equal edge ranges per task both hub rows are cut across many tasks."""
+    from workloads import Workload, csr_from_pairs
+
+    dst = np.concatenate([np.zeros(hub, np.int64), rng.integers(0, n, hub), rng.integers(0, n, rest)])
+    src = np.concatenate([rng.integers(0, n, hub), np.ones(hub, np.int64), rng.integers(0, n, rest)])
+    row_ptr, s, _ = csr_from_pairs(n, dst, src)
+    E, D = len(s), (L + 1) ** 2
+    return Workload("hubs", L, C, P, row_ptr, s, rng.standard_normal((E, 3), dtype=np.float32),
+                    rng.standard_normal((n, D, C), dtype=np.float32),
+                    rng.standard_normal((E, P, C), dtype=np.float32) / np.float32(np.sqrt(P)),
+                    rng.standard_normal((n, D, C), dtype=np.float32))

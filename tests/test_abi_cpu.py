@@ -23,7 +23,7 @@ def lib():
 
 def test_exports_every_declared_symbol(lib):
     names = etp.declared_symbols()
-    assert len(names) == 27
+    assert len(names) == 28
     for n in names:
         assert hasattr(lib, n), n
 
@@ -83,27 +83,35 @@ def test_host_argument_checks(lib):
     ok = ctypes.c_void_p(0x10000)       # never dereferenced: each call fails a host check
     bad = ctypes.c_void_p(0x10004)      # not 16-byte aligned
     F = lib.etp_forward
-    assert F(None, 4, 4, ok, ok, ok, None, ok, ok, ok, None) == etp.ETP_ERR_INVALID_ARG       # no plan
-    assert F(h, -1, 4, ok, ok, ok, None, ok, ok, ok, None) == etp.ETP_ERR_INVALID_ARG         # N < 0
-    assert F(h, 4, -2, ok, ok, ok, None, ok, ok, ok, None) == etp.ETP_ERR_INVALID_ARG         # E < 0
-    assert F(h, 0, 3, ok, ok, ok, None, ok, ok, ok, None) == etp.ETP_ERR_INVALID_ARG          # edges without nodes
-    assert F(h, 0, 0, None, None, None, None, None, None, None, None) == etp.ETP_OK           # nothing to do
-    assert F(h, 4, 4, None, ok, ok, None, ok, ok, ok, None) == etp.ETP_ERR_INVALID_ARG        # row_ptr NULL
-    assert F(h, 4, 4, ok, ok, ok, None, bad, ok, ok, None) == etp.ETP_ERR_INVALID_ARG         # x misaligned
-    assert F(h, 4, 4, ok, ok, ok, None, ok, bad, ok, None) == etp.ETP_ERR_INVALID_ARG         # w misaligned
-    assert F(h, 4, 4, ok, ok, ok, None, ok, ok, bad, None) == etp.ETP_ERR_INVALID_ARG         # out misaligned
-    assert F(h, 4, 4, ok, None, ok, None, ok, ok, ok, None) == etp.ETP_ERR_INVALID_ARG        # src NULL with E > 0
-    assert F(h, 4, 4, ok, ok, None, None, ok, ok, ok, None) == etp.ETP_ERR_INVALID_ARG     # neither r nor frames
-    assert F(h, 4, 4, ok, ok, None, bad, ok, ok, ok, None) == etp.ETP_ERR_INVALID_ARG      # frames misaligned
+    assert F(None, 4, 4, ok, ok, ok, None, ok, ok, ok, ok, 1 << 30, None) == etp.ETP_ERR_INVALID_ARG       # no plan
+    assert F(h, -1, 4, ok, ok, ok, None, ok, ok, ok, ok, 1 << 30, None) == etp.ETP_ERR_INVALID_ARG         # N < 0
+    assert F(h, 4, -2, ok, ok, ok, None, ok, ok, ok, ok, 1 << 30, None) == etp.ETP_ERR_INVALID_ARG         # E < 0
+    assert F(h, 0, 3, ok, ok, ok, None, ok, ok, ok, ok, 1 << 30, None) == etp.ETP_ERR_INVALID_ARG          # edges without nodes
+    assert F(h, 0, 0, None, None, None, None, None, None, None, ok, 1 << 30, None) == etp.ETP_OK           # nothing to do
+    assert F(h, 4, 4, None, ok, ok, None, ok, ok, ok, ok, 1 << 30, None) == etp.ETP_ERR_INVALID_ARG        # row_ptr NULL
+    assert F(h, 4, 4, ok, ok, ok, None, bad, ok, ok, ok, 1 << 30, None) == etp.ETP_ERR_INVALID_ARG         # x misaligned
+    assert F(h, 4, 4, ok, ok, ok, None, ok, bad, ok, ok, 1 << 30, None) == etp.ETP_ERR_INVALID_ARG         # w misaligned
+    assert F(h, 4, 4, ok, ok, ok, None, ok, ok, bad, ok, 1 << 30, None) == etp.ETP_ERR_INVALID_ARG         # out misaligned
+    assert F(h, 4, 4, ok, None, ok, None, ok, ok, ok, ok, 1 << 30, None) == etp.ETP_ERR_INVALID_ARG        # src NULL with E > 0
+    assert F(h, 4, 4, ok, ok, None, None, ok, ok, ok, ok, 1 << 30, None) == etp.ETP_ERR_INVALID_ARG     # neither r nor frames
+    assert F(h, 4, 4, ok, ok, None, bad, ok, ok, ok, ok, 1 << 30, None) == etp.ETP_ERR_INVALID_ARG      # frames misaligned
+    assert F(h, 4, 4, ok, ok, ok, None, ok, ok, ok, None, 1 << 30, None) == etp.ETP_ERR_INVALID_ARG  # no workspace
+    assert F(h, 4, 4, ok, ok, ok, None, ok, ok, ok, bad, 1 << 30, None) == etp.ETP_ERR_INVALID_ARG   # misaligned
+    assert F(h, 4, 4, ok, ok, ok, None, ok, ok, ok, ok, 0, None) == etp.ETP_ERR_WORKSPACE             # too small
     B = lib.etp_backward
-    assert B(h, 4, 4, ok, ok, None, ok, ok, ok, None, ok, ok, ok, ok, ok, ok, None) == etp.ETP_ERR_INVALID_ARG  # rev_ptr
-    assert B(h, 4, 4, ok, ok, ok, None, ok, ok, None, ok, ok, ok, ok, ok, ok, None) == etp.ETP_ERR_INVALID_ARG  # rev_perm
-    assert B(h, 4, 4, ok, ok, ok, ok, ok, ok, None, ok, ok, bad, ok, ok, ok, None) == etp.ETP_ERR_INVALID_ARG   # grad_out
-    assert B(h, 4, 4, ok, ok, ok, ok, ok, ok, None, ok, ok, ok, ok, bad, ok, None) == etp.ETP_ERR_INVALID_ARG   # grad_w
-    assert B(h, 4, 4, ok, ok, ok, ok, ok, ok, None, ok, ok, ok, bad, ok, ok, None) == etp.ETP_ERR_INVALID_ARG   # grad_x
-    assert B(h, 4, 4, ok, ok, ok, ok, ok, ok, None, ok, ok, ok, None, None, None, None) == etp.ETP_OK  # nothing wanted
-    assert B(h, 4, 4, ok, ok, ok, ok, ok, None, None, ok, ok, ok, ok, ok, ok, None) == etp.ETP_ERR_INVALID_ARG  # no r/frames
-    assert B(h, 4, 4, ok, ok, ok, ok, ok, None, bad, ok, ok, ok, ok, ok, ok, None) == etp.ETP_ERR_INVALID_ARG   # frames
+    assert B(h, 4, 4, ok, ok, None, ok, ok, ok, None, ok, ok, ok, ok, ok, ok, ok, 1 << 30, None) == etp.ETP_ERR_INVALID_ARG  # rev_ptr
+    assert B(h, 4, 4, ok, ok, ok, None, ok, ok, None, ok, ok, ok, ok, ok, ok, ok, 1 << 30, None) == etp.ETP_ERR_INVALID_ARG  # rev_perm
+    assert B(h, 4, 4, ok, ok, ok, ok, ok, ok, None, ok, ok, bad, ok, ok, ok, ok, 1 << 30, None) == etp.ETP_ERR_INVALID_ARG   # grad_out
+    assert B(h, 4, 4, ok, ok, ok, ok, ok, ok, None, ok, ok, ok, ok, bad, ok, ok, 1 << 30, None) == etp.ETP_ERR_INVALID_ARG   # grad_w
+    assert B(h, 4, 4, ok, ok, ok, ok, ok, ok, None, ok, ok, ok, bad, ok, ok, ok, 1 << 30, None) == etp.ETP_ERR_INVALID_ARG   # grad_x
+    assert B(h, 4, 4, ok, ok, ok, ok, ok, ok, None, ok, ok, ok, None, None, None, ok, 1 << 30, None) == etp.ETP_OK  # nothing wanted
+    assert B(h, 4, 4, ok, ok, ok, ok, ok, None, None, ok, ok, ok, ok, ok, ok, ok, 1 << 30, None) == etp.ETP_ERR_INVALID_ARG  # no r/frames
+    assert B(h, 4, 4, ok, ok, ok, ok, ok, None, bad, ok, ok, ok, ok, ok, ok, ok, 1 << 30, None) == etp.ETP_ERR_INVALID_ARG   # frames
+    assert B(h, 4, 4, ok, ok, ok, ok, ok, ok, None, ok, ok, ok, ok, ok, ok, ok, 0, None) == etp.ETP_ERR_WORKSPACE
+    tw = ctypes.c_size_t()
+    assert lib.etp_tp_workspace_size(h, 100, 1000, 0, ctypes.byref(tw)) == etp.ETP_OK and tw.value > 0
+    assert lib.etp_tp_workspace_size(h, 100, 0, 0, ctypes.byref(tw)) == etp.ETP_OK and tw.value == 0
+    assert lib.etp_tp_workspace_size(None, 100, 1000, 0, ctypes.byref(tw)) == etp.ETP_ERR_INVALID_ARG
     G = lib.etp_edge_frames
     assert G(None, 4, ok, ok, None) == etp.ETP_ERR_INVALID_ARG      # no plan
     assert G(h, -1, ok, ok, None) == etp.ETP_ERR_INVALID_ARG        # E < 0
@@ -156,14 +164,14 @@ def test_host_argument_checks(lib):
     assert LS(10, 100, ok, ok, ok, 4.5, *full, ctypes.c_void_p(0x10004), ls.value, None) == etp.ETP_ERR_INVALID_ARG
     assert LS(0, 0, None, None, None, 4.5, *([None] * 6), None, 0, None) == etp.ETP_OK            # nothing to do
     FO, BO = lib.etp_forward_ordered, lib.etp_backward_ordered
-    assert FO(h, 4, 4, None, ok, ok, ok, ok, None, ok, ok, ok, None) == etp.ETP_ERR_INVALID_ARG    # order NULL
-    assert FO(h, 4, 4, ok, ok, None, ok, ok, None, ok, ok, ok, None) == etp.ETP_ERR_INVALID_ARG    # ord_edge NULL
-    assert FO(h, 4, 4, ok, None, ok, ok, ok, None, ok, ok, ok, None) == etp.ETP_ERR_INVALID_ARG    # ord_ptr NULL
-    assert FO(h, 4, 4, ok, ok, ok, ok, ok, None, ok, ok, bad, None) == etp.ETP_ERR_INVALID_ARG     # out
-    assert BO(h, 4, 4, ok, ok, ok, None, ok, None, ok, ok, ok, ok, ok, ok, None) == etp.ETP_ERR_INVALID_ARG  # dst
-    assert BO(h, 4, 4, None, ok, ok, ok, ok, None, ok, ok, ok, ok, ok, ok, None) == etp.ETP_ERR_INVALID_ARG  # order
-    assert BO(h, 4, 4, ok, ok, ok, ok, ok, None, ok, ok, bad, ok, ok, ok, None) == etp.ETP_ERR_INVALID_ARG   # grad_out
-    assert BO(h, 4, 4, ok, ok, ok, ok, ok, None, ok, ok, ok, None, None, None, None) == etp.ETP_OK          # nothing
+    assert FO(h, 4, 4, None, ok, ok, ok, ok, None, ok, ok, ok, ok, 1 << 30, None) == etp.ETP_ERR_INVALID_ARG    # order NULL
+    assert FO(h, 4, 4, ok, ok, None, ok, ok, None, ok, ok, ok, ok, 1 << 30, None) == etp.ETP_ERR_INVALID_ARG    # ord_edge NULL
+    assert FO(h, 4, 4, ok, None, ok, ok, ok, None, ok, ok, ok, ok, 1 << 30, None) == etp.ETP_ERR_INVALID_ARG    # ord_ptr NULL
+    assert FO(h, 4, 4, ok, ok, ok, ok, ok, None, ok, ok, bad, ok, 1 << 30, None) == etp.ETP_ERR_INVALID_ARG     # out
+    assert BO(h, 4, 4, ok, ok, ok, None, ok, None, ok, ok, ok, ok, ok, ok, ok, 1 << 30, None) == etp.ETP_ERR_INVALID_ARG  # dst
+    assert BO(h, 4, 4, None, ok, ok, ok, ok, None, ok, ok, ok, ok, ok, ok, ok, 1 << 30, None) == etp.ETP_ERR_INVALID_ARG  # order
+    assert BO(h, 4, 4, ok, ok, ok, ok, ok, None, ok, ok, bad, ok, ok, ok, ok, 1 << 30, None) == etp.ETP_ERR_INVALID_ARG   # grad_out
+    assert BO(h, 4, 4, ok, ok, ok, ok, ok, None, ok, ok, ok, None, None, None, ok, 1 << 30, None) == etp.ETP_OK          # nothing
     V = lib.etp_validate_csr
     assert V(10, 100, None, ok, ok, None) == etp.ETP_ERR_INVALID_ARG
     assert V(10, 100, ok, ok, None, None) == etp.ETP_ERR_INVALID_ARG

@@ -139,3 +139,20 @@ def test_micro_sampled_rows(name):
     idx = torch.from_numpy(np.nonzero(keep)[0]).cuda()
     assert rel_err(gw[idx], ref[2]) <= VJP_TOL
     assert rel_err(gr[idx], ref[3]) <= VJP_TOL
+
+
+@pytest.mark.parametrize("C", [16, 128])
+def test_hub_rows_repeatable(C):
+    """Hub rows cut across many tasks: oracle parity, and two runs agree bit for bit."""
+    from gpu_helpers import hub_workload
+
+    wl = hub_workload(np.random.default_rng(37), 2, C, 15, hub=6000, rest=1000)
+    a = _run(wl, wl.irreps, wl.w, wl.r)
+    b = _run(wl, wl.irreps, wl.w, wl.r)
+    for x, y in zip(a, b):
+        assert torch.equal(x, y)
+    ref = _oracle(wl, wl.irreps, wl.w, wl.r)
+    assert rel_err(a[0], ref[0]) <= FWD_TOL
+    assert rel_err(a[1], ref[1]) <= VJP_TOL
+    assert rel_err(a[2], ref[2]) <= VJP_TOL
+    assert rel_err(a[3], ref[3]) <= VJP_TOL

@@ -169,3 +169,15 @@ def test_ordered_every_spec_ragged(L, o3, C):
     t, s = _schedule(wl, _random_pos(rng, wl.N), 3.0)
     res = _run_ordered(wl, plan, t, s, False)
     check_errs(compare_full(wl, res, irreps=irreps))
+
+
+def test_ordered_bitwise_repeatable():
+    """Two schedules of the same graph and two runs on them: every output repeats bit for bit."""
+    wl = workloads.make("water")
+    plan = etp.Plan(wl.irreps, wl.L, wl.irreps, wl.C)
+    t, s = _schedule(wl, wl.pos, wl.graph_cutoff)
+    a = _run_ordered(wl, plan, t, s, False)
+    _, s2 = _schedule(wl, wl.pos, wl.graph_cutoff)
+    b = _run_ordered(wl, plan, t, s2, False)
+    for k in a:
+        assert torch.equal(a[k], b[k]), k
