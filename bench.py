@@ -218,40 +218,43 @@ def recorded_traffic(kernel, framed, workload, n_nodes, scheduled=False):
 
 
 # ---------------------------------------------------------------------------
+def _oracle_sample(wl, tp, rows):
+    """The oracle's forward and VJP on the sub-graph of the given destination rows (their edges only, every
+    other row empty): out of those rows, grad_w and grad_r of their edges, grad_x of every source over them.
+    Returns (seconds, edges)."""
+    import numpy as np
+
+    edges = np.concatenate([np.arange(wl.row_ptr[i], wl.row_ptr[i + 1]) for i in rows])
+    counts = np.zeros(wl.N, dtype=np.int64)
+    counts[rows] = np.diff(wl.row_ptr)[rows]
+    sub_ptr = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    src, r, w = wl.src[edges], wl.r[edges], wl.w[edges]
+    t0 = time.perf_counter()
+    tp.forward(sub_ptr, src, r, wl.x, w, rows=rows)
+    tp.backward(sub_ptr, src, r, wl.x, w, wl.g)
+    return time.perf_counter() - t0, len(edges)
+
+
 def cpu_baseline(wl, seconds):
-    """The FP64 oracle, as it stands, on a bounded sample: fwd rows + VJP of the same edges."""
+    """The FP64 oracle, as it stands, on a bounded sample: fwd + VJP of the edges of random rows."""
     import numpy as np
 
     import oracle
 
     tp = oracle.OracleTP(wl.irreps, wl.L, wl.irreps, wl.C)
     rng = np.random.default_rng(1)
-
-    def run(n_rows):
-        rows = np.sort(rng.choice(wl.N, size=min(n_rows, wl.N), replace=False))
-        edges = np.concatenate([np.arange(wl.row_ptr[i], wl.row_ptr[i + 1]) for i in rows])
-        srcs = np.unique(wl.src[edges])[:n_rows]
-        t0 = time.perf_counter()
-        tp.forward(wl.row_ptr, wl.src, wl.r, wl.x, wl.w, rows=rows)
-        tp.backward(wl.row_ptr, wl.src, wl.r, wl.x, wl.w, wl.g, nodes=srcs, edges=edges)
-        dt = time.perf_counter() - t0
-        # the grad_x sample covers the edges whose source is in srcs
-        n_src_edges = int(np.isin(wl.src, srcs).sum())
-        return dt, len(edges), n_src_edges
-
-    # t(rows) ~ a + b rows (a: harmonics of every edge, b: the loops); size the sample to `seconds`
-    t2 = run(2)[0]
-    t6 = run(6)[0]
-    b = max((t6 - t2) / 4, 1e-4)
-    a = max(t2 - 2 * b, 0.0)
-    # the median of three samples of a third of the time each
-    n_rows = int(max(2, min(wl.N, (seconds / 3 - a) / b)))
-    runs = sorted((run(n_rows) for _ in range(3)), key=lambda t: t[1] / t[0])
-    dt, ne, nse = runs[1]
+    pick = lambda n: np.sort(rng.choice(wl.N, size=min(n, wl.N), replace=False))
+    # the work grows with the sampled edges; size the sample to `seconds` (three samples of a third each)
+    dt, ne = _oracle_sample(wl, tp, pick(max(2, wl.N // 64)))
+    per_edge = max(dt / max(ne, 1), 1e-9)
+    want_edges = (seconds / 3) / per_edge
+    n_rows = int(max(2, min(wl.N, want_edges / max(wl.E / max(wl.N, 1), 1))))
+    runs = sorted((_oracle_sample(wl, tp, pick(n_rows)) for _ in range(3)), key=lambda t: t[1] / t[0])
+    dt, ne = runs[1]
     return {"value": ne / dt, "unit": "edges/s", "cores": oracle.num_threads(), "kind": "oracle",
-            "sample": f"median of 3 samples, each {n_rows} random destination rows ({ne} edges): forward of those "
-                      f"rows, grad_w and grad_r of those edges, grad_x of {n_rows} of their sources ({nse} edges); "
-                      f"FP64 C loops with OpenMP, harmonics of all {wl.E} edges in numpy; {dt:.1f} s each"}
+            "sample": f"median of 3 samples, each the {ne} edges of {n_rows} random destination rows: forward of "
+                      f"those rows and the VJP (grad_x, grad_w, grad_r) over those edges; FP64 C loops with OpenMP, "
+                      f"harmonics of the sampled edges in numpy; {dt:.1f} s each"}
 
 
 def reference_arm(args):
@@ -271,22 +274,15 @@ def reference_arm(args):
 
     def step(n_rows):
         rows = np.sort(rng.choice(wl.N, size=n_rows, replace=False))
-        edges = np.concatenate([np.arange(wl.row_ptr[i], wl.row_ptr[i + 1]) for i in rows])
-        tp.forward(wl.row_ptr, wl.src, wl.r, wl.x, wl.w, rows=rows)
-        tp.backward(wl.row_ptr, wl.src, wl.r, wl.x, wl.w, wl.g, nodes=wl.src[edges[:n_rows]], edges=edges)
-        return len(edges)
+        return _oracle_sample(wl, tp, rows)[1]
 
-    # a step's time ~ a + b rows (a: the oracle's harmonics of every edge); size each step so that the whole
-    # run (warm-up + timed steps) takes about two minutes, and at most 2.5 s a step
+    # a step's time grows with its edges; size each step so that the whole run (warm-up + timed steps) takes
+    # about two minutes, and at most 2.5 s a step
     t_a = time.perf_counter()
-    step(2)
-    t_b = time.perf_counter()
-    step(10)
-    t_c = time.perf_counter()
-    b = max(((t_c - t_b) - (t_b - t_a)) / 8, 1e-4)
-    a = max((t_b - t_a) - 2 * b, 0.0)
+    ne = step(max(2, min(wl.N, wl.N // 64)))
+    per_edge = max((time.perf_counter() - t_a) / max(ne, 1), 1e-9)
     budget = min(2.5, 120.0 / max(args.steps + args.warmup, 1))
-    rows_per_step = int(max(1, min(wl.N, (budget - a) / b)))
+    rows_per_step = int(max(1, min(wl.N, budget / per_edge / max(wl.E / max(wl.N, 1), 1))))
 
     for _ in range(args.warmup):
         step(rows_per_step)
@@ -295,8 +291,8 @@ def reference_arm(args):
     dt = time.perf_counter() - t0
     value = ne / dt
     cores = oracle.num_threads()
-    sample = f"each step: {rows_per_step} random destination rows of {args.workload} (forward + grad_w + grad_r " \
-             f"of their edges, grad_x of {rows_per_step} sources); FP64 oracle"
+    sample = f"each step: the edges of {rows_per_step} random destination rows of {args.workload} (forward of " \
+             f"those rows and the VJP: grad_x, grad_w, grad_r over those edges); FP64 oracle"
     print(json.dumps({
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * dt / max(args.steps, 1),
@@ -521,13 +517,10 @@ def main():
             etp._check(lib.etp_edge_frames(plan.handle, E, P(b["r"]), P(frames), spp), "edge frames")
         if ev:
             ev[2].record(s)
-        if scheduled:
-            etp._check(lib.etp_forward_ordered(plan.handle, N, E, P(sched.order), P(sched.ord_ptr),
-                                               P(sched.ord_edge), P(b["src"]), P(b["r"]), P(frames), P(b["x"]),
-                                               P(b["w"]), P(b["out"]), P(ws), ws.numel(), spp), "forward (scheduled)")
-        else:
-            etp._check(lib.etp_forward(plan.handle, N, E, P(b["row_ptr"]), P(b["src"]), P(b["r"]), P(frames),
-                                       P(b["x"]), P(b["w"]), P(b["out"]), P(ws), ws.numel(), spp), "forward")
+        # the forward stays in CSR order: on the schedule it reads fewer bytes but is no faster (it is bound by
+        # its arithmetic there), while the VJP gains
+        etp._check(lib.etp_forward(plan.handle, N, E, P(b["row_ptr"]), P(b["src"]), P(b["r"]), P(frames),
+                                   P(b["x"]), P(b["w"]), P(b["out"]), P(ws), ws.numel(), spp), "forward")
         if ev:
             ev[3].record(s)
         if scheduled:
@@ -739,7 +732,8 @@ def main():
                "pipelining": "double-buffered: input copies, compute and output copies on three streams"}
 
     # kernels launched per step: the reverse CSR (one counting pass: counts, chunk scan, chunk-total scan,
-    # scatter, edge rows; otherwise counts, scan, edge rows and 3 per 8-bit radix pass), frames, forward, backward
+    # scatter, edge rows; otherwise counts, scan, edge rows and 4 per 8-bit radix pass: histograms, column scan,
+    # digit totals, scatter), frames, forward and backward with their row-combine passes
     n_tiles = (E + 1023) // 1024
     if E > 0 and 1 <= N <= 8192 and (N + 1) * n_tiles <= (1 << 22):
         rc_launches = 5
@@ -747,11 +741,11 @@ def main():
         passes = 0
         while (1 << (8 * passes)) < N and passes < 4:
             passes += 1
-        rc_launches = (1 if E > 0 else 0) + 1 + (1 if E > 0 else 0) + ((1 if passes == 0 else 3 * passes) if E > 0 else 0)
-    if scheduled:  # bounding box (2), Morton keys, 4 radix passes of 3; rank, degrees, scan (3); edge rows,
+        rc_launches = (1 if E > 0 else 0) + 1 + (1 if E > 0 else 0) + ((1 if passes == 0 else 4 * passes) if E > 0 else 0)
+    if scheduled:  # bounding box (2), Morton keys, 4 radix passes of 4; rank, degrees, scan (3); edge rows,
         # positions, source ranks (3 with edges); then the reverse CSR over the ranks
-        rc_launches = 3 + 12 + 3 + ((3 + rc_launches - 1) if E > 0 else 0)  # (its own edge-rows launch is skipped)
-    launches = K * (rc_launches + 2 + (1 if framed and E > 0 else 0))  # in the timed steps
+        rc_launches = 3 + 16 + 3 + ((3 + rc_launches - 1) if E > 0 else 0)  # (its own edge-rows launch is skipped)
+    launches = K * (rc_launches + 4 + (1 if framed and E > 0 else 0))  # in the timed steps
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -769,6 +763,7 @@ def main():
                    "P": plan.n_paths, "cg_nnz": nnz_total,
                    "step": (("locality schedule (Morton order of the positions, ordered CSRs) + " if scheduled
                              else "reverse CSR + ") + ("edge frames + " if framed else "") +
+                            ("forward in CSR order + VJP on the schedule: " if scheduled else "") +
                             "forward + VJP (grad_x, grad_w, grad_r), inputs resident in HBM"),
                    "l2": f"inputs larger than L2 (w = {wl.w.nbytes / 1e9:.2f} GB streamed per pass)",
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",

@@ -196,6 +196,7 @@ __global__ void __launch_bounds__(kThreads) etp_cart_fwd_kernel(Args a) {
         });
     }
     store_row<D>(row_slot(a.out, a.part, row, row_lo, row_hi, k0, k1, tm.task, D * C2, tm.cp), C2, acc);
+    if (tm.slice == 0 && tm.tl == 0) tail_record(a.part, a.ntasks, D * C2, tm.task, row, row_lo, row_hi, k0, k1);
 }
 
 template <int L, bool O3>
@@ -305,8 +306,10 @@ __global__ void __launch_bounds__(kThreads) etp_cart_bwd_kernel(Args a) {
             }
         }
     }
-    if (a.grad_x)
+    if (a.grad_x) {
         store_row<D>(row_slot(a.grad_x, a.part, row, row_lo, row_hi, k0, k1, tm.task, D * C2, tm.cp), C2, gx);
+        if (tm.slice == 0 && tm.tl == 0) tail_record(a.part, a.ntasks, D * C2, tm.task, row, row_lo, row_hi, k0, k1);
+    }
 }
 
 }  // namespace cart

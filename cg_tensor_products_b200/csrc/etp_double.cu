@@ -340,8 +340,10 @@ __global__ void __launch_bounds__(kThreads) etp_dd_dst_kernel(Args a) {
             });
         }
     }
-    if (a.grad_g)
+    if (a.grad_g) {
         store_row<D>(row_slot(a.grad_g, a.part, row, row_lo, row_hi, k0, k1, tm.task, D * C2, tm.cp), C2, acc);
+        if (tm.slice == 0 && tm.tl == 0) tail_record(a.part, a.ntasks, D * C2, tm.task, row, row_lo, row_hi, k0, k1);
+    }
 }
 
 
@@ -596,8 +598,10 @@ __global__ void __launch_bounds__(kThreads) etp_dd_src_kernel(Args a) {
             }
         }
     }
-    if (a.grad_x)
+    if (a.grad_x) {
         store_row<D>(row_slot(a.grad_x, a.part, row, row_lo, row_hi, k0, k1, tm.task, D * C2, tm.cp), C2, gx);
+        if (tm.slice == 0 && tm.tl == 0) tail_record(a.part, a.ntasks, D * C2, tm.task, row, row_lo, row_hi, k0, k1);
+    }
 }
 
 template <int L, bool O3>

@@ -536,6 +536,14 @@ __device__ __forceinline__ void store_row(float2* dst, int C2, const float2 (&ac
     for (int k = 0; k < D; ++k) dst[k * C2] = acc[k];
 }
 
+// The task's record after the partial rows: its last row (rank) when that row
+// goes on past the task and begins in it, else -1 (one lane per task writes it).
+__device__ __forceinline__ void tail_record(float2* part, int ntasks, int DC2, int task, int row, int lo, int hi,
+                                            int k0, int k1) {
+    int32_t* rec = reinterpret_cast<int32_t*>(part + (size_t)ntasks * 2 * DC2);
+    rec[task] = (hi > k1 && lo >= k0) ? row : -1;
+}
+
 // Where a task's finished row [lo, hi) of positions goes (this lane's channel
 // pair): the output row, or the task's partial slot.
 __device__ __forceinline__ float2* row_slot(float2* rows, float2* part, int node, int lo, int hi, int k0, int k1,
@@ -841,6 +849,7 @@ __global__ void __launch_bounds__(frame::kThreads, 4) etp_fwd_frame_kernel(FwdAr
         r_cur = r_next;
     }
     store_row<D>(row_slot(out2, part2, node, row_lo, row_hi, k0, k1, G.task, D * C2, cp), C2, acc);
+    if (G.slice == 0 && G.tl == 0) tail_record(part2, a.ntasks, D * C2, G.task, row, row_lo, row_hi, k0, k1);
 }
 
 // ===========================================================================
@@ -1131,7 +1140,10 @@ __global__ void __launch_bounds__(frame::kThreads, L <= 2 ? 6 : 4) etp_bwd_frame
         r_cur = r_next;
     }
     cp_async_wait_all();
-    if (gx2) store_row<D>(row_slot(gx2, part2, node, row_lo, row_hi, k0, k1, G.task, D * C2, cp), C2, gx);
+    if (gx2) {
+        store_row<D>(row_slot(gx2, part2, node, row_lo, row_hi, k0, k1, G.task, D * C2, cp), C2, gx);
+        if (G.slice == 0 && G.tl == 0) tail_record(part2, a.ntasks, D * C2, G.task, row, row_lo, row_hi, k0, k1);
+    }
 }
 
 namespace frame {

@@ -12,8 +12,8 @@
 // Otherwise the reverse grouping is a least-significant-digit radix sort of the source ids
 // with the edge ids as values, 8 bits per pass. Each pass is a stable counting
 // sort over tiles of kTile edges: (1) a per-tile digit histogram, (2) an
-// exclusive scan of the histogram table in (digit, tile) order, (3) a stable
-// scatter in which four warps split a tile into quarters, offset each other by
+// exclusive scan of the histogram table in (digit, tile) order (a parallel
+// column scan, then the digit totals), (3) a stable scatter in which four warps split a tile into quarters, offset each other by
 // their digit counts, and walk their quarter in order, ranking equal digits
 // inside each 32-edge chunk with __match_any_sync. Stability of every pass makes the result
 // unique: ties (equal sources) stay in increasing edge id, so the output is
@@ -89,30 +89,54 @@ __global__ void __launch_bounds__(kScanThreads) scan_exclusive(const int32_t* in
 }
 
 // Exclusive scan, in place, of the per-tile digit counts in tile-major order
-// hist[t * 256 + d], in the order (digit, tile): one block of 256 threads, thread
-// d runs down its digit over the tiles (coalesced rows, loads batched by 8),
-// then the 256 digit totals are scanned and added back. hist[256 * n_tiles] = total.
-__global__ void __launch_bounds__(256) scan_digit_columns(int32_t* hist, int n_tiles) {
+// hist[t * 256 + d], in the order (digit, tile), in two launches.
+// (1) scan_digit_column: block d scans its digit's column over the tiles (in
+// chunks of 1024 tiles, one per thread, carrying the running total) and leaves
+// the column total in hist[256 * n_tiles + d].
+__global__ void __launch_bounds__(1024) scan_digit_column(int32_t* hist, int n_tiles) {
+    __shared__ int32_t warp_sums[32];
+    __shared__ int32_t carry_s;
+    const int d = blockIdx.x, tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+    if (tid == 0) carry_s = 0;
+    __syncthreads();
+    for (int base = 0; base < n_tiles; base += 1024) {
+        const int t = base + tid;
+        const int v = t < n_tiles ? hist[(size_t)t * 256 + d] : 0;
+        int incl = v;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int u = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += u;
+        }
+        if (lane == 31) warp_sums[wid] = incl;
+        __syncthreads();
+        if (wid == 0) {
+            int ws = warp_sums[lane];
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int u = __shfl_up_sync(0xffffffffu, ws, o);
+                if (lane >= o) ws += u;
+            }
+            warp_sums[lane] = ws;  // inclusive over warps
+        }
+        __syncthreads();
+        const int carry = carry_s;
+        if (t < n_tiles) hist[(size_t)t * 256 + d] = carry + (wid ? warp_sums[wid - 1] : 0) + incl - v;
+        __syncthreads();
+        if (tid == 0) carry_s = carry + warp_sums[31];
+        __syncthreads();
+    }
+    if (tid == 0) hist[256 * (size_t)n_tiles + d] = carry_s;
+}
+
+// (2) scan_digit_totals: the 256 column totals become the digits' start offsets
+// (exclusive scan in place); hist[256 * n_tiles + 256] = the total. tile_scatter
+// adds a tile's column entry and its digit's start.
+__global__ void __launch_bounds__(256) scan_digit_totals(int32_t* hist, int n_tiles) {
     __shared__ int32_t tot[256];
     const int d = threadIdx.x;
-    int run = 0;
-    int t = 0;
-    for (; t + 8 <= n_tiles; t += 8) {
-        int v[8];
-#pragma unroll
-        for (int k = 0; k < 8; ++k) v[k] = hist[(size_t)(t + k) * 256 + d];
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-            hist[(size_t)(t + k) * 256 + d] = run;
-            run += v[k];
-        }
-    }
-    for (; t < n_tiles; ++t) {
-        const int v = hist[(size_t)t * 256 + d];
-        hist[(size_t)t * 256 + d] = run;
-        run += v;
-    }
-    tot[d] = run;
+    int32_t* col = hist + 256 * (size_t)n_tiles;
+    tot[d] = col[d];
     __syncthreads();
     for (int s = 1; s < 256; s <<= 1) {  // inclusive scan of the totals
         const int v = d >= s ? tot[d - s] : 0;
@@ -120,9 +144,8 @@ __global__ void __launch_bounds__(256) scan_digit_columns(int32_t* hist, int n_t
         tot[d] += v;
         __syncthreads();
     }
-    const int base = d ? tot[d - 1] : 0;
-    for (t = 0; t < n_tiles; ++t) hist[(size_t)t * 256 + d] += base;
-    if (d == 255) hist[256 * (size_t)n_tiles] = tot[255];
+    col[d] = d ? tot[d - 1] : 0;
+    if (d == 255) col[256] = tot[255];
 }
 
 // hist[t * 256 + d] = number of edges of tile t whose key has digit d.
@@ -138,9 +161,10 @@ __global__ void __launch_bounds__(256) tile_histogram(const int32_t* __restrict_
     hist[(size_t)t * 256 + threadIdx.x] = h[threadIdx.x];
 }
 
-// Stable scatter of one tile per block of 4 warps: warp w takes the w-th quarter
-// of the tile; (1) each warp counts its digits, (2) the per-digit counts are
-// prefix-summed over the warps on top of the tile's scanned offsets, (3) each
+// Stable scatter of one tile per block of 4 warps (one block per tile): warp w
+// takes the w-th quarter of the tile; (1) each warp counts its digits, (2) the
+// per-digit counts are prefix-summed over the warps on top of the tile's scanned
+// offsets (column entry plus digit start), (3) each
 // warp walks its quarter in order, ranking equal digits inside 32-edge chunks
 // with __match_any_sync. vals_in == nullptr means the identity (value = edge id).
 __global__ void __launch_bounds__(128) tile_scatter(const int32_t* __restrict__ keys_in,
@@ -160,7 +184,7 @@ __global__ void __launch_bounds__(128) tile_scatter(const int32_t* __restrict__ 
     }
     __syncthreads();
     for (int d = threadIdx.x; d < 256; d += 128) {  // warp-exclusive prefix per digit
-        int run = offsets[(size_t)t * 256 + d];
+        int run = offsets[(size_t)t * 256 + d] + offsets[256 * (size_t)gridDim.x + d];
 #pragma unroll
         for (int w = 0; w < 4; ++w) {
             const int v = cnt[w][d];
@@ -491,7 +515,7 @@ inline int radix_passes(int N) {
 
 // Stable LSD radix sort of the ids 0..n-1 by keys (8 bits per pass, `passes`
 // passes from the lowest digit); the sorted ids end in out. keys_a, keys_b,
-// vals_spare: n entries each; hist: 256 * tiles + 1.
+// vals_spare: n entries each; hist: 256 * (tiles + 1) + 1.
 void radix_sort_ids(const int32_t* keys, int n, int passes, int32_t* keys_a, int32_t* keys_b, int32_t* vals_spare,
                     int32_t* hist, int32_t* out, cudaStream_t s) {
     const int n_tiles = (n + kTile - 1) / kTile;
@@ -503,7 +527,8 @@ void radix_sort_ids(const int32_t* keys, int n, int passes, int32_t* keys_a, int
     for (int pass = 0; pass < passes; ++pass) {
         const int shift = 8 * pass;
         tile_histogram<<<n_tiles, 256, 0, s>>>(kin, n, shift, hist);
-        scan_digit_columns<<<1, 256, 0, s>>>(hist, n_tiles);
+        scan_digit_column<<<256, 1024, 0, s>>>(hist, n_tiles);
+        scan_digit_totals<<<1, 256, 0, s>>>(hist, n_tiles);
         int32_t* kout = kbuf[pass & 1];
         int32_t* vout = vbuf[pass & 1];
         tile_scatter<<<n_tiles, 128, 0, s>>>(kin, vin, n, shift, hist, kout, vout);
@@ -568,7 +593,7 @@ cudaError_t build_reverse_csr(int N, int E, const int32_t* row_ptr, const int32_
 
 size_t spatial_order_workspace_bytes(int N) {
     return align16(8 * sizeof(unsigned)) + 4 * align16(sizeof(int32_t) * (size_t)N) +
-           align16(sizeof(int32_t) * (256 * (size_t)radix_tiles(N) + 1));
+           align16(sizeof(int32_t) * (256 * ((size_t)radix_tiles(N) + 1) + 1));
 }
 
 cudaError_t spatial_order(int N, const float* pos, float cell, int32_t* order, void* ws, cudaStream_t s) {

@@ -78,14 +78,18 @@ cudaError_t launch_edge_frames(int E, const float* r, float* frames, cudaStream_
 // positions) over rows of row4 float4s; ptr: the CSR pointer the tasks ran over.
 cudaError_t launch_combine_rows(const int32_t* ptr, const int32_t* order, int N, int E, int ntasks, int row4,
                                 const float4* part, float4* rows, cudaStream_t s);
-// Bytes of the partial-row buffer of one launch shape.
-inline size_t partial_rows_bytes(int ntasks, int D, int C) { return 2 * (size_t)ntasks * D * C * sizeof(float); }
+// Bytes of the partial-row buffer of one launch shape: two rows of D x C floats
+// per task, then one int per task, the task's last row when that row is cut at
+// the task's end and begins in it (the task that starts its combine), else -1.
+inline size_t partial_rows_bytes(int ntasks, int D, int C) {
+    return 2 * (size_t)ntasks * D * C * sizeof(float) + (size_t)ntasks * sizeof(int32_t);
+}
 
 // Reverse CSR workspace. Up to kOnePassMaxNodes sources (and a bounded table)
 // the grouping is one stable counting pass over a (source, tile) count table;
 // otherwise a radix sort of the source ids, 8 bits per pass, whose workspace is
-// per-source counts, two key buffers, one value buffer and the digit-major table
-// of per-tile histograms (tiles of kRadixTile edges).
+// per-source counts, two key buffers, one value buffer and the table of per-tile
+// digit histograms (tiles of kRadixTile edges) with a row of digit totals.
 constexpr int kRadixTile = 1024;
 constexpr int kOnePassMaxNodes = 8192;
 constexpr long long kOnePassMaxEntries = 1ll << 22;
@@ -97,7 +101,7 @@ constexpr bool reverse_csr_one_pass(long long N, long long E) {
 }
 constexpr size_t radix_workspace_bytes_for(long long N, long long E) {
     return align16_bytes(4 * (size_t)(N + 1)) + 3 * align16_bytes(4 * (size_t)E) +
-           align16_bytes(4 * (256 * (size_t)radix_tiles(E) + 1));
+           align16_bytes(4 * (256 * ((size_t)radix_tiles(E) + 1) + 1));
 }
 constexpr size_t one_pass_workspace_bytes_for(long long N, long long E) {
     return align16_bytes(4 * (size_t)((N + 1) * radix_tiles(E))) +

@@ -18,21 +18,20 @@ int log2i(int t) {
 
 // Second pass of the segment sums, after the forward or backward kernel on the
 // same stream. (1) A row cut by task boundaries is stored by the block of the
-// task where it begins: the sum, in task order, of that task's slot 1 and the
-// slot 0 of each following task up to the one where the row ends. (2) Rows
+// task where it begins (found from the task's record after the partial rows):
+// the sum, in task order, of that task's slot 1 and the slot 0 of each
+// following task up to the one where the row ends. (2) Rows
 // without positions are zeroed, one warp per row. Every output row is thus
 // written exactly once, in a fixed order: no atomics, bitwise repeatable.
 __global__ void __launch_bounds__(256) etp_combine_rows_kernel(const int32_t* __restrict__ ptr,
                                                                const int32_t* __restrict__ order, int N, int E,
                                                                int ntasks, int row4, const float4* __restrict__ part,
                                                                float4* __restrict__ rows) {
+    const int32_t* rec = reinterpret_cast<const int32_t*>(part + (size_t)ntasks * 2 * row4);
     for (int t = blockIdx.x; t < ntasks; t += gridDim.x) {
-        int k0, k1;
-        frame::task_range(E, t, ntasks, k0, k1);
-        if (k0 >= k1) continue;
-        const int R = frame::segment_of(ptr, N, k1 - 1);
-        const int lo = __ldg(ptr + R), hi = __ldg(ptr + R + 1);
-        if (!(hi > k1 && lo >= k0)) continue;  // the task's last row ends in it, or began before it
+        const int R = rec[t];  // the task's last row if it goes on past the task and begins in it
+        if (R < 0) continue;
+        const int hi = __ldg(ptr + R + 1);
         const int node = order ? __ldg(order + R) : R;
         for (int f = threadIdx.x; f < row4; f += blockDim.x) {
             float4 acc = part[((size_t)t * 2 + 1) * row4 + f];

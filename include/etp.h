@@ -397,7 +397,7 @@ ETP_API etp_status etp_backward_ordered(etp_plan_t plan, int N, int E, const int
 /* Limits of etp_build_reverse_csr_static and the size of its scratch array. */
 #define ETP_STATIC_MAX_NODES (1 << 18)
 #define ETP_STATIC_MAX_EDGES (1 << 18)
-#define ETP_STATIC_SCRATCH_BYTES 4456480 /* device bytes held on every GPU that loads the library */
+#define ETP_STATIC_SCRATCH_BYTES 4457504 /* device bytes held on every GPU that loads the library */
 
 /* etp_build_reverse_csr without a workspace argument and without allocating:
  * for callers that cannot allocate device memory where they need the reverse
