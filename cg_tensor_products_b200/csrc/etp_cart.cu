@@ -23,7 +23,8 @@
 // Layout as the spherical kernels: x, out [N][(L+1)^2][C] (l blocks ascending, the
 // independent components above), w [E][P][C]; a team of lanes over the channels
 // (two per lane), equal contiguous ranges of edges, node rows summed in registers
-// (a row cut by a range boundary is added onto the zeroed output).
+// and stored once (a row cut by a range boundary leaves partial rows that the
+// row-combine pass sums in range order).
 #include <cuda_runtime.h>
 
 #include <cstdint>

@@ -28,8 +28,8 @@
 //
 // Two kernels, laid out like the first-order ones: edge-balanced tasks of
 // contiguous edges, a team of lanes over the channels (two per lane), node rows
-// summed in registers and stored once (a row cut by a task boundary is added by
-// vector reduction onto the zeroed output):
+// summed in registers and stored once (a row cut by a task boundary leaves partial
+// rows that the row-combine pass sums in task order):
 //   dd_dst: CSR order, grad_g;
 //   dd_src: reverse-CSR order, grad_x, and per edge grad_w and grad_r.
 // The frame vectors of an edge sit in lane-owned shared memory (registers), and so

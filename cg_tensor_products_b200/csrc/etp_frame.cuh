@@ -28,8 +28,9 @@
 // of T = min(32, C/2) lanes handles a slice of 2T channels of the task's edges
 // (lane t holds channels 2(sT + t), 2(sT + t) + 1 as a float2); with C = 128 a
 // task has two slices, the two warps of one block. Node sums accumulate in
-// registers and are stored once per row; a row cut by a task boundary is
-// combined with vector reductions onto the zeroed output. Per edge, one lane
+// registers and are stored once per row; a row cut by a task boundary leaves one
+// partial row per task, which a second launch sums in task order (no atomics).
+// Per edge, one lane
 // bulk-copies the next edge's weights (and frame record, and in the forward the
 // source row) into the other of two shared-memory buffers; each team expands its
 // edge's Wigner matrices into shared memory, from the record or built from r.
@@ -483,9 +484,9 @@ __device__ __forceinline__ float2 gen_form(const float2* v, const float2* s) {
 
 // ---------------------------------------------------------------------------
 // Work decomposition: equal contiguous ranges of edges ("tasks"), one per team
-// (or per pair of slice teams when C = 128, the block's two warps). Rows cut by a
-// range boundary are combined by vector reductions on a zeroed output; rows
-// inside a range are stored once.
+// (or per pair of slice teams when C = 128, the block's two warps). Rows inside a
+// range are stored once; rows cut by a range boundary go through the partial-row
+// slots (store_row, row_slot, tail_record below).
 struct Geometry {
     int T, S, team_in_block, task, slice, tl;
     unsigned tmask;
