@@ -195,9 +195,16 @@ template <int L, bool O3>
 constexpr int dst_team_floats(int T) {
     return frame::kTeamFloats + (2 * (L + 1) * (L + 1) + 2 * PathSet<L, O3>::P) * T * 2;
 }
+// The source kernel buffers the cotangent-weight row too for L <= 2; at L = 3 that
+// row (8.5 KB more per team) would leave room for three blocks per SM instead of
+// four, so there gg_w is read where it is used.
+template <int L>
+constexpr bool src_buffers_ggw() {
+    return L <= 2;
+}
 template <int L, bool O3>
 constexpr int src_team_floats(int T) {
-    return frame::kTeamFloats + (3 * (L + 1) * (L + 1) + 2 * PathSet<L, O3>::P) * T * 2;
+    return frame::kTeamFloats + (3 * (L + 1) * (L + 1) + (src_buffers_ggw<L>() ? 2 : 1) * PathSet<L, O3>::P) * T * 2;
 }
 
 // This lane's channel pair of every path of two weight rows, into lane-owned
@@ -431,7 +438,7 @@ __global__ void __launch_bounds__(kThreads) etp_dd_src_kernel(Args a) {
             continue;
         }
         // this edge's weight rows and g row, in flight while the frame is built
-        copy_weight_rows<P>(wbuf, gwbuf, wrow, gwrow, C2, T);
+        copy_weight_rows<P>(wbuf, gwbuf, wrow, src_buffers_ggw<L>() ? gwrow : nullptr, C2, T);
 #pragma unroll
         for (int k = 0; k < D; ++k) cp_async8(&V(GP, k), gs + k * C2);
         cp_async_commit();
@@ -485,7 +492,10 @@ __global__ void __launch_bounds__(kThreads) etp_dd_src_kernel(Args a) {
                     apply_MT<L, O3, l1, l3>(We, Wo, gp3, z);
                     apply_MT<L, O3, l1, l3>(We, Wo, gt3, zt);
                     if (gwrow) {
-                        group_weights<L, O3, l1, l3>(gwbuf, T, We, Wo);
+                        if constexpr (src_buffers_ggw<L>())
+                            group_weights<L, O3, l1, l3>(gwbuf, T, We, Wo);
+                        else
+                            group_weights_g<L, O3, l1, l3>(gwrow, C2, We, Wo);
                         apply_MT<L, O3, l1, l3>(We, Wo, gp3, z2);
                     }
                 }
@@ -538,7 +548,10 @@ __global__ void __launch_bounds__(kThreads) etp_dd_src_kernel(Args a) {
                     apply_M<L, O3, l1, l3>(We, Wo, xt1, yt);
                     apply_M<L, O3, l1, l3>(We, Wo, gxp1, y56);
                     if (gwrow) {
-                        group_weights<L, O3, l1, l3>(gwbuf, T, We, Wo);
+                        if constexpr (src_buffers_ggw<L>())
+                            group_weights<L, O3, l1, l3>(gwbuf, T, We, Wo);
+                        else
+                            group_weights_g<L, O3, l1, l3>(gwrow, C2, We, Wo);
                         apply_M<L, O3, l1, l3>(We, Wo, xp1, y56);
                     }
                     if (gwe) {
