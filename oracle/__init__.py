@@ -27,6 +27,7 @@ from . import sh as sh_mod
 from .forces import assemble_forces  # noqa: F401  (forces and per-atom virials from dE/dr)
 from . import radial  # noqa: F401  (radial-weight MLP of the edge length and its VJP)
 from . import cartesian  # noqa: F401  (the same edge convolution with Cartesian couplings)
+from . import nodelocal  # noqa: F401  (the node-local product, spherical and Cartesian)
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _BUILD = os.path.join(_HERE, "_build")
