@@ -342,7 +342,8 @@ def extra_timings(etp, lib, plan, wl, d, rev_ptr, rev_perm, dst, gw, stream, dev
         (3 TF32 products per FP32 product of the dense layer, TF32 peak = measured bf16 x 1/2);
       - the VJP of the VJP (all three cotangents), against its algorithmic bytes (HBM);
       - the Cartesian edge convolution (forward and VJP) beside the spherical kernels at equal rank, against
-        the same algorithmic bytes (HBM)."""
+        the same algorithmic bytes (HBM);
+      - the node-local product at its own fixed size (node_product_timings), against the FP32 pipes."""
     import numpy as np
     import torch
 
@@ -432,7 +433,53 @@ def extra_timings(etp, lib, plan, wl, d, rev_ptr, rev_perm, dst, gw, stream, dev
     cart["note"] = ("equal rank: the same graph, weights and path list; both read the edge vectors (no frame "
                     "records); algorithmic bytes of the spherical step for both")
     out["cartesian_vs_spherical"] = cart
+    out["node_product"] = node_product_timings(etp, stream, dev)
     return out
+
+
+def node_product_timings(etp, stream, dev, N=4096, C=128, L=3, K=4, reps=10, warm=3):
+    """The node-local product at the size the pages time it (4096 nodes x 128 channels, rank 3,
+    correlation order 4; the path-reduced product, forward), spherical and Cartesian couplings.
+    Each launch is timed alone with CUDA events after a 256 MB write that flushes L2 (its 67 MB of
+    input and output would otherwise stay resident). Bound by the FP32 pipes: the kernel's own
+    operation count (etp_node_product_ops: one multiply per operand product, one FMA per
+    coupling coefficient and per weighted output component) over 148 SMs x 128 FP32 lanes at
+    the 1965 MHz maximum SM clock."""
+    import torch
+
+    plan = etp.Plan(f"0..{L}", L, f"0..{L}", C)
+    g = torch.Generator(device=dev).manual_seed(5)
+    x = torch.randn((N, (L + 1) ** 2, C), device=dev, generator=g)
+    w = torch.randn((K - 1, plan.n_paths, C), device=dev, generator=g) / plan.n_paths ** 0.5
+    out = torch.empty_like(x)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    peak = 148 * 128 * 1.965e9 / 1e12
+    res = {"nodes": N, "channels": C, "rank": L, "order": K, "paths": plan.n_paths,
+           "page_ms_path_reduced": 0.40, "page_note": "the pages' time for this size and order, GPU not named: context"}
+    with torch.cuda.stream(stream):
+        for cart in (False, True):
+            fn = lambda: etp.node_product(plan, x, w, K=K, cartesian=cart, out=out, stream=stream)
+            for _ in range(warm):
+                fn()
+            total = 0.0
+            for _ in range(reps):
+                flush.zero_()
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                fn()
+                b.record(stream)
+                b.synchronize()
+                total += a.elapsed_time(b)
+            ms = total / reps
+            ops = etp.node_product_ops(plan, cart) * N * C * (K - 1)
+            res["cartesian" if cart else "spherical"] = {
+                "ms": ms, "ops_per_node_channel_step": etp.node_product_ops(plan, cart),
+                "roofline": {"bound": "alu", "achieved": ops / (ms * 1e9), "peak": peak, "unit": "Top/s",
+                             "frac": ops / (ms * 1e9) / peak,
+                             "peak_source": "148 SMs x 128 FP32 lanes x 1965 MHz (FMA or multiply: one op)"},
+                "hbm_bytes_per_launch": 2 * N * (L + 1) ** 2 * C * 4 + (K - 1) * plan.n_paths * C * 4}
+    del flush
+    return res
 
 
 # ---------------------------------------------------------------------------

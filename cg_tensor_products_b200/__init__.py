@@ -60,6 +60,8 @@ def _load():
         "etp_cart_forward": [vp, i32, i32, vp, vp, vp, vp, vp, vp, vp, sz, vp],
         "etp_cart_backward": [vp, i32, i32] + [vp] * 12 + [vp, sz, vp],
         "etp_assemble_forces": [i32, i32, vp, vp, vp, vp, vp, vp, vp, vp],
+        "etp_node_product": [vp, i32, i32, i32, vp, vp, vp, vp],
+        "etp_node_product_ops": [vp, i32, ctypes.POINTER(i32)],
         "etp_radial_workspace_size": [vp, i32, i32, i32, ctypes.POINTER(sz)],
         "etp_radial_forward": [vp, i32, i32, i32, ctypes.c_float, vp, vp, vp, vp, vp, sz, vp],
         "etp_radial_backward": [vp, i32, i32, i32, ctypes.c_float, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp],
@@ -313,6 +315,45 @@ def cart_forward(plan: Plan, row_ptr, src, r, x, w, out=None, workspace=None, st
     _launch(dev, "etp_cart_forward", _load().etp_cart_forward, plan.handle, N, E, _ptr(row_ptr), _ptr(src), _ptr(r),
             _ptr(x), _ptr(w), _ptr(out), _ptr(workspace), workspace.numel(), stream=stream)
     return out
+
+
+def node_product(plan: Plan, x, w, K=None, cartesian=False, out=None, stream=None):
+    """Node-local product of correlation order K (launches etp_node_product): out = B(K) with
+    B(1) = x, B(k+1) = sum_p w[k-1, p] couple_p(B(k), x). x [N, D, C]; w [K-1, P, C] (K defaults
+    to w.shape[0] + 1; w may be None for K = 1); spherical or Cartesian (independent STF
+    components) couplings."""
+    import torch
+
+    N = x.shape[0] if x.dim() == 3 else -1
+    _expect(x, "x", "float32", (N, plan.dim_in, plan.C))
+    if K is None:
+        if w is None:
+            raise ValueError("give K or w")
+        K = w.shape[0] + 1
+    if K < 1:
+        raise ValueError(f"K must be >= 1, got {K}")
+    if K > 1:
+        if w is None:
+            raise ValueError("w is required for K > 1")
+        _expect(w, "w", "float32", (K - 1, plan.n_paths, plan.C))
+    if out is None:
+        out = torch.empty((N, plan.dim_out, plan.C), device=x.device, dtype=torch.float32)
+    _expect(out, "out", "float32", (N, plan.dim_out, plan.C))
+    for t in (x, w if K > 1 else None):
+        if t is not None and t.numel() and out.numel() and \
+                out.data_ptr() < t.data_ptr() + 4 * t.numel() and t.data_ptr() < out.data_ptr() + 4 * out.numel():
+            raise ValueError("out must not overlap x or w")
+    dev = _need_cuda(x, out, *([w] if K > 1 else []))
+    _launch(dev, "etp_node_product", _load().etp_node_product, plan.handle, N, int(K), int(bool(cartesian)),
+            _ptr(x), _ptr(w) if K > 1 else None, _ptr(out), stream=stream)
+    return out
+
+
+def node_product_ops(plan: Plan, cartesian=False) -> int:
+    """FP32 operations per node, channel and step of the node-local product kernel."""
+    n = ctypes.c_int()
+    _check(_load().etp_node_product_ops(plan.handle, int(bool(cartesian)), ctypes.byref(n)), "node product ops")
+    return n.value
 
 
 def cart_backward(plan: Plan, row_ptr, src, rev_ptr, rev_perm, dst, r, x, w, grad_out, want=("x", "w", "r"),

@@ -80,7 +80,7 @@ def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False) 
     for L in range(4):
         jobs.append((os.path.join(CSRC, "etp_kernels_inst.cu"), os.path.join(BUILD_DIR, f"etp_kernels_l{L}.o"),
                      [f"-DETP_L={L}"]))
-    for name in ("etp_graph", "etp_forces", "etp_radial", "etp_radial_tc", "etp_fused", "etp_double", "etp_cart", "etp_api",
+    for name in ("etp_graph", "etp_forces", "etp_radial", "etp_radial_tc", "etp_fused", "etp_double", "etp_cart", "etp_nodeprod", "etp_api",
                  "etp_static_scratch", "etp_launch"):
         jobs.append((os.path.join(CSRC, name + ".cu"), os.path.join(BUILD_DIR, name + ".o"), []))
     extra = ["-Xptxas", "-v"] if ptxas_info else []

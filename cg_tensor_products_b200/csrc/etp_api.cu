@@ -475,6 +475,22 @@ etp_status etp_cart_backward(etp_plan_t plan, int N, int E, const int32_t* row_p
                                           reinterpret_cast<cudaStream_t>(stream)));
 }
 
+etp_status etp_node_product(etp_plan_t plan, int N, int K, int cartesian, const float* x, const float* w,
+                            float* out, etp_stream_t stream) {
+    if (!plan || N < 0 || K < 1 || (cartesian != 0 && cartesian != 1)) return ETP_ERR_INVALID_ARG;
+    if (N == 0) return ETP_OK;
+    if (!x || !out || !aligned16(x) || !aligned16(out)) return ETP_ERR_INVALID_ARG;
+    if (K > 1 && (!w || !aligned16(w))) return ETP_ERR_INVALID_ARG;
+    return cuda_status(etp::node_product(plan->L, plan->o3, cartesian != 0, plan->C, N, K, x, w, out,
+                                         reinterpret_cast<cudaStream_t>(stream)));
+}
+
+etp_status etp_node_product_ops(etp_plan_t plan, int cartesian, int* ops_per_step) {
+    if (!plan || !ops_per_step || (cartesian != 0 && cartesian != 1)) return ETP_ERR_INVALID_ARG;
+    *ops_per_step = etp::node_product_ops(plan->L, plan->o3, cartesian != 0);
+    return ETP_OK;
+}
+
 etp_status etp_assemble_forces(int N, int E, const int32_t* row_ptr, const int32_t* rev_ptr, const int32_t* rev_perm,
                                const float* r, const float* grad_r, float* forces, float* virial, etp_stream_t stream) {
     if (N < 0 || E < 0) return ETP_ERR_INVALID_ARG;

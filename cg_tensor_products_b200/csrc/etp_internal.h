@@ -168,6 +168,13 @@ cudaError_t cart_backward(int L, bool o3, int C, int N, int E, const int32_t* ro
                           const float* g, float* grad_x, float* grad_w, float* grad_r, void* part, size_t part_bytes,
                           cudaStream_t s);
 size_t cart_partial_bytes(int L, bool o3, int C, int N, int E);
+
+// node-local product (etp_nodeprod.cu): out = B(K), w [K-1][P][C]; cart selects the
+// Cartesian couplings
+cudaError_t node_product(int L, bool o3, bool cart, int C, int N, int K, const float* x, const float* w, float* out,
+                         cudaStream_t s);
+// FP32 operations per node, channel and step of that kernel's arithmetic
+int node_product_ops(int L, bool o3, bool cart);
 cudaError_t assemble_forces(int N, int E, const int32_t* row_ptr, const int32_t* rev_ptr, const int32_t* rev_perm,
                             const float* r, const float* grad_r, float* forces, float* virial, cudaStream_t s);
 cudaError_t validate_csr(int N, int E, const int32_t* row_ptr, const int32_t* src, int32_t* flag, cudaStream_t s);

@@ -251,6 +251,34 @@ ETP_API etp_status etp_cart_backward(etp_plan_t plan, int N, int E, const int32_
                                      float* grad_x, float* grad_w, float* grad_r, void* workspace,
                                      size_t workspace_bytes, etp_stream_t stream);
 
+/* Node-local product: features of higher correlation order from one node's own
+ * features ("FlashCart 如何让等变原子间势更快更准?", section "FlashCart 用笛卡尔内核替代
+ * 球谐耦合": equivariant features built recursively, brought back to a fixed width at
+ * every step; section "生成内核在高阶下胜过球谐基线": the node-local product at 4096
+ * nodes x 128 channels, rank 3, order 4, weighted products applied step by step and
+ * only ranks up to the maximum kept). The pages give no formula; this library's
+ * reading, with the plan's paths p = (l1, l2, l3) (l1 a rank of B, l2 a rank of x):
+ *   B(1) = x,  B(k+1)_l3[c] = sum_p w[k-1, p, c] couple_p(B(k)_l1[c], x_l2[c]),  k = 1 .. K-1,
+ *   out = B(K)   (K: the correlation order, the number of factors of x).
+ * Channels do not mix; w is shared by all nodes. cartesian = 0: spherical
+ * components and the plan's real Clebsch-Gordan couplings (x, out laid out as for
+ * etp_forward); cartesian = 1: STF tensors in the independent components and
+ * couplings of etp_cart_forward (a general STF second operand, not only the edge
+ * attribute).
+ * x: float32 [N][D][C] device; w: float32 [K-1][P][C] device (may be NULL when
+ * K = 1); out: float32 [N][D][C] device, written in full, must not overlap x or w.
+ * All three 16-byte aligned and owned by the caller; nothing is allocated. The call
+ * is asynchronous on `stream`; results repeat bit for bit (no atomics).
+ * Errors: ETP_ERR_INVALID_ARG for a NULL plan, N < 0, K < 1, cartesian not 0 or 1, or
+ * a NULL or misaligned pointer that is needed; N = 0 returns ETP_OK at once. */
+ETP_API etp_status etp_node_product(etp_plan_t plan, int N, int K, int cartesian, const float* x, const float* w,
+                                    float* out, etp_stream_t stream);
+/* The kernel's FP32 operations per node, channel and step (one multiply per operand
+ * product it forms, one FMA per coupling coefficient, one FMA per weighted output
+ * component): the cost model of etp_node_product, whose work is this times
+ * N * C * (K - 1). */
+ETP_API etp_status etp_node_product_ops(etp_plan_t plan, int cartesian, int* ops_per_step);
+
 /* Radial weights: the tensor product's per-edge weights as a function of the edge
  * length. The pages make these weights a learned function of |r| ("High-performance
  * training and inference for deep equivariant interatomic potentials", section

@@ -23,7 +23,7 @@ def lib():
 
 def test_exports_every_declared_symbol(lib):
     names = etp.declared_symbols()
-    assert len(names) == 28
+    assert len(names) == 30
     for n in names:
         assert hasattr(lib, n), n
 
@@ -172,6 +172,20 @@ def test_host_argument_checks(lib):
     assert BO(h, 4, 4, None, ok, ok, ok, ok, None, ok, ok, ok, ok, ok, ok, ok, 1 << 30, None) == etp.ETP_ERR_INVALID_ARG  # order
     assert BO(h, 4, 4, ok, ok, ok, ok, ok, None, ok, ok, bad, ok, ok, ok, ok, 1 << 30, None) == etp.ETP_ERR_INVALID_ARG   # grad_out
     assert BO(h, 4, 4, ok, ok, ok, ok, ok, None, ok, ok, ok, None, None, None, ok, 1 << 30, None) == etp.ETP_OK          # nothing
+    NP = lib.etp_node_product
+    assert NP(None, 4, 2, 0, ok, ok, ok, None) == etp.ETP_ERR_INVALID_ARG      # no plan
+    assert NP(h, -1, 2, 0, ok, ok, ok, None) == etp.ETP_ERR_INVALID_ARG        # N < 0
+    assert NP(h, 4, 0, 0, ok, ok, ok, None) == etp.ETP_ERR_INVALID_ARG         # K < 1
+    assert NP(h, 4, 2, 2, ok, ok, ok, None) == etp.ETP_ERR_INVALID_ARG         # cartesian not 0 / 1
+    assert NP(h, 4, 2, 0, None, ok, ok, None) == etp.ETP_ERR_INVALID_ARG       # x NULL
+    assert NP(h, 4, 2, 0, ok, None, ok, None) == etp.ETP_ERR_INVALID_ARG       # w NULL with K > 1
+    assert NP(h, 4, 2, 1, ok, bad, ok, None) == etp.ETP_ERR_INVALID_ARG        # w misaligned
+    assert NP(h, 4, 1, 0, ok, None, bad, None) == etp.ETP_ERR_INVALID_ARG      # out misaligned
+    assert NP(h, 0, 3, 1, None, None, None, None) == etp.ETP_OK                # nothing to do
+    n = ctypes.c_int()
+    assert lib.etp_node_product_ops(None, 0, ctypes.byref(n)) == etp.ETP_ERR_INVALID_ARG
+    assert lib.etp_node_product_ops(h, 3, ctypes.byref(n)) == etp.ETP_ERR_INVALID_ARG
+    assert lib.etp_node_product_ops(h, 0, None) == etp.ETP_ERR_INVALID_ARG
     V = lib.etp_validate_csr
     assert V(10, 100, None, ok, ok, None) == etp.ETP_ERR_INVALID_ARG
     assert V(10, 100, ok, ok, None, None) == etp.ETP_ERR_INVALID_ARG
@@ -216,6 +230,16 @@ def test_binding_checks_dtypes_and_shapes(lib):
         etp.assemble_forces(N, row_ptr, row_ptr, src, torch.zeros(E, 3), forces=torch.zeros(N, 2))
     with pytest.raises(ValueError, match="expected"):
         etp.build_reverse_csr(N, row_ptr.long(), src)
+    nplan = etp.Plan("0..1", 1, "0..1", 8)
+    xn, wn = torch.zeros(N, 4, 8), torch.zeros(2, nplan.n_paths, 8)
+    with pytest.raises(ValueError, match="expected"):
+        etp.node_product(nplan, xn, torch.zeros(2, 4, 8))
+    with pytest.raises(ValueError, match="overlap"):
+        etp.node_product(nplan, xn, wn, out=xn)
+    with pytest.raises(ValueError, match="required"):
+        etp.node_product(nplan, xn, None, K=3)
+    with pytest.raises(ValueError, match="CUDA"):
+        etp.node_product(nplan, xn, wn)
 
 
 def test_fused_workspace_size_and_refusals(lib):
@@ -235,3 +259,22 @@ def test_frames_advised_by_size(lib):
     assert etp.Plan("0..3", 3, "0..3", 128).frames_advised(131072)          # 46 MB of records
     assert not etp.Plan("0..3", 3, "0..3", 64).frames_advised(1250256)     # 440 MB
     assert not etp.Plan("0..1", 1, "0..1", 8).frames_advised(256)
+
+
+@pytest.mark.parametrize("L,o3", [(1, False), (2, True), (3, False), (3, True)])
+def test_node_product_ops_count(lib, L, o3):
+    """The kernel's cost model: one multiply per operand product that some path uses, one
+    FMA per coupling coefficient, one FMA per weighted output component; counted here from
+    the oracle's own couplings (spherical: nonzero real CG entries)."""
+    irreps = "+".join(f"{l}{'e' if l % 2 == 0 else 'o'}" for l in range(L + 1)) if o3 else f"0..{L}"
+    plan = etp.Plan(irreps, L, irreps, 8)
+    from oracle import nodelocal
+
+    nps = nodelocal.node_paths(irreps)
+    terms = sum(int(np.count_nonzero(cg.real_cg(*p))) for p in nps)
+    pairs = set()
+    for p in nps:
+        for a, b, _ in np.argwhere(cg.real_cg(*p) != 0):
+            pairs.add((p[0], p[1], int(a), int(b)))
+    outs = sum(2 * p[2] + 1 for p in nps)
+    assert etp.node_product_ops(plan, False) == len(pairs) + terms + outs

@@ -3,7 +3,6 @@ against the FP64 Cartesian oracle (oracle/cartesian.py, full 3^l tensors, VJP by
 autograd). The library holds a rank-l STF tensor by its 2l + 1 entries with at most
 one z index; the test maps those to and from full tensors with its own expansion
 (STF completion) and entry picks. Tolerances: forward 1e-5, VJP 1e-4."""
-import itertools
 
 import numpy as np
 import pytest
@@ -14,6 +13,7 @@ import oracle
 import workloads
 from cg_tensor_products_b200 import build as etp_build
 from gpu_helpers import FWD_TOL, VJP_TOL, rel_err
+from cart_layout import expand as _expand, from_full as _from_full, pick as _pick, to_full as _to_full
 from oracle import cartesian as ct
 
 pytestmark = pytest.mark.gpu
@@ -25,49 +25,6 @@ def _built():
         pytest.skip("no CUDA device")
     etp_build.build()
     oracle.build()
-
-
-def _counts(l):
-    return [(l - b, b, 0) for b in range(l + 1)] + [(l - 1 - b, b, 1) for b in range(l)]
-
-
-def _pick(l):
-    """S [2l+1, 3^l]: the independent entries of a full rank-l tensor."""
-    if l == 0:
-        return np.ones((1, 1))
-    pos = {t: i for i, t in enumerate(itertools.product(range(3), repeat=l))}
-    S = np.zeros((2 * l + 1, 3 ** l))
-    for i, (a, b, c) in enumerate(_counts(l)):
-        S[i, pos[(0,) * a + (1,) * b + (2,) * c]] = 1.0
-    return S
-
-
-def _expand(l):
-    """E [3^l, 2l+1]: the STF tensor with the given independent entries (S E = I)."""
-    if l == 0:
-        return np.ones((1, 1))
-    u, s, _ = np.linalg.svd(ct.stf_projector(l))
-    Q = u[:, s > 0.5]
-    return Q @ np.linalg.inv(_pick(l) @ Q)
-
-
-def _to_full(a, L):
-    """[N, (L+1)^2, C] independent components -> {l: [N, C] + [3] * l} full tensors."""
-    out = {}
-    for l in range(L + 1):
-        blk = a[:, l * l:(l + 1) ** 2, :].astype(np.float64)             # [N, 2l+1, C]
-        full = np.einsum("fi,nic->ncf", _expand(l), blk)
-        out[l] = torch.from_numpy(full.reshape(a.shape[0], a.shape[2], *([3] * l)) if l else full[..., 0])
-    return out
-
-
-def _from_full(d, L, op):
-    """{l: [N, C] + [3]*l} -> [N, (L+1)^2, C] with op(l) ([2l+1, 3^l]) applied to each tensor."""
-    blocks = []
-    for l in range(L + 1):
-        t = d[l].detach().numpy().reshape(d[l].shape[0], d[l].shape[1], -1)
-        blocks.append(np.einsum("if,ncf->nic", op(l), t))
-    return np.concatenate(blocks, axis=1)
 
 
 def _run(wl, irreps, w, r):
