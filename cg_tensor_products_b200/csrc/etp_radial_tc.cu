@@ -7,18 +7,21 @@
 // whose dropped term A_lo B_lo and rounding of the halves leave a relative error
 // near 2^-21 per product, below the 1e-5 tolerance of the forward.
 //
-// Per CTA (4 warps, one per SM: 225 KB of shared memory) and tile of 128 edges:
-//   1. each thread builds its edge's row of H (Bessel basis, first layer, SiLU),
-//      splits it into TF32 halves and stores both into shared memory in the
-//      tensor core's K-major layout without swizzle: 8-row x 16-byte core matrices,
-//      LBO = 128 B between core matrices along K, SBO = 2048 B between 8-row groups;
-//   2. per chunk of up to 128 output columns, one thread bulk-copies the chunk of
-//      W2^T (halves pre-split by radial_tc_prepare into the same layout) into shared
-//      memory, issues 8 K-steps x 3 products of tcgen05.mma (M = 128, N = chunk,
-//      K = 8, kind::tf32) into a TMEM accumulator and commits them to an mbarrier;
-//   3. the 4 warps read the accumulator back (tcgen05.ld, warp w owns TMEM lanes
-//      32w..32w+31, i.e. edges), stage it in shared memory and store w in whole
-//      row segments.
+// Per CTA (9 warps, one CTA per SM: 224 KB of shared memory) and tile of 128 edges:
+//   1. the 8 epilogue warps build the tile's rows of H (Bessel basis, first layer,
+//      SiLU; two threads per edge), split them into TF32 halves and store both into
+//      shared memory in the tensor core's K-major layout without swizzle: 8-row x
+//      16-byte core matrices, LBO = 128 B between core matrices along K, SBO = 2048 B
+//      between 8-row groups;
+//   2. per chunk of up to 128 output columns, one thread of the ninth warp
+//      bulk-copies the chunk of W2^T (halves pre-split by radial_tc_prepare into the
+//      same layout) into one of two shared-memory slots, issues 8 K-steps x 3
+//      products of tcgen05.mma (M = 128, N = chunk, K = 8, kind::tf32) into one of
+//      two TMEM accumulators and commits them to an mbarrier;
+//   3. the 8 epilogue warps read the accumulator back (tcgen05.ld; warps w and w + 4
+//      own TMEM lanes 32w..32w+31, i.e. edges, and half of the columns each), hand it
+//      back to the MMA thread by an mbarrier, and store w in whole 128-byte row
+//      segments through a per-warp stage. No block barrier inside the chunk loop.
 // The VJP's two dense products, dL/dH = grad_w W2^T and grad_W2 = H^T grad_w, follow
 // below as warp-specialised kernels with the same operand layout and split.
 // Every wait is bounded; on time-out the kernel raises its fault flag and leaves.
@@ -35,7 +38,6 @@ constexpr int kRows = 128;                    // edges per tile (MMA M)
 constexpr int kBasis = 8;                     // Bessel functions (compile-time: registers, unrolled)
 constexpr int kHidden = 64;                   // K of the product (the hidden width)
 constexpr int kChunk = 128;                   // output columns per MMA group (N)
-constexpr int kThreads = 128;
 constexpr uint32_t kLBO = 128, kSBO = 2048;   // bytes: next K core matrix, next 8-row group
 constexpr uint32_t kTileBytes = kRows * kHidden * 4;  // 32 KB: one operand half of a tile
 constexpr int kWaitLimit = 1 << 22;
@@ -104,14 +106,17 @@ __global__ void radial_tc_prepare(const float* __restrict__ W2, int PC, int n_ch
 }
 
 // Shared memory: A halves (64 KB), two B slots of two halves (128 KB), the
-// epilogue stage (128 rows x 68 floats: 16-byte rows whose vector accesses hit
-// all 32 banks once per 8 threads), 4 mbarriers, the TMEM address.
-constexpr int kStageStride = 68;
-constexpr uint32_t kStageFloats = kRows * kStageStride;
+// epilogue stage (8 warps x 32 rows x 32 floats, 16-byte units XOR-swizzled by the
+// row so that a phase of 8 lanes writing one row each, or reading 8 units of one
+// row, touches 8 distinct bank quads), 6 mbarriers, the TMEM address, a flag.
+constexpr int kEpiWarps = 8;                   // two per TMEM lane quarter, each half of a chunk's columns
+constexpr int kFwdThreads = (kEpiWarps + 1) * 32;
+constexpr uint32_t kStageFloats = kEpiWarps * 32 * 32;
 constexpr uint32_t kOffB = 2 * kTileBytes, kOffStage = 6 * kTileBytes;
 constexpr uint32_t kOffBars = kOffStage + kStageFloats * 4;
 constexpr uint32_t kSmemBytes = kOffBars + 64;
 static_assert(kOffBars % 16 == 0 && kSmemBytes <= 232448, "radial tensor-core kernel shared memory");
+static_assert(kBasis * kHidden <= (int)kStageFloats, "W1 is staged in the epilogue buffer");
 
 __device__ __forceinline__ void load_b(const float* Bhi, const float* Blo, int c, unsigned char* slot_hi,
                                        unsigned char* slot_lo, uint64_t* bar) {
@@ -127,10 +132,20 @@ __device__ __forceinline__ void load_b(const float* Bhi, const float* Blo, int c
                  : "memory");
 }
 
-// Two-stage pipeline over the output chunks: while the tensor cores work on chunk
-// c (B slot c % 2, TMEM columns 128 (c % 2)), the warps write chunk c - 1 out and
-// the copy engine brings in chunk c + 1.
-__global__ void __launch_bounds__(kThreads, 1)
+__device__ __forceinline__ void mbar_arrive_one(uint64_t* bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+// Warp-specialised pipeline over the output chunks, with no block barrier in the
+// loop. The MMA warp (one thread) issues chunk c into accumulator c % 2 once its
+// W2 slot is filled (bar_b) and the epilogue has drained chunk c - 2 from that
+// accumulator (bar_free, one arrival per epilogue warp), commits to bar_m, and
+// refills the slot of chunk c - 1 with chunk c + 1 once chunk c - 1's MMAs are done.
+// Each epilogue warp (TMEM lane quarter w % 4, column half w / 4) waits for bar_m,
+// reads its 32 rows x 64 columns into registers, frees the accumulator, and writes
+// the rows out through its own stage: every store instruction writes four whole
+// 128-byte row segments.
+__global__ void __launch_bounds__(kFwdThreads, 1)
     radial_tc_forward(int E, int PC, int nb, float rc, const float* __restrict__ r, const float* __restrict__ W1,
                       const float* __restrict__ Bhi, const float* __restrict__ Blo, float* __restrict__ w) {
     extern __shared__ __align__(1024) unsigned char smem[];
@@ -139,34 +154,39 @@ __global__ void __launch_bounds__(kThreads, 1)
     float* stage = reinterpret_cast<float*>(smem + kOffStage);
     uint64_t* bar_b = reinterpret_cast<uint64_t*>(smem + kOffBars);       // [2] B slot filled
     uint64_t* bar_m = bar_b + 2;                                            // [2] accumulator ready
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffBars + 32);
-    int* abort_flag = reinterpret_cast<int*>(smem + kOffBars + 36);
+    uint64_t* bar_free = bar_b + 4;                                         // [2] accumulator drained
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffBars + 48);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffBars + 52);
     const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
     const int m0 = blockIdx.x * kRows;
     const int n_chunks = (PC + kChunk - 1) / kChunk;
+    constexpr int kMmaWarp = kEpiWarps;
     auto slot_hi = [&](int s) { return smem + kOffB + (uint32_t)s * 2 * kTileBytes; };
     auto slot_lo = [&](int s) { return smem + kOffB + (uint32_t)s * 2 * kTileBytes + kTileBytes; };
 
-    if (warp == 0) {  // two accumulators of 128 fp32 columns
+    if (warp == kMmaWarp) {  // two accumulators of 128 fp32 columns
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
                      "r"(256)
                      : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
-    }
-    if (t == 0) {
-        for (int i = 0; i < 4; ++i) mbar_init(&bar_b[i], 1);
-        *abort_flag = 0;
-        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-        load_b(Bhi, Blo, 0, slot_hi(0), slot_lo(0), &bar_b[0]);  // the first two chunks, behind H
-        if (n_chunks > 1) load_b(Bhi, Blo, 1, slot_hi(1), slot_lo(1), &bar_b[1]);
+        if (lane == 0) {
+            for (int i = 0; i < 4; ++i) mbar_init(&bar_b[i], 1);
+            for (int i = 0; i < 2; ++i) mbar_init(&bar_free[i], kEpiWarps);
+            *abort_flag = 0;
+            asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+            load_b(Bhi, Blo, 0, slot_hi(0), slot_lo(0), &bar_b[0]);  // the first two chunks, behind H
+            if (n_chunks > 1) load_b(Bhi, Blo, 1, slot_hi(1), slot_lo(1), &bar_b[1]);
+        }
     }
 
-    // 1. the tile's rows of H, split into TF32 halves (W1 read from the epilogue
-    // stage, which is free until the first chunk is written out)
-    for (int i = t; i < kBasis * kHidden; i += kThreads) stage[i] = __ldg(W1 + i);
+    // 1. the tile's rows of H, split into TF32 halves: two epilogue threads per row,
+    // 32 hidden units each (W1 read from the epilogue stage, free until the first
+    // chunk is written out)
+    for (int i = t; i < kBasis * kHidden; i += kFwdThreads) stage[i] = __ldg(W1 + i);
     __syncthreads();
-    {
-        const int e = m0 + t;
+    if (warp < kEpiWarps) {
+        const int row = t & (kRows - 1), k0 = (t >> 7) * (kHidden / 2);
+        const int e = m0 + row;
         float b[kBasis];
 #pragma unroll
         for (int n = 0; n < kBasis; ++n) b[n] = 0.f;
@@ -181,7 +201,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
 #pragma unroll 4
-        for (int k = 0; k < kHidden; ++k) {
+        for (int k = k0; k < k0 + kHidden / 2; ++k) {
             float h = 0.f;
             if (e < E) {
                 float zz = 0.f;
@@ -190,8 +210,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 h = zz / (1.f + expf(-zz));
             }
             const float hh = tf32_round(h);
-            *reinterpret_cast<float*>(a_hi + tile_offset(t, k)) = hh;
-            *reinterpret_cast<float*>(a_lo + tile_offset(t, k)) = tf32_round(h - hh);
+            *reinterpret_cast<float*>(a_hi + tile_offset(row, k)) = hh;
+            *reinterpret_cast<float*>(a_lo + tile_offset(row, k)) = tf32_round(h - hh);
         }
     }
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // generic-proxy writes -> tensor core
@@ -199,15 +219,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
     const uint32_t tmem = *tmem_slot;
-    int last_committed = -1;  // (thread 0) the last chunk whose MMAs were committed
 
-    for (int c = 0; c <= n_chunks; ++c) {
-        // 2. the MMAs of chunk c
-        if (c < n_chunks && t == 0 && !*abort_flag) {
-            const int sb = c & 1;
-            if (!mbar_wait(&bar_b[sb], (c >> 1) & 1)) {
-                *abort_flag = 1;
-            } else {
+    if (warp == kMmaWarp) {
+        // 2. the MMA thread
+        if (lane == 0) {
+            int committed = -1, loaded = n_chunks > 1 ? 1 : 0;  // last chunk committed / loaded
+            for (int c = 0; c < n_chunks && !*abort_flag; ++c) {
+                const int sb = c & 1, u = c >> 1;
+                if (!mbar_wait(&bar_b[sb], u & 1) || (c >= 2 && !mbar_wait(&bar_free[sb], (u - 1) & 1))) {
+                    *abort_flag = 1;
+                    break;
+                }
                 asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
                 const int n = min(kChunk, PC - c * kChunk);  // a multiple of 16
                 const uint32_t idesc = instr_desc(n);
@@ -229,23 +251,43 @@ __global__ void __launch_bounds__(kThreads, 1)
                 asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
                                  smem_u32(&bar_m[sb]))
                              : "memory");
-                last_committed = c;
+                committed = c;
+                // the slot of chunk c - 1 takes chunk c + 1 once chunk c - 1's products are done
+                if (c >= 1 && c + 1 < n_chunks) {
+                    if (!mbar_wait(&bar_m[sb ^ 1], ((c - 1) >> 1) & 1)) {
+                        *abort_flag = 1;
+                        break;
+                    }
+                    load_b(Bhi, Blo, c + 1, slot_hi(sb ^ 1), slot_lo(sb ^ 1), &bar_b[sb ^ 1]);
+                    loaded = c + 1;
+                }
+            }
+            if (*abort_flag) {
+                atomicOr(&g_fault, 1);
+                // leave nothing in flight on the freed TMEM and shared memory: one bounded wait each
+                if (committed >= 0) mbar_wait(&bar_m[committed & 1], (committed >> 1) & 1);
+                if (committed >= 1) mbar_wait(&bar_m[(committed - 1) & 1], ((committed - 1) >> 1) & 1);
+                for (int c = committed + 1; c <= loaded; ++c) mbar_wait(&bar_b[c & 1], (c >> 1) & 1);
             }
         }
-        if (c == 0) continue;
-        // 3. chunk c - 1: wait for its accumulator, refill its B slot, write it out
-        const int cp = c - 1, sp = cp & 1;
-        __syncthreads();
-        if (*abort_flag) break;
-        if (!mbar_wait(&bar_m[sp], (cp >> 1) & 1)) atomicOr(abort_flag, 1);
-        __syncthreads();
-        if (*abort_flag) break;
-        if (t == 0 && cp + 2 < n_chunks) load_b(Bhi, Blo, cp + 2, slot_hi(sp), slot_lo(sp), &bar_b[sp]);
-        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-        const int n = min(kChunk, PC - cp * kChunk);
-        for (int h0 = 0; h0 < n; h0 += 64) {
-            const int hn = min(64, n - h0);
-            uint32_t v[64];  // this thread's row of the half-chunk: all loads in flight, one wait
+    } else {
+        // 3. the epilogue warps
+        const int q = warp & 3, hf = warp >> 2;
+        float* st = stage + warp * 32 * 32;
+        for (int c = 0; c < n_chunks; ++c) {
+            const int sb = c & 1, u = c >> 1;
+            const int n = min(kChunk, PC - c * kChunk);
+            const int hn = max(0, min(64, n - 64 * hf));  // this warp's columns of the chunk
+            const bool got = mbar_wait(&bar_m[sb], u & 1);
+            if (__any_sync(0xffffffffu, !got || *abort_flag)) {  // warp-uniform
+                if (lane == 0) {
+                    *abort_flag = 1;
+                    atomicOr(&g_fault, 1);
+                }
+                break;
+            }
+            asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+            uint32_t v[64];
 #pragma unroll
             for (int jj = 0; jj < 4; ++jj) {
                 if (jj * 16 < hn)
@@ -256,38 +298,44 @@ __global__ void __launch_bounds__(kThreads, 1)
                           "=r"(v[16 * jj + 4]), "=r"(v[16 * jj + 5]), "=r"(v[16 * jj + 6]), "=r"(v[16 * jj + 7]),
                           "=r"(v[16 * jj + 8]), "=r"(v[16 * jj + 9]), "=r"(v[16 * jj + 10]), "=r"(v[16 * jj + 11]),
                           "=r"(v[16 * jj + 12]), "=r"(v[16 * jj + 13]), "=r"(v[16 * jj + 14]), "=r"(v[16 * jj + 15])
-                        : "r"(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(sp * 128 + h0 + 16 * jj)));
+                        : "r"(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(sb * 128 + 64 * hf + 16 * jj)));
+                else
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) v[16 * jj + i] = 0u;
             }
             asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+            asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+            __syncwarp();
+            if (lane == 0) mbar_arrive_one(&bar_free[sb]);  // the accumulator may take chunk c + 2
+            const int e_base = m0 + q * 32;
+            const size_t col0 = (size_t)c * kChunk + 64 * hf;
 #pragma unroll
-            for (int q = 0; q < 16; ++q)
-                if (q * 4 < hn)
-                    *reinterpret_cast<float4*>(stage + t * kStageStride + 4 * q) =
-                        make_float4(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1]),
-                                    __uint_as_float(v[4 * q + 2]), __uint_as_float(v[4 * q + 3]));
-            __syncthreads();
-            // each half-warp stores one 64-float row segment per step: 16 lanes x 16 bytes
-            const int col = (lane & 15) * 4;
-            for (int rr = 0; rr < 32; rr += 2) {
-                const int row = warp * 32 + rr + (lane >> 4), e = m0 + row;
-                if (e < E && col < hn)
-                    *reinterpret_cast<float4*>(w + (size_t)e * PC + cp * kChunk + h0 + col) =
-                        *reinterpret_cast<const float4*>(stage + row * kStageStride + col);
+            for (int sbk = 0; sbk < 2; ++sbk) {
+                if (32 * sbk >= hn) break;
+#pragma unroll
+                for (int j = 0; j < 8; ++j)
+                    *reinterpret_cast<float4*>(st + lane * 32 + 4 * (j ^ (lane & 7))) =
+                        make_float4(__uint_as_float(v[32 * sbk + 4 * j]), __uint_as_float(v[32 * sbk + 4 * j + 1]),
+                                    __uint_as_float(v[32 * sbk + 4 * j + 2]), __uint_as_float(v[32 * sbk + 4 * j + 3]));
+                __syncwarp();
+                const int jj = lane & 7;
+#pragma unroll
+                for (int rr = 0; rr < 8; ++rr) {
+                    const int row = 4 * rr + (lane >> 3), e = e_base + row;
+                    const int col = 32 * sbk + 4 * jj;
+                    if (e < E && col < hn)
+                        *reinterpret_cast<float4*>(w + (size_t)e * PC + col0 + col) =
+                            *reinterpret_cast<const float4*>(st + row * 32 + 4 * (jj ^ (row & 7)));
+                }
+                __syncwarp();
             }
-            __syncthreads();
         }
-        asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");  // accumulator sp free for chunk c + 1
     }
     __syncthreads();
-    if (t == 0 && *abort_flag) {
-        atomicOr(&g_fault, 1);
-        // leave nothing in flight on the freed TMEM and shared memory: one more bounded wait each
-        if (last_committed >= 0) mbar_wait(&bar_m[last_committed & 1], (last_committed >> 1) & 1);
-        for (int s2 = 0; s2 < 2 && s2 < n_chunks; ++s2) mbar_wait(&bar_b[s2], 0);
-    }
-    __syncthreads();
-    if (warp == 0)
+    if (warp == kMmaWarp) {
+        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(256) : "memory");
+    }
 }
 
 // ---------------------------------------------------------------------------
@@ -830,8 +878,8 @@ cudaError_t radial_tc_forward(int E, int nb, int PC, float rc, const float* r, c
     cudaError_t err = cudaFuncSetAttribute(rtc::radial_tc_forward, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                            (int)smem);
     if (err != cudaSuccess) return err;
-    rtc::radial_tc_forward<<<(E + rtc::kRows - 1) / rtc::kRows, rtc::kThreads, smem, s>>>(E, PC, nb, rc, r, W1, hi, lo,
-                                                                                         w);
+    rtc::radial_tc_forward<<<(E + rtc::kRows - 1) / rtc::kRows, rtc::kFwdThreads, smem, s>>>(E, PC, nb, rc, r, W1, hi,
+                                                                                            lo, w);
     return cudaGetLastError();
 }
 

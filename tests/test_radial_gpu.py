@@ -31,7 +31,7 @@ def _params(seed, P, C, nb=8, hidden=64):
 
 @pytest.mark.parametrize("L,C,nb,hidden,E", [(2, 64, 8, 64, 5000), (3, 128, 8, 64, 3000), (1, 8, 5, 32, 777),
                                              (2, 16, 32, 256, 2000), (3, 32, 8, 64, 1),
-                                             (2, 64, 8, 64, 60000)])
+                                             (2, 64, 8, 64, 60000), (1, 16, 8, 64, 3001), (2, 32, 8, 64, 129)])
 def test_radial_weights_and_vjp_match_oracle(L, C, nb, hidden, E):
     P = workloads.N_PATHS_SO3[L]
     W1, W2, rng = _params(L * 100 + C, P, C, nb, hidden)
