@@ -10,14 +10,14 @@
 // Per CTA (9 warps, one CTA per SM: 224 KB of shared memory) and tile of 128 edges:
 //   1. the 8 epilogue warps build the tile's rows of H (Bessel basis, first layer,
 //      SiLU; two threads per edge), split them into TF32 halves and store both into
-//      shared memory in the tensor core's K-major layout without swizzle: 8-row x
-//      16-byte core matrices, LBO = 128 B between core matrices along K, SBO = 2048 B
-//      between 8-row groups;
+//      tensor memory (tcgen05.st; TMEM lane = edge, one column per hidden unit);
 //   2. per chunk of up to 128 output columns, one thread of the ninth warp
 //      bulk-copies the chunk of W2^T (halves pre-split by radial_tc_prepare into the
-//      same layout) into one of two shared-memory slots, issues 8 K-steps x 3
-//      products of tcgen05.mma (M = 128, N = chunk, K = 8, kind::tf32) into one of
-//      two TMEM accumulators and commits them to an mbarrier;
+//      K-major shared-memory layout without swizzle: 8-row x 16-byte core matrices,
+//      LBO = 128 B between core matrices along K, SBO = 2048 B between 8-row groups)
+//      into one of three slots, issues 8 K-steps x 3 products of tcgen05.mma
+//      (M = 128, N = chunk, K = 8, kind::tf32, A from tensor memory) into one of two
+//      TMEM accumulators and commits them to an mbarrier;
 //   3. the 8 epilogue warps read the accumulator back (tcgen05.ld; warps w and w + 4
 //      own TMEM lanes 32w..32w+31, i.e. edges, and half of the columns each), hand it
 //      back to the MMA thread by an mbarrier, and store w in whole 128-byte row
@@ -105,16 +105,21 @@ __global__ void radial_tc_prepare(const float* __restrict__ W2, int PC, int n_ch
     }
 }
 
-// Shared memory: A halves (64 KB), two B slots of two halves (128 KB), the
-// epilogue stage (8 warps x 32 rows x 32 floats, 16-byte units XOR-swizzled by the
-// row so that a phase of 8 lanes writing one row each, or reading 8 units of one
-// row, touches 8 distinct bank quads), 6 mbarriers, the TMEM address, a flag.
+// Shared memory: three W2 slots of two TF32 halves (192 KB), the epilogue stage (8
+// warps x 32 rows x 32 floats, 16-byte units XOR-swizzled by the row so that a phase
+// of 8 lanes writing one row each, or reading 8 units of one row, touches 8 distinct
+// bank quads), 7 mbarriers, the TMEM address, a flag. The H operand lives in tensor
+// memory, next to the two accumulators.
 constexpr int kEpiWarps = 8;                   // two per TMEM lane quarter, each half of a chunk's columns
 constexpr int kFwdThreads = (kEpiWarps + 1) * 32;
+constexpr int kSlots = 3;
+constexpr uint32_t kSlotBytes = 2 * kTileBytes;
 constexpr uint32_t kStageFloats = kEpiWarps * 32 * 32;
-constexpr uint32_t kOffB = 2 * kTileBytes, kOffStage = 6 * kTileBytes;
+constexpr uint32_t kOffStage = kSlots * kSlotBytes;
 constexpr uint32_t kOffBars = kOffStage + kStageFloats * 4;
-constexpr uint32_t kSmemBytes = kOffBars + 64;
+constexpr uint32_t kSmemBytes = kOffBars + 96;
+// TMEM columns: accumulators 0..127 and 128..255, H's TF32 halves 256..319 and 320..383
+constexpr uint32_t kTmemCols = 512, kTmemAHi = 256, kTmemALo = 320;
 static_assert(kOffBars % 16 == 0 && kSmemBytes <= 232448, "radial tensor-core kernel shared memory");
 static_assert(kBasis * kHidden <= (int)kStageFloats, "W1 is staged in the epilogue buffer");
 
@@ -136,54 +141,62 @@ __device__ __forceinline__ void mbar_arrive_one(uint64_t* bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&v)[32]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+        "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr),
+        "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]),
+        "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]), "r"(v[16]), "r"(v[17]), "r"(v[18]),
+        "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]),
+        "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
+        : "memory");
+}
+
 // Warp-specialised pipeline over the output chunks, with no block barrier in the
-// loop. The MMA warp (one thread) issues chunk c into accumulator c % 2 once its
-// W2 slot is filled (bar_b) and the epilogue has drained chunk c - 2 from that
+// loop. The H operand (128 edges x 64 hidden units, both TF32 halves) is written
+// into tensor memory once per tile (tcgen05.st); the products read it from there
+// (the A-from-TMEM form of tcgen05.mma) and only W2 from shared memory. The MMA
+// warp (one thread) issues chunk c into accumulator c % 2 once its W2 slot
+// (c % 3) is filled (bar_b) and the epilogue has drained chunk c - 2 from that
 // accumulator (bar_free, one arrival per epilogue warp), commits to bar_m, and
-// refills the slot of chunk c - 1 with chunk c + 1 once chunk c - 1's MMAs are done.
-// Each epilogue warp (TMEM lane quarter w % 4, column half w / 4) waits for bar_m,
-// reads its 32 rows x 64 columns into registers, frees the accumulator, and writes
-// the rows out through its own stage: every store instruction writes four whole
-// 128-byte row segments.
+// refills the slot of chunk c - 1 with chunk c + 2 once chunk c - 1's products are
+// done. Each epilogue warp (TMEM lane quarter w % 4, column half w / 4) waits for
+// bar_m, reads its 32 rows x 64 columns into registers, frees the accumulator, and
+// writes the rows out through its own stage: every store instruction writes four
+// whole 128-byte row segments.
 __global__ void __launch_bounds__(kFwdThreads, 1)
     radial_tc_forward(int E, int PC, int nb, float rc, const float* __restrict__ r, const float* __restrict__ W1,
-                      const float* __restrict__ Bhi, const float* __restrict__ Blo, float* __restrict__ w) {
+                       const float* __restrict__ Bhi, const float* __restrict__ Blo, float* __restrict__ w) {
     extern __shared__ __align__(1024) unsigned char smem[];
-    unsigned char* a_hi = smem;
-    unsigned char* a_lo = smem + kTileBytes;
     float* stage = reinterpret_cast<float*>(smem + kOffStage);
-    uint64_t* bar_b = reinterpret_cast<uint64_t*>(smem + kOffBars);       // [2] B slot filled
-    uint64_t* bar_m = bar_b + 2;                                            // [2] accumulator ready
-    uint64_t* bar_free = bar_b + 4;                                         // [2] accumulator drained
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffBars + 48);
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffBars + 52);
+    uint64_t* bar_b = reinterpret_cast<uint64_t*>(smem + kOffBars);  // [3]
+    uint64_t* bar_m = bar_b + 3;                                       // [2]
+    uint64_t* bar_free = bar_b + 5;                                    // [2]
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffBars + 64);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffBars + 68);
     const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
     const int m0 = blockIdx.x * kRows;
     const int n_chunks = (PC + kChunk - 1) / kChunk;
     constexpr int kMmaWarp = kEpiWarps;
-    auto slot_hi = [&](int s) { return smem + kOffB + (uint32_t)s * 2 * kTileBytes; };
-    auto slot_lo = [&](int s) { return smem + kOffB + (uint32_t)s * 2 * kTileBytes + kTileBytes; };
-
-    if (warp == kMmaWarp) {  // two accumulators of 128 fp32 columns
+    auto slot_hi = [&](int s) { return smem + (uint32_t)s * kSlotBytes; };
+    auto slot_lo = [&](int s) { return smem + (uint32_t)s * kSlotBytes + kTileBytes; };
+    if (warp == kMmaWarp) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
-                     "r"(256)
+                     "r"(kTmemCols)
                      : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
         if (lane == 0) {
-            for (int i = 0; i < 4; ++i) mbar_init(&bar_b[i], 1);
+            for (int i = 0; i < 5; ++i) mbar_init(&bar_b[i], 1);
             for (int i = 0; i < 2; ++i) mbar_init(&bar_free[i], kEpiWarps);
             *abort_flag = 0;
             asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-            load_b(Bhi, Blo, 0, slot_hi(0), slot_lo(0), &bar_b[0]);  // the first two chunks, behind H
-            if (n_chunks > 1) load_b(Bhi, Blo, 1, slot_hi(1), slot_lo(1), &bar_b[1]);
+            for (int c = 0; c < kSlots && c < n_chunks; ++c) load_b(Bhi, Blo, c, slot_hi(c), slot_lo(c), &bar_b[c]);
         }
     }
-
-    // 1. the tile's rows of H, split into TF32 halves: two epilogue threads per row,
-    // 32 hidden units each (W1 read from the epilogue stage, free until the first
-    // chunk is written out)
     for (int i = t; i < kBasis * kHidden; i += kFwdThreads) stage[i] = __ldg(W1 + i);
     __syncthreads();
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+    const uint32_t tmem = *tmem_slot;
     if (warp < kEpiWarps) {
         const int row = t & (kRows - 1), k0 = (t >> 7) * (kHidden / 2);
         const int e = m0 + row;
@@ -200,51 +213,51 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                 b[n] = d >= 1e-12f ? c * sinf(k * d) / d : c * k;
             }
         }
-#pragma unroll 4
-        for (int k = k0; k < k0 + kHidden / 2; ++k) {
+        uint32_t vh[32], vl[32];
+#pragma unroll
+        for (int k = 0; k < 32; ++k) {
             float h = 0.f;
             if (e < E) {
                 float zz = 0.f;
 #pragma unroll
-                for (int n = 0; n < kBasis; ++n) zz = fmaf(b[n], stage[n * kHidden + k], zz);
+                for (int n = 0; n < kBasis; ++n) zz = fmaf(b[n], stage[n * kHidden + k0 + k], zz);
                 h = zz / (1.f + expf(-zz));
             }
             const float hh = tf32_round(h);
-            *reinterpret_cast<float*>(a_hi + tile_offset(row, k)) = hh;
-            *reinterpret_cast<float*>(a_lo + tile_offset(row, k)) = tf32_round(h - hh);
+            vh[k] = __float_as_uint(hh);
+            vl[k] = __float_as_uint(tf32_round(h - hh));
         }
+        const uint32_t lanebase = (uint32_t)((warp & 3) * 32) << 16;
+        tmem_st32(tmem + lanebase + kTmemAHi + k0, vh);
+        tmem_st32(tmem + lanebase + kTmemALo + k0, vl);
+        asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
     }
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // generic-proxy writes -> tensor core
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
     __syncthreads();
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-    const uint32_t tmem = *tmem_slot;
-
     if (warp == kMmaWarp) {
-        // 2. the MMA thread
         if (lane == 0) {
-            int committed = -1, loaded = n_chunks > 1 ? 1 : 0;  // last chunk committed / loaded
+            int committed = -1, loaded = min(kSlots, n_chunks) - 1;
             for (int c = 0; c < n_chunks && !*abort_flag; ++c) {
-                const int sb = c & 1, u = c >> 1;
-                if (!mbar_wait(&bar_b[sb], u & 1) || (c >= 2 && !mbar_wait(&bar_free[sb], (u - 1) & 1))) {
+                const int sb = c & 1, u = c >> 1, sl = c % kSlots, ul = c / kSlots;
+                if (!mbar_wait(&bar_b[sl], ul & 1) || (c >= 2 && !mbar_wait(&bar_free[sb], (u - 1) & 1))) {
                     *abort_flag = 1;
                     break;
                 }
                 asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-                const int n = min(kChunk, PC - c * kChunk);  // a multiple of 16
+                const int n = min(kChunk, PC - c * kChunk);
                 const uint32_t idesc = instr_desc(n);
                 const uint32_t d_tmem = tmem + (uint32_t)sb * 128;
-                const uint32_t A[3] = {smem_u32(a_hi), smem_u32(a_hi), smem_u32(a_lo)};
-                const uint32_t B[3] = {smem_u32(slot_hi(sb)), smem_u32(slot_lo(sb)), smem_u32(slot_hi(sb))};
+                const uint32_t At[3] = {tmem + kTmemAHi, tmem + kTmemAHi, tmem + kTmemALo};
+                const uint32_t B[3] = {smem_u32(slot_hi(sl)), smem_u32(slot_lo(sl)), smem_u32(slot_hi(sl))};
                 for (int s = 0; s < kHidden / 8; ++s) {
                     for (int q = 0; q < 3; ++q) {
-                        const uint64_t da = smem_desc(A[q] + s * 2 * kLBO);
                         const uint64_t db = smem_desc(B[q] + s * 2 * kLBO);
                         const uint32_t acc = (s | q) ? 1u : 0u;
                         asm volatile(
                             "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
-                            " tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n}" ::"r"(d_tmem),
-                            "l"(da), "l"(db), "r"(idesc), "r"(acc)
+                            " tcgen05.mma.cta_group::1.kind::tf32 [%0], [%1], %2, %3, p;\n}" ::"r"(d_tmem),
+                            "r"(At[q] + 8 * s), "l"(db), "r"(idesc), "r"(acc)
                             : "memory");
                     }
                 }
@@ -252,34 +265,32 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                                  smem_u32(&bar_m[sb]))
                              : "memory");
                 committed = c;
-                // the slot of chunk c - 1 takes chunk c + 1 once chunk c - 1's products are done
-                if (c >= 1 && c + 1 < n_chunks) {
+                if (c >= 1 && c + 2 < n_chunks) {
                     if (!mbar_wait(&bar_m[sb ^ 1], ((c - 1) >> 1) & 1)) {
                         *abort_flag = 1;
                         break;
                     }
-                    load_b(Bhi, Blo, c + 1, slot_hi(sb ^ 1), slot_lo(sb ^ 1), &bar_b[sb ^ 1]);
-                    loaded = c + 1;
+                    const int s2 = (c + 2) % kSlots;
+                    load_b(Bhi, Blo, c + 2, slot_hi(s2), slot_lo(s2), &bar_b[s2]);
+                    loaded = c + 2;
                 }
             }
             if (*abort_flag) {
                 atomicOr(&g_fault, 1);
-                // leave nothing in flight on the freed TMEM and shared memory: one bounded wait each
                 if (committed >= 0) mbar_wait(&bar_m[committed & 1], (committed >> 1) & 1);
                 if (committed >= 1) mbar_wait(&bar_m[(committed - 1) & 1], ((committed - 1) >> 1) & 1);
-                for (int c = committed + 1; c <= loaded; ++c) mbar_wait(&bar_b[c & 1], (c >> 1) & 1);
+                for (int c = committed + 1; c <= loaded; ++c) mbar_wait(&bar_b[c % kSlots], (c / kSlots) & 1);
             }
         }
     } else {
-        // 3. the epilogue warps
         const int q = warp & 3, hf = warp >> 2;
         float* st = stage + warp * 32 * 32;
         for (int c = 0; c < n_chunks; ++c) {
             const int sb = c & 1, u = c >> 1;
             const int n = min(kChunk, PC - c * kChunk);
-            const int hn = max(0, min(64, n - 64 * hf));  // this warp's columns of the chunk
+            const int hn = max(0, min(64, n - 64 * hf));
             const bool got = mbar_wait(&bar_m[sb], u & 1);
-            if (__any_sync(0xffffffffu, !got || *abort_flag)) {  // warp-uniform
+            if (__any_sync(0xffffffffu, !got || *abort_flag)) {
                 if (lane == 0) {
                     *abort_flag = 1;
                     atomicOr(&g_fault, 1);
@@ -306,7 +317,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
             asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
             __syncwarp();
-            if (lane == 0) mbar_arrive_one(&bar_free[sb]);  // the accumulator may take chunk c + 2
+            if (lane == 0) mbar_arrive_one(&bar_free[sb]);
             const int e_base = m0 + q * 32;
             const size_t col0 = (size_t)c * kChunk + 64 * hf;
 #pragma unroll
@@ -334,7 +345,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     __syncthreads();
     if (warp == kMmaWarp) {
         asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(256) : "memory");
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
     }
 }
 
