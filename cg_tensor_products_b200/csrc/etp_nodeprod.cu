@@ -20,8 +20,9 @@
 // operand ranks (l1, l2): every product B_l1[m1] x_l2[m2] that some path uses is
 // formed once (one packed multiply) and scattered, with its compile-time
 // coefficients, into the accumulators of all paths (l1, l2, *); each path's sum is
-// then weighted into B(k+1)_l3. Channels never mix: no shared memory, no
-// synchronisation, no atomics.
+// then weighted into B(k+1)_l3. Every step is a packed fp32x2 instruction for the
+// thread's two channels (the coefficient as a register pair). Channels never mix:
+// no shared memory, no synchronisation, no atomics.
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -33,7 +34,7 @@
 namespace etp {
 namespace nodeprod {
 
-constexpr int kThreads = 128;
+constexpr int kThreads = 64;
 constexpr int kMaxGroups = (etp_gen::kLmax + 1) * (etp_gen::kLmax + 1);
 constexpr int kMaxPairs = kMaxGroups * (2 * etp_gen::kLmax + 1) * (2 * etp_gen::kLmax + 1);
 constexpr int kMaxTerms = etp_gen::kCgTotal > etp_gen::kCartTotal ? etp_gen::kCgTotal : etp_gen::kCartTotal;
@@ -156,7 +157,7 @@ __global__ void __launch_bounds__(kThreads) etp_node_product_kernel(int N, int K
                 const float2 q = f2_mul(B[G.l1 * G.l1 + pr.m1], xv[G.l2 * G.l2 + pr.m2]);
                 static_for<0, pr.count>([&](auto qc) {
                     constexpr Term tm = kTable<L, O3, CART>.tm[pr.first + decltype(qc)::value];
-                    f2_fma(t[tm.slot], tm.v, q);
+                    t[tm.slot] = __ffma2_rn(make_float2(tm.v, tm.v), q, t[tm.slot]);
                 });
             });
             static_for<0, G.npaths>([&](auto kc) {
