@@ -51,3 +51,18 @@ def from_full(d, L, op):
         t = d[l].detach().numpy().reshape(d[l].shape[0], d[l].shape[1], -1)
         blocks.append(np.einsum("if,ncf->nic", op(l), t))
     return np.concatenate(blocks, axis=1)
+
+
+def coupling_table(l1, l2, l3):
+    """T [2l1+1, 2l2+1, 2l3+1]: the oracle's Cartesian coupling of path (l1, l2, l3) in the
+    library's independent components, out[i3] = sum T[i1, i2, i3] A[i1] B[i2] (A, B expanded
+    to full STF tensors, the result's independent entries picked)."""
+    d1, d2 = 2 * l1 + 1, 2 * l2 + 1
+    T = np.zeros((d1, d2, 2 * l3 + 1))
+    for i in range(d1):
+        for j in range(d2):
+            a = torch.from_numpy(expand(l1)[:, i].reshape((1,) + (3,) * l1))
+            b = torch.from_numpy(expand(l2)[:, j].reshape((1,) + (3,) * l2))
+            full = ct.couple(a, b, l1, l2, l3).reshape(-1).numpy()
+            T[i, j] = pick(l3) @ full
+    return T

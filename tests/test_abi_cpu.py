@@ -265,7 +265,8 @@ def test_frames_advised_by_size(lib):
 def test_node_product_ops_count(lib, L, o3):
     """The kernel's cost model: one multiply per operand product that some path uses, one
     FMA per coupling coefficient, one FMA per weighted output component; counted here from
-    the oracle's own couplings (spherical: nonzero real CG entries)."""
+    the oracle's own couplings (nonzero real CG entries; nonzero Cartesian coefficients in
+    the independent STF components), which also pins the sparsity of the compiled tables."""
     irreps = "+".join(f"{l}{'e' if l % 2 == 0 else 'o'}" for l in range(L + 1)) if o3 else f"0..{L}"
     plan = etp.Plan(irreps, L, irreps, 8)
     from oracle import nodelocal
@@ -278,3 +279,12 @@ def test_node_product_ops_count(lib, L, o3):
             pairs.add((p[0], p[1], int(a), int(b)))
     outs = sum(2 * p[2] + 1 for p in nps)
     assert etp.node_product_ops(plan, False) == len(pairs) + terms + outs
+    # Cartesian: the same count from the oracle's Cartesian couplings in independent components
+    from cart_layout import coupling_table
+
+    terms, pairs = 0, set()
+    for p in nps:
+        nz = np.argwhere(np.abs(coupling_table(*p)) > 1e-12)
+        terms += len(nz)
+        pairs.update((p[0], p[1], int(a), int(b)) for a, b, _ in nz)
+    assert etp.node_product_ops(plan, True) == len(pairs) + terms + outs
