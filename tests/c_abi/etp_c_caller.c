@@ -43,6 +43,13 @@ static int host_checks(void) {
     CHECK(etp_plan_create(&bad, "0..4", 4, "0..4", 128, ETP_F32) == ETP_ERR_UNSUPPORTED, "L = 4 unsupported");
     CHECK(etp_plan_create(&bad, "0..2", 2, "0..2", 6, ETP_F32) == ETP_ERR_UNSUPPORTED, "C = 6 unsupported");
     CHECK(strlen(etp_status_string(ETP_ERR_CUDA)) > 0, "status string");
+    int ops = 0;
+    ETP(etp_node_product_ops(plan, 0, &ops));
+    CHECK(ops == 1023, "node-local product cost model (spherical, L = 3)");
+    ETP(etp_node_product_ops(plan, 1, &ops));
+    CHECK(ops == 1128, "node-local product cost model (Cartesian, L = 3)");
+    CHECK(etp_node_product(plan, 4, 0, 0, NULL, NULL, NULL, NULL) == ETP_ERR_INVALID_ARG, "node product K < 1 rejected");
+    CHECK(etp_node_product(plan, 0, 3, 1, NULL, NULL, NULL, NULL) == ETP_OK, "node product with no nodes");
     ETP(etp_plan_destroy(plan));
     return 0;
 }
