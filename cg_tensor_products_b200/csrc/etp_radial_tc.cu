@@ -7,10 +7,12 @@
 // whose dropped term A_lo B_lo and rounding of the halves leave a relative error
 // near 2^-21 per product, below the 1e-5 tolerance of the forward.
 //
-// Per CTA (9 warps, one CTA per SM: 224 KB of shared memory) and tile of 128 edges:
+// Per CTA (9 warps, one persistent CTA per SM: 226 KB of shared memory) and tile of
+// 128 edges, the tiles of a CTA taken in turn:
 //   1. the 8 epilogue warps build the tile's rows of H (Bessel basis, first layer,
 //      SiLU; two threads per edge), split them into TF32 halves and store both into
-//      tensor memory (tcgen05.st; TMEM lane = edge, one column per hidden unit);
+//      tensor memory (tcgen05.st; TMEM lane = edge, one column per hidden unit; two
+//      buffers, so the next tile's H is built while this tile's last chunk multiplies);
 //   2. per chunk of up to 128 output columns, one thread of the ninth warp
 //      bulk-copies the chunk of W2^T (halves pre-split by radial_tc_prepare into the
 //      K-major shared-memory layout without swizzle: 8-row x 16-byte core matrices,
@@ -116,12 +118,12 @@ constexpr int kSlots = 3;
 constexpr uint32_t kSlotBytes = 2 * kTileBytes;
 constexpr uint32_t kStageFloats = kEpiWarps * 32 * 32;
 constexpr uint32_t kOffStage = kSlots * kSlotBytes;
-constexpr uint32_t kOffBars = kOffStage + kStageFloats * 4;
-constexpr uint32_t kSmemBytes = kOffBars + 96;
-// TMEM columns: accumulators 0..127 and 128..255, H's TF32 halves 256..319 and 320..383
-constexpr uint32_t kTmemCols = 512, kTmemAHi = 256, kTmemALo = 320;
+constexpr uint32_t kOffW1 = kOffStage + kStageFloats * 4;
+constexpr uint32_t kOffBars = kOffW1 + kBasis * kHidden * 4;
+constexpr uint32_t kSmemBytes = kOffBars + 128;
+// TMEM columns: accumulators 0..127 and 128..255; H's TF32 halves of two tiles (hi, lo): 256.., 384..
+constexpr uint32_t kTmemCols = 512;
 static_assert(kOffBars % 16 == 0 && kSmemBytes <= 232448, "radial tensor-core kernel shared memory");
-static_assert(kBasis * kHidden <= (int)kStageFloats, "W1 is staged in the epilogue buffer");
 
 __device__ __forceinline__ void load_b(const float* Bhi, const float* Blo, int c, unsigned char* slot_hi,
                                        unsigned char* slot_lo, uint64_t* bar) {
@@ -152,34 +154,80 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&v)[32
         : "memory");
 }
 
-// Warp-specialised pipeline over the output chunks, with no block barrier in the
-// loop. The H operand (128 edges x 64 hidden units, both TF32 halves) is written
-// into tensor memory once per tile (tcgen05.st); the products read it from there
-// (the A-from-TMEM form of tcgen05.mma) and only W2 from shared memory. The MMA
-// warp (one thread) issues chunk c into accumulator c % 2 once its W2 slot
-// (c % 3) is filled (bar_b) and the epilogue has drained chunk c - 2 from that
-// accumulator (bar_free, one arrival per epilogue warp), commits to bar_m, and
-// refills the slot of chunk c - 1 with chunk c + 2 once chunk c - 1's products are
-// done. Each epilogue warp (TMEM lane quarter w % 4, column half w / 4) waits for
-// bar_m, reads its 32 rows x 64 columns into registers, frees the accumulator, and
-// writes the rows out through its own stage: every store instruction writes four
-// whole 128-byte row segments.
+// The H operand of one tile (128 edges x 64 hidden units, both TF32 halves) from the
+// edge lengths: two epilogue threads per edge, 32 hidden units each, written into tensor
+// memory (tcgen05.st; TMEM lane = edge) at columns col_hi / col_lo.
+__device__ __forceinline__ void build_h(int t, int warp, int m0, int E, float rc, const float* __restrict__ r,
+                                        const float* w1s, uint32_t tmem, uint32_t col_hi, uint32_t col_lo) {
+    const int row = t & (kRows - 1), k0 = (t >> 7) * (kHidden / 2);
+    const int e = m0 + row;
+    float b[kBasis];
+#pragma unroll
+    for (int n = 0; n < kBasis; ++n) b[n] = 0.f;
+    if (e < E) {
+        const float x = __ldg(r + 3 * (size_t)e), y = __ldg(r + 3 * (size_t)e + 1), z = __ldg(r + 3 * (size_t)e + 2);
+        const float d = sqrtf(x * x + y * y + z * z);
+        const float c = sqrtf(2.f / rc);
+#pragma unroll
+        for (int n = 0; n < kBasis; ++n) {
+            const float k = (float)(n + 1) * kPi / rc;
+            b[n] = d >= 1e-12f ? c * sinf(k * d) / d : c * k;
+        }
+    }
+    uint32_t vh[32], vl[32];
+#pragma unroll
+    for (int k = 0; k < 32; ++k) {
+        float h = 0.f;
+        if (e < E) {
+            float zz = 0.f;
+#pragma unroll
+            for (int n = 0; n < kBasis; ++n) zz = fmaf(b[n], w1s[n * kHidden + k0 + k], zz);
+            h = zz / (1.f + expf(-zz));
+        }
+        const float hh = tf32_round(h);
+        vh[k] = __float_as_uint(hh);
+        vl[k] = __float_as_uint(tf32_round(h - hh));
+    }
+    const uint32_t lanebase = (uint32_t)((warp & 3) * 32) << 16;
+    tmem_st32(tmem + lanebase + col_hi + k0, vh);
+    tmem_st32(tmem + lanebase + col_lo + k0, vl);
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+// Persistent warp-specialised pipeline: one CTA per SM walks tiles blockIdx.x,
+// blockIdx.x + gridDim.x, .., and the chunks of all its tiles form one sequence g (tile
+// major), with no block barrier in the loop. The MMA warp (one thread) issues chunk g
+// into accumulator g % 2 once its W2 slot (g % 3) is filled (bar_b), the epilogue has
+// drained chunk g - 2 from that accumulator (bar_free, one arrival per epilogue warp)
+// and, for a tile's first chunk, the tile's H is in tensor memory (bar_h, H buffer
+// tile % 2); the products read A from tensor memory (the A-from-TMEM form of
+// tcgen05.mma) and only W2 from shared memory. It commits to bar_m and refills the slot
+// of chunk g - 1 with chunk g + 2 once chunk g - 1's products are done. Each epilogue
+// warp (TMEM lane quarter w % 4, column half w / 4) builds the next tile's H while the
+// current tile's last chunk multiplies, waits for bar_m, reads its 32 rows x 64 columns
+// into registers, frees the accumulator, and writes the rows out through its own stage:
+// every store instruction writes four whole 128-byte row segments.
 __global__ void __launch_bounds__(kFwdThreads, 1)
     radial_tc_forward(int E, int PC, int nb, float rc, const float* __restrict__ r, const float* __restrict__ W1,
-                       const float* __restrict__ Bhi, const float* __restrict__ Blo, float* __restrict__ w) {
+                        const float* __restrict__ Bhi, const float* __restrict__ Blo, float* __restrict__ w) {
     extern __shared__ __align__(1024) unsigned char smem[];
     float* stage = reinterpret_cast<float*>(smem + kOffStage);
+    float* w1s = reinterpret_cast<float*>(smem + kOffW1);
     uint64_t* bar_b = reinterpret_cast<uint64_t*>(smem + kOffBars);  // [3]
-    uint64_t* bar_m = bar_b + 3;                                       // [2]
-    uint64_t* bar_free = bar_b + 5;                                    // [2]
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffBars + 64);
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffBars + 68);
+    uint64_t* bar_m = bar_b + 3;                                        // [2]
+    uint64_t* bar_free = bar_b + 5;                                     // [2]
+    uint64_t* bar_h = bar_b + 7;                                        // [2] H buffer written
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffBars + 96);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffBars + 100);
     const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
-    const int m0 = blockIdx.x * kRows;
+    const int n_tiles = (E + kRows - 1) / kRows;
+    const int n_local = n_tiles > (int)blockIdx.x ? (n_tiles - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
     const int n_chunks = (PC + kChunk - 1) / kChunk;
+    const int total = n_local * n_chunks;  // this CTA's chunks, tile-major
     constexpr int kMmaWarp = kEpiWarps;
     auto slot_hi = [&](int s) { return smem + (uint32_t)s * kSlotBytes; };
     auto slot_lo = [&](int s) { return smem + (uint32_t)s * kSlotBytes + kTileBytes; };
+    auto hcol = [&](int hb, int lo) { return (uint32_t)(256 + 128 * hb + 64 * lo); };
     if (warp == kMmaWarp) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
                      "r"(kTmemCols)
@@ -188,59 +236,25 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         if (lane == 0) {
             for (int i = 0; i < 5; ++i) mbar_init(&bar_b[i], 1);
             for (int i = 0; i < 2; ++i) mbar_init(&bar_free[i], kEpiWarps);
+            for (int i = 0; i < 2; ++i) mbar_init(&bar_h[i], kEpiWarps);
             *abort_flag = 0;
             asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-            for (int c = 0; c < kSlots && c < n_chunks; ++c) load_b(Bhi, Blo, c, slot_hi(c), slot_lo(c), &bar_b[c]);
+            for (int g = 0; g < kSlots && g < total; ++g)
+                load_b(Bhi, Blo, g % n_chunks, slot_hi(g), slot_lo(g), &bar_b[g]);
         }
     }
-    for (int i = t; i < kBasis * kHidden; i += kFwdThreads) stage[i] = __ldg(W1 + i);
+    for (int i = t; i < kBasis * kHidden; i += kFwdThreads) w1s[i] = __ldg(W1 + i);
     __syncthreads();
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
     const uint32_t tmem = *tmem_slot;
-    if (warp < kEpiWarps) {
-        const int row = t & (kRows - 1), k0 = (t >> 7) * (kHidden / 2);
-        const int e = m0 + row;
-        float b[kBasis];
-#pragma unroll
-        for (int n = 0; n < kBasis; ++n) b[n] = 0.f;
-        if (e < E) {
-            const float x = __ldg(r + 3 * (size_t)e), y = __ldg(r + 3 * (size_t)e + 1), z = __ldg(r + 3 * (size_t)e + 2);
-            const float d = sqrtf(x * x + y * y + z * z);
-            const float c = sqrtf(2.f / rc);
-#pragma unroll
-            for (int n = 0; n < kBasis; ++n) {
-                const float k = (float)(n + 1) * kPi / rc;
-                b[n] = d >= 1e-12f ? c * sinf(k * d) / d : c * k;
-            }
-        }
-        uint32_t vh[32], vl[32];
-#pragma unroll
-        for (int k = 0; k < 32; ++k) {
-            float h = 0.f;
-            if (e < E) {
-                float zz = 0.f;
-#pragma unroll
-                for (int n = 0; n < kBasis; ++n) zz = fmaf(b[n], stage[n * kHidden + k0 + k], zz);
-                h = zz / (1.f + expf(-zz));
-            }
-            const float hh = tf32_round(h);
-            vh[k] = __float_as_uint(hh);
-            vl[k] = __float_as_uint(tf32_round(h - hh));
-        }
-        const uint32_t lanebase = (uint32_t)((warp & 3) * 32) << 16;
-        tmem_st32(tmem + lanebase + kTmemAHi + k0, vh);
-        tmem_st32(tmem + lanebase + kTmemALo + k0, vl);
-        asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-    }
-    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-    __syncthreads();
-    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
     if (warp == kMmaWarp) {
         if (lane == 0) {
-            int committed = -1, loaded = min(kSlots, n_chunks) - 1;
-            for (int c = 0; c < n_chunks && !*abort_flag; ++c) {
-                const int sb = c & 1, u = c >> 1, sl = c % kSlots, ul = c / kSlots;
-                if (!mbar_wait(&bar_b[sl], ul & 1) || (c >= 2 && !mbar_wait(&bar_free[sb], (u - 1) & 1))) {
+            int committed = -1, loaded = min(kSlots, total) - 1;
+            for (int g = 0; g < total && !*abort_flag; ++g) {
+                const int i = g / n_chunks, c = g - i * n_chunks;
+                const int sb = g & 1, u = g >> 1, sl = g % kSlots, ul = g / kSlots;
+                if (!mbar_wait(&bar_b[sl], ul & 1) || (g >= 2 && !mbar_wait(&bar_free[sb], (u - 1) & 1)) ||
+                    (c == 0 && !mbar_wait(&bar_h[i & 1], (i >> 1) & 1))) {
                     *abort_flag = 1;
                     break;
                 }
@@ -248,7 +262,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                 const int n = min(kChunk, PC - c * kChunk);
                 const uint32_t idesc = instr_desc(n);
                 const uint32_t d_tmem = tmem + (uint32_t)sb * 128;
-                const uint32_t At[3] = {tmem + kTmemAHi, tmem + kTmemAHi, tmem + kTmemALo};
+                const uint32_t At[3] = {tmem + hcol(i & 1, 0), tmem + hcol(i & 1, 0), tmem + hcol(i & 1, 1)};
                 const uint32_t B[3] = {smem_u32(slot_hi(sl)), smem_u32(slot_lo(sl)), smem_u32(slot_hi(sl))};
                 for (int s = 0; s < kHidden / 8; ++s) {
                     for (int q = 0; q < 3; ++q) {
@@ -264,29 +278,44 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                 asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
                                  smem_u32(&bar_m[sb]))
                              : "memory");
-                committed = c;
-                if (c >= 1 && c + 2 < n_chunks) {
-                    if (!mbar_wait(&bar_m[sb ^ 1], ((c - 1) >> 1) & 1)) {
+                committed = g;
+                if (g >= 1 && g + 2 < total) {
+                    if (!mbar_wait(&bar_m[sb ^ 1], ((g - 1) >> 1) & 1)) {
                         *abort_flag = 1;
                         break;
                     }
-                    const int s2 = (c + 2) % kSlots;
-                    load_b(Bhi, Blo, c + 2, slot_hi(s2), slot_lo(s2), &bar_b[s2]);
-                    loaded = c + 2;
+                    const int s2 = (g + 2) % kSlots;
+                    load_b(Bhi, Blo, (g + 2) % n_chunks, slot_hi(s2), slot_lo(s2), &bar_b[s2]);
+                    loaded = g + 2;
                 }
             }
             if (*abort_flag) {
                 atomicOr(&g_fault, 1);
                 if (committed >= 0) mbar_wait(&bar_m[committed & 1], (committed >> 1) & 1);
                 if (committed >= 1) mbar_wait(&bar_m[(committed - 1) & 1], ((committed - 1) >> 1) & 1);
-                for (int c = committed + 1; c <= loaded; ++c) mbar_wait(&bar_b[c % kSlots], (c / kSlots) & 1);
+                for (int g = committed + 1; g <= loaded; ++g) mbar_wait(&bar_b[g % kSlots], (g / kSlots) & 1);
             }
         }
     } else {
         const int q = warp & 3, hf = warp >> 2;
         float* st = stage + warp * 32 * 32;
-        for (int c = 0; c < n_chunks; ++c) {
-            const int sb = c & 1, u = c >> 1;
+        if (n_local > 0) {
+            build_h(t, warp, (int)blockIdx.x * kRows, E, rc, r, w1s, tmem, hcol(0, 0), hcol(0, 1));
+            asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+            __syncwarp();
+            if (lane == 0) mbar_arrive_one(&bar_h[0]);
+        }
+        for (int g = 0; g < total; ++g) {
+            const int i = g / n_chunks, c = g - i * n_chunks;
+            const int m0 = ((int)blockIdx.x + i * (int)gridDim.x) * kRows;
+            if (c == n_chunks - 1 && i + 1 < n_local) {  // the next tile's H, while this tile's last chunk multiplies
+                build_h(t, warp, ((int)blockIdx.x + (i + 1) * (int)gridDim.x) * kRows, E, rc, r, w1s, tmem,
+                        hcol((i + 1) & 1, 0), hcol((i + 1) & 1, 1));
+                asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+                __syncwarp();
+                if (lane == 0) mbar_arrive_one(&bar_h[(i + 1) & 1]);
+            }
+            const int sb = g & 1, u = g >> 1;
             const int n = min(kChunk, PC - c * kChunk);
             const int hn = max(0, min(64, n - 64 * hf));
             const bool got = mbar_wait(&bar_m[sb], u & 1);
@@ -312,7 +341,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                         : "r"(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(sb * 128 + 64 * hf + 16 * jj)));
                 else
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) v[16 * jj + i] = 0u;
+                    for (int ii = 0; ii < 16; ++ii) v[16 * jj + ii] = 0u;
             }
             asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
             asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
@@ -889,8 +918,8 @@ cudaError_t radial_tc_forward(int E, int nb, int PC, float rc, const float* r, c
     cudaError_t err = cudaFuncSetAttribute(rtc::radial_tc_forward, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                            (int)smem);
     if (err != cudaSuccess) return err;
-    rtc::radial_tc_forward<<<(E + rtc::kRows - 1) / rtc::kRows, rtc::kFwdThreads, smem, s>>>(E, PC, nb, rc, r, W1, hi,
-                                                                                            lo, w);
+    const int tiles = (E + rtc::kRows - 1) / rtc::kRows;
+    rtc::radial_tc_forward<<<tiles < 148 ? tiles : 148, rtc::kFwdThreads, smem, s>>>(E, PC, nb, rc, r, W1, hi, lo, w);
     return cudaGetLastError();
 }
 
